@@ -1,0 +1,414 @@
+"""Benchmark of the GuidedQuant + LNQ hot path on B200.
+
+One step = the whole hot path on one synthetic Llama-2-7B q_proj layer (d_in = d_out = 4096,
+n = 16384 calibration tokens, 4 Fisher groups, 4-bit codebooks, 3 LNQ iterations):
+guided Fisher build (s_g reduction, operand scaling, tcgen05 SYRK), codebook initialisation,
+3 x (codebook step + assignment sweep), and the per-row objective.
+
+    python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+
+With N > 1 (launched by torchrun, one process per GPU) every rank quantises its own layer (the
+rows, groups and layers of the method are independent), so per-GPU work is fixed: weak scaling,
+with no collective on the data path. Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+METRIC = "LNQ rows quantized/s per layer (guided Fisher build + init + LNQ iterations)"
+UNIT = "rows/s"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                  "sm_max_mhz": 1965.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        d["source"] = "measured"
+        return d
+    d = dict(PEAKS_FALLBACK)
+    d["source"] = "fallback"
+    return d
+
+
+# ------------------------------------------------------------------------------------------
+# Clock sampling during the timed region
+# ------------------------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.path = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            ident = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+        except Exception:
+            ident = str(device_index)
+        self.ident = ident
+
+    def start(self):
+        import tempfile
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.ident, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) == 7:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[0]) for r in rows if r[0].replace(".", "").isdigit()]
+        mx = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[k] for r in rows for k in range(4) if r[3 + k] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows),
+                "power_w_max": max((float(r[2]) for r in rows
+                                    if r[2].replace(".", "").isdigit()), default=None)}
+
+
+# ------------------------------------------------------------------------------------------
+# Algorithmic work per kernel (units and per-unit figures are stated in the design doc)
+# ------------------------------------------------------------------------------------------
+def algorithmic_work(layer, kernel: str, launches: int, moves_per_sweep: float):
+    """(amount, unit kind) per launch for a kernel of one step on `layer`."""
+    d, n, g, dout, m = layer.d_in, layer.n, layer.groups, layer.d_out, layer.m
+    if kernel == "fisher_syrk":
+        return 2.0 * g * n * d * d, "flop"                     # dense-equivalent
+    if kernel == "group_scales":
+        return 2.0 * n * dout + 4.0 * g * n, "byte"            # read G, write S
+    if kernel == "scale_rows":
+        return 2.0 * n * d + 4.0 * g * n + 2.0 * g * n * d, "byte"
+    if kernel == "lnq_codebook":
+        return 1.0 * dout * d * d, "lane_op"                    # one bin-add per F entry per row
+    if kernel == "lnq_sweep":
+        # u = F r refresh (d^2 per row) plus the trailing updates of the moved coordinates
+        return dout * (d * d + moves_per_sweep * d / 2.0), "lane_op"
+    if kernel == "lnq_objective":
+        return 1.0 * dout * d * d, "lane_op"
+    if kernel == "lnq_init":
+        return 4.0 * dout * d + dout * d, "byte"
+    return 0.0, "unknown"
+
+
+def roofline_for(kernel, per_launch_work, unit, avg_ms, peaks, clocks, num_sms):
+    sec = avg_ms / 1e3
+    if unit == "flop":
+        peak = peaks["bf16_tflops"]
+        achieved = per_launch_work / sec / 1e12
+        return {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak}
+    if unit == "byte":
+        peak = peaks["hbm_gbs"]
+        achieved = per_launch_work / sec / 1e9
+        return {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                "frac": achieved / peak}
+    # FP32 lane operations: 128 FP32 lanes per SM at the maximum SM clock
+    mhz = peaks.get("sm_max_mhz", 1965.0)
+    peak = num_sms * 128 * mhz * 1e6 / 1e12
+    achieved = per_launch_work / sec / 1e12
+    return {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "Tlane-op/s",
+            "frac": achieved / peak}
+
+
+# ------------------------------------------------------------------------------------------
+# Oracle (CPU) baseline on a bounded sample
+# ------------------------------------------------------------------------------------------
+def cpu_baseline(layer, X, G, W, F_gpu, budget_s=20.0, threads=None):
+    """Oracle throughput in rows/s on a bounded sample of the same layer, extrapolated:
+    Fisher = measured 64x64 tiles of group 0 scaled to all groups' full blocks; LNQ = measured
+    rows of group 0 (init + all iterations on the GPU's F) scaled to all rows."""
+    from oracle import oracle as orc
+    threads = threads or os.cpu_count()
+    d, n, R = layer.d_in, layer.n, layer.rows_per_group
+    t_start = time.perf_counter()
+    s = np.empty(n)
+    Rg = layer.rows_per_group
+    for r0 in range(0, n, 4096):
+        Gh = G[r0:r0 + 4096, 0:Rg].double().cpu().numpy()
+        s[r0:r0 + Gh.shape[0]] = orc.group_scales(Gh, Gh.shape[0], Rg, 1)[0]
+    t_s = time.perf_counter() - t_start
+    tiles, t_tiles = 0, 0.0
+    rng = np.random.default_rng(0)
+    while t_tiles < budget_s * 0.3 and tiles < 64:
+        i0, k0 = (int(v) for v in rng.integers(0, d - 64, 2))
+        A = X[:, i0:i0 + 64].double().cpu().numpy()
+        B = X[:, k0:k0 + 64].double().cpu().numpy()
+        t0 = time.perf_counter()
+        orc.fisher_block(A, B, s, 1.0)
+        t_tiles += time.perf_counter() - t0
+        tiles += 1
+    fisher_s = (t_tiles / tiles) * layer.groups * (d / 64.0) ** 2 + t_s * layer.groups
+    Fh = F_gpu[0].double().cpu().numpy()
+    Wh = W[:R].double().cpu().numpy()
+    rows, t_rows = 0, 0.0
+    while t_rows < budget_s * 0.6 and rows < R:
+        k = min(threads, R - rows)
+        t0 = time.perf_counter()
+        orc.lnq_rows(Fh, Wh[rows:rows + k], layer.m, layer.iters, init=True, nthreads=threads)
+        t_rows += time.perf_counter() - t0
+        rows += k
+    lnq_s = t_rows / rows * layer.d_out
+    value = layer.d_out / (fisher_s + lnq_s)
+    return {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": (f"Fisher: {tiles} 64x64 tiles of group 0 (n={n}) extrapolated to "
+                       f"{layer.groups} full {d}x{d} blocks; LNQ: {rows} rows of group 0, init + "
+                       f"{layer.iters} iterations on the GPU's F, extrapolated to {layer.d_out} "
+                       f"rows; FP64, {threads} OpenMP threads"),
+            "fisher_s_extrapolated": fisher_s, "lnq_s_extrapolated": lnq_s}
+
+
+# ------------------------------------------------------------------------------------------
+# Main arm
+# ------------------------------------------------------------------------------------------
+def run_ours(args, rank, world, device):
+    import post_weight_quantization_guided_b200 as lnq
+    from post_weight_quantization_guided_b200 import binding as b
+    from post_weight_quantization_guided_b200 import workloads as wl
+
+    lnq.binding.lib()
+    layer = wl.scaled(wl.Q_PROJ, seed=wl.Q_PROJ.seed + 100 * rank,
+                      x_seed=wl.Q_PROJ.x_seed + 100 * rank)
+    torch.cuda.set_device(device)
+    X, G, W = wl.make_layer(layer, device)
+    d, dout, m, it = layer.d_in, layer.d_out, layer.m, layer.iters
+    F = torch.empty((layer.groups, d, d), dtype=torch.float32, device=device)
+    C = torch.empty((dout, m), dtype=torch.float32, device=device)
+    Q = torch.empty((dout, d), dtype=torch.uint8, device=device)
+    J = torch.empty(dout, dtype=torch.float64, device=device)
+    st = torch.empty(dout, dtype=torch.int32, device=device)
+    ws_f = b.workspace(b.LNQ_OP_BUILD_FISHER, layer.n, d, dout, layer.groups, m, device)
+    ws_q = b.workspace(b.LNQ_OP_QUANTIZE_ROWS, 0, d, dout, layer.groups, m, device)
+    ws_i = b.workspace(b.LNQ_OP_INIT_CODEBOOK, 0, d, dout, 1, m, device)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step(Xs, Gs, Ws):
+        lnq.lnq_build_fisher(Xs, Gs, layer.groups, F=F, ws=ws_f)
+        lnq.lnq_init_codebook(Ws, m, C, Q, ws=ws_i)
+        lnq.lnq_quantize_rows(F, Ws, m, it, C, Q, J, st, ws=ws_q)
+
+    for _ in range(args.warmup):
+        step(X, G, W)
+    torch.cuda.synchronize(device)
+    assert b.lnq_workspace_check(ws_f) == b.LNQ_OK
+
+    # ---------------------------------------------------------------- device-timed region
+    sampler = ClockSampler(device.index) if rank == 0 else None
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(device)
+    if sampler:
+        sampler.start()
+    b.lnq_profile_read()
+    b.lnq_profile_enable(True)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    for k in range(args.steps):
+        flush.fill_(k & 0xFF)           # evict L2 between timed steps (untimed)
+        evs[k][0].record(stream)
+        step(X, G, W)
+        evs[k][1].record(stream)
+    torch.cuda.synchronize(device)
+    if world > 1:
+        torch.distributed.barrier()
+    b.lnq_profile_enable(False)
+    prof = b.lnq_profile_read()
+    clocks = sampler.stop() if sampler else None
+    step_ms = [a.elapsed_time(z) for a, z in evs]
+    total_ms = float(sum(step_ms))
+    assert b.lnq_workspace_check(ws_f) == b.LNQ_OK
+    Jh = J.cpu().numpy()
+    assert np.all(np.isfinite(Jh)) and int(st.abs().sum()) == 0
+
+    # ---------------------------------------------------------------- end to end (host buffers)
+    Xp, Gp, Wp = X.cpu().pin_memory(), G.cpu().pin_memory(), W.cpu().pin_memory()
+    Cp = torch.empty_like(C, device="cpu").pin_memory()
+    Qp = torch.empty_like(Q, device="cpu").pin_memory()
+    Jp = torch.empty_like(J, device="cpu").pin_memory()
+    Xd, Gd, Wd = torch.empty_like(X), torch.empty_like(G), torch.empty_like(W)
+    h2d = X.numel() * 2 + G.numel() * 2 + W.numel() * 4
+    d2h = C.numel() * 4 + Q.numel() + J.numel() * 8
+    e2e_steps = max(1, min(args.steps, 3))
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        Xd.copy_(Xp, non_blocking=True)
+        Gd.copy_(Gp, non_blocking=True)
+        Wd.copy_(Wp, non_blocking=True)
+        step(Xd, Gd, Wd)
+        Cp.copy_(C, non_blocking=True)
+        Qp.copy_(Q, non_blocking=True)
+        Jp.copy_(J, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    e2e_ms = e0.elapsed_time(e1)
+
+    # ---------------------------------------------------------------- max over ranks
+    t = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    total_ms, e2e_ms = float(t[0]), float(t[1])
+
+    if rank != 0:
+        return None
+    ms_per_step = total_ms / args.steps
+    value = world * dout / (ms_per_step / 1e3)
+    e2e_value = world * dout * e2e_steps / (e2e_ms / 1e3)
+
+    peaks = load_peaks()
+    num_sms = torch.cuda.get_device_properties(device).multi_processor_count
+    kernels = {}
+    for name, (launches, ms) in prof.items():
+        per_step = launches / args.steps
+        per_launch, unit = algorithmic_work(layer, name, launches, 0.0)
+        avg = ms / launches
+        kernels[name] = {"launches_per_step": per_step, "avg_ms": avg,
+                         "share": ms / sum(v[1] for v in prof.values()),
+                         "roofline": roofline_for(name, per_launch, unit, avg, peaks, clocks,
+                                                  num_sms)}
+    dominant = max(kernels, key=lambda k: kernels[k]["share"])
+    roof = dict(kernels[dominant]["roofline"])
+    roof["kernel"] = dominant
+    roof["traffic"] = None
+    roof["peak_source"] = peaks["source"]
+    fisher_ms = kernels.get("fisher_syrk", {}).get("avg_ms")
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16+f32",
+        "data": "synthetic (seeded draws with the q_proj layer's shapes and distributions)",
+        "config": {"workload": layer.name, "d_in": d, "d_out": dout, "n": layer.n,
+                   "groups": layer.groups, "m": m, "iters": it,
+                   "rows_per_step": world * dout, "parallelism": f"layer-per-gpu x{world}",
+                   "l2": "flushed between timed steps (256 MB write)"},
+        "gpu_launches": int(sum(v[0] for v in prof.values()) / args.steps) * args.steps,
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "roofline": roof,
+        "fisher_tflops": (layer.fisher_flops / (fisher_ms / 1e3) / 1e12) if fisher_ms else None,
+        "kernels": kernels,
+        "clocks": clocks,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(layer, X, G, W, F, budget_s=args.cpu_budget)
+    return line
+
+
+def run_reference(args, rank, world):
+    """The oracle (plain FP64 CPU code) on the host cores, same metric and workload, each step a
+    bounded sample extrapolated to the whole layer."""
+    if rank != 0:
+        return None
+    from post_weight_quantization_guided_b200 import workloads as wl
+    from oracle import oracle as orc
+    orc.build()
+    layer = wl.Q_PROJ
+    X, G, W = wl.make_layer(layer, "cpu")
+    d = layer.d_in
+    s = orc.group_scales(G[:, :layer.rows_per_group].double().numpy(), layer.n,
+                         layer.rows_per_group, 1)[0]
+    # Untimed preparation: group 0's Fisher block as input for the LNQ sample (a plain float64
+    # product; the oracle's own Fisher routine is what the timed sample below measures).
+    Xh = X.double().numpy()
+    F0 = (Xh * s[:, None]).T @ Xh
+    vals = []
+    for k in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        A = X[:, 0:64].double().numpy()
+        orc.fisher_block(A, A, s, 1.0)
+        t_tile = time.perf_counter() - t0
+        t1 = time.perf_counter()
+        orc.lnq_rows(F0, W[:8].double().numpy(), layer.m, layer.iters, init=True, nthreads=0)
+        t_rows = time.perf_counter() - t1
+        per_layer = t_tile * layer.groups * (d / 64.0) ** 2 + t_rows / 8 * layer.d_out
+        if k >= args.warmup:
+            vals.append(layer.d_out / per_layer)
+    value = statistics.median(vals)
+    threads = os.cpu_count()
+    return {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * layer.d_out / value, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": layer.name, "d_in": d, "d_out": layer.d_out, "n": layer.n,
+                       "groups": layer.groups, "m": layer.m, "iters": layer.iters},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                             "sample": "per step: one 64x64 Fisher tile (n=16384) and 8 rows "
+                                       "of LNQ (init + 3 iterations), extrapolated to the layer"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=20.0)
+    args = ap.parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+    from datetime import timedelta
+    if world > 1:
+        torch.distributed.init_process_group("nccl", timeout=timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local))
+    device = torch.device("cuda", local)
+    try:
+        line = run_ours(args, rank, world, device)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+    if line is not None:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,158 @@
+/*
+ * lnq.h -- C ABI of the B200 (sm_100a) library for the GuidedQuant + LNQ hot path.
+ *
+ * What it computes (source pages: "GuidedQuant" blog post on jinukkim.me, and the GuidedQuant
+ * abstract on the aitopics "squeezellm" tag page):
+ *
+ *   1. Guided Fisher blocks -- GuidedQuant section, third equation and the sentence after it.
+ *      The gradient-weighted output error ||dL/dZ (.) (XW - XW^)||_F^2 equals
+ *      n * sum_j (w_j - w^_j)^T F_j (w_j - w^_j) with F_j = (1/n) X^T diag(G_:,j^2) X. The blocks
+ *      are grouped and averaged within each group, which gives
+ *          F_g = alpha * X^T diag(s_g) X,   s_g[t] = mean_{j in g} G[t,j]^2.
+ *      Groups are contiguous, equal slices of output rows. With G == NULL every gradient is 1, and
+ *      then F = alpha * X^T X, the Hessian of the plain layer-wise objective (first equation).
+ *   2. LNQ -- LNQ section, both equations. Output row j gets a codebook c_j (m values) and a
+ *      one-hot assignment q_j (d_in indices). These minimise
+ *          J_j = (c_j[q_j] - w_j)^T F_g (c_j[q_j] - w_j)
+ *      by alternating two steps: the closed-form codebook update c <- (P^T F P)^-1 P^T F w, and a
+ *      coordinate-descent assignment sweep over i = 0..d_in-1 in order.
+ *
+ * Readings the pages leave open, and what this library does:
+ *   - Initial codebook: c_q = sort(w)[floor((2q+1) d_in / (2m))]. Each weight then takes its
+ *     nearest codeword, with ties going to the lower index. Every iteration starts with the
+ *     codebook step.
+ *   - Assignment: a coordinate moves only if the move strictly lowers J_j. Among equal best
+ *     candidates, the lowest index wins.
+ *   - Codebook: solved over the non-empty codewords only; empty codewords keep their value; no
+ *     damping. If the Cholesky factorisation meets a non-positive pivot, the row keeps its old
+ *     codebook and its row_status is set to LNQ_ROW_SINGULAR.
+ *
+ * Conventions for every entry point:
+ *   - Pointers: every array pointer is DEVICE memory that the caller allocates and owns. The
+ *     library allocates no device memory. It keeps no state between calls except a cached TMA
+ *     encoder function pointer.
+ *   - Layout: all matrices are dense and row-major with no padding.
+ *       X  [n][d_in]      bf16, passed as raw 16-bit patterns (uint16_t)
+ *       G  [n][d_out]     bf16 (raw 16-bit), or NULL
+ *       W  [d_out][d_in]  fp32, row j = output channel w_j
+ *       F  [groups][d_in][d_in] fp32, full symmetric blocks
+ *       C  [d_out][m]     fp32
+ *       Q  [d_out][d_in]  uint8 codeword indices
+ *   - Streams: each call enqueues its work on `stream` and returns without synchronising. A NULL
+ *     stream is the legacy default stream. Results are valid once the stream has synchronised.
+ *   - Workspace: `ws` is caller-owned device scratch of at least lnq_workspace_size(op, ...) bytes,
+ *     aligned to 256 bytes. Two calls that share one workspace must not overlap in time.
+ *   - Errors: a call returns LNQ_ERR_INVALID_ARG (bad sizes or misaligned pointers) or
+ *     LNQ_ERR_WORKSPACE (ws too small, NULL or misaligned) before it launches anything.
+ *     It returns LNQ_ERR_CUDA if a launch fails. Kernels never trap. Every wait inside them is
+ *     bounded. A wait that gives up sets a flag in the workspace and the kernel returns early;
+ *     lnq_workspace_check() reports that flag as LNQ_ERR_TIMEOUT.
+ */
+#ifndef LNQ_H
+#define LNQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define LNQ_API __attribute__((visibility("default")))
+#else
+#define LNQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t (struct CUstream_st *); NULL is the legacy default stream. */
+typedef struct CUstream_st *lnq_stream_t;
+
+typedef enum {
+    LNQ_OK = 0,
+    LNQ_ERR_INVALID_ARG = 1,
+    LNQ_ERR_CUDA = 2,
+    LNQ_ERR_WORKSPACE = 3,
+    LNQ_ERR_UNSUPPORTED = 4,
+    LNQ_ERR_TIMEOUT = 5
+} lnq_status;
+
+/* Per-row outcome written to row_status by lnq_quantize_rows. */
+enum { LNQ_ROW_OK = 0, LNQ_ROW_SINGULAR = 1 };
+
+/* Operation selector for lnq_workspace_size. */
+typedef enum {
+    LNQ_OP_BUILD_FISHER = 0,
+    LNQ_OP_INIT_CODEBOOK = 1,
+    LNQ_OP_QUANTIZE_ROWS = 2,
+    LNQ_OP_OBJECTIVE = 3
+} lnq_op;
+
+/* Bytes of device workspace the operation needs for these sizes (0 if the sizes are invalid).
+ * Arguments an operation does not use are ignored. */
+LNQ_API size_t lnq_workspace_size(lnq_op op, int64_t n, int64_t d_in, int64_t d_out, int groups, int m);
+
+/* Guided Fisher blocks F_g = alpha * X^T diag(s_g) X, g = 0..groups-1 (GuidedQuant section, third
+ * equation and the grouping sentence).
+ *   X      [n][d_in] bf16; G [n][d_out] bf16 or NULL (all gradients 1, requires groups == 1)
+ *   alpha  overall scale (1 gives X^T X for G == NULL; 1/n gives the blocks of the equation)
+ *   F      out, [groups][d_in][d_in] fp32, both triangles written
+ * Requirements: n >= 1; d_in >= 1 and d_in % 8 == 0; d_out >= 1; groups >= 1 and
+ * d_out % groups == 0; X, G and F 16-byte aligned. Arithmetic: the s_g reduction in fp32. The
+ * products run on tensor cores with bf16 operands and fp32 accumulation. When G != NULL, the
+ * operand is bf16(sqrt(s_g[t]) * X[t][:]), rounded once. */
+LNQ_API lnq_status lnq_build_fisher(const uint16_t *X, const uint16_t *G, int64_t n, int64_t d_in,
+                            int64_t d_out, int groups, float alpha, float *F, void *ws,
+                            size_t ws_bytes, lnq_stream_t stream);
+
+/* Initial codebooks and assignments for every row (reading above).
+ *   W  [d_out][d_in] fp32 in; C [d_out][m] fp32 out; Q [d_out][d_in] uint8 out
+ * Requirements: m in {2, 4, 8, 16}; 1 <= d_in <= 16384; d_out >= 1. */
+LNQ_API lnq_status lnq_init_codebook(const float *W, int64_t d_out, int64_t d_in, int m, float *C,
+                             uint8_t *Q, void *ws, size_t ws_bytes, lnq_stream_t stream);
+
+/* `iters` LNQ iterations (codebook step, then assignment sweep) for every row, starting from
+ * (C, Q) and updating them in place (LNQ section, second equation). Row j uses
+ * F[j / (d_out/groups)].
+ *   J_out       [d_out] fp64 out (objective after the last sweep), or NULL
+ *   row_status  [d_out] int32 out (LNQ_ROW_OK / LNQ_ROW_SINGULAR), or NULL
+ * Resuming: calling with iters = a and then with iters = b gives bit-identical (C, Q) to one call
+ * with iters = a + b.
+ * Requirements: as lnq_init_codebook, plus groups >= 1, d_out % groups == 0, 0 <= iters. */
+LNQ_API lnq_status lnq_quantize_rows(const float *F, int groups, const float *W, int64_t d_out,
+                             int64_t d_in, int m, int iters, float *C, uint8_t *Q,
+                             double *J_out, int32_t *row_status, void *ws, size_t ws_bytes,
+                             lnq_stream_t stream);
+
+/* Per-row objective J[j] = r^T F_g r with r = C[j][Q[j]] - W[j] (fp32 products, fp64 sums). */
+LNQ_API lnq_status lnq_objective(const float *F, int groups, const float *W, const float *C,
+                         const uint8_t *Q, int64_t d_out, int64_t d_in, int m, double *J,
+                         void *ws, size_t ws_bytes, lnq_stream_t stream);
+
+/* Synchronises `stream`, then reads and clears the flag that a bounded in-kernel wait sets when it
+ * gives up. Returns LNQ_OK, LNQ_ERR_TIMEOUT or LNQ_ERR_CUDA. */
+LNQ_API lnq_status lnq_workspace_check(void *ws, lnq_stream_t stream);
+
+/* Testing knob: upper bound, in SM clock cycles, on every in-kernel wait of later calls from this
+ * process (0 makes every wait give up at once). A negative value restores the default of about
+ * 2^31 cycles, roughly a second. */
+LNQ_API void lnq_set_wait_limit(int64_t cycles);
+
+/* Tracing aid: when switched on (on != 0), every kernel launch of later calls is bracketed by two
+ * CUDA events on the launching stream. Off by default; events are host objects, so profiling
+ * allocates no device memory. */
+LNQ_API void lnq_profile_enable(int on);
+
+/* Waits for the recorded events, then writes at most max_kernels entries: names[k] (static
+ * strings owned by the library), total_ms[k] (summed device time) and launches[k]. Clears the
+ * records. Returns the number of entries written. */
+LNQ_API int lnq_profile_read(int max_kernels, const char **names, double *total_ms,
+                             int64_t *launches);
+
+/* Static description of a status code. */
+LNQ_API const char *lnq_status_string(lnq_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LNQ_H */

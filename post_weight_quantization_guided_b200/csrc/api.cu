@@ -1,0 +1,236 @@
+// api.cu -- the extern "C" entry points declared in include/lnq.h.
+//
+// Host-side only: argument validation, workspace carving, TMA descriptor encoding and kernel
+// launches on the caller's stream. No device memory is allocated here.
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <mutex>
+
+#include "common.cuh"
+#include "profile.cuh"
+
+namespace lnq {
+
+// Kernels defined in fisher.cu / lnq.cu.
+__global__ void group_scales_kernel(const __nv_bfloat16 *, int64_t, int64_t, int, float *);
+__global__ void scale_rows_kernel(const __nv_bfloat16 *, const float *, int64_t, int64_t, int,
+                                  __nv_bfloat16 *);
+cudaError_t fisher_syrk(const __nv_bfloat16 *Y, int64_t n, int64_t d, int groups, float alpha,
+                        float *F, DeviceErr err, cudaStream_t s, int num_sms);
+cudaError_t lnq_init_launch(const float *W, int64_t d_out, int64_t d, int m, float *C,
+                            uint8_t *Q, cudaStream_t s);
+cudaError_t lnq_iterate_launch(const float *F, int groups, const float *W, int64_t d_out,
+                               int64_t d, int m, int iters, float *C, uint8_t *Q, double *J,
+                               int32_t *status, cudaStream_t s);
+cudaError_t lnq_objective_launch(const float *F, int groups, const float *W, const float *C,
+                                 const uint8_t *Q, int64_t d_out, int64_t d, int m, double *J,
+                                 cudaStream_t s);
+
+static std::atomic<long long> g_wait_limit{kDefaultWaitLimit};
+
+static int device_sm_count()
+{
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess)
+        return 148;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+        return 148;
+    return sms;
+}
+
+static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+static bool valid_m(int m) { return m == 2 || m == 4 || m == 8 || m == 16; }
+
+// Workspace layout (all offsets 256-byte aligned):
+//   BUILD_FISHER:   header | S [groups][n] f32 | Y [groups][n][d_in] bf16
+//   QUANTIZE_ROWS:  header | status [d_out] i32
+//   INIT, OBJECTIVE: header
+struct FisherWs {
+    size_t s_off, y_off, total;
+};
+static FisherWs fisher_ws(int64_t n, int64_t d_in, int groups)
+{
+    FisherWs w;
+    w.s_off = kWsHeader;
+    w.y_off = align_up(w.s_off + static_cast<size_t>(groups) * n * sizeof(float), 256);
+    w.total = align_up(w.y_off + static_cast<size_t>(groups) * n * d_in * 2, 256);
+    return w;
+}
+
+}  // namespace lnq
+
+using namespace lnq;
+
+extern "C" {
+
+const char *lnq_status_string(lnq_status s)
+{
+    switch (s) {
+    case LNQ_OK: return "ok";
+    case LNQ_ERR_INVALID_ARG: return "invalid argument";
+    case LNQ_ERR_CUDA: return "CUDA error";
+    case LNQ_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case LNQ_ERR_UNSUPPORTED: return "unsupported configuration";
+    case LNQ_ERR_TIMEOUT: return "a bounded in-kernel wait gave up";
+    }
+    return "unknown status";
+}
+
+void lnq_set_wait_limit(int64_t cycles)
+{
+    g_wait_limit.store(cycles < 0 ? kDefaultWaitLimit : static_cast<long long>(cycles));
+}
+
+size_t lnq_workspace_size(lnq_op op, int64_t n, int64_t d_in, int64_t d_out, int groups, int m)
+{
+    (void)m;
+    switch (op) {
+    case LNQ_OP_BUILD_FISHER:
+        if (n < 1 || d_in < 1 || groups < 1)
+            return 0;
+        return fisher_ws(n, d_in, groups).total;
+    case LNQ_OP_QUANTIZE_ROWS:
+        if (d_out < 1)
+            return 0;
+        return align_up(kWsHeader + static_cast<size_t>(d_out) * sizeof(int32_t), 256);
+    case LNQ_OP_INIT_CODEBOOK:
+    case LNQ_OP_OBJECTIVE:
+        return kWsHeader;
+    }
+    return 0;
+}
+
+static lnq_status check_ws(void *ws, size_t ws_bytes, size_t need)
+{
+    if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0 || ws_bytes < need)
+        return LNQ_ERR_WORKSPACE;
+    return LNQ_OK;
+}
+
+lnq_status lnq_build_fisher(const uint16_t *X, const uint16_t *G, int64_t n, int64_t d_in,
+                            int64_t d_out, int groups, float alpha, float *F, void *ws,
+                            size_t ws_bytes, lnq_stream_t stream)
+{
+    if (X == nullptr || F == nullptr || n < 1 || d_in < 1 || d_in % 8 != 0 || d_out < 1 ||
+        groups < 1 || d_out % groups != 0 || !aligned16(X) || !aligned16(F) ||
+        (G != nullptr && !aligned16(G)) || (G == nullptr && groups != 1) ||
+        n > (int64_t(1) << 31) - 64 || d_in > (int64_t(1) << 30))
+        return LNQ_ERR_INVALID_ARG;
+    const FisherWs lay = fisher_ws(n, d_in, groups);
+    const size_t need = (G == nullptr) ? kWsHeader : lay.total;
+    lnq_status st = check_ws(ws, ws_bytes, need);
+    if (st != LNQ_OK)
+        return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t *base = static_cast<uint8_t *>(ws);
+    DeviceErr err{reinterpret_cast<uint32_t *>(base), g_wait_limit.load()};
+    if (cudaMemsetAsync(base, 0, kWsHeader, s) != cudaSuccess)
+        return LNQ_ERR_CUDA;
+    const __nv_bfloat16 *Y = reinterpret_cast<const __nv_bfloat16 *>(X);
+    if (G != nullptr) {
+        float *S = reinterpret_cast<float *>(base + lay.s_off);
+        __nv_bfloat16 *Yw = reinterpret_cast<__nv_bfloat16 *>(base + lay.y_off);
+        const int64_t warps = n * groups;
+        const int threads = 256;
+        const int64_t blocks = (warps * 32 + threads - 1) / threads;
+        {
+            KernelTimer timer("group_scales", s);
+            group_scales_kernel<<<static_cast<unsigned>(blocks), threads, 0, s>>>(
+                reinterpret_cast<const __nv_bfloat16 *>(G), n, d_out, groups, S);
+        }
+        const int64_t vecs = n * (d_in / 8);
+        {
+            KernelTimer timer("scale_rows", s);
+            scale_rows_kernel<<<static_cast<unsigned>((vecs + threads - 1) / threads), threads, 0,
+                                s>>>(reinterpret_cast<const __nv_bfloat16 *>(X), S, n, d_in,
+                                     groups, Yw);
+        }
+        if (cudaGetLastError() != cudaSuccess)
+            return LNQ_ERR_CUDA;
+        Y = Yw;
+    }
+    cudaError_t e = fisher_syrk(Y, n, d_in, groups, alpha, F, err, s, device_sm_count());
+    if (e == cudaErrorNotSupported)
+        return LNQ_ERR_UNSUPPORTED;
+    return e == cudaSuccess ? LNQ_OK : LNQ_ERR_CUDA;
+}
+
+lnq_status lnq_init_codebook(const float *W, int64_t d_out, int64_t d_in, int m, float *C,
+                             uint8_t *Q, void *ws, size_t ws_bytes, lnq_stream_t stream)
+{
+    if (W == nullptr || C == nullptr || Q == nullptr || d_out < 1 || d_in < 1 || d_in > 16384 ||
+        !valid_m(m) || d_out > (int64_t(1) << 31) - 1)
+        return LNQ_ERR_INVALID_ARG;
+    lnq_status st = check_ws(ws, ws_bytes, kWsHeader);
+    if (st != LNQ_OK)
+        return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    return lnq_init_launch(W, d_out, d_in, m, C, Q, s) == cudaSuccess ? LNQ_OK : LNQ_ERR_CUDA;
+}
+
+lnq_status lnq_quantize_rows(const float *F, int groups, const float *W, int64_t d_out,
+                             int64_t d_in, int m, int iters, float *C, uint8_t *Q,
+                             double *J_out, int32_t *row_status, void *ws, size_t ws_bytes,
+                             lnq_stream_t stream)
+{
+    if (F == nullptr || W == nullptr || C == nullptr || Q == nullptr || groups < 1 ||
+        d_out < 1 || d_out % groups != 0 || d_in < 1 || d_in > 16384 || !valid_m(m) ||
+        iters < 0 || d_out > (int64_t(1) << 31) - 1)
+        return LNQ_ERR_INVALID_ARG;
+    const size_t need = lnq_workspace_size(LNQ_OP_QUANTIZE_ROWS, 0, d_in, d_out, groups, m);
+    lnq_status st = check_ws(ws, ws_bytes, need);
+    if (st != LNQ_OK)
+        return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t *base = static_cast<uint8_t *>(ws);
+    int32_t *status = reinterpret_cast<int32_t *>(base + kWsHeader);
+    if (cudaMemsetAsync(base, 0, kWsHeader + static_cast<size_t>(d_out) * sizeof(int32_t), s) !=
+        cudaSuccess)
+        return LNQ_ERR_CUDA;
+    if (lnq_iterate_launch(F, groups, W, d_out, d_in, m, iters, C, Q, J_out, status, s) !=
+        cudaSuccess)
+        return LNQ_ERR_CUDA;
+    if (row_status != nullptr &&
+        cudaMemcpyAsync(row_status, status, static_cast<size_t>(d_out) * sizeof(int32_t),
+                        cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+        return LNQ_ERR_CUDA;
+    return LNQ_OK;
+}
+
+lnq_status lnq_objective(const float *F, int groups, const float *W, const float *C,
+                         const uint8_t *Q, int64_t d_out, int64_t d_in, int m, double *J,
+                         void *ws, size_t ws_bytes, lnq_stream_t stream)
+{
+    if (F == nullptr || W == nullptr || C == nullptr || Q == nullptr || J == nullptr ||
+        groups < 1 || d_out < 1 || d_out % groups != 0 || d_in < 1 || d_in > 16384 ||
+        !valid_m(m) || d_out > (int64_t(1) << 31) - 1)
+        return LNQ_ERR_INVALID_ARG;
+    lnq_status st = check_ws(ws, ws_bytes, kWsHeader);
+    if (st != LNQ_OK)
+        return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    return lnq_objective_launch(F, groups, W, C, Q, d_out, d_in, m, J, s) == cudaSuccess
+               ? LNQ_OK
+               : LNQ_ERR_CUDA;
+}
+
+lnq_status lnq_workspace_check(void *ws, lnq_stream_t stream)
+{
+    if (ws == nullptr)
+        return LNQ_ERR_WORKSPACE;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint32_t flags[2] = {0, 0};
+    if (cudaMemcpyAsync(flags, ws, sizeof(flags), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+        return LNQ_ERR_CUDA;
+    if (flags[0] != 0u) {
+        if (cudaMemsetAsync(ws, 0, sizeof(flags), s) != cudaSuccess ||
+            cudaStreamSynchronize(s) != cudaSuccess)
+            return LNQ_ERR_CUDA;
+        return LNQ_ERR_TIMEOUT;
+    }
+    return LNQ_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,202 @@
+"""GPU-versus-oracle parity through the C ABI (needs a B200 and the built library).
+
+Fisher blocks: "GuidedQuant" blog post, GuidedQuant section (third equation, grouping sentence).
+LNQ: same post, LNQ section (problem and iteration). Tolerances are in parity_helpers.
+"""
+import numpy as np
+import pytest
+import torch
+
+from parity_helpers import (check_fisher_full, check_fisher_sampled, lnq_follow_parity, J_TOL)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def lnq():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from post_weight_quantization_guided_b200 import build
+    build.build_library()
+    import post_weight_quantization_guided_b200 as pkg
+    return pkg
+
+
+@pytest.fixture(scope="module")
+def wl():
+    from post_weight_quantization_guided_b200 import workloads
+    return workloads
+
+
+def _dev():
+    return torch.device("cuda:0")
+
+
+# --------------------------------------------------------------------------------- Fisher
+
+def test_fisher_tiny_layer_full(orc, lnq, wl):
+    layer = wl.TINY
+    X, G, W = wl.make_layer(layer, _dev())
+    F = lnq.lnq_build_fisher(X, G, layer.groups)
+    check_fisher_full(orc, F, X, G, layer.groups)
+
+
+@pytest.mark.parametrize("n,d_in,d_out,groups,guided", [
+    (200, 136, 6, 3, True),    # ragged n and d_in (one partial row block and column block)
+    (77, 8, 4, 1, True),       # smallest d_in
+    (64, 264, 5, 1, False),    # unguided, ragged
+    (1, 64, 2, 2, True),       # a single token
+    (130, 512, 8, 8, True),    # 4 x 2 tile grid, diagonal and off-diagonal tiles
+    (1000, 392, 12, 4, True),
+])
+def test_fisher_ragged_shapes(orc, lnq, wl, n, d_in, d_out, groups, guided):
+    layer = wl.scaled(wl.TINY, n=n, d_in=d_in, d_out=d_out, groups=groups,
+                      x_outlier_cols=min(4, d_in), g_kind="normal" if guided else "ones")
+    X, G, _ = wl.make_layer(layer, _dev())
+    F = lnq.lnq_build_fisher(X, G, groups)
+    check_fisher_full(orc, F, X, G, groups)
+
+
+def test_fisher_unit_gradients_and_alpha(orc, lnq, wl):
+    layer = wl.scaled(wl.TINY, n=333, d_in=200, d_out=16, groups=1)
+    X, _, _ = wl.make_layer(layer, _dev())
+    F0 = lnq.lnq_build_fisher(X, None, 1)
+    ones = torch.ones((layer.n, layer.d_out), dtype=torch.bfloat16, device=_dev())
+    F1 = lnq.lnq_build_fisher(X, ones, 1)
+    torch.cuda.synchronize()
+    assert torch.equal(F0, F1)            # sqrt(1) * x == x exactly
+    Xh = X.double().cpu().numpy()
+    ref = Xh.T @ Xh                        # library matmul, independent of the oracle
+    dg = np.sqrt(np.outer(np.diag(ref), np.diag(ref)))
+    assert np.max(np.abs(F0[0].double().cpu().numpy() - ref) / dg) < 1e-5
+    Fa = lnq.lnq_build_fisher(X, None, 1, alpha=1.0 / layer.n)
+    check_fisher_full(orc, Fa, X, None, 1, alpha=1.0 / layer.n)
+
+
+def test_fisher_symmetric(lnq, wl):
+    layer = wl.scaled(wl.TINY, n=500, d_in=392, d_out=12, groups=3)
+    X, G, _ = wl.make_layer(layer, _dev())
+    F = lnq.lnq_build_fisher(X, G, 3)
+    assert torch.equal(F, F.transpose(1, 2))
+
+
+def test_fisher_q_proj_full_size_sampled(orc, lnq, wl):
+    layer = wl.Q_PROJ
+    X, G, _ = wl.make_layer(layer, _dev())
+    F = lnq.lnq_build_fisher(X, G, layer.groups)
+    check_fisher_sampled(orc, F, X, G, layer.groups, tiles_per_group=6)
+
+
+# --------------------------------------------------------------------------------- LNQ
+
+def test_lnq_tiny_layer_all_rows(orc, lnq, wl):
+    layer = wl.TINY
+    X, G, W = wl.make_layer(layer, _dev())
+    F = lnq.lnq_build_fisher(X, G, layer.groups)
+    summary, _, _ = lnq_follow_parity(orc, lnq, F, W, layer.m, layer.iters)
+    assert summary["moves"] > 0
+
+
+def test_lnq_resume_is_bit_identical(lnq, wl):
+    layer = wl.TINY
+    X, G, W = wl.make_layer(layer, _dev())
+    F = lnq.lnq_build_fisher(X, G, layer.groups)
+    C, Q = lnq.lnq_init_codebook(W, layer.m)
+    Ca, Qa = C.clone(), Q.clone()
+    lnq.lnq_quantize_rows(F, W, layer.m, 3, C, Q)
+    lnq.lnq_quantize_rows(F, W, layer.m, 1, Ca, Qa)
+    lnq.lnq_quantize_rows(F, W, layer.m, 2, Ca, Qa)
+    torch.cuda.synchronize()
+    assert torch.equal(C, Ca) and torch.equal(Q, Qa)
+
+
+def test_lnq_q_proj_full_size_sampled_rows(orc, lnq, wl):
+    layer = wl.Q_PROJ
+    X, G, W = wl.make_layer(layer, _dev())
+    F = lnq.lnq_build_fisher(X, G, layer.groups)
+    del X, G
+    summary, _, _ = lnq_follow_parity(orc, lnq, F, W, layer.m, layer.iters, rows_per_group=16)
+    assert summary["moves"] > 0
+
+
+@pytest.mark.parametrize("m", [2, 4, 8, 16])
+def test_lnq_every_codebook_size(orc, lnq, wl, m):
+    layer = wl.scaled(wl.TINY, d_in=96, d_out=8, n=300, groups=2, m=m)
+    X, G, W = wl.make_layer(layer, _dev())
+    F = lnq.lnq_build_fisher(X, G, layer.groups)
+    lnq_follow_parity(orc, lnq, F, W, m, 3)
+
+
+def test_lnq_empty_codewords_and_tiny_rows(orc, lnq, wl):
+    # Rows with only 3 distinct values and m = 8 leave codewords empty; d_in = 5 is not a
+    # multiple of anything.
+    torch.manual_seed(0)
+    d, d_out, m = 5, 4, 8
+    A = torch.randn(20, d, dtype=torch.float64)
+    F = (A.T @ A).float().unsqueeze(0).contiguous().to(_dev())
+    W = torch.tensor([[0.1, 0.1, 0.2, 0.2, 0.3]] * d_out, dtype=torch.float32)
+    W[1] = torch.tensor([1.0, -1.0, 0.5, 0.25, 0.0])
+    W = W.to(_dev())
+    lnq_follow_parity(orc, lnq, F, W, m, 3)
+
+
+def test_lnq_singular_rows(orc, lnq):
+    # Coordinates 0..3 see an all-zero block of F, so any codeword used only there has a zero
+    # pivot: the row keeps its codebook and reports LNQ_ROW_SINGULAR, exactly as the oracle.
+    d, m = 16, 4
+    torch.manual_seed(1)
+    A = torch.randn(40, d, dtype=torch.float64)
+    F = A.T @ A
+    F[:4, :] = 0
+    F[:, :4] = 0
+    F = F.float().unsqueeze(0).contiguous().to(_dev())
+    W = torch.cat([torch.full((1, 4), 5.0), torch.randn(1, d - 4) * 0.01], dim=1).to(_dev())
+    W = W.float().contiguous()
+    st = torch.empty(1, dtype=torch.int32, device=_dev())
+    C, Q = lnq.lnq_init_codebook(W, m)
+    C0 = C.clone()
+    lnq.lnq_quantize_rows(F, W, m, 1, C, Q, None, st)
+    torch.cuda.synchronize()
+    Fh = F[0].double().cpu().numpy()
+    c_or, status = orc.codebook_row(Fh, W[0].double().cpu().numpy(), Q.cpu().numpy()[0],
+                                    C0[0].double().cpu().numpy())
+    assert status == 1 and int(st[0]) == 1
+    assert torch.equal(C, C0)
+
+
+def test_objective_entry_point(orc, lnq, wl):
+    layer = wl.TINY
+    X, G, W = wl.make_layer(layer, _dev())
+    F = lnq.lnq_build_fisher(X, G, layer.groups)
+    C, Q = lnq.lnq_init_codebook(W, layer.m)
+    lnq.lnq_quantize_rows(F, W, layer.m, 2, C, Q)
+    J = lnq.lnq_objective(F, W, C, Q)
+    torch.cuda.synchronize()
+    Fh, Wh, Ch, Qh = (F.double().cpu().numpy(), W.double().cpu().numpy(),
+                      C.double().cpu().numpy(), Q.cpu().numpy())
+    R = layer.rows_per_group
+    for j in range(layer.d_out):
+        Jo = orc.objective_row(Fh[j // R], Wh[j], Ch[j], Qh[j])
+        assert abs(J[j].item() - Jo) <= J_TOL * Jo
+
+
+# --------------------------------------------------------------------------------- failures
+
+def test_wait_limit_zero_reports_timeout_and_recovers(lnq, wl):
+    """Every in-kernel wait gives up at once: the call reports a timeout through the workspace
+    flag, the context stays usable, and the next call with the default limit is correct."""
+    from post_weight_quantization_guided_b200 import binding as b
+    layer = wl.scaled(wl.TINY, n=512, d_in=256, d_out=8, groups=2)
+    X, G, _ = wl.make_layer(layer, _dev())
+    ws = b.workspace(b.LNQ_OP_BUILD_FISHER, layer.n, layer.d_in, layer.d_out, layer.groups)
+    try:
+        b.lnq_set_wait_limit(0)
+        lnq.lnq_build_fisher(X, G, layer.groups, ws=ws)
+        assert b.lnq_workspace_check(ws) == b.LNQ_ERR_TIMEOUT
+    finally:
+        b.lnq_set_wait_limit(-1)
+    F = lnq.lnq_build_fisher(X, G, layer.groups, ws=ws)
+    assert b.lnq_workspace_check(ws) == b.LNQ_OK
+    F2 = lnq.lnq_build_fisher(X, G, layer.groups)
+    torch.cuda.synchronize()
+    assert torch.equal(F, F2)
