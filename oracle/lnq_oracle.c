@@ -234,16 +234,19 @@ int orc_codebook_row(const double *F, int64_t d, const double *w, int m, const u
  *
  * Follow mode: when `hint` is not NULL it holds another solver's assignment after the same sweep.
  * Where the hint differs from this sweep's choice and the hinted candidate's Delta is within
- * tie_rel * J_current of the best Delta, the hint is adopted and counted as a tie-follow;
- * otherwise this sweep's choice is kept and the coordinate is counted as a mismatch.
+ * max(tie_rel * J_current, tie_abs) of the best Delta, the hint is adopted and counted as a
+ * tie-follow; otherwise this sweep's choice is kept and the coordinate is counted as a mismatch.
+ * The absolute floor tie_abs matters only for rows whose objective reaches (nearly) zero: there
+ * duplicate codewords make many assignments equally good, and the candidates differ only by
+ * rounding noise, far below any fraction of J.
  *
  * stats (may be NULL): [0] moves, [1] tie-follows, [2] mismatches, [3] smallest gap
  * (second-best minus best Delta, over all coordinates, in units of J_current) encoded as a
  * double bit pattern.  J_trace (may be NULL, length d+1): J before the sweep and after each
  * coordinate.  Returns J after the sweep (tracked incrementally from J before the sweep). */
 double orc_sweep_row(const double *F, int64_t d, const double *w, int m, const double *c,
-                     uint8_t *q, const uint8_t *hint, double tie_rel, int64_t *stats,
-                     double *J_trace)
+                     uint8_t *q, const uint8_t *hint, double tie_rel, double tie_abs,
+                     int64_t *stats, double *J_trace)
 {
     double *u = (double *)malloc((size_t)d * sizeof(double));
     double *delta = (double *)malloc((size_t)m * sizeof(double));
@@ -279,15 +282,15 @@ double orc_sweep_row(const double *F, int64_t d, const double *w, int m, const d
         for (int a = 0; a < m; ++a)
             if (a != best && delta[a] < second)
                 second = delta[a];
-        double Jref = fabs(J) > 0.0 ? fabs(J) : 1.0;
-        double gap = (second - bestD) / Jref;
+        const double band = fmax(tie_rel * fabs(J), tie_abs);
+        double gap = (second - bestD) / (fabs(J) > 0.0 ? fabs(J) : 1.0);
         if (gap < min_gap)
             min_gap = gap;
         int chosen = best;
         double chosenD = bestD;
         if (hint != NULL && hint[i] != best) {
             double hD = hint[i] < m ? delta[hint[i]] : INFINITY;
-            if (hD - bestD <= tie_rel * Jref) {
+            if (hD - bestD <= band) {
                 chosen = hint[i];
                 chosenD = hD;
                 ++follows;
@@ -344,7 +347,7 @@ void orc_lnq_rows(const double *F, int64_t d, const double *W, int64_t nrows, in
                 st = ORC_ROW_SINGULAR;
             if (J_hist)
                 J_hist[j * 2 * iters + 2 * it] = orc_objective_row(F, d, w, c, q);
-            orc_sweep_row(F, d, w, m, c, q, NULL, 0.0, NULL, NULL);
+            orc_sweep_row(F, d, w, m, c, q, NULL, 0.0, 0.0, NULL, NULL);
             if (J_hist)
                 J_hist[j * 2 * iters + 2 * it + 1] = orc_objective_row(F, d, w, c, q);
         }
@@ -355,14 +358,16 @@ void orc_lnq_rows(const double *F, int64_t d, const double *W, int64_t nrows, in
 
 /* One LNQ iteration in follow mode for `nrows` rows sharing F.
  * In:  C_start, Q_start (another solver's state at the start of the iteration) and Q_hint (that
- *      solver's assignment at the end of the iteration).
+ *      solver's assignment at the end of the iteration); tie_abs (nrows, may be NULL) the
+ *      per-row absolute floor of the tie band.
  * Out: C_out = this oracle's codebook step applied to (C_start, Q_start); Q_out = this oracle's
  *      sweep from Q_start with C_out, following the hint inside the tie band; J_out = objective of
  *      (C_out, Q_out) from its definition; stats (nrows x 4) as in orc_sweep_row;
  *      status (nrows) the codebook status. */
 void orc_follow_iteration(const double *F, int64_t d, const double *W, int64_t nrows, int m,
                           const double *C_start, const uint8_t *Q_start, const uint8_t *Q_hint,
-                          double tie_rel, double *C_out, uint8_t *Q_out, double *J_out,
+                          double tie_rel, const double *tie_abs, double *C_out, uint8_t *Q_out,
+                          double *J_out,
                           int64_t *stats, int32_t *status, int nthreads)
 {
 #ifdef _OPENMP
@@ -377,7 +382,8 @@ void orc_follow_iteration(const double *F, int64_t d, const double *W, int64_t n
         memcpy(c, C_start + j * m, (size_t)m * sizeof(double));
         memcpy(q, Q_start + j * d, (size_t)d);
         status[j] = orc_codebook_row(F, d, w, m, q, c);
-        orc_sweep_row(F, d, w, m, c, q, Q_hint + j * d, tie_rel, stats + 4 * j, NULL);
+        orc_sweep_row(F, d, w, m, c, q, Q_hint + j * d, tie_rel, tie_abs ? tie_abs[j] : 0.0,
+                      stats + 4 * j, NULL);
         J_out[j] = orc_objective_row(F, d, w, c, q);
     }
 }

@@ -51,12 +51,12 @@ def _bind(path: str):
     lib.orc_codebook_row.argtypes = [_DP, _I64, _DP, ctypes.c_int, _U8P, _DP]
     lib.orc_codebook_row.restype = ctypes.c_int
     lib.orc_sweep_row.argtypes = [_DP, _I64, _DP, ctypes.c_int, _DP, _U8P, _U8P,
-                                  ctypes.c_double, _I64P, _DP]
+                                  ctypes.c_double, ctypes.c_double, _I64P, _DP]
     lib.orc_sweep_row.restype = ctypes.c_double
     lib.orc_lnq_rows.argtypes = [_DP, _I64, _DP, _I64, ctypes.c_int, ctypes.c_int,
                                  ctypes.c_int, _DP, _U8P, _DP, _I32P, ctypes.c_int]
     lib.orc_follow_iteration.argtypes = [_DP, _I64, _DP, _I64, ctypes.c_int, _DP, _U8P,
-                                         _U8P, ctypes.c_double, _DP, _U8P, _DP, _I64P,
+                                         _U8P, ctypes.c_double, _DP, _DP, _U8P, _DP, _I64P,
                                          _I32P, ctypes.c_int]
     return lib
 
@@ -181,7 +181,8 @@ def codebook_row(F, w, q, c):
     return c, st
 
 
-def sweep_row(F, w, c, q, hint=None, tie_rel: float = 0.0, trace: bool = False):
+def sweep_row(F, w, c, q, hint=None, tie_rel: float = 0.0, trace: bool = False,
+              tie_abs: float = 0.0):
     """Returns (q after the sweep, J after, stats dict, J trace or None)."""
     F, w, c = _f64(F), _f64(w), _f64(c)
     q = _u8(q).copy()
@@ -190,7 +191,7 @@ def sweep_row(F, w, c, q, hint=None, tie_rel: float = 0.0, trace: bool = False):
     jt = np.empty(d + 1, dtype=np.float64) if trace else None
     hp = _p(_u8(hint), _U8P) if hint is not None else None
     J = _load().orc_sweep_row(_p(F, _DP), d, _p(w, _DP), c.shape[0], _p(c, _DP), _p(q, _U8P),
-                              hp, tie_rel, _p(stats, _I64P),
+                              hp, tie_rel, tie_abs, _p(stats, _I64P),
                               _p(jt, _DP) if trace else None)
     st = {"moves": int(stats[0]), "follows": int(stats[1]), "mismatches": int(stats[2]),
           "min_gap": float(stats[3:4].view(np.float64)[0])}
@@ -212,8 +213,9 @@ def lnq_rows(F, W, m: int, iters: int, init: bool = True, C=None, Q=None,
 
 
 def follow_iteration(F, W, m: int, C_start, Q_start, Q_hint, tie_rel: float,
-                     nthreads: int = 0):
+                     nthreads: int = 0, tie_abs=None):
     """One oracle iteration from another solver's state, following its choices at near-ties.
+    tie_abs: optional per-row absolute floor of the tie band.
 
     Returns (C_out, Q_out, J_out, stats [rows, 4] with the gap column as float64, status)."""
     F, W = _f64(F), _f64(W)
@@ -224,8 +226,10 @@ def follow_iteration(F, W, m: int, C_start, Q_start, Q_hint, tie_rel: float,
     J_out = np.empty(nrows, dtype=np.float64)
     stats = np.zeros((nrows, 4), dtype=np.int64)
     status = np.zeros(nrows, dtype=np.int32)
+    ta = None if tie_abs is None else _f64(tie_abs)
     _load().orc_follow_iteration(_p(F, _DP), d, _p(W, _DP), nrows, m, _p(C_start, _DP),
-                                 _p(Q_start, _U8P), _p(Q_hint, _U8P), tie_rel, _p(C_out, _DP),
+                                 _p(Q_start, _U8P), _p(Q_hint, _U8P), tie_rel,
+                                 None if ta is None else _p(ta, _DP), _p(C_out, _DP),
                                  _p(Q_out, _U8P), _p(J_out, _DP), _p(stats, _I64P),
                                  _p(status, _I32P), nthreads)
     return C_out, Q_out, J_out, stats, status

@@ -343,3 +343,27 @@ def test_pins_catch_planted_mistakes(orc, tmp_path, anchor, mistake, pin):
     with orc.mutated(anchor, mistake, str(tmp_path)):
         assert not _pins_pass(orc, pin), f"pin '{pin}' missed: {mistake}"
     assert _pins_pass(orc, pin)
+
+
+def test_follow_mode_absolute_floor_for_exactly_representable_rows(orc):
+    """A row the codebook represents exactly reaches J ~ 0; candidates among equal codewords then
+    differ only by rounding noise. Without a floor every such difference is a 'mismatch'; with a
+    floor tied to the row's scale w^T F w they are followed, and nothing else changes."""
+    rng = np.random.default_rng(12)
+    A = rng.standard_normal((20, 5))
+    F = A.T @ A
+    w = np.array([0.1, 0.1, 0.2, 0.2, 0.3])
+    c0, q0 = orc.init_row(w, 8)
+    c, _ = orc.codebook_row(F, w, q0, c0)
+    assert orc.objective_row(F, w, c, q0) < 1e-28
+    hint = q0.copy()
+    q_strict, _, st, _ = orc.sweep_row(F, w, c, q0, hint=hint, tie_rel=1e-6, tie_abs=0.0)
+    Jw = w @ F @ w
+    q_floor, _, st2, _ = orc.sweep_row(F, w, c, q0, hint=hint, tie_rel=1e-6, tie_abs=1e-12 * Jw)
+    assert st2["mismatches"] == 0
+    np.testing.assert_array_equal(q_floor, hint)
+    # a genuinely worse hint is still a mismatch with the floor
+    bad = q0.copy()
+    bad[4] = 0
+    _, _, st3, _ = orc.sweep_row(F, w, c, q0, hint=bad, tie_rel=1e-6, tie_abs=1e-12 * Jw)
+    assert st3["mismatches"] == 1
