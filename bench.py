@@ -110,20 +110,21 @@ def algorithmic_work(layer, kernel: str, launches: int, moves_per_sweep: float):
     """(amount, unit kind) per launch for a kernel of one step on `layer`."""
     d, n, g, dout, m = layer.d_in, layer.n, layer.groups, layer.d_out, layer.m
     if kernel == "fisher_syrk":
-        return 2.0 * g * n * d * d, "flop"                     # dense-equivalent
-    if kernel == "group_scales":
-        return 2.0 * n * dout + 4.0 * g * n, "byte"            # read G, write S
-    if kernel == "scale_rows":
-        return 2.0 * n * d + 4.0 * g * n + 2.0 * g * n * d, "byte"
+        # every unique entry of each symmetric block: 2 n flops for each of d(d+1)/2 entries
+        return float(g) * n * d * (d + 1), "flop"
+    if kernel == "token_stats":
+        return 2.0 * n * (d + dout) + 4.0 * n * (g + 1), "byte"    # read X and G, write S and M
+    if kernel == "guided_operands":
+        return 2.0 * n * d * (2 + g) + 4.0 * n * (g + 1), "byte"   # read X, S, M; write A, B_g
+    if kernel == "lnq_init":
+        return 4.0 * dout * d + dout * d + 4.0 * dout * m, "byte"  # read W, write Q and C
     if kernel == "lnq_codebook":
-        return 1.0 * dout * d * d, "lane_op"                    # one bin-add per F entry per row
+        return 2.0 * dout * d * d, "lane_op"   # a class-bin add and an FMA per F entry per row
     if kernel == "lnq_sweep":
-        # u = F r refresh (d^2 per row) plus the trailing updates of the moved coordinates
+        # u = F r refresh (d^2 FMA per row) plus the trailing updates of the moved coordinates
         return dout * (d * d + moves_per_sweep * d / 2.0), "lane_op"
     if kernel == "lnq_objective":
         return 1.0 * dout * d * d, "lane_op"
-    if kernel == "lnq_init":
-        return 4.0 * dout * d + dout * d, "byte"
     return 0.0, "unknown"
 
 
@@ -311,7 +312,8 @@ def run_ours(args, rank, world, device):
     roof["kernel"] = dominant
     roof["traffic"] = None
     roof["peak_source"] = peaks["source"]
-    fisher_ms = kernels.get("fisher_syrk", {}).get("avg_ms")
+    fisher_ms = sum(kernels[k]["avg_ms"] for k in ("token_stats", "guided_operands", "fisher_syrk")
+                    if k in kernels) or None
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
@@ -325,7 +327,9 @@ def run_ours(args, rank, world, device):
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "roofline": roof,
-        "fisher_tflops": (layer.fisher_flops / (fisher_ms / 1e3) / 1e12) if fisher_ms else None,
+        # the whole Fisher build (statistics, operands, SYRK) at the unique-entry flop count
+        "fisher_tflops": (layer.groups * layer.n * d * (d + 1) / (fisher_ms / 1e3) / 1e12)
+        if fisher_ms else None,
         "kernels": kernels,
         "clocks": clocks,
     }

@@ -12,12 +12,15 @@
 
 namespace lnq {
 
-// Kernels defined in fisher.cu / lnq.cu.
-__global__ void group_scales_kernel(const __nv_bfloat16 *, int64_t, int64_t, int, float *);
-__global__ void scale_rows_kernel(const __nv_bfloat16 *, const float *, int64_t, int64_t, int,
-                                  __nv_bfloat16 *);
-cudaError_t fisher_syrk(const __nv_bfloat16 *Y, int64_t n, int64_t d, int groups, float alpha,
-                        float *F, DeviceErr err, cudaStream_t s, int num_sms);
+// Kernels and launchers defined in fisher.cu / lnq.cu.
+__global__ void token_stats_kernel(const __nv_bfloat16 *, const __nv_bfloat16 *, int64_t, int64_t,
+                                   int64_t, int, float *, float *, unsigned *);
+__global__ void guided_operands_kernel(const __nv_bfloat16 *, const float *, const float *,
+                                       const unsigned *, int64_t, int64_t, int, __half *,
+                                       __half *);
+cudaError_t fisher_syrk(const void *A, const void *B, bool f16, const unsigned *pimax, int64_t n,
+                        int64_t d, int groups, float alpha, float *F, DeviceErr err,
+                        cudaStream_t s, int num_sms);
 cudaError_t lnq_init_launch(const float *W, int64_t d_out, int64_t d, int m, float *C,
                             uint8_t *Q, cudaStream_t s);
 cudaError_t lnq_iterate_launch(const float *F, int groups, const float *W, int64_t d_out,
@@ -43,18 +46,22 @@ static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 
 static bool valid_m(int m) { return m == 2 || m == 4 || m == 8 || m == 16; }
 
 // Workspace layout (all offsets 256-byte aligned):
-//   BUILD_FISHER:   header | S [groups][n] f32 | Y [groups][n][d_in] bf16
+//   BUILD_FISHER:   header | S [groups][n] f32 | M [n] f32 | pimax [groups] u32
+//                   | A [n][d_in] f16 | B [groups][n][d_in] f16
 //   QUANTIZE_ROWS:  header | status [d_out] i32
 //   INIT, OBJECTIVE: header
 struct FisherWs {
-    size_t s_off, y_off, total;
+    size_t s_off, m_off, pi_off, a_off, b_off, total;
 };
 static FisherWs fisher_ws(int64_t n, int64_t d_in, int groups)
 {
     FisherWs w;
     w.s_off = kWsHeader;
-    w.y_off = align_up(w.s_off + static_cast<size_t>(groups) * n * sizeof(float), 256);
-    w.total = align_up(w.y_off + static_cast<size_t>(groups) * n * d_in * 2, 256);
+    w.m_off = align_up(w.s_off + static_cast<size_t>(groups) * n * sizeof(float), 256);
+    w.pi_off = align_up(w.m_off + static_cast<size_t>(n) * sizeof(float), 256);
+    w.a_off = align_up(w.pi_off + static_cast<size_t>(groups) * sizeof(unsigned), 256);
+    w.b_off = align_up(w.a_off + static_cast<size_t>(n) * d_in * 2, 256);
+    w.total = align_up(w.b_off + static_cast<size_t>(groups) * n * d_in * 2, 256);
     return w;
 }
 
@@ -127,30 +134,36 @@ lnq_status lnq_build_fisher(const uint16_t *X, const uint16_t *G, int64_t n, int
     DeviceErr err{reinterpret_cast<uint32_t *>(base), g_wait_limit.load()};
     if (cudaMemsetAsync(base, 0, kWsHeader, s) != cudaSuccess)
         return LNQ_ERR_CUDA;
-    const __nv_bfloat16 *Y = reinterpret_cast<const __nv_bfloat16 *>(X);
+    const __nv_bfloat16 *Xb = reinterpret_cast<const __nv_bfloat16 *>(X);
+    cudaError_t e;
     if (G != nullptr) {
         float *S = reinterpret_cast<float *>(base + lay.s_off);
-        __nv_bfloat16 *Yw = reinterpret_cast<__nv_bfloat16 *>(base + lay.y_off);
-        const int64_t warps = n * groups;
+        float *M = reinterpret_cast<float *>(base + lay.m_off);
+        unsigned *pimax = reinterpret_cast<unsigned *>(base + lay.pi_off);
+        __half *A = reinterpret_cast<__half *>(base + lay.a_off);
+        __half *B = reinterpret_cast<__half *>(base + lay.b_off);
+        if (cudaMemsetAsync(pimax, 0, static_cast<size_t>(groups) * sizeof(unsigned), s) !=
+            cudaSuccess)
+            return LNQ_ERR_CUDA;
         const int threads = 256;
-        const int64_t blocks = (warps * 32 + threads - 1) / threads;
         {
-            KernelTimer timer("group_scales", s);
-            group_scales_kernel<<<static_cast<unsigned>(blocks), threads, 0, s>>>(
-                reinterpret_cast<const __nv_bfloat16 *>(G), n, d_out, groups, S);
+            KernelTimer timer("token_stats", s);
+            token_stats_kernel<<<static_cast<unsigned>((n * 32 + threads - 1) / threads), threads,
+                                 0, s>>>(Xb, reinterpret_cast<const __nv_bfloat16 *>(G), n, d_in,
+                                         d_out, groups, S, M, pimax);
         }
         const int64_t vecs = n * (d_in / 8);
         {
-            KernelTimer timer("scale_rows", s);
-            scale_rows_kernel<<<static_cast<unsigned>((vecs + threads - 1) / threads), threads, 0,
-                                s>>>(reinterpret_cast<const __nv_bfloat16 *>(X), S, n, d_in,
-                                     groups, Yw);
+            KernelTimer timer("guided_operands", s);
+            guided_operands_kernel<<<static_cast<unsigned>((vecs + threads - 1) / threads),
+                                     threads, 0, s>>>(Xb, S, M, pimax, n, d_in, groups, A, B);
         }
         if (cudaGetLastError() != cudaSuccess)
             return LNQ_ERR_CUDA;
-        Y = Yw;
+        e = fisher_syrk(A, B, true, pimax, n, d_in, groups, alpha, F, err, s, device_sm_count());
+    } else {
+        e = fisher_syrk(Xb, Xb, false, nullptr, n, d_in, 1, alpha, F, err, s, device_sm_count());
     }
-    cudaError_t e = fisher_syrk(Y, n, d_in, groups, alpha, F, err, s, device_sm_count());
     if (e == cudaErrorNotSupported)
         return LNQ_ERR_UNSUPPORTED;
     return e == cudaSuccess ? LNQ_OK : LNQ_ERR_CUDA;

@@ -7,6 +7,7 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -205,13 +206,13 @@ __device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t start, uint32_t lbo
     return d;
 }
 
-// Instruction descriptor for kind::f16 with bf16 A/B, fp32 D.
-__host__ __device__ constexpr uint32_t umma_idesc_bf16(int M, int N, bool a_mn_major,
-                                                       bool b_mn_major)
+// Instruction descriptor for kind::f16 with fp16 (f16 = true) or bf16 A/B and fp32 D.
+__host__ __device__ constexpr uint32_t umma_idesc_f16kind(int M, int N, bool a_mn_major,
+                                                          bool b_mn_major, bool f16)
 {
     return (1u << 4)                                // D format: f32
-           | (1u << 7)                              // A format: bf16
-           | (1u << 10)                             // B format: bf16
+           | ((f16 ? 0u : 1u) << 7)                 // A format: f16 = 0, bf16 = 1
+           | ((f16 ? 0u : 1u) << 10)                // B format (same type as A)
            | ((a_mn_major ? 1u : 0u) << 15)         // A major
            | ((b_mn_major ? 1u : 0u) << 16)         // B major
            | (static_cast<uint32_t>(N >> 3) << 17)  // N / 8

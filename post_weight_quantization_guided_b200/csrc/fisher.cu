@@ -5,40 +5,40 @@
 // F_j = (1/n) X^T diag(G_:,j^2) X) and the sentence after it (blocks are grouped and averaged
 // within each group, so F_g uses s_g[t] = mean_{j in g} G[t,j]^2).
 //
-// Three kernels:
-//   group_scales_kernel  s_g[t]: one warp per (token, group), 16-byte loads of G, fp32 sums.
-//   scale_rows_kernel    Y_g[t,:] = bf16(sqrt(s_g[t]) * X[t,:]) so that F_g = alpha * Y_g^T Y_g.
-//                        Skipped when G == NULL (then Y = X and s == 1).
-//   fisher_syrk_kernel   persistent tcgen05 GEMM over the upper-triangle tiles of every F_g.
-//                        TMA brings 64(t) x 64(i) bf16 boxes of Y_g into shared memory in the
-//                        128-byte-swizzled MN-major layout; one thread issues
-//                        tcgen05.mma.kind::f16 (M=128, N=256, K=16) into a TMEM accumulator;
-//                        four epilogue warps read TMEM, scale by alpha and write the tile and its
-//                        mirror image. Two TMEM accumulators let the epilogue of one tile overlap
-//                        the main loop of the next.
+// Kernels:
+//   token_stats_kernel      per token t: s_g[t] for every group (16-byte loads of G, fp32 sums),
+//                           M_t = max_i |X[t,i]|, and per group the maximum of s_g[t] M_t^2.
+//   guided_operands_kernel  A = X scaled by a power of two per token (exact in fp16) and
+//                           B_g = fp16(s_g * X) scaled by powers of two (one rounding, 2^-11
+//                           relative), so that F_g = alpha * Pi_g * A^T B_g. Keeping X exact on
+//                           one side and fp16 on the other bounds the error of every F entry by
+//                           about 5e-4 * sqrt(F_ii F_kk) even for a single token; bf16 on both
+//                           sides can reach 8e-3.
+//   fisher_syrk_kernel      persistent tcgen05 GEMM over the upper-triangle tiles of every F_g.
+//                           TMA brings 64(t) x 64(i) boxes of A and B_g into shared memory in the
+//                           128-byte-swizzled MN-major layout (no transpose of X is needed); one
+//                           thread issues tcgen05.mma.kind::f16 (M=128, N=256, K=16) into a TMEM
+//                           accumulator; four epilogue warps read TMEM, scale and write the tile
+//                           and its mirror image. Two TMEM accumulators let the epilogue of one
+//                           tile overlap the main loop of the next.
+// Without gradients (G == NULL) the product is X^T X: A = B = X in bf16, no preparation pass.
+#include <cuda_fp16.h>
+
 #include "common.cuh"
 #include "profile.cuh"
 
 namespace lnq {
 
 // ------------------------------------------------------------------------------------------
-// s_g reduction
+// Per-token statistics: s_g[t] and the row maximum M_t = max_i |X[t,i]|
 // ------------------------------------------------------------------------------------------
-__global__ void group_scales_kernel(const __nv_bfloat16 *__restrict__ G, int64_t n, int64_t d_out,
-                                    int groups, float *__restrict__ S)
+__device__ __forceinline__ float sum_squares_bf16(const __nv_bfloat16 *__restrict__ p, int64_t len,
+                                                  int lane)
 {
-    const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-    const int lane = threadIdx.x & 31;
-    if (warp >= n * groups)
-        return;
-    const int64_t t = warp / groups;
-    const int g = static_cast<int>(warp % groups);
-    const int64_t R = d_out / groups;
-    const __nv_bfloat16 *row = G + t * d_out + g * R;
     float acc = 0.f;
-    if ((reinterpret_cast<uintptr_t>(row) & 15u) == 0 && (R & 7) == 0) {
-        const uint4 *v = reinterpret_cast<const uint4 *>(row);
-        for (int64_t k = lane; k < R / 8; k += 32) {
+    if ((reinterpret_cast<uintptr_t>(p) & 15u) == 0 && (len & 7) == 0) {
+        const uint4 *v = reinterpret_cast<const uint4 *>(p);
+        for (int64_t k = lane; k < len / 8; k += 32) {
             uint4 x = __ldg(v + k);
             const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&x);
 #pragma unroll
@@ -49,21 +49,74 @@ __global__ void group_scales_kernel(const __nv_bfloat16 *__restrict__ G, int64_t
             }
         }
     } else {
-        for (int64_t k = lane; k < R; k += 32) {
-            float f = __bfloat162float(row[k]);
+        for (int64_t k = lane; k < len; k += 32) {
+            float f = __bfloat162float(p[k]);
             acc = fmaf(f, f, acc);
         }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1)
         acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    if (lane == 0)
-        S[static_cast<int64_t>(g) * n + t] = acc / static_cast<float>(R);
+    return acc;
 }
 
-// Y[g][t][:] = bf16(sqrt(S[g][t]) * X[t][:]); one thread per 8 consecutive elements of a row.
-__global__ void scale_rows_kernel(const __nv_bfloat16 *__restrict__ X, const float *__restrict__ S,
-                                  int64_t n, int64_t d, int groups, __nv_bfloat16 *__restrict__ Y)
+// One warp per token t: S[g][t] = mean_{j in g} G[t,j]^2 for every group, M[t] = max_i |X[t,i]|,
+// and pimax[g] = max over tokens of S[g][t] * M[t]^2 (positive floats compare as their bits).
+__global__ void token_stats_kernel(const __nv_bfloat16 *__restrict__ X,
+                                   const __nv_bfloat16 *__restrict__ G, int64_t n, int64_t d,
+                                   int64_t d_out, int groups, float *__restrict__ S,
+                                   float *__restrict__ M, unsigned *__restrict__ pimax)
+{
+    const int64_t t = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (t >= n)
+        return;
+    const uint4 *xv = reinterpret_cast<const uint4 *>(X + t * d);
+    float mx = 0.f;
+    for (int64_t k = lane; k < d / 8; k += 32) {
+        uint4 x = __ldg(xv + k);
+        const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&x);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            float2 f = __bfloat1622float2(h[e]);
+            mx = fmaxf(mx, fmaxf(fabsf(f.x), fabsf(f.y)));
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if (lane == 0)
+        M[t] = mx;
+    const int64_t R = d_out / groups;
+    for (int g = 0; g < groups; ++g) {
+        const float sg = sum_squares_bf16(G + t * d_out + g * R, R, lane) / static_cast<float>(R);
+        if (lane == 0) {
+            S[static_cast<int64_t>(g) * n + t] = sg;
+            atomicMax(&pimax[g], __float_as_uint(sg * mx * mx));
+        }
+    }
+}
+
+// Smallest power of two >= v for finite v > 0; 1 for v == 0.
+__device__ __forceinline__ float pow2_ceil(float v)
+{
+    if (!(v > 0.f))
+        return 1.f;
+    const unsigned u = __float_as_uint(v);
+    if ((u & 0x007FFFFFu) == 0u)
+        return v;
+    return __uint_as_float((u & 0x7F800000u) + 0x00800000u);
+}
+
+// Operands of the guided product, one thread per 8 consecutive elements of a token row:
+//   A[t][:]    = fp16(X[t][:] / P_t),                          P_t = pow2_ceil(M[t])  (exact)
+//   B[g][t][:] = fp16(X[t][:] * S[g][t] * P_t / Pi_g),         Pi_g = pow2_ceil(pimax[g])
+// so that A[t][i] * B[g][t][k] = s_g[t] X[t][i] X[t][k] / Pi_g with one fp16 rounding, |A| <= 1
+// and |B| <= 2. The GEMM epilogue multiplies by alpha * Pi_g.
+__global__ void guided_operands_kernel(const __nv_bfloat16 *__restrict__ X,
+                                       const float *__restrict__ S, const float *__restrict__ M,
+                                       const unsigned *__restrict__ pimax, int64_t n, int64_t d,
+                                       int groups, __half *__restrict__ A, __half *__restrict__ B)
 {
     const int64_t vec_per_row = d / 8;
     const int64_t v = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -76,14 +129,20 @@ __global__ void scale_rows_kernel(const __nv_bfloat16 *__restrict__ X, const flo
 #pragma unroll
     for (int e = 0; e < 4; ++e)
         f[e] = __bfloat1622float2(h[e]);
+    const float Pt = pow2_ceil(M[t]);
+    const float inv = 1.f / Pt;  // exact: Pt is a power of two
+    uint4 out;
+    __half2 *o = reinterpret_cast<__half2 *>(&out);
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+        o[e] = __floats2half2_rn(f[e].x * inv, f[e].y * inv);
+    reinterpret_cast<uint4 *>(A)[v] = out;
     for (int g = 0; g < groups; ++g) {
-        const float sc = sqrtf(S[static_cast<int64_t>(g) * n + t]);
-        uint4 out;
-        __nv_bfloat162 *o = reinterpret_cast<__nv_bfloat162 *>(&out);
+        const float factor = S[static_cast<int64_t>(g) * n + t] * Pt / pow2_ceil(__uint_as_float(pimax[g]));
 #pragma unroll
         for (int e = 0; e < 4; ++e)
-            o[e] = __floats2bfloat162_rn(sc * f[e].x, sc * f[e].y);
-        reinterpret_cast<uint4 *>(Y + static_cast<int64_t>(g) * n * d)[v] = out;
+            o[e] = __floats2half2_rn(f[e].x * factor, f[e].y * factor);
+        reinterpret_cast<uint4 *>(B + static_cast<int64_t>(g) * n * d)[v] = out;
     }
 }
 
@@ -103,11 +162,11 @@ constexpr int STAGE_BYTES = A_BYTES + B_BYTES;           // 48 KB
 constexpr int NUM_THREADS = 192;                         // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
 constexpr int TMEM_COLS = 2 * BN;                        // two accumulators
 constexpr size_t SMEM_BYTES = static_cast<size_t>(STAGES) * STAGE_BYTES + 1024 /*align*/ + 256;
-constexpr uint32_t IDESC = umma_idesc_bf16(BM, BN, /*a_mn_major=*/true, /*b_mn_major=*/true);
 }  // namespace syrk
 
 struct SyrkParams {
     float *F;            // [groups][d][d]
+    const unsigned *pimax;  // [groups] per-group operand scale (guided), or nullptr
     int64_t n, d;
     int groups;
     float alpha;
@@ -135,10 +194,14 @@ __device__ __forceinline__ void syrk_tile_coords(const SyrkParams &p, int tile, 
     bi = r;
 }
 
+template <bool kF16>
 __global__ void __launch_bounds__(syrk::NUM_THREADS, 1)
-    fisher_syrk_kernel(const __grid_constant__ CUtensorMap ymap, SyrkParams p)
+    fisher_syrk_kernel(const __grid_constant__ CUtensorMap amap,
+                       const __grid_constant__ CUtensorMap bmap, SyrkParams p)
 {
     using namespace syrk;
+    constexpr uint32_t IDESC = umma_idesc_f16kind(BM, BN, /*a_mn_major=*/true,
+                                                  /*b_mn_major=*/true, kF16);
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(align_up(reinterpret_cast<uintptr_t>(smem_raw), 1024));
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + STAGES * STAGE_BYTES);
@@ -163,7 +226,8 @@ __global__ void __launch_bounds__(syrk::NUM_THREADS, 1)
         }
         mbar_init(drain, 1);
         fence_barrier_init();
-        tma_prefetch_desc(&ymap);
+        tma_prefetch_desc(&amap);
+        tma_prefetch_desc(&bmap);
     }
     if (warp == 1)
         tmem_alloc(tmem_holder, TMEM_COLS);
@@ -196,9 +260,9 @@ __global__ void __launch_bounds__(syrk::NUM_THREADS, 1)
                     mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
                     const int t0 = kb * BK;
                     for (int b = 0; b < BM / BOX; ++b)
-                        tma_load_3d(sa + b * BOX_BYTES, &ymap, &full[stage], bi * BM + b * BOX, t0, g);
+                        tma_load_3d(sa + b * BOX_BYTES, &amap, &full[stage], bi * BM + b * BOX, t0, 0);
                     for (int b = 0; b < BN / BOX; ++b)
-                        tma_load_3d(sb + b * BOX_BYTES, &ymap, &full[stage], bk * BN + b * BOX, t0, g);
+                        tma_load_3d(sb + b * BOX_BYTES, &bmap, &full[stage], bk * BN + b * BOX, t0, g);
                     ++fills[stage];
                     stage = (stage + 1 == STAGES) ? 0 : stage + 1;
                 }
@@ -282,6 +346,8 @@ __global__ void __launch_bounds__(syrk::NUM_THREADS, 1)
             int g, bi, bk;
             syrk_tile_coords(p, tile, g, bi, bk);
             float *Fg = p.F + static_cast<int64_t>(g) * p.d * p.d;
+            const float scale =
+                p.pimax ? p.alpha * pow2_ceil(__uint_as_float(p.pimax[g])) : p.alpha;
             const int64_t i = static_cast<int64_t>(bi) * BM + row_in_tile;
             for (int chunk = 0; chunk < BN / 32; ++chunk) {
                 float v[32];
@@ -296,14 +362,14 @@ __global__ void __launch_bounds__(syrk::NUM_THREADS, 1)
 #pragma unroll
                         for (int e = 0; e < 32; e += 4)
                             *reinterpret_cast<float4 *>(rowp + k0 + e) =
-                                make_float4(p.alpha * v[e], p.alpha * v[e + 1],
-                                            p.alpha * v[e + 2], p.alpha * v[e + 3]);
+                                make_float4(scale * v[e], scale * v[e + 1],
+                                            scale * v[e + 2], scale * v[e + 3]);
                     } else {
 #pragma unroll
                         for (int e = 0; e < 32; ++e) {
                             const int64_t k = k0 + e;
                             if (k >= i && k < p.d)
-                                rowp[k] = p.alpha * v[e];
+                                rowp[k] = scale * v[e];
                         }
                     }
                     // the mirror: element (k, i) for k > i; lanes are consecutive i (coalesced)
@@ -311,7 +377,7 @@ __global__ void __launch_bounds__(syrk::NUM_THREADS, 1)
                     for (int e = 0; e < 32; ++e) {
                         const int64_t k = k0 + e;
                         if (k > i && k < p.d)
-                            Fg[k * p.d + i] = p.alpha * v[e];
+                            Fg[k * p.d + i] = scale * v[e];
                     }
                 }
             }
@@ -353,28 +419,41 @@ static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
     return fn;
 }
 
-// F_g = alpha * Y_g^T Y_g for Y [groups][n][d] bf16 (row-major), both triangles of F written.
-cudaError_t fisher_syrk(const __nv_bfloat16 *Y, int64_t n, int64_t d, int groups, float alpha,
-                        float *F, DeviceErr err, cudaStream_t s, int num_sms)
+static bool encode_operand(CUtensorMap *map, const void *base, int64_t n, int64_t d, int groups,
+                           bool f16)
 {
     using namespace syrk;
     auto encode = tensor_map_encoder();
     if (encode == nullptr)
-        return cudaErrorNotSupported;
-    CUtensorMap map;
+        return false;
     cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(n),
                           static_cast<cuuint64_t>(groups)};
     cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(n * d) * 2};
     cuuint32_t box[3] = {BOX, BK, 1};
     cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = encode(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<__nv_bfloat16 *>(Y),
-                        dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS)
+    return encode(map, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                  const_cast<void *>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// F_g = scale_g * A^T B_g, both triangles written, for A [n][d] and B [groups][n][d] (row-major):
+//   f16 == false: A = B = X in bf16 (groups == 1), scale = alpha;
+//   f16 == true:  the guided operands above, scale_g = alpha * pow2_ceil(pimax[g]).
+cudaError_t fisher_syrk(const void *A, const void *B, bool f16, const unsigned *pimax, int64_t n,
+                        int64_t d, int groups, float alpha, float *F, DeviceErr err,
+                        cudaStream_t s, int num_sms)
+{
+    using namespace syrk;
+    CUtensorMap amap, bmap;
+    if (tensor_map_encoder() == nullptr)
+        return cudaErrorNotSupported;
+    if (!encode_operand(&amap, A, n, d, 1, f16) || !encode_operand(&bmap, B, n, d, groups, f16))
         return cudaErrorInvalidValue;
     SyrkParams p;
     p.F = F;
+    p.pimax = pimax;
     p.n = n;
     p.d = d;
     p.groups = groups;
@@ -387,14 +466,14 @@ cudaError_t fisher_syrk(const __nv_bfloat16 *Y, int64_t n, int64_t d, int groups
     p.num_tiles = p.tiles_per_group * groups;
     p.err = err;
     const int grid = p.num_tiles < num_sms ? p.num_tiles : num_sms;
-    cudaError_t e = cudaFuncSetAttribute(fisher_syrk_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+    auto kernel = f16 ? fisher_syrk_kernel<true> : fisher_syrk_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(SMEM_BYTES));
     if (e != cudaSuccess)
         return e;
     {
         KernelTimer timer("fisher_syrk", s);
-        fisher_syrk_kernel<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(map, p);
+        kernel<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(amap, bmap, p);
     }
     return cudaGetLastError();
 }

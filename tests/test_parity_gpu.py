@@ -62,13 +62,13 @@ def test_fisher_unit_gradients_and_alpha(orc, lnq, wl):
     X, _, _ = wl.make_layer(layer, _dev())
     F0 = lnq.lnq_build_fisher(X, None, 1)
     ones = torch.ones((layer.n, layer.d_out), dtype=torch.bfloat16, device=_dev())
-    F1 = lnq.lnq_build_fisher(X, ones, 1)
+    F1 = lnq.lnq_build_fisher(X, ones, 1)       # the guided (fp16 operand) path with s == 1
     torch.cuda.synchronize()
-    assert torch.equal(F0, F1)            # sqrt(1) * x == x exactly
     Xh = X.double().cpu().numpy()
     ref = Xh.T @ Xh                        # library matmul, independent of the oracle
     dg = np.sqrt(np.outer(np.diag(ref), np.diag(ref)))
-    assert np.max(np.abs(F0[0].double().cpu().numpy() - ref) / dg) < 1e-5
+    assert np.max(np.abs(F0[0].double().cpu().numpy() - ref) / dg) < 1e-5   # exact bf16 inputs
+    assert np.max(np.abs(F1[0].double().cpu().numpy() - ref) / dg) < 1e-5   # power-of-2 scaling
     Fa = lnq.lnq_build_fisher(X, None, 1, alpha=1.0 / layer.n)
     check_fisher_full(orc, Fa, X, None, 1, alpha=1.0 / layer.n)
 
