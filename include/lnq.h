@@ -104,6 +104,30 @@ LNQ_API lnq_status lnq_build_fisher(const uint16_t *X, const uint16_t *G, int64_
                             int64_t d_out, int groups, float alpha, float *F, void *ws,
                             size_t ws_bytes, lnq_stream_t stream);
 
+/* Size in bytes of the static device scratch behind lnq_build_fisher_noalloc (64 MiB). */
+#define LNQ_NOALLOC_SCRATCH_BYTES (64ull << 20)
+
+/* lnq_build_fisher without a workspace argument. The pages have no counterpart: this entry point
+ * is an addition of this library, for callers that cannot allocate device memory at the moment
+ * they need F. Examples are a plugin with no allocator handle, code that runs inside another
+ * framework's fixed memory pool, or a latency-critical path that cannot afford the implicit
+ * synchronisation of cudaMalloc.
+ *   Scratch: a file-scope device array of LNQ_NOALLOC_SCRATCH_BYTES inside the library. Every GPU
+ *   that loads the library holds it until the process exits. The call itself allocates nothing
+ *   (no cudaMalloc, no cudaFree, no allocating library routine).
+ *   Set-up: the first call on each device looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current. Make that first call before any stream
+ *   capture, and call with the device that owns `stream` current.
+ *   Sharing: all calls share the one array, which keeps the last call's contents. Each call
+ *   clears what must start at zero and overwrites the rest, but calls that overlap on the GPU
+ *   (different streams or host threads) race on the array, so serialise them.
+ *   Arguments, results and requirements: as lnq_build_fisher. Returns LNQ_ERR_WORKSPACE, before
+ *   touching the device, when the problem needs more than LNQ_NOALLOC_SCRATCH_BYTES of scratch
+ *   (lnq_workspace_size(LNQ_OP_BUILD_FISHER, ...) bytes with G, 256 bytes without G). */
+LNQ_API lnq_status lnq_build_fisher_noalloc(const uint16_t *X, const uint16_t *G, int64_t n,
+                                            int64_t d_in, int64_t d_out, int groups, float alpha,
+                                            float *F, lnq_stream_t stream);
+
 /* Initial codebooks and assignments for every row (reading above).
  *   W  [d_out][d_in] fp32 in; C [d_out][m] fp32 out; Q [d_out][d_in] uint8 out
  * Requirements: m in {2, 4, 8, 16}; 1 <= d_in <= 16384; d_out >= 1. */

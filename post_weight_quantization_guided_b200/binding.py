@@ -22,7 +22,7 @@ LNQ_OP_BUILD_FISHER, LNQ_OP_INIT_CODEBOOK, LNQ_OP_QUANTIZE_ROWS, LNQ_OP_OBJECTIV
 
 EXPORTED = ("lnq_workspace_size", "lnq_build_fisher", "lnq_init_codebook", "lnq_quantize_rows",
             "lnq_objective", "lnq_workspace_check", "lnq_set_wait_limit", "lnq_status_string",
-            "lnq_profile_enable", "lnq_profile_read")
+            "lnq_profile_enable", "lnq_profile_read", "lnq_build_fisher_noalloc")
 
 _lib = None
 _VP, _I64, _INT, _SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
@@ -45,6 +45,8 @@ def lib():
         L.lnq_workspace_size.restype = _SZ
         L.lnq_build_fisher.argtypes = [_VP, _VP, _I64, _I64, _I64, _INT, ctypes.c_float, _VP,
                                        _VP, _SZ, _VP]
+        L.lnq_build_fisher_noalloc.argtypes = [_VP, _VP, _I64, _I64, _I64, _INT, ctypes.c_float,
+                                               _VP, _VP]
         L.lnq_init_codebook.argtypes = [_VP, _I64, _I64, _INT, _VP, _VP, _VP, _SZ, _VP]
         L.lnq_quantize_rows.argtypes = [_VP, _INT, _VP, _I64, _I64, _INT, _INT, _VP, _VP, _VP,
                                         _VP, _VP, _SZ, _VP]
@@ -61,7 +63,8 @@ def lib():
         L.lnq_profile_read.restype = _INT
         L.lnq_status_string.argtypes = [_INT]
         L.lnq_status_string.restype = ctypes.c_char_p
-        for name in ("lnq_build_fisher", "lnq_init_codebook", "lnq_quantize_rows",
+        for name in ("lnq_build_fisher", "lnq_build_fisher_noalloc", "lnq_init_codebook",
+                     "lnq_quantize_rows",
                      "lnq_objective", "lnq_workspace_check"):
             getattr(L, name).restype = _INT
         _lib = L
@@ -136,6 +139,24 @@ def lnq_build_fisher(X: torch.Tensor, G: Optional[torch.Tensor], groups: int, al
         ws = workspace(LNQ_OP_BUILD_FISHER, n, d_in, d_out, groups, device=X.device)
     _check(lib().lnq_build_fisher(_ptr(X), _ptr(G), n, d_in, d_out, groups, alpha, _ptr(F),
                                   _ptr(ws), ws.numel(), _stream(stream)), "lnq_build_fisher")
+    return F
+
+
+def lnq_build_fisher_noalloc(X: torch.Tensor, G: Optional[torch.Tensor], groups: int,
+                             alpha: float = 1.0, F: Optional[torch.Tensor] = None,
+                             stream=None) -> torch.Tensor:
+    """lnq_build_fisher with the library's static scratch instead of a workspace (F is still
+    caller memory; pass it in to keep the call free of any allocation)."""
+    n, d_in = X.shape
+    d_out = G.shape[1] if G is not None else groups
+    _need(X, torch.bfloat16, (n, d_in), "X")
+    if G is not None:
+        _need(G, torch.bfloat16, (n, d_out), "G")
+    if F is None:
+        F = torch.empty((groups, d_in, d_in), dtype=torch.float32, device=X.device)
+    _need(F, torch.float32, (groups, d_in, d_in), "F")
+    _check(lib().lnq_build_fisher_noalloc(_ptr(X), _ptr(G), n, d_in, d_out, groups, alpha,
+                                          _ptr(F), _stream(stream)), "lnq_build_fisher_noalloc")
     return F
 
 

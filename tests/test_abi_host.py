@@ -29,7 +29,7 @@ def test_header_declares_the_entry_points():
     assert names == sorted(["lnq_build_fisher", "lnq_init_codebook", "lnq_objective",
                             "lnq_quantize_rows", "lnq_set_wait_limit", "lnq_status_string",
                             "lnq_workspace_check", "lnq_workspace_size", "lnq_profile_enable",
-                            "lnq_profile_read"])
+                            "lnq_profile_read", "lnq_build_fisher_noalloc"])
 
 
 def test_library_exports_every_declared_symbol(L):
