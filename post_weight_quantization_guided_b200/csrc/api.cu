@@ -8,6 +8,7 @@
 #include <mutex>
 
 #include "common.cuh"
+#include "lnq_internal.cuh"
 #include "profile.cuh"
 
 namespace lnq {
@@ -21,14 +22,6 @@ __global__ void guided_operands_kernel(const __nv_bfloat16 *, const float *, con
 cudaError_t fisher_syrk(const void *A, const void *B, bool f16, const unsigned *pimax, int64_t n,
                         int64_t d, int groups, float alpha, float *F, DeviceErr err,
                         cudaStream_t s, int num_sms);
-cudaError_t lnq_init_launch(const float *W, int64_t d_out, int64_t d, int m, float *C,
-                            uint8_t *Q, cudaStream_t s);
-cudaError_t lnq_iterate_launch(const float *F, int groups, const float *W, int64_t d_out,
-                               int64_t d, int m, int iters, float *C, uint8_t *Q, double *J,
-                               int32_t *status, cudaStream_t s);
-cudaError_t lnq_objective_launch(const float *F, int groups, const float *W, const float *C,
-                                 const uint8_t *Q, int64_t d_out, int64_t d, int m, double *J,
-                                 cudaStream_t s);
 
 static std::atomic<long long> g_wait_limit{kDefaultWaitLimit};
 
@@ -48,8 +41,11 @@ static bool valid_m(int m) { return m == 2 || m == 4 || m == 8 || m == 16; }
 // Workspace layout (all offsets 256-byte aligned):
 //   BUILD_FISHER:   header | S [groups][n] f32 | M [n] f32 | pimax [groups] u32
 //                   | A [n][d_in] f16 | B [groups][n][d_in] f16
-//   QUANTIZE_ROWS:  header | status [d_out] i32
-//   INIT, OBJECTIVE: header
+//   QUANTIZE_ROWS:  header | status [d_out] i32 | Fp [groups][3][d_in][ld] bf16 (ld = d_in
+//                   rounded up to a multiple of 8)
+//                   | V [d_out][d_in][m] f32 | uT [d_in][d_out] f32 | dC [d_out][m] f32
+//   OBJECTIVE:      the same layout (status, V and dC unused)
+//   INIT:           header
 struct FisherWs {
     size_t s_off, m_off, pi_off, a_off, b_off, total;
 };
@@ -62,6 +58,34 @@ static FisherWs fisher_ws(int64_t n, int64_t d_in, int groups)
     w.a_off = align_up(w.pi_off + static_cast<size_t>(groups) * sizeof(unsigned), 256);
     w.b_off = align_up(w.a_off + static_cast<size_t>(n) * d_in * 2, 256);
     w.total = align_up(w.b_off + static_cast<size_t>(groups) * n * d_in * 2, 256);
+    return w;
+}
+
+struct LnqWs {
+    size_t st_off, fp_off, v_off, ut_off, dc_off, total;
+};
+static LnqWs lnq_ws(int64_t d_in, int64_t d_out, int groups, int m)
+{
+    LnqWs w;
+    w.st_off = kWsHeader;
+    w.fp_off = align_up(w.st_off + static_cast<size_t>(d_out) * 4, 256);
+    const size_t ld = static_cast<size_t>((d_in + 7) / 8 * 8);  // bf16 piece row stride
+    w.v_off = align_up(w.fp_off + static_cast<size_t>(groups) * 3 * d_in * ld * 2, 256);
+    w.ut_off = align_up(w.v_off + static_cast<size_t>(d_out) * d_in * m * 4, 256);
+    w.dc_off = align_up(w.ut_off + static_cast<size_t>(d_in) * d_out * 4, 256);
+    w.total = align_up(w.dc_off + static_cast<size_t>(d_out) * m * 4, 256);
+    return w;
+}
+
+static LnqWorkspace carve(void *ws, const LnqWs &lay)
+{
+    uint8_t *b = static_cast<uint8_t *>(ws);
+    LnqWorkspace w;
+    w.status = reinterpret_cast<int32_t *>(b + lay.st_off);
+    w.Fp = reinterpret_cast<__nv_bfloat16 *>(b + lay.fp_off);
+    w.V = reinterpret_cast<float *>(b + lay.v_off);
+    w.uT = reinterpret_cast<float *>(b + lay.ut_off);
+    w.dC = reinterpret_cast<float *>(b + lay.dc_off);
     return w;
 }
 
@@ -98,11 +122,11 @@ size_t lnq_workspace_size(lnq_op op, int64_t n, int64_t d_in, int64_t d_out, int
             return 0;
         return fisher_ws(n, d_in, groups).total;
     case LNQ_OP_QUANTIZE_ROWS:
-        if (d_out < 1)
-            return 0;
-        return align_up(kWsHeader + static_cast<size_t>(d_out) * sizeof(int32_t), 256);
-    case LNQ_OP_INIT_CODEBOOK:
     case LNQ_OP_OBJECTIVE:
+        if (d_out < 1 || d_in < 1 || groups < 1 || !valid_m(m))
+            return 0;
+        return lnq_ws(d_in, d_out, groups, m).total;
+    case LNQ_OP_INIT_CODEBOOK:
         return kWsHeader;
     }
     return 0;
@@ -191,21 +215,20 @@ lnq_status lnq_quantize_rows(const float *F, int groups, const float *W, int64_t
         d_out < 1 || d_out % groups != 0 || d_in < 1 || d_in > 16384 || !valid_m(m) ||
         iters < 0 || d_out > (int64_t(1) << 31) - 1)
         return LNQ_ERR_INVALID_ARG;
-    const size_t need = lnq_workspace_size(LNQ_OP_QUANTIZE_ROWS, 0, d_in, d_out, groups, m);
-    lnq_status st = check_ws(ws, ws_bytes, need);
+    const LnqWs lay = lnq_ws(d_in, d_out, groups, m);
+    lnq_status st = check_ws(ws, ws_bytes, lay.total);
     if (st != LNQ_OK)
         return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    uint8_t *base = static_cast<uint8_t *>(ws);
-    int32_t *status = reinterpret_cast<int32_t *>(base + kWsHeader);
-    if (cudaMemsetAsync(base, 0, kWsHeader + static_cast<size_t>(d_out) * sizeof(int32_t), s) !=
-        cudaSuccess)
+    const LnqWorkspace w = carve(ws, lay);
+    DeviceErr err{reinterpret_cast<uint32_t *>(ws), g_wait_limit.load()};
+    if (cudaMemsetAsync(ws, 0, lay.fp_off, s) != cudaSuccess)   // header and row status
         return LNQ_ERR_CUDA;
-    if (lnq_iterate_launch(F, groups, W, d_out, d_in, m, iters, C, Q, J_out, status, s) !=
-        cudaSuccess)
+    if (lnq_iterate_launch(F, groups, W, d_out, d_in, m, iters, C, Q, J_out, w, err,
+                           device_sm_count(), s) != cudaSuccess)
         return LNQ_ERR_CUDA;
     if (row_status != nullptr &&
-        cudaMemcpyAsync(row_status, status, static_cast<size_t>(d_out) * sizeof(int32_t),
+        cudaMemcpyAsync(row_status, w.status, static_cast<size_t>(d_out) * sizeof(int32_t),
                         cudaMemcpyDeviceToDevice, s) != cudaSuccess)
         return LNQ_ERR_CUDA;
     return LNQ_OK;
@@ -219,11 +242,19 @@ lnq_status lnq_objective(const float *F, int groups, const float *W, const float
         groups < 1 || d_out < 1 || d_out % groups != 0 || d_in < 1 || d_in > 16384 ||
         !valid_m(m) || d_out > (int64_t(1) << 31) - 1)
         return LNQ_ERR_INVALID_ARG;
-    lnq_status st = check_ws(ws, ws_bytes, kWsHeader);
+    const LnqWs lay = lnq_ws(d_in, d_out, groups, m);
+    lnq_status st = check_ws(ws, ws_bytes, lay.total);
     if (st != LNQ_OK)
         return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    return lnq_objective_launch(F, groups, W, C, Q, d_out, d_in, m, J, s) == cudaSuccess
+    const LnqWorkspace w = carve(ws, lay);
+    DeviceErr err{reinterpret_cast<uint32_t *>(ws), g_wait_limit.load()};
+    if (cudaMemsetAsync(ws, 0, kWsHeader, s) != cudaSuccess)
+        return LNQ_ERR_CUDA;
+    // iters = 0 with J requested: only the objective pass runs (C and Q are not modified).
+    return lnq_iterate_launch(F, groups, W, d_out, d_in, m, 0, const_cast<float *>(C),
+                              const_cast<uint8_t *>(Q), J, w, err, device_sm_count(),
+                              s) == cudaSuccess
                ? LNQ_OK
                : LNQ_ERR_CUDA;
 }

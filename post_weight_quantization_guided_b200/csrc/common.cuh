@@ -100,6 +100,25 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, long l
     return false;
 }
 
+// Named barrier among `n` threads (id 1..15; id 0 is __syncthreads).
+__device__ __forceinline__ void named_bar_sync(int id, int n)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
+// Named barrier that also ANDs a predicate over the `n` participating threads.
+__device__ __forceinline__ int named_bar_and(int id, int n, int pred)
+{
+    int out;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\tsetp.ne.b32 q, %1, 0;\n\t"
+        "bar.red.and.pred p, %2, %3, q;\n\tselp.b32 %0, 1, 0, p;\n\t}"
+        : "=r"(out)
+        : "r"(pred), "r"(id), "r"(n)
+        : "memory");
+    return out;
+}
+
 // ------------------------------------------------------------------------------------------
 // TMA (bulk tensor copies; plain loads, never multicast)
 // ------------------------------------------------------------------------------------------

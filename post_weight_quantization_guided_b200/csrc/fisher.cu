@@ -25,6 +25,7 @@
 #include <cuda_fp16.h>
 
 #include "common.cuh"
+#include "lnq_internal.cuh"
 #include "profile.cuh"
 
 namespace lnq {
@@ -404,7 +405,7 @@ __global__ void __launch_bounds__(syrk::NUM_THREADS, 1)
 
 namespace lnq {
 
-static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
 {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
     static std::once_flag once;

@@ -1,0 +1,48 @@
+// lnq_internal.cuh -- declarations shared between the library's translation units (not part of
+// the C ABI).
+#pragma once
+
+#include <cudaTypedefs.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+
+namespace lnq {
+
+// cuTensorMapEncodeTiled from the driver, looked up once; nullptr if unavailable.
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
+
+// Device scratch of lnq_quantize_rows / lnq_objective, carved from the caller's workspace.
+struct LnqWorkspace {
+    int32_t *status;     // [d_out] sticky per-row status
+    __nv_bfloat16 *Fp;   // [groups][3][d][d] bf16 pieces of F
+    float *V;            // [d_out][d][m]
+    float *uT;           // [d][d_out]
+    float *dC;           // [d_out][m]
+};
+
+// lnq.cu
+cudaError_t lnq_init_launch(const float *W, int64_t d_out, int64_t d, int m, float *C,
+                            uint8_t *Q, cudaStream_t s);
+cudaError_t lnq_iterate_launch(const float *F, int groups, const float *W, int64_t d_out,
+                               int64_t d, int m, int iters, float *C, uint8_t *Q, double *J,
+                               const LnqWorkspace &w, DeviceErr err, int num_sms, cudaStream_t s);
+
+// lnq_vgemm.cu
+cudaError_t lnq_split_f(const float *F, int64_t d, int groups, __nv_bfloat16 *Fp, cudaStream_t s);
+cudaError_t lnq_vgemm(const __nv_bfloat16 *Fp, int groups, const uint8_t *Q, const float *W,
+                      const float *C, float *V, float *uT, int64_t d, int64_t d_out, int m,
+                      bool residual_only, DeviceErr err, int num_sms, cudaStream_t s);
+
+// lnq_sweep.cu
+cudaError_t lnq_solve(const float *V, const float *uT, const uint8_t *Q, float *C, float *dC,
+                      int32_t *status, int64_t d, int64_t d_out, int m, cudaStream_t s);
+cudaError_t lnq_sweep(const float *F, int groups, const float *V, const float *dC, float *uT,
+                      const float *C, uint8_t *Q, int64_t d, int64_t d_out, int m,
+                      cudaStream_t s);
+cudaError_t lnq_objective_from_u(const float *uT, const float *W, const float *C,
+                                 const uint8_t *Q, double *J, int64_t d, int64_t d_out, int m,
+                                 cudaStream_t s);
+
+}  // namespace lnq

@@ -3,7 +3,10 @@
 Tolerances (per entry unless stated), from the accuracy targets of the hot path:
   F          |F_gpu - F_oracle| <= 1e-3 * sqrt(F_ii F_kk)  (bf16 operands, fp32 accumulation)
   codebook   |c_gpu - c_oracle| <= 1e-4 * max_q |c_oracle|  (per row)
-  objective  |J_gpu - J_oracle| <= 1e-5 * J_oracle
+  objective  |J_gpu - J_oracle(same state)| <= 1e-5 * J: the GPU's reported objective against
+             the oracle's objective of the GPU's own (C, Q). Along the trajectory the oracle keeps
+             its fp64 codebook, which may differ from the fp32 one within the codebook tolerance,
+             and J follows that difference to first order: there J agrees within 1e-4.
   indices    identical, except where the oracle's best two candidates are within 1e-6 * J
              (the oracle then follows the GPU's choice and counts it; any other difference is a
              mismatch and fails)
@@ -18,6 +21,7 @@ import torch
 F_TOL = 1e-3
 C_TOL = 1e-4
 J_TOL = 1e-5
+J_TRAJ_TOL = 1e-4
 TIE_TOL = 1e-6
 # Absolute floor of the tie band and of the objective tolerance, relative to the row's scale
 # w^T F w. It only matters when a row's objective reaches ~0 (an exactly representable row), where
@@ -108,7 +112,7 @@ def lnq_follow_parity(orc, lnq, F: torch.Tensor, W: torch.Tensor, m: int, iters:
     J = torch.empty(d_out, dtype=torch.float64, device=W.device)
     st = torch.empty(d_out, dtype=torch.int32, device=W.device)
     summary = {"follows": 0, "moves": 0, "rows": int(sum(len(r) for r in rows)),
-               "max_c_err": 0.0, "max_J_err": 0.0}
+               "max_c_err": 0.0, "max_J_err": 0.0, "max_J_same_state_err": 0.0}
     Fh = [None] * groups
     for it in range(iters):
         C0, Q0 = C.double().cpu().numpy(), Q.cpu().numpy()
@@ -131,10 +135,15 @@ def lnq_follow_parity(orc, lnq, F: torch.Tensor, W: torch.Tensor, m: int, iters:
             cscale = np.abs(Cf).max(axis=1, keepdims=True)
             cerr = float((np.abs(C1[r] - Cf) / cscale).max())
             jerr = float((np.abs(J1[r] - Jf) / (Jf + SCALE_FLOOR * Jw / J_TOL)).max())
+            # the oracle's objective of the GPU's own state (its fp32 codebook and assignment)
+            Js = np.array([orc.objective_row(Fh[g], Wh[jj], C1[jj], Q1[jj]) for jj in r])
+            serr = float((np.abs(J1[r] - Js) / (Js + SCALE_FLOOR * Jw / J_TOL)).max())
             assert cerr <= C_TOL, f"iteration {it} group {g}: codebook error {cerr:.3e}"
-            assert jerr <= J_TOL, f"iteration {it} group {g}: objective error {jerr:.3e}"
+            assert serr <= J_TOL, f"iteration {it} group {g}: objective error {serr:.3e}"
+            assert jerr <= J_TRAJ_TOL, f"iteration {it} group {g}: trajectory objective {jerr:.3e}"
             summary["follows"] += int(stats[:, 1].sum())
             summary["moves"] += int(stats[:, 0].sum())
             summary["max_c_err"] = max(summary["max_c_err"], cerr)
             summary["max_J_err"] = max(summary["max_J_err"], jerr)
+            summary["max_J_same_state_err"] = max(summary["max_J_same_state_err"], serr)
     return summary, C, Q
