@@ -26,7 +26,7 @@
 namespace lnq {
 
 constexpr int kSolveThreads = 256;
-constexpr int kSweepWarps = 16;
+constexpr int kSweepWarps = 8;
 constexpr int kObjWarps = 8;
 constexpr int kBlk = 32;
 
@@ -187,9 +187,9 @@ __global__ void __launch_bounds__(kSweepWarps * 32)
 {
     __shared__ float c_s[kBlk][M + 1];
     __shared__ float fblk[kBlk][kBlk + 1];
-    __shared__ float dl_s[kBlk][kBlk];
+    __shared__ __align__(16) float dl_s[kBlk][kBlk];
     __shared__ uint8_t qb_s[kBlk][kBlk + 4];
-    __shared__ int moved_s;
+    __shared__ unsigned moved_s;  // bit ii: some row moved at coordinate b0 + ii
 
     const int g = blockIdx.x / blocks_per_group;
     const int rb = blockIdx.x - g * blocks_per_group;
@@ -254,7 +254,7 @@ __global__ void __launch_bounds__(kSweepWarps * 32)
 #pragma unroll
             for (int ii = 0; ii < kBlk; ++ii)
                 ub[ii] = (valid && ii < nb) ? uT[(b0 + ii) * d_out + j] : 0.f;
-            int moved = 0;
+            unsigned colmask = 0u;
 #pragma unroll
             for (int ii = 0; ii < kBlk; ++ii) {
                 float dlt = 0.f;
@@ -274,69 +274,84 @@ __global__ void __launch_bounds__(kSweepWarps * 32)
                             best = a;
                         }
                     }
-                    if (best != qi) {
+                    if (best != qi) {  // a strictly negative Delta implies c[best] != cur
                         dlt = c_s[lane][best] - cur;
                         qb_s[lane][ii] = static_cast<uint8_t>(best);
-                        moved = 1;
                     }
                 }
 #pragma unroll
                 for (int i2 = ii + 1; i2 < kBlk; ++i2)
                     ub[i2] = fmaf(dlt, fblk[ii][i2], ub[i2]);
                 dl_s[ii][lane] = dlt;
+                colmask |= (__ballot_sync(0xffffffffu, dlt != 0.f) != 0u ? 1u : 0u) << ii;
             }
-            moved = __any_sync(0xffffffffu, moved);
             if (lane == 0)
-                moved_s = moved;
-            if (valid && moved) {
+                moved_s = colmask;
+            if (valid && colmask != 0u) {
                 for (int ii = 0; ii < nb; ++ii)
                     Q[j * d + b0 + ii] = qb_s[lane][ii];
             }
         }
         __syncthreads();
-        if (moved_s) {
-            float dl[kBlk];
+        const unsigned colmask = moved_s;
+        if (colmask != 0u) {
+            // Trailing update with one coordinate k per thread: the thread holds u[k] of the
+            // block's 32 rows and F[k][b0..b0+31], and adds sum_ii delta[ii][row] F[k][b0+ii] over
+            // the coordinates ii where some row moved (delta is read from shared memory as a
+            // broadcast). Every thread has 64 independent loads in flight.
+            const int nrows = static_cast<int>(row_end - row0);
+            for (int64_t k = b0 + nb + threadIdx.x; k < d; k += blockDim.x) {
+                float* urow = uT + k * d_out + row0;
+                const float *frow = Fg + k * d + b0;
+                float u[kBlk], f[kBlk];
+                const bool vec_u = nrows == kBlk && (reinterpret_cast<uintptr_t>(urow) & 15u) == 0;
+                const bool vec_f = nb == kBlk && (reinterpret_cast<uintptr_t>(frow) & 15u) == 0;
+                if (vec_u) {
 #pragma unroll
-            for (int ii = 0; ii < kBlk; ++ii)
-                dl[ii] = dl_s[ii][lane];
-            if (valid) {
-                const int64_t kfirst = b0 + nb + warp;
-                if (nb == kBlk && (d & 3) == 0) {
-                    // F[k][b0..b0+31] is one 128-byte line read by the whole warp (broadcast);
-                    // two coordinates per trip keep more loads in flight.
-                    for (int64_t k = kfirst; k < d; k += 2 * kSweepWarps) {
-                        const int64_t k2 = k + kSweepWarps;
-                        const bool has2 = k2 < d;
-                        const float4 *f1 = reinterpret_cast<const float4 *>(Fg + k * d + b0);
-                        const float4 *f2 = reinterpret_cast<const float4 *>(Fg + (has2 ? k2 : k) * d + b0);
-                        float a1 = uT[k * d_out + j];
-                        float a2 = has2 ? uT[k2 * d_out + j] : 0.f;
-#pragma unroll
-                        for (int v = 0; v < kBlk / 4; ++v) {
-                            const float4 x = f1[v], y = f2[v];
-                            a1 = fmaf(dl[4 * v], x.x, a1);
-                            a1 = fmaf(dl[4 * v + 1], x.y, a1);
-                            a1 = fmaf(dl[4 * v + 2], x.z, a1);
-                            a1 = fmaf(dl[4 * v + 3], x.w, a1);
-                            a2 = fmaf(dl[4 * v], y.x, a2);
-                            a2 = fmaf(dl[4 * v + 1], y.y, a2);
-                            a2 = fmaf(dl[4 * v + 2], y.z, a2);
-                            a2 = fmaf(dl[4 * v + 3], y.w, a2);
-                        }
-                        uT[k * d_out + j] = a1;
-                        if (has2)
-                            uT[k2 * d_out + j] = a2;
+                    for (int v = 0; v < kBlk / 4; ++v) {
+                        const float4 x = reinterpret_cast<const float4 *>(urow)[v];
+                        u[4 * v] = x.x; u[4 * v + 1] = x.y; u[4 * v + 2] = x.z; u[4 * v + 3] = x.w;
                     }
                 } else {
-                    for (int64_t k = kfirst; k < d; k += kSweepWarps) {
-                        const float *fk = Fg + k * d + b0;
-                        float acc = uT[k * d_out + j];
 #pragma unroll
-                        for (int ii = 0; ii < kBlk; ++ii)
-                            if (ii < nb)
-                                acc = fmaf(dl[ii], fk[ii], acc);
-                        uT[k * d_out + j] = acc;
+                    for (int r = 0; r < kBlk; ++r)
+                        u[r] = r < nrows ? urow[r] : 0.f;
+                }
+                if (vec_f) {
+#pragma unroll
+                    for (int v = 0; v < kBlk / 4; ++v) {
+                        const float4 x = reinterpret_cast<const float4 *>(frow)[v];
+                        f[4 * v] = x.x; f[4 * v + 1] = x.y; f[4 * v + 2] = x.z; f[4 * v + 3] = x.w;
                     }
+                } else {
+#pragma unroll
+                    for (int ii = 0; ii < kBlk; ++ii)
+                        f[ii] = ii < nb ? frow[ii] : 0.f;
+                }
+#pragma unroll
+                for (int ii = 0; ii < kBlk; ++ii) {
+                    if ((colmask >> ii) & 1u) {
+                        const float fi = f[ii];
+#pragma unroll
+                        for (int v = 0; v < kBlk / 4; ++v) {
+                            const float4 dd = *reinterpret_cast<const float4 *>(&dl_s[ii][4 * v]);
+                            u[4 * v] = fmaf(dd.x, fi, u[4 * v]);
+                            u[4 * v + 1] = fmaf(dd.y, fi, u[4 * v + 1]);
+                            u[4 * v + 2] = fmaf(dd.z, fi, u[4 * v + 2]);
+                            u[4 * v + 3] = fmaf(dd.w, fi, u[4 * v + 3]);
+                        }
+                    }
+                }
+                if (vec_u) {
+#pragma unroll
+                    for (int v = 0; v < kBlk / 4; ++v)
+                        reinterpret_cast<float4 *>(urow)[v] =
+                            make_float4(u[4 * v], u[4 * v + 1], u[4 * v + 2], u[4 * v + 3]);
+                } else {
+#pragma unroll
+                    for (int r = 0; r < kBlk; ++r)
+                        if (r < nrows)
+                            urow[r] = u[r];
                 }
             }
         }

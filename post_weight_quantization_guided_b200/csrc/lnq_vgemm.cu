@@ -30,24 +30,23 @@ namespace lnq {
 
 namespace vg {
 constexpr int BM = 128;
-constexpr int BN = 256;
 constexpr int BK = 64;
-constexpr int STAGES = 2;
 constexpr int PIECES = 3;
-constexpr int A_TILE = BM * BK * 2;              // 16 KB per piece
-constexpr int A_BYTES = PIECES * A_TILE;         // 48 KB
-constexpr int B_BYTES = BN * BK * 2;             // 32 KB
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;   // 80 KB
+constexpr int A_TILE = BM * BK * 2;              // one bf16 piece of a 128 x 64 F tile: 16 KB
+constexpr int B_STAGES = 2;
 constexpr int NUM_THREADS = 320;                 // w0 TMA, w1 MMA, w2-5 epilogue, w6-9 operand
 constexpr int PRODUCER_THREADS = 128;
-constexpr int TMEM_COLS = 2 * BN;
-constexpr size_t SMEM_BYTES = static_cast<size_t>(STAGES) * STAGE_BYTES + 1024 + 256 + 33 * 1024;
+constexpr int TMEM_COLS = 512;
+constexpr int MAX_DYN_SMEM = 232448;             // opt-in dynamic shared memory per block
+constexpr int BAR_BYTES = 512;
 }  // namespace vg
 
 // Tile shapes. With one-hot columns (M > 0) a tile is 256 columns and two TMEM accumulators
 // alternate between tiles. The residual-only product (M == 0) feeds the objective, which sums
 // r_i u_i with cancellation; there a tile is 128 columns and the K range is cut into four
 // segments with one accumulator each, so each fp32 accumulator takes a quarter of the additions.
+// Shared memory: A arrives one bf16 piece (16 KB) per slot, in as many slots as fit next to the two
+// right-operand stages and the staging area, so that several K blocks of F are in flight.
 template <int M>
 struct VgShape {
     static constexpr int NCOLS = M > 0 ? 256 : 128;     // MMA N
@@ -57,8 +56,16 @@ struct VgShape {
     static constexpr int ONEHOT = RT * M;               // one-hot columns
     static constexpr int USED = RT * (M + 3);           // columns carrying data
     static constexpr int CHUNKS = (USED + 31) / 32;     // 32-column TMEM loads per accumulator
-    static_assert(SETS * SEGS * NCOLS <= 512, "TMEM holds 512 fp32 columns");
-    static_assert(RT <= 64, "staging holds 64 rows");
+    static constexpr int B_BYTES = NCOLS * 128;         // N rows x 64 k of bf16
+    static constexpr int STG_BYTES = RT * 512;          // staging: classes, residual pieces, codebook
+    static constexpr int A_FIT = (vg::MAX_DYN_SMEM - 1024 - vg::BAR_BYTES -
+                                  vg::B_STAGES * B_BYTES - STG_BYTES) / vg::A_TILE;
+    static constexpr int A_SLOTS = A_FIT < 12 ? A_FIT : 12;
+    static constexpr size_t SMEM = 1024 + static_cast<size_t>(A_SLOTS) * vg::A_TILE +
+                                   vg::B_STAGES * B_BYTES + vg::BAR_BYTES + STG_BYTES;
+    static_assert(SETS * SEGS * NCOLS <= vg::TMEM_COLS, "TMEM holds 512 fp32 columns");
+    static_assert(A_SLOTS >= 2 * vg::PIECES, "at least two K blocks of F in flight");
+    static_assert(SMEM <= vg::MAX_DYN_SMEM, "shared memory");
 };
 
 __device__ __forceinline__ uint16_t bf16_bits(float x)
@@ -129,37 +136,12 @@ __device__ __forceinline__ void vg_tile_coords(const VgParams &p, int tile, int 
 //   q[r][kk]     class of coordinate k0+kk in row row0+r (0xFF outside the problem)
 //   rp[r][p][kk] bf16 piece p of the residual c[q] - w of that coordinate (0 outside)
 //   c[r][b]      codebook of row row0+r
-constexpr int kMaxRT = 64;
+template <int RT>
 struct VgStage {
-    uint8_t q[kMaxRT][64];
-    uint16_t rp[kMaxRT][3][64];
-    float c[kMaxRT][16];
+    uint8_t q[RT][64];
+    uint16_t rp[RT][3][64];
+    float c[RT][16];
 };
-
-// One 16-byte chunk (8 consecutive k) of row n of the right operand, from the staging area.
-template <int M>
-__device__ __forceinline__ uint4 vg_operand_chunk(const VgStage &st, int n, int c)
-{
-    constexpr int ONEHOT = VgShape<M>::ONEHOT, USED = VgShape<M>::USED;
-    if constexpr (M > 0) {
-        if (n < ONEHOT) {
-            const int r = n / M, b = n - (n / M) * M;
-            const uint2 qq = *reinterpret_cast<const uint2 *>(&st.q[r][8 * c]);
-            const uint32_t bbbb = 0x01010101u * static_cast<uint32_t>(b);
-            const uint32_t m0 = __vcmpeq4(qq.x, bbbb), m1 = __vcmpeq4(qq.y, bbbb);
-            // byte e of the mask (0xFF or 0) -> bf16 1.0 (0x3F80) or 0 in half-word e
-            return make_uint4(__byte_perm(m0, 0u, 0x1100) & 0x3F803F80u,
-                              __byte_perm(m0, 0u, 0x3322) & 0x3F803F80u,
-                              __byte_perm(m1, 0u, 0x1100) & 0x3F803F80u,
-                              __byte_perm(m1, 0u, 0x3322) & 0x3F803F80u);
-        }
-    }
-    if (n < USED) {
-        const int r = (n - ONEHOT) / 3, piece = (n - ONEHOT) - 3 * ((n - ONEHOT) / 3);
-        return *reinterpret_cast<const uint4 *>(&st.rp[r][piece][8 * c]);
-    }
-    return make_uint4(0u, 0u, 0u, 0u);
-}
 
 template <int M>
 __global__ void __launch_bounds__(vg::NUM_THREADS, 1)
@@ -167,28 +149,36 @@ __global__ void __launch_bounds__(vg::NUM_THREADS, 1)
 {
     using namespace vg;
     using S = VgShape<M>;
+    constexpr int NSLOT = S::A_SLOTS;
     constexpr uint32_t IDESC = umma_idesc_f16kind(BM, S::NCOLS, false, false, /*f16=*/false);
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(align_up(reinterpret_cast<uintptr_t>(smem_raw), 1024));
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + STAGES * STAGE_BYTES);
-    uint64_t *a_full = bars;                   // [STAGES]
-    uint64_t *b_full = bars + STAGES;          // [STAGES]
-    uint64_t *empty = bars + 2 * STAGES;       // [STAGES]
-    uint64_t *tfull = bars + 3 * STAGES;       // [2]
-    uint64_t *tempty = bars + 3 * STAGES + 2;  // [2]
-    uint64_t *drain = bars + 3 * STAGES + 4;
-    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + 3 * STAGES + 5);
-    VgStage &stg = *reinterpret_cast<VgStage *>(smem + STAGES * STAGE_BYTES + 256);
+    uint8_t *a_base = smem;                                       // [NSLOT][16 KB]
+    uint8_t *b_base = smem + NSLOT * A_TILE;                      // [B_STAGES][B_BYTES]
+    uint64_t *bars = reinterpret_cast<uint64_t *>(b_base + B_STAGES * S::B_BYTES);
+    uint64_t *a_full = bars;                                      // [NSLOT]
+    uint64_t *a_empty = a_full + NSLOT;                           // [NSLOT]
+    uint64_t *b_full = a_empty + NSLOT;                           // [B_STAGES]
+    uint64_t *b_empty = b_full + B_STAGES;                        // [B_STAGES]
+    uint64_t *tfull = b_empty + B_STAGES;                         // [SETS]
+    uint64_t *tempty = tfull + S::SETS;                           // [SETS]
+    uint64_t *drain = tempty + S::SETS;
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(drain + 1);
+    VgStage<S::RT> &stg = *reinterpret_cast<VgStage<S::RT> *>(
+        b_base + B_STAGES * S::B_BYTES + BAR_BYTES);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
-        for (int s = 0; s < STAGES; ++s) {
+        for (int s = 0; s < NSLOT; ++s) {
             mbar_init(&a_full[s], 1);
-            mbar_init(&b_full[s], PRODUCER_THREADS);
-            mbar_init(&empty[s], 1);
+            mbar_init(&a_empty[s], 1);
         }
-        for (int a = 0; a < 2; ++a) {
+        for (int s = 0; s < B_STAGES; ++s) {
+            mbar_init(&b_full[s], PRODUCER_THREADS);
+            mbar_init(&b_empty[s], 1);
+        }
+        for (int a = 0; a < S::SETS; ++a) {
             mbar_init(&tfull[a], 1);
             mbar_init(&tempty[a], 4 * 32);
         }
@@ -207,59 +197,84 @@ __global__ void __launch_bounds__(vg::NUM_THREADS, 1)
 
     if (warp == 0) {
         // ---------------------------------------------------------------- TMA: F pieces
+        // One 16 KB piece tile per slot, slots in round-robin order.
         if (lane == 0) {
-            int fills[STAGES] = {};
-            int stage = 0;
+            int fills[NSLOT] = {};
+            int slot = 0;
             bool ok = true;
             for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
                 int g, it;
                 int64_t row0, row_end;
                 vg_tile_coords<M>(p, tile, g, row0, row_end, it);
-                for (int kb = 0; kb < nk; ++kb) {
-                    if (!mbar_wait(&empty[stage], (fills[stage] & 1) ^ 1, limit)) {
-                        raise_error(p.err, kErrTimeout, 11);
-                        ok = false;
-                        break;
-                    }
-                    uint8_t *sa = smem + stage * STAGE_BYTES;
-                    mbar_arrive_expect_tx(&a_full[stage], A_BYTES);
-                    for (int pc = 0; pc < PIECES; ++pc)
-                        tma_load_3d(sa + pc * A_TILE, &fmap, &a_full[stage], kb * BK, it * BM,
+                for (int kb = 0; kb < nk && ok; ++kb) {
+                    for (int pc = 0; pc < PIECES; ++pc) {
+                        if (!mbar_wait(&a_empty[slot], (fills[slot] & 1) ^ 1, limit)) {
+                            raise_error(p.err, kErrTimeout, 11);
+                            ok = false;
+                            break;
+                        }
+                        mbar_arrive_expect_tx(&a_full[slot], A_TILE);
+                        tma_load_3d(a_base + slot * A_TILE, &fmap, &a_full[slot], kb * BK, it * BM,
                                     g * PIECES + pc);
-                    ++fills[stage];
-                    stage = (stage + 1 == STAGES) ? 0 : stage + 1;
+                        ++fills[slot];
+                        slot = (slot + 1 == NSLOT) ? 0 : slot + 1;
+                    }
                 }
             }
             if (!ok)
-                for (int s = 0; s < STAGES; ++s)
+                for (int s = 0; s < NSLOT; ++s)
                     if (fills[s] > 0)
                         mbar_wait(&a_full[s], (fills[s] - 1) & 1, kDrainLimit);
         }
     } else if (warp >= 6) {
         // ---------------------------------------------------------------- right operand
-        // Four warps stage the classes and the bf16 pieces of the residuals with coalesced loads
-        // (the next K block's loads are issued before this block's tile is expanded), then expand
-        // them into the swizzled bf16 tile. The stage wait is ANDed over the four warps, so they
-        // leave together on a timeout and the named barriers cannot deadlock.
+        // Four warps build the right operand of each K block in two phases, separated by a named
+        // barrier. Staging: each thread takes quads of 4 consecutive k of one row (prefetched into
+        // registers during the previous block) and writes the classes and the three bf16 pieces of
+        // the residuals. Expansion: each thread takes one (row, 16-byte column chunk): it reads the
+        // 8 classes once and writes the chunk of every one-hot row of that row, then copies residual
+        // chunks. Loads are issued before stores so that shared-memory accesses overlap. The stage
+        // wait is ANDed over the four warps, so they leave together on a timeout and the named
+        // barriers cannot deadlock. Columns beyond S::USED are never written: the epilogue ignores
+        // them.
         constexpr int kBar = 1;
-        constexpr int PER = (S::RT * 64 + PRODUCER_THREADS - 1) / PRODUCER_THREADS;
+        constexpr int QUADS = S::RT * 16;
+        constexpr int PER = (QUADS + PRODUCER_THREADS - 1) / PRODUCER_THREADS;
+        constexpr int PAIRS = S::RT * 8;
+        constexpr int RCH = 3 * S::RT * 8;  // residual chunks
+        constexpr int RPER = (RCH + PRODUCER_THREADS - 1) / PRODUCER_THREADS;
         const int t = threadIdx.x - 6 * 32;
-        int uses[STAGES] = {};
+        const bool vec = (p.d & 3) == 0 && (reinterpret_cast<uintptr_t>(p.Q) & 3u) == 0 &&
+                         (reinterpret_cast<uintptr_t>(p.W) & 15u) == 0;
+        int uses[B_STAGES] = {};
         int stage = 0;
         bool ok = true;
-        uint8_t qpre[PER];
-        float wpre[PER];
+        uint32_t qpre[PER];
+        float4 wpre[PER];
         auto fetch = [&](int64_t row0, int64_t row_end, int64_t k0) {
 #pragma unroll
             for (int s2 = 0; s2 < PER; ++s2) {
                 const int e = t + s2 * PRODUCER_THREADS;
-                const int r = e >> 6, kk = e & 63;
+                const int r = e >> 4, kk = (e & 15) * 4;
                 const int64_t j = row0 + r, k = k0 + kk;
-                qpre[s2] = 0xFFu;
-                wpre[s2] = 0.f;
-                if (e < S::RT * 64 && j < row_end && k < p.d) {
-                    qpre[s2] = static_cast<uint8_t>(p.Q[j * p.d + k] & (p.m - 1));
-                    wpre[s2] = p.W[j * p.d + k];
+                qpre[s2] = 0xFFFFFFFFu;
+                wpre[s2] = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (e < QUADS && j < row_end && k < p.d) {
+                    if (vec) {
+                        qpre[s2] = *reinterpret_cast<const uint32_t *>(p.Q + j * p.d + k);
+                        wpre[s2] = *reinterpret_cast<const float4 *>(p.W + j * p.d + k);
+                    } else {
+                        uint32_t qv = 0;
+                        float wv[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                        for (int e4 = 0; e4 < 4; ++e4) {
+                            const bool in = k + e4 < p.d;
+                            qv |= static_cast<uint32_t>(in ? p.Q[j * p.d + k + e4] : 0xFFu) << (8 * e4);
+                            wv[e4] = in ? p.W[j * p.d + k + e4] : 0.f;
+                        }
+                        qpre[s2] = qv;
+                        wpre[s2] = make_float4(wv[0], wv[1], wv[2], wv[3]);
+                    }
                 }
             }
         };
@@ -269,7 +284,7 @@ __global__ void __launch_bounds__(vg::NUM_THREADS, 1)
             vg_tile_coords<M>(p, tile, g, row0, row_end, it);
             fetch(row0, row_end, 0);
             for (int kb = 0; kb < nk; ++kb) {
-                const int mine = mbar_wait(&empty[stage], (uses[stage] & 1) ^ 1, limit) ? 1 : 0;
+                const int mine = mbar_wait(&b_empty[stage], (uses[stage] & 1) ^ 1, limit) ? 1 : 0;
                 if (!named_bar_and(kBar, PRODUCER_THREADS, mine)) {
                     if (t == 0)
                         raise_error(p.err, kErrTimeout, 12);
@@ -284,42 +299,102 @@ __global__ void __launch_bounds__(vg::NUM_THREADS, 1)
                     }
                     named_bar_sync(kBar, PRODUCER_THREADS);
                 }
+                // staging: classes and residual pieces of this K block
+                float cq[PER][4];
 #pragma unroll
                 for (int s2 = 0; s2 < PER; ++s2) {
                     const int e = t + s2 * PRODUCER_THREADS;
-                    if (e < S::RT * 64) {
-                        const int r = e >> 6, kk = e & 63;
-                        const uint8_t qv = qpre[s2];
-                        float p0 = 0.f, p1 = 0.f, p2 = 0.f;
-                        if (qv != 0xFFu)
-                            split3(stg.c[r][qv] - wpre[s2], p0, p1, p2);
-                        stg.q[r][kk] = qv;
-                        stg.rp[r][0][kk] = bf16_bits(p0);
-                        stg.rp[r][1][kk] = bf16_bits(p1);
-                        stg.rp[r][2][kk] = bf16_bits(p2);
+                    const int r = (e < QUADS) ? (e >> 4) : 0;
+#pragma unroll
+                    for (int e4 = 0; e4 < 4; ++e4) {
+                        const uint32_t qv = (qpre[s2] >> (8 * e4)) & 0xFFu;
+                        cq[s2][e4] = stg.c[r][(qv == 0xFFu ? 0u : qv) & (p.m - 1)];
+                    }
+                }
+#pragma unroll
+                for (int s2 = 0; s2 < PER; ++s2) {
+                    const int e = t + s2 * PRODUCER_THREADS;
+                    if (e < QUADS) {
+                        const int r = e >> 4, kk = (e & 15) * 4;
+                        const float wv[4] = {wpre[s2].x, wpre[s2].y, wpre[s2].z, wpre[s2].w};
+                        uint32_t pk[3][2] = {{0u, 0u}, {0u, 0u}, {0u, 0u}};
+                        uint32_t qmask = 0u;
+#pragma unroll
+                        for (int e4 = 0; e4 < 4; ++e4) {
+                            const uint32_t qv = (qpre[s2] >> (8 * e4)) & 0xFFu;
+                            float p0 = 0.f, p1 = 0.f, p2 = 0.f;
+                            if (qv != 0xFFu) {
+                                split3(cq[s2][e4] - wv[e4], p0, p1, p2);
+                                qmask |= (qv & (p.m - 1)) << (8 * e4);
+                            } else {
+                                qmask |= 0xFFu << (8 * e4);
+                            }
+                            pk[0][e4 >> 1] |= static_cast<uint32_t>(bf16_bits(p0)) << (16 * (e4 & 1));
+                            pk[1][e4 >> 1] |= static_cast<uint32_t>(bf16_bits(p1)) << (16 * (e4 & 1));
+                            pk[2][e4 >> 1] |= static_cast<uint32_t>(bf16_bits(p2)) << (16 * (e4 & 1));
+                        }
+                        *reinterpret_cast<uint32_t *>(&stg.q[r][kk]) = qmask;
+#pragma unroll
+                        for (int pc = 0; pc < 3; ++pc)
+                            *reinterpret_cast<uint2 *>(&stg.rp[r][pc][kk]) = make_uint2(pk[pc][0], pk[pc][1]);
                     }
                 }
                 if (kb + 1 < nk)
                     fetch(row0, row_end, static_cast<int64_t>(kb + 1) * BK);
                 named_bar_sync(kBar, PRODUCER_THREADS);
-                uint8_t *sb = smem + stage * STAGE_BYTES + A_BYTES;
-                for (int idx = t; idx < S::NCOLS * 8; idx += PRODUCER_THREADS) {
-                    const int n = idx >> 3, c = idx & 7;
-                    const uint4 v = vg_operand_chunk<M>(stg, n, c);
-                    *reinterpret_cast<uint4 *>(sb + n * 128 + ((c ^ (n & 7)) << 4)) = v;
+                // expansion into the swizzled K-major tile
+                uint8_t *sb = b_base + stage * S::B_BYTES;
+                if constexpr (M > 0) {
+                    for (int pi = t; pi < PAIRS; pi += PRODUCER_THREADS) {
+                        const int r = pi >> 3, c = pi & 7;
+                        const uint2 qq = *reinterpret_cast<const uint2 *>(&stg.q[r][8 * c]);
+#pragma unroll
+                        for (int b = 0; b < M; ++b) {
+                            const int n = r * M + b;
+                            const uint32_t bbbb = 0x01010101u * static_cast<uint32_t>(b);
+                            const uint32_t m0 = __vcmpeq4(qq.x, bbbb), m1 = __vcmpeq4(qq.y, bbbb);
+                            // byte e of the mask (0xFF or 0) -> bf16 1.0 (0x3F80) or 0, half-word e
+                            *reinterpret_cast<uint4 *>(sb + n * 128 + ((c ^ (n & 7)) << 4)) =
+                                make_uint4(__byte_perm(m0, 0u, 0x1100) & 0x3F803F80u,
+                                           __byte_perm(m0, 0u, 0x3322) & 0x3F803F80u,
+                                           __byte_perm(m1, 0u, 0x1100) & 0x3F803F80u,
+                                           __byte_perm(m1, 0u, 0x3322) & 0x3F803F80u);
+                        }
+                    }
+                }
+                {
+                    uint4 rv[RPER];
+#pragma unroll
+                    for (int s2 = 0; s2 < RPER; ++s2) {
+                        const int ci = t + s2 * PRODUCER_THREADS;
+                        const int nr = ci >> 3, c = ci & 7;   // nr = 3 r + piece
+                        if (ci < RCH)
+                            rv[s2] = *reinterpret_cast<const uint4 *>(&stg.rp[nr / 3][nr % 3][8 * c]);
+                    }
+#pragma unroll
+                    for (int s2 = 0; s2 < RPER; ++s2) {
+                        const int ci = t + s2 * PRODUCER_THREADS;
+                        const int nr = ci >> 3, c = ci & 7;
+                        const int n = S::ONEHOT + nr;
+                        if (ci < RCH)
+                            *reinterpret_cast<uint4 *>(sb + n * 128 + ((c ^ (n & 7)) << 4)) = rv[s2];
+                    }
                 }
                 // make the generic-proxy writes visible to the tensor core (async proxy)
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                 mbar_arrive(&b_full[stage]);
                 ++uses[stage];
-                stage = (stage + 1 == STAGES) ? 0 : stage + 1;
+                stage = (stage + 1 == B_STAGES) ? 0 : stage + 1;
             }
         }
     } else if (warp == 1) {
         // ---------------------------------------------------------------- MMA issuer
+        // Per K block: wait for the right operand, then for each piece wait for its A slot, issue
+        // four K=16 MMAs and release the slot; release the right-operand stage after the block.
         if (lane == 0) {
-            int stage = 0;
-            uint32_t phase[STAGES] = {};
+            int bstage = 0, slot = 0;
+            uint32_t bphase[B_STAGES] = {};
+            uint32_t aphase[NSLOT] = {};
             bool ok = true;
             int itn = 0;
             for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x, ++itn) {
@@ -331,38 +406,45 @@ __global__ void __launch_bounds__(vg::NUM_THREADS, 1)
                     break;
                 }
                 tc_fence_after();
-                for (int kb = 0; kb < nk; ++kb) {
-                    if (!mbar_wait(&a_full[stage], phase[stage], limit) ||
-                        !mbar_wait(&b_full[stage], phase[stage], limit)) {
+                for (int kb = 0; kb < nk && ok; ++kb) {
+                    if (!mbar_wait(&b_full[bstage], bphase[bstage], limit)) {
                         raise_error(p.err, kErrTimeout, 14);
                         ok = false;
                         break;
                     }
-                    phase[stage] ^= 1u;
-                    tc_fence_after();
+                    bphase[bstage] ^= 1u;
                     const int seg = (kb * S::SEGS) / nk;
                     const bool seg_start = (kb == 0) || (((kb - 1) * S::SEGS) / nk != seg);
                     const uint32_t d_tmem =
                         tmem_base + static_cast<uint32_t>((acc * S::SEGS + seg) * S::NCOLS);
-                    const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES);
-                    const uint32_t sb = sa + A_BYTES;
-#pragma unroll
+                    const uint32_t sb = smem_u32(b_base + bstage * S::B_BYTES);
                     for (int pc = 0; pc < PIECES; ++pc) {
+                        if (!mbar_wait(&a_full[slot], aphase[slot], limit)) {
+                            raise_error(p.err, kErrTimeout, 16);
+                            ok = false;
+                            break;
+                        }
+                        aphase[slot] ^= 1u;
+                        tc_fence_after();
+                        const uint32_t sa = smem_u32(a_base + slot * A_TILE);
 #pragma unroll
                         for (int kk = 0; kk < BK / 16; ++kk) {
                             // K-major, 128-byte swizzle: 16 k = 32 bytes along the row.
-                            const uint64_t ad = umma_desc_sw128(sa + pc * A_TILE + kk * 32, 16, 1024);
+                            const uint64_t ad = umma_desc_sw128(sa + kk * 32, 16, 1024);
                             const uint64_t bd = umma_desc_sw128(sb + kk * 32, 16, 1024);
-                            umma_f16(d_tmem, ad, bd, IDESC, (!seg_start || pc != 0 || kk != 0) ? 1u : 0u);
+                            umma_f16(d_tmem, ad, bd, IDESC,
+                                     (!seg_start || pc != 0 || kk != 0) ? 1u : 0u);
                         }
+                        umma_commit(&a_empty[slot]);
+                        slot = (slot + 1 == NSLOT) ? 0 : slot + 1;
                     }
-                    umma_commit(&empty[stage]);
-                    stage = (stage + 1 == STAGES) ? 0 : stage + 1;
+                    if (!ok)
+                        break;
+                    umma_commit(&b_empty[bstage]);
+                    bstage = (bstage + 1 == B_STAGES) ? 0 : bstage + 1;
                 }
                 if (!ok)
                     break;
-                // Segments that received no K block (tiny d) hold stale data: the epilogue only
-                // reads segments that started.
                 umma_commit(&tfull[acc]);
             }
             umma_commit(drain);
@@ -497,11 +579,11 @@ static cudaError_t launch_vgemm_m(const CUtensorMap &map, VgParams p, int num_sm
     const int grid = p.num_tiles < num_sms ? p.num_tiles : num_sms;
     cudaError_t e = cudaFuncSetAttribute(lnq_vgemm_kernel<M>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(vg::SMEM_BYTES));
+                                         static_cast<int>(S::SMEM));
     if (e != cudaSuccess)
         return e;
     KernelTimer timer(name, s);
-    lnq_vgemm_kernel<M><<<grid, vg::NUM_THREADS, vg::SMEM_BYTES, s>>>(map, p);
+    lnq_vgemm_kernel<M><<<grid, vg::NUM_THREADS, S::SMEM, s>>>(map, p);
     return cudaGetLastError();
 }
 
