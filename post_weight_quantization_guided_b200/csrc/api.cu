@@ -44,6 +44,7 @@ static bool valid_m(int m) { return m == 2 || m == 4 || m == 8 || m == 16; }
 //   QUANTIZE_ROWS:  header | status [d_out] i32 | Fp [groups][3][d_in][ld] bf16 (ld = d_in
 //                   rounded up to a multiple of 8)
 //                   | V [d_out][d_in][m] f32 | uT [d_in][d_out] f32 | dC [d_out][m] f32
+//                   | sweep history [CTAs][2 ceil(d_in / 128)][3][4 KB] (Delta pieces)
 //   OBJECTIVE:      the same layout (status, V and dC unused)
 //   INIT:           header
 struct FisherWs {
@@ -62,7 +63,7 @@ static FisherWs fisher_ws(int64_t n, int64_t d_in, int groups)
 }
 
 struct LnqWs {
-    size_t st_off, fp_off, v_off, ut_off, dc_off, total;
+    size_t st_off, fp_off, v_off, ut_off, dc_off, hist_off, total;
 };
 static LnqWs lnq_ws(int64_t d_in, int64_t d_out, int groups, int m)
 {
@@ -73,7 +74,8 @@ static LnqWs lnq_ws(int64_t d_in, int64_t d_out, int groups, int m)
     w.v_off = align_up(w.fp_off + static_cast<size_t>(groups) * 3 * d_in * ld * 2, 256);
     w.ut_off = align_up(w.v_off + static_cast<size_t>(d_out) * d_in * m * 4, 256);
     w.dc_off = align_up(w.ut_off + static_cast<size_t>(d_in) * d_out * 4, 256);
-    w.total = align_up(w.dc_off + static_cast<size_t>(d_out) * m * 4, 256);
+    w.hist_off = align_up(w.dc_off + static_cast<size_t>(d_out) * m * 4, 256);
+    w.total = align_up(w.hist_off + lnq_sweep_history_bytes(d_in, d_out, groups), 256);
     return w;
 }
 
@@ -86,6 +88,7 @@ static LnqWorkspace carve(void *ws, const LnqWs &lay)
     w.V = reinterpret_cast<float *>(b + lay.v_off);
     w.uT = reinterpret_cast<float *>(b + lay.ut_off);
     w.dC = reinterpret_cast<float *>(b + lay.dc_off);
+    w.hist = b + lay.hist_off;
     return w;
 }
 

@@ -20,6 +20,7 @@ struct LnqWorkspace {
     float *V;            // [d_out][d][m]
     float *uT;           // [d][d_out]
     float *dC;           // [d_out][m]
+    uint8_t *hist;       // sweep history, lnq_sweep_history_bytes()
 };
 
 // lnq.cu
@@ -30,19 +31,23 @@ cudaError_t lnq_iterate_launch(const float *F, int groups, const float *W, int64
                                const LnqWorkspace &w, DeviceErr err, int num_sms, cudaStream_t s);
 
 // lnq_vgemm.cu
+bool encode_f_pieces(CUtensorMap *map, const __nv_bfloat16 *Fp, int64_t d, int groups);
 cudaError_t lnq_split_f(const float *F, int64_t d, int groups, __nv_bfloat16 *Fp, cudaStream_t s);
 cudaError_t lnq_vgemm(const __nv_bfloat16 *Fp, int groups, const uint8_t *Q, const float *W,
                       const float *C, float *V, float *uT, int64_t d, int64_t d_out, int m,
                       bool residual_only, DeviceErr err, int num_sms, cudaStream_t s);
 
-// lnq_sweep.cu
+// lnq_solve.cu
 cudaError_t lnq_solve(const float *V, const float *uT, const uint8_t *Q, float *C, float *dC,
                       int32_t *status, int64_t d, int64_t d_out, int m, cudaStream_t s);
-cudaError_t lnq_sweep(const float *F, int groups, const float *V, const float *dC, float *uT,
-                      const float *C, uint8_t *Q, int64_t d, int64_t d_out, int m,
-                      cudaStream_t s);
 cudaError_t lnq_objective_from_u(const float *uT, const float *W, const float *C,
                                  const uint8_t *Q, double *J, int64_t d, int64_t d_out, int m,
                                  cudaStream_t s);
+
+// lnq_sweep.cu
+size_t lnq_sweep_history_bytes(int64_t d, int64_t d_out, int groups);
+cudaError_t lnq_sweep(const float *F, const __nv_bfloat16 *Fp, int groups, const float *V,
+                      const float *dC, const float *uT, const float *C, uint8_t *Q, uint8_t *hist,
+                      int64_t d, int64_t d_out, int m, DeviceErr err, cudaStream_t s);
 
 }  // namespace lnq

@@ -1,462 +1,683 @@
-// lnq_sweep.cu -- codebook solve, assignment sweep and objective of an LNQ iteration.
+// lnq_sweep.cu -- the assignment sweep of an LNQ iteration (coordinate descent) on sm_100a.
 //
-// Source: "GuidedQuant" (jinukkim.me blog), LNQ section: the codebook step
-// c <- (P^T F P)^-1 P^T F w and the assignment step "for i = 1..d_in: give coordinate i the
-// codeword minimising (w^ - w)^T F (w^ - w)".
+// Source: "GuidedQuant" (jinukkim.me blog), LNQ section: after the codebook update, coordinate
+// i = 1..d_in in turn takes the codeword minimising (w^ - w)^T F (w^ - w). With u = F r
+// (r = w^ - w), moving coordinate i by delta changes the objective by delta (2 u_i + delta F_ii)
+// and changes u by delta F[:, i].
 //
-// solve_kernel (one CTA per row). From V = F P and u = F r (lnq_vgemm.cu) it forms
-// M = P^T V and t = P^T u in fp64. The coordinates are sorted by class first (a stable
-// counting sort), and every sum runs in a fixed order, so results do not depend on scheduling.
-// An fp64 Cholesky over the non-empty codewords then solves M dc = -t (the closed-form update in
-// residual form), and the kernel writes c + dc in fp32 together with the exact fp32 change.
-//
-// sweep_kernel (one CTA per 32 rows of one group; lane = row). First u += V dc, so that u is
-// F r for the new codebook. Then it walks blocks of 32 coordinates in order. One warp takes the
-// block's decisions, coordinate after coordinate: candidate a changes the objective by
-// Delta_a = delta_a (2 u_i + delta_a F_ii), the best strictly negative Delta moves the
-// coordinate (lowest index on ties), and the block's later coordinates are corrected at once
-// from the 32 x 32 diagonal tile of F. Then all warps apply the block's moves to every later
-// coordinate, u[k] += sum_b delta_b F[k][b], skipping the update when no row moved.
-//
-// objective_kernel: J_j = r_j^T u_j with u = F r from the residual-only product, fp64 sums.
+// One CTA per 32 rows of one Fisher group. Coordinates are taken in windows of 128 (the height
+// of a tensor-core tile), each window in four blocks of 32.
+//   * Before a window starts, its u is assembled left-looking: the value at the start of the
+//     sweep, u0 + V dc (u0 = F r for the previous codebook and V = F P from lnq_vgemm, dc the
+//     codebook change from lnq_solve), plus F[window][earlier coordinates] x Delta[earlier
+//     coordinates], Delta being the moves made so far in this sweep. That product runs on tcgen05
+//     tensor cores: F as its three exact bf16 pieces (the operand lnq_vgemm uses), Delta as three
+//     exact bf16 pieces per value, and the six piece products of weight >= 2^-16 accumulate in
+//     fp32 in TMEM; the three dropped ones are below 2^-25 of |F_ki delta_i|.
+//   * Delta of finished windows is kept per CTA in a global history, already in the swizzled
+//     K-major layout the MMA reads, written and read back with byte-exact bulk copies.
+//   * The product for window T+1 over windows < T runs while window T is being decided; only the
+//     contribution of window T itself waits for its last decision.
+//   * Inside a window one warp (lane = row) decides a block of 32 coordinates, correcting the
+//     block's later coordinates in registers from the 32 x 32 diagonal tile of F; then four warps
+//     correct the window's later blocks in shared memory from a 32 x 128 strip of F.
+// Warp roles: 0 TMA and bulk copies, 1 MMA issue, 2-5 window assembly (TMEM -> shared memory),
+// 6-9 the sweep (6 decides; 6-9 correct). Every wait is bounded; a wait that gives up sets the
+// workspace error flag and its role stops, and every role drains what it has in flight.
 #include "common.cuh"
 #include "lnq_internal.cuh"
 #include "profile.cuh"
 
 namespace lnq {
 
-constexpr int kSolveThreads = 256;
-constexpr int kSweepWarps = 8;
-constexpr int kObjWarps = 8;
-constexpr int kBlk = 32;
+namespace sw {
+constexpr int RB = 32;                    // rows per CTA (MMA N)
+constexpr int WIN = 128;                  // coordinates per window (MMA M)
+constexpr int BLK = 32;                   // coordinates per decision block
+constexpr int NBLK = WIN / BLK;
+constexpr int CH = 64;                    // coordinates per K chunk: one 128-byte bf16 swizzle row
+constexpr int A_TILE = WIN * CH * 2;      // one bf16 piece of F[window][chunk]: 16 KB
+constexpr int H_PIECE = RB * CH * 2;      // one bf16 piece of Delta[chunk][rows]: 4 KB
+constexpr int H_CHUNK = 3 * H_PIECE;      // 12 KB
+constexpr int NA = 6;                     // F piece slots
+constexpr int NH = 2;                     // history chunk slots
+constexpr int UW_LD = WIN + 1;            // row stride (floats) of a window's u in shared memory
+constexpr int NUM_THREADS = 320;
+constexpr int SWEEP_THREADS = 128;
+constexpr int TMEM_COLS = 64;             // two fp32 accumulators of RB columns
+constexpr int MAX_WIN = 16384 / WIN;      // d_in <= 16384
+constexpr int SWEEP_BAR = 2;              // named barrier of the sweep warps
 
-// ------------------------------------------------------------------------------------------
-// codebook solve
-// ------------------------------------------------------------------------------------------
-template <int M>
-__global__ void __launch_bounds__(kSolveThreads)
-    solve_kernel(const float *__restrict__ V, const float *__restrict__ uT,
-                 const uint8_t *__restrict__ Q, float *__restrict__ C, float *__restrict__ dC,
-                 int32_t *__restrict__ status, int64_t d, int64_t d_out)
+// shared memory carve-up (bytes from a 1024-aligned base)
+constexpr int OFF_A = 0;
+constexpr int OFF_H = OFF_A + NA * A_TILE;
+constexpr int OFF_BS = OFF_H + NH * H_CHUNK;
+constexpr int OFF_STRIP = OFF_BS + 2 * H_CHUNK;
+constexpr int OFF_UW = OFF_STRIP + 2 * BLK * WIN * 4;
+constexpr int OFF_DL = OFF_UW + 2 * RB * UW_LD * 4;
+constexpr int OFF_C = OFF_DL + BLK * RB * 4;
+constexpr int OFF_DC = OFF_C + RB * 17 * 4;
+constexpr int OFF_QB = OFF_DC + RB * 16 * 4;
+constexpr int OFF_WM = OFF_QB + RB * (BLK + 4);
+constexpr int OFF_BAR = (OFF_WM + MAX_WIN + 7) / 8 * 8;
+constexpr int NBARS = 2 * NA + 2 * NH + 2 + 2 + 2 + 2 + 3;
+constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
+constexpr size_t SMEM = 1024 + OFF_MISC + 16;
+static_assert(SMEM <= 232448, "shared memory");
+static_assert(OFF_H % 1024 == 0 && OFF_BS % 1024 == 0, "swizzle atoms are 1024-byte aligned");
+}  // namespace sw
+
+struct SwParams {
+    const float *F;      // [groups][d][d]
+    const float *V;      // [d_out][d][m]
+    const float *dC;     // [d_out][m]
+    const float *uT;     // [d][d_out]
+    const float *C;      // [d_out][m]
+    uint8_t *Q;          // [d_out][d]
+    uint8_t *hist;       // [CTAs][2 * windows][3][4 KB]
+    int64_t d, d_out, rows_per_group;
+    int blocks_per_group, nwin;
+    DeviceErr err;
+};
+
+__device__ __forceinline__ uint32_t bf16_pair(float lo, float hi)
 {
-    constexpr int T = kSolveThreads;
-    constexpr int PAIRS = M * M;
-    constexpr int PPARTS = T / PAIRS;  // threads per (class, column) pair: 1, 4, 16, 64
-    constexpr int TPARTS = T / M;      // threads per class for t
-    extern __shared__ __align__(16) uint8_t sm[];
-    int *cnt = reinterpret_cast<int *>(sm);               // [T][M] per-thread class counts
-    int *list = cnt + T * M;                              // [d] class-sorted coordinates
-    __shared__ int start[M + 1];
-    __shared__ double Msum[PAIRS * PPARTS], tsum[M * TPARTS];
-    __shared__ double Mm[M * M], tv[M], L[M * M], y[M];
-
-    const int64_t j = blockIdx.x;
-    const int tid = threadIdx.x;
-    const uint8_t *q = Q + j * d;
-    const int64_t chunk = (d + T - 1) / T;
-    const int64_t lo = min(d, tid * chunk), hi = min(d, lo + chunk);
-
-    // 1. stable counting sort of the coordinates by class
-    for (int b = 0; b < M; ++b)
-        cnt[tid * M + b] = 0;
-    for (int64_t i = lo; i < hi; ++i)
-        cnt[tid * M + (q[i] & (M - 1))] += 1;
-    __syncthreads();
-    if (tid < M) {  // exclusive scan over threads, per class
-        int run = 0;
-        for (int t = 0; t < T; ++t) {
-            const int c = cnt[t * M + tid];
-            cnt[t * M + tid] = run;
-            run += c;
-        }
-        start[tid + 1] = run;  // class total, turned into starts below
-    }
-    __syncthreads();
-    if (tid == 0) {
-        start[0] = 0;
-        for (int b = 0; b < M; ++b)
-            start[b + 1] += start[b];
-    }
-    __syncthreads();
-    {
-        int off[M];
-#pragma unroll
-        for (int b = 0; b < M; ++b)
-            off[b] = start[b] + cnt[tid * M + b];
-        for (int64_t i = lo; i < hi; ++i) {
-            const int b = q[i] & (M - 1);
-#pragma unroll
-            for (int bb = 0; bb < M; ++bb)
-                if (bb == b)
-                    list[off[bb]++] = static_cast<int>(i);
-        }
-    }
-    __syncthreads();
-
-    // 2. M[a][b] = sum_{i in class a} V[i][b], t[a] = sum_{i in class a} u[i]  (fp64, fixed order)
-    {
-        const int pair = tid / PPARTS, part = tid % PPARTS;
-        const int a = pair / M, b = pair % M;
-        double acc = 0.0;
-        for (int e = start[a] + part; e < start[a + 1]; e += PPARTS)
-            acc += static_cast<double>(V[(j * d + list[e]) * M + b]);
-        Msum[pair * PPARTS + part] = acc;
-        const int ta = tid / TPARTS, tpart = tid % TPARTS;
-        double tacc = 0.0;
-        for (int e = start[ta] + tpart; e < start[ta + 1]; e += TPARTS)
-            tacc += static_cast<double>(uT[static_cast<int64_t>(list[e]) * d_out + j]);
-        tsum[ta * TPARTS + tpart] = tacc;
-    }
-    __syncthreads();
-    if (tid < PAIRS) {
-        double s = 0.0;
-        for (int part = 0; part < PPARTS; ++part)
-            s += Msum[tid * PPARTS + part];
-        Mm[tid] = s;
-    }
-    if (tid < M) {
-        double s = 0.0;
-        for (int part = 0; part < TPARTS; ++part)
-            s += tsum[tid * TPARTS + part];
-        tv[tid] = s;
-    }
-    __syncthreads();
-
-    // 3. Cholesky over the non-empty codewords, dc = -M^-1 t
-    if (tid == 0) {
-        int idx[M];
-        int nn = 0;
-        for (int b = 0; b < M; ++b)
-            if (start[b + 1] > start[b])
-                idx[nn++] = b;
-        bool singular = false;
-        for (int r = 0; r < nn && !singular; ++r) {
-            for (int c = 0; c <= r; ++c) {
-                double s = Mm[idx[r] * M + idx[c]];
-                for (int k = 0; k < c; ++k)
-                    s -= L[r * M + k] * L[c * M + k];
-                if (r == c) {
-                    if (!(s > 0.0)) {
-                        singular = true;
-                        break;
-                    }
-                    L[r * M + r] = sqrt(s);
-                } else {
-                    L[r * M + c] = s / L[c * M + c];
-                }
-            }
-        }
-        float *c = C + j * M;
-        float *dc = dC + j * M;
-        for (int b = 0; b < M; ++b)
-            dc[b] = 0.f;
-        if (singular) {
-            status[j] |= LNQ_ROW_SINGULAR;
-        } else {
-            for (int r = 0; r < nn; ++r) {
-                double s = -tv[idx[r]];
-                for (int k = 0; k < r; ++k)
-                    s -= L[r * M + k] * y[k];
-                y[r] = s / L[r * M + r];
-            }
-            for (int r = nn - 1; r >= 0; --r) {
-                double s = y[r];
-                for (int k = r + 1; k < nn; ++k)
-                    s -= L[k * M + r] * y[k];
-                y[r] = s / L[r * M + r];
-            }
-            for (int r = 0; r < nn; ++r) {
-                const float old = c[idx[r]];
-                const float nw = static_cast<float>(static_cast<double>(old) + y[r]);
-                c[idx[r]] = nw;
-                dc[idx[r]] = static_cast<float>(static_cast<double>(nw) - static_cast<double>(old));
-            }
-        }
-    }
+    return static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(lo))) |
+           (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(hi))) << 16);
 }
 
-// ------------------------------------------------------------------------------------------
-// assignment sweep
-// ------------------------------------------------------------------------------------------
-template <int M>
-__global__ void __launch_bounds__(kSweepWarps * 32)
-    sweep_kernel(const float *__restrict__ F, const float *__restrict__ V,
-                 const float *__restrict__ dC, float *__restrict__ uT,
-                 const float *__restrict__ C, uint8_t *__restrict__ Q, int64_t d, int64_t d_out,
-                 int64_t rows_per_group, int blocks_per_group)
+// The three bf16 pieces of x: x == p0 + p1 + p2 exactly for normal fp32 x.
+__device__ __forceinline__ void split3_sw(float x, float &p0, float &p1, float &p2)
 {
-    __shared__ float c_s[kBlk][M + 1];
-    __shared__ float fblk[kBlk][kBlk + 1];
-    __shared__ __align__(16) float dl_s[kBlk][kBlk];
-    __shared__ uint8_t qb_s[kBlk][kBlk + 4];
-    __shared__ unsigned moved_s;  // bit ii: some row moved at coordinate b0 + ii
+    p0 = __bfloat162float(__float2bfloat16_rn(x));
+    const float r1 = x - p0;
+    p1 = __bfloat162float(__float2bfloat16_rn(r1));
+    p2 = r1 - p1;
+}
 
-    const int g = blockIdx.x / blocks_per_group;
-    const int rb = blockIdx.x - g * blocks_per_group;
-    const int64_t gstart = static_cast<int64_t>(g) * rows_per_group;
-    const int64_t row0 = gstart + static_cast<int64_t>(rb) * kBlk;
-    const int64_t row_end = min(row0 + kBlk, gstart + rows_per_group);
-    const float *Fg = F + static_cast<int64_t>(g) * d * d;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t j = row0 + lane;
-    const bool valid = j < row_end;
+template <int M>
+__global__ void __launch_bounds__(sw::NUM_THREADS, 1)
+    sweep_kernel(const __grid_constant__ CUtensorMap fmap, SwParams p)
+{
+    using namespace sw;
+    constexpr uint32_t IDESC = umma_idesc_f16kind(WIN, RB, false, false, /*f16=*/false);
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(align_up(reinterpret_cast<uintptr_t>(smem_raw), 1024));
+    uint8_t *a_base = smem + OFF_A;                                  // [NA][16 KB]
+    uint8_t *h_base = smem + OFF_H;                                  // [NH][12 KB]
+    uint8_t *bs_base = smem + OFF_BS;                                // [2 chunks][3][4 KB]
+    float *strip = reinterpret_cast<float *>(smem + OFF_STRIP);      // [2][BLK][WIN]
+    float *uwb = reinterpret_cast<float *>(smem + OFF_UW);           // [2][RB][UW_LD]
+    float(*dl_s)[RB] = reinterpret_cast<float(*)[RB]>(smem + OFF_DL);       // [BLK][RB]
+    float(*c_s)[17] = reinterpret_cast<float(*)[17]>(smem + OFF_C);         // [RB][m]
+    float(*dc_s)[16] = reinterpret_cast<float(*)[16]>(smem + OFF_DC);       // [RB][m]
+    uint8_t(*qb_s)[BLK + 4] = reinterpret_cast<uint8_t(*)[BLK + 4]>(smem + OFF_QB);
+    volatile uint8_t *wmask = smem + OFF_WM;                         // [window]: some row moved
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
+    uint64_t *a_full = bars;
+    uint64_t *a_empty = a_full + NA;
+    uint64_t *h_full = a_empty + NA;
+    uint64_t *h_empty = h_full + NH;
+    uint64_t *acc_full = h_empty + NH;
+    uint64_t *acc_empty = acc_full + 2;
+    uint64_t *uw_ready = acc_empty + 2;
+    uint64_t *uw_free = uw_ready + 2;
+    uint64_t *bs_ready = uw_free + 2;
+    uint64_t *bs_free = bs_ready + 1;
+    uint64_t *drain = bs_free + 1;
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + OFF_MISC);
+    volatile unsigned *moved_s = reinterpret_cast<volatile unsigned *>(smem + OFF_MISC + 4);
 
-    for (int e = threadIdx.x; e < kBlk * M; e += blockDim.x) {
-        const int r = e / M, b = e % M;
-        c_s[r][b] = (row0 + r < row_end) ? C[(row0 + r) * M + b] : 0.f;
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int g = blockIdx.x / p.blocks_per_group;
+    const int rb = blockIdx.x - g * p.blocks_per_group;
+    const int64_t gstart = static_cast<int64_t>(g) * p.rows_per_group;
+    const int64_t row0 = gstart + static_cast<int64_t>(rb) * RB;
+    const int64_t row_end = min(row0 + RB, gstart + p.rows_per_group);
+    const int nrows = static_cast<int>(row_end - row0);
+    const int64_t d = p.d;
+    const int nwin = p.nwin;
+    uint8_t *hist = p.hist + static_cast<size_t>(blockIdx.x) * (2 * nwin) * H_CHUNK;
+    const long long limit = p.err.limit;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < NA; ++s) {
+            mbar_init(&a_full[s], 1);
+            mbar_init(&a_empty[s], 1);
+        }
+        for (int s = 0; s < NH; ++s) {
+            mbar_init(&h_full[s], 1);
+            mbar_init(&h_empty[s], 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&acc_full[s], 1);
+            mbar_init(&acc_empty[s], 128);
+            mbar_init(&uw_ready[s], 128);
+            mbar_init(&uw_free[s], SWEEP_THREADS);
+        }
+        mbar_init(bs_ready, 32);
+        mbar_init(bs_free, 2);
+        mbar_init(drain, 1);
+        fence_barrier_init();
+        tma_prefetch_desc(&fmap);
     }
-    // 0. u <- u + V dc for every coordinate (u then equals F r for the new codebook)
-    if (valid) {
-        float dc[M];
+    for (int e = threadIdx.x; e < RB * 16; e += blockDim.x) {
+        const int r = e >> 4, b = e & 15;
+        const bool in = r < nrows && b < M;
+        c_s[r][b] = in ? p.C[(row0 + r) * M + b] : 0.f;
+        dc_s[r][b] = in ? p.dC[(row0 + r) * M + b] : 0.f;
+    }
+    if (warp == 1)
+        tmem_alloc(tmem_holder, TMEM_COLS);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_holder;
+
+    if (warp == 0) {
+        // ---------------------------------------------------------------- TMA and bulk copies
+        // Pass T (window T's u): for each earlier window w <= T-2 that had a move, its two history
+        // chunks (Delta pieces) and the F pieces F[T][chunk]; then the F pieces of window T-1's two
+        // chunks (whose Delta the sweep is still producing). Then, once window T-1 is decided, its
+        // Delta pieces go from shared memory to the history.
+        if (lane == 0) {
+            int aslot = 0, hslot = 0;
+            // per slot: bit = parity of the number of fills, and whether it was ever filled
+            uint32_t apar = 0u, aused = 0u, hpar = 0u, hused = 0u;
+            int stored = 0, confirmed = 0;  // history chunks written / known complete
+            bool ok = true;
+            auto load_f = [&](int c, int T) -> bool {
+                for (int pc = 0; pc < 3; ++pc) {
+                    if (!mbar_wait(&a_empty[aslot], ((apar >> aslot) & 1u) ^ 1u, limit))
+                        return false;
+                    mbar_arrive_expect_tx(&a_full[aslot], A_TILE);
+                    tma_load_3d(a_base + aslot * A_TILE, &fmap, &a_full[aslot], c * CH, T * WIN,
+                                g * 3 + pc);
+                    apar ^= 1u << aslot;
+                    aused |= 1u << aslot;
+                    aslot = (aslot + 1 == NA) ? 0 : aslot + 1;
+                }
+                return true;
+            };
+            for (int T = 1; T < nwin && ok; ++T) {
+                for (int w = 0; w + 1 < T && ok; ++w) {
+                    if (!wmask[w])
+                        continue;
+                    for (int h = 0; h < 2 && ok; ++h) {
+                        const int c = 2 * w + h;
+                        if (c >= confirmed) {
+                            bulk_wait_all();
+                            confirmed = stored;
+                        }
+                        if (!mbar_wait(&h_empty[hslot], ((hpar >> hslot) & 1u) ^ 1u, limit)) {
+                            ok = false;
+                            break;
+                        }
+                        mbar_arrive_expect_tx(&h_full[hslot], H_CHUNK);
+                        bulk_load(h_base + hslot * H_CHUNK, hist + static_cast<size_t>(c) * H_CHUNK,
+                                  H_CHUNK, &h_full[hslot]);
+                        hpar ^= 1u << hslot;
+                        hused |= 1u << hslot;
+                        hslot = (hslot + 1 == NH) ? 0 : hslot + 1;
+                        ok = load_f(c, T);
+                    }
+                }
+                for (int h = 0; h < 2 && ok; ++h)
+                    ok = load_f(2 * (T - 1) + h, T);
+                if (ok && !mbar_wait(bs_ready, (T - 1) & 1, limit))
+                    ok = false;
+                if (!ok) {
+                    raise_error(p.err, kErrTimeout, 31);
+                    break;
+                }
+                if (wmask[T - 1]) {
+                    bulk_store(hist + static_cast<size_t>(2 * (T - 1)) * H_CHUNK, bs_base,
+                               2 * H_CHUNK);
+                    bulk_commit();
+                    stored = 2 * T;
+                    bulk_wait_read_all();
+                }
+                mbar_arrive(bs_free);
+            }
+            if (!ok) {
+                // the last fill of slot s completed phase (fills - 1), parity = fills parity ^ 1
+                for (int s = 0; s < NA; ++s)
+                    if ((aused >> s) & 1u)
+                        mbar_wait(&a_full[s], ((apar >> s) & 1u) ^ 1u, kDrainLimit);
+                for (int s = 0; s < NH; ++s)
+                    if ((hused >> s) & 1u)
+                        mbar_wait(&h_full[s], ((hpar >> s) & 1u) ^ 1u, kDrainLimit);
+            }
+            bulk_wait_all();
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------------------- MMA issue
+        // Accumulator T & 1 (32 TMEM columns, lane = coordinate of window T, column = row) gets
+        // sum over chunks c of F[T][c] x Delta[c], six piece products of four K=16 MMAs each.
+        if (lane == 0) {
+            int aslot = 0, hslot = 0;
+            uint32_t aph = 0u, hph = 0u, uses = 0u;  // bit per slot / accumulator: phase parity
+            bool ok = true;
+            for (int T = 1; T < nwin && ok; ++T) {
+                const int acc = T & 1;
+                if (!mbar_wait(&acc_empty[acc], ((uses >> acc) & 1u) ^ 1u, limit)) {
+                    raise_error(p.err, kErrTimeout, 32);
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * RB);
+                int n = 0;
+                auto chunk = [&](uint32_t b_addr, bool math) -> bool {
+                    for (int pa = 0; pa < 3; ++pa) {
+                        if (!mbar_wait(&a_full[aslot], (aph >> aslot) & 1u, limit))
+                            return false;
+                        aph ^= 1u << aslot;
+                        tc_fence_after();
+                        if (math) {
+                            const uint32_t sa = smem_u32(a_base + aslot * A_TILE);
+                            for (int pb = 0; pa + pb < 3; ++pb) {
 #pragma unroll
-        for (int b = 0; b < M; ++b)
-            dc[b] = dC[j * M + b];
-        const float *vj = V + j * d * M;
-#pragma unroll 2
-        for (int64_t k = warp; k < d; k += kSweepWarps) {
-            const float *vk = vj + k * M;
-            float acc = uT[k * d_out + j];
-            if constexpr (M >= 4) {
+                                for (int kk = 0; kk < CH / 16; ++kk) {
+                                    // K-major, 128-byte swizzle: 16 k = 32 bytes along the row
+                                    const uint64_t ad = umma_desc_sw128(sa + kk * 32, 16, 1024);
+                                    const uint64_t bd =
+                                        umma_desc_sw128(b_addr + pb * H_PIECE + kk * 32, 16, 1024);
+                                    umma_f16(d_tmem, ad, bd, IDESC, n > 0 ? 1u : 0u);
+                                    ++n;
+                                }
+                            }
+                        }
+                        umma_commit(&a_empty[aslot]);
+                        aslot = (aslot + 1 == NA) ? 0 : aslot + 1;
+                    }
+                    return true;
+                };
+                for (int w = 0; w + 1 < T && ok; ++w) {
+                    if (!wmask[w])
+                        continue;
+                    for (int h = 0; h < 2 && ok; ++h) {
+                        if (!mbar_wait(&h_full[hslot], (hph >> hslot) & 1u, limit)) {
+                            ok = false;
+                            break;
+                        }
+                        hph ^= 1u << hslot;
+                        ok = chunk(smem_u32(h_base + hslot * H_CHUNK), true);
+                        umma_commit(&h_empty[hslot]);
+                        hslot = (hslot + 1 == NH) ? 0 : hslot + 1;
+                    }
+                }
+                if (ok && !mbar_wait(bs_ready, (T - 1) & 1, limit))
+                    ok = false;
+                const bool mv = ok && wmask[T - 1] != 0;
+                for (int h = 0; h < 2 && ok; ++h)
+                    ok = chunk(smem_u32(bs_base + h * H_CHUNK), mv);
+                if (!ok) {
+                    raise_error(p.err, kErrTimeout, 33);
+                    break;
+                }
+                umma_commit(bs_free);
+                umma_commit(&acc_full[acc]);
+                uses ^= 1u << acc;
+            }
+            umma_commit(drain);
+            mbar_wait(drain, 0, kDrainLimit);
+        }
+    } else if (warp < 6) {
+        // ---------------------------------------------------------------- window assembly
+        // Thread = coordinate kl of the window (= TMEM lane; warp w reads lanes 32 (w % 4)..).
+        // u of window T for the CTA's rows: uT (F r for the previous codebook) + V dc, plus the
+        // accumulator of the moves made before the window, written to the window buffer T & 1.
+        const int quarter = warp & 3;
+        const int kl = quarter * 32 + lane;
+        uint32_t uses = 0u, wuses = 0u;  // bit per buffer: phase parity
+        bool anyw = false;
+        for (int T = 0; T < nwin; ++T) {
+            const int64_t k = static_cast<int64_t>(T) * WIN + kl;
+            const bool kin = k < d;
+            float u0[RB];
+            const float *ut = p.uT + k * p.d_out + row0;
+            if (kin && nrows == RB && (reinterpret_cast<uintptr_t>(ut) & 15u) == 0) {
 #pragma unroll
-                for (int b4 = 0; b4 < M / 4; ++b4) {
-                    const float4 v4 = reinterpret_cast<const float4 *>(vk)[b4];
-                    acc = fmaf(v4.x, dc[4 * b4], acc);
-                    acc = fmaf(v4.y, dc[4 * b4 + 1], acc);
-                    acc = fmaf(v4.z, dc[4 * b4 + 2], acc);
-                    acc = fmaf(v4.w, dc[4 * b4 + 3], acc);
+                for (int v = 0; v < RB / 4; ++v) {
+                    const float4 x = reinterpret_cast<const float4 *>(ut)[v];
+                    u0[4 * v] = x.x;
+                    u0[4 * v + 1] = x.y;
+                    u0[4 * v + 2] = x.z;
+                    u0[4 * v + 3] = x.w;
                 }
             } else {
 #pragma unroll
-                for (int b = 0; b < M; ++b)
-                    acc = fmaf(vk[b], dc[b], acc);
+                for (int r = 0; r < RB; ++r)
+                    u0[r] = (kin && r < nrows) ? ut[r] : 0.f;
             }
-            uT[k * d_out + j] = acc;
-        }
-    }
-    __syncthreads();
-    float c_reg[M];
+            if (kin) {
 #pragma unroll
-    for (int b = 0; b < M; ++b)
-        c_reg[b] = c_s[lane][b];
-
-    for (int64_t b0 = 0; b0 < d; b0 += kBlk) {
-        const int nb = (d - b0 < kBlk) ? static_cast<int>(d - b0) : kBlk;
-        // stage the diagonal tile of F and the block's codeword indices
-        for (int e = threadIdx.x; e < kBlk * kBlk; e += blockDim.x) {
-            const int r = e / kBlk, c = e % kBlk;
-            fblk[r][c] = (r < nb && c < nb) ? Fg[(b0 + r) * d + b0 + c] : 0.f;
-            const int64_t jr = row0 + r;
-            qb_s[r][c] = (jr < row_end && c < nb) ? (Q[jr * d + b0 + c] & (M - 1)) : 0;
-        }
-        __syncthreads();
-        if (warp == 0) {
-            float ub[kBlk];
+                for (int r = 0; r < RB; ++r) {
+                    if (r < nrows) {
+                        const float *vk = p.V + ((row0 + r) * d + k) * M;
+                        float acc = u0[r];
+                        if constexpr (M >= 4) {
 #pragma unroll
-            for (int ii = 0; ii < kBlk; ++ii)
-                ub[ii] = (valid && ii < nb) ? uT[(b0 + ii) * d_out + j] : 0.f;
-            unsigned colmask = 0u;
-#pragma unroll
-            for (int ii = 0; ii < kBlk; ++ii) {
-                float dlt = 0.f;
-                if (ii < nb && valid) {
-                    const int qi = qb_s[lane][ii];
-                    const float cur = c_s[lane][qi];
-                    const float fii = fblk[ii][ii];
-                    const float two_u = 2.f * ub[ii];
-                    int best = qi;
-                    float bestD = 0.f;
-#pragma unroll
-                    for (int a = 0; a < M; ++a) {
-                        const float da = c_reg[a] - cur;
-                        const float D = da * fmaf(da, fii, two_u);
-                        if (D < bestD) {
-                            bestD = D;
-                            best = a;
+                            for (int b4 = 0; b4 < M / 4; ++b4) {
+                                const float4 v4 = reinterpret_cast<const float4 *>(vk)[b4];
+                                acc = fmaf(v4.x, dc_s[r][4 * b4], acc);
+                                acc = fmaf(v4.y, dc_s[r][4 * b4 + 1], acc);
+                                acc = fmaf(v4.z, dc_s[r][4 * b4 + 2], acc);
+                                acc = fmaf(v4.w, dc_s[r][4 * b4 + 3], acc);
+                            }
+                        } else {
+                            const float2 v2 = *reinterpret_cast<const float2 *>(vk);
+                            acc = fmaf(v2.x, dc_s[r][0], acc);
+                            acc = fmaf(v2.y, dc_s[r][1], acc);
                         }
-                    }
-                    if (best != qi) {  // a strictly negative Delta implies c[best] != cur
-                        dlt = c_s[lane][best] - cur;
-                        qb_s[lane][ii] = static_cast<uint8_t>(best);
+                        u0[r] = acc;
                     }
                 }
-#pragma unroll
-                for (int i2 = ii + 1; i2 < kBlk; ++i2)
-                    ub[i2] = fmaf(dlt, fblk[ii][i2], ub[i2]);
-                dl_s[ii][lane] = dlt;
-                colmask |= (__ballot_sync(0xffffffffu, dlt != 0.f) != 0u ? 1u : 0u) << ii;
             }
+            if (T > 0) {
+                const int acc = T & 1;
+                int okw = 0;
+                if (lane == 0)
+                    okw = (mbar_wait(bs_ready, (T - 1) & 1, limit) &&
+                           mbar_wait(&acc_full[acc], (uses >> acc) & 1u, limit)) ? 1 : 0;
+                okw = __shfl_sync(0xffffffffu, okw, 0);
+                if (!okw) {
+                    if (lane == 0)
+                        raise_error(p.err, kErrTimeout, 34);
+                    break;
+                }
+                __syncwarp();
+                tc_fence_after();
+                uses ^= 1u << acc;
+                anyw = anyw || wmask[T - 1] != 0;
+                if (anyw) {
+                    float D[RB];
+                    tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
+                                           static_cast<uint32_t>(acc * RB),
+                                       D);
+#pragma unroll
+                    for (int r = 0; r < RB; ++r)
+                        u0[r] += D[r];
+                }
+                tc_fence_before();
+                mbar_arrive(&acc_empty[acc]);
+            }
+            const int buf = T & 1;
+            int okw = 0;
             if (lane == 0)
-                moved_s = colmask;
-            if (valid && colmask != 0u) {
-                for (int ii = 0; ii < nb; ++ii)
-                    Q[j * d + b0 + ii] = qb_s[lane][ii];
+                okw = mbar_wait(&uw_free[buf], ((wuses >> buf) & 1u) ^ 1u, limit) ? 1 : 0;
+            okw = __shfl_sync(0xffffffffu, okw, 0);
+            if (!okw) {
+                if (lane == 0)
+                    raise_error(p.err, kErrTimeout, 35);
+                break;
             }
+            __syncwarp();
+            wuses ^= 1u << buf;
+            float *uw = uwb + buf * (RB * UW_LD);
+#pragma unroll
+            for (int r = 0; r < RB; ++r)
+                uw[r * UW_LD + kl] = (kin && r < nrows) ? u0[r] : 0.f;
+            mbar_arrive(&uw_ready[buf]);
         }
-        __syncthreads();
-        const unsigned colmask = moved_s;
-        if (colmask != 0u) {
-            // Trailing update with one coordinate k per thread: the thread holds u[k] of the
-            // block's 32 rows and F[k][b0..b0+31], and adds sum_ii delta[ii][row] F[k][b0+ii] over
-            // the coordinates ii where some row moved (delta is read from shared memory as a
-            // broadcast). Every thread has 64 independent loads in flight.
-            const int nrows = static_cast<int>(row_end - row0);
-            for (int64_t k = b0 + nb + threadIdx.x; k < d; k += blockDim.x) {
-                float* urow = uT + k * d_out + row0;
-                const float *frow = Fg + k * d + b0;
-                float u[kBlk], f[kBlk];
-                const bool vec_u = nrows == kBlk && (reinterpret_cast<uintptr_t>(urow) & 15u) == 0;
-                const bool vec_f = nb == kBlk && (reinterpret_cast<uintptr_t>(frow) & 15u) == 0;
-                if (vec_u) {
+    } else {
+        // ---------------------------------------------------------------- the sweep
+        const int t = threadIdx.x - 6 * 32;  // 0..127
+        const bool decider = warp == 6;
+        const int64_t j = row0 + lane;
+        const bool valid = decider && lane < nrows;
+        const float *Fg = p.F + static_cast<int64_t>(g) * d * d;
+        const bool vecF = (d & 3) == 0 && (reinterpret_cast<uintptr_t>(p.F) & 15u) == 0;
+        float c_reg[M];
 #pragma unroll
-                    for (int v = 0; v < kBlk / 4; ++v) {
-                        const float4 x = reinterpret_cast<const float4 *>(urow)[v];
-                        u[4 * v] = x.x; u[4 * v + 1] = x.y; u[4 * v + 2] = x.z; u[4 * v + 3] = x.w;
-                    }
-                } else {
-#pragma unroll
-                    for (int r = 0; r < kBlk; ++r)
-                        u[r] = r < nrows ? urow[r] : 0.f;
+        for (int b = 0; b < M; ++b)
+            c_reg[b] = c_s[lane][b];
+        // F rows b0..b0+31, columns wstart..wstart+127 of the group (zero outside F) -> strip buf
+        auto load_strip = [&](int buf, int64_t b0, int64_t wstart) {
+            float *st = strip + buf * (BLK * WIN);
+            if (vecF) {
+                for (int e = t; e < BLK * WIN / 4; e += SWEEP_THREADS) {
+                    const int r = e / (WIN / 4), c4 = e % (WIN / 4);
+                    const int64_t row = b0 + r, col = wstart + 4 * c4;
+                    float *dst = st + r * WIN + 4 * c4;
+                    if (row < d && col < d)
+                        cp_async16(dst, Fg + row * d + col);
+                    else
+                        *reinterpret_cast<float4 *>(dst) = make_float4(0.f, 0.f, 0.f, 0.f);
                 }
-                if (vec_f) {
-#pragma unroll
-                    for (int v = 0; v < kBlk / 4; ++v) {
-                        const float4 x = reinterpret_cast<const float4 *>(frow)[v];
-                        f[4 * v] = x.x; f[4 * v + 1] = x.y; f[4 * v + 2] = x.z; f[4 * v + 3] = x.w;
-                    }
-                } else {
-#pragma unroll
-                    for (int ii = 0; ii < kBlk; ++ii)
-                        f[ii] = ii < nb ? frow[ii] : 0.f;
+                cp_async_commit();
+            } else {
+                for (int e = t; e < BLK * WIN; e += SWEEP_THREADS) {
+                    const int r = e / WIN, c = e % WIN;
+                    const int64_t row = b0 + r, col = wstart + c;
+                    st[r * WIN + c] = (row < d && col < d) ? Fg[row * d + col] : 0.f;
                 }
+            }
+        };
+        uint32_t wuses = 0u;  // bit per window buffer: phase parity
+        int bi = 0;  // block counter: the strip of block bi sits in buffer bi & 1
+        load_strip(0, 0, 0);
+        for (int T = 0; T < nwin; ++T) {
+            const int64_t wstart = static_cast<int64_t>(T) * WIN;
+            const int buf = T & 1;
+            const bool keep = T + 1 < nwin;  // later windows need this window's Delta
+            int mine = mbar_wait(&uw_ready[buf], (wuses >> buf) & 1u, limit) ? 1 : 0;
+            if (mine && T >= 1 && keep)
+                mine = mbar_wait(bs_free, (T - 1) & 1, limit) ? 1 : 0;
+            if (!named_bar_and(SWEEP_BAR, SWEEP_THREADS, mine)) {
+                if (t == 0)
+                    raise_error(p.err, kErrTimeout, 36);
+                break;
+            }
+            wuses ^= 1u << buf;
+            float *uw = uwb + buf * (RB * UW_LD);
+            bool wmoved = false;
+            for (int lb = 0; lb < NBLK; ++lb, ++bi) {
+                const int64_t b0 = wstart + lb * BLK;
+                if (b0 >= d)
+                    break;  // only in the last window
+                const int nb = (d - b0 < BLK) ? static_cast<int>(d - b0) : BLK;
+                cp_async_wait_all();
+                named_bar_sync(SWEEP_BAR, SWEEP_THREADS);  // strip of this block complete
+                {
+                    const int64_t nb0 = b0 + BLK;
+                    if (nb0 < d)
+                        load_strip((bi + 1) & 1, nb0, lb + 1 < NBLK ? wstart : wstart + WIN);
+                }
+                const float *st = strip + (bi & 1) * (BLK * WIN) + lb * BLK;  // st[ii * WIN + c]
+                if (decider) {
+                    // codes of the block for this row
+                    if (valid && nb == BLK && (d & 3) == 0 &&
+                        (reinterpret_cast<uintptr_t>(p.Q) & 3u) == 0) {
+                        const uint32_t *qs = reinterpret_cast<const uint32_t *>(p.Q + j * d + b0);
 #pragma unroll
-                for (int ii = 0; ii < kBlk; ++ii) {
-                    if ((colmask >> ii) & 1u) {
-                        const float fi = f[ii];
+                        for (int v = 0; v < BLK / 4; ++v)
+                            *reinterpret_cast<uint32_t *>(&qb_s[lane][4 * v]) = qs[v];
+                    } else {
+                        for (int ii = 0; ii < BLK; ++ii)
+                            qb_s[lane][ii] = (valid && ii < nb) ? p.Q[j * d + b0 + ii] : 0;
+                    }
+                    __syncwarp();
+                    float ub[BLK], dl[BLK];
 #pragma unroll
-                        for (int v = 0; v < kBlk / 4; ++v) {
-                            const float4 dd = *reinterpret_cast<const float4 *>(&dl_s[ii][4 * v]);
-                            u[4 * v] = fmaf(dd.x, fi, u[4 * v]);
-                            u[4 * v + 1] = fmaf(dd.y, fi, u[4 * v + 1]);
-                            u[4 * v + 2] = fmaf(dd.z, fi, u[4 * v + 2]);
-                            u[4 * v + 3] = fmaf(dd.w, fi, u[4 * v + 3]);
+                    for (int ii = 0; ii < BLK; ++ii)
+                        ub[ii] = uw[lane * UW_LD + lb * BLK + ii];
+                    unsigned colmask = 0u;
+#pragma unroll
+                    for (int ii = 0; ii < BLK; ++ii) {
+                        float dlt = 0.f;
+                        if (ii < nb && valid) {
+                            const int qi = qb_s[lane][ii] & (M - 1);
+                            const float cur = c_s[lane][qi];
+                            const float fii = st[ii * WIN + ii];
+                            const float two_u = 2.f * ub[ii];
+                            // Delta_a = delta_a (2 u + delta_a F_ii); staying is Delta 0; the lowest
+                            // index wins among equal strictly negative values
+                            int best = qi;
+                            float bestD = 0.f;
+#pragma unroll
+                            for (int a = 0; a < M; ++a) {
+                                const float da = c_reg[a] - cur;
+                                const float D = da * fmaf(da, fii, two_u);
+                                if (D < bestD) {
+                                    bestD = D;
+                                    best = a;
+                                }
+                            }
+                            if (best != qi) {  // a strictly negative Delta implies c[best] != cur
+                                dlt = c_s[lane][best] - cur;
+                                qb_s[lane][ii] = static_cast<uint8_t>(best);
+                            }
+                        }
+#pragma unroll
+                        for (int v = (ii + 1) / 4; v < BLK / 4; ++v) {
+                            const float4 f4 = *reinterpret_cast<const float4 *>(st + ii * WIN + 4 * v);
+                            if (4 * v > ii) ub[4 * v] = fmaf(dlt, f4.x, ub[4 * v]);
+                            if (4 * v + 1 > ii) ub[4 * v + 1] = fmaf(dlt, f4.y, ub[4 * v + 1]);
+                            if (4 * v + 2 > ii) ub[4 * v + 2] = fmaf(dlt, f4.z, ub[4 * v + 2]);
+                            if (4 * v + 3 > ii) ub[4 * v + 3] = fmaf(dlt, f4.w, ub[4 * v + 3]);
+                        }
+                        dl[ii] = dlt;
+                        dl_s[ii][lane] = dlt;
+                        colmask |= (__ballot_sync(0xffffffffu, dlt != 0.f) != 0u ? 1u : 0u) << ii;
+                    }
+                    if (lane == 0)
+                        *moved_s = colmask;
+                    wmoved = wmoved || colmask != 0u;
+                    if (valid && colmask != 0u) {
+                        for (int ii = 0; ii < nb; ++ii)
+                            p.Q[j * d + b0 + ii] = qb_s[lane][ii];
+                    }
+                    if (keep) {
+                        // Delta pieces of this block into the K-major, 128-byte-swizzled operand:
+                        // row = lane, K = 32 (lb & 1) + ii within chunk lb >> 1
+                        uint8_t *bs = bs_base + (lb >> 1) * H_CHUNK + lane * 128;
+#pragma unroll
+                        for (int cc = 0; cc < BLK / 8; ++cc) {
+                            uint32_t pk[3][4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                float a0, a1, a2, b0p, b1p, b2p;
+                                split3_sw(dl[8 * cc + 2 * e], a0, a1, a2);
+                                split3_sw(dl[8 * cc + 2 * e + 1], b0p, b1p, b2p);
+                                pk[0][e] = bf16_pair(a0, b0p);
+                                pk[1][e] = bf16_pair(a1, b1p);
+                                pk[2][e] = bf16_pair(a2, b2p);
+                            }
+                            const int chunk16 = (4 * (lb & 1) + cc) ^ (lane & 7);
+#pragma unroll
+                            for (int pc = 0; pc < 3; ++pc)
+                                *reinterpret_cast<uint4 *>(bs + pc * H_PIECE + chunk16 * 16) =
+                                    make_uint4(pk[pc][0], pk[pc][1], pk[pc][2], pk[pc][3]);
                         }
                     }
                 }
-                if (vec_u) {
+                named_bar_sync(SWEEP_BAR, SWEEP_THREADS);
+                const unsigned colmask = *moved_s;
+                const int kend = (d - wstart < WIN) ? static_cast<int>(d - wstart) : WIN;
+                if (colmask != 0u && (lb + 1) * BLK < kend) {
+                    // u[r][k] += sum_ii Delta[ii][r] F[b0 + ii][wstart + k] for the window's
+                    // later blocks; thread = (row, 4 consecutive k), F read as a broadcast
+                    const int r = t & 31, wq = t >> 5;
+                    const float *stw = strip + (bi & 1) * (BLK * WIN);
+                    float dr[BLK];
 #pragma unroll
-                    for (int v = 0; v < kBlk / 4; ++v)
-                        reinterpret_cast<float4 *>(urow)[v] =
-                            make_float4(u[4 * v], u[4 * v + 1], u[4 * v + 2], u[4 * v + 3]);
-                } else {
+                    for (int ii = 0; ii < BLK; ++ii)
+                        dr[ii] = dl_s[ii][r];
+                    for (int k0 = (lb + 1) * BLK + 4 * wq; k0 < kend; k0 += 16) {
+                        float a0 = uw[r * UW_LD + k0], a1 = uw[r * UW_LD + k0 + 1];
+                        float a2 = uw[r * UW_LD + k0 + 2], a3 = uw[r * UW_LD + k0 + 3];
 #pragma unroll
-                    for (int r = 0; r < kBlk; ++r)
-                        if (r < nrows)
-                            urow[r] = u[r];
+                        for (int ii = 0; ii < BLK; ++ii) {
+                            if ((colmask >> ii) & 1u) {
+                                const float4 f = *reinterpret_cast<const float4 *>(stw + ii * WIN + k0);
+                                a0 = fmaf(dr[ii], f.x, a0);
+                                a1 = fmaf(dr[ii], f.y, a1);
+                                a2 = fmaf(dr[ii], f.z, a2);
+                                a3 = fmaf(dr[ii], f.w, a3);
+                            }
+                        }
+                        uw[r * UW_LD + k0] = a0;
+                        uw[r * UW_LD + k0 + 1] = a1;
+                        uw[r * UW_LD + k0 + 2] = a2;
+                        uw[r * UW_LD + k0 + 3] = a3;
+                    }
+                }
+                named_bar_sync(SWEEP_BAR, SWEEP_THREADS);
+            }
+            if (decider) {
+                if (lane == 0)
+                    wmask[T] = wmoved ? 1 : 0;
+                if (keep) {
+                    fence_proxy_async_smem();
+                    mbar_arrive(bs_ready);
                 }
             }
+            mbar_arrive(&uw_free[buf]);
         }
-        __syncthreads();
+        cp_async_wait_all();
     }
-}
 
-// ------------------------------------------------------------------------------------------
-// objective J = r^T (F r)
-// ------------------------------------------------------------------------------------------
-template <int M>
-__global__ void __launch_bounds__(kObjWarps * 32)
-    objective_u_kernel(const float *__restrict__ uT, const float *__restrict__ W,
-                       const float *__restrict__ C, const uint8_t *__restrict__ Q,
-                       double *__restrict__ J, int64_t d, int64_t d_out)
-{
-    __shared__ double part[kObjWarps][32];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t j = static_cast<int64_t>(blockIdx.x) * 32 + lane;
-    double acc = 0.0;
-    if (j < d_out) {
-        for (int64_t i = warp; i < d; i += kObjWarps) {
-            const float r = C[j * M + (Q[j * d + i] & (M - 1))] - W[j * d + i];
-            acc += static_cast<double>(r) * static_cast<double>(uT[i * d_out + j]);
-        }
-    }
-    part[warp][lane] = acc;
+    tc_fence_before();
     __syncthreads();
-    if (warp == 0 && j < d_out) {
-        double s = 0.0;
-        for (int w = 0; w < kObjWarps; ++w)
-            s += part[w][lane];
-        J[j] = s;
-    }
+    tc_fence_after();
+    if (warp == 1)
+        tmem_dealloc(tmem_base, TMEM_COLS);
 }
 
 // ------------------------------------------------------------------------------------------
-// Host launchers
+// Host side
 // ------------------------------------------------------------------------------------------
-template <int M>
-static cudaError_t solve_m(const float *V, const float *uT, const uint8_t *Q, float *C, float *dC,
-                           int32_t *status, int64_t d, int64_t d_out, cudaStream_t s)
-{
-    const size_t smem = static_cast<size_t>(kSolveThreads) * M * 4 + static_cast<size_t>(d) * 4;
-    cudaError_t e = cudaFuncSetAttribute(solve_kernel<M>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
-    if (e != cudaSuccess)
-        return e;
-    KernelTimer timer("lnq_solve", s);
-    solve_kernel<M><<<static_cast<unsigned>(d_out), kSolveThreads, smem, s>>>(V, uT, Q, C, dC,
-                                                                              status, d, d_out);
-    return cudaGetLastError();
-}
-
-cudaError_t lnq_solve(const float *V, const float *uT, const uint8_t *Q, float *C, float *dC,
-                      int32_t *status, int64_t d, int64_t d_out, int m, cudaStream_t s)
-{
-    switch (m) {
-    case 2: return solve_m<2>(V, uT, Q, C, dC, status, d, d_out, s);
-    case 4: return solve_m<4>(V, uT, Q, C, dC, status, d, d_out, s);
-    case 8: return solve_m<8>(V, uT, Q, C, dC, status, d, d_out, s);
-    case 16: return solve_m<16>(V, uT, Q, C, dC, status, d, d_out, s);
-    }
-    return cudaErrorInvalidValue;
-}
-
-template <int M>
-static cudaError_t sweep_m(const float *F, int groups, const float *V, const float *dC, float *uT,
-                           const float *C, uint8_t *Q, int64_t d, int64_t d_out, cudaStream_t s)
+size_t lnq_sweep_history_bytes(int64_t d, int64_t d_out, int groups)
 {
     const int64_t R = d_out / groups;
-    const int bpg = static_cast<int>((R + kBlk - 1) / kBlk);
+    const int64_t ctas = groups * ((R + sw::RB - 1) / sw::RB);
+    const int64_t nwin = (d + sw::WIN - 1) / sw::WIN;
+    return static_cast<size_t>(ctas) * 2 * nwin * sw::H_CHUNK;
+}
+
+template <int M>
+static cudaError_t sweep_m(const CUtensorMap &map, const SwParams &p, unsigned grid, cudaStream_t s)
+{
+    cudaError_t e = cudaFuncSetAttribute(sweep_kernel<M>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(sw::SMEM));
+    if (e != cudaSuccess)
+        return e;
     KernelTimer timer("lnq_sweep", s);
-    sweep_kernel<M><<<static_cast<unsigned>(bpg * groups), kSweepWarps * 32, 0, s>>>(
-        F, V, dC, uT, C, Q, d, d_out, R, bpg);
+    sweep_kernel<M><<<grid, sw::NUM_THREADS, sw::SMEM, s>>>(map, p);
     return cudaGetLastError();
 }
 
-cudaError_t lnq_sweep(const float *F, int groups, const float *V, const float *dC, float *uT,
-                      const float *C, uint8_t *Q, int64_t d, int64_t d_out, int m, cudaStream_t s)
+cudaError_t lnq_sweep(const float *F, const __nv_bfloat16 *Fp, int groups, const float *V,
+                      const float *dC, const float *uT, const float *C, uint8_t *Q, uint8_t *hist,
+                      int64_t d, int64_t d_out, int m, DeviceErr err, cudaStream_t s)
 {
+    CUtensorMap map;
+    if (!encode_f_pieces(&map, Fp, d, groups))
+        return cudaErrorInvalidValue;
+    SwParams p{};
+    p.F = F;
+    p.V = V;
+    p.dC = dC;
+    p.uT = uT;
+    p.C = C;
+    p.Q = Q;
+    p.hist = hist;
+    p.d = d;
+    p.d_out = d_out;
+    p.rows_per_group = d_out / groups;
+    p.blocks_per_group = static_cast<int>((p.rows_per_group + sw::RB - 1) / sw::RB);
+    p.nwin = static_cast<int>((d + sw::WIN - 1) / sw::WIN);
+    p.err = err;
+    const unsigned grid = static_cast<unsigned>(p.blocks_per_group) * static_cast<unsigned>(groups);
     switch (m) {
-    case 2: return sweep_m<2>(F, groups, V, dC, uT, C, Q, d, d_out, s);
-    case 4: return sweep_m<4>(F, groups, V, dC, uT, C, Q, d, d_out, s);
-    case 8: return sweep_m<8>(F, groups, V, dC, uT, C, Q, d, d_out, s);
-    case 16: return sweep_m<16>(F, groups, V, dC, uT, C, Q, d, d_out, s);
+    case 2: return sweep_m<2>(map, p, grid, s);
+    case 4: return sweep_m<4>(map, p, grid, s);
+    case 8: return sweep_m<8>(map, p, grid, s);
+    case 16: return sweep_m<16>(map, p, grid, s);
     }
     return cudaErrorInvalidValue;
-}
-
-cudaError_t lnq_objective_from_u(const float *uT, const float *W, const float *C,
-                                 const uint8_t *Q, double *J, int64_t d, int64_t d_out, int m,
-                                 cudaStream_t s)
-{
-    const unsigned blocks = static_cast<unsigned>((d_out + 31) / 32);
-    KernelTimer timer("lnq_objective", s);
-    switch (m) {
-    case 2: objective_u_kernel<2><<<blocks, kObjWarps * 32, 0, s>>>(uT, W, C, Q, J, d, d_out); break;
-    case 4: objective_u_kernel<4><<<blocks, kObjWarps * 32, 0, s>>>(uT, W, C, Q, J, d, d_out); break;
-    case 8: objective_u_kernel<8><<<blocks, kObjWarps * 32, 0, s>>>(uT, W, C, Q, J, d, d_out); break;
-    case 16: objective_u_kernel<16><<<blocks, kObjWarps * 32, 0, s>>>(uT, W, C, Q, J, d, d_out); break;
-    default: return cudaErrorInvalidValue;
-    }
-    return cudaGetLastError();
 }
 
 }  // namespace lnq

@@ -550,7 +550,9 @@ cudaError_t lnq_split_f(const float *F, int64_t d, int groups, __nv_bfloat16 *Fp
     return cudaGetLastError();
 }
 
-static bool encode_pieces(CUtensorMap *map, const __nv_bfloat16 *Fp, int64_t d, int groups)
+// Tensor map over the pieces Fp [groups * 3][d][ld]: 64 x 128 (column x row) bf16 boxes,
+// 128-byte swizzle; reads outside d x d return zeros.
+bool encode_f_pieces(CUtensorMap *map, const __nv_bfloat16 *Fp, int64_t d, int groups)
 {
     auto encode = tensor_map_encoder();
     if (encode == nullptr)
@@ -593,7 +595,7 @@ cudaError_t lnq_vgemm(const __nv_bfloat16 *Fp, int groups, const uint8_t *Q, con
                       bool residual_only, DeviceErr err, int num_sms, cudaStream_t s)
 {
     CUtensorMap map;
-    if (!encode_pieces(&map, Fp, d, groups))
+    if (!encode_f_pieces(&map, Fp, d, groups))
         return cudaErrorInvalidValue;
     VgParams p{};
     p.Q = Q;
