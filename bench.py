@@ -118,14 +118,34 @@ def algorithmic_work(layer, kernel: str, launches: int, moves_per_sweep: float):
         return 2.0 * n * d * (2 + g) + 4.0 * n * (g + 1), "byte"   # read X, S, M; write A, B_g
     if kernel == "lnq_init":
         return 4.0 * dout * d + dout * d + 4.0 * dout * m, "byte"  # read W, write Q and C
-    if kernel == "lnq_codebook":
-        return 2.0 * dout * d * d, "lane_op"   # a class-bin add and an FMA per F entry per row
+    ld = (d + 7) // 8 * 8
+    if kernel == "lnq_split_f":
+        return 4.0 * g * d * d + 6.0 * g * d * ld, "byte"           # read F, write 3 bf16 pieces
+    if kernel == "lnq_vgemm":
+        # the dense product F x [P_j | r_j] over all rows: 2 d^2 (m + 1) flops per row
+        return 2.0 * d * d * (m + 1) * dout, "flop"
+    if kernel == "lnq_residual_gemm":
+        return 2.0 * d * d * dout, "flop"                           # u = F r for every row
+    if kernel == "lnq_solve":
+        return dout * (d * (4.0 * m + 4 + 1) + 8.0 * m), "byte"    # read V, uT, Q; write C, dC
     if kernel == "lnq_sweep":
-        # u = F r refresh (d^2 FMA per row) plus the trailing updates of the moved coordinates
-        return dout * (d * d + moves_per_sweep * d / 2.0), "lane_op"
+        # coordinate descent: the triangular u update d^2/2 FMA per row (the blocked scheme does
+        # it whenever a block moved) plus 2 d m for the candidates and the V dc refresh
+        return dout * (d * d / 2.0 + 2.0 * d * m), "lane_op"
     if kernel == "lnq_objective":
-        return 1.0 * dout * d * d, "lane_op"
+        return dout * d * (4.0 + 4 + 1), "byte"                     # read uT, W, Q
     return 0.0, "unknown"
+
+
+# tcgen05 work per unit of algorithmic work: F enters as three exact bf16 pieces; the one-hot
+# columns are exact, the residual columns are three pieces as well (nine products).
+def hw_flop_factor(layer, kernel):
+    m = layer.m
+    if kernel == "lnq_vgemm":
+        return (3.0 * m + 9.0) / (m + 1)
+    if kernel == "lnq_residual_gemm":
+        return 9.0
+    return None
 
 
 def roofline_for(kernel, per_launch_work, unit, avg_ms, peaks, clocks, num_sms):
@@ -307,6 +327,10 @@ def run_ours(args, rank, world, device):
                          "share": ms / sum(v[1] for v in prof.values()),
                          "roofline": roofline_for(name, per_launch, unit, avg, peaks, clocks,
                                                   num_sms)}
+        hf = hw_flop_factor(layer, name)
+        if hf is not None:
+            kernels[name]["roofline"]["hw_flop_factor"] = hf
+            kernels[name]["roofline"]["hw_frac"] = kernels[name]["roofline"]["frac"] * hf
     dominant = max(kernels, key=lambda k: kernels[k]["share"])
     roof = dict(kernels[dominant]["roofline"])
     roof["kernel"] = dominant

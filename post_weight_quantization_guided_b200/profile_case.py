@@ -1,0 +1,45 @@
+"""One small run of the whole path for profiler captures.
+
+    python -m post_weight_quantization_guided_b200.profile_case --workload q_proj --rows 1024
+
+builds the guided Fisher blocks, initialises the codebooks and runs `--iters` LNQ iterations plus
+the objective on a named synthetic workload, optionally with fewer output rows (`--rows`, a
+multiple of the group count) so that a capture stays small. It prints the objective's sum so that
+a run can be checked to have completed.
+"""
+from __future__ import annotations
+
+import argparse
+
+import torch
+
+from . import binding as api
+from . import workloads as wl
+
+WORKLOADS = {"tiny": wl.TINY, "q_proj": wl.Q_PROJ, "down_proj": wl.DOWN_PROJ, "up_proj": wl.UP_PROJ}
+
+
+def main(argv=None) -> None:
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--workload", default="q_proj", choices=sorted(WORKLOADS))
+    ap.add_argument("--rows", type=int, default=0, help="output rows (default: the workload's)")
+    ap.add_argument("--iters", type=int, default=1)
+    args = ap.parse_args(argv)
+    layer = WORKLOADS[args.workload]
+    if args.rows:
+        if args.rows % layer.groups:
+            raise SystemExit(f"--rows must be a multiple of {layer.groups}")
+        layer = wl.scaled(layer, d_out=args.rows)
+    dev = torch.device("cuda:0")
+    X, G, W = wl.make_layer(layer, dev)
+    F = api.lnq_build_fisher(X, G, layer.groups)
+    C, Q = api.lnq_init_codebook(W, layer.m)
+    J = torch.empty(layer.d_out, dtype=torch.float64, device=dev)
+    st = torch.empty(layer.d_out, dtype=torch.int32, device=dev)
+    api.lnq_quantize_rows(F, W, layer.m, args.iters, C, Q, J, st)
+    torch.cuda.synchronize()
+    print(f"{layer.name} rows={layer.d_out} iters={args.iters} sum(J)={float(J.sum()):.6e}")
+
+
+if __name__ == "__main__":
+    main()
