@@ -33,9 +33,9 @@ constexpr int BM = 128;
 constexpr int BK = 64;
 constexpr int PIECES = 3;
 constexpr int A_TILE = BM * BK * 2;              // one bf16 piece of a 128 x 64 F tile: 16 KB
-constexpr int B_STAGES = 2;
-constexpr int NUM_THREADS = 320;                 // w0 TMA, w1 MMA, w2-5 epilogue, w6-9 operand
-constexpr int PRODUCER_THREADS = 128;
+constexpr int B_STAGES = 2;                      // stage g belongs to producer group g
+constexpr int NUM_THREADS = 448;                 // w0 TMA, w1 MMA, w2-5 epilogue, w6-13 operand
+constexpr int PRODUCER_THREADS = 256;           // two groups of 4 warps
 constexpr int TMEM_COLS = 512;
 constexpr int MAX_DYN_SMEM = 232448;             // opt-in dynamic shared memory per block
 constexpr int BAR_BYTES = 512;
@@ -57,7 +57,7 @@ struct VgShape {
     static constexpr int USED = RT * (M + 3);           // columns carrying data
     static constexpr int CHUNKS = (USED + 31) / 32;     // 32-column TMEM loads per accumulator
     static constexpr int B_BYTES = NCOLS * 128;         // N rows x 64 k of bf16
-    static constexpr int STG_BYTES = RT * 512;          // staging: classes, residual pieces, codebook
+    static constexpr int STG_BYTES = 2 * RT * 64;       // codebooks of the tile's rows, per group
     static constexpr int A_FIT = (vg::MAX_DYN_SMEM - 1024 - vg::BAR_BYTES -
                                   vg::B_STAGES * B_BYTES - STG_BYTES) / vg::A_TILE;
     static constexpr int A_SLOTS = A_FIT < 12 ? A_FIT : 12;
@@ -132,17 +132,6 @@ __device__ __forceinline__ void vg_tile_coords(const VgParams &p, int tile, int 
     row_end = min(row0 + RT, gstart + p.rows_per_group);
 }
 
-// Per-K-block staging of the right operand's sources, shared by the producer warps:
-//   q[r][kk]     class of coordinate k0+kk in row row0+r (0xFF outside the problem)
-//   rp[r][p][kk] bf16 piece p of the residual c[q] - w of that coordinate (0 outside)
-//   c[r][b]      codebook of row row0+r
-template <int RT>
-struct VgStage {
-    uint8_t q[RT][64];
-    uint16_t rp[RT][3][64];
-    float c[RT][16];
-};
-
 template <int M>
 __global__ void __launch_bounds__(vg::NUM_THREADS, 1)
     lnq_vgemm_kernel(const __grid_constant__ CUtensorMap fmap, VgParams p)
@@ -164,8 +153,8 @@ __global__ void __launch_bounds__(vg::NUM_THREADS, 1)
     uint64_t *tempty = tfull + S::SETS;                           // [SETS]
     uint64_t *drain = tempty + S::SETS;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(drain + 1);
-    VgStage<S::RT> &stg = *reinterpret_cast<VgStage<S::RT> *>(
-        b_base + B_STAGES * S::B_BYTES + BAR_BYTES);
+    // per producer group: the codebooks of the tile's rows
+    float(*stg_c)[16] = reinterpret_cast<float(*)[16]>(b_base + B_STAGES * S::B_BYTES + BAR_BYTES);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -175,7 +164,7 @@ __global__ void __launch_bounds__(vg::NUM_THREADS, 1)
             mbar_init(&a_empty[s], 1);
         }
         for (int s = 0; s < B_STAGES; ++s) {
-            mbar_init(&b_full[s], PRODUCER_THREADS);
+            mbar_init(&b_full[s], PRODUCER_THREADS / 2);  // one producer group per stage
             mbar_init(&b_empty[s], 1);
         }
         for (int a = 0; a < S::SETS; ++a) {
@@ -228,52 +217,53 @@ __global__ void __launch_bounds__(vg::NUM_THREADS, 1)
         }
     } else if (warp >= 6) {
         // ---------------------------------------------------------------- right operand
-        // Four warps build the right operand of each K block in two phases, separated by a named
-        // barrier. Staging: each thread takes quads of 4 consecutive k of one row (prefetched into
-        // registers during the previous block) and writes the classes and the three bf16 pieces of
-        // the residuals. Expansion: each thread takes one (row, 16-byte column chunk): it reads the
-        // 8 classes once and writes the chunk of every one-hot row of that row, then copies residual
-        // chunks. Loads are issued before stores so that shared-memory accesses overlap. The stage
-        // wait is ANDed over the four warps, so they leave together on a timeout and the named
-        // barriers cannot deadlock. Columns beyond S::USED are never written: the epilogue ignores
-        // them.
-        constexpr int kBar = 1;
-        constexpr int QUADS = S::RT * 16;
-        constexpr int PER = (QUADS + PRODUCER_THREADS - 1) / PRODUCER_THREADS;
-        constexpr int PAIRS = S::RT * 8;
-        constexpr int RCH = 3 * S::RT * 8;  // residual chunks
-        constexpr int RPER = (RCH + PRODUCER_THREADS - 1) / PRODUCER_THREADS;
+        // Two groups of four warps take alternate K blocks (group g fills stage g with blocks
+        // kb = g, g + 2, ...), so each group has two MMA blocks' time to build one. A thread owns
+        // (row, 8-coordinate chunk) items and writes, from its own loads of Q and W, the chunk of
+        // every one-hot row of that row and of its three residual-piece rows, in the 128-byte
+        // swizzled K-major layout. Columns beyond S::USED are never written: the epilogue ignores
+        // them. The stage wait is ANDed over the group's warps so that they leave together on a
+        // timeout.
+        constexpr int GT = PRODUCER_THREADS / 2;
+        constexpr int ITEMS = S::RT * 8;
+        constexpr int IPT = (ITEMS + GT - 1) / GT;
         const int t = threadIdx.x - 6 * 32;
-        const bool vec = (p.d & 3) == 0 && (reinterpret_cast<uintptr_t>(p.Q) & 3u) == 0 &&
+        const int grp = t / GT, tg = t - grp * GT;
+        const int bar_id = 1 + grp;
+        float(*cs)[16] = stg_c + grp * S::RT;
+        const bool vec = (p.d & 7) == 0 && (reinterpret_cast<uintptr_t>(p.Q) & 7u) == 0 &&
                          (reinterpret_cast<uintptr_t>(p.W) & 15u) == 0;
-        int uses[B_STAGES] = {};
-        int stage = 0;
+        const int stage = grp;
+        int uses = 0;
         bool ok = true;
-        uint32_t qpre[PER];
-        float4 wpre[PER];
+        uint2 qn[IPT];   // next block's classes (0xFF outside the problem)
+        float4 wn[IPT][2];
         auto fetch = [&](int64_t row0, int64_t row_end, int64_t k0) {
 #pragma unroll
-            for (int s2 = 0; s2 < PER; ++s2) {
-                const int e = t + s2 * PRODUCER_THREADS;
-                const int r = e >> 4, kk = (e & 15) * 4;
-                const int64_t j = row0 + r, k = k0 + kk;
-                qpre[s2] = 0xFFFFFFFFu;
-                wpre[s2] = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (e < QUADS && j < row_end && k < p.d) {
-                    if (vec) {
-                        qpre[s2] = *reinterpret_cast<const uint32_t *>(p.Q + j * p.d + k);
-                        wpre[s2] = *reinterpret_cast<const float4 *>(p.W + j * p.d + k);
+            for (int s2 = 0; s2 < IPT; ++s2) {
+                const int e = tg + s2 * GT;
+                const int r = e >> 3, c = e & 7;
+                const int64_t j = row0 + r, k = k0 + 8 * c;
+                qn[s2] = make_uint2(0xFFFFFFFFu, 0xFFFFFFFFu);
+                wn[s2][0] = wn[s2][1] = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (e < ITEMS && j < row_end && k < p.d) {
+                    if (vec && k + 8 <= p.d) {
+                        qn[s2] = *reinterpret_cast<const uint2 *>(p.Q + j * p.d + k);
+                        wn[s2][0] = *reinterpret_cast<const float4 *>(p.W + j * p.d + k);
+                        wn[s2][1] = *reinterpret_cast<const float4 *>(p.W + j * p.d + k + 4);
                     } else {
-                        uint32_t qv = 0;
-                        float wv[4] = {0.f, 0.f, 0.f, 0.f};
+                        uint32_t q2[2] = {0u, 0u};
+                        float wv[8];
 #pragma unroll
-                        for (int e4 = 0; e4 < 4; ++e4) {
-                            const bool in = k + e4 < p.d;
-                            qv |= static_cast<uint32_t>(in ? p.Q[j * p.d + k + e4] : 0xFFu) << (8 * e4);
-                            wv[e4] = in ? p.W[j * p.d + k + e4] : 0.f;
+                        for (int e8 = 0; e8 < 8; ++e8) {
+                            const bool in = k + e8 < p.d;
+                            q2[e8 >> 2] |= static_cast<uint32_t>(in ? p.Q[j * p.d + k + e8] : 0xFFu)
+                                           << (8 * (e8 & 3));
+                            wv[e8] = in ? p.W[j * p.d + k + e8] : 0.f;
                         }
-                        qpre[s2] = qv;
-                        wpre[s2] = make_float4(wv[0], wv[1], wv[2], wv[3]);
+                        qn[s2] = make_uint2(q2[0], q2[1]);
+                        wn[s2][0] = make_float4(wv[0], wv[1], wv[2], wv[3]);
+                        wn[s2][1] = make_float4(wv[4], wv[5], wv[6], wv[7]);
                     }
                 }
             }
@@ -282,77 +272,70 @@ __global__ void __launch_bounds__(vg::NUM_THREADS, 1)
             int g, it;
             int64_t row0, row_end;
             vg_tile_coords<M>(p, tile, g, row0, row_end, it);
-            fetch(row0, row_end, 0);
-            for (int kb = 0; kb < nk; ++kb) {
-                const int mine = mbar_wait(&b_empty[stage], (uses[stage] & 1) ^ 1, limit) ? 1 : 0;
-                if (!named_bar_and(kBar, PRODUCER_THREADS, mine)) {
-                    if (t == 0)
+            if (grp >= nk)
+                continue;
+            // the group's copy of the tile's codebooks (the previous tile's readers are done:
+            // every thread passed the group's last stage wait after its last read)
+            named_bar_sync(bar_id, GT);
+            for (int e = tg; e < S::RT * 16; e += GT) {
+                const int r = e >> 4, b = e & 15;
+                const int64_t j = row0 + r;
+                cs[r][b] = (j < row_end && b < p.m) ? p.C[j * p.m + b] : 0.f;
+            }
+            fetch(row0, row_end, static_cast<int64_t>(grp) * BK);
+            named_bar_sync(bar_id, GT);
+            for (int kb = grp; kb < nk; kb += 2) {
+                const int mine = mbar_wait(&b_empty[stage], (uses & 1) ^ 1, limit) ? 1 : 0;
+                if (!named_bar_and(bar_id, GT, mine)) {
+                    if (tg == 0)
                         raise_error(p.err, kErrTimeout, 12);
                     ok = false;
                     break;
                 }
-                if (kb == 0) {
-                    for (int e = t; e < S::RT * 16; e += PRODUCER_THREADS) {
-                        const int r = e >> 4, b = e & 15;
-                        const int64_t j = row0 + r;
-                        stg.c[r][b] = (j < row_end && b < p.m) ? p.C[j * p.m + b] : 0.f;
-                    }
-                    named_bar_sync(kBar, PRODUCER_THREADS);
+                uint2 qc[IPT];
+                float4 wc[IPT][2];
+#pragma unroll
+                for (int s2 = 0; s2 < IPT; ++s2) {
+                    qc[s2] = qn[s2];
+                    wc[s2][0] = wn[s2][0];
+                    wc[s2][1] = wn[s2][1];
                 }
-                // staging: classes and residual pieces of this K block
-                float cq[PER][4];
-#pragma unroll
-                for (int s2 = 0; s2 < PER; ++s2) {
-                    const int e = t + s2 * PRODUCER_THREADS;
-                    const int r = (e < QUADS) ? (e >> 4) : 0;
-#pragma unroll
-                    for (int e4 = 0; e4 < 4; ++e4) {
-                        const uint32_t qv = (qpre[s2] >> (8 * e4)) & 0xFFu;
-                        cq[s2][e4] = stg.c[r][(qv == 0xFFu ? 0u : qv) & (p.m - 1)];
-                    }
-                }
-#pragma unroll
-                for (int s2 = 0; s2 < PER; ++s2) {
-                    const int e = t + s2 * PRODUCER_THREADS;
-                    if (e < QUADS) {
-                        const int r = e >> 4, kk = (e & 15) * 4;
-                        const float wv[4] = {wpre[s2].x, wpre[s2].y, wpre[s2].z, wpre[s2].w};
-                        uint32_t pk[3][2] = {{0u, 0u}, {0u, 0u}, {0u, 0u}};
-                        uint32_t qmask = 0u;
-#pragma unroll
-                        for (int e4 = 0; e4 < 4; ++e4) {
-                            const uint32_t qv = (qpre[s2] >> (8 * e4)) & 0xFFu;
-                            float p0 = 0.f, p1 = 0.f, p2 = 0.f;
-                            if (qv != 0xFFu) {
-                                split3(cq[s2][e4] - wv[e4], p0, p1, p2);
-                                qmask |= (qv & (p.m - 1)) << (8 * e4);
-                            } else {
-                                qmask |= 0xFFu << (8 * e4);
-                            }
-                            pk[0][e4 >> 1] |= static_cast<uint32_t>(bf16_bits(p0)) << (16 * (e4 & 1));
-                            pk[1][e4 >> 1] |= static_cast<uint32_t>(bf16_bits(p1)) << (16 * (e4 & 1));
-                            pk[2][e4 >> 1] |= static_cast<uint32_t>(bf16_bits(p2)) << (16 * (e4 & 1));
-                        }
-                        *reinterpret_cast<uint32_t *>(&stg.q[r][kk]) = qmask;
-#pragma unroll
-                        for (int pc = 0; pc < 3; ++pc)
-                            *reinterpret_cast<uint2 *>(&stg.rp[r][pc][kk]) = make_uint2(pk[pc][0], pk[pc][1]);
-                    }
-                }
-                if (kb + 1 < nk)
-                    fetch(row0, row_end, static_cast<int64_t>(kb + 1) * BK);
-                named_bar_sync(kBar, PRODUCER_THREADS);
-                // expansion into the swizzled K-major tile
+                if (kb + 2 < nk)
+                    fetch(row0, row_end, static_cast<int64_t>(kb + 2) * BK);
                 uint8_t *sb = b_base + stage * S::B_BYTES;
-                if constexpr (M > 0) {
-                    for (int pi = t; pi < PAIRS; pi += PRODUCER_THREADS) {
-                        const int r = pi >> 3, c = pi & 7;
-                        const uint2 qq = *reinterpret_cast<const uint2 *>(&stg.q[r][8 * c]);
+#pragma unroll
+                for (int s2 = 0; s2 < IPT; ++s2) {
+                    const int e = tg + s2 * GT;
+                    if (e >= ITEMS)
+                        continue;
+                    const int r = e >> 3, c = e & 7;
+                    // residual pieces of the chunk's 8 coordinates
+                    const float wv[8] = {wc[s2][0].x, wc[s2][0].y, wc[s2][0].z, wc[s2][0].w,
+                                         wc[s2][1].x, wc[s2][1].y, wc[s2][1].z, wc[s2][1].w};
+                    uint32_t pk[3][4] = {};
+#pragma unroll
+                    for (int e8 = 0; e8 < 8; ++e8) {
+                        const uint32_t qv = ((e8 < 4 ? qc[s2].x : qc[s2].y) >> (8 * (e8 & 3))) & 0xFFu;
+                        float p0 = 0.f, p1 = 0.f, p2 = 0.f;
+                        if (qv != 0xFFu)
+                            split3(cs[r][qv & (p.m - 1)] - wv[e8], p0, p1, p2);
+                        const int sh = 16 * (e8 & 1);
+                        pk[0][e8 >> 1] |= static_cast<uint32_t>(bf16_bits(p0)) << sh;
+                        pk[1][e8 >> 1] |= static_cast<uint32_t>(bf16_bits(p1)) << sh;
+                        pk[2][e8 >> 1] |= static_cast<uint32_t>(bf16_bits(p2)) << sh;
+                    }
+#pragma unroll
+                    for (int pc = 0; pc < 3; ++pc) {
+                        const int n = S::ONEHOT + 3 * r + pc;
+                        *reinterpret_cast<uint4 *>(sb + n * 128 + ((c ^ (n & 7)) << 4)) =
+                            make_uint4(pk[pc][0], pk[pc][1], pk[pc][2], pk[pc][3]);
+                    }
+                    if constexpr (M > 0) {
 #pragma unroll
                         for (int b = 0; b < M; ++b) {
                             const int n = r * M + b;
                             const uint32_t bbbb = 0x01010101u * static_cast<uint32_t>(b);
-                            const uint32_t m0 = __vcmpeq4(qq.x, bbbb), m1 = __vcmpeq4(qq.y, bbbb);
+                            const uint32_t m0 = __vcmpeq4(qc[s2].x, bbbb), m1 = __vcmpeq4(qc[s2].y, bbbb);
                             // byte e of the mask (0xFF or 0) -> bf16 1.0 (0x3F80) or 0, half-word e
                             *reinterpret_cast<uint4 *>(sb + n * 128 + ((c ^ (n & 7)) << 4)) =
                                 make_uint4(__byte_perm(m0, 0u, 0x1100) & 0x3F803F80u,
@@ -362,29 +345,10 @@ __global__ void __launch_bounds__(vg::NUM_THREADS, 1)
                         }
                     }
                 }
-                {
-                    uint4 rv[RPER];
-#pragma unroll
-                    for (int s2 = 0; s2 < RPER; ++s2) {
-                        const int ci = t + s2 * PRODUCER_THREADS;
-                        const int nr = ci >> 3, c = ci & 7;   // nr = 3 r + piece
-                        if (ci < RCH)
-                            rv[s2] = *reinterpret_cast<const uint4 *>(&stg.rp[nr / 3][nr % 3][8 * c]);
-                    }
-#pragma unroll
-                    for (int s2 = 0; s2 < RPER; ++s2) {
-                        const int ci = t + s2 * PRODUCER_THREADS;
-                        const int nr = ci >> 3, c = ci & 7;
-                        const int n = S::ONEHOT + nr;
-                        if (ci < RCH)
-                            *reinterpret_cast<uint4 *>(sb + n * 128 + ((c ^ (n & 7)) << 4)) = rv[s2];
-                    }
-                }
                 // make the generic-proxy writes visible to the tensor core (async proxy)
-                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                fence_proxy_async_smem();
                 mbar_arrive(&b_full[stage]);
-                ++uses[stage];
-                stage = (stage + 1 == B_STAGES) ? 0 : stage + 1;
+                ++uses;
             }
         }
     } else if (warp == 1) {
@@ -392,7 +356,7 @@ __global__ void __launch_bounds__(vg::NUM_THREADS, 1)
         // Per K block: wait for the right operand, then for each piece wait for its A slot, issue
         // four K=16 MMAs and release the slot; release the right-operand stage after the block.
         if (lane == 0) {
-            int bstage = 0, slot = 0;
+            int slot = 0;
             uint32_t bphase[B_STAGES] = {};
             uint32_t aphase[NSLOT] = {};
             bool ok = true;
@@ -407,6 +371,7 @@ __global__ void __launch_bounds__(vg::NUM_THREADS, 1)
                 }
                 tc_fence_after();
                 for (int kb = 0; kb < nk && ok; ++kb) {
+                    const int bstage = kb & 1;  // K block kb comes from producer group kb & 1
                     if (!mbar_wait(&b_full[bstage], bphase[bstage], limit)) {
                         raise_error(p.err, kErrTimeout, 14);
                         ok = false;
@@ -441,7 +406,6 @@ __global__ void __launch_bounds__(vg::NUM_THREADS, 1)
                     if (!ok)
                         break;
                     umma_commit(&b_empty[bstage]);
-                    bstage = (bstage + 1 == B_STAGES) ? 0 : bstage + 1;
                 }
                 if (!ok)
                     break;
