@@ -42,7 +42,8 @@ static bool valid_m(int m) { return m == 2 || m == 4 || m == 8 || m == 16; }
 //   BUILD_FISHER:   header | S [groups][n] f32 | M [n] f32 | pimax [groups] u32
 //                   | A [n][d_in] f16 | B [groups][n][d_in] f16
 //   QUANTIZE_ROWS:  header | status [d_out] i32 | Fp [groups][3][d_in][ld] bf16 (ld = d_in
-//                   rounded up to a multiple of 8)
+//                   rounded up to a multiple of 8) | Fh [groups][2][d_in][ld] f16 | fexp
+//                   [groups][d_in] i32 | rexp [d_out] i32
 //                   | V [d_out][d_in][m] f32 | uT [d_in][d_out] f32 | dC [d_out][m] f32
 //                   | sweep history [CTAs][2 ceil(d_in / 128)][3][4 KB] (Delta pieces)
 //   OBJECTIVE:      the same layout (status, V and dC unused)
@@ -63,7 +64,7 @@ static FisherWs fisher_ws(int64_t n, int64_t d_in, int groups)
 }
 
 struct LnqWs {
-    size_t st_off, fp_off, v_off, ut_off, dc_off, hist_off, total;
+    size_t st_off, fp_off, fh_off, fexp_off, rexp_off, v_off, ut_off, dc_off, hist_off, total;
 };
 static LnqWs lnq_ws(int64_t d_in, int64_t d_out, int groups, int m)
 {
@@ -71,7 +72,10 @@ static LnqWs lnq_ws(int64_t d_in, int64_t d_out, int groups, int m)
     w.st_off = kWsHeader;
     w.fp_off = align_up(w.st_off + static_cast<size_t>(d_out) * 4, 256);
     const size_t ld = static_cast<size_t>((d_in + 7) / 8 * 8);  // bf16 piece row stride
-    w.v_off = align_up(w.fp_off + static_cast<size_t>(groups) * 3 * d_in * ld * 2, 256);
+    w.fh_off = align_up(w.fp_off + static_cast<size_t>(groups) * 3 * d_in * ld * 2, 256);
+    w.fexp_off = align_up(w.fh_off + static_cast<size_t>(groups) * 2 * d_in * ld * 2, 256);
+    w.rexp_off = align_up(w.fexp_off + static_cast<size_t>(groups) * d_in * 4, 256);
+    w.v_off = align_up(w.rexp_off + static_cast<size_t>(d_out) * 4, 256);
     w.ut_off = align_up(w.v_off + static_cast<size_t>(d_out) * d_in * m * 4, 256);
     w.dc_off = align_up(w.ut_off + static_cast<size_t>(d_in) * d_out * 4, 256);
     w.hist_off = align_up(w.dc_off + static_cast<size_t>(d_out) * m * 4, 256);
@@ -85,6 +89,9 @@ static LnqWorkspace carve(void *ws, const LnqWs &lay)
     LnqWorkspace w;
     w.status = reinterpret_cast<int32_t *>(b + lay.st_off);
     w.Fp = reinterpret_cast<__nv_bfloat16 *>(b + lay.fp_off);
+    w.Fh = reinterpret_cast<__half *>(b + lay.fh_off);
+    w.fexp = reinterpret_cast<int32_t *>(b + lay.fexp_off);
+    w.rexp = reinterpret_cast<int32_t *>(b + lay.rexp_off);
     w.V = reinterpret_cast<float *>(b + lay.v_off);
     w.uT = reinterpret_cast<float *>(b + lay.ut_off);
     w.dC = reinterpret_cast<float *>(b + lay.dc_off);

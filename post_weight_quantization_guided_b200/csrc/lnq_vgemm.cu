@@ -8,19 +8,22 @@
 //      [V_j1 | u_j1 | V_j2 | u_j2 | ...] = F x [P_j1 | r_j1 | P_j2 | r_j2 | ...]
 //
 // whose left operand F is shared by every row of the group. This kernel computes it with
-// tcgen05.mma.kind::f16, exactly in fp32 terms:
+// tcgen05.mma.cta_group::2.kind::f16, exactly in fp32 terms:
 //   * F (fp32) is split into three bf16 pieces F = F1 + F2 + F3 (exact for normal values), and
 //     the three products accumulate into one TMEM accumulator;
 //   * the one-hot columns are 0/1 (exact in bf16); r is split the same way into three bf16
 //     pieces, one column each, so u = sum of nine exact bf16 x bf16 products;
 //   * accumulation is fp32 in TMEM.
-// A tile is 128 coordinates (i) x 256 columns (RT rows x (m one-hot + 3 residual pieces), RT =
-// floor(256 / (m + 3))). F tiles arrive by TMA (K-major, 128-byte swizzle); the 256 x 64 right
-// operand tile is generated in shared memory from Q, C and W by four producer warps, in the
-// same swizzled K-major layout. The epilogue writes V[j][i][b] and uT[i][j] (u transposed, so
-// the sweep reads it coalesced). With m = 0 the kernel computes u = F r only (85 rows per tile),
-// which the objective uses.
+// Two CTAs (a cluster pair on two SMs) share one MMA of 256 coordinates (i) x 256 columns
+// (RT rows x (m one-hot + 3 residual-piece columns), RT = floor(256 / (m + 3))): each CTA loads
+// the F tiles of its own 128 coordinates by TMA (K-major, 128-byte swizzle, no multicast) and
+// builds half of the right operand's columns in shared memory from Q, W and C, so that each SM
+// reads half of the right operand per MMA. The even CTA issues the MMAs; each CTA's TMEM holds
+// its 128 coordinates x all columns, and its epilogue writes V[j][i][b] and uT[i][j] (u
+// transposed, so the sweep reads a coordinate's rows contiguously). With m = 0 the kernel
+// computes u = F r only (42 rows per 128-column tile), which the objective uses.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "common.cuh"
 #include "lnq_internal.cuh"
@@ -29,42 +32,50 @@
 namespace lnq {
 
 namespace vg {
-constexpr int BM = 128;
+constexpr int BM = 128;                          // coordinates per CTA; a pair covers 256
 constexpr int BK = 64;
-constexpr int PIECES = 3;
 constexpr int A_TILE = BM * BK * 2;              // one bf16 piece of a 128 x 64 F tile: 16 KB
 constexpr int B_STAGES = 2;                      // stage g belongs to producer group g
 constexpr int NUM_THREADS = 448;                 // w0 TMA, w1 MMA, w2-5 epilogue, w6-13 operand
-constexpr int PRODUCER_THREADS = 256;           // two groups of 4 warps
+constexpr int PRODUCER_THREADS = 256;            // two groups of 4 warps
+constexpr int GROUP_THREADS = PRODUCER_THREADS / 2;
+constexpr int EPI_THREADS = 128;
 constexpr int TMEM_COLS = 512;
 constexpr int MAX_DYN_SMEM = 232448;             // opt-in dynamic shared memory per block
 constexpr int BAR_BYTES = 512;
+constexpr uint16_t PAIR = 0x3;                   // both CTAs of the cluster
+// After an error, how long a CTA lets its own copies land before the pair exits.
+constexpr long long kPairDrainLimit = 1LL << 22;
 }  // namespace vg
 
-// Tile shapes. With one-hot columns (M > 0) a tile is 256 columns and two TMEM accumulators
-// alternate between tiles. The residual-only product (M == 0) feeds the objective, which sums
-// r_i u_i with cancellation; there a tile is 128 columns and the K range is cut into four
-// segments with one accumulator each, so each fp32 accumulator takes a quarter of the additions.
-// Shared memory: A arrives one bf16 piece (16 KB) per slot, in as many slots as fit next to the two
-// right-operand stages and the staging area, so that several K blocks of F are in flight.
+// Tile shapes. With one-hot columns (M > 0) the MMA is 256 columns wide and two TMEM
+// accumulators alternate between tiles. The residual-only product (M == 0) feeds the objective,
+// which sums r_i u_i with cancellation; there the MMA is 128 columns wide and the K range is cut
+// into four segments with one accumulator each, so each fp32 accumulator takes a quarter of the
+// additions. Each CTA holds HALF = NCOLS / 2 rows of the right operand per stage.
 template <int M>
 struct VgShape {
+    static constexpr bool F16 = M > 0;                  // fp16 pieces (V, u) or exact bf16 (J)
+    static constexpr int PIECES = F16 ? 2 : 3;          // pieces of F in the left operand
     static constexpr int NCOLS = M > 0 ? 256 : 128;     // MMA N
+    static constexpr int HALF = NCOLS / 2;              // right-operand rows held by one CTA
     static constexpr int SEGS = M > 0 ? 1 : 4;          // K segments (one accumulator each)
     static constexpr int SETS = M > 0 ? 2 : 1;          // accumulator sets (tile double-buffer)
     static constexpr int RT = NCOLS / (M + 3);          // rows per tile
     static constexpr int ONEHOT = RT * M;               // one-hot columns
     static constexpr int USED = RT * (M + 3);           // columns carrying data
     static constexpr int CHUNKS = (USED + 31) / 32;     // 32-column TMEM loads per accumulator
-    static constexpr int B_BYTES = NCOLS * 128;         // N rows x 64 k of bf16
-    static constexpr int STG_BYTES = 2 * RT * 64;       // codebooks of the tile's rows, per group
+    static constexpr int B_BYTES = HALF * 128;          // HALF rows x 64 k of bf16
+    static constexpr int STG_BYTES = 2 * RT * 68;       // per group: codebooks and residual scales
     static constexpr int A_FIT = (vg::MAX_DYN_SMEM - 1024 - vg::BAR_BYTES -
                                   vg::B_STAGES * B_BYTES - STG_BYTES) / vg::A_TILE;
     static constexpr int A_SLOTS = A_FIT < 12 ? A_FIT : 12;
     static constexpr size_t SMEM = 1024 + static_cast<size_t>(A_SLOTS) * vg::A_TILE +
                                    vg::B_STAGES * B_BYTES + vg::BAR_BYTES + STG_BYTES;
     static_assert(SETS * SEGS * NCOLS <= vg::TMEM_COLS, "TMEM holds 512 fp32 columns");
-    static_assert(A_SLOTS >= 2 * vg::PIECES, "at least two K blocks of F in flight");
+    static_assert(A_SLOTS >= 2 * PIECES, "at least two K blocks of F in flight");
+    static_assert(A_SLOTS <= 32, "slot phases are kept in 32-bit masks");
+    static_assert(HALF % (M > 0 ? M : 1) == 0, "a row's one-hot columns lie in one CTA's half");
     static_assert(SMEM <= vg::MAX_DYN_SMEM, "shared memory");
 };
 
@@ -106,27 +117,112 @@ __global__ void split_f_kernel(const float *__restrict__ F, int64_t d, int group
     }
 }
 
+// 2^e as a float, exact for |e| <= 126; scale exponents are kept within +-100.
+__device__ __forceinline__ float pow2f(int e) { return __int_as_float((127 + e) << 23); }
+__device__ __forceinline__ int clamp_scale(int e) { return e < -100 ? -100 : (e > 100 ? 100 : e); }
+
+// F (fp32 [groups][d][d]) -> Fh (fp16 [groups][2][d][ld]) with a power-of-two scale per row:
+// F[i][k] 2^fexp[i] = H1 + H2 up to 2^-22 relative (2^-39 of the row's largest entry for entries
+// near the fp16 subnormal range), the row's largest entry scaled into [2^14, 2^15). One CTA per
+// row. The epilogue of the product multiplies by 2^-fexp[i], exactly.
+__global__ void __launch_bounds__(256)
+    split_f16_kernel(const float *__restrict__ F, int64_t d, __half *__restrict__ Fh,
+                     int32_t *__restrict__ fexp)
+{
+    __shared__ float red[8];
+    const int64_t row = blockIdx.x;            // g * d + i
+    const int64_t g = row / d, i = row - g * d;
+    const float *src = F + row * d;
+    float mx = 0.f;
+    for (int64_t k = threadIdx.x; k < d; k += blockDim.x)
+        mx = fmaxf(mx, fabsf(src[k]));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if ((threadIdx.x & 31) == 0)
+        red[threadIdx.x >> 5] = mx;
+    __syncthreads();
+    mx = red[0];
+    for (int w = 1; w < static_cast<int>(blockDim.x >> 5); ++w)
+        mx = fmaxf(mx, red[w]);
+    const int s = mx > 0.f ? clamp_scale(14 - ilogbf(mx)) : 0;
+    if (threadIdx.x == 0)
+        fexp[row] = s;
+    const float sc = pow2f(s);
+    const int64_t ld = pieces_stride(d);
+    __half *h1 = Fh + (g * 2 * d + i) * ld;
+    __half *h2 = h1 + d * ld;
+    for (int64_t k = threadIdx.x; k < ld; k += blockDim.x) {
+        float x = 0.f;
+        if (k < d)
+            x = src[k] * sc;
+        const __half a = __float2half_rn(x);
+        h1[k] = a;
+        h2[k] = __float2half_rn(x - __half2float(a));
+    }
+}
+
+// Per-row power-of-two scale of the residual r_j = c_j[q_j] - w_j for the fp16 right operand:
+// max_k |r_jk| 2^rexp[j] in [2^14, 2^15). One warp per row.
+__global__ void __launch_bounds__(256)
+    residual_scale_kernel(const uint8_t *__restrict__ Q, const float *__restrict__ W,
+                          const float *__restrict__ C, int64_t d, int64_t d_out, int m,
+                          int32_t *__restrict__ rexp)
+{
+    const int64_t j = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (j >= d_out)
+        return;
+    float mx = 0.f;
+    for (int64_t k = lane; k < d; k += 32)
+        mx = fmaxf(mx, fabsf(C[j * m + (Q[j * d + k] & (m - 1))] - W[j * d + k]));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if (lane == 0)
+        rexp[j] = mx > 0.f ? clamp_scale(14 - ilogbf(mx)) : 0;
+}
+
+// The three fp16 pieces of x (|x| <= 2^15): x == p0 + p1 + p2 up to 2^-33 relative (2^-24
+// absolute, the fp16 subnormal step).
+__device__ __forceinline__ void split3_f16(float x, uint16_t &p0, uint16_t &p1, uint16_t &p2)
+{
+    const __half a = __float2half_rn(x);
+    const float r1 = x - __half2float(a);
+    const __half b = __float2half_rn(r1);
+    const __half c = __float2half_rn(r1 - __half2float(b));
+    p0 = __half_as_ushort(a);
+    p1 = __half_as_ushort(b);
+    p2 = __half_as_ushort(c);
+}
+
 struct VgParams {
     const uint8_t *Q;   // [d_out][d]
     const float *W;     // [d_out][d]
     const float *C;     // [d_out][m]
     float *V;           // [d_out][d][m] (m > 0)
     float *uT;          // [d][d_out]
+    const int32_t *fexp;  // [groups][d] row scales of the fp16 pieces of F (fp16 mode)
+    const int32_t *rexp;  // [d_out] residual scales (fp16 mode)
     int64_t d, d_out, rows_per_group;
     int m;
-    int row_tiles_per_group, i_tiles, num_tiles;
+    int row_tiles_per_group, i_pairs, num_tiles;
     DeviceErr err;
 };
 
+// Tile -> (group, rows [row0, row_end), coordinate pair block ip), ordered group, then pair
+// block, then row tile: the pairs running at the same time read the same 256-coordinate panel of
+// F (a few MB, served from L2), and a group's Q and W stay in L2 across its pair blocks.
 template <int M>
 __device__ __forceinline__ void vg_tile_coords(const VgParams &p, int tile, int &g, int64_t &row0,
-                                               int64_t &row_end, int &it)
+                                               int64_t &row_end, int &ip)
 {
     constexpr int RT = VgShape<M>::RT;
-    it = tile % p.i_tiles;
-    const int rt_all = tile / p.i_tiles;
-    g = rt_all / p.row_tiles_per_group;
-    const int rt = rt_all - g * p.row_tiles_per_group;
+    const int per_group = p.i_pairs * p.row_tiles_per_group;
+    g = tile / per_group;
+    const int rem = tile - g * per_group;
+    ip = rem / p.row_tiles_per_group;
+    const int rt = rem - ip * p.row_tiles_per_group;
     const int64_t gstart = static_cast<int64_t>(g) * p.rows_per_group;
     row0 = gstart + static_cast<int64_t>(rt) * RT;
     row_end = min(row0 + RT, gstart + p.rows_per_group);
@@ -139,46 +235,50 @@ __global__ void __launch_bounds__(vg::NUM_THREADS, 1)
     using namespace vg;
     using S = VgShape<M>;
     constexpr int NSLOT = S::A_SLOTS;
-    constexpr uint32_t IDESC = umma_idesc_f16kind(BM, S::NCOLS, false, false, /*f16=*/false);
+    constexpr uint32_t IDESC = umma_idesc_f16kind(2 * BM, S::NCOLS, false, false, S::F16);
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(align_up(reinterpret_cast<uintptr_t>(smem_raw), 1024));
     uint8_t *a_base = smem;                                       // [NSLOT][16 KB]
     uint8_t *b_base = smem + NSLOT * A_TILE;                      // [B_STAGES][B_BYTES]
     uint64_t *bars = reinterpret_cast<uint64_t *>(b_base + B_STAGES * S::B_BYTES);
-    uint64_t *a_full = bars;                                      // [NSLOT]
+    uint64_t *a_full = bars;                                      // [NSLOT] (the even CTA's count)
     uint64_t *a_empty = a_full + NSLOT;                           // [NSLOT]
-    uint64_t *b_full = a_empty + NSLOT;                           // [B_STAGES]
+    uint64_t *b_full = a_empty + NSLOT;                           // [B_STAGES] (even CTA's count)
     uint64_t *b_empty = b_full + B_STAGES;                        // [B_STAGES]
     uint64_t *tfull = b_empty + B_STAGES;                         // [SETS]
-    uint64_t *tempty = tfull + S::SETS;                           // [SETS]
+    uint64_t *tempty = tfull + S::SETS;                           // [SETS] (even CTA's count)
     uint64_t *drain = tempty + S::SETS;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(drain + 1);
     // per producer group: the codebooks of the tile's rows
     float(*stg_c)[16] = reinterpret_cast<float(*)[16]>(b_base + B_STAGES * S::B_BYTES + BAR_BYTES);
+    float *stg_t = reinterpret_cast<float *>(stg_c + 2 * S::RT);  // [2][RT] 2^rexp of each row
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    const uint32_t cr = cluster_ctarank();  // 0: issues the pair's MMAs; 1: its peer
+    const int pair = static_cast<int>(blockIdx.x >> 1);
+    const int npairs = static_cast<int>(gridDim.x >> 1);
     if (threadIdx.x == 0) {
         for (int s = 0; s < NSLOT; ++s) {
             mbar_init(&a_full[s], 1);
             mbar_init(&a_empty[s], 1);
         }
         for (int s = 0; s < B_STAGES; ++s) {
-            mbar_init(&b_full[s], PRODUCER_THREADS / 2);  // one producer group per stage
+            mbar_init(&b_full[s], 2 * GROUP_THREADS);   // one producer group of each CTA
             mbar_init(&b_empty[s], 1);
         }
         for (int a = 0; a < S::SETS; ++a) {
             mbar_init(&tfull[a], 1);
-            mbar_init(&tempty[a], 4 * 32);
+            mbar_init(&tempty[a], 2 * EPI_THREADS);     // the epilogues of both CTAs
         }
         mbar_init(drain, 1);
         fence_barrier_init();
         tma_prefetch_desc(&fmap);
     }
     if (warp == 1)
-        tmem_alloc(tmem_holder, TMEM_COLS);
+        tmem_alloc_pair(tmem_holder, TMEM_COLS);
     tc_fence_before();
-    __syncthreads();
+    cluster_sync();  // barriers of both CTAs initialised, TMEM allocated in both
     tc_fence_after();
     const uint32_t tmem_base = *tmem_holder;
     const int nk = static_cast<int>((p.d + BK - 1) / BK);
@@ -186,71 +286,111 @@ __global__ void __launch_bounds__(vg::NUM_THREADS, 1)
 
     if (warp == 0) {
         // ---------------------------------------------------------------- TMA: F pieces
-        // One 16 KB piece tile per slot, slots in round-robin order.
+        // One 16 KB piece tile of this CTA's 128 coordinates per slot, slots in round-robin order;
+        // the bytes of both CTAs are counted on the even CTA's a_full (armed by its thread for
+        // both), and the even CTA's MMA commits release the slot in both CTAs.
         if (lane == 0) {
-            int fills[NSLOT] = {};
             int slot = 0;
+            uint32_t apar = 0u, aused = 0u;  // per slot: parity of the fills, ever filled
             bool ok = true;
-            for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
-                int g, it;
+            for (int tile = pair; tile < p.num_tiles && ok; tile += npairs) {
+                int g, ip;
                 int64_t row0, row_end;
-                vg_tile_coords<M>(p, tile, g, row0, row_end, it);
+                vg_tile_coords<M>(p, tile, g, row0, row_end, ip);
+                const int i0 = ip * 2 * BM + static_cast<int>(cr) * BM;
                 for (int kb = 0; kb < nk && ok; ++kb) {
-                    for (int pc = 0; pc < PIECES; ++pc) {
-                        if (!mbar_wait(&a_empty[slot], (fills[slot] & 1) ^ 1, limit)) {
+                    for (int pc = 0; pc < S::PIECES; ++pc) {
+                        if (!mbar_wait(&a_empty[slot], ((apar >> slot) & 1u) ^ 1u, limit)) {
                             raise_error(p.err, kErrTimeout, 11);
                             ok = false;
                             break;
                         }
-                        mbar_arrive_expect_tx(&a_full[slot], A_TILE);
-                        tma_load_3d(a_base + slot * A_TILE, &fmap, &a_full[slot], kb * BK, it * BM,
-                                    g * PIECES + pc);
-                        ++fills[slot];
+                        if (cr == 0)
+                            mbar_arrive_expect_tx(&a_full[slot], 2 * A_TILE);
+                        tma_load_3d_pair(a_base + slot * A_TILE, &fmap, cluster_addr(&a_full[slot], 0),
+                                         kb * BK, i0, g * S::PIECES + pc);
+                        apar ^= 1u << slot;
+                        aused |= 1u << slot;
                         slot = (slot + 1 == NSLOT) ? 0 : slot + 1;
                     }
                 }
             }
-            if (!ok)
-                for (int s = 0; s < NSLOT; ++s)
-                    if (fills[s] > 0)
-                        mbar_wait(&a_full[s], (fills[s] - 1) & 1, kDrainLimit);
+            if (!ok) {
+                // let this CTA's copies land before the pair exits: the even CTA waits for the last
+                // phase of each slot it armed; the odd CTA's copies are counted there, so it waits
+                // a fixed time
+                if (cr == 0) {
+                    for (int s = 0; s < NSLOT; ++s)
+                        if ((aused >> s) & 1u)
+                            mbar_wait(&a_full[s], ((apar >> s) & 1u) ^ 1u, kPairDrainLimit);
+                } else {
+                    const long long t0 = clock64();
+                    while (clock64() - t0 < kPairDrainLimit) {
+                    }
+                }
+            }
         }
     } else if (warp >= 6) {
         // ---------------------------------------------------------------- right operand
-        // Two groups of four warps take alternate K blocks (group g fills stage g with blocks
-        // kb = g, g + 2, ...), so each group has two MMA blocks' time to build one. A thread owns
-        // (row, 8-coordinate chunk) items and writes, from its own loads of Q and W, the chunk of
-        // every one-hot row of that row and of its three residual-piece rows, in the 128-byte
-        // swizzled K-major layout. Columns beyond S::USED are never written: the epilogue ignores
-        // them. The stage wait is ANDed over the group's warps so that they leave together on a
-        // timeout.
-        constexpr int GT = PRODUCER_THREADS / 2;
-        constexpr int ITEMS = S::RT * 8;
-        constexpr int IPT = (ITEMS + GT - 1) / GT;
+        // This CTA builds right-operand columns [n_lo, n_lo + HALF) of the pair's MMA. Two groups
+        // of four warps take alternate K blocks (group g fills stage g with blocks kb = g, g + 2,
+        // ...). A thread owns (row, 8-coordinate chunk) items and writes, from its own loads of Q
+        // and W, the chunk of each one-hot row and residual-piece row of that row that falls in
+        // this CTA's columns, in the 128-byte swizzled K-major layout. Columns beyond S::USED are
+        // never written: the epilogue ignores them. The stage wait is ANDed over the group's warps
+        // so that they leave together on a timeout.
+        constexpr int GT = GROUP_THREADS;
+        constexpr int IPT = (S::RT * 8 + GT - 1) / GT;
         const int t = threadIdx.x - 6 * 32;
         const int grp = t / GT, tg = t - grp * GT;
         const int bar_id = 1 + grp;
         float(*cs)[16] = stg_c + grp * S::RT;
+        float *ts = stg_t + grp * S::RT;
+        const int n_lo = static_cast<int>(cr) * S::HALF, n_hi = n_lo + S::HALF;
+        // rows with a column in [n_lo, n_hi): one-hot columns r M + b, residual ONEHOT + 3 r + pc
+        int r_lo = S::RT, r_hi = 0;
+        if constexpr (M > 0) {
+            const int lo = min(S::RT, n_lo / M), hi = min(S::RT, n_hi / M);
+            if (lo < hi) {
+                r_lo = lo;
+                r_hi = hi;
+            }
+        }
+        {
+            const int a = n_lo - S::ONEHOT - 2, b = n_hi - S::ONEHOT - 1;
+            const int lo = a <= 0 ? 0 : (a + 2) / 3;
+            const int hi = b < 0 ? 0 : min(S::RT, b / 3 + 1);
+            if (lo < hi) {
+                r_lo = min(r_lo, lo);
+                r_hi = max(r_hi, hi);
+            }
+        }
+        const int items = r_hi > r_lo ? (r_hi - r_lo) * 8 : 0;
         const bool vec = (p.d & 7) == 0 && (reinterpret_cast<uintptr_t>(p.Q) & 7u) == 0 &&
                          (reinterpret_cast<uintptr_t>(p.W) & 15u) == 0;
         const int stage = grp;
+        const uint32_t b_full_leader = cluster_addr(&b_full[stage], 0);
         int uses = 0;
         bool ok = true;
         uint2 qn[IPT];   // next block's classes (0xFF outside the problem)
         float4 wn[IPT][2];
+        auto has_res = [&](int r) { return S::ONEHOT + 3 * r + 2 >= n_lo && S::ONEHOT + 3 * r < n_hi; };
         auto fetch = [&](int64_t row0, int64_t row_end, int64_t k0) {
 #pragma unroll
             for (int s2 = 0; s2 < IPT; ++s2) {
                 const int e = tg + s2 * GT;
-                const int r = e >> 3, c = e & 7;
+                const int r = r_lo + (e >> 3), c = e & 7;
                 const int64_t j = row0 + r, k = k0 + 8 * c;
                 qn[s2] = make_uint2(0xFFFFFFFFu, 0xFFFFFFFFu);
                 wn[s2][0] = wn[s2][1] = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (e < ITEMS && j < row_end && k < p.d) {
+                if (e < items && j < row_end && k < p.d) {
+                    const bool need_w = has_res(r);
                     if (vec && k + 8 <= p.d) {
                         qn[s2] = *reinterpret_cast<const uint2 *>(p.Q + j * p.d + k);
-                        wn[s2][0] = *reinterpret_cast<const float4 *>(p.W + j * p.d + k);
-                        wn[s2][1] = *reinterpret_cast<const float4 *>(p.W + j * p.d + k + 4);
+                        if (need_w) {
+                            wn[s2][0] = *reinterpret_cast<const float4 *>(p.W + j * p.d + k);
+                            wn[s2][1] = *reinterpret_cast<const float4 *>(p.W + j * p.d + k + 4);
+                        }
                     } else {
                         uint32_t q2[2] = {0u, 0u};
                         float wv[8];
@@ -259,7 +399,7 @@ __global__ void __launch_bounds__(vg::NUM_THREADS, 1)
                             const bool in = k + e8 < p.d;
                             q2[e8 >> 2] |= static_cast<uint32_t>(in ? p.Q[j * p.d + k + e8] : 0xFFu)
                                            << (8 * (e8 & 3));
-                            wv[e8] = in ? p.W[j * p.d + k + e8] : 0.f;
+                            wv[e8] = (in && need_w) ? p.W[j * p.d + k + e8] : 0.f;
                         }
                         qn[s2] = make_uint2(q2[0], q2[1]);
                         wn[s2][0] = make_float4(wv[0], wv[1], wv[2], wv[3]);
@@ -268,10 +408,10 @@ __global__ void __launch_bounds__(vg::NUM_THREADS, 1)
                 }
             }
         };
-        for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
-            int g, it;
+        for (int tile = pair; tile < p.num_tiles && ok; tile += npairs) {
+            int g, ip;
             int64_t row0, row_end;
-            vg_tile_coords<M>(p, tile, g, row0, row_end, it);
+            vg_tile_coords<M>(p, tile, g, row0, row_end, ip);
             if (grp >= nk)
                 continue;
             // the group's copy of the tile's codebooks (the previous tile's readers are done:
@@ -281,6 +421,10 @@ __global__ void __launch_bounds__(vg::NUM_THREADS, 1)
                 const int r = e >> 4, b = e & 15;
                 const int64_t j = row0 + r;
                 cs[r][b] = (j < row_end && b < p.m) ? p.C[j * p.m + b] : 0.f;
+            }
+            if constexpr (S::F16) {
+                for (int r = tg; r < S::RT; r += GT)
+                    ts[r] = pow2f((row0 + r < row_end) ? p.rexp[row0 + r] : 0);
             }
             fetch(row0, row_end, static_cast<int64_t>(grp) * BK);
             named_bar_sync(bar_id, GT);
@@ -306,65 +450,83 @@ __global__ void __launch_bounds__(vg::NUM_THREADS, 1)
 #pragma unroll
                 for (int s2 = 0; s2 < IPT; ++s2) {
                     const int e = tg + s2 * GT;
-                    if (e >= ITEMS)
+                    if (e >= items)
                         continue;
-                    const int r = e >> 3, c = e & 7;
-                    // residual pieces of the chunk's 8 coordinates
-                    const float wv[8] = {wc[s2][0].x, wc[s2][0].y, wc[s2][0].z, wc[s2][0].w,
-                                         wc[s2][1].x, wc[s2][1].y, wc[s2][1].z, wc[s2][1].w};
-                    uint32_t pk[3][4] = {};
+                    const int r = r_lo + (e >> 3), c = e & 7;
+                    if (has_res(r)) {
+                        // residual pieces of the chunk's 8 coordinates
+                        const float wv[8] = {wc[s2][0].x, wc[s2][0].y, wc[s2][0].z, wc[s2][0].w,
+                                             wc[s2][1].x, wc[s2][1].y, wc[s2][1].z, wc[s2][1].w};
+                        uint32_t pk[3][4] = {};
 #pragma unroll
-                    for (int e8 = 0; e8 < 8; ++e8) {
-                        const uint32_t qv = ((e8 < 4 ? qc[s2].x : qc[s2].y) >> (8 * (e8 & 3))) & 0xFFu;
-                        float p0 = 0.f, p1 = 0.f, p2 = 0.f;
-                        if (qv != 0xFFu)
-                            split3(cs[r][qv & (p.m - 1)] - wv[e8], p0, p1, p2);
-                        const int sh = 16 * (e8 & 1);
-                        pk[0][e8 >> 1] |= static_cast<uint32_t>(bf16_bits(p0)) << sh;
-                        pk[1][e8 >> 1] |= static_cast<uint32_t>(bf16_bits(p1)) << sh;
-                        pk[2][e8 >> 1] |= static_cast<uint32_t>(bf16_bits(p2)) << sh;
-                    }
+                        for (int e8 = 0; e8 < 8; ++e8) {
+                            const uint32_t qv = ((e8 < 4 ? qc[s2].x : qc[s2].y) >> (8 * (e8 & 3))) & 0xFFu;
+                            uint16_t b0 = 0, b1 = 0, b2 = 0;
+                            if (qv != 0xFFu) {
+                                const float rv = cs[r][qv & (p.m - 1)] - wv[e8];
+                                if constexpr (S::F16) {
+                                    split3_f16(rv * ts[r], b0, b1, b2);
+                                } else {
+                                    float p0, p1, p2;
+                                    split3(rv, p0, p1, p2);
+                                    b0 = bf16_bits(p0);
+                                    b1 = bf16_bits(p1);
+                                    b2 = bf16_bits(p2);
+                                }
+                            }
+                            const int sh = 16 * (e8 & 1);
+                            pk[0][e8 >> 1] |= static_cast<uint32_t>(b0) << sh;
+                            pk[1][e8 >> 1] |= static_cast<uint32_t>(b1) << sh;
+                            pk[2][e8 >> 1] |= static_cast<uint32_t>(b2) << sh;
+                        }
 #pragma unroll
-                    for (int pc = 0; pc < 3; ++pc) {
-                        const int n = S::ONEHOT + 3 * r + pc;
-                        *reinterpret_cast<uint4 *>(sb + n * 128 + ((c ^ (n & 7)) << 4)) =
-                            make_uint4(pk[pc][0], pk[pc][1], pk[pc][2], pk[pc][3]);
+                        for (int pc = 0; pc < 3; ++pc) {
+                            const int n = S::ONEHOT + 3 * r + pc - n_lo;
+                            if (n >= 0 && n < S::HALF)
+                                *reinterpret_cast<uint4 *>(sb + n * 128 + ((c ^ (n & 7)) << 4)) =
+                                    make_uint4(pk[pc][0], pk[pc][1], pk[pc][2], pk[pc][3]);
+                        }
                     }
                     if constexpr (M > 0) {
+                        if (r * M >= n_lo && r * M < n_hi) {
 #pragma unroll
-                        for (int b = 0; b < M; ++b) {
-                            const int n = r * M + b;
-                            const uint32_t bbbb = 0x01010101u * static_cast<uint32_t>(b);
-                            const uint32_t m0 = __vcmpeq4(qc[s2].x, bbbb), m1 = __vcmpeq4(qc[s2].y, bbbb);
-                            // byte e of the mask (0xFF or 0) -> bf16 1.0 (0x3F80) or 0, half-word e
-                            *reinterpret_cast<uint4 *>(sb + n * 128 + ((c ^ (n & 7)) << 4)) =
-                                make_uint4(__byte_perm(m0, 0u, 0x1100) & 0x3F803F80u,
-                                           __byte_perm(m0, 0u, 0x3322) & 0x3F803F80u,
-                                           __byte_perm(m1, 0u, 0x1100) & 0x3F803F80u,
-                                           __byte_perm(m1, 0u, 0x3322) & 0x3F803F80u);
+                            for (int b = 0; b < M; ++b) {
+                                const int n = r * M + b - n_lo;
+                                const uint32_t bbbb = 0x01010101u * static_cast<uint32_t>(b);
+                                const uint32_t m0 = __vcmpeq4(qc[s2].x, bbbb), m1 = __vcmpeq4(qc[s2].y, bbbb);
+                                // byte e of the mask (0xFF or 0) -> 1.0 or 0 in half-word e
+                                // (fp16 1.0 = 0x3C00, bf16 1.0 = 0x3F80)
+                                constexpr uint32_t ONE2 = S::F16 ? 0x3C003C00u : 0x3F803F80u;
+                                *reinterpret_cast<uint4 *>(sb + n * 128 + ((c ^ (n & 7)) << 4)) =
+                                    make_uint4(__byte_perm(m0, 0u, 0x1100) & ONE2,
+                                               __byte_perm(m0, 0u, 0x3322) & ONE2,
+                                               __byte_perm(m1, 0u, 0x1100) & ONE2,
+                                               __byte_perm(m1, 0u, 0x3322) & ONE2);
+                            }
                         }
                     }
                 }
-                // make the generic-proxy writes visible to the tensor core (async proxy)
+                // make the generic-proxy writes visible to the tensor core (async proxy), then
+                // count them on the even CTA's stage barrier
                 fence_proxy_async_smem();
-                mbar_arrive(&b_full[stage]);
+                mbar_arrive_cluster(b_full_leader);
                 ++uses;
             }
         }
     } else if (warp == 1) {
-        // ---------------------------------------------------------------- MMA issuer
-        // Per K block: wait for the right operand, then for each piece wait for its A slot, issue
-        // four K=16 MMAs and release the slot; release the right-operand stage after the block.
-        if (lane == 0) {
+        // ---------------------------------------------------------------- MMA issue (even CTA)
+        // Per K block: wait for both CTAs' right-operand halves, then for each piece wait for
+        // both CTAs' F tiles, issue four K=16 MMAs (M = 256 over the pair) and release the slot
+        // in both CTAs; release the stage after the block, the accumulator after the tile.
+        if (cr == 0 && lane == 0) {
             int slot = 0;
-            uint32_t bphase[B_STAGES] = {};
-            uint32_t aphase[NSLOT] = {};
+            uint32_t aph = 0u, bph = 0u;  // phase parity per slot / stage
             bool ok = true;
             int itn = 0;
-            for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x, ++itn) {
+            for (int tile = pair; tile < p.num_tiles && ok; tile += npairs, ++itn) {
                 const int acc = itn % S::SETS;
                 const int use = itn / S::SETS;
-                if (!mbar_wait(&tempty[acc], (use & 1) ^ 1, limit)) {
+                if (!mbar_wait_cluster(&tempty[acc], (use & 1) ^ 1, limit)) {
                     raise_error(p.err, kErrTimeout, 13);
                     ok = false;
                     break;
@@ -372,53 +534,59 @@ __global__ void __launch_bounds__(vg::NUM_THREADS, 1)
                 tc_fence_after();
                 for (int kb = 0; kb < nk && ok; ++kb) {
                     const int bstage = kb & 1;  // K block kb comes from producer group kb & 1
-                    if (!mbar_wait(&b_full[bstage], bphase[bstage], limit)) {
+                    if (!mbar_wait_cluster(&b_full[bstage], (bph >> bstage) & 1u, limit)) {
                         raise_error(p.err, kErrTimeout, 14);
                         ok = false;
                         break;
                     }
-                    bphase[bstage] ^= 1u;
+                    bph ^= 1u << bstage;
+                    tc_fence_after();
                     const int seg = (kb * S::SEGS) / nk;
                     const bool seg_start = (kb == 0) || (((kb - 1) * S::SEGS) / nk != seg);
                     const uint32_t d_tmem =
                         tmem_base + static_cast<uint32_t>((acc * S::SEGS + seg) * S::NCOLS);
                     const uint32_t sb = smem_u32(b_base + bstage * S::B_BYTES);
-                    for (int pc = 0; pc < PIECES; ++pc) {
-                        if (!mbar_wait(&a_full[slot], aphase[slot], limit)) {
+                    for (int pc = 0; pc < S::PIECES; ++pc) {
+                        if (!mbar_wait(&a_full[slot], (aph >> slot) & 1u, limit)) {
                             raise_error(p.err, kErrTimeout, 16);
                             ok = false;
                             break;
                         }
-                        aphase[slot] ^= 1u;
+                        aph ^= 1u << slot;
                         tc_fence_after();
                         const uint32_t sa = smem_u32(a_base + slot * A_TILE);
 #pragma unroll
                         for (int kk = 0; kk < BK / 16; ++kk) {
-                            // K-major, 128-byte swizzle: 16 k = 32 bytes along the row.
+                            // K-major, 128-byte swizzle: 16 k = 32 bytes along the row
                             const uint64_t ad = umma_desc_sw128(sa + kk * 32, 16, 1024);
                             const uint64_t bd = umma_desc_sw128(sb + kk * 32, 16, 1024);
-                            umma_f16(d_tmem, ad, bd, IDESC,
-                                     (!seg_start || pc != 0 || kk != 0) ? 1u : 0u);
+                            umma_f16_pair(d_tmem, ad, bd, IDESC,
+                                          (!seg_start || pc != 0 || kk != 0) ? 1u : 0u);
                         }
-                        umma_commit(&a_empty[slot]);
+                        umma_commit_pair(&a_empty[slot], PAIR);
                         slot = (slot + 1 == NSLOT) ? 0 : slot + 1;
                     }
                     if (!ok)
                         break;
-                    umma_commit(&b_empty[bstage]);
+                    umma_commit_pair(&b_empty[bstage], PAIR);
                 }
                 if (!ok)
                     break;
-                umma_commit(&tfull[acc]);
+                umma_commit_pair(&tfull[acc], PAIR);
             }
-            umma_commit(drain);
+            umma_commit_pair(drain, 0x1);
             mbar_wait(drain, 0, kDrainLimit);
         }
     } else {
         // ---------------------------------------------------------------- epilogue (warps 2-5)
+        // This CTA's TMEM: lane = one of its 128 coordinates, columns = all of the tile's columns.
         const int quarter = warp & 3;
+        uint32_t tempty_leader[S::SETS];
+#pragma unroll
+        for (int a = 0; a < S::SETS; ++a)
+            tempty_leader[a] = cluster_addr(&tempty[a], 0);
         int itn = 0;
-        for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++itn) {
+        for (int tile = pair; tile < p.num_tiles; tile += npairs, ++itn) {
             const int acc = itn % S::SETS;
             const int use = itn / S::SETS;
             int ok = 0;
@@ -432,14 +600,18 @@ __global__ void __launch_bounds__(vg::NUM_THREADS, 1)
             }
             __syncwarp();
             tc_fence_after();
-            int g, it;
+            int g, ip;
             int64_t row0, row_end;
-            vg_tile_coords<M>(p, tile, g, row0, row_end, it);
-            const int64_t i = static_cast<int64_t>(it) * BM + quarter * 32 + lane;
+            vg_tile_coords<M>(p, tile, g, row0, row_end, ip);
+            const int64_t i = static_cast<int64_t>(ip) * 2 * BM + static_cast<int64_t>(cr) * BM +
+                              quarter * 32 + lane;
             float uacc[S::RT];
 #pragma unroll
             for (int r = 0; r < S::RT; ++r)
                 uacc[r] = 0.f;
+            // fp16 mode: the accumulator carries 2^fexp[i] (and 2^rexp[j] on residual columns)
+            const float inv_si =
+                pow2f((S::F16 && i < p.d) ? -p.fexp[static_cast<int64_t>(g) * p.d + i] : 0);
             for (int seg = 0; seg < S::SEGS; ++seg) {
                 // K block kb feeds segment kb * SEGS / nk; skip segments that received none
                 const int first = (seg * nk + S::SEGS - 1) / S::SEGS;
@@ -464,12 +636,12 @@ __global__ void __launch_bounds__(vg::NUM_THREADS, 1)
                                     if constexpr (M >= 4) {
 #pragma unroll
                                         for (int b4 = 0; b4 < M / 4; ++b4)
-                                            reinterpret_cast<float4 *>(dst)[b4] =
-                                                make_float4(v[e + 4 * b4], v[e + 4 * b4 + 1],
-                                                            v[e + 4 * b4 + 2], v[e + 4 * b4 + 3]);
+                                            reinterpret_cast<float4 *>(dst)[b4] = make_float4(
+                                                v[e + 4 * b4] * inv_si, v[e + 4 * b4 + 1] * inv_si,
+                                                v[e + 4 * b4 + 2] * inv_si, v[e + 4 * b4 + 3] * inv_si);
                                     } else {
                                         *reinterpret_cast<float2 *>(dst) =
-                                            make_float2(v[e], v[e + 1]);
+                                            make_float2(v[e] * inv_si, v[e + 1] * inv_si);
                                     }
                                 }
                             }
@@ -484,19 +656,22 @@ __global__ void __launch_bounds__(vg::NUM_THREADS, 1)
                 for (int r = 0; r < S::RT; ++r) {
                     const int64_t j = row0 + r;
                     if (j < row_end)
-                        p.uT[i * p.d_out + j] = uacc[r];
+                        p.uT[i * p.d_out + j] =
+                            S::F16 ? (uacc[r] * inv_si) * pow2f(-p.rexp[j]) : uacc[r];
                 }
             }
             tc_fence_before();
-            mbar_arrive(&tempty[acc]);
+            mbar_arrive_cluster(tempty_leader[acc]);
         }
     }
 
+    // Both CTAs stay until the pair is done: the MMAs read both CTAs' shared memory and every
+    // role signals barriers in the even CTA.
     tc_fence_before();
-    __syncthreads();
+    cluster_sync();
     tc_fence_after();
     if (warp == 1)
-        tmem_dealloc(tmem_base, TMEM_COLS);
+        tmem_dealloc_pair(tmem_base, TMEM_COLS);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -514,23 +689,47 @@ cudaError_t lnq_split_f(const float *F, int64_t d, int groups, __nv_bfloat16 *Fp
     return cudaGetLastError();
 }
 
-// Tensor map over the pieces Fp [groups * 3][d][ld]: 64 x 128 (column x row) bf16 boxes,
-// 128-byte swizzle; reads outside d x d return zeros.
-bool encode_f_pieces(CUtensorMap *map, const __nv_bfloat16 *Fp, int64_t d, int groups)
+cudaError_t lnq_split_f16(const float *F, int64_t d, int groups, __half *Fh, int32_t *fexp,
+                          cudaStream_t s)
+{
+    KernelTimer timer("lnq_split_f16", s);
+    split_f16_kernel<<<static_cast<unsigned>(d * groups), 256, 0, s>>>(F, d, Fh, fexp);
+    return cudaGetLastError();
+}
+
+cudaError_t lnq_residual_scale(const uint8_t *Q, const float *W, const float *C, int64_t d,
+                               int64_t d_out, int m, int32_t *rexp, cudaStream_t s)
+{
+    KernelTimer timer("lnq_residual_scale", s);
+    residual_scale_kernel<<<static_cast<unsigned>((d_out + 7) / 8), 256, 0, s>>>(Q, W, C, d, d_out,
+                                                                                m, rexp);
+    return cudaGetLastError();
+}
+
+// Tensor map over F's pieces [groups * planes][d][ld] (bf16: three planes per group, fp16: two):
+// 64 x 128 (column x row) boxes, 128-byte swizzle; reads outside d x d return zeros.
+static bool encode_pieces_map(CUtensorMap *map, const void *pieces, int64_t d, int planes,
+                              CUtensorMapDataType type)
 {
     auto encode = tensor_map_encoder();
     if (encode == nullptr)
         return false;
     const int64_t ld = pieces_stride(d);
     cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(d),
-                          static_cast<cuuint64_t>(groups) * 3};
+                          static_cast<cuuint64_t>(planes)};
     cuuint64_t strides[2] = {static_cast<cuuint64_t>(ld) * 2, static_cast<cuuint64_t>(d * ld) * 2};
     cuuint32_t box[3] = {vg::BK, vg::BM, 1};
     cuuint32_t estr[3] = {1, 1, 1};
-    return encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<__nv_bfloat16 *>(Fp), dims,
-                  strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+    return encode(map, type, 3, const_cast<void *>(pieces), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Tensor map over the bf16 pieces Fp [groups][3][d][ld].
+bool encode_f_pieces(CUtensorMap *map, const __nv_bfloat16 *Fp, int64_t d, int groups)
+{
+    return encode_pieces_map(map, Fp, d, groups * 3, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
 }
 
 template <int M>
@@ -539,27 +738,61 @@ static cudaError_t launch_vgemm_m(const CUtensorMap &map, VgParams p, int num_sm
 {
     using S = VgShape<M>;
     p.row_tiles_per_group = static_cast<int>((p.rows_per_group + S::RT - 1) / S::RT);
-    p.i_tiles = static_cast<int>((p.d + vg::BM - 1) / vg::BM);
+    p.i_pairs = static_cast<int>((p.d + 2 * vg::BM - 1) / (2 * vg::BM));
     const int64_t groups = p.d_out / p.rows_per_group;
-    p.num_tiles = static_cast<int>(groups * p.row_tiles_per_group * p.i_tiles);
-    const int grid = p.num_tiles < num_sms ? p.num_tiles : num_sms;
+    p.num_tiles = static_cast<int>(groups * p.row_tiles_per_group * p.i_pairs);
     cudaError_t e = cudaFuncSetAttribute(lnq_vgemm_kernel<M>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(S::SMEM));
     if (e != cudaSuccess)
         return e;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.blockDim = dim3(vg::NUM_THREADS);
+    cfg.dynamicSmemBytes = S::SMEM;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    // persistent: as many pairs as can be resident at once (at most one CTA per SM)
+    static int resident[5] = {0, 0, 0, 0, 0};
+    constexpr int slot = M == 0 ? 0 : (M == 2 ? 1 : (M == 4 ? 2 : (M == 8 ? 3 : 4)));
+    if (resident[slot] == 0) {
+        cfg.gridDim = dim3(static_cast<unsigned>(num_sms & ~1));
+        int clusters = 0;
+        if (cudaOccupancyMaxActiveClusters(&clusters, lnq_vgemm_kernel<M>, &cfg) != cudaSuccess ||
+            clusters < 1)
+            clusters = num_sms / 2;
+        resident[slot] = clusters;
+    }
+    int pairs = resident[slot];
+    if (pairs > p.num_tiles)
+        pairs = p.num_tiles;
+    if (pairs < 1)
+        pairs = 1;
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
     KernelTimer timer(name, s);
-    lnq_vgemm_kernel<M><<<grid, vg::NUM_THREADS, S::SMEM, s>>>(map, p);
+    e = cudaLaunchKernelEx(&cfg, lnq_vgemm_kernel<M>, map, p);
+    if (e != cudaSuccess)
+        return e;
     return cudaGetLastError();
 }
 
-// m in {2,4,8,16}: V and uT for every row; m == 0: uT = F r only.
-cudaError_t lnq_vgemm(const __nv_bfloat16 *Fp, int groups, const uint8_t *Q, const float *W,
+// m in {2,4,8,16}: V and uT for every row from the fp16 pieces (Fh, fexp) and the residual scales
+// rexp; residual_only: uT = F r from the exact bf16 pieces Fp.
+cudaError_t lnq_vgemm(const __nv_bfloat16 *Fp, const __half *Fh, const int32_t *fexp,
+                      const int32_t *rexp, int groups, const uint8_t *Q, const float *W,
                       const float *C, float *V, float *uT, int64_t d, int64_t d_out, int m,
                       bool residual_only, DeviceErr err, int num_sms, cudaStream_t s)
 {
     CUtensorMap map;
-    if (!encode_f_pieces(&map, Fp, d, groups))
+    const bool ok = residual_only
+                        ? encode_f_pieces(&map, Fp, d, groups)
+                        : encode_pieces_map(&map, Fh, d, groups * 2, CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
+    if (!ok)
         return cudaErrorInvalidValue;
     VgParams p{};
     p.Q = Q;
@@ -567,6 +800,8 @@ cudaError_t lnq_vgemm(const __nv_bfloat16 *Fp, int groups, const uint8_t *Q, con
     p.C = C;
     p.V = V;
     p.uT = uT;
+    p.fexp = fexp;
+    p.rexp = rexp;
     p.d = d;
     p.d_out = d_out;
     p.rows_per_group = d_out / groups;
