@@ -46,6 +46,7 @@ static bool valid_m(int m) { return m == 2 || m == 4 || m == 8 || m == 16; }
 //                   [groups][d_in] i32 | rexp [d_out] i32
 //                   | V [d_out][d_in][m] f32 | uT [d_in][d_out] f32 | dC [d_out][m] f32
 //                   | sweep history [CTAs][2 ceil(d_in / 128)][3][4 KB] (Delta pieces)
+//                   | right-operand image of the product [row tiles][K blocks][N][64] 16-bit
 //   OBJECTIVE:      the same layout (status, V and dC unused)
 //   INIT:           header
 struct FisherWs {
@@ -64,7 +65,8 @@ static FisherWs fisher_ws(int64_t n, int64_t d_in, int groups)
 }
 
 struct LnqWs {
-    size_t st_off, fp_off, fh_off, fexp_off, rexp_off, v_off, ut_off, dc_off, hist_off, total;
+    size_t st_off, fp_off, fh_off, fexp_off, rexp_off, v_off, ut_off, dc_off, hist_off, img_off,
+        total;
 };
 static LnqWs lnq_ws(int64_t d_in, int64_t d_out, int groups, int m)
 {
@@ -79,7 +81,8 @@ static LnqWs lnq_ws(int64_t d_in, int64_t d_out, int groups, int m)
     w.ut_off = align_up(w.v_off + static_cast<size_t>(d_out) * d_in * m * 4, 256);
     w.dc_off = align_up(w.ut_off + static_cast<size_t>(d_in) * d_out * 4, 256);
     w.hist_off = align_up(w.dc_off + static_cast<size_t>(d_out) * m * 4, 256);
-    w.total = align_up(w.hist_off + lnq_sweep_history_bytes(d_in, d_out, groups), 256);
+    w.img_off = align_up(w.hist_off + lnq_sweep_history_bytes(d_in, d_out, groups), 256);
+    w.total = align_up(w.img_off + lnq_vgemm_image_bytes(d_in, d_out, groups, m), 256);
     return w;
 }
 
@@ -96,6 +99,7 @@ static LnqWorkspace carve(void *ws, const LnqWs &lay)
     w.uT = reinterpret_cast<float *>(b + lay.ut_off);
     w.dC = reinterpret_cast<float *>(b + lay.dc_off);
     w.hist = b + lay.hist_off;
+    w.img = reinterpret_cast<uint16_t *>(b + lay.img_off);
     return w;
 }
 

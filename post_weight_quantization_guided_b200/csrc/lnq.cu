@@ -116,8 +116,8 @@ cudaError_t lnq_iterate_launch(const float *F, int groups, const float *W, int64
     for (int it = 0; it < iters; ++it) {
         if ((e = lnq_residual_scale(Q, W, C, d, d_out, m, w.rexp, s)) != cudaSuccess)
             return e;
-        if ((e = lnq_vgemm(w.Fp, w.Fh, w.fexp, w.rexp, groups, Q, W, C, w.V, w.uT, d, d_out, m,
-                           false, err, num_sms, s)) != cudaSuccess)
+        if ((e = lnq_vgemm(w.Fp, w.Fh, w.fexp, w.rexp, groups, Q, W, C, w.V, w.uT, w.img, d, d_out,
+                           m, false, err, num_sms, s)) != cudaSuccess)
             return e;
         if ((e = lnq_solve(w.V, w.uT, Q, C, w.dC, w.status, d, d_out, m, s)) != cudaSuccess)
             return e;
@@ -126,8 +126,8 @@ cudaError_t lnq_iterate_launch(const float *F, int groups, const float *W, int64
             return e;
     }
     if (J != nullptr) {
-        if ((e = lnq_vgemm(w.Fp, w.Fh, w.fexp, w.rexp, groups, Q, W, C, nullptr, w.uT, d, d_out,
-                           m, true, err, num_sms, s)) != cudaSuccess)
+        if ((e = lnq_vgemm(w.Fp, w.Fh, w.fexp, w.rexp, groups, Q, W, C, nullptr, w.uT, w.img, d,
+                           d_out, m, true, err, num_sms, s)) != cudaSuccess)
             return e;
         if ((e = lnq_objective_from_u(w.uT, W, C, Q, J, d, d_out, m, s)) != cudaSuccess)
             return e;

@@ -21,6 +21,7 @@ struct LnqWorkspace {
     __half *Fh;          // [groups][2][d][ld] fp16 pieces of F, rows scaled by 2^fexp
     int32_t *fexp;       // [groups][d]
     int32_t *rexp;       // [d_out] residual scales
+    uint16_t *img;       // right-operand image of the product, lnq_vgemm_image_bytes()
     float *V;            // [d_out][d][m]
     float *uT;           // [d][d_out]
     float *dC;           // [d_out][m]
@@ -41,10 +42,11 @@ cudaError_t lnq_split_f16(const float *F, int64_t d, int groups, __half *Fh, int
                           cudaStream_t s);
 cudaError_t lnq_residual_scale(const uint8_t *Q, const float *W, const float *C, int64_t d,
                                int64_t d_out, int m, int32_t *rexp, cudaStream_t s);
+size_t lnq_vgemm_image_bytes(int64_t d, int64_t d_out, int groups, int m);
 cudaError_t lnq_vgemm(const __nv_bfloat16 *Fp, const __half *Fh, const int32_t *fexp,
                       const int32_t *rexp, int groups, const uint8_t *Q, const float *W,
-                      const float *C, float *V, float *uT, int64_t d, int64_t d_out, int m,
-                      bool residual_only, DeviceErr err, int num_sms, cudaStream_t s);
+                      const float *C, float *V, float *uT, uint16_t *img, int64_t d, int64_t d_out,
+                      int m, bool residual_only, DeviceErr err, int num_sms, cudaStream_t s);
 
 // lnq_solve.cu
 cudaError_t lnq_solve(const float *V, const float *uT, const uint8_t *Q, float *C, float *dC,

@@ -35,10 +35,8 @@ namespace vg {
 constexpr int BM = 128;                          // coordinates per CTA; a pair covers 256
 constexpr int BK = 64;
 constexpr int A_TILE = BM * BK * 2;              // one bf16 piece of a 128 x 64 F tile: 16 KB
-constexpr int B_STAGES = 2;                      // stage g belongs to producer group g
-constexpr int NUM_THREADS = 448;                 // w0 TMA, w1 MMA, w2-5 epilogue, w6-13 operand
-constexpr int PRODUCER_THREADS = 256;            // two groups of 4 warps
-constexpr int GROUP_THREADS = PRODUCER_THREADS / 2;
+constexpr int B_STAGES = 4;                      // right-operand half tiles in flight
+constexpr int NUM_THREADS = 192;                 // w0 TMA, w1 MMA, w2-5 epilogue
 constexpr int EPI_THREADS = 128;
 constexpr int TMEM_COLS = 512;
 constexpr int MAX_DYN_SMEM = 232448;             // opt-in dynamic shared memory per block
@@ -65,17 +63,15 @@ struct VgShape {
     static constexpr int ONEHOT = RT * M;               // one-hot columns
     static constexpr int USED = RT * (M + 3);           // columns carrying data
     static constexpr int CHUNKS = (USED + 31) / 32;     // 32-column TMEM loads per accumulator
-    static constexpr int B_BYTES = HALF * 128;          // HALF rows x 64 k of bf16
-    static constexpr int STG_BYTES = 2 * RT * 68;       // per group: codebooks and residual scales
+    static constexpr int B_BYTES = HALF * 128;          // HALF rows x 64 k of 16-bit values
     static constexpr int A_FIT = (vg::MAX_DYN_SMEM - 1024 - vg::BAR_BYTES -
-                                  vg::B_STAGES * B_BYTES - STG_BYTES) / vg::A_TILE;
+                                  vg::B_STAGES * B_BYTES) / vg::A_TILE;
     static constexpr int A_SLOTS = A_FIT < 12 ? A_FIT : 12;
     static constexpr size_t SMEM = 1024 + static_cast<size_t>(A_SLOTS) * vg::A_TILE +
-                                   vg::B_STAGES * B_BYTES + vg::BAR_BYTES + STG_BYTES;
+                                   vg::B_STAGES * B_BYTES + vg::BAR_BYTES;
     static_assert(SETS * SEGS * NCOLS <= vg::TMEM_COLS, "TMEM holds 512 fp32 columns");
     static_assert(A_SLOTS >= 2 * PIECES, "at least two K blocks of F in flight");
     static_assert(A_SLOTS <= 32, "slot phases are kept in 32-bit masks");
-    static_assert(HALF % (M > 0 ? M : 1) == 0, "a row's one-hot columns lie in one CTA's half");
     static_assert(SMEM <= vg::MAX_DYN_SMEM, "shared memory");
 };
 
@@ -196,6 +192,101 @@ __device__ __forceinline__ void split3_f16(float x, uint16_t &p0, uint16_t &p1, 
     p2 = __half_as_ushort(c);
 }
 
+// The right operand of every (row tile, K block), written once per call of the product and then
+// loaded by TMA like F: NCOLS rows (the product's columns) x 64 coordinates, row-major
+// [row tiles][K blocks][NCOLS][64]. Column n < ONEHOT of a row tile is the indicator of class n % M
+// for its row n / M; ONEHOT <= n < USED is residual piece (n - ONEHOT) % 3 of row (n - ONEHOT) / 3;
+// the rest is zero, as is everything outside the problem. fp16 (residuals scaled by 2^rexp) when
+// there are one-hot columns, exact bf16 pieces for the residual-only product.
+template <int M>
+__global__ void __launch_bounds__(256)
+    operand_image_kernel(const uint8_t *__restrict__ Q, const float *__restrict__ W,
+                         const float *__restrict__ C, const int32_t *__restrict__ rexp, int64_t d,
+                         int64_t rows_per_group, int row_tiles_per_group, int num_rt_all, int nk,
+                         int m, uint16_t *__restrict__ img)
+{
+    using S = VgShape<M>;
+    const bool vec = (d & 7) == 0 && (reinterpret_cast<uintptr_t>(Q) & 7u) == 0 &&
+                     (reinterpret_cast<uintptr_t>(W) & 15u) == 0;
+    const int64_t total = static_cast<int64_t>(num_rt_all) * nk * S::NCOLS * 8;  // 16-byte chunks
+    for (int64_t u = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; u < total;
+         u += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int c = static_cast<int>(u & 7);
+        const int64_t rest = u >> 3;
+        const int n = static_cast<int>(rest % S::NCOLS);
+        const int64_t tb = rest / S::NCOLS;  // row tile * nk + K block
+        const int kb = static_cast<int>(tb % nk);
+        const int rt_all = static_cast<int>(tb / nk);
+        const int g = rt_all / row_tiles_per_group;
+        const int rt = rt_all - g * row_tiles_per_group;
+        const int64_t gstart = static_cast<int64_t>(g) * rows_per_group;
+        const int64_t row0 = gstart + static_cast<int64_t>(rt) * S::RT;
+        const int64_t row_end = min(row0 + S::RT, gstart + rows_per_group);
+        const int64_t k0 = static_cast<int64_t>(kb) * 64 + 8 * c;
+        uint32_t out[4] = {0u, 0u, 0u, 0u};
+        if (n < S::USED) {
+            const bool onehot = n < S::ONEHOT;
+            const int r = onehot ? n / (M > 0 ? M : 1) : (n - S::ONEHOT) / 3;
+            const int64_t j = row0 + r;
+            if (j < row_end && k0 < d) {
+                uint8_t qv[8];
+                float wv[8];
+                if (vec && k0 + 8 <= d) {
+                    const uint2 q2 = *reinterpret_cast<const uint2 *>(Q + j * d + k0);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        qv[e] = static_cast<uint8_t>(q2.x >> (8 * e));
+                        qv[4 + e] = static_cast<uint8_t>(q2.y >> (8 * e));
+                    }
+                    if (!onehot) {
+                        const float4 w0 = *reinterpret_cast<const float4 *>(W + j * d + k0);
+                        const float4 w1 = *reinterpret_cast<const float4 *>(W + j * d + k0 + 4);
+                        wv[0] = w0.x; wv[1] = w0.y; wv[2] = w0.z; wv[3] = w0.w;
+                        wv[4] = w1.x; wv[5] = w1.y; wv[6] = w1.z; wv[7] = w1.w;
+                    }
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const bool in = k0 + e < d;
+                        qv[e] = in ? Q[j * d + k0 + e] : 0xFFu;
+                        wv[e] = (in && !onehot) ? W[j * d + k0 + e] : 0.f;
+                    }
+                }
+                if (onehot) {
+                    constexpr uint16_t ONE = S::F16 ? 0x3C00u : 0x3F80u;  // 1.0 in fp16 / bf16
+                    const int b = n - r * (M > 0 ? M : 1);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        if (qv[e] == b)
+                            out[e >> 1] |= static_cast<uint32_t>(ONE) << (16 * (e & 1));
+                } else {
+                    const int pc = (n - S::ONEHOT) % 3;
+                    const float sc = S::F16 ? pow2f(rexp[j]) : 1.f;
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        if (qv[e] == 0xFFu)
+                            continue;
+                        const float rv = C[j * m + (qv[e] & (m - 1))] - wv[e];
+                        uint16_t bits;
+                        if constexpr (S::F16) {
+                            uint16_t b0, b1, b2;
+                            split3_f16(rv * sc, b0, b1, b2);
+                            bits = pc == 0 ? b0 : (pc == 1 ? b1 : b2);
+                        } else {
+                            float p0, p1, p2;
+                            split3(rv, p0, p1, p2);
+                            bits = bf16_bits(pc == 0 ? p0 : (pc == 1 ? p1 : p2));
+                        }
+                        out[e >> 1] |= static_cast<uint32_t>(bits) << (16 * (e & 1));
+                    }
+                }
+            }
+        }
+        *reinterpret_cast<uint4 *>(img + (tb * S::NCOLS + n) * 64 + 8 * c) =
+            make_uint4(out[0], out[1], out[2], out[3]);
+    }
+}
+
 struct VgParams {
     const uint8_t *Q;   // [d_out][d]
     const float *W;     // [d_out][d]
@@ -210,19 +301,18 @@ struct VgParams {
     DeviceErr err;
 };
 
-// Tile -> (group, rows [row0, row_end), coordinate pair block ip), ordered group, then pair
-// block, then row tile: the pairs running at the same time read the same 256-coordinate panel of
-// F (a few MB, served from L2), and a group's Q and W stay in L2 across its pair blocks.
+// Tile -> (group, rows [row0, row_end), coordinate pair block ip, row tile rt_all over all
+// groups). Consecutive tiles share a row tile, so the pairs running at the same time read the same
+// right-operand tiles, and a group's F pieces (fp16: 2 d^2 x 2 bytes) stay in L2 across its rows.
 template <int M>
 __device__ __forceinline__ void vg_tile_coords(const VgParams &p, int tile, int &g, int64_t &row0,
-                                               int64_t &row_end, int &ip)
+                                               int64_t &row_end, int &ip, int &rt_all)
 {
     constexpr int RT = VgShape<M>::RT;
-    const int per_group = p.i_pairs * p.row_tiles_per_group;
-    g = tile / per_group;
-    const int rem = tile - g * per_group;
-    ip = rem / p.row_tiles_per_group;
-    const int rt = rem - ip * p.row_tiles_per_group;
+    ip = tile % p.i_pairs;
+    rt_all = tile / p.i_pairs;
+    g = rt_all / p.row_tiles_per_group;
+    const int rt = rt_all - g * p.row_tiles_per_group;
     const int64_t gstart = static_cast<int64_t>(g) * p.rows_per_group;
     row0 = gstart + static_cast<int64_t>(rt) * RT;
     row_end = min(row0 + RT, gstart + p.rows_per_group);
@@ -230,7 +320,8 @@ __device__ __forceinline__ void vg_tile_coords(const VgParams &p, int tile, int 
 
 template <int M>
 __global__ void __launch_bounds__(vg::NUM_THREADS, 1)
-    lnq_vgemm_kernel(const __grid_constant__ CUtensorMap fmap, VgParams p)
+    lnq_vgemm_kernel(const __grid_constant__ CUtensorMap fmap, const __grid_constant__ CUtensorMap bmap,
+                     VgParams p)
 {
     using namespace vg;
     using S = VgShape<M>;
@@ -243,15 +334,12 @@ __global__ void __launch_bounds__(vg::NUM_THREADS, 1)
     uint64_t *bars = reinterpret_cast<uint64_t *>(b_base + B_STAGES * S::B_BYTES);
     uint64_t *a_full = bars;                                      // [NSLOT] (the even CTA's count)
     uint64_t *a_empty = a_full + NSLOT;                           // [NSLOT]
-    uint64_t *b_full = a_empty + NSLOT;                           // [B_STAGES] (even CTA's count)
+    uint64_t *b_full = a_empty + NSLOT;                           // [B_STAGES] (the even CTA's count)
     uint64_t *b_empty = b_full + B_STAGES;                        // [B_STAGES]
     uint64_t *tfull = b_empty + B_STAGES;                         // [SETS]
     uint64_t *tempty = tfull + S::SETS;                           // [SETS] (even CTA's count)
     uint64_t *drain = tempty + S::SETS;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(drain + 1);
-    // per producer group: the codebooks of the tile's rows
-    float(*stg_c)[16] = reinterpret_cast<float(*)[16]>(b_base + B_STAGES * S::B_BYTES + BAR_BYTES);
-    float *stg_t = reinterpret_cast<float *>(stg_c + 2 * S::RT);  // [2][RT] 2^rexp of each row
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -264,7 +352,7 @@ __global__ void __launch_bounds__(vg::NUM_THREADS, 1)
             mbar_init(&a_empty[s], 1);
         }
         for (int s = 0; s < B_STAGES; ++s) {
-            mbar_init(&b_full[s], 2 * GROUP_THREADS);   // one producer group of each CTA
+            mbar_init(&b_full[s], 1);
             mbar_init(&b_empty[s], 1);
         }
         for (int a = 0; a < S::SETS; ++a) {
@@ -274,6 +362,7 @@ __global__ void __launch_bounds__(vg::NUM_THREADS, 1)
         mbar_init(drain, 1);
         fence_barrier_init();
         tma_prefetch_desc(&fmap);
+        tma_prefetch_desc(&bmap);
     }
     if (warp == 1)
         tmem_alloc_pair(tmem_holder, TMEM_COLS);
@@ -285,20 +374,33 @@ __global__ void __launch_bounds__(vg::NUM_THREADS, 1)
     const long long limit = p.err.limit;
 
     if (warp == 0) {
-        // ---------------------------------------------------------------- TMA: F pieces
-        // One 16 KB piece tile of this CTA's 128 coordinates per slot, slots in round-robin order;
-        // the bytes of both CTAs are counted on the even CTA's a_full (armed by its thread for
-        // both), and the even CTA's MMA commits release the slot in both CTAs.
+        // ---------------------------------------------------------------- TMA: operands
+        // Per K block: this CTA's half of the right-operand tile (HALF rows of the operand image),
+        // then one 16 KB piece tile of F for this CTA's 128 coordinates per slot. The bytes of both
+        // CTAs are counted on the even CTA's barriers (armed by its thread for both), and the even
+        // CTA's MMA commits release stages and slots in both CTAs.
         if (lane == 0) {
-            int slot = 0;
-            uint32_t apar = 0u, aused = 0u;  // per slot: parity of the fills, ever filled
+            int slot = 0, bs = 0;
+            uint32_t apar = 0u, aused = 0u, bpar = 0u, bused = 0u;  // parity of fills, ever filled
             bool ok = true;
             for (int tile = pair; tile < p.num_tiles && ok; tile += npairs) {
-                int g, ip;
+                int g, ip, rt_all;
                 int64_t row0, row_end;
-                vg_tile_coords<M>(p, tile, g, row0, row_end, ip);
+                vg_tile_coords<M>(p, tile, g, row0, row_end, ip, rt_all);
                 const int i0 = ip * 2 * BM + static_cast<int>(cr) * BM;
                 for (int kb = 0; kb < nk && ok; ++kb) {
+                    if (!mbar_wait(&b_empty[bs], ((bpar >> bs) & 1u) ^ 1u, limit)) {
+                        raise_error(p.err, kErrTimeout, 17);
+                        ok = false;
+                        break;
+                    }
+                    if (cr == 0)
+                        mbar_arrive_expect_tx(&b_full[bs], 2 * S::B_BYTES);
+                    tma_load_2d_pair(b_base + bs * S::B_BYTES, &bmap, cluster_addr(&b_full[bs], 0), 0,
+                                     (rt_all * nk + kb) * S::NCOLS + static_cast<int>(cr) * S::HALF);
+                    bpar ^= 1u << bs;
+                    bused |= 1u << bs;
+                    bs = (bs + 1 == B_STAGES) ? 0 : bs + 1;
                     for (int pc = 0; pc < S::PIECES; ++pc) {
                         if (!mbar_wait(&a_empty[slot], ((apar >> slot) & 1u) ^ 1u, limit)) {
                             raise_error(p.err, kErrTimeout, 11);
@@ -323,194 +425,14 @@ __global__ void __launch_bounds__(vg::NUM_THREADS, 1)
                     for (int s = 0; s < NSLOT; ++s)
                         if ((aused >> s) & 1u)
                             mbar_wait(&a_full[s], ((apar >> s) & 1u) ^ 1u, kPairDrainLimit);
+                    for (int s = 0; s < B_STAGES; ++s)
+                        if ((bused >> s) & 1u)
+                            mbar_wait(&b_full[s], ((bpar >> s) & 1u) ^ 1u, kPairDrainLimit);
                 } else {
                     const long long t0 = clock64();
                     while (clock64() - t0 < kPairDrainLimit) {
                     }
                 }
-            }
-        }
-    } else if (warp >= 6) {
-        // ---------------------------------------------------------------- right operand
-        // This CTA builds right-operand columns [n_lo, n_lo + HALF) of the pair's MMA. Two groups
-        // of four warps take alternate K blocks (group g fills stage g with blocks kb = g, g + 2,
-        // ...). A thread owns (row, 8-coordinate chunk) items and writes, from its own loads of Q
-        // and W, the chunk of each one-hot row and residual-piece row of that row that falls in
-        // this CTA's columns, in the 128-byte swizzled K-major layout. Columns beyond S::USED are
-        // never written: the epilogue ignores them. The stage wait is ANDed over the group's warps
-        // so that they leave together on a timeout.
-        constexpr int GT = GROUP_THREADS;
-        constexpr int IPT = (S::RT * 8 + GT - 1) / GT;
-        const int t = threadIdx.x - 6 * 32;
-        const int grp = t / GT, tg = t - grp * GT;
-        const int bar_id = 1 + grp;
-        float(*cs)[16] = stg_c + grp * S::RT;
-        float *ts = stg_t + grp * S::RT;
-        const int n_lo = static_cast<int>(cr) * S::HALF, n_hi = n_lo + S::HALF;
-        // rows with a column in [n_lo, n_hi): one-hot columns r M + b, residual ONEHOT + 3 r + pc
-        int r_lo = S::RT, r_hi = 0;
-        if constexpr (M > 0) {
-            const int lo = min(S::RT, n_lo / M), hi = min(S::RT, n_hi / M);
-            if (lo < hi) {
-                r_lo = lo;
-                r_hi = hi;
-            }
-        }
-        {
-            const int a = n_lo - S::ONEHOT - 2, b = n_hi - S::ONEHOT - 1;
-            const int lo = a <= 0 ? 0 : (a + 2) / 3;
-            const int hi = b < 0 ? 0 : min(S::RT, b / 3 + 1);
-            if (lo < hi) {
-                r_lo = min(r_lo, lo);
-                r_hi = max(r_hi, hi);
-            }
-        }
-        const int items = r_hi > r_lo ? (r_hi - r_lo) * 8 : 0;
-        const bool vec = (p.d & 7) == 0 && (reinterpret_cast<uintptr_t>(p.Q) & 7u) == 0 &&
-                         (reinterpret_cast<uintptr_t>(p.W) & 15u) == 0;
-        const int stage = grp;
-        const uint32_t b_full_leader = cluster_addr(&b_full[stage], 0);
-        int uses = 0;
-        bool ok = true;
-        uint2 qn[IPT];   // next block's classes (0xFF outside the problem)
-        float4 wn[IPT][2];
-        auto has_res = [&](int r) { return S::ONEHOT + 3 * r + 2 >= n_lo && S::ONEHOT + 3 * r < n_hi; };
-        auto fetch = [&](int64_t row0, int64_t row_end, int64_t k0) {
-#pragma unroll
-            for (int s2 = 0; s2 < IPT; ++s2) {
-                const int e = tg + s2 * GT;
-                const int r = r_lo + (e >> 3), c = e & 7;
-                const int64_t j = row0 + r, k = k0 + 8 * c;
-                qn[s2] = make_uint2(0xFFFFFFFFu, 0xFFFFFFFFu);
-                wn[s2][0] = wn[s2][1] = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (e < items && j < row_end && k < p.d) {
-                    const bool need_w = has_res(r);
-                    if (vec && k + 8 <= p.d) {
-                        qn[s2] = *reinterpret_cast<const uint2 *>(p.Q + j * p.d + k);
-                        if (need_w) {
-                            wn[s2][0] = *reinterpret_cast<const float4 *>(p.W + j * p.d + k);
-                            wn[s2][1] = *reinterpret_cast<const float4 *>(p.W + j * p.d + k + 4);
-                        }
-                    } else {
-                        uint32_t q2[2] = {0u, 0u};
-                        float wv[8];
-#pragma unroll
-                        for (int e8 = 0; e8 < 8; ++e8) {
-                            const bool in = k + e8 < p.d;
-                            q2[e8 >> 2] |= static_cast<uint32_t>(in ? p.Q[j * p.d + k + e8] : 0xFFu)
-                                           << (8 * (e8 & 3));
-                            wv[e8] = (in && need_w) ? p.W[j * p.d + k + e8] : 0.f;
-                        }
-                        qn[s2] = make_uint2(q2[0], q2[1]);
-                        wn[s2][0] = make_float4(wv[0], wv[1], wv[2], wv[3]);
-                        wn[s2][1] = make_float4(wv[4], wv[5], wv[6], wv[7]);
-                    }
-                }
-            }
-        };
-        for (int tile = pair; tile < p.num_tiles && ok; tile += npairs) {
-            int g, ip;
-            int64_t row0, row_end;
-            vg_tile_coords<M>(p, tile, g, row0, row_end, ip);
-            if (grp >= nk)
-                continue;
-            // the group's copy of the tile's codebooks (the previous tile's readers are done:
-            // every thread passed the group's last stage wait after its last read)
-            named_bar_sync(bar_id, GT);
-            for (int e = tg; e < S::RT * 16; e += GT) {
-                const int r = e >> 4, b = e & 15;
-                const int64_t j = row0 + r;
-                cs[r][b] = (j < row_end && b < p.m) ? p.C[j * p.m + b] : 0.f;
-            }
-            if constexpr (S::F16) {
-                for (int r = tg; r < S::RT; r += GT)
-                    ts[r] = pow2f((row0 + r < row_end) ? p.rexp[row0 + r] : 0);
-            }
-            fetch(row0, row_end, static_cast<int64_t>(grp) * BK);
-            named_bar_sync(bar_id, GT);
-            for (int kb = grp; kb < nk; kb += 2) {
-                const int mine = mbar_wait(&b_empty[stage], (uses & 1) ^ 1, limit) ? 1 : 0;
-                if (!named_bar_and(bar_id, GT, mine)) {
-                    if (tg == 0)
-                        raise_error(p.err, kErrTimeout, 12);
-                    ok = false;
-                    break;
-                }
-                uint2 qc[IPT];
-                float4 wc[IPT][2];
-#pragma unroll
-                for (int s2 = 0; s2 < IPT; ++s2) {
-                    qc[s2] = qn[s2];
-                    wc[s2][0] = wn[s2][0];
-                    wc[s2][1] = wn[s2][1];
-                }
-                if (kb + 2 < nk)
-                    fetch(row0, row_end, static_cast<int64_t>(kb + 2) * BK);
-                uint8_t *sb = b_base + stage * S::B_BYTES;
-#pragma unroll
-                for (int s2 = 0; s2 < IPT; ++s2) {
-                    const int e = tg + s2 * GT;
-                    if (e >= items)
-                        continue;
-                    const int r = r_lo + (e >> 3), c = e & 7;
-                    if (has_res(r)) {
-                        // residual pieces of the chunk's 8 coordinates
-                        const float wv[8] = {wc[s2][0].x, wc[s2][0].y, wc[s2][0].z, wc[s2][0].w,
-                                             wc[s2][1].x, wc[s2][1].y, wc[s2][1].z, wc[s2][1].w};
-                        uint32_t pk[3][4] = {};
-#pragma unroll
-                        for (int e8 = 0; e8 < 8; ++e8) {
-                            const uint32_t qv = ((e8 < 4 ? qc[s2].x : qc[s2].y) >> (8 * (e8 & 3))) & 0xFFu;
-                            uint16_t b0 = 0, b1 = 0, b2 = 0;
-                            if (qv != 0xFFu) {
-                                const float rv = cs[r][qv & (p.m - 1)] - wv[e8];
-                                if constexpr (S::F16) {
-                                    split3_f16(rv * ts[r], b0, b1, b2);
-                                } else {
-                                    float p0, p1, p2;
-                                    split3(rv, p0, p1, p2);
-                                    b0 = bf16_bits(p0);
-                                    b1 = bf16_bits(p1);
-                                    b2 = bf16_bits(p2);
-                                }
-                            }
-                            const int sh = 16 * (e8 & 1);
-                            pk[0][e8 >> 1] |= static_cast<uint32_t>(b0) << sh;
-                            pk[1][e8 >> 1] |= static_cast<uint32_t>(b1) << sh;
-                            pk[2][e8 >> 1] |= static_cast<uint32_t>(b2) << sh;
-                        }
-#pragma unroll
-                        for (int pc = 0; pc < 3; ++pc) {
-                            const int n = S::ONEHOT + 3 * r + pc - n_lo;
-                            if (n >= 0 && n < S::HALF)
-                                *reinterpret_cast<uint4 *>(sb + n * 128 + ((c ^ (n & 7)) << 4)) =
-                                    make_uint4(pk[pc][0], pk[pc][1], pk[pc][2], pk[pc][3]);
-                        }
-                    }
-                    if constexpr (M > 0) {
-                        if (r * M >= n_lo && r * M < n_hi) {
-#pragma unroll
-                            for (int b = 0; b < M; ++b) {
-                                const int n = r * M + b - n_lo;
-                                const uint32_t bbbb = 0x01010101u * static_cast<uint32_t>(b);
-                                const uint32_t m0 = __vcmpeq4(qc[s2].x, bbbb), m1 = __vcmpeq4(qc[s2].y, bbbb);
-                                // byte e of the mask (0xFF or 0) -> 1.0 or 0 in half-word e
-                                // (fp16 1.0 = 0x3C00, bf16 1.0 = 0x3F80)
-                                constexpr uint32_t ONE2 = S::F16 ? 0x3C003C00u : 0x3F803F80u;
-                                *reinterpret_cast<uint4 *>(sb + n * 128 + ((c ^ (n & 7)) << 4)) =
-                                    make_uint4(__byte_perm(m0, 0u, 0x1100) & ONE2,
-                                               __byte_perm(m0, 0u, 0x3322) & ONE2,
-                                               __byte_perm(m1, 0u, 0x1100) & ONE2,
-                                               __byte_perm(m1, 0u, 0x3322) & ONE2);
-                            }
-                        }
-                    }
-                }
-                // make the generic-proxy writes visible to the tensor core (async proxy), then
-                // count them on the even CTA's stage barrier
-                fence_proxy_async_smem();
-                mbar_arrive_cluster(b_full_leader);
-                ++uses;
             }
         }
     } else if (warp == 1) {
@@ -519,7 +441,7 @@ __global__ void __launch_bounds__(vg::NUM_THREADS, 1)
         // both CTAs' F tiles, issue four K=16 MMAs (M = 256 over the pair) and release the slot
         // in both CTAs; release the stage after the block, the accumulator after the tile.
         if (cr == 0 && lane == 0) {
-            int slot = 0;
+            int slot = 0, bstage = 0;
             uint32_t aph = 0u, bph = 0u;  // phase parity per slot / stage
             bool ok = true;
             int itn = 0;
@@ -533,8 +455,7 @@ __global__ void __launch_bounds__(vg::NUM_THREADS, 1)
                 }
                 tc_fence_after();
                 for (int kb = 0; kb < nk && ok; ++kb) {
-                    const int bstage = kb & 1;  // K block kb comes from producer group kb & 1
-                    if (!mbar_wait_cluster(&b_full[bstage], (bph >> bstage) & 1u, limit)) {
+                    if (!mbar_wait(&b_full[bstage], (bph >> bstage) & 1u, limit)) {
                         raise_error(p.err, kErrTimeout, 14);
                         ok = false;
                         break;
@@ -569,6 +490,7 @@ __global__ void __launch_bounds__(vg::NUM_THREADS, 1)
                     if (!ok)
                         break;
                     umma_commit_pair(&b_empty[bstage], PAIR);
+                    bstage = (bstage + 1 == B_STAGES) ? 0 : bstage + 1;
                 }
                 if (!ok)
                     break;
@@ -600,9 +522,9 @@ __global__ void __launch_bounds__(vg::NUM_THREADS, 1)
             }
             __syncwarp();
             tc_fence_after();
-            int g, ip;
+            int g, ip, rt_all;
             int64_t row0, row_end;
-            vg_tile_coords<M>(p, tile, g, row0, row_end, ip);
+            vg_tile_coords<M>(p, tile, g, row0, row_end, ip, rt_all);
             const int64_t i = static_cast<int64_t>(ip) * 2 * BM + static_cast<int64_t>(cr) * BM +
                               quarter * 32 + lane;
             float uacc[S::RT];
@@ -665,8 +587,8 @@ __global__ void __launch_bounds__(vg::NUM_THREADS, 1)
         }
     }
 
-    // Both CTAs stay until the pair is done: the MMAs read both CTAs' shared memory and every
-    // role signals barriers in the even CTA.
+    // Both CTAs stay until the pair is done: the MMAs read both CTAs' shared memory and the
+    // copies and epilogues of both signal barriers in the even CTA.
     tc_fence_before();
     cluster_sync();
     tc_fence_after();
@@ -732,15 +654,74 @@ bool encode_f_pieces(CUtensorMap *map, const __nv_bfloat16 *Fp, int64_t d, int g
     return encode_pieces_map(map, Fp, d, groups * 3, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
 }
 
+// Right-operand image rows for m (M > 0 layout) or for the residual-only product: the workspace
+// holds the larger of the two.
 template <int M>
-static cudaError_t launch_vgemm_m(const CUtensorMap &map, VgParams p, int num_sms, cudaStream_t s,
-                                  const char *name)
+static int64_t image_rows_m(int64_t d, int64_t d_out, int groups)
+{
+    using S = VgShape<M>;
+    const int64_t R = d_out / groups;
+    const int64_t nk = (d + vg::BK - 1) / vg::BK;
+    return groups * ((R + S::RT - 1) / S::RT) * nk * S::NCOLS;
+}
+
+size_t lnq_vgemm_image_bytes(int64_t d, int64_t d_out, int groups, int m)
+{
+    int64_t rows = image_rows_m<0>(d, d_out, groups);
+    int64_t rm = 0;
+    switch (m) {
+    case 2: rm = image_rows_m<2>(d, d_out, groups); break;
+    case 4: rm = image_rows_m<4>(d, d_out, groups); break;
+    case 8: rm = image_rows_m<8>(d, d_out, groups); break;
+    case 16: rm = image_rows_m<16>(d, d_out, groups); break;
+    }
+    if (rm > rows)
+        rows = rm;
+    return static_cast<size_t>(rows) * 64 * 2;
+}
+
+template <int M>
+static cudaError_t launch_vgemm_m(const CUtensorMap &map, VgParams p, uint16_t *img, int num_sms,
+                                  cudaStream_t s, const char *name)
 {
     using S = VgShape<M>;
     p.row_tiles_per_group = static_cast<int>((p.rows_per_group + S::RT - 1) / S::RT);
     p.i_pairs = static_cast<int>((p.d + 2 * vg::BM - 1) / (2 * vg::BM));
     const int64_t groups = p.d_out / p.rows_per_group;
-    p.num_tiles = static_cast<int>(groups * p.row_tiles_per_group * p.i_pairs);
+    const int nk = static_cast<int>((p.d + vg::BK - 1) / vg::BK);
+    const int64_t num_rt_all = groups * p.row_tiles_per_group;
+    const int64_t img_rows = num_rt_all * nk * S::NCOLS;
+    if (img_rows > 0x7fffffffLL || num_rt_all * p.i_pairs > 0x7fffffffLL)
+        return cudaErrorInvalidValue;
+    p.num_tiles = static_cast<int>(num_rt_all * p.i_pairs);
+    {
+        KernelTimer timer(S::F16 ? "lnq_operand_image" : "lnq_residual_image", s);
+        const int64_t chunks = img_rows * 8;
+        int64_t blocks = (chunks + 255) / 256;
+        if (blocks > static_cast<int64_t>(num_sms) * 16)
+            blocks = static_cast<int64_t>(num_sms) * 16;
+        operand_image_kernel<M><<<static_cast<unsigned>(blocks), 256, 0, s>>>(
+            p.Q, p.W, p.C, p.rexp, p.d, p.rows_per_group, p.row_tiles_per_group,
+            static_cast<int>(num_rt_all), nk, p.m, img);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess)
+            return e;
+    }
+    CUtensorMap bmap;
+    {
+        auto encode = tensor_map_encoder();
+        if (encode == nullptr)
+            return cudaErrorInvalidValue;
+        cuuint64_t dims[2] = {64, static_cast<cuuint64_t>(img_rows)};
+        cuuint64_t strides[1] = {128};
+        cuuint32_t box[2] = {64, static_cast<cuuint32_t>(S::HALF)};
+        cuuint32_t estr[2] = {1, 1};
+        if (encode(&bmap, S::F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                   2, img, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
+    }
     cudaError_t e = cudaFuncSetAttribute(lnq_vgemm_kernel<M>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(S::SMEM));
@@ -775,7 +756,7 @@ static cudaError_t launch_vgemm_m(const CUtensorMap &map, VgParams p, int num_sm
         pairs = 1;
     cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
     KernelTimer timer(name, s);
-    e = cudaLaunchKernelEx(&cfg, lnq_vgemm_kernel<M>, map, p);
+    e = cudaLaunchKernelEx(&cfg, lnq_vgemm_kernel<M>, map, bmap, p);
     if (e != cudaSuccess)
         return e;
     return cudaGetLastError();
@@ -785,8 +766,8 @@ static cudaError_t launch_vgemm_m(const CUtensorMap &map, VgParams p, int num_sm
 // rexp; residual_only: uT = F r from the exact bf16 pieces Fp.
 cudaError_t lnq_vgemm(const __nv_bfloat16 *Fp, const __half *Fh, const int32_t *fexp,
                       const int32_t *rexp, int groups, const uint8_t *Q, const float *W,
-                      const float *C, float *V, float *uT, int64_t d, int64_t d_out, int m,
-                      bool residual_only, DeviceErr err, int num_sms, cudaStream_t s)
+                      const float *C, float *V, float *uT, uint16_t *img, int64_t d, int64_t d_out,
+                      int m, bool residual_only, DeviceErr err, int num_sms, cudaStream_t s)
 {
     CUtensorMap map;
     const bool ok = residual_only
@@ -808,12 +789,12 @@ cudaError_t lnq_vgemm(const __nv_bfloat16 *Fp, const __half *Fh, const int32_t *
     p.m = m;
     p.err = err;
     if (residual_only)
-        return launch_vgemm_m<0>(map, p, num_sms, s, "lnq_residual_gemm");
+        return launch_vgemm_m<0>(map, p, img, num_sms, s, "lnq_residual_gemm");
     switch (m) {
-    case 2: return launch_vgemm_m<2>(map, p, num_sms, s, "lnq_vgemm");
-    case 4: return launch_vgemm_m<4>(map, p, num_sms, s, "lnq_vgemm");
-    case 8: return launch_vgemm_m<8>(map, p, num_sms, s, "lnq_vgemm");
-    case 16: return launch_vgemm_m<16>(map, p, num_sms, s, "lnq_vgemm");
+    case 2: return launch_vgemm_m<2>(map, p, img, num_sms, s, "lnq_vgemm");
+    case 4: return launch_vgemm_m<4>(map, p, img, num_sms, s, "lnq_vgemm");
+    case 8: return launch_vgemm_m<8>(map, p, img, num_sms, s, "lnq_vgemm");
+    case 16: return launch_vgemm_m<16>(map, p, img, num_sms, s, "lnq_vgemm");
     }
     return cudaErrorInvalidValue;
 }
