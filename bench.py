@@ -70,10 +70,17 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", self.ident, f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "20"],
                 stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
+            return
+        # the timed region starts once the sampler is producing samples
+        t0 = time.time()
+        while time.time() - t0 < 10.0:
+            if os.path.getsize(self.path) > 0:
+                break
+            time.sleep(0.01)
 
     def stop(self):
         if self.proc is None:
@@ -121,6 +128,17 @@ def algorithmic_work(layer, kernel: str, launches: int, moves_per_sweep: float):
     ld = (d + 7) // 8 * 8
     if kernel == "lnq_split_f":
         return 4.0 * g * d * d + 6.0 * g * d * ld, "byte"           # read F, write 3 bf16 pieces
+    if kernel in ("lnq_operand_image", "lnq_residual_image"):
+        # write the right-operand image (N columns x d coordinates x 2 bytes per row tile), read Q
+        # and W once
+        rt = max(1, 256 // (m + 3)) if kernel == "lnq_operand_image" else 128 // 3
+        ncols = 256 if kernel == "lnq_operand_image" else 128
+        tiles = g * -(-(dout // g) // rt)
+        return tiles * ncols * (-(-d // 64) * 64) * 2.0 + 5.0 * dout * d, "byte"
+    if kernel == "lnq_split_f16":
+        return 4.0 * g * d * d + 4.0 * g * d * ld, "byte"           # read F, write 2 fp16 pieces
+    if kernel == "lnq_residual_scale":
+        return 5.0 * dout * d, "byte"                               # read W and Q
     if kernel == "lnq_vgemm":
         # the dense product F x [P_j | r_j] over all rows: 2 d^2 (m + 1) flops per row
         return 2.0 * d * d * (m + 1) * dout, "flop"
@@ -137,12 +155,13 @@ def algorithmic_work(layer, kernel: str, launches: int, moves_per_sweep: float):
     return 0.0, "unknown"
 
 
-# tcgen05 work per unit of algorithmic work: F enters as three exact bf16 pieces; the one-hot
-# columns are exact, the residual columns are three pieces as well (nine products).
+# tcgen05 work per unit of algorithmic work. The V/u product takes F as two fp16 pieces against
+# m exact one-hot columns and three residual-piece columns per row; the objective's residual
+# product takes F as three exact bf16 pieces against three residual pieces (nine products).
 def hw_flop_factor(layer, kernel):
     m = layer.m
     if kernel == "lnq_vgemm":
-        return (3.0 * m + 9.0) / (m + 1)
+        return (2.0 * m + 6.0) / (m + 1)
     if kernel == "lnq_residual_gemm":
         return 9.0
     return None

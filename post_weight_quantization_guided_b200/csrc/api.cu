@@ -44,7 +44,7 @@ static bool valid_m(int m) { return m == 2 || m == 4 || m == 8 || m == 16; }
 //   QUANTIZE_ROWS:  header | status [d_out] i32 | Fp [groups][3][d_in][ld] bf16 (ld = d_in
 //                   rounded up to a multiple of 8) | Fh [groups][2][d_in][ld] f16 | fexp
 //                   [groups][d_in] i32 | rexp [d_out] i32
-//                   | V [d_out][d_in][m] f32 | uT [d_in][d_out] f32 | dC [d_out][m] f32
+//                   | V [d_out][d_in][m] f32 | U [d_out][d_in] f32 (u = F r) | dC [d_out][m] f32
 //                   | sweep history [CTAs][2 ceil(d_in / 128)][3][4 KB] (Delta pieces)
 //                   | right-operand image of the product [row tiles][K blocks][N][64] 16-bit
 //   OBJECTIVE:      the same layout (status, V and dC unused)
@@ -96,7 +96,7 @@ static LnqWorkspace carve(void *ws, const LnqWs &lay)
     w.fexp = reinterpret_cast<int32_t *>(b + lay.fexp_off);
     w.rexp = reinterpret_cast<int32_t *>(b + lay.rexp_off);
     w.V = reinterpret_cast<float *>(b + lay.v_off);
-    w.uT = reinterpret_cast<float *>(b + lay.ut_off);
+    w.U = reinterpret_cast<float *>(b + lay.ut_off);
     w.dC = reinterpret_cast<float *>(b + lay.dc_off);
     w.hist = b + lay.hist_off;
     w.img = reinterpret_cast<uint16_t *>(b + lay.img_off);

@@ -116,20 +116,20 @@ cudaError_t lnq_iterate_launch(const float *F, int groups, const float *W, int64
     for (int it = 0; it < iters; ++it) {
         if ((e = lnq_residual_scale(Q, W, C, d, d_out, m, w.rexp, s)) != cudaSuccess)
             return e;
-        if ((e = lnq_vgemm(w.Fp, w.Fh, w.fexp, w.rexp, groups, Q, W, C, w.V, w.uT, w.img, d, d_out,
+        if ((e = lnq_vgemm(w.Fp, w.Fh, w.fexp, w.rexp, groups, Q, W, C, w.V, w.U, w.img, d, d_out,
                            m, false, err, num_sms, s)) != cudaSuccess)
             return e;
-        if ((e = lnq_solve(w.V, w.uT, Q, C, w.dC, w.status, d, d_out, m, s)) != cudaSuccess)
+        if ((e = lnq_solve(w.V, w.U, Q, C, w.dC, w.status, d, d_out, m, s)) != cudaSuccess)
             return e;
-        if ((e = lnq_sweep(F, w.Fp, groups, w.V, w.dC, w.uT, C, Q, w.hist, d, d_out, m, err,
+        if ((e = lnq_sweep(F, w.Fp, groups, w.V, w.dC, w.U, C, Q, w.hist, d, d_out, m, err,
                            s)) != cudaSuccess)
             return e;
     }
     if (J != nullptr) {
-        if ((e = lnq_vgemm(w.Fp, w.Fh, w.fexp, w.rexp, groups, Q, W, C, nullptr, w.uT, w.img, d,
+        if ((e = lnq_vgemm(w.Fp, w.Fh, w.fexp, w.rexp, groups, Q, W, C, nullptr, w.U, w.img, d,
                            d_out, m, true, err, num_sms, s)) != cudaSuccess)
             return e;
-        if ((e = lnq_objective_from_u(w.uT, W, C, Q, J, d, d_out, m, s)) != cudaSuccess)
+        if ((e = lnq_objective_from_u(w.U, W, C, Q, J, d, d_out, m, s)) != cudaSuccess)
             return e;
     }
     return cudaGetLastError();

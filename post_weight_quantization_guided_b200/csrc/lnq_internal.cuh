@@ -23,7 +23,7 @@ struct LnqWorkspace {
     int32_t *rexp;       // [d_out] residual scales
     uint16_t *img;       // right-operand image of the product, lnq_vgemm_image_bytes()
     float *V;            // [d_out][d][m]
-    float *uT;           // [d][d_out]
+    float *U;            // [d_out][d] u = F r per row
     float *dC;           // [d_out][m]
     uint8_t *hist;       // sweep history, lnq_sweep_history_bytes()
 };
@@ -45,20 +45,20 @@ cudaError_t lnq_residual_scale(const uint8_t *Q, const float *W, const float *C,
 size_t lnq_vgemm_image_bytes(int64_t d, int64_t d_out, int groups, int m);
 cudaError_t lnq_vgemm(const __nv_bfloat16 *Fp, const __half *Fh, const int32_t *fexp,
                       const int32_t *rexp, int groups, const uint8_t *Q, const float *W,
-                      const float *C, float *V, float *uT, uint16_t *img, int64_t d, int64_t d_out,
+                      const float *C, float *V, float *U, uint16_t *img, int64_t d, int64_t d_out,
                       int m, bool residual_only, DeviceErr err, int num_sms, cudaStream_t s);
 
 // lnq_solve.cu
-cudaError_t lnq_solve(const float *V, const float *uT, const uint8_t *Q, float *C, float *dC,
+cudaError_t lnq_solve(const float *V, const float *U, const uint8_t *Q, float *C, float *dC,
                       int32_t *status, int64_t d, int64_t d_out, int m, cudaStream_t s);
-cudaError_t lnq_objective_from_u(const float *uT, const float *W, const float *C,
+cudaError_t lnq_objective_from_u(const float *U, const float *W, const float *C,
                                  const uint8_t *Q, double *J, int64_t d, int64_t d_out, int m,
                                  cudaStream_t s);
 
 // lnq_sweep.cu
 size_t lnq_sweep_history_bytes(int64_t d, int64_t d_out, int groups);
 cudaError_t lnq_sweep(const float *F, const __nv_bfloat16 *Fp, int groups, const float *V,
-                      const float *dC, const float *uT, const float *C, uint8_t *Q, uint8_t *hist,
+                      const float *dC, const float *U, const float *C, uint8_t *Q, uint8_t *hist,
                       int64_t d, int64_t d_out, int m, DeviceErr err, cudaStream_t s);
 
 }  // namespace lnq

@@ -4,12 +4,14 @@
 // c <- (P^T F P)^-1 P^T F w, and the objective (w^ - w)^T F (w^ - w) of each row.
 //
 // solve_kernel (one CTA per row). From V = F P and u = F r (lnq_vgemm.cu) it forms
-// M = P^T V and t = P^T u in fp64. The coordinates are sorted by class first (a stable
-// counting sort), and every sum runs in a fixed order, so results do not depend on scheduling.
-// An fp64 Cholesky over the non-empty codewords then solves M dc = -t (the closed-form update in
+// M = P^T V and t = P^T u, streaming the row's V and u once with coalesced loads: fp32 partial
+// sums over 32-coordinate chunks (a few terms each), fp64 across chunks; every sum runs in a
+// fixed order, so results do not depend on scheduling. An fp64 Cholesky over the
+// non-empty codewords (one warp, a lane per row) then solves M dc = -t (the closed-form update in
 // residual form), and the kernel writes c + dc in fp32 together with the exact fp32 change.
 //
-// objective_u_kernel: J_j = r_j^T u_j with u = F r from the residual-only product, fp64 sums.
+// objective_u_kernel: J_j = r_j^T u_j with u = F r from the residual-only product, fp64 sums in a
+// fixed order.
 #include "common.cuh"
 #include "lnq_internal.cuh"
 #include "profile.cuh"
@@ -17,148 +19,205 @@
 namespace lnq {
 
 constexpr int kSolveThreads = 256;
-constexpr int kObjWarps = 8;
+constexpr int kObjThreads = 256;
 
 // ------------------------------------------------------------------------------------------
 // codebook solve
 // ------------------------------------------------------------------------------------------
 template <int M>
 __global__ void __launch_bounds__(kSolveThreads)
-    solve_kernel(const float *__restrict__ V, const float *__restrict__ uT,
+    solve_kernel(const float *__restrict__ V, const float *__restrict__ U,
                  const uint8_t *__restrict__ Q, float *__restrict__ C, float *__restrict__ dC,
-                 int32_t *__restrict__ status, int64_t d, int64_t d_out)
+                 int32_t *__restrict__ status, int64_t d)
 {
-    constexpr int T = kSolveThreads;
+    constexpr int NW = kSolveThreads / 32;
     constexpr int PAIRS = M * M;
-    constexpr int PPARTS = T / PAIRS;  // threads per (class, column) pair: 1, 4, 16, 64
-    constexpr int TPARTS = T / M;      // threads per class for t
-    extern __shared__ __align__(16) uint8_t sm[];
-    int *cnt = reinterpret_cast<int *>(sm);               // [T][M] per-thread class counts
-    int *list = cnt + T * M;                              // [d] class-sorted coordinates
-    __shared__ int start[M + 1];
-    __shared__ double Msum[PAIRS * PPARTS], tsum[M * TPARTS];
-    __shared__ double Mm[M * M], tv[M], L[M * M], y[M];
+    constexpr int PPL = (PAIRS + 31) / 32;     // (class, column) pairs per lane, same class
+    __shared__ float stv[NW][32][M + 1];       // staged V rows and u of 32 coordinates
+    __shared__ uint8_t stq[NW][32];
+    __shared__ double Mp[NW][PAIRS], tp[NW][M];
+    __shared__ int cp[NW][M];
+    __shared__ double Mm[PAIRS], tv[M], Ls[16][16];
+    __shared__ int cnt[M];
 
     const int64_t j = blockIdx.x;
-    const int tid = threadIdx.x;
-    const uint8_t *q = Q + j * d;
-    const int64_t chunk = (d + T - 1) / T;
-    const int64_t lo = min(d, tid * chunk), hi = min(d, lo + chunk);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const float *Vj = V + j * d * M;
+    const float *Uj = U + j * d;
+    const uint8_t *qj = Q + j * d;
 
-    // 1. stable counting sort of the coordinates by class
-    for (int b = 0; b < M; ++b)
-        cnt[tid * M + b] = 0;
-    for (int64_t i = lo; i < hi; ++i)
-        cnt[tid * M + (q[i] & (M - 1))] += 1;
-    __syncthreads();
-    if (tid < M) {  // exclusive scan over threads, per class
-        int run = 0;
-        for (int t = 0; t < T; ++t) {
-            const int c = cnt[t * M + tid];
-            cnt[t * M + tid] = run;
-            run += c;
-        }
-        start[tid + 1] = run;  // class total, turned into starts below
-    }
-    __syncthreads();
-    if (tid == 0) {
-        start[0] = 0;
-        for (int b = 0; b < M; ++b)
-            start[b + 1] += start[b];
-    }
-    __syncthreads();
-    {
-        int off[M];
+    // 1. M[a][b] = sum over class-a coordinates of V[i][b], t[a] = sum of u[i], per warp in a
+    //    fixed order: warp w takes 32-coordinate chunks w, w + NW, ...; a chunk is staged with
+    //    coalesced loads, then lane (a, columns b0..b0+PPL) adds the staged rows of class a.
+    const int p0 = lane * PPL;
+    const bool owner = p0 < PAIRS;
+    const int a = owner ? p0 / M : M;          // M: no class
+    const int b0 = owner ? p0 % M : 0;
+    double acc[PPL], tacc = 0.0;
+    int n = 0;
 #pragma unroll
-        for (int b = 0; b < M; ++b)
-            off[b] = start[b] + cnt[tid * M + b];
-        for (int64_t i = lo; i < hi; ++i) {
-            const int b = q[i] & (M - 1);
+    for (int q = 0; q < PPL; ++q)
+        acc[q] = 0.0;
+    const int64_t nch = (d + 31) / 32;
+    for (int64_t ch = warp; ch < nch; ch += NW) {
+        const int64_t i = ch * 32 + lane;
+        if (i < d) {
+            const float *vi = Vj + i * M;
+            if constexpr (M >= 4) {
 #pragma unroll
-            for (int bb = 0; bb < M; ++bb)
-                if (bb == b)
-                    list[off[bb]++] = static_cast<int>(i);
+                for (int b4 = 0; b4 < M / 4; ++b4) {
+                    const float4 x = reinterpret_cast<const float4 *>(vi)[b4];
+                    stv[warp][lane][4 * b4] = x.x;
+                    stv[warp][lane][4 * b4 + 1] = x.y;
+                    stv[warp][lane][4 * b4 + 2] = x.z;
+                    stv[warp][lane][4 * b4 + 3] = x.w;
+                }
+            } else {
+                const float2 x = *reinterpret_cast<const float2 *>(vi);
+                stv[warp][lane][0] = x.x;
+                stv[warp][lane][1] = x.y;
+            }
+            stv[warp][lane][M] = Uj[i];
+            stq[warp][lane] = qj[i] & (M - 1);
+        } else {
+            stq[warp][lane] = 0xFF;
+        }
+        __syncwarp();
+        // the chunk's coordinates of this lane's class (one ballot per class), visited in lane
+        // order: fp32 partials of the chunk, added to the fp64 sums once per chunk
+        const int mq = stq[warp][lane];
+        uint32_t mine = 0u;
+#pragma unroll
+        for (int c = 0; c < M; ++c) {
+            const uint32_t mc = __ballot_sync(0xffffffffu, mq == c);
+            mine = (a == c) ? mc : mine;
+        }
+        float pf[PPL], tf = 0.f;
+#pragma unroll
+        for (int q = 0; q < PPL; ++q)
+            pf[q] = 0.f;
+        n += __popc(mine);
+        while (mine != 0u) {
+            const int e = __ffs(mine) - 1;
+            mine &= mine - 1u;
+#pragma unroll
+            for (int q = 0; q < PPL; ++q)
+                pf[q] += stv[warp][e][b0 + q];
+            tf += stv[warp][e][M];
+        }
+#pragma unroll
+        for (int q = 0; q < PPL; ++q)
+            acc[q] += static_cast<double>(pf[q]);
+        tacc += static_cast<double>(tf);
+        __syncwarp();
+    }
+    if (owner) {
+#pragma unroll
+        for (int q = 0; q < PPL; ++q)
+            Mp[warp][p0 + q] = acc[q];
+        if (b0 == 0) {
+            tp[warp][a] = tacc;
+            cp[warp][a] = n;
         }
     }
     __syncthreads();
-
-    // 2. M[a][b] = sum_{i in class a} V[i][b], t[a] = sum_{i in class a} u[i]  (fp64, fixed order)
-    {
-        const int pair = tid / PPARTS, part = tid % PPARTS;
-        const int a = pair / M, b = pair % M;
-        double acc = 0.0;
-        for (int e = start[a] + part; e < start[a + 1]; e += PPARTS)
-            acc += static_cast<double>(V[(j * d + list[e]) * M + b]);
-        Msum[pair * PPARTS + part] = acc;
-        const int ta = tid / TPARTS, tpart = tid % TPARTS;
-        double tacc = 0.0;
-        for (int e = start[ta] + tpart; e < start[ta + 1]; e += TPARTS)
-            tacc += static_cast<double>(uT[static_cast<int64_t>(list[e]) * d_out + j]);
-        tsum[ta * TPARTS + tpart] = tacc;
-    }
-    __syncthreads();
-    if (tid < PAIRS) {
+    for (int e = threadIdx.x; e < PAIRS; e += kSolveThreads) {
         double s = 0.0;
-        for (int part = 0; part < PPARTS; ++part)
-            s += Msum[tid * PPARTS + part];
-        Mm[tid] = s;
+        for (int w = 0; w < NW; ++w)
+            s += Mp[w][e];
+        Mm[e] = s;
     }
-    if (tid < M) {
+    if (threadIdx.x < M) {
         double s = 0.0;
-        for (int part = 0; part < TPARTS; ++part)
-            s += tsum[tid * TPARTS + part];
-        tv[tid] = s;
+        int c = 0;
+        for (int w = 0; w < NW; ++w) {
+            s += tp[w][threadIdx.x];
+            c += cp[w][threadIdx.x];
+        }
+        tv[threadIdx.x] = s;
+        cnt[threadIdx.x] = c;
     }
     __syncthreads();
 
-    // 3. Cholesky over the non-empty codewords, dc = -M^-1 t
-    if (tid == 0) {
+    // 2. Cholesky over the non-empty codewords (one warp, lane = row, right-looking), then
+    //    dc = -M^-1 t by forward and back substitution.
+    if (warp == 0) {
         int idx[M];
         int nn = 0;
+#pragma unroll
         for (int b = 0; b < M; ++b)
-            if (start[b + 1] > start[b])
+            if (cnt[b] > 0)
                 idx[nn++] = b;
+        const int myc = lane < nn ? idx[lane < M ? lane : 0] : 0;
+        double arow[M];
+#pragma unroll
+        for (int c = 0; c < M; ++c)
+            arow[c] = (lane < nn && c < nn) ? Mm[myc * M + idx[c]] : 0.0;
         bool singular = false;
-        for (int r = 0; r < nn && !singular; ++r) {
-            for (int c = 0; c <= r; ++c) {
-                double s = Mm[idx[r] * M + idx[c]];
-                for (int k = 0; k < c; ++k)
-                    s -= L[r * M + k] * L[c * M + k];
-                if (r == c) {
-                    if (!(s > 0.0)) {
-                        singular = true;
-                        break;
-                    }
-                    L[r * M + r] = sqrt(s);
+#pragma unroll
+        for (int k = 0; k < M; ++k) {
+            if (k < nn && !singular) {
+                const double piv = __shfl_sync(0xffffffffu, arow[k], k);
+                if (!(piv > 0.0)) {
+                    singular = true;
                 } else {
-                    L[r * M + c] = s / L[c * M + c];
+                    const double lkk = sqrt(piv);
+                    const double inv = 1.0 / lkk;
+                    const double lik = lane > k ? arow[k] * inv : (lane == k ? lkk : 0.0);
+                    arow[k] = lik;  // column k of the row now holds L[lane][k]
+#pragma unroll
+                    for (int jj = k + 1; jj < M; ++jj) {
+                        if (jj < nn) {
+                            const double ljk = __shfl_sync(0xffffffffu, lik, jj);
+                            if (lane >= jj)
+                                arow[jj] -= lik * ljk;
+                        }
+                    }
                 }
             }
         }
         float *c = C + j * M;
         float *dc = dC + j * M;
-        for (int b = 0; b < M; ++b)
-            dc[b] = 0.f;
         if (singular) {
-            status[j] |= LNQ_ROW_SINGULAR;
+            if (lane < M)
+                dc[lane] = 0.f;
+            if (lane == 0)
+                status[j] |= LNQ_ROW_SINGULAR;
         } else {
-            for (int r = 0; r < nn; ++r) {
-                double s = -tv[idx[r]];
-                for (int k = 0; k < r; ++k)
-                    s -= L[r * M + k] * y[k];
-                y[r] = s / L[r * M + r];
+            if (lane < nn) {
+#pragma unroll
+                for (int k = 0; k < M; ++k)
+                    Ls[lane][k] = (k <= lane) ? arow[k] : 0.0;
             }
-            for (int r = nn - 1; r >= 0; --r) {
-                double s = y[r];
-                for (int k = r + 1; k < nn; ++k)
-                    s -= L[k * M + r] * y[k];
-                y[r] = s / L[r * M + r];
+            __syncwarp();
+            // forward: L y = -t; lane r keeps its running sum
+            double s = lane < nn ? -tv[myc] : 0.0;
+            double y = 0.0;
+            for (int k = 0; k < nn; ++k) {
+                if (lane == k)
+                    y = s / Ls[k][k];
+                const double yk = __shfl_sync(0xffffffffu, y, k);
+                if (lane > k && lane < nn)
+                    s -= Ls[lane][k] * yk;
             }
-            for (int r = 0; r < nn; ++r) {
-                const float old = c[idx[r]];
-                const float nw = static_cast<float>(static_cast<double>(old) + y[r]);
-                c[idx[r]] = nw;
-                dc[idx[r]] = static_cast<float>(static_cast<double>(nw) - static_cast<double>(old));
+            // back: L^T x = y
+            s = y;
+            double x = 0.0;
+            for (int k = nn - 1; k >= 0; --k) {
+                if (lane == k)
+                    x = s / Ls[k][k];
+                const double xk = __shfl_sync(0xffffffffu, x, k);
+                if (lane < k)
+                    s -= Ls[k][lane] * xk;
+            }
+            if (lane < M)
+                dc[lane] = 0.f;
+            __syncwarp();
+            if (lane < nn) {
+                const float old = c[myc];
+                const float nw = static_cast<float>(static_cast<double>(old) + x);
+                c[myc] = nw;
+                dc[myc] = static_cast<float>(static_cast<double>(nw) - static_cast<double>(old));
             }
         }
     }
@@ -167,28 +226,31 @@ __global__ void __launch_bounds__(kSolveThreads)
 // ------------------------------------------------------------------------------------------
 // objective J = r^T (F r)
 // ------------------------------------------------------------------------------------------
+// One CTA per row: fp64 sum of r_i u_i over the row, each thread over a fixed stride of
+// coordinates, then a fixed-order tree, so the result does not depend on scheduling.
 template <int M>
-__global__ void __launch_bounds__(kObjWarps * 32)
-    objective_u_kernel(const float *__restrict__ uT, const float *__restrict__ W,
+__global__ void __launch_bounds__(kObjThreads)
+    objective_u_kernel(const float *__restrict__ U, const float *__restrict__ W,
                        const float *__restrict__ C, const uint8_t *__restrict__ Q,
-                       double *__restrict__ J, int64_t d, int64_t d_out)
+                       double *__restrict__ J, int64_t d)
 {
-    __shared__ double part[kObjWarps][32];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t j = static_cast<int64_t>(blockIdx.x) * 32 + lane;
+    __shared__ double part[kObjThreads / 32];
+    const int64_t j = blockIdx.x;
     double acc = 0.0;
-    if (j < d_out) {
-        for (int64_t i = warp; i < d; i += kObjWarps) {
-            const float r = C[j * M + (Q[j * d + i] & (M - 1))] - W[j * d + i];
-            acc += static_cast<double>(r) * static_cast<double>(uT[i * d_out + j]);
-        }
+    for (int64_t i = threadIdx.x; i < d; i += kObjThreads) {
+        const float r = C[j * M + (Q[j * d + i] & (M - 1))] - W[j * d + i];
+        acc += static_cast<double>(r) * static_cast<double>(U[j * d + i]);
     }
-    part[warp][lane] = acc;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        acc += __shfl_down_sync(0xffffffffu, acc, o);
+    if ((threadIdx.x & 31) == 0)
+        part[threadIdx.x >> 5] = acc;
     __syncthreads();
-    if (warp == 0 && j < d_out) {
+    if (threadIdx.x == 0) {
         double s = 0.0;
-        for (int w = 0; w < kObjWarps; ++w)
-            s += part[w][lane];
+        for (int w = 0; w < kObjThreads / 32; ++w)
+            s += part[w];
         J[j] = s;
     }
 }
@@ -197,44 +259,37 @@ __global__ void __launch_bounds__(kObjWarps * 32)
 // Host launchers
 // ------------------------------------------------------------------------------------------
 template <int M>
-static cudaError_t solve_m(const float *V, const float *uT, const uint8_t *Q, float *C, float *dC,
+static cudaError_t solve_m(const float *V, const float *U, const uint8_t *Q, float *C, float *dC,
                            int32_t *status, int64_t d, int64_t d_out, cudaStream_t s)
 {
-    const size_t smem = static_cast<size_t>(kSolveThreads) * M * 4 + static_cast<size_t>(d) * 4;
-    cudaError_t e = cudaFuncSetAttribute(solve_kernel<M>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
-    if (e != cudaSuccess)
-        return e;
     KernelTimer timer("lnq_solve", s);
-    solve_kernel<M><<<static_cast<unsigned>(d_out), kSolveThreads, smem, s>>>(V, uT, Q, C, dC,
-                                                                              status, d, d_out);
+    solve_kernel<M><<<static_cast<unsigned>(d_out), kSolveThreads, 0, s>>>(V, U, Q, C, dC, status, d);
     return cudaGetLastError();
 }
 
-cudaError_t lnq_solve(const float *V, const float *uT, const uint8_t *Q, float *C, float *dC,
+cudaError_t lnq_solve(const float *V, const float *U, const uint8_t *Q, float *C, float *dC,
                       int32_t *status, int64_t d, int64_t d_out, int m, cudaStream_t s)
 {
     switch (m) {
-    case 2: return solve_m<2>(V, uT, Q, C, dC, status, d, d_out, s);
-    case 4: return solve_m<4>(V, uT, Q, C, dC, status, d, d_out, s);
-    case 8: return solve_m<8>(V, uT, Q, C, dC, status, d, d_out, s);
-    case 16: return solve_m<16>(V, uT, Q, C, dC, status, d, d_out, s);
+    case 2: return solve_m<2>(V, U, Q, C, dC, status, d, d_out, s);
+    case 4: return solve_m<4>(V, U, Q, C, dC, status, d, d_out, s);
+    case 8: return solve_m<8>(V, U, Q, C, dC, status, d, d_out, s);
+    case 16: return solve_m<16>(V, U, Q, C, dC, status, d, d_out, s);
     }
     return cudaErrorInvalidValue;
 }
 
-cudaError_t lnq_objective_from_u(const float *uT, const float *W, const float *C,
+cudaError_t lnq_objective_from_u(const float *U, const float *W, const float *C,
                                  const uint8_t *Q, double *J, int64_t d, int64_t d_out, int m,
                                  cudaStream_t s)
 {
-    const unsigned blocks = static_cast<unsigned>((d_out + 31) / 32);
+    const unsigned blocks = static_cast<unsigned>(d_out);
     KernelTimer timer("lnq_objective", s);
     switch (m) {
-    case 2: objective_u_kernel<2><<<blocks, kObjWarps * 32, 0, s>>>(uT, W, C, Q, J, d, d_out); break;
-    case 4: objective_u_kernel<4><<<blocks, kObjWarps * 32, 0, s>>>(uT, W, C, Q, J, d, d_out); break;
-    case 8: objective_u_kernel<8><<<blocks, kObjWarps * 32, 0, s>>>(uT, W, C, Q, J, d, d_out); break;
-    case 16: objective_u_kernel<16><<<blocks, kObjWarps * 32, 0, s>>>(uT, W, C, Q, J, d, d_out); break;
+    case 2: objective_u_kernel<2><<<blocks, kObjThreads, 0, s>>>(U, W, C, Q, J, d); break;
+    case 4: objective_u_kernel<4><<<blocks, kObjThreads, 0, s>>>(U, W, C, Q, J, d); break;
+    case 8: objective_u_kernel<8><<<blocks, kObjThreads, 0, s>>>(U, W, C, Q, J, d); break;
+    case 16: objective_u_kernel<16><<<blocks, kObjThreads, 0, s>>>(U, W, C, Q, J, d); break;
     default: return cudaErrorInvalidValue;
     }
     return cudaGetLastError();

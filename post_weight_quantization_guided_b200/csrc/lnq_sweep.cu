@@ -71,7 +71,7 @@ struct SwParams {
     const float *F;      // [groups][d][d]
     const float *V;      // [d_out][d][m]
     const float *dC;     // [d_out][m]
-    const float *uT;     // [d][d_out]
+    const float *U;      // [d_out][d] u = F r for the previous codebook
     const float *C;      // [d_out][m]
     uint8_t *Q;          // [d_out][d]
     uint8_t *hist;       // [CTAs][2 * windows][3][4 KB]
@@ -326,7 +326,7 @@ __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
     } else if (warp < 6) {
         // ---------------------------------------------------------------- window assembly
         // Thread = coordinate kl of the window (= TMEM lane; warp w reads lanes 32 (w % 4)..).
-        // u of window T for the CTA's rows: uT (F r for the previous codebook) + V dc, plus the
+        // u of window T for the CTA's rows: U (F r for the previous codebook) + V dc, plus the
         // accumulator of the moves made before the window, written to the window buffer T & 1.
         const int quarter = warp & 3;
         const int kl = quarter * 32 + lane;
@@ -336,21 +336,10 @@ __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
             const int64_t k = static_cast<int64_t>(T) * WIN + kl;
             const bool kin = k < d;
             float u0[RB];
-            const float *ut = p.uT + k * p.d_out + row0;
-            if (kin && nrows == RB && (reinterpret_cast<uintptr_t>(ut) & 15u) == 0) {
+            // u of the CTA's rows at coordinate k (row-major u: a warp reads 128 contiguous bytes)
 #pragma unroll
-                for (int v = 0; v < RB / 4; ++v) {
-                    const float4 x = reinterpret_cast<const float4 *>(ut)[v];
-                    u0[4 * v] = x.x;
-                    u0[4 * v + 1] = x.y;
-                    u0[4 * v + 2] = x.z;
-                    u0[4 * v + 3] = x.w;
-                }
-            } else {
-#pragma unroll
-                for (int r = 0; r < RB; ++r)
-                    u0[r] = (kin && r < nrows) ? ut[r] : 0.f;
-            }
+            for (int r = 0; r < RB; ++r)
+                u0[r] = (kin && r < nrows) ? p.U[(row0 + r) * d + k] : 0.f;
             if (kin) {
 #pragma unroll
                 for (int r = 0; r < RB; ++r) {
@@ -650,7 +639,7 @@ static cudaError_t sweep_m(const CUtensorMap &map, const SwParams &p, unsigned g
 }
 
 cudaError_t lnq_sweep(const float *F, const __nv_bfloat16 *Fp, int groups, const float *V,
-                      const float *dC, const float *uT, const float *C, uint8_t *Q, uint8_t *hist,
+                      const float *dC, const float *U, const float *C, uint8_t *Q, uint8_t *hist,
                       int64_t d, int64_t d_out, int m, DeviceErr err, cudaStream_t s)
 {
     CUtensorMap map;
@@ -660,7 +649,7 @@ cudaError_t lnq_sweep(const float *F, const __nv_bfloat16 *Fp, int groups, const
     p.F = F;
     p.V = V;
     p.dC = dC;
-    p.uT = uT;
+    p.U = U;
     p.C = C;
     p.Q = Q;
     p.hist = hist;

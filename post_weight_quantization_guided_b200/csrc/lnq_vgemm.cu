@@ -19,8 +19,8 @@
 // the F tiles of its own 128 coordinates by TMA (K-major, 128-byte swizzle, no multicast) and
 // builds half of the right operand's columns in shared memory from Q, W and C, so that each SM
 // reads half of the right operand per MMA. The even CTA issues the MMAs; each CTA's TMEM holds
-// its 128 coordinates x all columns, and its epilogue writes V[j][i][b] and uT[i][j] (u
-// transposed, so the sweep reads a coordinate's rows contiguously). With m = 0 the kernel
+// its 128 coordinates x all columns, and its epilogue writes V[j][i][b] and U[j][i] (both
+// contiguous across a warp's coordinates). With m = 0 the kernel
 // computes u = F r only (42 rows per 128-column tile), which the objective uses.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -208,20 +208,19 @@ __global__ void __launch_bounds__(256)
     using S = VgShape<M>;
     const bool vec = (d & 7) == 0 && (reinterpret_cast<uintptr_t>(Q) & 7u) == 0 &&
                      (reinterpret_cast<uintptr_t>(W) & 15u) == 0;
-    const int64_t total = static_cast<int64_t>(num_rt_all) * nk * S::NCOLS * 8;  // 16-byte chunks
-    for (int64_t u = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; u < total;
-         u += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-        const int c = static_cast<int>(u & 7);
-        const int64_t rest = u >> 3;
-        const int n = static_cast<int>(rest % S::NCOLS);
-        const int64_t tb = rest / S::NCOLS;  // row tile * nk + K block
-        const int kb = static_cast<int>(tb % nk);
-        const int rt_all = static_cast<int>(tb / nk);
-        const int g = rt_all / row_tiles_per_group;
-        const int rt = rt_all - g * row_tiles_per_group;
-        const int64_t gstart = static_cast<int64_t>(g) * rows_per_group;
-        const int64_t row0 = gstart + static_cast<int64_t>(rt) * S::RT;
-        const int64_t row_end = min(row0 + S::RT, gstart + rows_per_group);
+    // one (row tile, K block) per CTA iteration: NCOLS x 8 chunks of 16 bytes
+    const int ntb = num_rt_all * nk;
+    for (int tb = blockIdx.x; tb < ntb; tb += gridDim.x) {
+      const int kb = tb % nk;
+      const int rt_all = tb / nk;
+      const int g = rt_all / row_tiles_per_group;
+      const int rt = rt_all - g * row_tiles_per_group;
+      const int64_t gstart = static_cast<int64_t>(g) * rows_per_group;
+      const int64_t row0 = gstart + static_cast<int64_t>(rt) * S::RT;
+      const int64_t row_end = min(row0 + S::RT, gstart + rows_per_group);
+      for (int v = threadIdx.x; v < S::NCOLS * 8; v += blockDim.x) {
+        const int c = v & 7;
+        const int n = v >> 3;
         const int64_t k0 = static_cast<int64_t>(kb) * 64 + 8 * c;
         uint32_t out[4] = {0u, 0u, 0u, 0u};
         if (n < S::USED) {
@@ -282,8 +281,9 @@ __global__ void __launch_bounds__(256)
                 }
             }
         }
-        *reinterpret_cast<uint4 *>(img + (tb * S::NCOLS + n) * 64 + 8 * c) =
+        *reinterpret_cast<uint4 *>(img + (static_cast<int64_t>(tb) * S::NCOLS + n) * 64 + 8 * c) =
             make_uint4(out[0], out[1], out[2], out[3]);
+      }
     }
 }
 
@@ -292,7 +292,7 @@ struct VgParams {
     const float *W;     // [d_out][d]
     const float *C;     // [d_out][m]
     float *V;           // [d_out][d][m] (m > 0)
-    float *uT;          // [d][d_out]
+    float *U;           // [d_out][d] u = F r per row
     const int32_t *fexp;  // [groups][d] row scales of the fp16 pieces of F (fp16 mode)
     const int32_t *rexp;  // [d_out] residual scales (fp16 mode)
     int64_t d, d_out, rows_per_group;
@@ -578,7 +578,7 @@ __global__ void __launch_bounds__(vg::NUM_THREADS, 1)
                 for (int r = 0; r < S::RT; ++r) {
                     const int64_t j = row0 + r;
                     if (j < row_end)
-                        p.uT[i * p.d_out + j] =
+                        p.U[j * p.d + i] =
                             S::F16 ? (uacc[r] * inv_si) * pow2f(-p.rexp[j]) : uacc[r];
                 }
             }
@@ -696,8 +696,7 @@ static cudaError_t launch_vgemm_m(const CUtensorMap &map, VgParams p, uint16_t *
     p.num_tiles = static_cast<int>(num_rt_all * p.i_pairs);
     {
         KernelTimer timer(S::F16 ? "lnq_operand_image" : "lnq_residual_image", s);
-        const int64_t chunks = img_rows * 8;
-        int64_t blocks = (chunks + 255) / 256;
+        int64_t blocks = num_rt_all * nk;
         if (blocks > static_cast<int64_t>(num_sms) * 16)
             blocks = static_cast<int64_t>(num_sms) * 16;
         operand_image_kernel<M><<<static_cast<unsigned>(blocks), 256, 0, s>>>(
@@ -762,11 +761,11 @@ static cudaError_t launch_vgemm_m(const CUtensorMap &map, VgParams p, uint16_t *
     return cudaGetLastError();
 }
 
-// m in {2,4,8,16}: V and uT for every row from the fp16 pieces (Fh, fexp) and the residual scales
-// rexp; residual_only: uT = F r from the exact bf16 pieces Fp.
+// m in {2,4,8,16}: V and U for every row from the fp16 pieces (Fh, fexp) and the residual scales
+// rexp; residual_only: U = F r from the exact bf16 pieces Fp.
 cudaError_t lnq_vgemm(const __nv_bfloat16 *Fp, const __half *Fh, const int32_t *fexp,
                       const int32_t *rexp, int groups, const uint8_t *Q, const float *W,
-                      const float *C, float *V, float *uT, uint16_t *img, int64_t d, int64_t d_out,
+                      const float *C, float *V, float *U, uint16_t *img, int64_t d, int64_t d_out,
                       int m, bool residual_only, DeviceErr err, int num_sms, cudaStream_t s)
 {
     CUtensorMap map;
@@ -780,7 +779,7 @@ cudaError_t lnq_vgemm(const __nv_bfloat16 *Fp, const __half *Fh, const int32_t *
     p.W = W;
     p.C = C;
     p.V = V;
-    p.uT = uT;
+    p.U = U;
     p.fexp = fexp;
     p.rexp = rexp;
     p.d = d;
