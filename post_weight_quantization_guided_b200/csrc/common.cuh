@@ -101,6 +101,22 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, long l
     return false;
 }
 
+// Like mbar_wait, sleeping about `ns` nanoseconds between tries: for waits that are expected to
+// be long, so that the waiting warp leaves its issue slots to the warps doing the work.
+__device__ __forceinline__ bool mbar_wait_sleep(uint64_t *bar, uint32_t parity, long long limit,
+                                                unsigned ns)
+{
+    if (mbar_try_wait(bar, parity))
+        return true;
+    const long long t0 = clock64();
+    while (clock64() - t0 < limit) {
+        __nanosleep(ns);
+        if (mbar_try_wait(bar, parity))
+            return true;
+    }
+    return false;
+}
+
 // Named barrier among `n` threads (id 1..15; id 0 is __syncthreads).
 __device__ __forceinline__ void named_bar_sync(int id, int n)
 {

@@ -18,11 +18,12 @@
 //     K-major layout the MMA reads, written and read back with byte-exact bulk copies.
 //   * The product for window T+1 over windows < T runs while window T is being decided; only the
 //     contribution of window T itself waits for its last decision.
-//   * Inside a window one warp (lane = row) decides a block of 32 coordinates, correcting the
-//     block's later coordinates in registers from the 32 x 32 diagonal tile of F; then four warps
-//     correct the window's later blocks in shared memory from a 32 x 128 strip of F.
+//   * Inside a window the four sweep warps decide a block of 32 coordinates (four threads per
+//     row, each evaluating a quarter of the codewords), correcting the block's later coordinates
+//     in registers from the 32 x 32 diagonal tile of F; then they correct the window's later
+//     blocks in shared memory from a 32 x 128 strip of F.
 // Warp roles: 0 TMA and bulk copies, 1 MMA issue, 2-5 window assembly (TMEM -> shared memory),
-// 6-9 the sweep (6 decides; 6-9 correct). Every wait is bounded; a wait that gives up sets the
+// 6-9 the sweep. Every wait is bounded; a wait that gives up sets the
 // workspace error flag and its role stops, and every role drains what it has in flight.
 #include "common.cuh"
 #include "lnq_internal.cuh"
@@ -62,7 +63,7 @@ constexpr int OFF_WM = OFF_QB + RB * (BLK + 4);
 constexpr int OFF_BAR = (OFF_WM + MAX_WIN + 7) / 8 * 8;
 constexpr int NBARS = 2 * NA + 2 * NH + 2 + 2 + 2 + 2 + 3;
 constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
-constexpr size_t SMEM = 1024 + OFF_MISC + 16;
+constexpr size_t SMEM = 1024 + OFF_MISC + 32;
 static_assert(SMEM <= 232448, "shared memory");
 static_assert(OFF_H % 1024 == 0 && OFF_BS % 1024 == 0, "swizzle atoms are 1024-byte aligned");
 }  // namespace sw
@@ -126,7 +127,7 @@ __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
     uint64_t *bs_free = bs_ready + 1;
     uint64_t *drain = bs_free + 1;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + OFF_MISC);
-    volatile unsigned *moved_s = reinterpret_cast<volatile unsigned *>(smem + OFF_MISC + 4);
+    volatile unsigned *moved_s = reinterpret_cast<volatile unsigned *>(smem + OFF_MISC + 16);  // [4]
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -156,7 +157,7 @@ __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
             mbar_init(&uw_ready[s], 128);
             mbar_init(&uw_free[s], SWEEP_THREADS);
         }
-        mbar_init(bs_ready, 32);
+        mbar_init(bs_ready, SWEEP_THREADS);
         mbar_init(bs_free, 2);
         mbar_init(drain, 1);
         fence_barrier_init();
@@ -189,7 +190,7 @@ __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
             bool ok = true;
             auto load_f = [&](int c, int T) -> bool {
                 for (int pc = 0; pc < 3; ++pc) {
-                    if (!mbar_wait(&a_empty[aslot], ((apar >> aslot) & 1u) ^ 1u, limit))
+                    if (!mbar_wait_sleep(&a_empty[aslot], ((apar >> aslot) & 1u) ^ 1u, limit, 64))
                         return false;
                     mbar_arrive_expect_tx(&a_full[aslot], A_TILE);
                     tma_load_3d(a_base + aslot * A_TILE, &fmap, &a_full[aslot], c * CH, T * WIN,
@@ -210,7 +211,7 @@ __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
                             bulk_wait_all();
                             confirmed = stored;
                         }
-                        if (!mbar_wait(&h_empty[hslot], ((hpar >> hslot) & 1u) ^ 1u, limit)) {
+                        if (!mbar_wait_sleep(&h_empty[hslot], ((hpar >> hslot) & 1u) ^ 1u, limit, 64)) {
                             ok = false;
                             break;
                         }
@@ -225,7 +226,7 @@ __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
                 }
                 for (int h = 0; h < 2 && ok; ++h)
                     ok = load_f(2 * (T - 1) + h, T);
-                if (ok && !mbar_wait(bs_ready, (T - 1) & 1, limit))
+                if (ok && !mbar_wait_sleep(bs_ready, (T - 1) & 1, limit, 64))
                     ok = false;
                 if (!ok) {
                     raise_error(p.err, kErrTimeout, 31);
@@ -261,7 +262,7 @@ __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
             bool ok = true;
             for (int T = 1; T < nwin && ok; ++T) {
                 const int acc = T & 1;
-                if (!mbar_wait(&acc_empty[acc], ((uses >> acc) & 1u) ^ 1u, limit)) {
+                if (!mbar_wait_sleep(&acc_empty[acc], ((uses >> acc) & 1u) ^ 1u, limit, 64)) {
                     raise_error(p.err, kErrTimeout, 32);
                     break;
                 }
@@ -270,7 +271,7 @@ __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
                 int n = 0;
                 auto chunk = [&](uint32_t b_addr, bool math) -> bool {
                     for (int pa = 0; pa < 3; ++pa) {
-                        if (!mbar_wait(&a_full[aslot], (aph >> aslot) & 1u, limit))
+                        if (!mbar_wait_sleep(&a_full[aslot], (aph >> aslot) & 1u, limit, 64))
                             return false;
                         aph ^= 1u << aslot;
                         tc_fence_after();
@@ -297,7 +298,7 @@ __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
                     if (!wmask[w])
                         continue;
                     for (int h = 0; h < 2 && ok; ++h) {
-                        if (!mbar_wait(&h_full[hslot], (hph >> hslot) & 1u, limit)) {
+                        if (!mbar_wait_sleep(&h_full[hslot], (hph >> hslot) & 1u, limit, 64)) {
                             ok = false;
                             break;
                         }
@@ -307,7 +308,7 @@ __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
                         hslot = (hslot + 1 == NH) ? 0 : hslot + 1;
                     }
                 }
-                if (ok && !mbar_wait(bs_ready, (T - 1) & 1, limit))
+                if (ok && !mbar_wait_sleep(bs_ready, (T - 1) & 1, limit, 64))
                     ok = false;
                 const bool mv = ok && wmask[T - 1] != 0;
                 for (int h = 0; h < 2 && ok; ++h)
@@ -368,8 +369,8 @@ __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
                 const int acc = T & 1;
                 int okw = 0;
                 if (lane == 0)
-                    okw = (mbar_wait(bs_ready, (T - 1) & 1, limit) &&
-                           mbar_wait(&acc_full[acc], (uses >> acc) & 1u, limit)) ? 1 : 0;
+                    okw = (mbar_wait_sleep(bs_ready, (T - 1) & 1, limit, 64) &&
+                           mbar_wait_sleep(&acc_full[acc], (uses >> acc) & 1u, limit, 64)) ? 1 : 0;
                 okw = __shfl_sync(0xffffffffu, okw, 0);
                 if (!okw) {
                     if (lane == 0)
@@ -395,7 +396,7 @@ __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
             const int buf = T & 1;
             int okw = 0;
             if (lane == 0)
-                okw = mbar_wait(&uw_free[buf], ((wuses >> buf) & 1u) ^ 1u, limit) ? 1 : 0;
+                okw = mbar_wait_sleep(&uw_free[buf], ((wuses >> buf) & 1u) ^ 1u, limit, 64) ? 1 : 0;
             okw = __shfl_sync(0xffffffffu, okw, 0);
             if (!okw) {
                 if (lane == 0)
@@ -413,15 +414,8 @@ __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
     } else {
         // ---------------------------------------------------------------- the sweep
         const int t = threadIdx.x - 6 * 32;  // 0..127
-        const bool decider = warp == 6;
-        const int64_t j = row0 + lane;
-        const bool valid = decider && lane < nrows;
         const float *Fg = p.F + static_cast<int64_t>(g) * d * d;
         const bool vecF = (d & 3) == 0 && (reinterpret_cast<uintptr_t>(p.F) & 15u) == 0;
-        float c_reg[M];
-#pragma unroll
-        for (int b = 0; b < M; ++b)
-            c_reg[b] = c_s[lane][b];
         // F rows b0..b0+31, columns wstart..wstart+127 of the group (zero outside F) -> strip buf
         auto load_strip = [&](int buf, int64_t b0, int64_t wstart) {
             float *st = strip + buf * (BLK * WIN);
@@ -475,48 +469,79 @@ __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
                         load_strip((bi + 1) & 1, nb0, lb + 1 < NBLK ? wstart : wstart + WIN);
                 }
                 const float *st = strip + (bi & 1) * (BLK * WIN) + lb * BLK;  // st[ii * WIN + c]
-                if (decider) {
-                    // codes of the block for this row
-                    if (valid && nb == BLK && (d & 3) == 0 &&
-                        (reinterpret_cast<uintptr_t>(p.Q) & 3u) == 0) {
-                        const uint32_t *qs = reinterpret_cast<const uint32_t *>(p.Q + j * d + b0);
+                {
+                    // Decisions: thread (row r = t / 4, sub s = t % 4). The row's four threads
+                    // hold the block's u redundantly, each evaluates a quarter of the codewords,
+                    // and the lexicographic minimum of (Delta, index) over the four is formed
+                    // with two shuffles: the lowest index wins among equal values, and a
+                    // coordinate moves only for a strictly negative Delta (staying is Delta 0).
+                    const int r = t >> 2, s = t & 3;
+                    const int64_t jr = row0 + r;
+                    const bool vr = r < nrows;
+                    // codes of the block (sub s loads 8 of them) and their codeword values
 #pragma unroll
-                        for (int v = 0; v < BLK / 4; ++v)
-                            *reinterpret_cast<uint32_t *>(&qb_s[lane][4 * v]) = qs[v];
-                    } else {
-                        for (int ii = 0; ii < BLK; ++ii)
-                            qb_s[lane][ii] = (valid && ii < nb) ? p.Q[j * d + b0 + ii] : 0;
+                    for (int e = 0; e < 8; ++e) {
+                        const int k = 8 * s + e;
+                        qb_s[r][k] = (vr && k < nb) ? (p.Q[jr * d + b0 + k] & (M - 1)) : 0;
                     }
                     __syncwarp();
-                    float ub[BLK], dl[BLK];
+                    constexpr int NPL = (M + 3) / 4;  // codewords per thread: a = s + 4 k
+                    float ca[NPL];
 #pragma unroll
-                    for (int ii = 0; ii < BLK; ++ii)
-                        ub[ii] = uw[lane * UW_LD + lb * BLK + ii];
-                    unsigned colmask = 0u;
+                    for (int k = 0; k < NPL; ++k)
+                        ca[k] = (s + 4 * k < M) ? c_s[r][s + 4 * k] : 0.f;
+                    // the block's u, current codeword values, codes (byte ii of qw) and moves stay
+                    // in registers for the whole walk: no shared-memory stores inside it, so the
+                    // loads of F can be issued ahead
+                    float ub[BLK], cur[BLK], dl[BLK];
+                    uint32_t qw[BLK / 4];
+#pragma unroll
+                    for (int v = 0; v < BLK / 4; ++v)
+                        qw[v] = *reinterpret_cast<const uint32_t *>(&qb_s[r][4 * v]);
+#pragma unroll
+                    for (int ii = 0; ii < BLK; ++ii) {
+                        ub[ii] = uw[r * UW_LD + lb * BLK + ii];
+                        cur[ii] = c_s[r][(qw[ii >> 2] >> (8 * (ii & 3))) & 0xFFu];
+                    }
+                    unsigned rowmask = 0u;
 #pragma unroll
                     for (int ii = 0; ii < BLK; ++ii) {
                         float dlt = 0.f;
-                        if (ii < nb && valid) {
-                            const int qi = qb_s[lane][ii] & (M - 1);
-                            const float cur = c_s[lane][qi];
+                        if (ii < nb) {
                             const float fii = st[ii * WIN + ii];
                             const float two_u = 2.f * ub[ii];
-                            // Delta_a = delta_a (2 u + delta_a F_ii); staying is Delta 0; the lowest
-                            // index wins among equal strictly negative values
-                            int best = qi;
-                            float bestD = 0.f;
+                            float Dm = __int_as_float(0x7f800000);  // +inf
+                            int am = M;
+                            float cm = 0.f;
 #pragma unroll
-                            for (int a = 0; a < M; ++a) {
-                                const float da = c_reg[a] - cur;
-                                const float D = da * fmaf(da, fii, two_u);
-                                if (D < bestD) {
-                                    bestD = D;
-                                    best = a;
+                            for (int k = 0; k < NPL; ++k) {
+                                if (s + 4 * k < M) {
+                                    const float da = ca[k] - cur[ii];
+                                    const float D = da * fmaf(da, fii, two_u);
+                                    if (D < Dm) {
+                                        Dm = D;
+                                        am = s + 4 * k;
+                                        cm = ca[k];
+                                    }
                                 }
                             }
-                            if (best != qi) {  // a strictly negative Delta implies c[best] != cur
-                                dlt = c_s[lane][best] - cur;
-                                qb_s[lane][ii] = static_cast<uint8_t>(best);
+#pragma unroll
+                            for (int o = 1; o <= 2; o <<= 1) {
+                                const float D2 = __shfl_xor_sync(0xffffffffu, Dm, o);
+                                const int a2 = __shfl_xor_sync(0xffffffffu, am, o);
+                                const float c2 = __shfl_xor_sync(0xffffffffu, cm, o);
+                                if (D2 < Dm || (D2 == Dm && a2 < am)) {
+                                    Dm = D2;
+                                    am = a2;
+                                    cm = c2;
+                                }
+                            }
+                            if (vr && Dm < 0.f) {  // a strictly negative Delta implies c[am] != cur
+                                dlt = cm - cur[ii];
+                                rowmask |= 1u << ii;
+                                const int sh = 8 * (ii & 3);
+                                qw[ii >> 2] = (qw[ii >> 2] & ~(0xFFu << sh)) |
+                                              (static_cast<uint32_t>(am) << sh);
                             }
                         }
 #pragma unroll
@@ -528,42 +553,53 @@ __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
                             if (4 * v + 3 > ii) ub[4 * v + 3] = fmaf(dlt, f4.w, ub[4 * v + 3]);
                         }
                         dl[ii] = dlt;
-                        dl_s[ii][lane] = dlt;
-                        colmask |= (__ballot_sync(0xffffffffu, dlt != 0.f) != 0u ? 1u : 0u) << ii;
                     }
+                    if (s == 0) {
+#pragma unroll
+                        for (int ii = 0; ii < BLK; ++ii)
+                            dl_s[ii][r] = dl[ii];
+#pragma unroll
+                        for (int v = 0; v < BLK / 4; ++v)
+                            *reinterpret_cast<uint32_t *>(&qb_s[r][4 * v]) = qw[v];
+                    }
+                    const unsigned wm = __reduce_or_sync(0xffffffffu, rowmask);
                     if (lane == 0)
-                        *moved_s = colmask;
-                    wmoved = wmoved || colmask != 0u;
-                    if (valid && colmask != 0u) {
-                        for (int ii = 0; ii < nb; ++ii)
-                            p.Q[j * d + b0 + ii] = qb_s[lane][ii];
+                        moved_s[warp - 6] = wm;
+                    __syncwarp();
+                    // new codes of the row (sub s writes 8 of them) and, for later windows, the
+                    // Delta pieces in the K-major, 128-byte-swizzled operand: row r, K = 32 (lb & 1)
+                    // + k within chunk lb >> 1, sub s writes the 16-byte chunk of k = 8 s .. 8 s + 7
+                    if (vr && rowmask != 0u) {
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            const int k = 8 * s + e;
+                            if (k < nb)
+                                p.Q[jr * d + b0 + k] = qb_s[r][k];
+                        }
                     }
                     if (keep) {
-                        // Delta pieces of this block into the K-major, 128-byte-swizzled operand:
-                        // row = lane, K = 32 (lb & 1) + ii within chunk lb >> 1
-                        uint8_t *bs = bs_base + (lb >> 1) * H_CHUNK + lane * 128;
+                        uint32_t pk[3][4];
 #pragma unroll
-                        for (int cc = 0; cc < BLK / 8; ++cc) {
-                            uint32_t pk[3][4];
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                float a0, a1, a2, b0p, b1p, b2p;
-                                split3_sw(dl[8 * cc + 2 * e], a0, a1, a2);
-                                split3_sw(dl[8 * cc + 2 * e + 1], b0p, b1p, b2p);
-                                pk[0][e] = bf16_pair(a0, b0p);
-                                pk[1][e] = bf16_pair(a1, b1p);
-                                pk[2][e] = bf16_pair(a2, b2p);
-                            }
-                            const int chunk16 = (4 * (lb & 1) + cc) ^ (lane & 7);
-#pragma unroll
-                            for (int pc = 0; pc < 3; ++pc)
-                                *reinterpret_cast<uint4 *>(bs + pc * H_PIECE + chunk16 * 16) =
-                                    make_uint4(pk[pc][0], pk[pc][1], pk[pc][2], pk[pc][3]);
+                        for (int e = 0; e < 4; ++e) {
+                            float a0, a1, a2, c0, c1, c2;
+                            split3_sw(dl_s[8 * s + 2 * e][r], a0, a1, a2);
+                            split3_sw(dl_s[8 * s + 2 * e + 1][r], c0, c1, c2);
+                            pk[0][e] = bf16_pair(a0, c0);
+                            pk[1][e] = bf16_pair(a1, c1);
+                            pk[2][e] = bf16_pair(a2, c2);
                         }
+                        uint8_t *bs = bs_base + (lb >> 1) * H_CHUNK + r * 128;
+                        const int chunk16 = (4 * (lb & 1) + s) ^ (r & 7);
+#pragma unroll
+                        for (int pc = 0; pc < 3; ++pc)
+                            *reinterpret_cast<uint4 *>(bs + pc * H_PIECE + chunk16 * 16) =
+                                make_uint4(pk[pc][0], pk[pc][1], pk[pc][2], pk[pc][3]);
                     }
                 }
                 named_bar_sync(SWEEP_BAR, SWEEP_THREADS);
-                const unsigned colmask = *moved_s;
+                const unsigned colmask = moved_s[0] | moved_s[1] | moved_s[2] | moved_s[3];
+                wmoved = wmoved || colmask != 0u;
+
                 const int kend = (d - wstart < WIN) ? static_cast<int>(d - wstart) : WIN;
                 if (colmask != 0u && (lb + 1) * BLK < kend) {
                     // u[r][k] += sum_ii Delta[ii][r] F[b0 + ii][wstart + k] for the window's
@@ -595,13 +631,11 @@ __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
                 }
                 named_bar_sync(SWEEP_BAR, SWEEP_THREADS);
             }
-            if (decider) {
-                if (lane == 0)
-                    wmask[T] = wmoved ? 1 : 0;
-                if (keep) {
-                    fence_proxy_async_smem();
-                    mbar_arrive(bs_ready);
-                }
+            if (t == 0)
+                wmask[T] = wmoved ? 1 : 0;
+            if (keep) {
+                fence_proxy_async_smem();
+                mbar_arrive(bs_ready);
             }
             mbar_arrive(&uw_free[buf]);
         }
