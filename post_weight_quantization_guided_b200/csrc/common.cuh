@@ -42,6 +42,26 @@ __device__ __forceinline__ void raise_error(const DeviceErr &e, uint32_t flag, u
 __host__ __device__ constexpr size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // ------------------------------------------------------------------------------------------
+// Exact power-of-two scaling and fp16 pieces
+// ------------------------------------------------------------------------------------------
+// 2^e as a float, exact for |e| <= 126; scale exponents are kept within +-100.
+__device__ __forceinline__ float pow2f(int e) { return __int_as_float((127 + e) << 23); }
+__device__ __forceinline__ int clamp_scale(int e) { return e < -100 ? -100 : (e > 100 ? 100 : e); }
+
+// The three fp16 pieces of x (|x| <= 2^15): x == p0 + p1 + p2 up to 2^-33 relative (2^-24
+// absolute, the fp16 subnormal step).
+__device__ __forceinline__ void split3_f16(float x, uint16_t &p0, uint16_t &p1, uint16_t &p2)
+{
+    const __half a = __float2half_rn(x);
+    const float r1 = x - __half2float(a);
+    const __half b = __float2half_rn(r1);
+    const __half c = __float2half_rn(r1 - __half2float(b));
+    p0 = __half_as_ushort(a);
+    p1 = __half_as_ushort(b);
+    p2 = __half_as_ushort(c);
+}
+
+// ------------------------------------------------------------------------------------------
 // Shared-memory addresses and mbarriers
 // ------------------------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t smem_u32(const void *p)

@@ -121,8 +121,8 @@ cudaError_t lnq_iterate_launch(const float *F, int groups, const float *W, int64
             return e;
         if ((e = lnq_solve(w.V, w.U, Q, C, w.dC, w.status, d, d_out, m, s)) != cudaSuccess)
             return e;
-        if ((e = lnq_sweep(F, w.Fp, groups, w.V, w.dC, w.U, C, Q, w.hist, d, d_out, m, err,
-                           s)) != cudaSuccess)
+        if ((e = lnq_sweep(F, w.Fh, w.fexp, groups, w.V, w.dC, w.U, C, Q, w.hist, d, d_out, m,
+                           err, s)) != cudaSuccess)
             return e;
     }
     if (J != nullptr) {

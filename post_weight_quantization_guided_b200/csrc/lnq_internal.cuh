@@ -37,6 +37,7 @@ cudaError_t lnq_iterate_launch(const float *F, int groups, const float *W, int64
 
 // lnq_vgemm.cu
 bool encode_f_pieces(CUtensorMap *map, const __nv_bfloat16 *Fp, int64_t d, int groups);
+bool encode_f16_pieces(CUtensorMap *map, const __half *Fh, int64_t d, int groups);
 cudaError_t lnq_split_f(const float *F, int64_t d, int groups, __nv_bfloat16 *Fp, cudaStream_t s);
 cudaError_t lnq_split_f16(const float *F, int64_t d, int groups, __half *Fh, int32_t *fexp,
                           cudaStream_t s);
@@ -57,8 +58,8 @@ cudaError_t lnq_objective_from_u(const float *U, const float *W, const float *C,
 
 // lnq_sweep.cu
 size_t lnq_sweep_history_bytes(int64_t d, int64_t d_out, int groups);
-cudaError_t lnq_sweep(const float *F, const __nv_bfloat16 *Fp, int groups, const float *V,
-                      const float *dC, const float *U, const float *C, uint8_t *Q, uint8_t *hist,
-                      int64_t d, int64_t d_out, int m, DeviceErr err, cudaStream_t s);
+cudaError_t lnq_sweep(const float *F, const __half *Fh, const int32_t *fexp, int groups,
+                      const float *V, const float *dC, const float *U, const float *C, uint8_t *Q,
+                      uint8_t *hist, int64_t d, int64_t d_out, int m, DeviceErr err, cudaStream_t s);
 
 }  // namespace lnq

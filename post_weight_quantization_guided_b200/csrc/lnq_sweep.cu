@@ -11,11 +11,12 @@
 //     sweep, u0 + V dc (u0 = F r for the previous codebook and V = F P from lnq_vgemm, dc the
 //     codebook change from lnq_solve), plus F[window][earlier coordinates] x Delta[earlier
 //     coordinates], Delta being the moves made so far in this sweep. That product runs on tcgen05
-//     tensor cores: F as its three exact bf16 pieces (the operand lnq_vgemm uses), Delta as three
-//     exact bf16 pieces per value, and the six piece products of weight >= 2^-16 accumulate in
-//     fp32 in TMEM; the three dropped ones are below 2^-25 of |F_ki delta_i|.
-//   * Delta of finished windows is kept per CTA in a global history, already in the swizzled
-//     K-major layout the MMA reads, written and read back with byte-exact bulk copies.
+//     tensor cores: F as its two fp16 pieces with a power-of-two scale per row (the operand of
+//     lnq_vgemm, 22 bits per entry), Delta as three fp16 pieces with a power-of-two scale per
+//     row of W (exact), five piece products accumulated in fp32 in TMEM (the dropped one is below
+//     2^-33 of |F_ki delta_i|); the scales are undone exactly when the window is assembled.
+//   * Delta of finished windows is kept per CTA in a global history (fp16 pieces), already in
+//     the swizzled K-major layout the MMA reads, written and read back with byte-exact copies.
 //   * The product for window T+1 over windows < T runs while window T is being decided; only the
 //     contribution of window T itself waits for its last decision.
 //   * Inside a window the four sweep warps decide a block of 32 coordinates (four threads per
@@ -37,8 +38,9 @@ constexpr int WIN = 128;                  // coordinates per window (MMA M)
 constexpr int BLK = 32;                   // coordinates per decision block
 constexpr int NBLK = WIN / BLK;
 constexpr int CH = 64;                    // coordinates per K chunk: one 128-byte bf16 swizzle row
-constexpr int A_TILE = WIN * CH * 2;      // one bf16 piece of F[window][chunk]: 16 KB
-constexpr int H_PIECE = RB * CH * 2;      // one bf16 piece of Delta[chunk][rows]: 4 KB
+constexpr int FPIECES = 2;                // fp16 pieces of F
+constexpr int A_TILE = WIN * CH * 2;      // one fp16 piece of F[window][chunk]: 16 KB
+constexpr int H_PIECE = RB * CH * 2;      // one fp16 piece of Delta[chunk][rows]: 4 KB
 constexpr int H_CHUNK = 3 * H_PIECE;      // 12 KB
 constexpr int NA = 6;                     // F piece slots
 constexpr int NH = 2;                     // history chunk slots
@@ -59,13 +61,15 @@ constexpr int OFF_DL = OFF_UW + 2 * RB * UW_LD * 4;
 constexpr int OFF_C = OFF_DL + BLK * RB * 4;
 constexpr int OFF_DC = OFF_C + RB * 17 * 4;
 constexpr int OFF_QB = OFF_DC + RB * 16 * 4;
-constexpr int OFF_WM = OFF_QB + RB * (BLK + 4);
-constexpr int OFF_BAR = (OFF_WM + MAX_WIN + 7) / 8 * 8;
+constexpr int OFF_WM = OFF_QB + RB * (BLK + 8);
+constexpr int OFF_TS = (OFF_WM + MAX_WIN + 15) / 16 * 16;  // [2][RB] Delta scales 2^t, 2^-t
+constexpr int OFF_BAR = OFF_TS + 2 * RB * 4;
 constexpr int NBARS = 2 * NA + 2 * NH + 2 + 2 + 2 + 2 + 3;
 constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
 constexpr size_t SMEM = 1024 + OFF_MISC + 32;
 static_assert(SMEM <= 232448, "shared memory");
 static_assert(OFF_H % 1024 == 0 && OFF_BS % 1024 == 0, "swizzle atoms are 1024-byte aligned");
+static_assert(OFF_QB % 8 == 0 && OFF_STRIP % 16 == 0, "vector accesses to the code and strip tiles");
 }  // namespace sw
 
 struct SwParams {
@@ -76,32 +80,18 @@ struct SwParams {
     const float *C;      // [d_out][m]
     uint8_t *Q;          // [d_out][d]
     uint8_t *hist;       // [CTAs][2 * windows][3][4 KB]
+    const int32_t *fexp; // [groups][d] row scales of the fp16 pieces of F
     int64_t d, d_out, rows_per_group;
     int blocks_per_group, nwin;
     DeviceErr err;
 };
-
-__device__ __forceinline__ uint32_t bf16_pair(float lo, float hi)
-{
-    return static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(lo))) |
-           (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(hi))) << 16);
-}
-
-// The three bf16 pieces of x: x == p0 + p1 + p2 exactly for normal fp32 x.
-__device__ __forceinline__ void split3_sw(float x, float &p0, float &p1, float &p2)
-{
-    p0 = __bfloat162float(__float2bfloat16_rn(x));
-    const float r1 = x - p0;
-    p1 = __bfloat162float(__float2bfloat16_rn(r1));
-    p2 = r1 - p1;
-}
 
 template <int M>
 __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
     sweep_kernel(const __grid_constant__ CUtensorMap fmap, SwParams p)
 {
     using namespace sw;
-    constexpr uint32_t IDESC = umma_idesc_f16kind(WIN, RB, false, false, /*f16=*/false);
+    constexpr uint32_t IDESC = umma_idesc_f16kind(WIN, RB, false, false, /*f16=*/true);
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(align_up(reinterpret_cast<uintptr_t>(smem_raw), 1024));
     uint8_t *a_base = smem + OFF_A;                                  // [NA][16 KB]
@@ -112,8 +102,10 @@ __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
     float(*dl_s)[RB] = reinterpret_cast<float(*)[RB]>(smem + OFF_DL);       // [BLK][RB]
     float(*c_s)[17] = reinterpret_cast<float(*)[17]>(smem + OFF_C);         // [RB][m]
     float(*dc_s)[16] = reinterpret_cast<float(*)[16]>(smem + OFF_DC);       // [RB][m]
-    uint8_t(*qb_s)[BLK + 4] = reinterpret_cast<uint8_t(*)[BLK + 4]>(smem + OFF_QB);
+    uint8_t(*qb_s)[BLK + 8] = reinterpret_cast<uint8_t(*)[BLK + 8]>(smem + OFF_QB);  // rows 8-byte aligned
     volatile uint8_t *wmask = smem + OFF_WM;                         // [window]: some row moved
+    float *dsc = reinterpret_cast<float *>(smem + OFF_TS);            // [RB] 2^t_r of Delta row r
+    float *dinv = dsc + RB;                                           // [RB] 2^-t_r
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
     uint64_t *a_full = bars;
     uint64_t *a_empty = a_full + NA;
@@ -169,6 +161,21 @@ __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
         c_s[r][b] = in ? p.C[(row0 + r) * M + b] : 0.f;
         dc_s[r][b] = in ? p.dC[(row0 + r) * M + b] : 0.f;
     }
+    if (threadIdx.x < RB) {
+        // every Delta of row r is a difference of two of its codewords: |Delta| <= max c - min c
+        const int r = threadIdx.x;
+        float lo = 0.f, hi = 0.f;
+        if (r < nrows) {
+            lo = hi = p.C[(row0 + r) * M];
+            for (int b = 1; b < M; ++b) {
+                lo = fminf(lo, p.C[(row0 + r) * M + b]);
+                hi = fmaxf(hi, p.C[(row0 + r) * M + b]);
+            }
+        }
+        const int tr = hi > lo ? clamp_scale(14 - ilogbf(hi - lo)) : 0;
+        dsc[r] = pow2f(tr);
+        dinv[r] = pow2f(-tr);
+    }
     if (warp == 1)
         tmem_alloc(tmem_holder, TMEM_COLS);
     tc_fence_before();
@@ -189,12 +196,12 @@ __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
             int stored = 0, confirmed = 0;  // history chunks written / known complete
             bool ok = true;
             auto load_f = [&](int c, int T) -> bool {
-                for (int pc = 0; pc < 3; ++pc) {
+                for (int pc = 0; pc < FPIECES; ++pc) {
                     if (!mbar_wait_sleep(&a_empty[aslot], ((apar >> aslot) & 1u) ^ 1u, limit, 64))
                         return false;
                     mbar_arrive_expect_tx(&a_full[aslot], A_TILE);
                     tma_load_3d(a_base + aslot * A_TILE, &fmap, &a_full[aslot], c * CH, T * WIN,
-                                g * 3 + pc);
+                                g * FPIECES + pc);
                     apar ^= 1u << aslot;
                     aused |= 1u << aslot;
                     aslot = (aslot + 1 == NA) ? 0 : aslot + 1;
@@ -255,7 +262,7 @@ __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
     } else if (warp == 1) {
         // ---------------------------------------------------------------- MMA issue
         // Accumulator T & 1 (32 TMEM columns, lane = coordinate of window T, column = row) gets
-        // sum over chunks c of F[T][c] x Delta[c], six piece products of four K=16 MMAs each.
+        // sum over chunks c of F[T][c] x Delta[c], five piece products of four K=16 MMAs each.
         if (lane == 0) {
             int aslot = 0, hslot = 0;
             uint32_t aph = 0u, hph = 0u, uses = 0u;  // bit per slot / accumulator: phase parity
@@ -270,14 +277,15 @@ __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * RB);
                 int n = 0;
                 auto chunk = [&](uint32_t b_addr, bool math) -> bool {
-                    for (int pa = 0; pa < 3; ++pa) {
+                    for (int pa = 0; pa < FPIECES; ++pa) {
                         if (!mbar_wait_sleep(&a_full[aslot], (aph >> aslot) & 1u, limit, 64))
                             return false;
                         aph ^= 1u << aslot;
                         tc_fence_after();
                         if (math) {
                             const uint32_t sa = smem_u32(a_base + aslot * A_TILE);
-                            for (int pb = 0; pa + pb < 3; ++pb) {
+                            // F piece pa times Delta piece pb, all but F2 x Delta3
+                            for (int pb = 0; pb < 3 - pa; ++pb) {
 #pragma unroll
                                 for (int kk = 0; kk < CH / 16; ++kk) {
                                     // K-major, 128-byte swizzle: 16 k = 32 bytes along the row
@@ -386,9 +394,11 @@ __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
                     tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                                            static_cast<uint32_t>(acc * RB),
                                        D);
+                    // the accumulator carries 2^fexp[k] 2^t_r
+                    const float inv_fk = pow2f(kin ? -p.fexp[static_cast<int64_t>(g) * d + k] : 0);
 #pragma unroll
                     for (int r = 0; r < RB; ++r)
-                        u0[r] += D[r];
+                        u0[r] += (D[r] * inv_fk) * dinv[r];
                 }
                 tc_fence_before();
                 mbar_arrive(&acc_empty[acc]);
@@ -439,7 +449,31 @@ __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
             }
         };
         uint32_t wuses = 0u;  // bit per window buffer: phase parity
-        int bi = 0;  // block counter: the strip of block bi sits in buffer bi & 1
+        int bi = 0;
+        // codes of this thread's row (r = t / 4) at coordinates k0 + 8 (t % 4) .. + 7, classes
+        // masked, 0 outside the problem
+        const bool qvec = (d & 7) == 0 && (reinterpret_cast<uintptr_t>(p.Q) & 7u) == 0;
+        auto fetch_codes = [&](int64_t k0) -> uint2 {
+            const int r = t >> 2, s = t & 3;
+            const int64_t k = k0 + 8 * s;
+            uint32_t w[2] = {0u, 0u};
+            if (r < nrows && k < d) {
+                const uint8_t *src = p.Q + (row0 + r) * d + k;
+                if (qvec && k + 8 <= d) {
+                    const uint2 v = *reinterpret_cast<const uint2 *>(src);
+                    w[0] = v.x;
+                    w[1] = v.y;
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        if (k + e < d)
+                            w[e >> 2] |= static_cast<uint32_t>(src[e]) << (8 * (e & 3));
+                }
+            }
+            constexpr uint32_t MASK4 = 0x01010101u * static_cast<uint32_t>(M - 1);
+            return make_uint2(w[0] & MASK4, w[1] & MASK4);
+        };
+        uint2 qpf = fetch_codes(0);  // block counter: the strip of block bi sits in buffer bi & 1
         load_strip(0, 0, 0);
         for (int T = 0; T < nwin; ++T) {
             const int64_t wstart = static_cast<int64_t>(T) * WIN;
@@ -478,12 +512,10 @@ __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
                     const int r = t >> 2, s = t & 3;
                     const int64_t jr = row0 + r;
                     const bool vr = r < nrows;
-                    // codes of the block (sub s loads 8 of them) and their codeword values
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const int k = 8 * s + e;
-                        qb_s[r][k] = (vr && k < nb) ? (p.Q[jr * d + b0 + k] & (M - 1)) : 0;
-                    }
+                    // codes of the block (sub s holds 8 of them, fetched during the previous block),
+                    // then the fetch of the next block's codes, hidden behind this block's walk
+                    *reinterpret_cast<uint2 *>(&qb_s[r][8 * s]) = qpf;
+                    qpf = fetch_codes(b0 + BLK);
                     __syncwarp();
                     constexpr int NPL = (M + 3) / 4;  // codewords per thread: a = s + 4 k
                     float ca[NPL];
@@ -570,23 +602,29 @@ __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
                     // Delta pieces in the K-major, 128-byte-swizzled operand: row r, K = 32 (lb & 1)
                     // + k within chunk lb >> 1, sub s writes the 16-byte chunk of k = 8 s .. 8 s + 7
                     if (vr && rowmask != 0u) {
+                        if (qvec && 8 * s + 8 <= nb) {
+                            *reinterpret_cast<uint2 *>(p.Q + jr * d + b0 + 8 * s) =
+                                *reinterpret_cast<const uint2 *>(&qb_s[r][8 * s]);
+                        } else {
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            const int k = 8 * s + e;
-                            if (k < nb)
-                                p.Q[jr * d + b0 + k] = qb_s[r][k];
+                            for (int e = 0; e < 8; ++e) {
+                                const int k = 8 * s + e;
+                                if (k < nb)
+                                    p.Q[jr * d + b0 + k] = qb_s[r][k];
+                            }
                         }
                     }
                     if (keep) {
                         uint32_t pk[3][4];
+                        const float sc = dsc[r];
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
-                            float a0, a1, a2, c0, c1, c2;
-                            split3_sw(dl_s[8 * s + 2 * e][r], a0, a1, a2);
-                            split3_sw(dl_s[8 * s + 2 * e + 1][r], c0, c1, c2);
-                            pk[0][e] = bf16_pair(a0, c0);
-                            pk[1][e] = bf16_pair(a1, c1);
-                            pk[2][e] = bf16_pair(a2, c2);
+                            uint16_t a0, a1, a2, c0, c1, c2;
+                            split3_f16(dl_s[8 * s + 2 * e][r] * sc, a0, a1, a2);
+                            split3_f16(dl_s[8 * s + 2 * e + 1][r] * sc, c0, c1, c2);
+                            pk[0][e] = static_cast<uint32_t>(a0) | (static_cast<uint32_t>(c0) << 16);
+                            pk[1][e] = static_cast<uint32_t>(a1) | (static_cast<uint32_t>(c1) << 16);
+                            pk[2][e] = static_cast<uint32_t>(a2) | (static_cast<uint32_t>(c2) << 16);
                         }
                         uint8_t *bs = bs_base + (lb >> 1) * H_CHUNK + r * 128;
                         const int chunk16 = (4 * (lb & 1) + s) ^ (r & 7);
@@ -672,12 +710,12 @@ static cudaError_t sweep_m(const CUtensorMap &map, const SwParams &p, unsigned g
     return cudaGetLastError();
 }
 
-cudaError_t lnq_sweep(const float *F, const __nv_bfloat16 *Fp, int groups, const float *V,
-                      const float *dC, const float *U, const float *C, uint8_t *Q, uint8_t *hist,
-                      int64_t d, int64_t d_out, int m, DeviceErr err, cudaStream_t s)
+cudaError_t lnq_sweep(const float *F, const __half *Fh, const int32_t *fexp, int groups,
+                      const float *V, const float *dC, const float *U, const float *C, uint8_t *Q,
+                      uint8_t *hist, int64_t d, int64_t d_out, int m, DeviceErr err, cudaStream_t s)
 {
     CUtensorMap map;
-    if (!encode_f_pieces(&map, Fp, d, groups))
+    if (!encode_f16_pieces(&map, Fh, d, groups))
         return cudaErrorInvalidValue;
     SwParams p{};
     p.F = F;
@@ -687,6 +725,7 @@ cudaError_t lnq_sweep(const float *F, const __nv_bfloat16 *Fp, int groups, const
     p.C = C;
     p.Q = Q;
     p.hist = hist;
+    p.fexp = fexp;
     p.d = d;
     p.d_out = d_out;
     p.rows_per_group = d_out / groups;

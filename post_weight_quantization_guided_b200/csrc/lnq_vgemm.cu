@@ -113,10 +113,6 @@ __global__ void split_f_kernel(const float *__restrict__ F, int64_t d, int group
     }
 }
 
-// 2^e as a float, exact for |e| <= 126; scale exponents are kept within +-100.
-__device__ __forceinline__ float pow2f(int e) { return __int_as_float((127 + e) << 23); }
-__device__ __forceinline__ int clamp_scale(int e) { return e < -100 ? -100 : (e > 100 ? 100 : e); }
-
 // F (fp32 [groups][d][d]) -> Fh (fp16 [groups][2][d][ld]) with a power-of-two scale per row:
 // F[i][k] 2^fexp[i] = H1 + H2 up to 2^-22 relative (2^-39 of the row's largest entry for entries
 // near the fp16 subnormal range), the row's largest entry scaled into [2^14, 2^15). One CTA per
@@ -179,18 +175,6 @@ __global__ void __launch_bounds__(256)
         rexp[j] = mx > 0.f ? clamp_scale(14 - ilogbf(mx)) : 0;
 }
 
-// The three fp16 pieces of x (|x| <= 2^15): x == p0 + p1 + p2 up to 2^-33 relative (2^-24
-// absolute, the fp16 subnormal step).
-__device__ __forceinline__ void split3_f16(float x, uint16_t &p0, uint16_t &p1, uint16_t &p2)
-{
-    const __half a = __float2half_rn(x);
-    const float r1 = x - __half2float(a);
-    const __half b = __float2half_rn(r1);
-    const __half c = __float2half_rn(r1 - __half2float(b));
-    p0 = __half_as_ushort(a);
-    p1 = __half_as_ushort(b);
-    p2 = __half_as_ushort(c);
-}
 
 // The right operand of every (row tile, K block), written once per call of the product and then
 // loaded by TMA like F: NCOLS rows (the product's columns) x 64 coordinates, row-major
@@ -652,6 +636,12 @@ static bool encode_pieces_map(CUtensorMap *map, const void *pieces, int64_t d, i
 bool encode_f_pieces(CUtensorMap *map, const __nv_bfloat16 *Fp, int64_t d, int groups)
 {
     return encode_pieces_map(map, Fp, d, groups * 3, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
+}
+
+// Tensor map over the fp16 pieces Fh [groups][2][d][ld].
+bool encode_f16_pieces(CUtensorMap *map, const __half *Fh, int64_t d, int groups)
+{
+    return encode_pieces_map(map, Fh, d, groups * 2, CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
 }
 
 // Right-operand image rows for m (M > 0 layout) or for the residual-only product: the workspace
