@@ -127,6 +127,27 @@ def test_lnq_every_codebook_size(orc, lnq, wl, m):
     lnq_follow_parity(orc, lnq, F, W, m, 3)
 
 
+@pytest.mark.parametrize("m,d_in,d_out,groups", [
+    (2, 300, 72, 2),     # three windows, ragged last one; 36 rows per group (a ragged row block)
+    (4, 517, 40, 1),     # odd d_in: unaligned rows, scalar paths, ragged K block
+    (8, 640, 48, 3),     # five full windows
+    (16, 1000, 34, 2),   # eight windows, 17 rows per group
+])
+def test_lnq_multi_window_shapes(orc, lnq, wl, m, d_in, d_out, groups):
+    # Several 128-coordinate windows, so the left-looking product over earlier moves (tensor
+    # cores, fp16 pieces, history copies) and the window hand-over all take part; every row is
+    # checked against the oracle in follow mode for two iterations.
+    layer = wl.scaled(wl.TINY, d_in=d_in, d_out=d_out, n=640, groups=groups, m=m)
+    X, G, W = wl.make_layer(layer, _dev())
+    # the Fisher build takes d_in % 8 == 0: build on X padded with zero columns and keep the
+    # leading d_in x d_in block, which is X^T diag(s) X of the real columns
+    pad = (-d_in) % 8
+    Xp = torch.cat([X, torch.zeros(X.shape[0], pad, dtype=X.dtype, device=X.device)], dim=1)
+    F = lnq.lnq_build_fisher(Xp, G, layer.groups)[:, :d_in, :d_in].contiguous()
+    summary, _, _ = lnq_follow_parity(orc, lnq, F, W, m, 2)
+    assert summary["moves"] > 0
+
+
 def test_lnq_empty_codewords_and_tiny_rows(orc, lnq, wl):
     # Rows with only 3 distinct values and m = 8 leave codewords empty; d_in = 5 is not a
     # multiple of anything.
