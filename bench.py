@@ -237,14 +237,37 @@ def cpu_baseline(layer, X, G, W, F_gpu, budget_s=20.0, threads=None):
 # ------------------------------------------------------------------------------------------
 # Main arm
 # ------------------------------------------------------------------------------------------
+# Multi-rank host logic (one layer per rank, weak scaling, no data-path collective)
+# ------------------------------------------------------------------------------------------
+def per_rank_layer(wl, rank):
+    """Rank r quantises its own q_proj-shaped layer: same shapes and distributions, seeds offset by
+    100 r, so the ranks' inputs differ."""
+    base = wl.Q_PROJ
+    return wl.scaled(base, seed=base.seed + 100 * rank, x_seed=base.x_seed + 100 * rank)
+
+
+def max_over_ranks(values, world, device):
+    """Element-wise maximum over the ranks of a list of timings (the job ends with its slowest
+    rank)."""
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return [float(x) for x in t]
+
+
+def job_throughput(world, rows_per_rank, ms_per_step):
+    """Whole-job rows per second: every rank quantises rows_per_rank rows per step."""
+    return world * rows_per_rank / (ms_per_step / 1e3)
+
+
+# ------------------------------------------------------------------------------------------
 def run_ours(args, rank, world, device):
     import post_weight_quantization_guided_b200 as lnq
     from post_weight_quantization_guided_b200 import binding as b
     from post_weight_quantization_guided_b200 import workloads as wl
 
     lnq.binding.lib()
-    layer = wl.scaled(wl.Q_PROJ, seed=wl.Q_PROJ.seed + 100 * rank,
-                      x_seed=wl.Q_PROJ.x_seed + 100 * rank)
+    layer = per_rank_layer(wl, rank)
     torch.cuda.set_device(device)
     X, G, W = wl.make_layer(layer, device)
     d, dout, m, it = layer.d_in, layer.d_out, layer.m, layer.iters
@@ -324,16 +347,13 @@ def run_ours(args, rank, world, device):
     e2e_ms = e0.elapsed_time(e1)
 
     # ---------------------------------------------------------------- max over ranks
-    t = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device=device)
-    if world > 1:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    total_ms, e2e_ms = float(t[0]), float(t[1])
+    total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], world, device)
 
     if rank != 0:
         return None
     ms_per_step = total_ms / args.steps
-    value = world * dout / (ms_per_step / 1e3)
-    e2e_value = world * dout * e2e_steps / (e2e_ms / 1e3)
+    value = job_throughput(world, dout, ms_per_step)
+    e2e_value = job_throughput(world, dout, e2e_ms / e2e_steps)
 
     peaks = load_peaks()
     num_sms = torch.cuda.get_device_properties(device).multi_processor_count
