@@ -12,9 +12,9 @@
 //     codebook change from lnq_solve), plus F[window][earlier coordinates] x Delta[earlier
 //     coordinates], Delta being the moves made so far in this sweep. That product runs on tcgen05
 //     tensor cores: F as its two fp16 pieces with a power-of-two scale per row (the operand of
-//     lnq_vgemm, 22 bits per entry), Delta as three fp16 pieces with a power-of-two scale per
-//     row of W (exact), five piece products accumulated in fp32 in TMEM (the dropped one is below
-//     2^-33 of |F_ki delta_i|); the scales are undone exactly when the window is assembled.
+//     lnq_vgemm, 22 bits per entry), Delta as two fp16 pieces with a power-of-two scale per
+//     row of W (22 bits), the four piece products accumulated in fp32 in TMEM; the scales are
+//     undone exactly when the window is assembled.
 //   * Delta of finished windows is kept per CTA in a global history (fp16 pieces), already in
 //     the swizzled K-major layout the MMA reads, written and read back with byte-exact copies.
 //   * The product for window T+1 over windows < T runs while window T is being decided; only the
@@ -41,9 +41,10 @@ constexpr int CH = 64;                    // coordinates per K chunk: one 128-by
 constexpr int FPIECES = 2;                // fp16 pieces of F
 constexpr int A_TILE = WIN * CH * 2;      // one fp16 piece of F[window][chunk]: 16 KB
 constexpr int H_PIECE = RB * CH * 2;      // one fp16 piece of Delta[chunk][rows]: 4 KB
-constexpr int H_CHUNK = 3 * H_PIECE;      // 12 KB
+constexpr int DPIECES = 2;                // fp16 pieces of Delta
+constexpr int H_CHUNK = DPIECES * H_PIECE;  // 8 KB
 constexpr int NA = 6;                     // F piece slots
-constexpr int NH = 2;                     // history chunk slots
+constexpr int NH = 3;                     // history chunk slots
 constexpr int UW_LD = WIN + 1;            // row stride (floats) of a window's u in shared memory
 constexpr int NUM_THREADS = 320;
 constexpr int SWEEP_THREADS = 128;
@@ -79,7 +80,7 @@ struct SwParams {
     const float *U;      // [d_out][d] u = F r for the previous codebook
     const float *C;      // [d_out][m]
     uint8_t *Q;          // [d_out][d]
-    uint8_t *hist;       // [CTAs][2 * windows][3][4 KB]
+    uint8_t *hist;       // [CTAs][2 * windows][2][4 KB]
     const int32_t *fexp; // [groups][d] row scales of the fp16 pieces of F
     int64_t d, d_out, rows_per_group;
     int blocks_per_group, nwin;
@@ -96,7 +97,7 @@ __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
     uint8_t *smem = reinterpret_cast<uint8_t *>(align_up(reinterpret_cast<uintptr_t>(smem_raw), 1024));
     uint8_t *a_base = smem + OFF_A;                                  // [NA][16 KB]
     uint8_t *h_base = smem + OFF_H;                                  // [NH][12 KB]
-    uint8_t *bs_base = smem + OFF_BS;                                // [2 chunks][3][4 KB]
+    uint8_t *bs_base = smem + OFF_BS;                                // [2 chunks][2][4 KB]
     float *strip = reinterpret_cast<float *>(smem + OFF_STRIP);      // [2][BLK][WIN]
     float *uwb = reinterpret_cast<float *>(smem + OFF_UW);           // [2][RB][UW_LD]
     float(*dl_s)[RB] = reinterpret_cast<float(*)[RB]>(smem + OFF_DL);       // [BLK][RB]
@@ -262,7 +263,7 @@ __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
     } else if (warp == 1) {
         // ---------------------------------------------------------------- MMA issue
         // Accumulator T & 1 (32 TMEM columns, lane = coordinate of window T, column = row) gets
-        // sum over chunks c of F[T][c] x Delta[c], five piece products of four K=16 MMAs each.
+        // sum over chunks c of F[T][c] x Delta[c], four piece products of four K=16 MMAs each.
         if (lane == 0) {
             int aslot = 0, hslot = 0;
             uint32_t aph = 0u, hph = 0u, uses = 0u;  // bit per slot / accumulator: phase parity
@@ -284,8 +285,8 @@ __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
                         tc_fence_after();
                         if (math) {
                             const uint32_t sa = smem_u32(a_base + aslot * A_TILE);
-                            // F piece pa times Delta piece pb, all but F2 x Delta3
-                            for (int pb = 0; pb < 3 - pa; ++pb) {
+                            // every F piece times every Delta piece
+                            for (int pb = 0; pb < DPIECES; ++pb) {
 #pragma unroll
                                 for (int kk = 0; kk < CH / 16; ++kk) {
                                     // K-major, 128-byte swizzle: 16 k = 32 bytes along the row
@@ -615,21 +616,24 @@ __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
                         }
                     }
                     if (keep) {
-                        uint32_t pk[3][4];
+                        uint32_t pk[DPIECES][4];
                         const float sc = dsc[r];
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
-                            uint16_t a0, a1, a2, c0, c1, c2;
-                            split3_f16(dl_s[8 * s + 2 * e][r] * sc, a0, a1, a2);
-                            split3_f16(dl_s[8 * s + 2 * e + 1][r] * sc, c0, c1, c2);
-                            pk[0][e] = static_cast<uint32_t>(a0) | (static_cast<uint32_t>(c0) << 16);
-                            pk[1][e] = static_cast<uint32_t>(a1) | (static_cast<uint32_t>(c1) << 16);
-                            pk[2][e] = static_cast<uint32_t>(a2) | (static_cast<uint32_t>(c2) << 16);
+                            const float x0 = dl_s[8 * s + 2 * e][r] * sc;
+                            const float x1 = dl_s[8 * s + 2 * e + 1][r] * sc;
+                            const __half a0 = __float2half_rn(x0), c0 = __float2half_rn(x1);
+                            const __half a1 = __float2half_rn(x0 - __half2float(a0));
+                            const __half c1 = __float2half_rn(x1 - __half2float(c0));
+                            pk[0][e] = static_cast<uint32_t>(__half_as_ushort(a0)) |
+                                       (static_cast<uint32_t>(__half_as_ushort(c0)) << 16);
+                            pk[1][e] = static_cast<uint32_t>(__half_as_ushort(a1)) |
+                                       (static_cast<uint32_t>(__half_as_ushort(c1)) << 16);
                         }
                         uint8_t *bs = bs_base + (lb >> 1) * H_CHUNK + r * 128;
                         const int chunk16 = (4 * (lb & 1) + s) ^ (r & 7);
 #pragma unroll
-                        for (int pc = 0; pc < 3; ++pc)
+                        for (int pc = 0; pc < DPIECES; ++pc)
                             *reinterpret_cast<uint4 *>(bs + pc * H_PIECE + chunk16 * 16) =
                                 make_uint4(pk[pc][0], pk[pc][1], pk[pc][2], pk[pc][3]);
                     }
