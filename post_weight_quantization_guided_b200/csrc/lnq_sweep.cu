@@ -19,10 +19,12 @@
 //     the swizzled K-major layout the MMA reads, written and read back with byte-exact copies.
 //   * The product for window T+1 over windows < T runs while window T is being decided; only the
 //     contribution of window T itself waits for its last decision.
-//   * Inside a window the four sweep warps decide a block of 32 coordinates (four threads per
-//     row, each evaluating a quarter of the codewords), correcting the block's later coordinates
-//     in registers from the 32 x 32 diagonal tile of F; then they correct the window's later
-//     blocks in shared memory from a 32 x 128 strip of F.
+//   * Inside a window one warp (lane = row) decides a block of 32 coordinates: the best codeword
+//     for a coordinate is the one nearest to t = w^_i - u_i / F_ii, found among the midpoints of
+//     the row's sorted codebook, and the coordinate moves only if its exact change is strictly
+//     negative; the block's later coordinates are corrected in registers from the 32 x 32 diagonal
+//     tile of F. Then the four sweep warps write the codes and moves and correct the window's
+//     later blocks in shared memory from a 32 x 128 strip of F.
 // Warp roles: 0 TMA and bulk copies, 1 MMA issue, 2-5 window assembly (TMEM -> shared memory),
 // 6-9 the sweep. Every wait is bounded; a wait that gives up sets the
 // workspace error flag and its role stops, and every role drains what it has in flight.
@@ -64,7 +66,12 @@ constexpr int OFF_DC = OFF_C + RB * 17 * 4;
 constexpr int OFF_QB = OFF_DC + RB * 16 * 4;
 constexpr int OFF_WM = OFF_QB + RB * (BLK + 8);
 constexpr int OFF_TS = (OFF_WM + MAX_WIN + 15) / 16 * 16;  // [2][RB] Delta scales 2^t, 2^-t
-constexpr int OFF_BAR = OFF_TS + 2 * RB * 4;
+constexpr int OFF_SRT = OFF_TS + 2 * RB * 4;               // [RB][17] sorted codebook
+constexpr int OFF_ORD = OFF_SRT + RB * 17 * 4;             // [RB][16] its codeword indices
+constexpr int OFF_FINV = OFF_ORD + RB * 16;                // [BLK] 1 / F_ii of the block
+constexpr int OFF_FDG = OFF_FINV + BLK * 4;                // [BLK] F_ii of the block
+constexpr int OFF_RM = OFF_FDG + BLK * 4;                  // [RB] moved-coordinate mask per row
+constexpr int OFF_BAR = OFF_RM + RB * 4;
 constexpr int NBARS = 2 * NA + 2 * NH + 2 + 2 + 2 + 2 + 3;
 constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
 constexpr size_t SMEM = 1024 + OFF_MISC + 32;
@@ -107,6 +114,11 @@ __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
     volatile uint8_t *wmask = smem + OFF_WM;                         // [window]: some row moved
     float *dsc = reinterpret_cast<float *>(smem + OFF_TS);            // [RB] 2^t_r of Delta row r
     float *dinv = dsc + RB;                                           // [RB] 2^-t_r
+    float(*srt_s)[17] = reinterpret_cast<float(*)[17]>(smem + OFF_SRT);
+    uint8_t(*ord_s)[16] = reinterpret_cast<uint8_t(*)[16]>(smem + OFF_ORD);
+    float *finv_s = reinterpret_cast<float *>(smem + OFF_FINV);
+    float *fdg_s = reinterpret_cast<float *>(smem + OFF_FDG);
+    unsigned *rm_s = reinterpret_cast<unsigned *>(smem + OFF_RM);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
     uint64_t *a_full = bars;
     uint64_t *a_empty = a_full + NA;
@@ -474,7 +486,27 @@ __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
             constexpr uint32_t MASK4 = 0x01010101u * static_cast<uint32_t>(M - 1);
             return make_uint2(w[0] & MASK4, w[1] & MASK4);
         };
-        uint2 qpf = fetch_codes(0);  // block counter: the strip of block bi sits in buffer bi & 1
+        uint2 qpf = fetch_codes(0);
+        // warp 6 (lane = row): the row's codebook sorted, equal values in index order, and the
+        // midpoints between neighbours, for the decisions of the whole sweep
+        float mid[M > 1 ? M - 1 : 1];
+        if (warp == 6) {
+            const int r = lane;
+            for (int a = 0; a < M; ++a) {
+                const float ca = c_s[r][a];
+                int rank = 0;
+                for (int b = 0; b < M; ++b) {
+                    const float cb = c_s[r][b];
+                    rank += (cb < ca || (cb == ca && b < a)) ? 1 : 0;
+                }
+                srt_s[r][rank] = ca;
+                ord_s[r][rank] = static_cast<uint8_t>(a);
+            }
+            __syncwarp();
+#pragma unroll
+            for (int k = 0; k + 1 < M; ++k)
+                mid[k] = 0.5f * (srt_s[r][k] + srt_s[r][k + 1]);
+        }
         load_strip(0, 0, 0);
         for (int T = 0; T < nwin; ++T) {
             const int64_t wstart = static_cast<int64_t>(T) * WIN;
@@ -505,78 +537,66 @@ __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
                 }
                 const float *st = strip + (bi & 1) * (BLK * WIN) + lb * BLK;  // st[ii * WIN + c]
                 {
-                    // Decisions: thread (row r = t / 4, sub s = t % 4). The row's four threads
-                    // hold the block's u redundantly, each evaluates a quarter of the codewords,
-                    // and the lexicographic minimum of (Delta, index) over the four is formed
-                    // with two shuffles: the lowest index wins among equal values, and a
-                    // coordinate moves only for a strictly negative Delta (staying is Delta 0).
+                    // codes of the block (thread (r = t / 4, s = t % 4) holds 8 of them, fetched
+                    // during the previous block), then the fetch of the next block's codes
                     const int r = t >> 2, s = t & 3;
-                    const int64_t jr = row0 + r;
-                    const bool vr = r < nrows;
-                    // codes of the block (sub s holds 8 of them, fetched during the previous block),
-                    // then the fetch of the next block's codes, hidden behind this block's walk
                     *reinterpret_cast<uint2 *>(&qb_s[r][8 * s]) = qpf;
                     qpf = fetch_codes(b0 + BLK);
-                    __syncwarp();
-                    constexpr int NPL = (M + 3) / 4;  // codewords per thread: a = s + 4 k
-                    float ca[NPL];
-#pragma unroll
-                    for (int k = 0; k < NPL; ++k)
-                        ca[k] = (s + 4 * k < M) ? c_s[r][s + 4 * k] : 0.f;
-                    // the block's u, current codeword values, codes (byte ii of qw) and moves stay
-                    // in registers for the whole walk: no shared-memory stores inside it, so the
-                    // loads of F can be issued ahead
-                    float ub[BLK], cur[BLK], dl[BLK];
+                }
+                if (t < BLK) {
+                    const float f = st[t * WIN + t];
+                    fdg_s[t] = f;
+                    finv_s[t] = f > 0.f ? __frcp_rn(f) : __int_as_float(0x7f800000);  // 1/0 -> +inf
+                }
+                named_bar_sync(SWEEP_BAR, SWEEP_THREADS);
+                if (warp == 6) {
+                    // Decisions (lane = row). With F_ii > 0, candidate a changes the objective by
+                    // F_ii ((c_a - t)^2 - (cur - t)^2), t = cur - u_i / F_ii, so the best candidate
+                    // is the codeword nearest to t: the number of midpoints of the sorted codebook
+                    // below t gives it. Its change delta (2 u_i + delta F_ii) is then evaluated
+                    // and the coordinate moves only if that is strictly negative. (F_ii = 0 gives
+                    // t = -+inf, the extreme codeword, which is the best one for a linear change.)
+                    const int r = lane;
+                    const bool vr = r < nrows;
+                    // registers hold the block's u and codes only (fewer live values, no spills on
+                    // the chain); each coordinate's current value is read and its move written in
+                    // shared memory
+                    float ub[BLK];
                     uint32_t qw[BLK / 4];
 #pragma unroll
                     for (int v = 0; v < BLK / 4; ++v)
                         qw[v] = *reinterpret_cast<const uint32_t *>(&qb_s[r][4 * v]);
 #pragma unroll
-                    for (int ii = 0; ii < BLK; ++ii) {
+                    for (int ii = 0; ii < BLK; ++ii)
                         ub[ii] = uw[r * UW_LD + lb * BLK + ii];
-                        cur[ii] = c_s[r][(qw[ii >> 2] >> (8 * (ii & 3))) & 0xFFu];
-                    }
                     unsigned rowmask = 0u;
 #pragma unroll
                     for (int ii = 0; ii < BLK; ++ii) {
-                        float dlt = 0.f;
-                        if (ii < nb) {
-                            const float fii = st[ii * WIN + ii];
-                            const float two_u = 2.f * ub[ii];
-                            float Dm = __int_as_float(0x7f800000);  // +inf
-                            int am = M;
-                            float cm = 0.f;
+                        const float u = ub[ii];
+                        const float cur = c_s[r][(qw[ii >> 2] >> (8 * (ii & 3))) & 0xFFu];
+                        const float tt = fmaf(-u, finv_s[ii], cur);
+                        // number of midpoints below t, summed as a balanced tree
+                        int cnt[M];
 #pragma unroll
-                            for (int k = 0; k < NPL; ++k) {
-                                if (s + 4 * k < M) {
-                                    const float da = ca[k] - cur[ii];
-                                    const float D = da * fmaf(da, fii, two_u);
-                                    if (D < Dm) {
-                                        Dm = D;
-                                        am = s + 4 * k;
-                                        cm = ca[k];
-                                    }
-                                }
-                            }
+                        for (int k = 0; k < M; ++k)
+                            cnt[k] = (k + 1 < M && tt > mid[k < M - 1 ? k : 0]) ? 1 : 0;
 #pragma unroll
-                            for (int o = 1; o <= 2; o <<= 1) {
-                                const float D2 = __shfl_xor_sync(0xffffffffu, Dm, o);
-                                const int a2 = __shfl_xor_sync(0xffffffffu, am, o);
-                                const float c2 = __shfl_xor_sync(0xffffffffu, cm, o);
-                                if (D2 < Dm || (D2 == Dm && a2 < am)) {
-                                    Dm = D2;
-                                    am = a2;
-                                    cm = c2;
-                                }
-                            }
-                            if (vr && Dm < 0.f) {  // a strictly negative Delta implies c[am] != cur
-                                dlt = cm - cur[ii];
-                                rowmask |= 1u << ii;
-                                const int sh = 8 * (ii & 3);
-                                qw[ii >> 2] = (qw[ii >> 2] & ~(0xFFu << sh)) |
-                                              (static_cast<uint32_t>(am) << sh);
-                            }
+                        for (int w2 = 1; w2 < M; w2 *= 2) {
+#pragma unroll
+                            for (int k = 0; k + w2 < M; k += 2 * w2)
+                                cnt[k] += cnt[k + w2];
                         }
+                        const int pos = cnt[0];
+                        const float da = srt_s[r][pos] - cur;
+                        const float D = da * fmaf(da, fdg_s[ii], 2.f * u);
+                        // a strictly negative change implies c != cur
+                        const bool mv = vr && ii < nb && D < 0.f;
+                        const float dlt = mv ? da : 0.f;
+                        rowmask |= (mv ? 1u : 0u) << ii;
+                        const int sh = 8 * (ii & 3);
+                        const uint32_t nq = (qw[ii >> 2] & ~(0xFFu << sh)) |
+                                            (static_cast<uint32_t>(ord_s[r][pos]) << sh);
+                        qw[ii >> 2] = mv ? nq : qw[ii >> 2];
 #pragma unroll
                         for (int v = (ii + 1) / 4; v < BLK / 4; ++v) {
                             const float4 f4 = *reinterpret_cast<const float4 *>(st + ii * WIN + 4 * v);
@@ -585,24 +605,24 @@ __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
                             if (4 * v + 2 > ii) ub[4 * v + 2] = fmaf(dlt, f4.z, ub[4 * v + 2]);
                             if (4 * v + 3 > ii) ub[4 * v + 3] = fmaf(dlt, f4.w, ub[4 * v + 3]);
                         }
-                        dl[ii] = dlt;
+                        dl_s[ii][r] = dlt;
                     }
-                    if (s == 0) {
 #pragma unroll
-                        for (int ii = 0; ii < BLK; ++ii)
-                            dl_s[ii][r] = dl[ii];
-#pragma unroll
-                        for (int v = 0; v < BLK / 4; ++v)
-                            *reinterpret_cast<uint32_t *>(&qb_s[r][4 * v]) = qw[v];
-                    }
+                    for (int v = 0; v < BLK / 4; ++v)
+                        *reinterpret_cast<uint32_t *>(&qb_s[r][4 * v]) = qw[v];
+                    rm_s[r] = rowmask;
                     const unsigned wm = __reduce_or_sync(0xffffffffu, rowmask);
                     if (lane == 0)
-                        moved_s[warp - 6] = wm;
-                    __syncwarp();
-                    // new codes of the row (sub s writes 8 of them) and, for later windows, the
+                        moved_s[0] = wm;
+                }
+                named_bar_sync(SWEEP_BAR, SWEEP_THREADS);
+                {
+                    // thread (r, s): the row's new codes (8 of them) and, for later windows, the
                     // Delta pieces in the K-major, 128-byte-swizzled operand: row r, K = 32 (lb & 1)
                     // + k within chunk lb >> 1, sub s writes the 16-byte chunk of k = 8 s .. 8 s + 7
-                    if (vr && rowmask != 0u) {
+                    const int r = t >> 2, s = t & 3;
+                    const int64_t jr = row0 + r;
+                    if (r < nrows && rm_s[r] != 0u) {
                         if (qvec && 8 * s + 8 <= nb) {
                             *reinterpret_cast<uint2 *>(p.Q + jr * d + b0 + 8 * s) =
                                 *reinterpret_cast<const uint2 *>(&qb_s[r][8 * s]);
@@ -638,8 +658,8 @@ __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
                                 make_uint4(pk[pc][0], pk[pc][1], pk[pc][2], pk[pc][3]);
                     }
                 }
-                named_bar_sync(SWEEP_BAR, SWEEP_THREADS);
-                const unsigned colmask = moved_s[0] | moved_s[1] | moved_s[2] | moved_s[3];
+                const unsigned colmask = moved_s[0];
+
                 wmoved = wmoved || colmask != 0u;
 
                 const int kend = (d - wstart < WIN) ? static_cast<int>(d - wstart) : WIN;
