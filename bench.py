@@ -126,13 +126,11 @@ def algorithmic_work(layer, kernel: str, launches: int, moves_per_sweep: float):
     if kernel == "lnq_init":
         return 4.0 * dout * d + dout * d + 4.0 * dout * m, "byte"  # read W, write Q and C
     ld = (d + 7) // 8 * 8
-    if kernel == "lnq_split_f":
-        return 4.0 * g * d * d + 6.0 * g * d * ld, "byte"           # read F, write 3 bf16 pieces
     if kernel in ("lnq_operand_image", "lnq_residual_image"):
         # write the right-operand image (N columns x d coordinates x 2 bytes per row tile), read Q
         # and W once
-        rt = max(1, 256 // (m + 3)) if kernel == "lnq_operand_image" else 128 // 3
-        ncols = 256 if kernel == "lnq_operand_image" else 128
+        rt = max(1, 256 // (m + 3)) if kernel == "lnq_operand_image" else 256 // 3
+        ncols = 256
         tiles = g * -(-(dout // g) // rt)
         return tiles * ncols * (-(-d // 64) * 64) * 2.0 + 5.0 * dout * d, "byte"
     if kernel == "lnq_split_f16":
@@ -155,23 +153,23 @@ def algorithmic_work(layer, kernel: str, launches: int, moves_per_sweep: float):
     return 0.0, "unknown"
 
 
-# tcgen05 work per unit of algorithmic work. The V/u product takes F as two fp16 pieces against
-# m exact one-hot columns and three residual-piece columns per row; the objective's residual
-# product takes F as three exact bf16 pieces against three residual pieces (nine products).
+# tcgen05 work per unit of algorithmic work. Both products take F as two fp16 pieces: the V/u
+# product against m exact one-hot columns and three residual-piece columns per row, the
+# objective's residual product against the three residual-piece columns alone (six products).
 def hw_flop_factor(layer, kernel):
     m = layer.m
     if kernel == "lnq_vgemm":
         return (2.0 * m + 6.0) / (m + 1)
     if kernel == "lnq_residual_gemm":
-        return 9.0
+        return 6.0
     return None
 
 
 # DRAM bytes per launch of the dominant kernel from an ncu capture (profiles/
 # dram_traffic_lnq_q_proj_rows1024.md: 1024 rows, scaled by 4 to the 4096-row launch), valid only
 # while the kernel's source is the one that was measured.
-TRAFFIC = {"lnq_vgemm": {"bytes": 4 * (1474252544 + 269069568), "source": "lnq_vgemm.cu",
-                         "sha256": "5efc3929f14fbbf906c511263b8c5bda727ce09fb1129ba4f39d5548bfaca71c"}}
+TRAFFIC = {"lnq_vgemm": {"bytes": 4 * (1365949184 + 270225152), "source": "lnq_vgemm.cu",
+                         "sha256": "556269b73b751b571ee70f646966983f5c0d0a608a1b7bfae7b6c8f3eb238c91"}}
 
 
 def measured_traffic(kernel):

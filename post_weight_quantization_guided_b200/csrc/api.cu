@@ -41,9 +41,8 @@ static bool valid_m(int m) { return m == 2 || m == 4 || m == 8 || m == 16; }
 // Workspace layout (all offsets 256-byte aligned):
 //   BUILD_FISHER:   header | S [groups][n] f32 | M [n] f32 | pimax [groups] u32
 //                   | A [n][d_in] f16 | B [groups][n][d_in] f16
-//   QUANTIZE_ROWS:  header | status [d_out] i32 | Fp [groups][3][d_in][ld] bf16 (ld = d_in
-//                   rounded up to a multiple of 8) | Fh [groups][2][d_in][ld] f16 | fexp
-//                   [groups][d_in] i32 | rexp [d_out] i32
+//   QUANTIZE_ROWS:  header | status [d_out] i32 | Fh [groups][2][d_in][ld] f16 (ld = d_in
+//                   rounded up to a multiple of 8) | fexp [groups][d_in] i32 | rexp [d_out] i32
 //                   | V [d_out][d_in][m] f32 | U [d_out][d_in] f32 (u = F r) | dC [d_out][m] f32
 //                   | sweep history [CTAs][2 ceil(d_in / 128)][3][4 KB] (Delta pieces)
 //                   | right-operand image of the product [row tiles][K blocks][N][64] 16-bit
@@ -65,16 +64,15 @@ static FisherWs fisher_ws(int64_t n, int64_t d_in, int groups)
 }
 
 struct LnqWs {
-    size_t st_off, fp_off, fh_off, fexp_off, rexp_off, v_off, ut_off, dc_off, hist_off, img_off,
+    size_t st_off, fh_off, fexp_off, rexp_off, v_off, ut_off, dc_off, hist_off, img_off,
         total;
 };
 static LnqWs lnq_ws(int64_t d_in, int64_t d_out, int groups, int m)
 {
     LnqWs w;
     w.st_off = kWsHeader;
-    w.fp_off = align_up(w.st_off + static_cast<size_t>(d_out) * 4, 256);
-    const size_t ld = static_cast<size_t>((d_in + 7) / 8 * 8);  // bf16 piece row stride
-    w.fh_off = align_up(w.fp_off + static_cast<size_t>(groups) * 3 * d_in * ld * 2, 256);
+    w.fh_off = align_up(w.st_off + static_cast<size_t>(d_out) * 4, 256);
+    const size_t ld = static_cast<size_t>((d_in + 7) / 8 * 8);  // fp16 piece row stride
     w.fexp_off = align_up(w.fh_off + static_cast<size_t>(groups) * 2 * d_in * ld * 2, 256);
     w.rexp_off = align_up(w.fexp_off + static_cast<size_t>(groups) * d_in * 4, 256);
     w.v_off = align_up(w.rexp_off + static_cast<size_t>(d_out) * 4, 256);
@@ -91,7 +89,6 @@ static LnqWorkspace carve(void *ws, const LnqWs &lay)
     uint8_t *b = static_cast<uint8_t *>(ws);
     LnqWorkspace w;
     w.status = reinterpret_cast<int32_t *>(b + lay.st_off);
-    w.Fp = reinterpret_cast<__nv_bfloat16 *>(b + lay.fp_off);
     w.Fh = reinterpret_cast<__half *>(b + lay.fh_off);
     w.fexp = reinterpret_cast<int32_t *>(b + lay.fexp_off);
     w.rexp = reinterpret_cast<int32_t *>(b + lay.rexp_off);
@@ -236,7 +233,7 @@ lnq_status lnq_quantize_rows(const float *F, int groups, const float *W, int64_t
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const LnqWorkspace w = carve(ws, lay);
     DeviceErr err{reinterpret_cast<uint32_t *>(ws), g_wait_limit.load()};
-    if (cudaMemsetAsync(ws, 0, lay.fp_off, s) != cudaSuccess)   // header and row status
+    if (cudaMemsetAsync(ws, 0, lay.fh_off, s) != cudaSuccess)   // header and row status
         return LNQ_ERR_CUDA;
     if (lnq_iterate_launch(F, groups, W, d_out, d_in, m, iters, C, Q, J_out, w, err,
                            device_sm_count(), s) != cudaSuccess)

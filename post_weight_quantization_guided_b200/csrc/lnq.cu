@@ -108,16 +108,13 @@ cudaError_t lnq_iterate_launch(const float *F, int groups, const float *W, int64
 {
     cudaError_t e;
     if (iters > 0 || J != nullptr)
-        if ((e = lnq_split_f(F, d, groups, w.Fp, s)) != cudaSuccess)
-            return e;
-    if (iters > 0)
         if ((e = lnq_split_f16(F, d, groups, w.Fh, w.fexp, s)) != cudaSuccess)
             return e;
     for (int it = 0; it < iters; ++it) {
         if ((e = lnq_residual_scale(Q, W, C, d, d_out, m, w.rexp, s)) != cudaSuccess)
             return e;
-        if ((e = lnq_vgemm(w.Fp, w.Fh, w.fexp, w.rexp, groups, Q, W, C, w.V, w.U, w.img, d, d_out,
-                           m, false, err, num_sms, s)) != cudaSuccess)
+        if ((e = lnq_vgemm(w.Fh, w.fexp, w.rexp, groups, Q, W, C, w.V, w.U, w.img, d, d_out, m,
+                           false, err, num_sms, s)) != cudaSuccess)
             return e;
         if ((e = lnq_solve(w.V, w.U, Q, C, w.dC, w.status, d, d_out, m, s)) != cudaSuccess)
             return e;
@@ -126,8 +123,10 @@ cudaError_t lnq_iterate_launch(const float *F, int groups, const float *W, int64
             return e;
     }
     if (J != nullptr) {
-        if ((e = lnq_vgemm(w.Fp, w.Fh, w.fexp, w.rexp, groups, Q, W, C, nullptr, w.U, w.img, d,
-                           d_out, m, true, err, num_sms, s)) != cudaSuccess)
+        if ((e = lnq_residual_scale(Q, W, C, d, d_out, m, w.rexp, s)) != cudaSuccess)
+            return e;
+        if ((e = lnq_vgemm(w.Fh, w.fexp, w.rexp, groups, Q, W, C, nullptr, w.U, w.img, d, d_out, m,
+                           true, err, num_sms, s)) != cudaSuccess)
             return e;
         if ((e = lnq_objective_from_u(w.U, W, C, Q, J, d, d_out, m, s)) != cudaSuccess)
             return e;

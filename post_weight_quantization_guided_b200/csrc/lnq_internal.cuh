@@ -17,7 +17,6 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
 // Device scratch of lnq_quantize_rows / lnq_objective, carved from the caller's workspace.
 struct LnqWorkspace {
     int32_t *status;     // [d_out] sticky per-row status
-    __nv_bfloat16 *Fp;   // [groups][3][d][ld] bf16 pieces of F (exact)
     __half *Fh;          // [groups][2][d][ld] fp16 pieces of F, rows scaled by 2^fexp
     int32_t *fexp;       // [groups][d]
     int32_t *rexp;       // [d_out] residual scales
@@ -36,15 +35,13 @@ cudaError_t lnq_iterate_launch(const float *F, int groups, const float *W, int64
                                const LnqWorkspace &w, DeviceErr err, int num_sms, cudaStream_t s);
 
 // lnq_vgemm.cu
-bool encode_f_pieces(CUtensorMap *map, const __nv_bfloat16 *Fp, int64_t d, int groups);
 bool encode_f16_pieces(CUtensorMap *map, const __half *Fh, int64_t d, int groups);
-cudaError_t lnq_split_f(const float *F, int64_t d, int groups, __nv_bfloat16 *Fp, cudaStream_t s);
 cudaError_t lnq_split_f16(const float *F, int64_t d, int groups, __half *Fh, int32_t *fexp,
                           cudaStream_t s);
 cudaError_t lnq_residual_scale(const uint8_t *Q, const float *W, const float *C, int64_t d,
                                int64_t d_out, int m, int32_t *rexp, cudaStream_t s);
 size_t lnq_vgemm_image_bytes(int64_t d, int64_t d_out, int groups, int m);
-cudaError_t lnq_vgemm(const __nv_bfloat16 *Fp, const __half *Fh, const int32_t *fexp,
+cudaError_t lnq_vgemm(const __half *Fh, const int32_t *fexp,
                       const int32_t *rexp, int groups, const uint8_t *Q, const float *W,
                       const float *C, float *V, float *U, uint16_t *img, int64_t d, int64_t d_out,
                       int m, bool residual_only, DeviceErr err, int num_sms, cudaStream_t s);

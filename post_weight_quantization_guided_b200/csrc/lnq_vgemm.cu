@@ -8,21 +8,22 @@
 //      [V_j1 | u_j1 | V_j2 | u_j2 | ...] = F x [P_j1 | r_j1 | P_j2 | r_j2 | ...]
 //
 // whose left operand F is shared by every row of the group. This kernel computes it with
-// tcgen05.mma.cta_group::2.kind::f16, exactly in fp32 terms:
-//   * F (fp32) is split into three bf16 pieces F = F1 + F2 + F3 (exact for normal values), and
-//     the three products accumulate into one TMEM accumulator;
-//   * the one-hot columns are 0/1 (exact in bf16); r is split the same way into three bf16
-//     pieces, one column each, so u = sum of nine exact bf16 x bf16 products;
-//   * accumulation is fp32 in TMEM.
-// Two CTAs (a cluster pair on two SMs) share one MMA of 256 coordinates (i) x 256 columns
-// (RT rows x (m one-hot + 3 residual-piece columns), RT = floor(256 / (m + 3))): each CTA loads
-// the F tiles of its own 128 coordinates by TMA (K-major, 128-byte swizzle, no multicast) and
-// builds half of the right operand's columns in shared memory from Q, W and C, so that each SM
-// reads half of the right operand per MMA. The even CTA issues the MMAs; each CTA's TMEM holds
-// its 128 coordinates x all columns, and its epilogue writes V[j][i][b] and U[j][i] (both
-// contiguous across a warp's coordinates). With m = 0 the kernel
-// computes u = F r only (42 rows per 128-column tile), which the objective uses.
-#include <cuda_bf16.h>
+// tcgen05.mma.cta_group::2.kind::f16 on fp16 pieces:
+//   * each row i of F (fp32) is scaled by a power of two 2^fexp[i] that puts its largest entry
+//     in [2^14, 2^15) and split into two fp16 pieces H1 + H2, 22 significant bits of every
+//     entry;
+//   * the one-hot columns are 0/1 (exact in fp16); r_j is scaled by 2^rexp[j] the same way and
+//     split into three fp16 pieces (33 bits, exact for fp32 r), one column each, so u takes six
+//     piece products and V two;
+//   * accumulation is fp32 in TMEM; the epilogue removes the power-of-two scales exactly.
+// The right operand [P | r pieces] of every (row tile, K block) is written once per call as an
+// image in HBM and loaded by TMA like F. Two CTAs (a cluster pair on two SMs) share one MMA of
+// 256 coordinates (i) x 256 columns (RT rows x (m one-hot + 3 residual-piece columns),
+// RT = floor(256 / (m + 3))): each CTA loads the F tiles of its own 128 coordinates and half of
+// the right operand's rows (K-major, 128-byte swizzle, no multicast). The even CTA issues the
+// MMAs; each CTA's TMEM holds its 128 coordinates x all columns, and its epilogue writes V[j][i][b]
+// and U[j][i] (both contiguous across a warp's coordinates). With m = 0 the kernel computes
+// u = F r only (85 rows per 256-column tile), which the objective uses.
 #include <cuda_fp16.h>
 
 #include "common.cuh"
@@ -46,18 +47,18 @@ constexpr uint16_t PAIR = 0x3;                   // both CTAs of the cluster
 constexpr long long kPairDrainLimit = 1LL << 22;
 }  // namespace vg
 
-// Tile shapes. With one-hot columns (M > 0) the MMA is 256 columns wide and two TMEM
-// accumulators alternate between tiles. The residual-only product (M == 0) feeds the objective,
-// which sums r_i u_i with cancellation; there the MMA is 128 columns wide and the K range is cut
-// into four segments with one accumulator each, so each fp32 accumulator takes a quarter of the
-// additions. Each CTA holds HALF = NCOLS / 2 rows of the right operand per stage.
+// Tile shapes. Both products take F as two fp16 pieces and the residual as three fp16 pieces, and
+// the MMA is 256 columns wide. With one-hot columns (M > 0) two TMEM accumulators alternate between
+// tiles. The residual-only product (M == 0) feeds the objective, which sums r_i u_i with
+// cancellation; there the K range is cut into two segments with one accumulator each, so each
+// fp32 accumulator takes half of the additions. Each CTA holds HALF = NCOLS / 2 rows of the right
+// operand per stage.
 template <int M>
 struct VgShape {
-    static constexpr bool F16 = M > 0;                  // fp16 pieces (V, u) or exact bf16 (J)
-    static constexpr int PIECES = F16 ? 2 : 3;          // pieces of F in the left operand
-    static constexpr int NCOLS = M > 0 ? 256 : 128;     // MMA N
+    static constexpr int PIECES = 2;                    // fp16 pieces of F in the left operand
+    static constexpr int NCOLS = 256;                   // MMA N
     static constexpr int HALF = NCOLS / 2;              // right-operand rows held by one CTA
-    static constexpr int SEGS = M > 0 ? 1 : 4;          // K segments (one accumulator each)
+    static constexpr int SEGS = M > 0 ? 1 : 2;          // K segments (one accumulator each)
     static constexpr int SETS = M > 0 ? 2 : 1;          // accumulator sets (tile double-buffer)
     static constexpr int RT = NCOLS / (M + 3);          // rows per tile
     static constexpr int ONEHOT = RT * M;               // one-hot columns
@@ -75,43 +76,8 @@ struct VgShape {
     static_assert(SMEM <= vg::MAX_DYN_SMEM, "shared memory");
 };
 
-__device__ __forceinline__ uint16_t bf16_bits(float x)
-{
-    return __bfloat16_as_ushort(__float2bfloat16_rn(x));
-}
-
-// The three bf16 pieces of x: x == p0 + p1 + p2 exactly for normal fp32 x.
-__device__ __forceinline__ void split3(float x, float &p0, float &p1, float &p2)
-{
-    p0 = __bfloat162float(__float2bfloat16_rn(x));
-    const float r1 = x - p0;
-    p1 = __bfloat162float(__float2bfloat16_rn(r1));
-    p2 = r1 - p1;
-}
-
-// Row stride (elements) of the bf16 pieces: TMA needs row strides that are multiples of 16 B.
+// Row stride (elements) of the fp16 pieces of F: TMA needs row strides that are multiples of 16 B.
 __host__ __device__ inline int64_t pieces_stride(int64_t d) { return (d + 7) / 8 * 8; }
-
-// F (fp32 [groups][d][d]) -> Fp (bf16 [groups][3][d][ld]), ld = pieces_stride(d), zero padded.
-__global__ void split_f_kernel(const float *__restrict__ F, int64_t d, int groups,
-                               __nv_bfloat16 *__restrict__ Fp)
-{
-    const int64_t ld = pieces_stride(d);
-    const int64_t plane = d * ld;
-    const int64_t total = plane * groups;
-    for (int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; e < total;
-         e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-        const int64_t g = e / plane, r = e - g * plane;
-        const int64_t row = r / ld, col = r - row * ld;
-        float p0 = 0.f, p1 = 0.f, p2 = 0.f;
-        if (col < d)
-            split3(F[(g * d + row) * d + col], p0, p1, p2);
-        __nv_bfloat16 *base = Fp + g * 3 * plane + r;
-        base[0] = __float2bfloat16_rn(p0);
-        base[plane] = __float2bfloat16_rn(p1);
-        base[2 * plane] = __float2bfloat16_rn(p2);
-    }
-}
 
 // F (fp32 [groups][d][d]) -> Fh (fp16 [groups][2][d][ld]) with a power-of-two scale per row:
 // F[i][k] 2^fexp[i] = H1 + H2 up to 2^-22 relative (2^-39 of the row's largest entry for entries
@@ -180,8 +146,8 @@ __global__ void __launch_bounds__(256)
 // loaded by TMA like F: NCOLS rows (the product's columns) x 64 coordinates, row-major
 // [row tiles][K blocks][NCOLS][64]. Column n < ONEHOT of a row tile is the indicator of class n % M
 // for its row n / M; ONEHOT <= n < USED is residual piece (n - ONEHOT) % 3 of row (n - ONEHOT) / 3;
-// the rest is zero, as is everything outside the problem. fp16 (residuals scaled by 2^rexp) when
-// there are one-hot columns, exact bf16 pieces for the residual-only product.
+// the rest is zero, as is everything outside the problem. All values are fp16, residuals scaled by
+// 2^rexp.
 template <int M>
 __global__ void __launch_bounds__(256)
     operand_image_kernel(const uint8_t *__restrict__ Q, const float *__restrict__ W,
@@ -236,7 +202,7 @@ __global__ void __launch_bounds__(256)
                     }
                 }
                 if (onehot) {
-                    constexpr uint16_t ONE = S::F16 ? 0x3C00u : 0x3F80u;  // 1.0 in fp16 / bf16
+                    constexpr uint16_t ONE = 0x3C00u;  // 1.0 in fp16
                     const int b = n - r * (M > 0 ? M : 1);
 #pragma unroll
                     for (int e = 0; e < 8; ++e)
@@ -244,22 +210,15 @@ __global__ void __launch_bounds__(256)
                             out[e >> 1] |= static_cast<uint32_t>(ONE) << (16 * (e & 1));
                 } else {
                     const int pc = (n - S::ONEHOT) % 3;
-                    const float sc = S::F16 ? pow2f(rexp[j]) : 1.f;
+                    const float sc = pow2f(rexp[j]);
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
                         if (qv[e] == 0xFFu)
                             continue;
                         const float rv = C[j * m + (qv[e] & (m - 1))] - wv[e];
-                        uint16_t bits;
-                        if constexpr (S::F16) {
-                            uint16_t b0, b1, b2;
-                            split3_f16(rv * sc, b0, b1, b2);
-                            bits = pc == 0 ? b0 : (pc == 1 ? b1 : b2);
-                        } else {
-                            float p0, p1, p2;
-                            split3(rv, p0, p1, p2);
-                            bits = bf16_bits(pc == 0 ? p0 : (pc == 1 ? p1 : p2));
-                        }
+                        uint16_t b0, b1, b2;
+                        split3_f16(rv * sc, b0, b1, b2);
+                        const uint16_t bits = pc == 0 ? b0 : (pc == 1 ? b1 : b2);
                         out[e >> 1] |= static_cast<uint32_t>(bits) << (16 * (e & 1));
                     }
                 }
@@ -310,7 +269,7 @@ __global__ void __launch_bounds__(vg::NUM_THREADS, 1)
     using namespace vg;
     using S = VgShape<M>;
     constexpr int NSLOT = S::A_SLOTS;
-    constexpr uint32_t IDESC = umma_idesc_f16kind(2 * BM, S::NCOLS, false, false, S::F16);
+    constexpr uint32_t IDESC = umma_idesc_f16kind(2 * BM, S::NCOLS, false, false, true);
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(align_up(reinterpret_cast<uintptr_t>(smem_raw), 1024));
     uint8_t *a_base = smem;                                       // [NSLOT][16 KB]
@@ -511,59 +470,65 @@ __global__ void __launch_bounds__(vg::NUM_THREADS, 1)
             vg_tile_coords<M>(p, tile, g, row0, row_end, ip, rt_all);
             const int64_t i = static_cast<int64_t>(ip) * 2 * BM + static_cast<int64_t>(cr) * BM +
                               quarter * 32 + lane;
-            float uacc[S::RT];
-#pragma unroll
-            for (int r = 0; r < S::RT; ++r)
-                uacc[r] = 0.f;
-            // fp16 mode: the accumulator carries 2^fexp[i] (and 2^rexp[j] on residual columns)
+            // the accumulator carries 2^fexp[i] (and 2^rexp[j] on residual columns)
             const float inv_si =
-                pow2f((S::F16 && i < p.d) ? -p.fexp[static_cast<int64_t>(g) * p.d + i] : 0);
-            for (int seg = 0; seg < S::SEGS; ++seg) {
-                // K block kb feeds segment kb * SEGS / nk; skip segments that received none
-                const int first = (seg * nk + S::SEGS - 1) / S::SEGS;
-                if (first >= nk || (first * S::SEGS) / nk != seg)
-                    continue;
+                pow2f(i < p.d ? -p.fexp[static_cast<int64_t>(g) * p.d + i] : 0);
+            // Chunks of 32 columns in order, each summed over the K segments that received a
+            // K block; a row's three residual columns are added as they come and its u is
+            // written at the third, so only one partial sum is live at a time.
+            float uacc = 0.f;
 #pragma unroll
-                for (int ch = 0; ch < S::CHUNKS; ++ch) {
-                    float v[32];
+            for (int ch = 0; ch < S::CHUNKS; ++ch) {
+                float v[32];
+#pragma unroll
+                for (int seg = 0; seg < S::SEGS; ++seg) {
+                    // K block kb feeds segment kb * SEGS / nk; skip segments that received none
+                    const int first = (seg * nk + S::SEGS - 1) / S::SEGS;
+                    const bool fed = seg == 0 || (first < nk && (first * S::SEGS) / nk == seg);
                     const uint32_t taddr =
                         tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                         static_cast<uint32_t>((acc * S::SEGS + seg) * S::NCOLS + ch * 32);
-                    tmem_ld_32x32b_x32(taddr, v);
+                    if (seg == 0) {
+                        tmem_ld_32x32b_x32(taddr, v);
+                    } else if (fed) {
+                        float w[32];
+                        tmem_ld_32x32b_x32(taddr, w);
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const int col = ch * 32 + e;
-                        if constexpr (M > 0) {
-                            // M divides 32, so each row's M columns sit inside one chunk.
-                            if (col < S::ONEHOT && col % M == 0) {
-                                const int64_t j = row0 + col / M;
-                                if (j < row_end && i < p.d) {
-                                    float *dst = p.V + (j * p.d + i) * M;
-                                    if constexpr (M >= 4) {
+                        for (int e = 0; e < 32; ++e)
+                            v[e] += w[e];
+                    }
+                }
 #pragma unroll
-                                        for (int b4 = 0; b4 < M / 4; ++b4)
-                                            reinterpret_cast<float4 *>(dst)[b4] = make_float4(
-                                                v[e + 4 * b4] * inv_si, v[e + 4 * b4 + 1] * inv_si,
-                                                v[e + 4 * b4 + 2] * inv_si, v[e + 4 * b4 + 3] * inv_si);
-                                    } else {
-                                        *reinterpret_cast<float2 *>(dst) =
-                                            make_float2(v[e] * inv_si, v[e + 1] * inv_si);
-                                    }
+                for (int e = 0; e < 32; ++e) {
+                    const int col = ch * 32 + e;
+                    if constexpr (M > 0) {
+                        // M divides 32, so each row's M columns sit inside one chunk.
+                        if (col < S::ONEHOT && col % M == 0) {
+                            const int64_t j = row0 + col / M;
+                            if (j < row_end && i < p.d) {
+                                float *dst = p.V + (j * p.d + i) * M;
+                                if constexpr (M >= 4) {
+#pragma unroll
+                                    for (int b4 = 0; b4 < M / 4; ++b4)
+                                        reinterpret_cast<float4 *>(dst)[b4] = make_float4(
+                                            v[e + 4 * b4] * inv_si, v[e + 4 * b4 + 1] * inv_si,
+                                            v[e + 4 * b4 + 2] * inv_si, v[e + 4 * b4 + 3] * inv_si);
+                                } else {
+                                    *reinterpret_cast<float2 *>(dst) =
+                                        make_float2(v[e] * inv_si, v[e + 1] * inv_si);
                                 }
                             }
                         }
-                        if (col >= S::ONEHOT && col < S::USED)
-                            uacc[(col - S::ONEHOT) / 3] += v[e];
                     }
-                }
-            }
-            if (i < p.d) {
-#pragma unroll
-                for (int r = 0; r < S::RT; ++r) {
-                    const int64_t j = row0 + r;
-                    if (j < row_end)
-                        p.U[j * p.d + i] =
-                            S::F16 ? (uacc[r] * inv_si) * pow2f(-p.rexp[j]) : uacc[r];
+                    if (col >= S::ONEHOT && col < S::USED) {
+                        uacc += v[e];
+                        if ((col - S::ONEHOT) % 3 == 2) {
+                            const int64_t j = row0 + (col - S::ONEHOT) / 3;
+                            if (j < row_end && i < p.d)
+                                p.U[j * p.d + i] = (uacc * inv_si) * pow2f(-p.rexp[j]);
+                            uacc = 0.f;
+                        }
+                    }
                 }
             }
             tc_fence_before();
@@ -583,18 +548,6 @@ __global__ void __launch_bounds__(vg::NUM_THREADS, 1)
 // ------------------------------------------------------------------------------------------
 // Host launchers
 // ------------------------------------------------------------------------------------------
-cudaError_t lnq_split_f(const float *F, int64_t d, int groups, __nv_bfloat16 *Fp, cudaStream_t s)
-{
-    const int64_t total = d * pieces_stride(d) * groups;
-    const int threads = 256;
-    int64_t blocks = (total + threads - 1) / threads;
-    if (blocks > 148 * 32)
-        blocks = 148 * 32;
-    KernelTimer timer("lnq_split_f", s);
-    split_f_kernel<<<static_cast<unsigned>(blocks), threads, 0, s>>>(F, d, groups, Fp);
-    return cudaGetLastError();
-}
-
 cudaError_t lnq_split_f16(const float *F, int64_t d, int groups, __half *Fh, int32_t *fexp,
                           cudaStream_t s)
 {
@@ -612,7 +565,7 @@ cudaError_t lnq_residual_scale(const uint8_t *Q, const float *W, const float *C,
     return cudaGetLastError();
 }
 
-// Tensor map over F's pieces [groups * planes][d][ld] (bf16: three planes per group, fp16: two):
+// Tensor map over F's pieces [groups * planes][d][ld] (two fp16 planes per group):
 // 64 x 128 (column x row) boxes, 128-byte swizzle; reads outside d x d return zeros.
 static bool encode_pieces_map(CUtensorMap *map, const void *pieces, int64_t d, int planes,
                               CUtensorMapDataType type)
@@ -630,12 +583,6 @@ static bool encode_pieces_map(CUtensorMap *map, const void *pieces, int64_t d, i
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-// Tensor map over the bf16 pieces Fp [groups][3][d][ld].
-bool encode_f_pieces(CUtensorMap *map, const __nv_bfloat16 *Fp, int64_t d, int groups)
-{
-    return encode_pieces_map(map, Fp, d, groups * 3, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
 }
 
 // Tensor map over the fp16 pieces Fh [groups][2][d][ld].
@@ -685,7 +632,7 @@ static cudaError_t launch_vgemm_m(const CUtensorMap &map, VgParams p, uint16_t *
         return cudaErrorInvalidValue;
     p.num_tiles = static_cast<int>(num_rt_all * p.i_pairs);
     {
-        KernelTimer timer(S::F16 ? "lnq_operand_image" : "lnq_residual_image", s);
+        KernelTimer timer(M > 0 ? "lnq_operand_image" : "lnq_residual_image", s);
         int64_t blocks = num_rt_all * nk;
         if (blocks > static_cast<int64_t>(num_sms) * 16)
             blocks = static_cast<int64_t>(num_sms) * 16;
@@ -705,8 +652,7 @@ static cudaError_t launch_vgemm_m(const CUtensorMap &map, VgParams p, uint16_t *
         cuuint64_t strides[1] = {128};
         cuuint32_t box[2] = {64, static_cast<cuuint32_t>(S::HALF)};
         cuuint32_t estr[2] = {1, 1};
-        if (encode(&bmap, S::F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
-                   2, img, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+        if (encode(&bmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, img, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return cudaErrorInvalidValue;
@@ -752,17 +698,14 @@ static cudaError_t launch_vgemm_m(const CUtensorMap &map, VgParams p, uint16_t *
 }
 
 // m in {2,4,8,16}: V and U for every row from the fp16 pieces (Fh, fexp) and the residual scales
-// rexp; residual_only: U = F r from the exact bf16 pieces Fp.
-cudaError_t lnq_vgemm(const __nv_bfloat16 *Fp, const __half *Fh, const int32_t *fexp,
+// rexp; residual_only: U = F r alone (the objective's product), from the same pieces.
+cudaError_t lnq_vgemm(const __half *Fh, const int32_t *fexp,
                       const int32_t *rexp, int groups, const uint8_t *Q, const float *W,
                       const float *C, float *V, float *U, uint16_t *img, int64_t d, int64_t d_out,
                       int m, bool residual_only, DeviceErr err, int num_sms, cudaStream_t s)
 {
     CUtensorMap map;
-    const bool ok = residual_only
-                        ? encode_f_pieces(&map, Fp, d, groups)
-                        : encode_pieces_map(&map, Fh, d, groups * 2, CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
-    if (!ok)
+    if (!encode_f16_pieces(&map, Fh, d, groups))
         return cudaErrorInvalidValue;
     VgParams p{};
     p.Q = Q;
