@@ -276,6 +276,13 @@ __device__ __forceinline__ void cp_async16(void *dst, const void *src)
                  "l"(reinterpret_cast<uint64_t>(src))
                  : "memory");
 }
+// 8-byte asynchronous global -> shared copy (both addresses 8-byte aligned).
+__device__ __forceinline__ void cp_async8(void *dst, const void *src)
+{
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(dst)),
+                 "l"(reinterpret_cast<uint64_t>(src))
+                 : "memory");
+}
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 

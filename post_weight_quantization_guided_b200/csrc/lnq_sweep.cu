@@ -24,10 +24,12 @@
 //     the row's sorted codebook, and the coordinate moves only if its exact change is strictly
 //     negative; the block's later coordinates are corrected in registers from the 32 x 32 diagonal
 //     tile of F. Then the four sweep warps write the codes and moves and correct the window's
-//     later blocks in shared memory from a 32 x 128 strip of F.
+//     later blocks in shared memory from a 32 x 128 strip of F (one TMA box per block).
 // Warp roles: 0 TMA and bulk copies, 1 MMA issue, 2-5 window assembly (TMEM -> shared memory),
 // 6-9 the sweep. Every wait is bounded; a wait that gives up sets the
 // workspace error flag and its role stops, and every role drains what it has in flight.
+#include <cstring>
+
 #include "common.cuh"
 #include "lnq_internal.cuh"
 #include "profile.cuh"
@@ -64,7 +66,7 @@ constexpr int OFF_DL = OFF_UW + 2 * RB * UW_LD * 4;
 constexpr int OFF_C = OFF_DL + BLK * RB * 4;
 constexpr int OFF_DC = OFF_C + RB * 17 * 4;
 constexpr int OFF_QB = OFF_DC + RB * 16 * 4;
-constexpr int OFF_WM = OFF_QB + RB * (BLK + 8);
+constexpr int OFF_WM = OFF_QB + 2 * RB * (BLK + 8);   // codes: two blocks in flight
 constexpr int OFF_TS = (OFF_WM + MAX_WIN + 15) / 16 * 16;  // [2][RB] Delta scales 2^t, 2^-t
 constexpr int OFF_SRT = OFF_TS + 2 * RB * 4;               // [RB][17] sorted codebook
 constexpr int OFF_ORD = OFF_SRT + RB * 17 * 4;             // [RB][16] its codeword indices
@@ -72,7 +74,7 @@ constexpr int OFF_FINV = OFF_ORD + RB * 16;                // [BLK] 1 / F_ii of 
 constexpr int OFF_FDG = OFF_FINV + BLK * 4;                // [BLK] F_ii of the block
 constexpr int OFF_RM = OFF_FDG + BLK * 4;                  // [RB] moved-coordinate mask per row
 constexpr int OFF_BAR = OFF_RM + RB * 4;
-constexpr int NBARS = 2 * NA + 2 * NH + 2 + 2 + 2 + 2 + 3;
+constexpr int NBARS = 2 * NA + 2 * NH + 2 + 2 + 2 + 2 + 3 + 2;
 constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
 constexpr size_t SMEM = 1024 + OFF_MISC + 32;
 static_assert(SMEM <= 232448, "shared memory");
@@ -90,13 +92,15 @@ struct SwParams {
     uint8_t *hist;       // [CTAs][2 * windows][2][4 KB]
     const int32_t *fexp; // [groups][d] row scales of the fp16 pieces of F
     int64_t d, d_out, rows_per_group;
+    int strip_tma;       // F strips by TMA (d % 4 == 0, F 16-byte aligned) or by plain loads
     int blocks_per_group, nwin;
     DeviceErr err;
 };
 
 template <int M>
 __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
-    sweep_kernel(const __grid_constant__ CUtensorMap fmap, SwParams p)
+    sweep_kernel(const __grid_constant__ CUtensorMap fmap, const __grid_constant__ CUtensorMap smap,
+                 SwParams p)
 {
     using namespace sw;
     constexpr uint32_t IDESC = umma_idesc_f16kind(WIN, RB, false, false, /*f16=*/true);
@@ -110,7 +114,8 @@ __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
     float(*dl_s)[RB] = reinterpret_cast<float(*)[RB]>(smem + OFF_DL);       // [BLK][RB]
     float(*c_s)[17] = reinterpret_cast<float(*)[17]>(smem + OFF_C);         // [RB][m]
     float(*dc_s)[16] = reinterpret_cast<float(*)[16]>(smem + OFF_DC);       // [RB][m]
-    uint8_t(*qb_s)[BLK + 8] = reinterpret_cast<uint8_t(*)[BLK + 8]>(smem + OFF_QB);  // rows 8-byte aligned
+    // [2][RB][BLK + 8] codes of the current and the next block, rows 8-byte aligned
+    uint8_t(*qb2)[RB][BLK + 8] = reinterpret_cast<uint8_t(*)[RB][BLK + 8]>(smem + OFF_QB);
     volatile uint8_t *wmask = smem + OFF_WM;                         // [window]: some row moved
     float *dsc = reinterpret_cast<float *>(smem + OFF_TS);            // [RB] 2^t_r of Delta row r
     float *dinv = dsc + RB;                                           // [RB] 2^-t_r
@@ -131,6 +136,7 @@ __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
     uint64_t *bs_ready = uw_free + 2;
     uint64_t *bs_free = bs_ready + 1;
     uint64_t *drain = bs_free + 1;
+    uint64_t *strip_full = drain + 1;                                // [2] F strip buffers
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + OFF_MISC);
     volatile unsigned *moved_s = reinterpret_cast<volatile unsigned *>(smem + OFF_MISC + 16);  // [4]
 
@@ -165,8 +171,12 @@ __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
         mbar_init(bs_ready, SWEEP_THREADS);
         mbar_init(bs_free, 2);
         mbar_init(drain, 1);
+        mbar_init(&strip_full[0], 1);
+        mbar_init(&strip_full[1], 1);
         fence_barrier_init();
         tma_prefetch_desc(&fmap);
+        if (p.strip_tma)
+            tma_prefetch_desc(&smap);
     }
     for (int e = threadIdx.x; e < RB * 16; e += blockDim.x) {
         const int r = e >> 4, b = e & 15;
@@ -439,10 +449,22 @@ __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
         const int t = threadIdx.x - 6 * 32;  // 0..127
         const float *Fg = p.F + static_cast<int64_t>(g) * d * d;
         const bool vecF = (d & 3) == 0 && (reinterpret_cast<uintptr_t>(p.F) & 15u) == 0;
-        // F rows b0..b0+31, columns wstart..wstart+127 of the group (zero outside F) -> strip buf
+        uint32_t spar = 0u, sused = 0u;  // strip buffers: parity of TMA fills, ever filled
+        // F rows b0..b0+31, columns wstart..wstart+127 of the group (zero outside F) -> strip buf:
+        // one TMA box (completing on strip_full[buf]) or, when F's rows are not 16-byte multiples,
+        // plain loads
         auto load_strip = [&](int buf, int64_t b0, int64_t wstart) {
             float *st = strip + buf * (BLK * WIN);
-            if (vecF) {
+            if (p.strip_tma) {
+                if (t == 0) {
+                    fence_proxy_async_smem();
+                    mbar_arrive_expect_tx(&strip_full[buf], BLK * WIN * 4);
+                    tma_load_3d(st, &smap, &strip_full[buf], static_cast<int32_t>(wstart),
+                                static_cast<int32_t>(b0), g);
+                }
+                spar ^= 1u << buf;
+                sused |= 1u << buf;
+            } else if (vecF) {
                 for (int e = t; e < BLK * WIN / 4; e += SWEEP_THREADS) {
                     const int r = e / (WIN / 4), c4 = e % (WIN / 4);
                     const int64_t row = b0 + r, col = wstart + 4 * c4;
@@ -463,30 +485,30 @@ __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
         };
         uint32_t wuses = 0u;  // bit per window buffer: phase parity
         int bi = 0;
-        // codes of this thread's row (r = t / 4) at coordinates k0 + 8 (t % 4) .. + 7, classes
-        // masked, 0 outside the problem
+        // codes of this thread's row (r = t / 4) at coordinates k0 + 8 (t % 4) .. + 7 into code
+        // buffer buf: an asynchronous copy (completed with the block's F strip), plain loads at a
+        // ragged end, 0 outside the problem. Readers mask the classes.
         const bool qvec = (d & 7) == 0 && (reinterpret_cast<uintptr_t>(p.Q) & 7u) == 0;
-        auto fetch_codes = [&](int64_t k0) -> uint2 {
+        auto fetch_codes = [&](int buf, int64_t k0) {
             const int r = t >> 2, s = t & 3;
             const int64_t k = k0 + 8 * s;
-            uint32_t w[2] = {0u, 0u};
-            if (r < nrows && k < d) {
-                const uint8_t *src = p.Q + (row0 + r) * d + k;
-                if (qvec && k + 8 <= d) {
-                    const uint2 v = *reinterpret_cast<const uint2 *>(src);
-                    w[0] = v.x;
-                    w[1] = v.y;
-                } else {
+            uint8_t *dst = &qb2[buf][r][8 * s];
+            if (r < nrows && k < d && qvec && k + 8 <= d) {
+                cp_async8(dst, p.Q + (row0 + r) * d + k);
+            } else {
+                uint32_t w[2] = {0u, 0u};
+                if (r < nrows && k < d) {
+                    const uint8_t *src = p.Q + (row0 + r) * d + k;
 #pragma unroll
                     for (int e = 0; e < 8; ++e)
                         if (k + e < d)
                             w[e >> 2] |= static_cast<uint32_t>(src[e]) << (8 * (e & 3));
                 }
+                *reinterpret_cast<uint2 *>(dst) = make_uint2(w[0], w[1]);
             }
-            constexpr uint32_t MASK4 = 0x01010101u * static_cast<uint32_t>(M - 1);
-            return make_uint2(w[0] & MASK4, w[1] & MASK4);
+            cp_async_commit();
         };
-        uint2 qpf = fetch_codes(0);
+        constexpr uint32_t MASK4 = 0x01010101u * static_cast<uint32_t>(M - 1);
         // warp 6 (lane = row): the row's codebook sorted, equal values in index order, and the
         // midpoints between neighbours, for the decisions of the whole sweep
         float mid[M > 1 ? M - 1 : 1];
@@ -507,7 +529,9 @@ __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
             for (int k = 0; k + 1 < M; ++k)
                 mid[k] = 0.5f * (srt_s[r][k] + srt_s[r][k + 1]);
         }
+        fetch_codes(0, 0);
         load_strip(0, 0, 0);
+        bool failed = false;
         for (int T = 0; T < nwin; ++T) {
             const int64_t wstart = static_cast<int64_t>(T) * WIN;
             const int buf = T & 1;
@@ -528,21 +552,26 @@ __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
                 if (b0 >= d)
                     break;  // only in the last window
                 const int nb = (d - b0 < BLK) ? static_cast<int>(d - b0) : BLK;
+                int sok = 1;
+                if (p.strip_tma)
+                    sok = mbar_wait(&strip_full[bi & 1], (bi >> 1) & 1, limit) ? 1 : 0;
                 cp_async_wait_all();
-                named_bar_sync(SWEEP_BAR, SWEEP_THREADS);  // strip of this block complete
+                // strip and codes of this block complete
+                if (!named_bar_and(SWEEP_BAR, SWEEP_THREADS, sok)) {
+                    if (t == 0)
+                        raise_error(p.err, kErrTimeout, 37);
+                    failed = true;
+                    break;
+                }
                 {
                     const int64_t nb0 = b0 + BLK;
-                    if (nb0 < d)
+                    if (nb0 < d) {
+                        fetch_codes((bi + 1) & 1, nb0);
                         load_strip((bi + 1) & 1, nb0, lb + 1 < NBLK ? wstart : wstart + WIN);
+                    }
                 }
+                uint8_t(*qb_s)[BLK + 8] = qb2[bi & 1];
                 const float *st = strip + (bi & 1) * (BLK * WIN) + lb * BLK;  // st[ii * WIN + c]
-                {
-                    // codes of the block (thread (r = t / 4, s = t % 4) holds 8 of them, fetched
-                    // during the previous block), then the fetch of the next block's codes
-                    const int r = t >> 2, s = t & 3;
-                    *reinterpret_cast<uint2 *>(&qb_s[r][8 * s]) = qpf;
-                    qpf = fetch_codes(b0 + BLK);
-                }
                 if (t < BLK) {
                     const float f = st[t * WIN + t];
                     fdg_s[t] = f;
@@ -565,7 +594,7 @@ __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
                     uint32_t qw[BLK / 4];
 #pragma unroll
                     for (int v = 0; v < BLK / 4; ++v)
-                        qw[v] = *reinterpret_cast<const uint32_t *>(&qb_s[r][4 * v]);
+                        qw[v] = *reinterpret_cast<const uint32_t *>(&qb_s[r][4 * v]) & MASK4;
 #pragma unroll
                     for (int ii = 0; ii < BLK; ++ii)
                         ub[ii] = uw[r * UW_LD + lb * BLK + ii];
@@ -693,6 +722,8 @@ __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
                 }
                 named_bar_sync(SWEEP_BAR, SWEEP_THREADS);
             }
+            if (failed)
+                break;
             if (t == 0)
                 wmask[T] = wmoved ? 1 : 0;
             if (keep) {
@@ -702,6 +733,12 @@ __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
             mbar_arrive(&uw_free[buf]);
         }
         cp_async_wait_all();
+        // after an early exit, let the strip copies in flight land (the last fill of buffer b
+        // completes phase fills - 1)
+        if (p.strip_tma && t == 0)
+            for (int b = 0; b < 2; ++b)
+                if ((sused >> b) & 1u)
+                    mbar_wait(&strip_full[b], ((spar >> b) & 1u) ^ 1u, kDrainLimit);
     }
 
     tc_fence_before();
@@ -722,15 +759,36 @@ size_t lnq_sweep_history_bytes(int64_t d, int64_t d_out, int groups)
     return static_cast<size_t>(ctas) * 2 * nwin * sw::H_CHUNK;
 }
 
+// Tensor map over F (fp32 [groups][d][d]) for the sweep's strips: 128 x 32 (column x row) boxes, no
+// swizzle, zeros outside d x d. Needs rows of 16-byte multiples (d % 4 == 0) and an aligned F.
+static bool encode_f32_strips(CUtensorMap *map, const float *F, int64_t d, int groups)
+{
+    if ((d & 3) != 0 || (reinterpret_cast<uintptr_t>(F) & 15u) != 0)
+        return false;
+    auto encode = tensor_map_encoder();
+    if (encode == nullptr)
+        return false;
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(d),
+                          static_cast<cuuint64_t>(groups)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 4, static_cast<cuuint64_t>(d * d) * 4};
+    cuuint32_t box[3] = {sw::WIN, sw::BLK, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float *>(F), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int M>
-static cudaError_t sweep_m(const CUtensorMap &map, const SwParams &p, unsigned grid, cudaStream_t s)
+static cudaError_t sweep_m(const CUtensorMap &map, const CUtensorMap &smap, const SwParams &p,
+                           unsigned grid, cudaStream_t s)
 {
     cudaError_t e = cudaFuncSetAttribute(sweep_kernel<M>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(sw::SMEM));
     if (e != cudaSuccess)
         return e;
     KernelTimer timer("lnq_sweep", s);
-    sweep_kernel<M><<<grid, sw::NUM_THREADS, sw::SMEM, s>>>(map, p);
+    sweep_kernel<M><<<grid, sw::NUM_THREADS, sw::SMEM, s>>>(map, smap, p);
     return cudaGetLastError();
 }
 
@@ -741,7 +799,11 @@ cudaError_t lnq_sweep(const float *F, const __half *Fh, const int32_t *fexp, int
     CUtensorMap map;
     if (!encode_f16_pieces(&map, Fh, d, groups))
         return cudaErrorInvalidValue;
+    CUtensorMap smap;
+    memset(&smap, 0, sizeof(smap));
+    const bool strip_tma = encode_f32_strips(&smap, F, d, groups);
     SwParams p{};
+    p.strip_tma = strip_tma ? 1 : 0;
     p.F = F;
     p.V = V;
     p.dC = dC;
@@ -758,10 +820,10 @@ cudaError_t lnq_sweep(const float *F, const __half *Fh, const int32_t *fexp, int
     p.err = err;
     const unsigned grid = static_cast<unsigned>(p.blocks_per_group) * static_cast<unsigned>(groups);
     switch (m) {
-    case 2: return sweep_m<2>(map, p, grid, s);
-    case 4: return sweep_m<4>(map, p, grid, s);
-    case 8: return sweep_m<8>(map, p, grid, s);
-    case 16: return sweep_m<16>(map, p, grid, s);
+    case 2: return sweep_m<2>(map, smap, p, grid, s);
+    case 4: return sweep_m<4>(map, smap, p, grid, s);
+    case 8: return sweep_m<8>(map, smap, p, grid, s);
+    case 16: return sweep_m<16>(map, smap, p, grid, s);
     }
     return cudaErrorInvalidValue;
 }
