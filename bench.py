@@ -129,7 +129,7 @@ def algorithmic_work(layer, kernel: str, launches: int, moves_per_sweep: float):
     if kernel in ("lnq_operand_image", "lnq_residual_image"):
         # write the right-operand image (N columns x d coordinates x 2 bytes per row tile), read Q
         # and W once
-        rt = max(1, 256 // (m + 3)) if kernel == "lnq_operand_image" else 256 // 3
+        rt = 256 // m if kernel == "lnq_operand_image" else 256 // 3
         ncols = 256
         tiles = g * -(-(dout // g) // rt)
         return tiles * ncols * (-(-d // 64) * 64) * 2.0 + 5.0 * dout * d, "byte"
@@ -138,8 +138,8 @@ def algorithmic_work(layer, kernel: str, launches: int, moves_per_sweep: float):
     if kernel == "lnq_residual_scale":
         return 5.0 * dout * d, "byte"                               # read W and Q
     if kernel == "lnq_vgemm":
-        # the dense product F x [P_j | r_j] over all rows: 2 d^2 (m + 1) flops per row
-        return 2.0 * d * d * (m + 1) * dout, "flop"
+        # the class-binned product V_j = F P_j over all rows: 2 d^2 m flops per row
+        return 2.0 * d * d * m * dout, "flop"
     if kernel == "lnq_residual_gemm":
         return 2.0 * d * d * dout, "flop"                           # u = F r for every row
     if kernel == "lnq_solve":
@@ -153,13 +153,12 @@ def algorithmic_work(layer, kernel: str, launches: int, moves_per_sweep: float):
     return 0.0, "unknown"
 
 
-# tcgen05 work per unit of algorithmic work. Both products take F as two fp16 pieces: the V/u
-# product against m exact one-hot columns and three residual-piece columns per row, the
-# objective's residual product against the three residual-piece columns alone (six products).
+# tcgen05 work per unit of algorithmic work. Both products take F as two fp16 pieces: the
+# class-binned product against m exact one-hot columns per row (two products), the residual
+# product (F w once per call, F r for the objective) against three residual-piece columns (six).
 def hw_flop_factor(layer, kernel):
-    m = layer.m
     if kernel == "lnq_vgemm":
-        return (2.0 * m + 6.0) / (m + 1)
+        return 2.0
     if kernel == "lnq_residual_gemm":
         return 6.0
     return None

@@ -14,9 +14,11 @@
 //   init_kernel   sort w_j in shared memory (bitonic), pick the midpoint order statistics
 //                 c_q = sorted[floor((2q+1) d / (2m))], assign each weight its nearest codeword
 //                 (fp64 distances, ties to the lower index). One CTA per row.
-//   iteration     lnq_vgemm (V = F P, u = F r on tensor cores) -> lnq_solve (codebook) ->
-//                 lnq_sweep (assignment); see lnq_vgemm.cu and lnq_sweep.cu.
-//   objective     residual-only lnq_vgemm (u = F r) -> J = r^T u.
+//   once          residual lnq_vgemm with the zero codebook: U = -F w (P^T F w for every
+//                 iteration's codebook, and u = F r = U + V c)
+//   iteration     lnq_vgemm (V = F P on tensor cores) -> lnq_solve (codebook) -> lnq_sweep
+//                 (assignment from u = U + V c); see lnq_vgemm.cu and lnq_sweep.cu.
+//   objective     residual lnq_vgemm (u = F r) -> J = r^T u.
 #include "common.cuh"
 #include "lnq_internal.cuh"
 #include "profile.cuh"
@@ -110,11 +112,17 @@ cudaError_t lnq_iterate_launch(const float *F, int groups, const float *W, int64
     if (iters > 0 || J != nullptr)
         if ((e = lnq_split_f16(F, d, groups, w.Fh, w.fexp, s)) != cudaSuccess)
             return e;
-    for (int it = 0; it < iters; ++it) {
-        if ((e = lnq_residual_scale(Q, W, C, d, d_out, m, w.rexp, s)) != cudaSuccess)
+    if (iters > 0) {
+        // U = -F w (the residual of the zero codebook), shared by every iteration
+        if ((e = lnq_residual_scale(Q, W, nullptr, d, d_out, m, w.rexp, s)) != cudaSuccess)
             return e;
-        if ((e = lnq_vgemm(w.Fh, w.fexp, w.rexp, groups, Q, W, C, w.V, w.U, w.img, d, d_out, m,
-                           false, err, num_sms, s)) != cudaSuccess)
+        if ((e = lnq_vgemm(w.Fh, w.fexp, w.rexp, groups, Q, W, nullptr, nullptr, w.U, w.img, d,
+                           d_out, m, true, err, num_sms, s)) != cudaSuccess)
+            return e;
+    }
+    for (int it = 0; it < iters; ++it) {
+        if ((e = lnq_vgemm(w.Fh, w.fexp, nullptr, groups, Q, W, C, w.V, nullptr, w.img, d, d_out,
+                           m, false, err, num_sms, s)) != cudaSuccess)
             return e;
         if ((e = lnq_solve(w.V, w.U, Q, C, w.dC, w.status, d, d_out, m, s)) != cudaSuccess)
             return e;

@@ -3,12 +3,14 @@
 // Source: "GuidedQuant" (jinukkim.me blog), LNQ section: the codebook step
 // c <- (P^T F P)^-1 P^T F w, and the objective (w^ - w)^T F (w^ - w) of each row.
 //
-// solve_kernel (one CTA per row). From V = F P and u = F r (lnq_vgemm.cu) it forms
-// M = P^T V and t = P^T u, streaming the row's V and u once with coalesced loads: fp32 partial
-// sums over 32-coordinate chunks (a few terms each), fp64 across chunks; every sum runs in a
-// fixed order, so results do not depend on scheduling. An fp64 Cholesky over the
-// non-empty codewords (one warp, a lane per row) then solves M dc = -t (the closed-form update in
-// residual form), and the kernel writes c + dc in fp32 together with the exact fp32 change.
+// solve_kernel (one CTA per row). From V = F P and U = -F w (lnq_vgemm.cu, the residual product
+// with a zero codebook) it forms M = P^T V and t = P^T U = -P^T F w, streaming the row's V and U
+// once with coalesced loads: fp32 partial sums over 32-coordinate chunks (a few terms each), fp64
+// across chunks; every sum runs in a fixed order, so results do not depend on scheduling. An fp64
+// Cholesky over the non-empty codewords (one warp, a lane per row) then solves M c = -t, the
+// closed form c = (P^T F P)^-1 P^T F w, and the kernel writes the new codebook in fp32 to C and to
+// dC (the sweep starts from u = U + V dC = F (c[q] - w)). Empty codewords keep their values; a
+// singular M leaves the codebook unchanged.
 //
 // objective_u_kernel: J_j = r_j^T u_j with u = F r from the residual-only product, fp64 sums in a
 // fixed order.
@@ -140,7 +142,7 @@ __global__ void __launch_bounds__(kSolveThreads)
     __syncthreads();
 
     // 2. Cholesky over the non-empty codewords (one warp, lane = row, right-looking), then
-    //    dc = -M^-1 t by forward and back substitution.
+    //    c = -M^-1 t by forward and back substitution.
     if (warp == 0) {
         int idx[M];
         int nn = 0;
@@ -177,10 +179,10 @@ __global__ void __launch_bounds__(kSolveThreads)
             }
         }
         float *c = C + j * M;
-        float *dc = dC + j * M;
+        float *cn = dC + j * M;
         if (singular) {
             if (lane < M)
-                dc[lane] = 0.f;
+                cn[lane] = c[lane];
             if (lane == 0)
                 status[j] |= LNQ_ROW_SINGULAR;
         } else {
@@ -211,13 +213,12 @@ __global__ void __launch_bounds__(kSolveThreads)
                     s -= Ls[k][lane] * xk;
             }
             if (lane < M)
-                dc[lane] = 0.f;
+                cn[lane] = c[lane];
             __syncwarp();
             if (lane < nn) {
-                const float old = c[myc];
-                const float nw = static_cast<float>(static_cast<double>(old) + x);
+                const float nw = static_cast<float>(x);
                 c[myc] = nw;
-                dc[myc] = static_cast<float>(static_cast<double>(nw) - static_cast<double>(old));
+                cn[myc] = nw;
             }
         }
     }

@@ -8,8 +8,8 @@
 // One CTA per 32 rows of one Fisher group. Coordinates are taken in windows of 128 (the height
 // of a tensor-core tile), each window in four blocks of 32.
 //   * Before a window starts, its u is assembled left-looking: the value at the start of the
-//     sweep, u0 + V dc (u0 = F r for the previous codebook and V = F P from lnq_vgemm, dc the
-//     codebook change from lnq_solve), plus F[window][earlier coordinates] x Delta[earlier
+//     sweep, U + V c (U = -F w and V = F P from lnq_vgemm, c the new codebook from lnq_solve,
+//     so U + V c = F (c[q] - w)), plus F[window][earlier coordinates] x Delta[earlier
 //     coordinates], Delta being the moves made so far in this sweep. That product runs on tcgen05
 //     tensor cores: F as its two fp16 pieces with a power-of-two scale per row (the operand of
 //     lnq_vgemm, 22 bits per entry), Delta as two fp16 pieces with a power-of-two scale per
@@ -85,7 +85,7 @@ static_assert(OFF_QB % 8 == 0 && OFF_STRIP % 16 == 0, "vector accesses to the co
 struct SwParams {
     const float *F;      // [groups][d][d]
     const float *V;      // [d_out][d][m]
-    const float *dC;     // [d_out][m]
+    const float *dC;     // [d_out][m] the new codebook (u at the start = U + V dC)
     const float *U;      // [d_out][d] u = F r for the previous codebook
     const float *C;      // [d_out][m]
     uint8_t *Q;          // [d_out][d]
@@ -358,7 +358,7 @@ __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
     } else if (warp < 6) {
         // ---------------------------------------------------------------- window assembly
         // Thread = coordinate kl of the window (= TMEM lane; warp w reads lanes 32 (w % 4)..).
-        // u of window T for the CTA's rows: U (F r for the previous codebook) + V dc, plus the
+        // u of window T for the CTA's rows: U (= -F w) + V c (c the new codebook), plus the
         // accumulator of the moves made before the window, written to the window buffer T & 1.
         const int quarter = warp & 3;
         const int kl = quarter * 32 + lane;

@@ -1,29 +1,30 @@
 // lnq_vgemm.cu -- the dense contraction of an LNQ iteration on tcgen05 tensor cores.
 //
 // Source: "GuidedQuant" (jinukkim.me blog), LNQ section. The codebook update
-// c <- (P^T F P)^-1 P^T F w needs, per output row j, the class-binned products V_j = F P_j
-// (d x m; P_j is the one-hot assignment) and the residual gradient u_j = F r_j with
-// r_j = c_j[q_j] - w_j. For all rows of one Fisher group these are a single product
+// c <- (P^T F P)^-1 P^T F w needs, per output row j, the class-binned product V_j = F P_j (d x m;
+// P_j is the one-hot assignment): M_j = P_j^T V_j. P^T F w comes from y_j = F w_j, which does not
+// change between iterations, and the sweep starts from u_j = F r_j = V_j c_j - y_j with
+// r_j = c_j[q_j] - w_j. Two products serve all rows of one Fisher group, whose left operand F
+// they share:
 //
-//      [V_j1 | u_j1 | V_j2 | u_j2 | ...] = F x [P_j1 | r_j1 | P_j2 | r_j2 | ...]
+//      [V_j1 | V_j2 | ...] = F x [P_j1 | P_j2 | ...]        (m one-hot columns per row)
+//      [u_j1 | u_j2 | ...] = F x [r_j1 | r_j2 | ...]        (residual; r = -w gives -y)
 //
-// whose left operand F is shared by every row of the group. This kernel computes it with
-// tcgen05.mma.cta_group::2.kind::f16 on fp16 pieces:
+// This kernel computes either with tcgen05.mma.cta_group::2.kind::f16 on fp16 pieces:
 //   * each row i of F (fp32) is scaled by a power of two 2^fexp[i] that puts its largest entry
 //     in [2^14, 2^15) and split into two fp16 pieces H1 + H2, 22 significant bits of every
 //     entry;
-//   * the one-hot columns are 0/1 (exact in fp16); r_j is scaled by 2^rexp[j] the same way and
-//     split into three fp16 pieces (33 bits, exact for fp32 r), one column each, so u takes six
-//     piece products and V two;
+//   * the one-hot columns are 0/1 (exact in fp16), two piece products; r_j is scaled by 2^rexp[j]
+//     the same way and split into three fp16 pieces (33 bits, exact for fp32 r), one column each,
+//     six piece products;
 //   * accumulation is fp32 in TMEM; the epilogue removes the power-of-two scales exactly.
-// The right operand [P | r pieces] of every (row tile, K block) is written once per call as an
-// image in HBM and loaded by TMA like F. Two CTAs (a cluster pair on two SMs) share one MMA of
-// 256 coordinates (i) x 256 columns (RT rows x (m one-hot + 3 residual-piece columns),
-// RT = floor(256 / (m + 3))): each CTA loads the F tiles of its own 128 coordinates and half of
+// The right operand (one-hot columns or residual pieces) of every (row tile, K block) is written
+// once per call as an image in HBM and loaded by TMA like F. Two CTAs (a cluster pair on two SMs)
+// share one MMA of 256 coordinates (i) x 256 columns (RT = 256 / m rows of m one-hot columns, or
+// 85 rows of 3 residual pieces): each CTA loads the F tiles of its own 128 coordinates and half of
 // the right operand's rows (K-major, 128-byte swizzle, no multicast). The even CTA issues the
 // MMAs; each CTA's TMEM holds its 128 coordinates x all columns, and its epilogue writes V[j][i][b]
-// and U[j][i] (both contiguous across a warp's coordinates). With m = 0 the kernel computes
-// u = F r only (85 rows per 256-column tile), which the objective uses.
+// or U[j][i] (both contiguous across a warp's coordinates).
 #include <cuda_fp16.h>
 
 #include "common.cuh"
@@ -47,12 +48,12 @@ constexpr uint16_t PAIR = 0x3;                   // both CTAs of the cluster
 constexpr long long kPairDrainLimit = 1LL << 22;
 }  // namespace vg
 
-// Tile shapes. Both products take F as two fp16 pieces and the residual as three fp16 pieces, and
-// the MMA is 256 columns wide. With one-hot columns (M > 0) two TMEM accumulators alternate between
-// tiles. The residual-only product (M == 0) feeds the objective, which sums r_i u_i with
-// cancellation; there the K range is cut into two segments with one accumulator each, so each
-// fp32 accumulator takes half of the additions. Each CTA holds HALF = NCOLS / 2 rows of the right
-// operand per stage.
+// Tile shapes. Both products take F as two fp16 pieces and the MMA is 256 columns wide. The
+// class-binned product (M > 0) has M one-hot columns per row and two TMEM accumulators that
+// alternate between tiles. The residual product (M == 0: three fp16 pieces of r per row) feeds the
+// objective, which sums r_i u_i with cancellation; there the K range is cut into two segments with
+// one accumulator each, so each fp32 accumulator takes half of the additions. Each CTA holds
+// HALF = NCOLS / 2 rows of the right operand per stage.
 template <int M>
 struct VgShape {
     static constexpr int PIECES = 2;                    // fp16 pieces of F in the left operand
@@ -60,9 +61,10 @@ struct VgShape {
     static constexpr int HALF = NCOLS / 2;              // right-operand rows held by one CTA
     static constexpr int SEGS = M > 0 ? 1 : 2;          // K segments (one accumulator each)
     static constexpr int SETS = M > 0 ? 2 : 1;          // accumulator sets (tile double-buffer)
-    static constexpr int RT = NCOLS / (M + 3);          // rows per tile
+    static constexpr int RES = M > 0 ? 0 : 3;           // residual-piece columns per row
+    static constexpr int RT = NCOLS / (M + RES);        // rows per tile
     static constexpr int ONEHOT = RT * M;               // one-hot columns
-    static constexpr int USED = RT * (M + 3);           // columns carrying data
+    static constexpr int USED = RT * (M + RES);         // columns carrying data
     static constexpr int CHUNKS = (USED + 31) / 32;     // 32-column TMEM loads per accumulator
     static constexpr int B_BYTES = HALF * 128;          // HALF rows x 64 k of 16-bit values
     static constexpr int A_FIT = (vg::MAX_DYN_SMEM - 1024 - vg::BAR_BYTES -
@@ -121,7 +123,8 @@ __global__ void __launch_bounds__(256)
 }
 
 // Per-row power-of-two scale of the residual r_j = c_j[q_j] - w_j for the fp16 right operand:
-// max_k |r_jk| 2^rexp[j] in [2^14, 2^15). One warp per row.
+// max_k |r_jk| 2^rexp[j] in [2^14, 2^15); C == nullptr stands for the zero codebook (r_j = -w_j).
+// One warp per row.
 __global__ void __launch_bounds__(256)
     residual_scale_kernel(const uint8_t *__restrict__ Q, const float *__restrict__ W,
                           const float *__restrict__ C, int64_t d, int64_t d_out, int m,
@@ -133,7 +136,7 @@ __global__ void __launch_bounds__(256)
         return;
     float mx = 0.f;
     for (int64_t k = lane; k < d; k += 32)
-        mx = fmaxf(mx, fabsf(C[j * m + (Q[j * d + k] & (m - 1))] - W[j * d + k]));
+        mx = fmaxf(mx, fabsf((C != nullptr ? C[j * m + (Q[j * d + k] & (m - 1))] : 0.f) - W[j * d + k]));
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1)
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
@@ -147,7 +150,7 @@ __global__ void __launch_bounds__(256)
 // [row tiles][K blocks][NCOLS][64]. Column n < ONEHOT of a row tile is the indicator of class n % M
 // for its row n / M; ONEHOT <= n < USED is residual piece (n - ONEHOT) % 3 of row (n - ONEHOT) / 3;
 // the rest is zero, as is everything outside the problem. All values are fp16, residuals scaled by
-// 2^rexp.
+// 2^rexp (C == nullptr: the zero codebook, r = -w).
 template <int M>
 __global__ void __launch_bounds__(256)
     operand_image_kernel(const uint8_t *__restrict__ Q, const float *__restrict__ W,
@@ -215,7 +218,7 @@ __global__ void __launch_bounds__(256)
                     for (int e = 0; e < 8; ++e) {
                         if (qv[e] == 0xFFu)
                             continue;
-                        const float rv = C[j * m + (qv[e] & (m - 1))] - wv[e];
+                        const float rv = (C != nullptr ? C[j * m + (qv[e] & (m - 1))] : 0.f) - wv[e];
                         uint16_t b0, b1, b2;
                         split3_f16(rv * sc, b0, b1, b2);
                         const uint16_t bits = pc == 0 ? b0 : (pc == 1 ? b1 : b2);
@@ -697,8 +700,8 @@ static cudaError_t launch_vgemm_m(const CUtensorMap &map, VgParams p, uint16_t *
     return cudaGetLastError();
 }
 
-// m in {2,4,8,16}: V and U for every row from the fp16 pieces (Fh, fexp) and the residual scales
-// rexp; residual_only: U = F r alone (the objective's product), from the same pieces.
+// V = F P for every row (m in {2,4,8,16}) or, with residual_only, U = F r with the residual scales
+// rexp (C == nullptr: the zero codebook, U = -F w), both from the fp16 pieces (Fh, fexp).
 cudaError_t lnq_vgemm(const __half *Fh, const int32_t *fexp,
                       const int32_t *rexp, int groups, const uint8_t *Q, const float *W,
                       const float *C, float *V, float *U, uint16_t *img, int64_t d, int64_t d_out,
