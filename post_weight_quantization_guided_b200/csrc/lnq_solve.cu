@@ -35,7 +35,9 @@ __global__ void __launch_bounds__(kSolveThreads)
     constexpr int NW = kSolveThreads / 32;
     constexpr int PAIRS = M * M;
     constexpr int PPL = (PAIRS + 31) / 32;     // (class, column) pairs per lane, same class
-    __shared__ float stv[NW][32][M + 1];       // staged V rows and u of 32 coordinates
+    constexpr int LOGM = M == 2 ? 1 : (M == 4 ? 2 : (M == 8 ? 3 : 4));
+    constexpr int SROW = M >= 4 ? M + 4 : 4;   // staged row: V[i][0..M-1], u[i]; 16-byte aligned
+    __shared__ __align__(16) float stv[NW][32][SROW];  // staged V rows and u of 32 coordinates
     __shared__ uint8_t stq[NW][32];
     __shared__ double Mp[NW][PAIRS], tp[NW][M];
     __shared__ int cp[NW][M];
@@ -67,13 +69,9 @@ __global__ void __launch_bounds__(kSolveThreads)
             const float *vi = Vj + i * M;
             if constexpr (M >= 4) {
 #pragma unroll
-                for (int b4 = 0; b4 < M / 4; ++b4) {
-                    const float4 x = reinterpret_cast<const float4 *>(vi)[b4];
-                    stv[warp][lane][4 * b4] = x.x;
-                    stv[warp][lane][4 * b4 + 1] = x.y;
-                    stv[warp][lane][4 * b4 + 2] = x.z;
-                    stv[warp][lane][4 * b4 + 3] = x.w;
-                }
+                for (int b4 = 0; b4 < M / 4; ++b4)
+                    reinterpret_cast<float4 *>(&stv[warp][lane][0])[b4] =
+                        reinterpret_cast<const float4 *>(vi)[b4];
             } else {
                 const float2 x = *reinterpret_cast<const float2 *>(vi);
                 stv[warp][lane][0] = x.x;
@@ -85,15 +83,17 @@ __global__ void __launch_bounds__(kSolveThreads)
             stq[warp][lane] = 0xFF;
         }
         __syncwarp();
-        // the chunk's coordinates of this lane's class (one ballot per class), visited in lane
-        // order: fp32 partials of the chunk, added to the fp64 sums once per chunk
+        // the chunk's coordinates of this lane's class (from one ballot per bit of the class),
+        // visited in lane order: fp32 partials of the chunk, added to the fp64 sums once per chunk
         const int mq = stq[warp][lane];
-        uint32_t mine = 0u;
+        uint32_t mine = __ballot_sync(0xffffffffu, mq < M);
 #pragma unroll
-        for (int c = 0; c < M; ++c) {
-            const uint32_t mc = __ballot_sync(0xffffffffu, mq == c);
-            mine = (a == c) ? mc : mine;
+        for (int k = 0; k < LOGM; ++k) {
+            const uint32_t bk = __ballot_sync(0xffffffffu, (mq >> k) & 1);
+            mine &= ((a >> k) & 1) ? bk : ~bk;
         }
+        if (!owner)
+            mine = 0u;
         float pf[PPL], tf = 0.f;
 #pragma unroll
         for (int q = 0; q < PPL; ++q)
@@ -102,9 +102,20 @@ __global__ void __launch_bounds__(kSolveThreads)
         while (mine != 0u) {
             const int e = __ffs(mine) - 1;
             mine &= mine - 1u;
+            if constexpr (PPL % 4 == 0) {
 #pragma unroll
-            for (int q = 0; q < PPL; ++q)
-                pf[q] += stv[warp][e][b0 + q];
+                for (int q4 = 0; q4 < PPL / 4; ++q4) {
+                    const float4 v4 = *reinterpret_cast<const float4 *>(&stv[warp][e][b0 + 4 * q4]);
+                    pf[4 * q4] += v4.x;
+                    pf[4 * q4 + 1] += v4.y;
+                    pf[4 * q4 + 2] += v4.z;
+                    pf[4 * q4 + 3] += v4.w;
+                }
+            } else {
+#pragma unroll
+                for (int q = 0; q < PPL; ++q)
+                    pf[q] += stv[warp][e][b0 + q];
+            }
             tf += stv[warp][e][M];
         }
 #pragma unroll
