@@ -59,8 +59,8 @@ struct VgShape {
     static constexpr int PIECES = 2;                    // fp16 pieces of F in the left operand
     static constexpr int NCOLS = 256;                   // MMA N
     static constexpr int HALF = NCOLS / 2;              // right-operand rows held by one CTA
-    static constexpr int SEGS = M > 0 ? 1 : 2;          // K segments (one accumulator each)
-    static constexpr int SETS = M > 0 ? 2 : 1;          // accumulator sets (tile double-buffer)
+    static constexpr int SEGS = 1;                      // K segments (one accumulator each)
+    static constexpr int SETS = 2;                      // accumulator sets (tile double-buffer)
     static constexpr int RES = M > 0 ? 0 : 3;           // residual-piece columns per row
     static constexpr int RT = NCOLS / (M + RES);        // rows per tile
     static constexpr int ONEHOT = RT * M;               // one-hot columns
