@@ -587,14 +587,18 @@ __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
                     // t = -+inf, the extreme codeword, which is the best one for a linear change.)
                     const int r = lane;
                     const bool vr = r < nrows;
-                    // registers hold the block's u and codes only (fewer live values, no spills on
-                    // the chain); each coordinate's current value is read and its move written in
-                    // shared memory
+                    // registers hold the block's u and codes; each coordinate's current value is
+                    // read and its move written in shared memory
                     float ub[BLK];
-                    uint32_t qw[BLK / 4];
+                    // qw: the block's codes as decided so far; qo: the codes before the block, from
+                    // which each coordinate's current value is read (no decision changes them, so
+                    // those reads do not wait for the previous coordinate)
+                    uint32_t qw[BLK / 4], qo[BLK / 4];
 #pragma unroll
-                    for (int v = 0; v < BLK / 4; ++v)
+                    for (int v = 0; v < BLK / 4; ++v) {
                         qw[v] = *reinterpret_cast<const uint32_t *>(&qb_s[r][4 * v]) & MASK4;
+                        qo[v] = qw[v];
+                    }
 #pragma unroll
                     for (int ii = 0; ii < BLK; ++ii)
                         ub[ii] = uw[r * UW_LD + lb * BLK + ii];
@@ -602,20 +606,22 @@ __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
 #pragma unroll
                     for (int ii = 0; ii < BLK; ++ii) {
                         const float u = ub[ii];
-                        const float cur = c_s[r][(qw[ii >> 2] >> (8 * (ii & 3))) & 0xFFu];
+                        const float cur = c_s[r][(qo[ii >> 2] >> (8 * (ii & 3))) & 0xFFu];
                         const float tt = fmaf(-u, finv_s[ii], cur);
-                        // number of midpoints below t, summed as a balanced tree
-                        int cnt[M];
+                        // number of midpoints below t, summed as a balanced tree of floats (exact
+                        // small integers; floating-point adds keep the tree's order, so the count is
+                        // four additions deep)
+                        float cnt[M];
 #pragma unroll
                         for (int k = 0; k < M; ++k)
-                            cnt[k] = (k + 1 < M && tt > mid[k < M - 1 ? k : 0]) ? 1 : 0;
+                            cnt[k] = (k + 1 < M && tt > mid[k < M - 1 ? k : 0]) ? 1.f : 0.f;
 #pragma unroll
                         for (int w2 = 1; w2 < M; w2 *= 2) {
 #pragma unroll
                             for (int k = 0; k + w2 < M; k += 2 * w2)
                                 cnt[k] += cnt[k + w2];
                         }
-                        const int pos = cnt[0];
+                        const int pos = static_cast<int>(cnt[0]);
                         const float da = srt_s[r][pos] - cur;
                         const float D = da * fmaf(da, fdg_s[ii], 2.f * u);
                         // a strictly negative change implies c != cur
