@@ -13,7 +13,8 @@
 //     coordinates], Delta being the moves made so far in this sweep. That product runs on tcgen05
 //     tensor cores: F as its two fp16 pieces with a power-of-two scale per row (the operand of
 //     lnq_vgemm, 22 bits per entry), Delta as two fp16 pieces with a power-of-two scale per
-//     row of W (22 bits), the four piece products accumulated in fp32 in TMEM; the scales are
+//     row of W (22 bits), three piece products (F2 x D2, below 2^-22 of each term, is left out)
+//     accumulated in fp32 in TMEM; the scales are
 //     undone exactly when the window is assembled.
 //   * Delta of finished windows is kept per CTA in a global history (fp16 pieces), already in
 //     the swizzled K-major layout the MMA reads, written and read back with byte-exact copies.
@@ -285,7 +286,7 @@ __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
     } else if (warp == 1) {
         // ---------------------------------------------------------------- MMA issue
         // Accumulator T & 1 (32 TMEM columns, lane = coordinate of window T, column = row) gets
-        // sum over chunks c of F[T][c] x Delta[c], four piece products of four K=16 MMAs each.
+        // sum over chunks c of F[T][c] x Delta[c], three piece products of four K=16 MMAs each.
         if (lane == 0) {
             int aslot = 0, hslot = 0;
             uint32_t aph = 0u, hph = 0u, uses = 0u;  // bit per slot / accumulator: phase parity
@@ -307,8 +308,9 @@ __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
                         tc_fence_after();
                         if (math) {
                             const uint32_t sa = smem_u32(a_base + aslot * A_TILE);
-                            // every F piece times every Delta piece
-                            for (int pb = 0; pb < DPIECES; ++pb) {
+                            // F1 x (D1 + D2) + F2 x D1: the dropped F2 x D2 is below 2^-22 of
+                            // each term, the size of the pieces' own rounding
+                            for (int pb = 0; pb < DPIECES - pa; ++pb) {
 #pragma unroll
                                 for (int kk = 0; kk < CH / 16; ++kk) {
                                     // K-major, 128-byte swizzle: 16 k = 32 bytes along the row
