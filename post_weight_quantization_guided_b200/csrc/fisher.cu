@@ -14,13 +14,17 @@
 //                           one side and fp16 on the other bounds the error of every F entry by
 //                           about 5e-4 * sqrt(F_ii F_kk) even for a single token; bf16 on both
 //                           sides can reach 8e-3.
-//   fisher_syrk_kernel      persistent tcgen05 GEMM over the upper-triangle tiles of every F_g.
-//                           TMA brings 64(t) x 64(i) boxes of A and B_g into shared memory in the
-//                           128-byte-swizzled MN-major layout (no transpose of X is needed); one
-//                           thread issues tcgen05.mma.kind::f16 (M=128, N=256, K=16) into a TMEM
-//                           accumulator; four epilogue warps read TMEM, scale and write the tile
-//                           and its mirror image. Two TMEM accumulators let the epilogue of one
-//                           tile overlap the main loop of the next.
+//   fisher_syrk_kernel      persistent tcgen05 GEMM over the upper-triangle 256 x 256 tiles of
+//                           every F_g, two CTAs (a cluster pair on two SMs) per tile. Each CTA's
+//                           TMA brings its 128 rows of A and its 128 of the tile's 256 columns of
+//                           B_g, as 64(t) x 64(i) boxes in the 128-byte-swizzled MN-major layout
+//                           (no transpose of X is needed), with the bytes of both counted on the
+//                           even CTA's barrier; the even CTA's thread issues
+//                           tcgen05.mma.cta_group::2.kind::f16 (M=256, N=256, K=16); each CTA's
+//                           four epilogue warps read its 128 rows from TMEM, scale and write them
+//                           and their mirror image. Two TMEM accumulators let the epilogue of one
+//                           tile overlap the main loop of the next. Per CTA and stage 32 KB feed
+//                           128 x 256 x 64 MACs (48 KB for a single CTA's tile of the same size).
 // Without gradients (G == NULL) the product is X^T X: A = B = X in bf16, no preparation pass.
 #include <cuda_fp16.h>
 
@@ -148,21 +152,26 @@ __global__ void guided_operands_kernel(const __nv_bfloat16 *__restrict__ X,
 }
 
 // ------------------------------------------------------------------------------------------
-// tcgen05 SYRK over upper-triangle tiles
+// tcgen05 SYRK over upper-triangle tiles, two CTAs (a cluster pair on two SMs) per tile
 // ------------------------------------------------------------------------------------------
 namespace syrk {
-constexpr int BM = 128;          // tile rows (i), TMEM lanes
+constexpr int BM = 128;          // tile rows (i) per CTA: TMEM lanes; the pair covers 2 BM
+constexpr int PM = 2 * BM;       // rows of a pair tile
 constexpr int BN = 256;          // tile columns (k), TMEM columns per accumulator
+constexpr int HALF = BN / 2;     // columns of the right operand each CTA loads
 constexpr int BK = 64;           // tokens per pipeline stage
-constexpr int STAGES = 4;
+constexpr int STAGES = 6;
 constexpr int BOX = 64;          // TMA box: 64 elements (128 B) along i/k  x  64 tokens
 constexpr int BOX_BYTES = BOX * BK * 2;                  // 8 KB
 constexpr int A_BYTES = (BM / BOX) * BOX_BYTES;          // 16 KB
-constexpr int B_BYTES = (BN / BOX) * BOX_BYTES;          // 32 KB
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;           // 48 KB
+constexpr int B_BYTES = (HALF / BOX) * BOX_BYTES;        // 16 KB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;           // 32 KB per CTA
 constexpr int NUM_THREADS = 192;                         // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
 constexpr int TMEM_COLS = 2 * BN;                        // two accumulators
 constexpr size_t SMEM_BYTES = static_cast<size_t>(STAGES) * STAGE_BYTES + 1024 /*align*/ + 256;
+constexpr uint16_t PAIR = 0x3;                           // both CTAs of the cluster
+constexpr long long kPairDrainLimit = 1LL << 22;
+static_assert(SMEM_BYTES <= 232448, "shared memory");
 }  // namespace syrk
 
 struct SyrkParams {
@@ -171,25 +180,21 @@ struct SyrkParams {
     int64_t n, d;
     int groups;
     float alpha;
-    int nbi, nbk;        // row blocks of 128, column blocks of 256
-    int tiles_per_group;
+    int nb;              // blocks of 256 along i and k
+    int tiles_per_group; // nb (nb + 1) / 2: the blocks (bi, bk) with bi <= bk
     int num_tiles;
     DeviceErr err;
 };
 
-// Tile t of one group, ordered by column block then row block; only tiles that touch the upper
-// triangle (row block start <= column block end) exist.
+// Pair tile t of one group, ordered by column block then row block: (bi, bk) with bi <= bk.
 __device__ __forceinline__ void syrk_tile_coords(const SyrkParams &p, int tile, int &g, int &bi,
                                                  int &bk)
 {
     g = tile / p.tiles_per_group;
     int r = tile - g * p.tiles_per_group;
     bk = 0;
-    for (;;) {
-        int cnt = min(2 * bk + 2, p.nbi);
-        if (r < cnt)
-            break;
-        r -= cnt;
+    while (r > bk) {
+        r -= bk + 1;
         ++bk;
     }
     bi = r;
@@ -201,20 +206,23 @@ __global__ void __launch_bounds__(syrk::NUM_THREADS, 1)
                        const __grid_constant__ CUtensorMap bmap, SyrkParams p)
 {
     using namespace syrk;
-    constexpr uint32_t IDESC = umma_idesc_f16kind(BM, BN, /*a_mn_major=*/true,
+    constexpr uint32_t IDESC = umma_idesc_f16kind(PM, BN, /*a_mn_major=*/true,
                                                   /*b_mn_major=*/true, kF16);
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(align_up(reinterpret_cast<uintptr_t>(smem_raw), 1024));
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + STAGES * STAGE_BYTES);
-    uint64_t *full = bars;                  // [STAGES]
+    uint64_t *full = bars;                  // [STAGES] (the even CTA's counts both CTAs' bytes)
     uint64_t *empty = bars + STAGES;        // [STAGES]
     uint64_t *tfull = bars + 2 * STAGES;    // [2]
-    uint64_t *tempty = bars + 2 * STAGES + 2;  // [2]
+    uint64_t *tempty = bars + 2 * STAGES + 2;  // [2] (the even CTA's counts both epilogues)
     uint64_t *drain = bars + 2 * STAGES + 4;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 5);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    const uint32_t cr = cluster_ctarank();  // 0: issues the pair's MMAs; 1: its peer
+    const int pair = static_cast<int>(blockIdx.x >> 1);
+    const int npairs = static_cast<int>(gridDim.x >> 1);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -223,7 +231,7 @@ __global__ void __launch_bounds__(syrk::NUM_THREADS, 1)
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(&tfull[a], 1);
-            mbar_init(&tempty[a], 4 * 32);
+            mbar_init(&tempty[a], 2 * 4 * 32);   // the epilogues of both CTAs
         }
         mbar_init(drain, 1);
         fence_barrier_init();
@@ -231,9 +239,9 @@ __global__ void __launch_bounds__(syrk::NUM_THREADS, 1)
         tma_prefetch_desc(&bmap);
     }
     if (warp == 1)
-        tmem_alloc(tmem_holder, TMEM_COLS);
+        tmem_alloc_pair(tmem_holder, TMEM_COLS);
     tc_fence_before();
-    __syncthreads();
+    cluster_sync();  // barriers of both CTAs initialised, TMEM allocated in both
     tc_fence_after();
     const uint32_t tmem_base = *tmem_holder;
     const int nk = static_cast<int>((p.n + BK - 1) / BK);
@@ -241,53 +249,64 @@ __global__ void __launch_bounds__(syrk::NUM_THREADS, 1)
 
     if (warp == 0) {
         // ---------------------------------------------------------------- TMA producer
+        // Per stage: this CTA's 128 rows of A and its 128 of the tile's 256 columns of B_g, the
+        // bytes of both CTAs counted on the even CTA's barrier (armed there for both).
         if (lane == 0) {
-            int fills[STAGES];
-            for (int s = 0; s < STAGES; ++s)
-                fills[s] = 0;
+            uint32_t fpar = 0u, fused = 0u;  // per stage: parity of the fills, ever filled
             int stage = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
+            for (int tile = pair; tile < p.num_tiles && ok; tile += npairs) {
                 int g, bi, bk;
                 syrk_tile_coords(p, tile, g, bi, bk);
+                const int i0 = bi * PM + static_cast<int>(cr) * BM;
+                const int k0 = bk * BN + static_cast<int>(cr) * HALF;
                 for (int kb = 0; kb < nk; ++kb) {
-                    if (!mbar_wait(&empty[stage], (fills[stage] & 1) ^ 1, limit)) {
+                    if (!mbar_wait(&empty[stage], ((fpar >> stage) & 1u) ^ 1u, limit)) {
                         raise_error(p.err, kErrTimeout, 1);
                         ok = false;
                         break;
                     }
                     uint8_t *sa = smem + stage * STAGE_BYTES;
                     uint8_t *sb = sa + A_BYTES;
-                    mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
+                    if (cr == 0)
+                        mbar_arrive_expect_tx(&full[stage], 2 * STAGE_BYTES);
+                    const uint32_t fb = cluster_addr(&full[stage], 0);
                     const int t0 = kb * BK;
                     for (int b = 0; b < BM / BOX; ++b)
-                        tma_load_3d(sa + b * BOX_BYTES, &amap, &full[stage], bi * BM + b * BOX, t0, 0);
-                    for (int b = 0; b < BN / BOX; ++b)
-                        tma_load_3d(sb + b * BOX_BYTES, &bmap, &full[stage], bk * BN + b * BOX, t0, g);
-                    ++fills[stage];
+                        tma_load_3d_pair(sa + b * BOX_BYTES, &amap, fb, i0 + b * BOX, t0, 0);
+                    for (int b = 0; b < HALF / BOX; ++b)
+                        tma_load_3d_pair(sb + b * BOX_BYTES, &bmap, fb, k0 + b * BOX, t0, g);
+                    fpar ^= 1u << stage;
+                    fused |= 1u << stage;
                     stage = (stage + 1 == STAGES) ? 0 : stage + 1;
                 }
             }
             if (!ok) {
-                // Let every load already issued land before the CTA can exit.
-                for (int s = 0; s < STAGES; ++s)
-                    if (fills[s] > 0)
-                        mbar_wait(&full[s], (fills[s] - 1) & 1, kDrainLimit);
+                // let this CTA's copies land before the pair exits: the even CTA waits for the
+                // last phase of each stage it armed; the odd CTA's copies are counted there, so it
+                // waits a fixed time
+                if (cr == 0) {
+                    for (int s = 0; s < STAGES; ++s)
+                        if ((fused >> s) & 1u)
+                            mbar_wait(&full[s], ((fpar >> s) & 1u) ^ 1u, kPairDrainLimit);
+                } else {
+                    const long long c0 = clock64();
+                    while (clock64() - c0 < kPairDrainLimit) {
+                    }
+                }
             }
         }
     } else if (warp == 1) {
-        // ---------------------------------------------------------------- MMA issuer
-        if (lane == 0) {
-            int stage = 0, uses = 0;
-            uint32_t full_phase[STAGES];
-            for (int s = 0; s < STAGES; ++s)
-                full_phase[s] = 0;
+        // ---------------------------------------------------------------- MMA issuer (even CTA)
+        if (cr == 0 && lane == 0) {
+            int stage = 0;
+            uint32_t fph = 0u;  // per stage: phase parity
             bool ok = true;
             int it = 0;
-            for (int tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x, ++it) {
+            for (int tile = pair; tile < p.num_tiles && ok; tile += npairs, ++it) {
                 const int acc = it & 1;
                 const int use = it >> 1;
-                if (!mbar_wait(&tempty[acc], (use & 1) ^ 1, limit)) {
+                if (!mbar_wait_cluster(&tempty[acc], (use & 1) ^ 1, limit)) {
                     raise_error(p.err, kErrTimeout, 2);
                     ok = false;
                     break;
@@ -295,12 +314,12 @@ __global__ void __launch_bounds__(syrk::NUM_THREADS, 1)
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
                 for (int kb = 0; kb < nk; ++kb) {
-                    if (!mbar_wait(&full[stage], full_phase[stage], limit)) {
+                    if (!mbar_wait(&full[stage], (fph >> stage) & 1u, limit)) {
                         raise_error(p.err, kErrTimeout, 3);
                         ok = false;
                         break;
                     }
-                    full_phase[stage] ^= 1u;
+                    fph ^= 1u << stage;
                     tc_fence_after();
                     const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES);
                     const uint32_t sb = sa + A_BYTES;
@@ -309,26 +328,26 @@ __global__ void __launch_bounds__(syrk::NUM_THREADS, 1)
                         // 16 tokens = two 8-row groups of the 128-byte swizzle atom.
                         const uint64_t ad = umma_desc_sw128(sa + kk * 16 * 128, BOX_BYTES, 1024);
                         const uint64_t bd = umma_desc_sw128(sb + kk * 16 * 128, BOX_BYTES, 1024);
-                        umma_f16(d_tmem, ad, bd, IDESC, (kb | kk) != 0 ? 1u : 0u);
+                        umma_f16_pair(d_tmem, ad, bd, IDESC, (kb | kk) != 0 ? 1u : 0u);
                     }
-                    umma_commit(&empty[stage]);
+                    umma_commit_pair(&empty[stage], PAIR);
                     stage = (stage + 1 == STAGES) ? 0 : stage + 1;
                 }
                 if (!ok)
                     break;
-                umma_commit(&tfull[acc]);
-                ++uses;
+                umma_commit_pair(&tfull[acc], PAIR);
             }
             // Every MMA issued by this thread has completed once `drain` flips.
-            umma_commit(drain);
+            umma_commit_pair(drain, 0x1);
             mbar_wait(drain, 0, kDrainLimit);
         }
     } else {
         // ---------------------------------------------------------------- epilogue (warps 2-5)
         const int quarter = warp & 3;  // TMEM lanes this warp may access
-        const int row_in_tile = quarter * 32 + lane;
+        const int row_in_tile = static_cast<int>(cr) * BM + quarter * 32 + lane;
+        const uint32_t tempty_leader[2] = {cluster_addr(&tempty[0], 0), cluster_addr(&tempty[1], 0)};
         int it = 0;
-        for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++it) {
+        for (int tile = pair; tile < p.num_tiles; tile += npairs, ++it) {
             const int acc = it & 1;
             const int use = it >> 1;
             // One lane waits and the warp follows its verdict, so the warp-collective TMEM loads
@@ -349,7 +368,7 @@ __global__ void __launch_bounds__(syrk::NUM_THREADS, 1)
             float *Fg = p.F + static_cast<int64_t>(g) * p.d * p.d;
             const float scale =
                 p.pimax ? p.alpha * pow2_ceil(__uint_as_float(p.pimax[g])) : p.alpha;
-            const int64_t i = static_cast<int64_t>(bi) * BM + row_in_tile;
+            const int64_t i = static_cast<int64_t>(bi) * PM + row_in_tile;
             for (int chunk = 0; chunk < BN / 32; ++chunk) {
                 float v[32];
                 const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
@@ -383,15 +402,17 @@ __global__ void __launch_bounds__(syrk::NUM_THREADS, 1)
                 }
             }
             tc_fence_before();
-            mbar_arrive(&tempty[acc]);
+            mbar_arrive_cluster(tempty_leader[acc]);
         }
     }
 
+    // Both CTAs stay until the pair is done: the MMAs read both CTAs' shared memory and the
+    // copies and epilogues of both signal barriers in the even CTA.
     tc_fence_before();
-    __syncthreads();
+    cluster_sync();
     tc_fence_after();
     if (warp == 1)
-        tmem_dealloc(tmem_base, TMEM_COLS);
+        tmem_dealloc_pair(tmem_base, TMEM_COLS);
 }
 
 }  // namespace lnq
@@ -459,23 +480,46 @@ cudaError_t fisher_syrk(const void *A, const void *B, bool f16, const unsigned *
     p.d = d;
     p.groups = groups;
     p.alpha = alpha;
-    p.nbi = static_cast<int>((d + BM - 1) / BM);
-    p.nbk = static_cast<int>((d + BN - 1) / BN);
-    p.tiles_per_group = 0;
-    for (int bk = 0; bk < p.nbk; ++bk)
-        p.tiles_per_group += (2 * bk + 2 < p.nbi) ? 2 * bk + 2 : p.nbi;
+    p.nb = static_cast<int>((d + PM - 1) / PM);
+    p.tiles_per_group = p.nb * (p.nb + 1) / 2;
     p.num_tiles = p.tiles_per_group * groups;
     p.err = err;
-    const int grid = p.num_tiles < num_sms ? p.num_tiles : num_sms;
     auto kernel = f16 ? fisher_syrk_kernel<true> : fisher_syrk_kernel<false>;
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(SMEM_BYTES));
     if (e != cudaSuccess)
         return e;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.blockDim = dim3(NUM_THREADS);
+    cfg.dynamicSmemBytes = SMEM_BYTES;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    // persistent: as many pairs as can be resident at once (one CTA per SM)
+    static int resident[2] = {0, 0};
+    int &res = resident[f16 ? 1 : 0];
+    if (res == 0) {
+        cfg.gridDim = dim3(static_cast<unsigned>(num_sms & ~1));
+        int clusters = 0;
+        if (cudaOccupancyMaxActiveClusters(&clusters, kernel, &cfg) != cudaSuccess || clusters < 1)
+            clusters = num_sms / 2;
+        res = clusters;
+    }
+    int pairs = res < p.num_tiles ? res : p.num_tiles;
+    if (pairs < 1)
+        pairs = 1;
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
     {
         KernelTimer timer("fisher_syrk", s);
-        kernel<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(amap, bmap, p);
+        e = cudaLaunchKernelEx(&cfg, kernel, amap, bmap, p);
     }
+    if (e != cudaSuccess)
+        return e;
     return cudaGetLastError();
 }
 
