@@ -129,8 +129,8 @@ def algorithmic_work(layer, kernel: str, launches: int, moves_per_sweep: float):
     if kernel in ("lnq_operand_image", "lnq_residual_image"):
         # write the right-operand image (N columns x d coordinates x 2 bytes per row tile), read Q
         # and W once
-        rt = 256 // m if kernel == "lnq_operand_image" else 256 // 3
-        ncols = 256
+        rt = 256 // m if kernel == "lnq_operand_image" else 64
+        ncols = 256 if kernel == "lnq_operand_image" else 192
         tiles = g * -(-(dout // g) // rt)
         return tiles * ncols * (-(-d // 64) * 64) * 2.0 + 5.0 * dout * d, "byte"
     if kernel == "lnq_split_f16":

@@ -48,19 +48,23 @@ constexpr uint16_t PAIR = 0x3;                   // both CTAs of the cluster
 constexpr long long kPairDrainLimit = 1LL << 22;
 }  // namespace vg
 
-// Tile shapes. Both products take F as two fp16 pieces and the MMA is 256 columns wide. The
-// class-binned product (M > 0) has M one-hot columns per row and two TMEM accumulators that
-// alternate between tiles. The residual product (M == 0: three fp16 pieces of r per row) feeds the
-// objective, which sums r_i u_i with cancellation; there the K range is cut into two segments with
-// one accumulator each, so each fp32 accumulator takes half of the additions. Each CTA holds
+// Tile shapes. Both products take F as two fp16 pieces and the MMA is 256 columns wide, with two
+// TMEM accumulators that alternate between accumulation segments. The class-binned product
+// (M > 0, M one-hot columns per row) accumulates a whole tile in one segment. The residual product
+// (M == 0: three fp16 pieces of r per row) feeds the objective and the solve, where u = F r is
+// small against its terms: its segments are SEGK K blocks long and the epilogue adds each
+// finished segment into fp32 sums per row, so no tensor-core accumulation chain runs longer than
+// SEGK x 64 coordinates (the accumulator's rounding error grows with the chain). Each CTA holds
 // HALF = NCOLS / 2 rows of the right operand per stage.
 template <int M>
 struct VgShape {
     static constexpr int PIECES = 2;                    // fp16 pieces of F in the left operand
-    static constexpr int NCOLS = 256;                   // MMA N
+    // MMA N: 256, or 192 (64 rows of three pieces) for the residual product, whose epilogue keeps
+    // a running sum per row in registers
+    static constexpr int NCOLS = M > 0 ? 256 : 192;
     static constexpr int HALF = NCOLS / 2;              // right-operand rows held by one CTA
-    static constexpr int SEGS = 1;                      // K segments (one accumulator each)
-    static constexpr int SETS = 2;                      // accumulator sets (tile double-buffer)
+    static constexpr int SEGK = M > 0 ? 0 : 8;          // K blocks per segment (0: whole tile)
+    static constexpr int SETS = 2;                      // accumulators (segment double-buffer)
     static constexpr int RES = M > 0 ? 0 : 3;           // residual-piece columns per row
     static constexpr int RT = NCOLS / (M + RES);        // rows per tile
     static constexpr int ONEHOT = RT * M;               // one-hot columns
@@ -72,7 +76,7 @@ struct VgShape {
     static constexpr int A_SLOTS = A_FIT < 12 ? A_FIT : 12;
     static constexpr size_t SMEM = 1024 + static_cast<size_t>(A_SLOTS) * vg::A_TILE +
                                    vg::B_STAGES * B_BYTES + vg::BAR_BYTES;
-    static_assert(SETS * SEGS * NCOLS <= vg::TMEM_COLS, "TMEM holds 512 fp32 columns");
+    static_assert(SETS * NCOLS <= vg::TMEM_COLS, "TMEM holds 512 fp32 columns");
     static_assert(A_SLOTS >= 2 * PIECES, "at least two K blocks of F in flight");
     static_assert(A_SLOTS <= 32, "slot phases are kept in 32-bit masks");
     static_assert(SMEM <= vg::MAX_DYN_SMEM, "shared memory");
@@ -385,22 +389,26 @@ __global__ void __launch_bounds__(vg::NUM_THREADS, 1)
         // ---------------------------------------------------------------- MMA issue (even CTA)
         // Per K block: wait for both CTAs' right-operand halves, then for each piece wait for
         // both CTAs' F tiles, issue four K=16 MMAs (M = 256 over the pair) and release the slot
-        // in both CTAs; release the stage after the block, the accumulator after the tile.
+        // in both CTAs; release the stage after the block, the accumulator after the segment.
         if (cr == 0 && lane == 0) {
             int slot = 0, bstage = 0;
             uint32_t aph = 0u, bph = 0u;  // phase parity per slot / stage
             bool ok = true;
-            int itn = 0;
-            for (int tile = pair; tile < p.num_tiles && ok; tile += npairs, ++itn) {
-                const int acc = itn % S::SETS;
-                const int use = itn / S::SETS;
-                if (!mbar_wait_cluster(&tempty[acc], (use & 1) ^ 1, limit)) {
-                    raise_error(p.err, kErrTimeout, 13);
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
+            int itn = 0;  // segments issued: accumulator itn % SETS
+            const int segk = S::SEGK > 0 ? S::SEGK : nk;
+            for (int tile = pair; tile < p.num_tiles && ok; tile += npairs) {
+                int acc = 0;
                 for (int kb = 0; kb < nk && ok; ++kb) {
+                    const bool seg_start = kb % segk == 0;
+                    if (seg_start) {
+                        acc = itn % S::SETS;
+                        if (!mbar_wait_cluster(&tempty[acc], ((itn / S::SETS) & 1) ^ 1, limit)) {
+                            raise_error(p.err, kErrTimeout, 13);
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                    }
                     if (!mbar_wait(&b_full[bstage], (bph >> bstage) & 1u, limit)) {
                         raise_error(p.err, kErrTimeout, 14);
                         ok = false;
@@ -408,10 +416,7 @@ __global__ void __launch_bounds__(vg::NUM_THREADS, 1)
                     }
                     bph ^= 1u << bstage;
                     tc_fence_after();
-                    const int seg = (kb * S::SEGS) / nk;
-                    const bool seg_start = (kb == 0) || (((kb - 1) * S::SEGS) / nk != seg);
-                    const uint32_t d_tmem =
-                        tmem_base + static_cast<uint32_t>((acc * S::SEGS + seg) * S::NCOLS);
+                    const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * S::NCOLS);
                     const uint32_t sb = smem_u32(b_base + bstage * S::B_BYTES);
                     for (int pc = 0; pc < S::PIECES; ++pc) {
                         if (!mbar_wait(&a_full[slot], (aph >> slot) & 1u, limit)) {
@@ -437,10 +442,11 @@ __global__ void __launch_bounds__(vg::NUM_THREADS, 1)
                         break;
                     umma_commit_pair(&b_empty[bstage], PAIR);
                     bstage = (bstage + 1 == B_STAGES) ? 0 : bstage + 1;
+                    if (kb % segk == segk - 1 || kb + 1 == nk) {
+                        umma_commit_pair(&tfull[acc], PAIR);
+                        ++itn;
+                    }
                 }
-                if (!ok)
-                    break;
-                umma_commit_pair(&tfull[acc], PAIR);
             }
             umma_commit_pair(drain, 0x1);
             mbar_wait(drain, 0, kDrainLimit);
@@ -453,21 +459,11 @@ __global__ void __launch_bounds__(vg::NUM_THREADS, 1)
 #pragma unroll
         for (int a = 0; a < S::SETS; ++a)
             tempty_leader[a] = cluster_addr(&tempty[a], 0);
-        int itn = 0;
-        for (int tile = pair; tile < p.num_tiles; tile += npairs, ++itn) {
-            const int acc = itn % S::SETS;
-            const int use = itn / S::SETS;
-            int ok = 0;
-            if (lane == 0)
-                ok = mbar_wait(&tfull[acc], use & 1, limit) ? 1 : 0;
-            ok = __shfl_sync(0xffffffffu, ok, 0);
-            if (!ok) {
-                if (lane == 0)
-                    raise_error(p.err, kErrTimeout, 15);
-                break;
-            }
-            __syncwarp();
-            tc_fence_after();
+        int itn = 0;  // segments read: accumulator itn % SETS
+        const int segk = S::SEGK > 0 ? S::SEGK : nk;
+        const int nseg = (nk + segk - 1) / segk;
+        bool ok = true;
+        for (int tile = pair; tile < p.num_tiles && ok; tile += npairs) {
             int g, ip, rt_all;
             int64_t row0, row_end;
             vg_tile_coords<M>(p, tile, g, row0, row_end, ip, rt_all);
@@ -476,66 +472,81 @@ __global__ void __launch_bounds__(vg::NUM_THREADS, 1)
             // the accumulator carries 2^fexp[i] (and 2^rexp[j] on residual columns)
             const float inv_si =
                 pow2f(i < p.d ? -p.fexp[static_cast<int64_t>(g) * p.d + i] : 0);
-            // Chunks of 32 columns in order, each summed over the K segments that received a
-            // K block; a row's three residual columns are added as they come and its u is
-            // written at the third, so only one partial sum is live at a time.
-            float uacc = 0.f;
+            // residual product: per row, the sum over segments of its three piece columns
+            float uacc[M > 0 ? 1 : S::RT];
 #pragma unroll
-            for (int ch = 0; ch < S::CHUNKS; ++ch) {
-                float v[32];
-#pragma unroll
-                for (int seg = 0; seg < S::SEGS; ++seg) {
-                    // K block kb feeds segment kb * SEGS / nk; skip segments that received none
-                    const int first = (seg * nk + S::SEGS - 1) / S::SEGS;
-                    const bool fed = seg == 0 || (first < nk && (first * S::SEGS) / nk == seg);
-                    const uint32_t taddr =
-                        tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
-                        static_cast<uint32_t>((acc * S::SEGS + seg) * S::NCOLS + ch * 32);
-                    if (seg == 0) {
-                        tmem_ld_32x32b_x32(taddr, v);
-                    } else if (fed) {
-                        float w[32];
-                        tmem_ld_32x32b_x32(taddr, w);
-#pragma unroll
-                        for (int e = 0; e < 32; ++e)
-                            v[e] += w[e];
-                    }
+            for (int r = 0; r < (M > 0 ? 1 : S::RT); ++r)
+                uacc[r] = 0.f;
+            for (int sg = 0; sg < nseg; ++sg, ++itn) {
+                const int acc = itn % S::SETS;
+                int okw = 0;
+                if (lane == 0)
+                    okw = mbar_wait(&tfull[acc], (itn / S::SETS) & 1, limit) ? 1 : 0;
+                okw = __shfl_sync(0xffffffffu, okw, 0);
+                if (!okw) {
+                    if (lane == 0)
+                        raise_error(p.err, kErrTimeout, 15);
+                    ok = false;
+                    break;
                 }
+                __syncwarp();
+                tc_fence_after();
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const int col = ch * 32 + e;
-                    if constexpr (M > 0) {
-                        // M divides 32, so each row's M columns sit inside one chunk.
-                        if (col < S::ONEHOT && col % M == 0) {
-                            const int64_t j = row0 + col / M;
-                            if (j < row_end && i < p.d) {
-                                float *dst = p.V + (j * p.d + i) * M;
-                                if constexpr (M >= 4) {
+                for (int ch = 0; ch < S::CHUNKS; ++ch) {
+                    float v[32];
+                    tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
+                                           static_cast<uint32_t>(acc * S::NCOLS + ch * 32),
+                                       v);
 #pragma unroll
-                                    for (int b4 = 0; b4 < M / 4; ++b4)
-                                        reinterpret_cast<float4 *>(dst)[b4] = make_float4(
-                                            v[e + 4 * b4] * inv_si, v[e + 4 * b4 + 1] * inv_si,
-                                            v[e + 4 * b4 + 2] * inv_si, v[e + 4 * b4 + 3] * inv_si);
-                                } else {
-                                    *reinterpret_cast<float2 *>(dst) =
-                                        make_float2(v[e] * inv_si, v[e + 1] * inv_si);
+                    for (int e = 0; e < 32; ++e) {
+                        const int col = ch * 32 + e;
+                        if constexpr (M > 0) {
+                            // M divides 32, so each row's M columns sit inside one chunk.
+                            if (col < S::ONEHOT && col % M == 0) {
+                                const int64_t j = row0 + col / M;
+                                if (j < row_end && i < p.d) {
+                                    float *dst = p.V + (j * p.d + i) * M;
+                                    if constexpr (M >= 4) {
+#pragma unroll
+                                        for (int b4 = 0; b4 < M / 4; ++b4)
+                                            reinterpret_cast<float4 *>(dst)[b4] = make_float4(
+                                                v[e + 4 * b4] * inv_si, v[e + 4 * b4 + 1] * inv_si,
+                                                v[e + 4 * b4 + 2] * inv_si,
+                                                v[e + 4 * b4 + 3] * inv_si);
+                                    } else {
+                                        *reinterpret_cast<float2 *>(dst) =
+                                            make_float2(v[e] * inv_si, v[e + 1] * inv_si);
+                                    }
                                 }
                             }
+                        } else {
+                            if (col < S::USED)
+                                uacc[col / 3] += v[e];
                         }
                     }
-                    if (col >= S::ONEHOT && col < S::USED) {
-                        uacc += v[e];
-                        if ((col - S::ONEHOT) % 3 == 2) {
-                            const int64_t j = row0 + (col - S::ONEHOT) / 3;
-                            if (j < row_end && i < p.d)
-                                p.U[j * p.d + i] = (uacc * inv_si) * pow2f(-p.rexp[j]);
-                            uacc = 0.f;
-                        }
+                    if constexpr (M == 0) {
+                        // the chunk's sums are complete here, before the next chunk is loaded
+                        // (otherwise the additions may be deferred and every chunk kept live)
+#pragma unroll
+                        for (int r = (ch * 32) / 3; r <= (ch * 32 + 31) / 3 && r < S::RT; ++r)
+                            asm volatile("" : "+f"(uacc[r]));
+                    }
+                }
+                tc_fence_before();
+                mbar_arrive_cluster(tempty_leader[acc]);
+            }
+            if (!ok)
+                break;
+            if constexpr (M == 0) {
+                if (i < p.d) {
+#pragma unroll
+                    for (int r = 0; r < S::RT; ++r) {
+                        const int64_t j = row0 + r;
+                        if (j < row_end)
+                            p.U[j * p.d + i] = (uacc[r] * inv_si) * pow2f(-p.rexp[j]);
                     }
                 }
             }
-            tc_fence_before();
-            mbar_arrive_cluster(tempty_leader[acc]);
         }
     }
 

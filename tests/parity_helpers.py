@@ -57,13 +57,13 @@ def check_fisher_full(orc, F: torch.Tensor, X: torch.Tensor, G, groups: int, alp
 
 
 def check_fisher_sampled(orc, F: torch.Tensor, X: torch.Tensor, G, groups: int, alpha=1.0,
-                         tiles_per_group=8, tile=64, seed=0):
+                         tiles_per_group=8, tile=64, seed=0, check_groups=None):
     """Full diagonal plus random tiles (always including one on the diagonal and one touching the
-    last, possibly ragged, columns) of every group."""
+    last, possibly ragged, columns) of every group (or of the groups in check_groups)."""
     n, d = X.shape
     rng = np.random.default_rng(seed)
     worst = 0.0
-    for g in range(groups):
+    for g in (range(groups) if check_groups is None else check_groups):
         s = np.ones(n) if G is None else group_scales_oracle(orc, G, groups, g)
         diag = np.empty(d)
         for c0 in range(0, d, 512):

@@ -87,6 +87,24 @@ def test_fisher_q_proj_full_size_sampled(orc, lnq, wl):
     check_fisher_sampled(orc, F, X, G, layer.groups, tiles_per_group=6)
 
 
+def test_fisher_down_proj_full_size_sampled(orc, lnq, wl):
+    """Unguided layer at d_in = 11008 (all gradients 1, one group): F = X^T X."""
+    layer = wl.DOWN_PROJ
+    X, G, _ = wl.make_layer(layer, _dev())
+    assert G is None and layer.groups == 1
+    F = lnq.lnq_build_fisher(X, None, 1)
+    check_fisher_sampled(orc, F, X, None, 1, tiles_per_group=6)
+
+
+def test_fisher_up_proj_full_size_sampled(orc, lnq, wl):
+    """Eight guided groups over 65536 tokens; the first, a middle and the last group are sampled."""
+    layer = wl.UP_PROJ
+    X, G, _ = wl.make_layer(layer, _dev())
+    F = lnq.lnq_build_fisher(X, G, layer.groups)
+    check_fisher_sampled(orc, F, X, G, layer.groups, tiles_per_group=3,
+                         check_groups=[0, layer.groups // 2, layer.groups - 1])
+
+
 # --------------------------------------------------------------------------------- LNQ
 
 def test_lnq_tiny_layer_all_rows(orc, lnq, wl):
@@ -116,6 +134,26 @@ def test_lnq_q_proj_full_size_sampled_rows(orc, lnq, wl):
     F = lnq.lnq_build_fisher(X, G, layer.groups)
     del X, G
     summary, _, _ = lnq_follow_parity(orc, lnq, F, W, layer.m, layer.iters, rows_per_group=16)
+    assert summary["moves"] > 0
+
+
+def test_lnq_down_proj_full_size_sampled_rows(orc, lnq, wl):
+    """d_in = 11008 (86 sweep windows, a ragged last one), m = 8, four iterations, one group."""
+    layer = wl.DOWN_PROJ
+    X, G, W = wl.make_layer(layer, _dev())
+    F = lnq.lnq_build_fisher(X, G, layer.groups)
+    del X, G
+    summary, _, _ = lnq_follow_parity(orc, lnq, F, W, layer.m, layer.iters, rows_per_group=6)
+    assert summary["moves"] > 0
+
+
+def test_lnq_up_proj_full_size_sampled_rows(orc, lnq, wl):
+    """d_out = 14336 in eight groups of 1792 rows, m = 4, five iterations."""
+    layer = wl.UP_PROJ
+    X, G, W = wl.make_layer(layer, _dev())
+    F = lnq.lnq_build_fisher(X, G, layer.groups)
+    del X, G
+    summary, _, _ = lnq_follow_parity(orc, lnq, F, W, layer.m, layer.iters, rows_per_group=3)
     assert summary["moves"] > 0
 
 
