@@ -167,8 +167,8 @@ def hw_flop_factor(layer, kernel):
 # DRAM bytes per launch of the dominant kernel from an ncu capture (profiles/
 # dram_traffic_lnq_q_proj_rows1024.md: 1024 rows, scaled by 4 to the 4096-row launch), valid only
 # while the kernel's source is the one that was measured.
-TRAFFIC = {"lnq_vgemm": {"bytes": 4 * (1195870976 + 249111808), "source": "lnq_vgemm.cu",
-                         "sha256": "85ad6d8b573cd5a5146499e74fc90997c893e3b95eeff99e1d2fcbd0ed17a2d7"}}
+TRAFFIC = {"lnq_vgemm": {"bytes": 4 * (1180144128 + 247361792), "source": "lnq_vgemm.cu",
+                         "sha256": "3070c2b2c610055c2a1d961ac335f278bedf3bcbdca574213921413cbce03f49"}}
 
 
 def measured_traffic(kernel):
