@@ -24,8 +24,10 @@
 //     for a coordinate is the one nearest to t = w^_i - u_i / F_ii, found among the midpoints of
 //     the row's sorted codebook, and the coordinate moves only if its exact change is strictly
 //     negative; the block's later coordinates are corrected in registers from the 32 x 32 diagonal
-//     tile of F. Then the four sweep warps write the codes and moves and correct the window's
-//     later blocks in shared memory from a 32 x 128 strip of F (one TMA box per block).
+//     tile of F. The four sweep warps then add the block's moves to the next block's coordinates,
+//     and while warp 6 decides that block, warps 7-9 write the finished block's codes and moves,
+//     correct the window's later blocks in shared memory from a 32 x 128 strip of F (one TMA box
+//     per block) and start the copies for the block after.
 // Warp roles: 0 TMA and bulk copies, 1 MMA issue, 2-5 window assembly (TMEM -> shared memory),
 // 6-9 the sweep. Every wait is bounded; a wait that gives up sets the
 // workspace error flag and its role stops, and every role drains what it has in flight.
@@ -56,6 +58,8 @@ constexpr int SWEEP_THREADS = 128;
 constexpr int TMEM_COLS = 64;             // two fp32 accumulators of RB columns
 constexpr int MAX_WIN = 16384 / WIN;      // d_in <= 16384
 constexpr int SWEEP_BAR = 2;              // named barrier of the sweep warps
+constexpr int HELP_BAR = 3;               // named barrier of sweep warps 7-9
+constexpr int LEAD = 32;                  // sweep thread that issues the F strip copies
 
 // shared memory carve-up (bytes from a 1024-aligned base)
 constexpr int OFF_A = 0;
@@ -64,7 +68,7 @@ constexpr int OFF_BS = OFF_H + NH * H_CHUNK;
 constexpr int OFF_STRIP = OFF_BS + 2 * H_CHUNK;
 constexpr int OFF_UW = OFF_STRIP + 2 * BLK * WIN * 4;
 constexpr int OFF_DL = OFF_UW + 2 * RB * UW_LD * 4;
-constexpr int OFF_C = OFF_DL + BLK * RB * 4;
+constexpr int OFF_C = OFF_DL + 2 * BLK * RB * 4;      // moves: two blocks in flight
 constexpr int OFF_DC = OFF_C + RB * 17 * 4;
 constexpr int OFF_QB = OFF_DC + RB * 16 * 4;
 constexpr int OFF_WM = OFF_QB + 2 * RB * (BLK + 8);   // codes: two blocks in flight
@@ -73,8 +77,8 @@ constexpr int OFF_SRT = OFF_TS + 2 * RB * 4;               // [RB][17] sorted co
 constexpr int OFF_ORD = OFF_SRT + RB * 17 * 4;             // [RB][16] its codeword indices
 constexpr int OFF_FINV = OFF_ORD + RB * 16;                // [BLK] 1 / F_ii of the block
 constexpr int OFF_FDG = OFF_FINV + BLK * 4;                // [BLK] F_ii of the block
-constexpr int OFF_RM = OFF_FDG + BLK * 4;                  // [RB] moved-coordinate mask per row
-constexpr int OFF_BAR = OFF_RM + RB * 4;
+constexpr int OFF_RM = OFF_FDG + BLK * 4;                  // [2][RB] moved-coordinate mask per row
+constexpr int OFF_BAR = OFF_RM + 2 * RB * 4;
 constexpr int NBARS = 2 * NA + 2 * NH + 2 + 2 + 2 + 2 + 3 + 2;
 constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
 constexpr size_t SMEM = 1024 + OFF_MISC + 32;
@@ -112,7 +116,7 @@ __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
     uint8_t *bs_base = smem + OFF_BS;                                // [2 chunks][2][4 KB]
     float *strip = reinterpret_cast<float *>(smem + OFF_STRIP);      // [2][BLK][WIN]
     float *uwb = reinterpret_cast<float *>(smem + OFF_UW);           // [2][RB][UW_LD]
-    float(*dl_s)[RB] = reinterpret_cast<float(*)[RB]>(smem + OFF_DL);       // [BLK][RB]
+    float(*dl2)[BLK][RB] = reinterpret_cast<float(*)[BLK][RB]>(smem + OFF_DL);  // [2][BLK][RB] moves
     float(*c_s)[17] = reinterpret_cast<float(*)[17]>(smem + OFF_C);         // [RB][m]
     float(*dc_s)[16] = reinterpret_cast<float(*)[16]>(smem + OFF_DC);       // [RB][m]
     // [2][RB][BLK + 8] codes of the current and the next block, rows 8-byte aligned
@@ -124,7 +128,7 @@ __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
     uint8_t(*ord_s)[16] = reinterpret_cast<uint8_t(*)[16]>(smem + OFF_ORD);
     float *finv_s = reinterpret_cast<float *>(smem + OFF_FINV);
     float *fdg_s = reinterpret_cast<float *>(smem + OFF_FDG);
-    unsigned *rm_s = reinterpret_cast<unsigned *>(smem + OFF_RM);
+    unsigned(*rm2)[RB] = reinterpret_cast<unsigned(*)[RB]>(smem + OFF_RM);  // [2][RB]
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
     uint64_t *a_full = bars;
     uint64_t *a_empty = a_full + NA;
@@ -139,7 +143,8 @@ __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
     uint64_t *drain = bs_free + 1;
     uint64_t *strip_full = drain + 1;                                // [2] F strip buffers
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(smem + OFF_MISC);
-    volatile unsigned *moved_s = reinterpret_cast<volatile unsigned *>(smem + OFF_MISC + 16);  // [4]
+    // [2] per block: the OR of its rows' move masks
+    volatile unsigned *mv2 = reinterpret_cast<volatile unsigned *>(smem + OFF_MISC + 16);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -453,21 +458,21 @@ __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
         const bool vecF = (d & 3) == 0 && (reinterpret_cast<uintptr_t>(p.F) & 15u) == 0;
         uint32_t spar = 0u, sused = 0u;  // strip buffers: parity of TMA fills, ever filled
         // F rows b0..b0+31, columns wstart..wstart+127 of the group (zero outside F) -> strip buf:
-        // one TMA box (completing on strip_full[buf]) or, when F's rows are not 16-byte multiples,
-        // plain loads
-        auto load_strip = [&](int buf, int64_t b0, int64_t wstart) {
+        // one TMA box issued by thread LEAD (completing on strip_full[buf]) or, when F's rows are not
+        // 16-byte multiples, loads by the threads tid = 0 .. nthr-1 of the caller
+        auto load_strip = [&](int buf, int64_t b0, int64_t wstart, int tid, int nthr) {
             float *st = strip + buf * (BLK * WIN);
             if (p.strip_tma) {
-                if (t == 0) {
+                if (t == LEAD) {
                     fence_proxy_async_smem();
                     mbar_arrive_expect_tx(&strip_full[buf], BLK * WIN * 4);
                     tma_load_3d(st, &smap, &strip_full[buf], static_cast<int32_t>(wstart),
                                 static_cast<int32_t>(b0), g);
+                    spar ^= 1u << buf;
+                    sused |= 1u << buf;
                 }
-                spar ^= 1u << buf;
-                sused |= 1u << buf;
             } else if (vecF) {
-                for (int e = t; e < BLK * WIN / 4; e += SWEEP_THREADS) {
+                for (int e = tid; e < BLK * WIN / 4; e += nthr) {
                     const int r = e / (WIN / 4), c4 = e % (WIN / 4);
                     const int64_t row = b0 + r, col = wstart + 4 * c4;
                     float *dst = st + r * WIN + 4 * c4;
@@ -478,7 +483,7 @@ __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
                 }
                 cp_async_commit();
             } else {
-                for (int e = t; e < BLK * WIN; e += SWEEP_THREADS) {
+                for (int e = tid; e < BLK * WIN; e += nthr) {
                     const int r = e / WIN, c = e % WIN;
                     const int64_t row = b0 + r, col = wstart + c;
                     st[r * WIN + c] = (row < d && col < d) ? Fg[row * d + col] : 0.f;
@@ -487,28 +492,105 @@ __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
         };
         uint32_t wuses = 0u;  // bit per window buffer: phase parity
         int bi = 0;
-        // codes of this thread's row (r = t / 4) at coordinates k0 + 8 (t % 4) .. + 7 into code
-        // buffer buf: an asynchronous copy (completed with the block's F strip), plain loads at a
-        // ragged end, 0 outside the problem. Readers mask the classes.
+        // codes of row r at coordinates k0 + 8 s .. + 7 (task e = 4 r + s of the threads tid = 0 ..
+        // nthr-1) into code buffer buf: asynchronous copies (completed with the block's F strip),
+        // plain loads at a ragged end, 0 outside the problem. Readers mask the classes.
         const bool qvec = (d & 7) == 0 && (reinterpret_cast<uintptr_t>(p.Q) & 7u) == 0;
-        auto fetch_codes = [&](int buf, int64_t k0) {
-            const int r = t >> 2, s = t & 3;
-            const int64_t k = k0 + 8 * s;
-            uint8_t *dst = &qb2[buf][r][8 * s];
-            if (r < nrows && k < d && qvec && k + 8 <= d) {
-                cp_async8(dst, p.Q + (row0 + r) * d + k);
-            } else {
-                uint32_t w[2] = {0u, 0u};
-                if (r < nrows && k < d) {
-                    const uint8_t *src = p.Q + (row0 + r) * d + k;
+        auto fetch_codes = [&](int buf, int64_t k0, int tid, int nthr) {
+            for (int e = tid; e < RB * 4; e += nthr) {
+                const int r = e >> 2, s = e & 3;
+                const int64_t k = k0 + 8 * s;
+                uint8_t *dst = &qb2[buf][r][8 * s];
+                if (r < nrows && k < d && qvec && k + 8 <= d) {
+                    cp_async8(dst, p.Q + (row0 + r) * d + k);
+                } else {
+                    uint32_t w[2] = {0u, 0u};
+                    if (r < nrows && k < d) {
+                        const uint8_t *src = p.Q + (row0 + r) * d + k;
 #pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        if (k + e < d)
-                            w[e >> 2] |= static_cast<uint32_t>(src[e]) << (8 * (e & 3));
+                        for (int e2 = 0; e2 < 8; ++e2)
+                            if (k + e2 < d)
+                                w[e2 >> 2] |= static_cast<uint32_t>(src[e2]) << (8 * (e2 & 3));
+                    }
+                    *reinterpret_cast<uint2 *>(dst) = make_uint2(w[0], w[1]);
                 }
-                *reinterpret_cast<uint2 *>(dst) = make_uint2(w[0], w[1]);
             }
             cp_async_commit();
+        };
+        // The rest of decided block j (buffers jb, local index jlb, coordinates jb0 .. jb0+jnb-1)
+        // by the threads tid = 0 .. nthr-1: task (row r, sub s) writes the row's new codes (8 of
+        // them) and, for later windows, the Delta pieces in the K-major, 128-byte-swizzled operand
+        // (row r, K = 32 (jlb & 1) + k within chunk jlb >> 1, sub s: the 16-byte chunk of
+        // k = 8 s .. 8 s + 7); then, from kfrom on (kfrom < 0: none), the window's later
+        // coordinates get u[r][k] += sum_ii Delta[ii][r] F[jb0 + ii][wstart + k] (thread = row and
+        // 4 consecutive k, F read as a broadcast, ii in increasing order).
+        auto finish_block = [&](int jb, int jlb, int64_t jb0, int jnb, int tid, int nthr, int kfrom,
+                                int kend, float *uw, bool keep) {
+            uint8_t(*qj)[BLK + 8] = qb2[jb];
+            float(*dlj)[RB] = dl2[jb];
+            for (int e = tid; e < RB * 4; e += nthr) {
+                const int r = e >> 2, s = e & 3;
+                const int64_t jr = row0 + r;
+                if (r < nrows && rm2[jb][r] != 0u) {
+                    if (qvec && 8 * s + 8 <= jnb) {
+                        *reinterpret_cast<uint2 *>(p.Q + jr * d + jb0 + 8 * s) =
+                            *reinterpret_cast<const uint2 *>(&qj[r][8 * s]);
+                    } else {
+#pragma unroll
+                        for (int e2 = 0; e2 < 8; ++e2) {
+                            const int k = 8 * s + e2;
+                            if (k < jnb)
+                                p.Q[jr * d + jb0 + k] = qj[r][k];
+                        }
+                    }
+                }
+                if (keep) {
+                    uint32_t pk[DPIECES][4];
+                    const float sc = dsc[r];
+#pragma unroll
+                    for (int e2 = 0; e2 < 4; ++e2) {
+                        const float x0 = dlj[8 * s + 2 * e2][r] * sc;
+                        const float x1 = dlj[8 * s + 2 * e2 + 1][r] * sc;
+                        const __half a0 = __float2half_rn(x0), c0 = __float2half_rn(x1);
+                        const __half a1 = __float2half_rn(x0 - __half2float(a0));
+                        const __half c1 = __float2half_rn(x1 - __half2float(c0));
+                        pk[0][e2] = static_cast<uint32_t>(__half_as_ushort(a0)) |
+                                    (static_cast<uint32_t>(__half_as_ushort(c0)) << 16);
+                        pk[1][e2] = static_cast<uint32_t>(__half_as_ushort(a1)) |
+                                    (static_cast<uint32_t>(__half_as_ushort(c1)) << 16);
+                    }
+                    uint8_t *bs = bs_base + (jlb >> 1) * H_CHUNK + r * 128;
+                    const int chunk16 = (4 * (jlb & 1) + s) ^ (r & 7);
+#pragma unroll
+                    for (int pc = 0; pc < DPIECES; ++pc)
+                        *reinterpret_cast<uint4 *>(bs + pc * H_PIECE + chunk16 * 16) =
+                            make_uint4(pk[pc][0], pk[pc][1], pk[pc][2], pk[pc][3]);
+                }
+            }
+            const unsigned colmask = mv2[jb];
+            if (colmask != 0u && kfrom >= 0 && kfrom < kend) {
+                const int r = tid & 31, wq = tid >> 5, nw = nthr >> 5;
+                const float *stw = strip + jb * (BLK * WIN);
+                for (int k0 = kfrom + 4 * wq; k0 < kend; k0 += 4 * nw) {
+                    float a0 = uw[r * UW_LD + k0], a1 = uw[r * UW_LD + k0 + 1];
+                    float a2 = uw[r * UW_LD + k0 + 2], a3 = uw[r * UW_LD + k0 + 3];
+#pragma unroll 4
+                    for (int ii = 0; ii < BLK; ++ii) {
+                        if ((colmask >> ii) & 1u) {
+                            const float dr = dlj[ii][r];
+                            const float4 f = *reinterpret_cast<const float4 *>(stw + ii * WIN + k0);
+                            a0 = fmaf(dr, f.x, a0);
+                            a1 = fmaf(dr, f.y, a1);
+                            a2 = fmaf(dr, f.z, a2);
+                            a3 = fmaf(dr, f.w, a3);
+                        }
+                    }
+                    uw[r * UW_LD + k0] = a0;
+                    uw[r * UW_LD + k0 + 1] = a1;
+                    uw[r * UW_LD + k0 + 2] = a2;
+                    uw[r * UW_LD + k0 + 3] = a3;
+                }
+            }
         };
         constexpr uint32_t MASK4 = 0x01010101u * static_cast<uint32_t>(M - 1);
         // warp 6 (lane = row): the row's codebook sorted, equal values in index order, and the
@@ -531,8 +613,8 @@ __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
             for (int k = 0; k + 1 < M; ++k)
                 mid[k] = 0.5f * (srt_s[r][k] + srt_s[r][k + 1]);
         }
-        fetch_codes(0, 0);
-        load_strip(0, 0, 0);
+        fetch_codes(0, 0, t, SWEEP_THREADS);
+        load_strip(0, 0, 0, t, SWEEP_THREADS);
         bool failed = false;
         for (int T = 0; T < nwin; ++T) {
             const int64_t wstart = static_cast<int64_t>(T) * WIN;
@@ -549,31 +631,58 @@ __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
             wuses ^= 1u << buf;
             float *uw = uwb + buf * (RB * UW_LD);
             bool wmoved = false;
-            for (int lb = 0; lb < NBLK; ++lb, ++bi) {
+            const int kend = (d - wstart < WIN) ? static_cast<int>(d - wstart) : WIN;
+            const int nblk = (kend + BLK - 1) / BLK;  // blocks of this window
+            for (int lb = 0; lb < nblk; ++lb, ++bi) {
                 const int64_t b0 = wstart + lb * BLK;
-                if (b0 >= d)
-                    break;  // only in the last window
                 const int nb = (d - b0 < BLK) ? static_cast<int>(d - b0) : BLK;
+                const int cb = bi & 1;  // strip, code and move buffers of this block
                 int sok = 1;
                 if (p.strip_tma)
-                    sok = mbar_wait(&strip_full[bi & 1], (bi >> 1) & 1, limit) ? 1 : 0;
+                    sok = mbar_wait(&strip_full[cb], (bi >> 1) & 1, limit) ? 1 : 0;
                 cp_async_wait_all();
-                // strip and codes of this block complete
+                // strip and codes of this block complete, the previous block decided
                 if (!named_bar_and(SWEEP_BAR, SWEEP_THREADS, sok)) {
                     if (t == 0)
                         raise_error(p.err, kErrTimeout, 37);
                     failed = true;
                     break;
                 }
-                {
-                    const int64_t nb0 = b0 + BLK;
-                    if (nb0 < d) {
-                        fetch_codes((bi + 1) & 1, nb0);
-                        load_strip((bi + 1) & 1, nb0, lb + 1 < NBLK ? wstart : wstart + WIN);
+                if (lb > 0) {
+                    // the previous block's moves into this block's u (thread: row t % 32 and 8
+                    // coordinates; ii in increasing order, as for the later blocks)
+                    const int pb = cb ^ 1;
+                    const unsigned colmask = mv2[pb];
+                    if (colmask != 0u) {
+                        const int r = t & 31;
+                        const int kb = lb * BLK + 8 * (t >> 5);
+                        const float *stw = strip + pb * (BLK * WIN) + kb;
+                        float a[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            a[e] = uw[r * UW_LD + kb + e];
+#pragma unroll
+                        for (int ii = 0; ii < BLK; ++ii) {
+                            if ((colmask >> ii) & 1u) {
+                                const float dr = dl2[pb][ii][r];
+                                const float4 f0 = *reinterpret_cast<const float4 *>(stw + ii * WIN);
+                                const float4 f1 = *reinterpret_cast<const float4 *>(stw + ii * WIN + 4);
+                                a[0] = fmaf(dr, f0.x, a[0]);
+                                a[1] = fmaf(dr, f0.y, a[1]);
+                                a[2] = fmaf(dr, f0.z, a[2]);
+                                a[3] = fmaf(dr, f0.w, a[3]);
+                                a[4] = fmaf(dr, f1.x, a[4]);
+                                a[5] = fmaf(dr, f1.y, a[5]);
+                                a[6] = fmaf(dr, f1.z, a[6]);
+                                a[7] = fmaf(dr, f1.w, a[7]);
+                            }
+                        }
+#pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            uw[r * UW_LD + kb + e] = a[e];
                     }
                 }
-                uint8_t(*qb_s)[BLK + 8] = qb2[bi & 1];
-                const float *st = strip + (bi & 1) * (BLK * WIN) + lb * BLK;  // st[ii * WIN + c]
+                const float *st = strip + cb * (BLK * WIN) + lb * BLK;  // st[ii * WIN + c]
                 if (t < BLK) {
                     const float f = st[t * WIN + t];
                     fdg_s[t] = f;
@@ -589,6 +698,7 @@ __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
                     // t = -+inf, the extreme codeword, which is the best one for a linear change.)
                     const int r = lane;
                     const bool vr = r < nrows;
+                    uint8_t(*qb_s)[BLK + 8] = qb2[cb];
                     // registers hold the block's u and codes; each coordinate's current value is
                     // read and its move written in shared memory
                     float ub[BLK];
@@ -642,93 +752,37 @@ __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
                             if (4 * v + 2 > ii) ub[4 * v + 2] = fmaf(dlt, f4.z, ub[4 * v + 2]);
                             if (4 * v + 3 > ii) ub[4 * v + 3] = fmaf(dlt, f4.w, ub[4 * v + 3]);
                         }
-                        dl_s[ii][r] = dlt;
+                        dl2[cb][ii][r] = dlt;
                     }
 #pragma unroll
                     for (int v = 0; v < BLK / 4; ++v)
                         *reinterpret_cast<uint32_t *>(&qb_s[r][4 * v]) = qw[v];
-                    rm_s[r] = rowmask;
+                    rm2[cb][r] = rowmask;
                     const unsigned wm = __reduce_or_sync(0xffffffffu, rowmask);
                     if (lane == 0)
-                        moved_s[0] = wm;
-                }
-                named_bar_sync(SWEEP_BAR, SWEEP_THREADS);
-                {
-                    // thread (r, s): the row's new codes (8 of them) and, for later windows, the
-                    // Delta pieces in the K-major, 128-byte-swizzled operand: row r, K = 32 (lb & 1)
-                    // + k within chunk lb >> 1, sub s writes the 16-byte chunk of k = 8 s .. 8 s + 7
-                    const int r = t >> 2, s = t & 3;
-                    const int64_t jr = row0 + r;
-                    if (r < nrows && rm_s[r] != 0u) {
-                        if (qvec && 8 * s + 8 <= nb) {
-                            *reinterpret_cast<uint2 *>(p.Q + jr * d + b0 + 8 * s) =
-                                *reinterpret_cast<const uint2 *>(&qb_s[r][8 * s]);
-                        } else {
-#pragma unroll
-                            for (int e = 0; e < 8; ++e) {
-                                const int k = 8 * s + e;
-                                if (k < nb)
-                                    p.Q[jr * d + b0 + k] = qb_s[r][k];
-                            }
-                        }
-                    }
-                    if (keep) {
-                        uint32_t pk[DPIECES][4];
-                        const float sc = dsc[r];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float x0 = dl_s[8 * s + 2 * e][r] * sc;
-                            const float x1 = dl_s[8 * s + 2 * e + 1][r] * sc;
-                            const __half a0 = __float2half_rn(x0), c0 = __float2half_rn(x1);
-                            const __half a1 = __float2half_rn(x0 - __half2float(a0));
-                            const __half c1 = __float2half_rn(x1 - __half2float(c0));
-                            pk[0][e] = static_cast<uint32_t>(__half_as_ushort(a0)) |
-                                       (static_cast<uint32_t>(__half_as_ushort(c0)) << 16);
-                            pk[1][e] = static_cast<uint32_t>(__half_as_ushort(a1)) |
-                                       (static_cast<uint32_t>(__half_as_ushort(c1)) << 16);
-                        }
-                        uint8_t *bs = bs_base + (lb >> 1) * H_CHUNK + r * 128;
-                        const int chunk16 = (4 * (lb & 1) + s) ^ (r & 7);
-#pragma unroll
-                        for (int pc = 0; pc < DPIECES; ++pc)
-                            *reinterpret_cast<uint4 *>(bs + pc * H_PIECE + chunk16 * 16) =
-                                make_uint4(pk[pc][0], pk[pc][1], pk[pc][2], pk[pc][3]);
-                    }
-                }
-                const unsigned colmask = moved_s[0];
-
-                wmoved = wmoved || colmask != 0u;
-
-                const int kend = (d - wstart < WIN) ? static_cast<int>(d - wstart) : WIN;
-                if (colmask != 0u && (lb + 1) * BLK < kend) {
-                    // u[r][k] += sum_ii Delta[ii][r] F[b0 + ii][wstart + k] for the window's
-                    // later blocks; thread = (row, 4 consecutive k), F read as a broadcast
-                    const int r = t & 31, wq = t >> 5;
-                    const float *stw = strip + (bi & 1) * (BLK * WIN);
-                    float dr[BLK];
-#pragma unroll
-                    for (int ii = 0; ii < BLK; ++ii)
-                        dr[ii] = dl_s[ii][r];
-                    for (int k0 = (lb + 1) * BLK + 4 * wq; k0 < kend; k0 += 16) {
-                        float a0 = uw[r * UW_LD + k0], a1 = uw[r * UW_LD + k0 + 1];
-                        float a2 = uw[r * UW_LD + k0 + 2], a3 = uw[r * UW_LD + k0 + 3];
-#pragma unroll
-                        for (int ii = 0; ii < BLK; ++ii) {
-                            if ((colmask >> ii) & 1u) {
-                                const float4 f = *reinterpret_cast<const float4 *>(stw + ii * WIN + k0);
-                                a0 = fmaf(dr[ii], f.x, a0);
-                                a1 = fmaf(dr[ii], f.y, a1);
-                                a2 = fmaf(dr[ii], f.z, a2);
-                                a3 = fmaf(dr[ii], f.w, a3);
-                            }
-                        }
-                        uw[r * UW_LD + k0] = a0;
-                        uw[r * UW_LD + k0 + 1] = a1;
-                        uw[r * UW_LD + k0 + 2] = a2;
-                        uw[r * UW_LD + k0 + 3] = a3;
+                        mv2[cb] = wm;
+                } else {
+                    // warps 7-9 while the block is decided: the rest of the previous block of this
+                    // window (its codes, Delta pieces and the window's coordinates after this
+                    // block), then the next block's codes and strip into the buffers it freed
+                    const int ht = t - 32;
+                    if (lb > 0)
+                        finish_block(cb ^ 1, lb - 1, b0 - BLK, BLK, ht, SWEEP_THREADS - 32,
+                                     (lb + 1) * BLK, kend, uw, keep);
+                    named_bar_sync(HELP_BAR, SWEEP_THREADS - 32);
+                    const int64_t nb0 = b0 + BLK;
+                    if (nb0 < d) {
+                        fetch_codes(cb ^ 1, nb0, ht, SWEEP_THREADS - 32);
+                        load_strip(cb ^ 1, nb0, lb + 1 < NBLK ? wstart : wstart + WIN, ht,
+                                   SWEEP_THREADS - 32);
                     }
                 }
                 named_bar_sync(SWEEP_BAR, SWEEP_THREADS);
+                wmoved = wmoved || mv2[cb] != 0u;
+                // the window's last block is finished before the window ends (its Delta pieces
+                // feed the next windows' product)
+                if (lb + 1 == nblk)
+                    finish_block(cb, lb, b0, nb, t, SWEEP_THREADS, -1, kend, uw, keep);
             }
             if (failed)
                 break;
@@ -743,7 +797,7 @@ __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
         cp_async_wait_all();
         // after an early exit, let the strip copies in flight land (the last fill of buffer b
         // completes phase fills - 1)
-        if (p.strip_tma && t == 0)
+        if (p.strip_tma && t == LEAD)
             for (int b = 0; b < 2; ++b)
                 if ((sused >> b) & 1u)
                     mbar_wait(&strip_full[b], ((spar >> b) & 1u) ^ 1u, kDrainLimit);

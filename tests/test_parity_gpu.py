@@ -157,6 +157,24 @@ def test_lnq_up_proj_full_size_sampled_rows(orc, lnq, wl):
     assert summary["moves"] > 0
 
 
+@pytest.mark.parametrize("d_in", [100, 256, 300, 1000, 1500, 4096, 6000, 11008])
+def test_init_every_sort_width(orc, lnq, d_in):
+    """Init is bit-exact against the oracle for every sort layout: the shared-memory sort
+    (d_in < 256) and the register sort with 1 to 64 keys per thread (p2 / 256)."""
+    g = torch.Generator(device="cpu").manual_seed(d_in)
+    W = (torch.randn(12, d_in, generator=g) * 0.02)
+    W[:, : d_in // 5] = torch.round(W[:, : d_in // 5] * 200) / 200   # ties among the weights
+    for m in (4, 16):
+        C, Q = lnq.lnq_init_codebook(W.to(_dev()), m)
+        torch.cuda.synchronize()
+        Ch, Qh = C.double().cpu().numpy(), Q.cpu().numpy()
+        Wh = W.double().numpy()
+        for j in range(W.shape[0]):
+            c0, q0 = orc.init_row(Wh[j], m)
+            np.testing.assert_array_equal(Ch[j], c0.astype(np.float32).astype(np.float64))
+            np.testing.assert_array_equal(Qh[j], q0)
+
+
 @pytest.mark.parametrize("m", [2, 4, 8, 16])
 def test_lnq_every_codebook_size(orc, lnq, wl, m):
     layer = wl.scaled(wl.TINY, d_in=96, d_out=8, n=300, groups=2, m=m)
