@@ -237,6 +237,61 @@ __global__ void __launch_bounds__(256)
     }
 }
 
+// The one-hot image (M > 0) with one task per (row tile, row, 8 coordinates): the task reads its
+// 8 codes once and writes its row's M class columns (16 bytes each; a warp's 32 tasks cover 4
+// rows x 64 coordinates, so each class store fills 4 whole 128-byte rows of the image).
+template <int M>
+__global__ void __launch_bounds__(256)
+    onehot_image_kernel(const uint8_t *__restrict__ Q, int64_t d, int64_t rows_per_group,
+                        int row_tiles_per_group, int64_t ntasks, int nk, uint16_t *__restrict__ img)
+{
+    using S = VgShape<M>;
+    static_assert(M > 0 && S::ONEHOT == S::NCOLS, "one-hot columns fill the tile");
+    const bool vec = (d & 7) == 0 && (reinterpret_cast<uintptr_t>(Q) & 7u) == 0;
+    for (int64_t task = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; task < ntasks;
+         task += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int c = static_cast<int>(task & 7);
+        const int r = static_cast<int>((task >> 3) % S::RT);
+        const int64_t tb = (task >> 3) / S::RT;
+        const int kb = static_cast<int>(tb % nk);
+        const int rt_all = static_cast<int>(tb / nk);
+        const int g = rt_all / row_tiles_per_group;
+        const int rt = rt_all - g * row_tiles_per_group;
+        const int64_t gstart = static_cast<int64_t>(g) * rows_per_group;
+        const int64_t j = gstart + static_cast<int64_t>(rt) * S::RT + r;
+        const int64_t k0 = static_cast<int64_t>(kb) * 64 + 8 * c;
+        uint8_t qv[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+            qv[e] = 0xFFu;  // no class: outside the problem
+        if (j < gstart + rows_per_group && k0 < d) {
+            if (vec && k0 + 8 <= d) {
+                const uint2 q2 = *reinterpret_cast<const uint2 *>(Q + j * d + k0);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    qv[e] = static_cast<uint8_t>(q2.x >> (8 * e));
+                    qv[4 + e] = static_cast<uint8_t>(q2.y >> (8 * e));
+                }
+            } else {
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    if (k0 + e < d)
+                        qv[e] = Q[j * d + k0 + e];
+            }
+        }
+        uint16_t *dst = img + (tb * S::NCOLS + static_cast<int64_t>(r) * M) * 64 + 8 * c;
+#pragma unroll
+        for (int b = 0; b < M; ++b) {
+            uint32_t out[4];
+#pragma unroll
+            for (int h = 0; h < 4; ++h)
+                out[h] = (qv[2 * h] == b ? 0x3C00u : 0u) | ((qv[2 * h + 1] == b ? 0x3C00u : 0u) << 16);
+            *reinterpret_cast<uint4 *>(dst + static_cast<int64_t>(b) * 64) =
+                make_uint4(out[0], out[1], out[2], out[3]);
+        }
+    }
+}
+
 struct VgParams {
     const uint8_t *Q;   // [d_out][d]
     const float *W;     // [d_out][d]
@@ -650,9 +705,18 @@ static cudaError_t launch_vgemm_m(const CUtensorMap &map, VgParams p, uint16_t *
         int64_t blocks = num_rt_all * nk;
         if (blocks > static_cast<int64_t>(num_sms) * 16)
             blocks = static_cast<int64_t>(num_sms) * 16;
-        operand_image_kernel<M><<<static_cast<unsigned>(blocks), 256, 0, s>>>(
-            p.Q, p.W, p.C, p.rexp, p.d, p.rows_per_group, p.row_tiles_per_group,
-            static_cast<int>(num_rt_all), nk, p.m, img);
+        if constexpr (M > 0) {
+            const int64_t ntasks = num_rt_all * nk * S::RT * 8;
+            int64_t tblocks = (ntasks + 255) / 256;
+            if (tblocks > static_cast<int64_t>(num_sms) * 16)
+                tblocks = static_cast<int64_t>(num_sms) * 16;
+            onehot_image_kernel<M><<<static_cast<unsigned>(tblocks), 256, 0, s>>>(
+                p.Q, p.d, p.rows_per_group, p.row_tiles_per_group, ntasks, nk, img);
+        } else {
+            operand_image_kernel<M><<<static_cast<unsigned>(blocks), 256, 0, s>>>(
+                p.Q, p.W, p.C, p.rexp, p.d, p.rows_per_group, p.row_tiles_per_group,
+                static_cast<int>(num_rt_all), nk, p.m, img);
+        }
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess)
             return e;
