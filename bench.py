@@ -167,8 +167,8 @@ def hw_flop_factor(layer, kernel):
 # DRAM bytes per launch of the dominant kernel from an ncu capture (profiles/
 # dram_traffic_lnq_q_proj_rows1024.md: 1024 rows, scaled by 4 to the 4096-row launch), valid only
 # while the kernel's source is the one that was measured.
-TRAFFIC = {"lnq_vgemm": {"bytes": 4 * (1180144128 + 247361792), "source": "lnq_vgemm.cu",
-                         "sha256": "3070c2b2c610055c2a1d961ac335f278bedf3bcbdca574213921413cbce03f49"}}
+TRAFFIC = {"lnq_vgemm": {"bytes": 4 * (1205451008 + 250055168), "source": "lnq_vgemm.cu",
+                         "sha256": "85b8ca24e3b69b4a4da631df276300ca7d62cb5a9e4e0d90557304f37f301c31"}}
 
 
 def measured_traffic(kernel):

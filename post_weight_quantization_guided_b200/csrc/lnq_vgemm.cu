@@ -154,88 +154,7 @@ __global__ void __launch_bounds__(256)
 // [row tiles][K blocks][NCOLS][64]. Column n < ONEHOT of a row tile is the indicator of class n % M
 // for its row n / M; ONEHOT <= n < USED is residual piece (n - ONEHOT) % 3 of row (n - ONEHOT) / 3;
 // the rest is zero, as is everything outside the problem. All values are fp16, residuals scaled by
-// 2^rexp (C == nullptr: the zero codebook, r = -w).
-template <int M>
-__global__ void __launch_bounds__(256)
-    operand_image_kernel(const uint8_t *__restrict__ Q, const float *__restrict__ W,
-                         const float *__restrict__ C, const int32_t *__restrict__ rexp, int64_t d,
-                         int64_t rows_per_group, int row_tiles_per_group, int num_rt_all, int nk,
-                         int m, uint16_t *__restrict__ img)
-{
-    using S = VgShape<M>;
-    const bool vec = (d & 7) == 0 && (reinterpret_cast<uintptr_t>(Q) & 7u) == 0 &&
-                     (reinterpret_cast<uintptr_t>(W) & 15u) == 0;
-    // one (row tile, K block) per CTA iteration: NCOLS x 8 chunks of 16 bytes
-    const int ntb = num_rt_all * nk;
-    for (int tb = blockIdx.x; tb < ntb; tb += gridDim.x) {
-      const int kb = tb % nk;
-      const int rt_all = tb / nk;
-      const int g = rt_all / row_tiles_per_group;
-      const int rt = rt_all - g * row_tiles_per_group;
-      const int64_t gstart = static_cast<int64_t>(g) * rows_per_group;
-      const int64_t row0 = gstart + static_cast<int64_t>(rt) * S::RT;
-      const int64_t row_end = min(row0 + S::RT, gstart + rows_per_group);
-      for (int v = threadIdx.x; v < S::NCOLS * 8; v += blockDim.x) {
-        const int c = v & 7;
-        const int n = v >> 3;
-        const int64_t k0 = static_cast<int64_t>(kb) * 64 + 8 * c;
-        uint32_t out[4] = {0u, 0u, 0u, 0u};
-        if (n < S::USED) {
-            const bool onehot = n < S::ONEHOT;
-            const int r = onehot ? n / (M > 0 ? M : 1) : (n - S::ONEHOT) / 3;
-            const int64_t j = row0 + r;
-            if (j < row_end && k0 < d) {
-                uint8_t qv[8];
-                float wv[8];
-                if (vec && k0 + 8 <= d) {
-                    const uint2 q2 = *reinterpret_cast<const uint2 *>(Q + j * d + k0);
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        qv[e] = static_cast<uint8_t>(q2.x >> (8 * e));
-                        qv[4 + e] = static_cast<uint8_t>(q2.y >> (8 * e));
-                    }
-                    if (!onehot) {
-                        const float4 w0 = *reinterpret_cast<const float4 *>(W + j * d + k0);
-                        const float4 w1 = *reinterpret_cast<const float4 *>(W + j * d + k0 + 4);
-                        wv[0] = w0.x; wv[1] = w0.y; wv[2] = w0.z; wv[3] = w0.w;
-                        wv[4] = w1.x; wv[5] = w1.y; wv[6] = w1.z; wv[7] = w1.w;
-                    }
-                } else {
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const bool in = k0 + e < d;
-                        qv[e] = in ? Q[j * d + k0 + e] : 0xFFu;
-                        wv[e] = (in && !onehot) ? W[j * d + k0 + e] : 0.f;
-                    }
-                }
-                if (onehot) {
-                    constexpr uint16_t ONE = 0x3C00u;  // 1.0 in fp16
-                    const int b = n - r * (M > 0 ? M : 1);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        if (qv[e] == b)
-                            out[e >> 1] |= static_cast<uint32_t>(ONE) << (16 * (e & 1));
-                } else {
-                    const int pc = (n - S::ONEHOT) % 3;
-                    const float sc = pow2f(rexp[j]);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        if (qv[e] == 0xFFu)
-                            continue;
-                        const float rv = (C != nullptr ? C[j * m + (qv[e] & (m - 1))] : 0.f) - wv[e];
-                        uint16_t b0, b1, b2;
-                        split3_f16(rv * sc, b0, b1, b2);
-                        const uint16_t bits = pc == 0 ? b0 : (pc == 1 ? b1 : b2);
-                        out[e >> 1] |= static_cast<uint32_t>(bits) << (16 * (e & 1));
-                    }
-                }
-            }
-        }
-        *reinterpret_cast<uint4 *>(img + (static_cast<int64_t>(tb) * S::NCOLS + n) * 64 + 8 * c) =
-            make_uint4(out[0], out[1], out[2], out[3]);
-      }
-    }
-}
+// 2^rexp (C == nullptr: the zero codebook, r = -w). Two writers follow.
 
 // The one-hot image (M > 0) with one task per (row tile, row, 8 coordinates): the task reads its
 // 8 codes once and writes its row's M class columns (16 bytes each; a warp's 32 tasks cover 4
@@ -289,6 +208,75 @@ __global__ void __launch_bounds__(256)
             *reinterpret_cast<uint4 *>(dst + static_cast<int64_t>(b) * 64) =
                 make_uint4(out[0], out[1], out[2], out[3]);
         }
+    }
+}
+
+// The residual image (M == 0) with one task per (row tile, row, 8 coordinates): the task forms its
+// 8 residuals r = c[q] - w (C == nullptr: r = -w) once, scales them by 2^rexp of the row and
+// writes the row's three fp16 piece columns (16 bytes each).
+__global__ void __launch_bounds__(256)
+    residual_image_kernel(const uint8_t *__restrict__ Q, const float *__restrict__ W,
+                          const float *__restrict__ C, const int32_t *__restrict__ rexp, int64_t d,
+                          int64_t rows_per_group, int row_tiles_per_group, int64_t ntasks, int nk,
+                          int m, uint16_t *__restrict__ img)
+{
+    using S = VgShape<0>;
+    const bool vec = (d & 7) == 0 && (reinterpret_cast<uintptr_t>(Q) & 7u) == 0 &&
+                     (reinterpret_cast<uintptr_t>(W) & 15u) == 0;
+    for (int64_t task = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; task < ntasks;
+         task += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int c = static_cast<int>(task & 7);
+        const int r = static_cast<int>((task >> 3) % S::RT);
+        const int64_t tb = (task >> 3) / S::RT;
+        const int kb = static_cast<int>(tb % nk);
+        const int rt_all = static_cast<int>(tb / nk);
+        const int g = rt_all / row_tiles_per_group;
+        const int rt = rt_all - g * row_tiles_per_group;
+        const int64_t gstart = static_cast<int64_t>(g) * rows_per_group;
+        const int64_t j = gstart + static_cast<int64_t>(rt) * S::RT + r;
+        const int64_t k0 = static_cast<int64_t>(kb) * 64 + 8 * c;
+        uint32_t out[3][4] = {{0u, 0u, 0u, 0u}, {0u, 0u, 0u, 0u}, {0u, 0u, 0u, 0u}};
+        if (j < gstart + rows_per_group && k0 < d) {
+            uint8_t qv[8];
+            float wv[8];
+            if (vec && k0 + 8 <= d) {
+                const uint2 q2 = *reinterpret_cast<const uint2 *>(Q + j * d + k0);
+                const float4 w0 = *reinterpret_cast<const float4 *>(W + j * d + k0);
+                const float4 w1 = *reinterpret_cast<const float4 *>(W + j * d + k0 + 4);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    qv[e] = static_cast<uint8_t>(q2.x >> (8 * e));
+                    qv[4 + e] = static_cast<uint8_t>(q2.y >> (8 * e));
+                }
+                wv[0] = w0.x; wv[1] = w0.y; wv[2] = w0.z; wv[3] = w0.w;
+                wv[4] = w1.x; wv[5] = w1.y; wv[6] = w1.z; wv[7] = w1.w;
+            } else {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const bool in = k0 + e < d;
+                    qv[e] = in ? Q[j * d + k0 + e] : 0xFFu;
+                    wv[e] = in ? W[j * d + k0 + e] : 0.f;
+                }
+            }
+            const float sc = pow2f(rexp[j]);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                if (qv[e] == 0xFFu)
+                    continue;
+                const float rv = (C != nullptr ? C[j * m + (qv[e] & (m - 1))] : 0.f) - wv[e];
+                uint16_t b0, b1, b2;
+                split3_f16(rv * sc, b0, b1, b2);
+                const int sh = 16 * (e & 1);
+                out[0][e >> 1] |= static_cast<uint32_t>(b0) << sh;
+                out[1][e >> 1] |= static_cast<uint32_t>(b1) << sh;
+                out[2][e >> 1] |= static_cast<uint32_t>(b2) << sh;
+            }
+        }
+        uint16_t *dst = img + (tb * S::NCOLS + static_cast<int64_t>(r) * 3) * 64 + 8 * c;
+#pragma unroll
+        for (int pc = 0; pc < 3; ++pc)
+            *reinterpret_cast<uint4 *>(dst + static_cast<int64_t>(pc) * 64) =
+                make_uint4(out[pc][0], out[pc][1], out[pc][2], out[pc][3]);
     }
 }
 
@@ -702,20 +690,18 @@ static cudaError_t launch_vgemm_m(const CUtensorMap &map, VgParams p, uint16_t *
     p.num_tiles = static_cast<int>(num_rt_all * p.i_pairs);
     {
         KernelTimer timer(M > 0 ? "lnq_operand_image" : "lnq_residual_image", s);
-        int64_t blocks = num_rt_all * nk;
-        if (blocks > static_cast<int64_t>(num_sms) * 16)
-            blocks = static_cast<int64_t>(num_sms) * 16;
+        // one task per (row tile, row, 8 coordinates)
+        const int64_t ntasks = num_rt_all * nk * S::RT * 8;
+        int64_t tblocks = (ntasks + 255) / 256;
+        if (tblocks > static_cast<int64_t>(num_sms) * 16)
+            tblocks = static_cast<int64_t>(num_sms) * 16;
         if constexpr (M > 0) {
-            const int64_t ntasks = num_rt_all * nk * S::RT * 8;
-            int64_t tblocks = (ntasks + 255) / 256;
-            if (tblocks > static_cast<int64_t>(num_sms) * 16)
-                tblocks = static_cast<int64_t>(num_sms) * 16;
             onehot_image_kernel<M><<<static_cast<unsigned>(tblocks), 256, 0, s>>>(
                 p.Q, p.d, p.rows_per_group, p.row_tiles_per_group, ntasks, nk, img);
         } else {
-            operand_image_kernel<M><<<static_cast<unsigned>(blocks), 256, 0, s>>>(
-                p.Q, p.W, p.C, p.rexp, p.d, p.rows_per_group, p.row_tiles_per_group,
-                static_cast<int>(num_rt_all), nk, p.m, img);
+            residual_image_kernel<<<static_cast<unsigned>(tblocks), 256, 0, s>>>(
+                p.Q, p.W, p.C, p.rexp, p.d, p.rows_per_group, p.row_tiles_per_group, ntasks, nk,
+                p.m, img);
         }
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess)
