@@ -17,6 +17,11 @@
  *               for i = 1..d_in: assign coordinate i the codeword minimising (w^-w)^T H (w^-w) }.
  *   [GQ-abs]    aitopics "squeezellm" tag page, GuidedQuant abstract: the non-uniform scalar
  *               quantiser decreases its objective monotonically.
+ *   [LUT]       same post, LNQ section, last sentence (LNQ runs on the same CUDA kernel as
+ *               SqueezeLLM), with the aitopics "squeezellm" tag page, SqueezeLLM abstract
+ *               (single-batch inference is memory-bound; weights stored as low-bit indices) and
+ *               GANQ abstract (lookup-table based mixed-precision GEMM): the consumer of (C, Q)
+ *               multiplies activations by W^ = C[Q] read through each row's codebook.
  *
  * READINGS (the pages leave these open; each routine below states the one it takes):
  *   R1 groups are contiguous, equal slices of output rows; s_g is the plain mean of squared
@@ -29,6 +34,9 @@
  *      among equal best candidates take the lowest index; coordinates are visited in natural order.
  *   R5 codebook: solve over non-empty codewords only, empty codewords keep their value, no
  *      damping; a non-positive Cholesky pivot keeps the old codebook and flags the row singular.
+ *   R6 packed codes (the pages fix no format): bits = log2(m); each row is a run of 32-bit words
+ *      holding floor(32 / bits) codes each, code i of the row in word i / floor(32 / bits) at bit
+ *      (i mod floor(32 / bits)) * bits; unused high bits and the tail of the last word are zero.
  *
  * Build:  gcc -O2 -fopenmp -shared -fPIC lnq_oracle.c -o liblnq_oracle.so -lm
  */
@@ -386,4 +394,48 @@ void orc_follow_iteration(const double *F, int64_t d, const double *W, int64_t n
                       stats + 4 * j, NULL);
         J_out[j] = orc_objective_row(F, d, w, c, q);
     }
+}
+
+/* ------------------------------------------------------------------------------------------ */
+/* Packed codes and the lookup-table product [LUT], reading R6                                  */
+/* ------------------------------------------------------------------------------------------ */
+
+/* P[j*words + w] for rows j < d_out, words = ceil(d_in / floor(32 / bits)) (R6). */
+void orc_pack_codes(const uint8_t *Q, int64_t d_out, int64_t d_in, int bits, uint32_t *P)
+{
+    const int64_t per = 32 / bits;
+    const int64_t words = (d_in + per - 1) / per;
+    for (int64_t j = 0; j < d_out; ++j) {
+        for (int64_t w = 0; w < words; ++w)
+            P[j * words + w] = 0u;
+        for (int64_t i = 0; i < d_in; ++i) {
+            const uint32_t code = (uint32_t)Q[j * d_in + i];
+            P[j * words + i / per] |= code << ((i % per) * bits);
+        }
+    }
+}
+
+/* The inverse of orc_pack_codes. */
+void orc_unpack_codes(const uint32_t *P, int64_t d_out, int64_t d_in, int bits, uint8_t *Q)
+{
+    const int64_t per = 32 / bits;
+    const int64_t words = (d_in + per - 1) / per;
+    const uint32_t mask = (1u << bits) - 1u;
+    for (int64_t j = 0; j < d_out; ++j)
+        for (int64_t i = 0; i < d_in; ++i)
+            Q[j * d_in + i] = (uint8_t)((P[j * words + i / per] >> ((i % per) * bits)) & mask);
+}
+
+/* y[b*d_out + j] = sum_i x[b*d_in + i] * C[j*m + Q[j*d_in + i]] for b < nb: the activations times
+ * the quantised weights W^[j][i] = c_j[q_ji], read through each row's codebook [LUT]. */
+void orc_lut_gemv(const double *x, int64_t nb, const double *C, int m, const uint8_t *Q,
+                  int64_t d_out, int64_t d_in, double *y)
+{
+    for (int64_t b = 0; b < nb; ++b)
+        for (int64_t j = 0; j < d_out; ++j) {
+            double acc = 0.0;
+            for (int64_t i = 0; i < d_in; ++i)
+                acc += x[b * d_in + i] * C[j * m + Q[j * d_in + i]];
+            y[b * d_out + j] = acc;
+        }
 }

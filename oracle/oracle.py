@@ -58,6 +58,10 @@ def _bind(path: str):
     lib.orc_follow_iteration.argtypes = [_DP, _I64, _DP, _I64, ctypes.c_int, _DP, _U8P,
                                          _U8P, ctypes.c_double, _DP, _DP, _U8P, _DP, _I64P,
                                          _I32P, ctypes.c_int]
+    u32p = ctypes.POINTER(ctypes.c_uint32)
+    lib.orc_pack_codes.argtypes = [_U8P, _I64, _I64, ctypes.c_int, u32p]
+    lib.orc_unpack_codes.argtypes = [u32p, _I64, _I64, ctypes.c_int, _U8P]
+    lib.orc_lut_gemv.argtypes = [_DP, _I64, _DP, ctypes.c_int, _U8P, _I64, _I64, _DP]
     return lib
 
 
@@ -233,3 +237,41 @@ def follow_iteration(F, W, m: int, C_start, Q_start, Q_hint, tie_rel: float,
                                  _p(Q_out, _U8P), _p(J_out, _DP), _p(stats, _I64P),
                                  _p(status, _I32P), nthreads)
     return C_out, Q_out, J_out, stats, status
+
+
+_U32P = ctypes.POINTER(ctypes.c_uint32)
+
+
+def packed_words(d_in: int, bits: int) -> int:
+    """32-bit words per row of packed codes (reading R6 in lnq_oracle.c)."""
+    per = 32 // bits
+    return (d_in + per - 1) // per
+
+
+def pack_codes(Q, bits: int):
+    """Q [d_out][d_in] uint8 -> packed uint32 [d_out][packed_words(d_in, bits)]."""
+    Q = _u8(Q)
+    d_out, d_in = Q.shape
+    P = np.empty((d_out, packed_words(d_in, bits)), dtype=np.uint32)
+    _load().orc_pack_codes(_p(Q, _U8P), d_out, d_in, bits, _p(P, _U32P))
+    return P
+
+
+def unpack_codes(P, d_in: int, bits: int):
+    P = np.ascontiguousarray(P, dtype=np.uint32)
+    d_out = P.shape[0]
+    Q = np.empty((d_out, d_in), dtype=np.uint8)
+    _load().orc_unpack_codes(_p(P, _U32P), d_out, d_in, bits, _p(Q, _U8P))
+    return Q
+
+
+def lut_gemv(x, C, Q):
+    """y [nb][d_out] = x [nb][d_in] times W^ = C[Q] (rows of W^ are the output channels)."""
+    x, C, Q = _f64(x), _f64(C), _u8(Q)
+    if x.ndim == 1:
+        x = x[None, :]
+    nb, d_in = x.shape
+    d_out, m = C.shape
+    y = np.empty((nb, d_out), dtype=np.float64)
+    _load().orc_lut_gemv(_p(x, _DP), nb, _p(C, _DP), m, _p(Q, _U8P), d_out, d_in, _p(y, _DP))
+    return y
