@@ -400,6 +400,37 @@ def run_ours(args, rank, world, device):
     e2e_ms = e0.elapsed_time(e1)
     assert np.array_equal(Qp[(e2e_steps - 1) % 2].numpy(), Q.cpu().numpy())
 
+    # ---------------------------------------------------------------- consumer of (C, Q)
+    # The lookup-table GEMV on the step's codes (batch 1), outside the step's timed region: the
+    # packed codes are cycled through enough copies that they come from HBM, not L2.
+    bits = m.bit_length() - 1
+    Pk = lnq.lnq_pack_codes(Q, bits)
+    copies = max(2, int(3 * 126e6 / (Pk.numel() * 4)) + 1)
+    Ps = [Pk.clone() for _ in range(copies)]
+    xg = torch.randn(1, d, device=device, generator=torch.Generator(device=device).manual_seed(5))
+    yg = torch.empty(1, dout, device=device)
+    for k in range(4):
+        lnq.lnq_lut_gemv(xg, Ps[k % copies], C, d, y=yg)
+    torch.cuda.synchronize(device)
+    # one CUDA graph of `copies` calls, so the timing sees the device, not the host's call rate
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for k in range(copies):
+            lnq.lnq_lut_gemv(xg, Ps[k], C, d, y=yg)
+    graph.replay()
+    torch.cuda.synchronize(device)
+    replays = 10
+    g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    g0.record(stream)
+    for _ in range(replays):
+        graph.replay()
+    g1.record(stream)
+    torch.cuda.synchronize(device)
+    lut_us = g0.elapsed_time(g1) * 1e3 / (replays * copies)
+    del graph
+    lut_bytes = Pk.numel() * 4 + C.numel() * 4 + d * 4 + dout * 4
+    del Ps
+
     # ---------------------------------------------------------------- max over ranks
     total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], world, device)
 
@@ -449,6 +480,12 @@ def run_ours(args, rank, world, device):
         if fisher_ms else None,
         "kernels": kernels,
         "clocks": clocks,
+        # the consumer of (C, Q): y = x W^T read through the codebooks from the packed codes
+        "lut_gemv": {"workload": f"{layer.name}: {bits}-bit packed codes, batch 1",
+                     "us_per_call": lut_us, "algorithmic_bytes": lut_bytes,
+                     "achieved_gbs": lut_bytes / (lut_us * 1e-6) / 1e9,
+                     "peak_gbs": peaks["hbm_gbs"],
+                     "frac": lut_bytes / (lut_us * 1e-6) / 1e9 / peaks["hbm_gbs"]},
     }
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(layer, X, G, W, F, budget_s=args.cpu_budget)

@@ -156,6 +156,36 @@ LNQ_API lnq_status lnq_objective(const float *F, int groups, const float *W, con
  * gives up. Returns LNQ_OK, LNQ_ERR_TIMEOUT or LNQ_ERR_CUDA. */
 LNQ_API lnq_status lnq_workspace_check(void *ws, lnq_stream_t stream);
 
+/* ---- Consumer of (C, Q): packed codes and the lookup-table GEMV ----------------------------
+ * "GuidedQuant" (jinukkim.me blog), LNQ section, last sentence (LNQ runs on SqueezeLLM's CUDA
+ * kernel); aitopics "squeezellm" tag page, SqueezeLLM and GANQ abstracts (single-batch inference
+ * is memory-bound; weights as low-bit indices into a lookup table).
+ * Packed format (the pages fix none): bits = log2(m) in {1, 2, 3, 4}; row j is a run of
+ * lnq_packed_words(d_in, bits) 32-bit words of floor(32 / bits) codes each, code i in word
+ * i / floor(32 / bits) at bit (i mod floor(32 / bits)) * bits, unused bits zero. */
+
+/* 32-bit words per packed row (0 if bits is not in 1..4 or d_in < 1). */
+LNQ_API int64_t lnq_packed_words(int64_t d_in, int bits);
+
+/* Packs Q [d_out][d_in] uint8 (device, codes < 2^bits; higher bits are dropped) into
+ * P [d_out][lnq_packed_words(d_in, bits)] uint32 (device, caller-owned).
+ * Requirements: bits in 1..4, d_out >= 1, d_in >= 1, non-NULL pointers; otherwise
+ * LNQ_ERR_INVALID_ARG. */
+LNQ_API lnq_status lnq_pack_codes(const uint8_t *Q, int64_t d_out, int64_t d_in, int bits,
+                                  uint32_t *P, lnq_stream_t stream);
+
+/* y[b][j] = sum_i x[b][i] * C[j][code(j, i)] for b < nb: nb activation vectors times the
+ * quantised weights W^ = C[Q], read from the packed codes.
+ *   x [nb][d_in] fp32, P packed as above, C [d_out][2^bits] fp32, y [nb][d_out] fp32 out; all
+ *   device memory, caller-owned.
+ * Arithmetic: fp32 products and sums (each lane sums its words in order, then a fixed-order warp
+ * tree), so results are bit-identical from run to run.
+ * Requirements: bits in 1..4, 1 <= nb <= 8, d_out >= 1, d_in >= 1, non-NULL pointers; otherwise
+ * LNQ_ERR_INVALID_ARG. */
+LNQ_API lnq_status lnq_lut_gemv(const float *x, int64_t nb, const uint32_t *P, const float *C,
+                                int64_t d_out, int64_t d_in, int bits, float *y,
+                                lnq_stream_t stream);
+
 /* Testing knob: upper bound, in SM clock cycles, on every in-kernel wait of later calls from this
  * process (0 makes every wait give up at once). A negative value restores the default of about
  * 2^31 cycles, roughly a second. */

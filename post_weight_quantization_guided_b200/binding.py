@@ -22,7 +22,8 @@ LNQ_OP_BUILD_FISHER, LNQ_OP_INIT_CODEBOOK, LNQ_OP_QUANTIZE_ROWS, LNQ_OP_OBJECTIV
 
 EXPORTED = ("lnq_workspace_size", "lnq_build_fisher", "lnq_init_codebook", "lnq_quantize_rows",
             "lnq_objective", "lnq_workspace_check", "lnq_set_wait_limit", "lnq_status_string",
-            "lnq_profile_enable", "lnq_profile_read", "lnq_build_fisher_noalloc")
+            "lnq_profile_enable", "lnq_profile_read", "lnq_build_fisher_noalloc",
+            "lnq_packed_words", "lnq_pack_codes", "lnq_lut_gemv")
 
 _lib = None
 _VP, _I64, _INT, _SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
@@ -63,9 +64,13 @@ def lib():
         L.lnq_profile_read.restype = _INT
         L.lnq_status_string.argtypes = [_INT]
         L.lnq_status_string.restype = ctypes.c_char_p
+        L.lnq_packed_words.argtypes = [_I64, _INT]
+        L.lnq_packed_words.restype = _I64
+        L.lnq_pack_codes.argtypes = [_VP, _I64, _I64, _INT, _VP, _VP]
+        L.lnq_lut_gemv.argtypes = [_VP, _I64, _VP, _VP, _I64, _I64, _INT, _VP, _VP]
         for name in ("lnq_build_fisher", "lnq_build_fisher_noalloc", "lnq_init_codebook",
-                     "lnq_quantize_rows",
-                     "lnq_objective", "lnq_workspace_check"):
+                     "lnq_quantize_rows", "lnq_objective", "lnq_workspace_check",
+                     "lnq_pack_codes", "lnq_lut_gemv"):
             getattr(L, name).restype = _INT
         _lib = L
     return _lib
@@ -221,3 +226,41 @@ def lnq_objective(F: torch.Tensor, W: torch.Tensor, C: torch.Tensor, Q: torch.Te
 def lnq_workspace_check(ws: torch.Tensor, stream=None) -> int:
     """Synchronises the stream and returns LNQ_OK or LNQ_ERR_TIMEOUT (see include/lnq.h)."""
     return int(lib().lnq_workspace_check(_ptr(ws), _stream(stream)))
+
+
+def lnq_packed_words(d_in: int, bits: int) -> int:
+    """32-bit words per packed row (see include/lnq.h)."""
+    return int(lib().lnq_packed_words(int(d_in), int(bits)))
+
+
+def lnq_pack_codes(Q: torch.Tensor, bits: int, P: Optional[torch.Tensor] = None,
+                   stream=None) -> torch.Tensor:
+    """Q [d_out][d_in] uint8 -> packed int32 words [d_out][lnq_packed_words(d_in, bits)]."""
+    d_out, d_in = Q.shape
+    _need(Q, torch.uint8, (d_out, d_in), "Q")
+    words = lnq_packed_words(d_in, bits)
+    if P is None:
+        P = torch.empty((d_out, words), dtype=torch.int32, device=Q.device)
+    _need(P, torch.int32, (d_out, words), "P")
+    _check(lib().lnq_pack_codes(_ptr(Q), d_out, d_in, int(bits), _ptr(P), _stream(stream)),
+           "lnq_pack_codes")
+    return P
+
+
+def lnq_lut_gemv(x: torch.Tensor, P: torch.Tensor, C: torch.Tensor, d_in: int,
+                 y: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """y [nb][d_out] = x [nb][d_in] times W^ = C[codes] (packed codes P, codebooks C [d_out][m])."""
+    d_out, m = C.shape
+    bits = m.bit_length() - 1
+    if x.dim() == 1:
+        x = x.view(1, -1)
+    nb = x.shape[0]
+    _need(x, torch.float32, (nb, d_in), "x")
+    _need(C, torch.float32, (d_out, m), "C")
+    _need(P, torch.int32, (d_out, lnq_packed_words(d_in, bits)), "P")
+    if y is None:
+        y = torch.empty((nb, d_out), dtype=torch.float32, device=x.device)
+    _need(y, torch.float32, (nb, d_out), "y")
+    _check(lib().lnq_lut_gemv(_ptr(x), nb, _ptr(P), _ptr(C), d_out, int(d_in), bits, _ptr(y),
+                              _stream(stream)), "lnq_lut_gemv")
+    return y

@@ -270,6 +270,37 @@ lnq_status lnq_objective(const float *F, int groups, const float *W, const float
                : LNQ_ERR_CUDA;
 }
 
+int64_t lnq_packed_words(int64_t d_in, int bits)
+{
+    if (bits < 1 || bits > 4 || d_in < 1)
+        return 0;
+    return lnq_lut_words(d_in, bits);
+}
+
+lnq_status lnq_pack_codes(const uint8_t *Q, int64_t d_out, int64_t d_in, int bits, uint32_t *P,
+                          lnq_stream_t stream)
+{
+    if (Q == nullptr || P == nullptr || bits < 1 || bits > 4 || d_out < 1 || d_in < 1)
+        return LNQ_ERR_INVALID_ARG;
+    return lnq_pack_launch(Q, d_out, d_in, bits, P, device_sm_count(),
+                           reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? LNQ_OK
+               : LNQ_ERR_CUDA;
+}
+
+lnq_status lnq_lut_gemv(const float *x, int64_t nb, const uint32_t *P, const float *C,
+                        int64_t d_out, int64_t d_in, int bits, float *y, lnq_stream_t stream)
+{
+    if (x == nullptr || P == nullptr || C == nullptr || y == nullptr || bits < 1 || bits > 4 ||
+        nb < 1 || nb > 8 || d_out < 1 || d_in < 1)
+        return LNQ_ERR_INVALID_ARG;
+    return lnq_lut_gemv_launch(x, static_cast<int>(nb), P, C, d_out, d_in, bits, y,
+                               device_sm_count(), reinterpret_cast<cudaStream_t>(stream)) ==
+                   cudaSuccess
+               ? LNQ_OK
+               : LNQ_ERR_CUDA;
+}
+
 lnq_status lnq_workspace_check(void *ws, lnq_stream_t stream)
 {
     if (ws == nullptr)

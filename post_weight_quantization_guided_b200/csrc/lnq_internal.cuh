@@ -59,4 +59,12 @@ cudaError_t lnq_sweep(const float *F, const __half *Fh, const int32_t *fexp, int
                       const float *V, const float *dC, const float *U, const float *C, uint8_t *Q,
                       uint8_t *hist, int64_t d, int64_t d_out, int m, DeviceErr err, cudaStream_t s);
 
+// lut.cu
+int64_t lnq_lut_words(int64_t d_in, int bits);
+cudaError_t lnq_pack_launch(const uint8_t *Q, int64_t d_out, int64_t d_in, int bits, uint32_t *P,
+                            int num_sms, cudaStream_t s);
+cudaError_t lnq_lut_gemv_launch(const float *x, int nb, const uint32_t *P, const float *C,
+                                int64_t d_out, int64_t d_in, int bits, float *y, int num_sms,
+                                cudaStream_t s);
+
 }  // namespace lnq

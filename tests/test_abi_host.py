@@ -29,7 +29,17 @@ def test_header_declares_the_entry_points():
     assert names == sorted(["lnq_build_fisher", "lnq_init_codebook", "lnq_objective",
                             "lnq_quantize_rows", "lnq_set_wait_limit", "lnq_status_string",
                             "lnq_workspace_check", "lnq_workspace_size", "lnq_profile_enable",
-                            "lnq_profile_read", "lnq_build_fisher_noalloc"])
+                            "lnq_profile_read", "lnq_build_fisher_noalloc", "lnq_packed_words",
+                            "lnq_pack_codes", "lnq_lut_gemv"])
+
+
+def test_packed_words_and_argument_checks(L):
+    """Host-side rules of the packed format and the consumer entry points (no GPU needed)."""
+    assert [L.lnq_packed_words(4096, b) for b in (1, 2, 3, 4)] == [128, 256, 410, 512]
+    assert L.lnq_packed_words(0, 4) == 0 and L.lnq_packed_words(10, 5) == 0
+    bad = 1  # LNQ_ERR_INVALID_ARG, returned before any device work
+    assert L.lnq_pack_codes(None, 4, 4, 4, None, None) == bad
+    assert L.lnq_lut_gemv(None, 1, None, None, 4, 4, 4, None, None) == bad
 
 
 def test_library_exports_every_declared_symbol(L):

@@ -277,3 +277,50 @@ def test_wait_limit_zero_reports_timeout_and_recovers(lnq, wl):
     F2 = lnq.lnq_build_fisher(X, G, layer.groups)
     torch.cuda.synchronize()
     assert torch.equal(F, F2)
+
+
+# --------------------------------------------------------------------------------- consumer
+
+@pytest.mark.parametrize("bits", [1, 2, 3, 4])
+@pytest.mark.parametrize("d_out,d_in,nb", [(37, 1, 1), (64, 100, 3), (130, 1027, 8),
+                                           (4096, 4096, 1)])
+def test_lut_pack_and_gemv(orc, lnq, bits, d_out, d_in, nb):
+    """Packed words bit-exact against the oracle's packing; y = x W^T within 1e-5 of
+    sum_i |x_i c_q| (fp32 sums of at most ~130 terms per lane, then a 5-level tree); bit-identical
+    on a second run."""
+    m = 1 << bits
+    g = torch.Generator().manual_seed(bits * 7919 + d_in)
+    Q = torch.randint(0, m, (d_out, d_in), generator=g, dtype=torch.uint8)
+    C = torch.randn(d_out, m, generator=g)
+    x = torch.randn(nb, d_in, generator=g)
+    P = lnq.lnq_pack_codes(Q.to(_dev()), bits)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(P.cpu().numpy().view(np.uint32), orc.pack_codes(Q.numpy(), bits))
+    y = lnq.lnq_lut_gemv(x.to(_dev()), P, C.to(_dev()), d_in)
+    y2 = lnq.lnq_lut_gemv(x.to(_dev()), P, C.to(_dev()), d_in)
+    torch.cuda.synchronize()
+    assert torch.equal(y, y2)
+    Qn, Cn, xn = Q.numpy(), C.double().numpy(), x.double().numpy()
+    yo = orc.lut_gemv(xn, Cn, Qn)
+    W_hat = np.take_along_axis(Cn, Qn.astype(np.int64), axis=1)
+    scale = np.abs(xn) @ np.abs(W_hat).T
+    err = np.abs(y.double().cpu().numpy() - yo)
+    assert np.all(err <= 1e-5 * scale + 1e-30), float((err / (scale + 1e-30)).max())
+
+
+def test_lut_gemv_on_a_quantised_layer(orc, lnq, wl):
+    """The consumer on the tiny layer's own LNQ result (C, Q after three iterations)."""
+    layer = wl.TINY
+    X, G, W = wl.make_layer(layer, _dev())
+    F = lnq.lnq_build_fisher(X, G, layer.groups)
+    C, Q = lnq.lnq_init_codebook(W, layer.m)
+    lnq.lnq_quantize_rows(F, W, layer.m, layer.iters, C, Q)
+    bits = layer.m.bit_length() - 1
+    P = lnq.lnq_pack_codes(Q, bits)
+    y = lnq.lnq_lut_gemv(X[:5].float().contiguous(), P, C, layer.d_in)
+    torch.cuda.synchronize()
+    xn = X[:5].double().cpu().numpy()
+    yo = orc.lut_gemv(xn, C.double().cpu().numpy(), Q.cpu().numpy())
+    W_hat = np.take_along_axis(C.double().cpu().numpy(), Q.cpu().numpy().astype(np.int64), axis=1)
+    scale = np.abs(xn) @ np.abs(W_hat).T
+    assert np.all(np.abs(y.double().cpu().numpy() - yo) <= 1e-5 * scale + 1e-30)
