@@ -6,6 +6,9 @@ builds the guided Fisher blocks, initialises the codebooks and runs `--iters` LN
 the objective on a named synthetic workload, optionally with fewer output rows (`--rows`, a
 multiple of the group count) so that a capture stays small. It prints the objective's sum so that
 a run can be checked to have completed.
+
+With `--lut N` it then packs the codes and runs the lookup-table GEMV N times on one activation
+vector (the codes cycled through enough copies that they come from HBM).
 """
 from __future__ import annotations
 
@@ -24,6 +27,7 @@ def main(argv=None) -> None:
     ap.add_argument("--workload", default="q_proj", choices=sorted(WORKLOADS))
     ap.add_argument("--rows", type=int, default=0, help="output rows (default: the workload's)")
     ap.add_argument("--iters", type=int, default=1)
+    ap.add_argument("--lut", type=int, default=0, help="lookup-table GEMV calls after the run")
     args = ap.parse_args(argv)
     layer = WORKLOADS[args.workload]
     if args.rows:
@@ -39,6 +43,16 @@ def main(argv=None) -> None:
     api.lnq_quantize_rows(F, W, layer.m, args.iters, C, Q, J, st)
     torch.cuda.synchronize()
     print(f"{layer.name} rows={layer.d_out} iters={args.iters} sum(J)={float(J.sum()):.6e}")
+    if args.lut:
+        bits = layer.m.bit_length() - 1
+        P = api.lnq_pack_codes(Q, bits)
+        Ps = [P.clone() for _ in range(max(2, int(3 * 126e6 / (P.numel() * 4)) + 1))]
+        x = torch.randn(1, layer.d_in, device=dev, generator=torch.Generator(device=dev).manual_seed(5))
+        y = torch.empty(1, layer.d_out, device=dev)
+        for k in range(args.lut):
+            api.lnq_lut_gemv(x, Ps[k % len(Ps)], C, layer.d_in, y=y)
+        torch.cuda.synchronize()
+        print(f"lut_gemv calls={args.lut} sum(y)={float(y.sum()):.6e}")
 
 
 if __name__ == "__main__":
