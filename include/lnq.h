@@ -147,6 +147,28 @@ LNQ_API lnq_status lnq_quantize_rows(const float *F, int groups, const float *W,
                              double *J_out, int32_t *row_status, void *ws, size_t ws_bytes,
                              lnq_stream_t stream);
 
+/* LNQ with a diagonal Fisher block: `iters` iterations of the same codebook step and assignment
+ * sweep as lnq_quantize_rows, with F_g = diag(Fd[g]).
+ * "GuidedQuant" (jinukkim.me blog), opening list, item 2 (diagonal-Fisher methods keep only the
+ * diagonal of the Fisher block); aitopics "squeezellm" tag page, SqueezeLLM abstract
+ * (sensitivity-based non-uniform quantization); the blog's LNQ section iteration.
+ * With a diagonal block the codebook step gives each non-empty codeword the weighted mean
+ * sum f_i w_i / sum f_i of its coordinates (a non-empty class with sum f_i <= 0 makes the row
+ * singular: it keeps its codebook and row_status reports it), and moves in the sweep do not
+ * interact, so every coordinate takes its nearest codeword in the f_i-weighted sense (only a
+ * strictly lower cost moves; the lowest index wins among equals).
+ *   Fd          [groups][d_in] fp32 device, row j uses Fd[j / (d_out/groups)]
+ *   W, C, Q     as lnq_quantize_rows (C, Q in/out; codes are read modulo m)
+ *   J_out       [d_out] fp64 out, sum_i f_i (C[j][Q[j][i]] - W[j][i])^2, or NULL
+ *   row_status  [d_out] int32 out, or NULL
+ * Arithmetic: class sums, cost changes and the objective in fp64, in a fixed order; results are
+ * bit-identical from run to run. Needs no workspace. Requirements as lnq_quantize_rows; otherwise
+ * LNQ_ERR_INVALID_ARG. */
+LNQ_API lnq_status lnq_quantize_rows_diag(const float *Fd, int groups, const float *W,
+                                          int64_t d_out, int64_t d_in, int m, int iters, float *C,
+                                          uint8_t *Q, double *J_out, int32_t *row_status,
+                                          lnq_stream_t stream);
+
 /* Per-row objective J[j] = r^T F_g r with r = C[j][Q[j]] - W[j] (fp32 products, fp64 sums). */
 LNQ_API lnq_status lnq_objective(const float *F, int groups, const float *W, const float *C,
                          const uint8_t *Q, int64_t d_out, int64_t d_in, int m, double *J,

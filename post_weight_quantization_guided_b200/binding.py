@@ -23,7 +23,7 @@ LNQ_OP_BUILD_FISHER, LNQ_OP_INIT_CODEBOOK, LNQ_OP_QUANTIZE_ROWS, LNQ_OP_OBJECTIV
 EXPORTED = ("lnq_workspace_size", "lnq_build_fisher", "lnq_init_codebook", "lnq_quantize_rows",
             "lnq_objective", "lnq_workspace_check", "lnq_set_wait_limit", "lnq_status_string",
             "lnq_profile_enable", "lnq_profile_read", "lnq_build_fisher_noalloc",
-            "lnq_packed_words", "lnq_pack_codes", "lnq_lut_gemv")
+            "lnq_packed_words", "lnq_pack_codes", "lnq_lut_gemv", "lnq_quantize_rows_diag")
 
 _lib = None
 _VP, _I64, _INT, _SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
@@ -68,9 +68,11 @@ def lib():
         L.lnq_packed_words.restype = _I64
         L.lnq_pack_codes.argtypes = [_VP, _I64, _I64, _INT, _VP, _VP]
         L.lnq_lut_gemv.argtypes = [_VP, _I64, _VP, _VP, _I64, _I64, _INT, _VP, _VP]
+        L.lnq_quantize_rows_diag.argtypes = [_VP, _INT, _VP, _I64, _I64, _INT, _INT, _VP, _VP,
+                                             _VP, _VP, _VP]
         for name in ("lnq_build_fisher", "lnq_build_fisher_noalloc", "lnq_init_codebook",
                      "lnq_quantize_rows", "lnq_objective", "lnq_workspace_check",
-                     "lnq_pack_codes", "lnq_lut_gemv"):
+                     "lnq_pack_codes", "lnq_lut_gemv", "lnq_quantize_rows_diag"):
             getattr(L, name).restype = _INT
         _lib = L
     return _lib
@@ -203,6 +205,27 @@ def lnq_quantize_rows(F: torch.Tensor, W: torch.Tensor, m: int, iters: int, C: t
     _check(lib().lnq_quantize_rows(_ptr(F), groups, _ptr(W), d_out, d_in, m, iters, _ptr(C),
                                    _ptr(Q), _ptr(J_out), _ptr(row_status), _ptr(ws), ws.numel(),
                                    _stream(stream)), "lnq_quantize_rows")
+    return C, Q, J_out, row_status
+
+
+def lnq_quantize_rows_diag(Fd: torch.Tensor, W: torch.Tensor, m: int, iters: int,
+                           C: torch.Tensor, Q: torch.Tensor, J_out: Optional[torch.Tensor] = None,
+                           row_status: Optional[torch.Tensor] = None, stream=None):
+    """`iters` LNQ iterations in place on (C, Q) with diagonal Fisher blocks Fd [groups][d_in];
+    returns (C, Q, J_out, row_status)."""
+    groups, d_in = Fd.shape
+    d_out = W.shape[0]
+    _need(Fd, torch.float32, (groups, d_in), "Fd")
+    _need(W, torch.float32, (d_out, d_in), "W")
+    _need(C, torch.float32, (d_out, m), "C")
+    _need(Q, torch.uint8, (d_out, d_in), "Q")
+    if J_out is not None:
+        _need(J_out, torch.float64, (d_out,), "J_out")
+    if row_status is not None:
+        _need(row_status, torch.int32, (d_out,), "row_status")
+    _check(lib().lnq_quantize_rows_diag(_ptr(Fd), groups, _ptr(W), d_out, d_in, m, iters,
+                                        _ptr(C), _ptr(Q), _ptr(J_out), _ptr(row_status),
+                                        _stream(stream)), "lnq_quantize_rows_diag")
     return C, Q, J_out, row_status
 
 

@@ -245,6 +245,20 @@ lnq_status lnq_quantize_rows(const float *F, int groups, const float *W, int64_t
     return LNQ_OK;
 }
 
+lnq_status lnq_quantize_rows_diag(const float *Fd, int groups, const float *W, int64_t d_out,
+                                  int64_t d_in, int m, int iters, float *C, uint8_t *Q,
+                                  double *J_out, int32_t *row_status, lnq_stream_t stream)
+{
+    if (Fd == nullptr || W == nullptr || C == nullptr || Q == nullptr || groups < 1 ||
+        d_out < 1 || d_out % groups != 0 || d_in < 1 || d_in > 16384 || !valid_m(m) ||
+        iters < 0 || d_out > (int64_t(1) << 31) - 1)
+        return LNQ_ERR_INVALID_ARG;
+    return lnq_diag_launch(Fd, groups, W, d_out, d_in, m, iters, C, Q, J_out, row_status,
+                           reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? LNQ_OK
+               : LNQ_ERR_CUDA;
+}
+
 lnq_status lnq_objective(const float *F, int groups, const float *W, const float *C,
                          const uint8_t *Q, int64_t d_out, int64_t d_in, int m, double *J,
                          void *ws, size_t ws_bytes, lnq_stream_t stream)

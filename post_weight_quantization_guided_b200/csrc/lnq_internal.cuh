@@ -67,4 +67,9 @@ cudaError_t lnq_lut_gemv_launch(const float *x, int nb, const uint32_t *P, const
                                 int64_t d_out, int64_t d_in, int bits, float *y, int num_sms,
                                 cudaStream_t s);
 
+// lnq_diag.cu
+cudaError_t lnq_diag_launch(const float *Fd, int groups, const float *W, int64_t d_out, int64_t d,
+                            int m, int iters, float *C, uint8_t *Q, double *J, int32_t *status,
+                            cudaStream_t s);
+
 }  // namespace lnq

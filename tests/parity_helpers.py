@@ -87,11 +87,13 @@ def check_fisher_sampled(orc, F: torch.Tensor, X: torch.Tensor, G, groups: int, 
 
 
 def lnq_follow_parity(orc, lnq, F: torch.Tensor, W: torch.Tensor, m: int, iters: int,
-                      rows_per_group=None, seed=0, nthreads=0):
+                      rows_per_group=None, seed=0, nthreads=0, diag=False):
     """Runs init and then `iters` single-iteration calls of the GPU path on every row, and checks
     sampled rows of each group against the oracle in follow mode after every step.
+    diag=True: F is [groups][d] (the diagonals), the GPU step is lnq_quantize_rows_diag and the
+    oracle runs its ordinary LNQ on the dense matrix diag(F[g]).
     Returns a summary dict."""
-    groups, d, _ = F.shape
+    groups, d = F.shape[0], F.shape[1]
     d_out = W.shape[0]
     R = d_out // groups
     rng = np.random.default_rng(seed)
@@ -116,13 +118,18 @@ def lnq_follow_parity(orc, lnq, F: torch.Tensor, W: torch.Tensor, m: int, iters:
     Fh = [None] * groups
     for it in range(iters):
         C0, Q0 = C.double().cpu().numpy(), Q.cpu().numpy()
-        lnq.lnq_quantize_rows(F, W, m, 1, C, Q, J, st)
+        if diag:
+            lnq.lnq_quantize_rows_diag(F, W, m, 1, C, Q, J, st)
+        else:
+            lnq.lnq_quantize_rows(F, W, m, 1, C, Q, J, st)
         torch.cuda.synchronize()
         C1, Q1 = C.double().cpu().numpy(), Q.cpu().numpy()
         J1, st1 = J.cpu().numpy(), st.cpu().numpy()
         for g in range(groups):
             if Fh[g] is None:
                 Fh[g] = F[g].double().cpu().numpy()
+                if diag:
+                    Fh[g] = np.diag(Fh[g])
             r = rows[g]
             Jw = np.einsum("ri,ik,rk->r", Wh[r], Fh[g], Wh[r])
             Cf, Qf, Jf, stats, status = orc.follow_iteration(Fh[g], Wh[r], m, C0[r], Q0[r], Q1[r],

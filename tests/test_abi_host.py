@@ -30,7 +30,7 @@ def test_header_declares_the_entry_points():
                             "lnq_quantize_rows", "lnq_set_wait_limit", "lnq_status_string",
                             "lnq_workspace_check", "lnq_workspace_size", "lnq_profile_enable",
                             "lnq_profile_read", "lnq_build_fisher_noalloc", "lnq_packed_words",
-                            "lnq_pack_codes", "lnq_lut_gemv"])
+                            "lnq_pack_codes", "lnq_lut_gemv", "lnq_quantize_rows_diag"])
 
 
 def test_packed_words_and_argument_checks(L):
@@ -104,6 +104,17 @@ def _quant(L, **kw):
 ])
 def test_quantize_rows_rejects_bad_arguments(L, kw):
     assert _quant(L, **kw) == 1
+
+
+@pytest.mark.parametrize("kw", [
+    dict(m=3), dict(m=32), dict(iters=-1), dict(groups=5), dict(d_out=0), dict(d_in=0),
+    dict(d_in=16385), dict(F=None), dict(C=None), dict(Q=None), dict(W=None),
+])
+def test_quantize_rows_diag_rejects_bad_arguments(L, kw):
+    a = dict(F=FAKE, groups=4, W=FAKE, d_out=64, d_in=128, m=8, iters=3, C=FAKE, Q=FAKE)
+    a.update(kw)
+    assert L.lnq_quantize_rows_diag(a["F"], a["groups"], a["W"], a["d_out"], a["d_in"], a["m"],
+                                    a["iters"], a["C"], a["Q"], None, None, None) == 1
 
 
 def test_quantize_rows_rejects_small_workspace(L):

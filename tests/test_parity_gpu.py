@@ -241,6 +241,81 @@ def test_lnq_singular_rows(orc, lnq):
     assert torch.equal(C, C0)
 
 
+# ----------------------------------------------------------------- LNQ, diagonal Fisher blocks
+
+def _fisher_diagonal(lnq, wl, layer):
+    X, G, W = wl.make_layer(layer, _dev())
+    F = lnq.lnq_build_fisher(X, G, layer.groups)
+    Fd = torch.diagonal(F, dim1=1, dim2=2).contiguous()
+    return Fd, W
+
+
+@pytest.mark.parametrize("m", [2, 4, 8, 16])
+def test_lnq_diag_tiny_layer_every_codebook_size(orc, lnq, wl, m):
+    Fd, W = _fisher_diagonal(lnq, wl, wl.TINY)
+    summary, _, _ = lnq_follow_parity(orc, lnq, Fd, W, m, 3, diag=True)
+    assert summary["moves"] > 0
+
+
+@pytest.mark.parametrize("d_in,d_out,groups", [(1, 3, 1), (5, 4, 2), (300, 66, 3), (1027, 40, 2)])
+def test_lnq_diag_ragged_shapes(orc, lnq, d_in, d_out, groups):
+    # d_in not a multiple of 8 (the Fisher build's rule), so log-normal weights stand in for the
+    # Fisher diagonal
+    gen = torch.Generator().manual_seed(d_in)
+    Fd = torch.exp(torch.randn(groups, d_in, generator=gen)).to(_dev())
+    W = (torch.randn(d_out, d_in, generator=gen) * 0.02).to(_dev())
+    lnq_follow_parity(orc, lnq, Fd, W, 8, 3, diag=True)
+
+
+def test_lnq_diag_q_proj_full_size_sampled_rows(orc, lnq, wl):
+    Fd, W = _fisher_diagonal(lnq, wl, wl.Q_PROJ)
+    summary, C, Q = lnq_follow_parity(orc, lnq, Fd, W, 16, 3, rows_per_group=16, diag=True)
+    assert summary["moves"] > 0
+    # run to run: bit-identical, and two calls of one iteration equal one call of two
+    C2, Q2 = lnq.lnq_init_codebook(W, 16)
+    C3, Q3 = C2.clone(), Q2.clone()
+    lnq.lnq_quantize_rows_diag(Fd, W, 16, 3, C2, Q2)
+    lnq.lnq_quantize_rows_diag(Fd, W, 16, 1, C3, Q3)
+    lnq.lnq_quantize_rows_diag(Fd, W, 16, 2, C3, Q3)
+    torch.cuda.synchronize()
+    assert torch.equal(C2, C) and torch.equal(Q2, Q)
+    assert torch.equal(C3, C) and torch.equal(Q3, Q)
+
+
+def test_lnq_diag_singular_rows(orc, lnq):
+    # Row 0 (group 0): f = 0 on coordinates 0..3, which hold the row's only large values, so a
+    # codeword used only there has no weight: the row keeps its codebook and reports
+    # LNQ_ROW_SINGULAR. Row 1 (group 1) has positive weights everywhere and is not singular.
+    d, m = 16, 4
+    torch.manual_seed(1)
+    f = torch.rand(2, d, dtype=torch.float32) + 0.5
+    f[0, :4] = 0
+    Fd = f.to(_dev())
+    W = torch.cat([torch.full((2, 4), 5.0), torch.randn(2, d - 4) * 0.01], dim=1)
+    W[1, :4] = torch.randn(4) * 0.01
+    W = W.float().contiguous().to(_dev())
+    st = torch.empty(2, dtype=torch.int32, device=_dev())
+    J = torch.empty(2, dtype=torch.float64, device=_dev())
+    C, Q = lnq.lnq_init_codebook(W, m)
+    C0, Q0 = C.clone(), Q.clone()
+    lnq.lnq_quantize_rows_diag(Fd, W, m, 1, C, Q, J, st)
+    torch.cuda.synchronize()
+    Fh = [np.diag(f[j].double().numpy()) for j in range(2)]
+    for j, want in ((0, 1), (1, 0)):
+        c_or, status = orc.codebook_row(Fh[j], W[j].double().cpu().numpy(), Q0.cpu().numpy()[j],
+                                        C0[j].double().cpu().numpy())
+        assert status == want and int(st[j]) == want
+    assert torch.equal(C[0], C0[0])
+    # the sweep still ran with the kept codebook: every coordinate with f > 0 is at its nearest
+    # codeword, and the reported objective is the oracle's of the final state
+    Ch, Qh, Wh = C.double().cpu().numpy(), Q.cpu().numpy(), W.double().cpu().numpy()
+    for j in range(2):
+        Jo = orc.objective_row(Fh[j], Wh[j], Ch[j], Qh[j])
+        assert abs(float(J[j]) - Jo) <= J_TOL * Jo + 1e-30
+        for i in range(4, d):
+            assert abs(Ch[j][Qh[j][i]] - Wh[j][i]) <= np.abs(Ch[j] - Wh[j][i]).min()
+
+
 def test_objective_entry_point(orc, lnq, wl):
     layer = wl.TINY
     X, G, W = wl.make_layer(layer, _dev())
