@@ -367,3 +367,38 @@ def test_follow_mode_absolute_floor_for_exactly_representable_rows(orc):
     bad[4] = 0
     _, _, st3, _ = orc.sweep_row(F, w, c, q0, hint=bad, tie_rel=1e-6, tie_abs=1e-12 * Jw)
     assert st3["mismatches"] == 1
+
+
+def _weighted_lloyd(f, w, c, q, iters):
+    """Textbook weighted 1-D k-means (Lloyd): each non-empty cluster's centre becomes the f-weighted
+    mean of its points, then every point takes its nearest centre (a point moves only to a
+    strictly nearer centre; the lowest index wins among equally near ones)."""
+    c, q = c.copy(), q.copy()
+    for _ in range(iters):
+        for a in range(len(c)):
+            sel = q == a
+            if sel.any():
+                c[a] = np.sum(f[sel] * w[sel]) / np.sum(f[sel])
+        dist = (w[:, None] - c[None, :]) ** 2
+        best = np.argmin(dist, axis=1)
+        stay = dist[np.arange(len(w)), q] <= dist[np.arange(len(w)), best]
+        q = np.where(stay, q, best).astype(np.uint8)
+    return c, q
+
+
+def test_lnq_with_diagonal_F_is_weighted_lloyd(orc):
+    """With F = diag(f) the LNQ iteration (codebook step, then the in-order sweep) is weighted
+    1-D k-means: the normal equations are diagonal and moves do not interact. The diagonal-Fisher
+    objective of the GuidedQuant post's opening list (SqueezeLLM's sensitivity-weighted
+    clustering, aitopics tag page) is exactly this case."""
+    rng = np.random.default_rng(21)
+    for d, m in ((64, 4), (300, 8), (1000, 16)):
+        W = rng.standard_t(5, (3, d)) * 0.02
+        f = np.exp(rng.standard_normal(d))
+        C, Q, _, st = orc.lnq_rows(np.diag(f), W, m, 4)
+        for j in range(3):
+            c0, q0 = orc.init_row(W[j], m)
+            c, q = _weighted_lloyd(f, W[j], c0, q0, 4)
+            np.testing.assert_array_equal(Q[j], q)
+            np.testing.assert_allclose(C[j], c, rtol=1e-12, atol=1e-15)
+        assert np.all(st == 0)
