@@ -1,0 +1,158 @@
+"""Several layers across ranks: every (linear, Fisher group) pair is one unit of independent work.
+
+"GuidedQuant" (jinukkim.me blog), GuidedQuant section, third equation and the sentence after it:
+the objective is a sum over layers l and output rows j of per-row terms, and rows share a Fisher
+block only inside their group. So a unit needs X of its layer, the G columns and W rows of its
+group, and nothing from any other unit: ranks run their units without a collective, and one
+all-gather of the results (codebooks C and codes Q) ends the job.
+
+  plan(layers, world)           units assigned to ranks, largest first to the least-loaded rank
+                                (ties to the lower rank); every rank computes the same plan
+  run(layers, rank, world, compute, group=None)
+                                runs this rank's units through `compute`, then all-gathers every
+                                unit's (C, Q) into whole-layer tensors on every rank
+  gpu_compute(lnq, wl, device)  the unit computation on the GPU library: guided Fisher block of the
+                                group (its G columns, one group), initial codebook, LNQ iterations
+"""
+from __future__ import annotations
+
+import dataclasses
+from typing import Callable, Dict, List, Tuple
+
+import torch
+import torch.distributed as dist
+
+
+@dataclasses.dataclass(frozen=True)
+class Unit:
+    layer: int        # index into the layer list
+    group: int        # Fisher group within the layer
+    row0: int         # first output row of the group
+    row1: int         # one past the last
+    cost: float       # flop estimate used for balancing
+
+
+def unit_cost(layer) -> float:
+    """Flops of one group: its Fisher block (n d_in (d_in + 1) unique-entry flops) plus the class-
+    binned product of every LNQ iteration (2 d_in^2 m flops per row), which dominate the step."""
+    R = layer.d_out // layer.groups
+    return (float(layer.n) * layer.d_in * (layer.d_in + 1)
+            + 2.0 * layer.d_in * layer.d_in * layer.m * R * layer.iters)
+
+
+def units_of(layers) -> List[Unit]:
+    out = []
+    for li, layer in enumerate(layers):
+        R = layer.d_out // layer.groups
+        c = unit_cost(layer)
+        for g in range(layer.groups):
+            out.append(Unit(li, g, g * R, (g + 1) * R, c))
+    return out
+
+
+def plan(layers, world: int) -> List[List[Unit]]:
+    """Longest-processing-time assignment: units by decreasing cost (then layer, group), each to
+    the rank with the least load so far (the lowest rank among equals). Deterministic, so every
+    rank derives the same plan without communication. Each rank's list is in assignment order."""
+    if world < 1:
+        raise ValueError("world must be >= 1")
+    order = sorted(units_of(layers), key=lambda u: (-u.cost, u.layer, u.group))
+    load = [0.0] * world
+    out: List[List[Unit]] = [[] for _ in range(world)]
+    for u in order:
+        r = min(range(world), key=lambda k: (load[k], k))
+        out[r].append(u)
+        load[r] += u.cost
+    return out
+
+
+def _unit_bytes(layers, u: Unit) -> int:
+    layer = layers[u.layer]
+    return (u.row1 - u.row0) * (4 * layer.m + layer.d_in)
+
+
+def _pack(layers, units, results, device) -> torch.Tensor:
+    parts = []
+    for u in units:
+        C, Q = results[(u.layer, u.group)]
+        parts.append(C.contiguous().view(torch.uint8).reshape(-1).to(device))
+        parts.append(Q.contiguous().reshape(-1).to(device))
+    if not parts:
+        return torch.empty(0, dtype=torch.uint8, device=device)
+    return torch.cat(parts)
+
+
+def gather(layers, assignment, results, device, group=None):
+    """All-gathers the units' (C, Q) of every rank. Returns, for every layer, (C [d_out][m] fp32,
+    Q [d_out][d_in] uint8) on `device`. Buffer sizes follow from the plan, so one all_gather of
+    equal-length byte buffers (padded to the largest rank) is the only exchange."""
+    world = len(assignment)
+    sizes = [sum(_unit_bytes(layers, u) for u in units) for units in assignment]
+    mx = max(sizes) if sizes else 0
+    rank = dist.get_rank(group) if world > 1 else 0
+    mine = _pack(layers, assignment[rank], results, device)
+    buf = torch.zeros(mx, dtype=torch.uint8, device=device)
+    buf[:mine.numel()] = mine
+    if world > 1:
+        bufs = [torch.empty(mx, dtype=torch.uint8, device=device) for _ in range(world)]
+        dist.all_gather(bufs, buf, group=group)
+    else:
+        bufs = [buf]
+    out = {li: (torch.empty((layer.d_out, layer.m), dtype=torch.float32, device=device),
+                torch.empty((layer.d_out, layer.d_in), dtype=torch.uint8, device=device))
+           for li, layer in enumerate(layers)}
+    for r, units in enumerate(assignment):
+        off = 0
+        for u in units:
+            layer = layers[u.layer]
+            R = u.row1 - u.row0
+            nc = R * layer.m * 4
+            C, Q = out[u.layer]
+            C[u.row0:u.row1] = bufs[r][off:off + nc].view(torch.float32).view(R, layer.m)
+            off += nc
+            nq = R * layer.d_in
+            Q[u.row0:u.row1] = bufs[r][off:off + nq].view(R, layer.d_in)
+            off += nq
+    return out
+
+
+def run(layers, rank: int, world: int,
+        compute: Callable[[object, int, int, int], Tuple[torch.Tensor, torch.Tensor]],
+        device, group=None):
+    """This rank's units through compute(layer, group, row0, row1) -> (C rows, Q rows), then the
+    all-gather. Returns (per-layer (C, Q) on `device`, this rank's units)."""
+    assignment = plan(layers, world)
+    results: Dict[Tuple[int, int], Tuple[torch.Tensor, torch.Tensor]] = {}
+    # layer order, so that units of one layer (and layers of one X draw) run back to back
+    for u in sorted(assignment[rank], key=lambda u: (u.layer, u.group)):
+        results[(u.layer, u.group)] = compute(layers[u.layer], u.group, u.row0, u.row1)
+    return gather(layers, assignment, results, device, group), assignment[rank]
+
+
+def gpu_compute(lnq, wl, device):
+    """compute() for run(): the unit on the GPU library. X is drawn once per distinct draw, G and
+    W once per layer, each kept while consecutive units use it; the group's G columns and W rows
+    are copied out contiguous. The group's block is built with groups = 1 over those columns,
+    which is the group's F_g of the whole layer (s_g averages only the group's columns); with
+    all-ones gradients (G is None) every group's block is X^T X."""
+    xs, gw = {}, {}
+
+    def compute(layer, g, row0, row1):
+        xkey = (layer.x_seed, layer.x_kind, layer.n, layer.d_in)
+        if xkey not in xs:
+            xs.clear()
+            xs[xkey] = wl.make_x(layer, device)
+        if layer.name not in gw:
+            gw.clear()
+            gw[layer.name] = (wl.make_g(layer, device), wl.make_w(layer, device))
+        X = xs[xkey]
+        G, W = gw[layer.name]
+        Gg = None if G is None else G[:, row0:row1].contiguous()
+        Wg = W[row0:row1].contiguous()
+        F = lnq.lnq_build_fisher(X, Gg, 1)
+        del Gg
+        C, Q = lnq.lnq_init_codebook(Wg, layer.m)
+        lnq.lnq_quantize_rows(F, Wg, layer.m, layer.iters, C, Q)
+        return C, Q
+
+    return compute
