@@ -111,7 +111,7 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------------------------------
-# Algorithmic work per kernel: the per-unit figure of each kernel times the units one launch processes
+# Algorithmic work per kernel: per-unit figure x the units one launch processes
 # ------------------------------------------------------------------------------------------
 def algorithmic_work(layer, kernel: str, launches: int, moves_per_sweep: float):
     """(amount, unit kind) per launch for a kernel of one step on `layer`."""
