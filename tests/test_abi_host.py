@@ -134,3 +134,28 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(b, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError, match="missing"):
         b.lib()
+
+
+def test_binding_refuses_host_tensors():
+    """No CPU path: every compute entry of the binding rejects host tensors before any call."""
+    import torch
+    import post_weight_quantization_guided_b200 as pkg
+    d, dout, m, g = 16, 8, 4, 2
+    X = torch.zeros(32, d, dtype=torch.bfloat16)
+    G = torch.zeros(32, dout, dtype=torch.bfloat16)
+    F = torch.zeros(g, d, d)
+    Fd = torch.zeros(g, d)
+    W = torch.zeros(dout, d)
+    C = torch.zeros(dout, m)
+    Q = torch.zeros(dout, d, dtype=torch.uint8)
+    P = torch.zeros(dout, 2, dtype=torch.int32)
+    calls = [lambda: pkg.lnq_build_fisher(X, G, g),
+             lambda: pkg.lnq_init_codebook(W, m),
+             lambda: pkg.lnq_quantize_rows(F, W, m, 1, C, Q),
+             lambda: pkg.lnq_quantize_rows_diag(Fd, W, m, 1, C, Q),
+             lambda: pkg.lnq_objective(F, W, C, Q),
+             lambda: pkg.lnq_pack_codes(Q, 2),
+             lambda: pkg.lnq_lut_gemv(torch.zeros(1, d), P, C, d)]
+    for call in calls:
+        with pytest.raises(ValueError, match="CUDA"):
+            call()
