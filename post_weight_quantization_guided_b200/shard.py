@@ -156,3 +156,64 @@ def gpu_compute(lnq, wl, device):
         return C, Q
 
     return compute
+
+
+def main(argv=None, compute=None, device=None, backend=None):
+    """Quantises the decoder block: one process per GPU (torchrun sets RANK and WORLD_SIZE), each
+    running its units, then the all-gather. Rank 0 prints one JSON line: rows quantised, the time
+    of the slowest rank (CUDA events on GPUs, wall clock on CPU) and rows per second.
+    compute / device / backend: overrides for running the host logic without a GPU."""
+    import argparse
+    import json
+    import os
+    import time
+
+    ap = argparse.ArgumentParser(description=main.__doc__)
+    ap.add_argument("--bits", type=int, default=4, choices=(1, 2, 3, 4))
+    args = ap.parse_args(argv)
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    from . import workloads as wl
+    if device is None:
+        local = int(os.environ.get("LOCAL_RANK", "0"))
+        device = torch.device("cuda", local)
+        torch.cuda.set_device(device)
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend or ("nccl" if device.type == "cuda" else "gloo"))
+    try:
+        if compute is None:
+            import post_weight_quantization_guided_b200 as lnq
+            compute = gpu_compute(lnq, wl, device)
+        layers = wl.decoder_block(1 << args.bits)
+        if world > 1:
+            dist.barrier()
+        if device.type == "cuda":
+            torch.cuda.synchronize(device)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+        t0 = time.perf_counter()
+        out, mine = run(layers, rank, world, compute, device)
+        if device.type == "cuda":
+            e1.record()
+            torch.cuda.synchronize(device)
+            ms = e0.elapsed_time(e1)
+        else:
+            ms = (time.perf_counter() - t0) * 1e3
+        t = torch.tensor([ms], dtype=torch.float64, device=device)
+        if world > 1:
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        rows = sum(layer.d_out for layer in layers)
+        line = {"workload": f"decoder block, {len(layers)} linears, n = {layers[0].n}, "
+                            f"m = {1 << args.bits}",
+                "ranks": world, "units": len(units_of(layers)), "rows": rows,
+                "ms": float(t.item()), "rows_per_s": rows / (float(t.item()) / 1e3)}
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+        return line, out
+    finally:
+        if world > 1 and dist.is_initialized():
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

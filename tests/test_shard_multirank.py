@@ -140,3 +140,39 @@ def test_one_rank_gather_needs_no_process_group():
     for g in range(3):
         Cg, Qg = fake(layers[0], g, 2 * g, 2 * g + 2)
         assert torch.equal(C[2 * g:2 * g + 2], Cg) and torch.equal(Q[2 * g:2 * g + 2], Qg)
+
+
+def _main_rank(rank, world, port, out):
+    sys.path.insert(0, ROOT)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world))
+    from post_weight_quantization_guided_b200 import shard
+
+    def fake(layer, g, row0, row1):
+        R = row1 - row0
+        return (torch.full((R, layer.m), float(g), dtype=torch.float32),
+                torch.full((R, layer.d_in), g, dtype=torch.uint8))
+
+    line, res = shard.main(["--bits", "3"], compute=fake, device=torch.device("cpu"))
+    out[rank] = (line, [(float(C.sum()), int(Q.sum())) for _, (C, Q) in sorted(res.items())])
+
+
+@pytest.mark.timeout(300)
+def test_main_runs_the_decoder_block_on_two_gloo_ranks():
+    """The command-line runner's host logic: the block's 28 units split over two ranks, the job
+    time is the slower rank's, and both ranks hold every layer's gathered result."""
+    from post_weight_quantization_guided_b200 import workloads as wl
+    world = 2
+    with mp.get_context("spawn").Manager() as mgr:
+        out = mgr.dict()
+        mp.spawn(_main_rank, args=(world, _free_port(), out), nprocs=world, join=True)
+        res = dict(out)
+    layers = wl.decoder_block(8)
+    want = [(float(sum(g * (l.d_out // l.groups) * l.m for g in range(l.groups))),
+             sum(g * (l.d_out // l.groups) * l.d_in for g in range(l.groups))) for l in layers]
+    for r in range(world):
+        line, sums = res[r]
+        assert line["units"] == 28 and line["ranks"] == 2
+        assert line["rows"] == sum(l.d_out for l in layers)
+        assert sums == want
+    assert res[0][0]["ms"] == res[1][0]["ms"]
