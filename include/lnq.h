@@ -162,8 +162,10 @@ LNQ_API lnq_status lnq_quantize_rows(const float *F, int groups, const float *W,
  *   J_out       [d_out] fp64 out, sum_i f_i (C[j][Q[j][i]] - W[j][i])^2, or NULL
  *   row_status  [d_out] int32 out, or NULL
  * Arithmetic: class sums, cost changes and the objective in fp64, in a fixed order; results are
- * bit-identical from run to run. Needs no workspace. Requirements as lnq_quantize_rows; otherwise
- * LNQ_ERR_INVALID_ARG. */
+ * bit-identical from run to run. Needs no workspace.
+ * Requirements: non-NULL Fd, W, C, Q; m in {2, 4, 8, 16}; 1 <= d_in <= 16384; 1 <= d_out < 2^31;
+ * groups >= 1 and d_out % groups == 0; iters >= 0. Otherwise LNQ_ERR_INVALID_ARG before any
+ * device work; a launch failure is LNQ_ERR_CUDA. */
 LNQ_API lnq_status lnq_quantize_rows_diag(const float *Fd, int groups, const float *W,
                                           int64_t d_out, int64_t d_in, int m, int iters, float *C,
                                           uint8_t *Q, double *J_out, int32_t *row_status,
