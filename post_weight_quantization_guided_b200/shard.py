@@ -13,6 +13,9 @@ all-gather of the results (codebooks C and codes Q) ends the job.
                                 unit's (C, Q) into whole-layer tensors on every rank
   gpu_compute(lnq, wl, device)  the unit computation on the GPU library: guided Fisher block of the
                                 group (its G columns, one group), initial codebook, LNQ iterations
+  token_range, reduce_fisher    the alternative for very large n: each rank builds the blocks
+                                over its own tokens, one all-reduce (or reduce-scatter of the
+                                groups) sums them
 """
 from __future__ import annotations
 
@@ -127,6 +130,40 @@ def run(layers, rank: int, world: int,
     for u in sorted(assignment[rank], key=lambda u: (u.layer, u.group)):
         results[(u.layer, u.group)] = compute(layers[u.layer], u.group, u.row0, u.row1)
     return gather(layers, assignment, results, device, group), assignment[rank]
+
+
+def token_range(n: int, rank: int, world: int) -> Tuple[int, int]:
+    """Rank `rank`'s contiguous slice [t0, t1) of n tokens (the first n % world ranks get one
+    more)."""
+    base, extra = divmod(n, world)
+    t0 = rank * base + min(rank, extra)
+    return t0, t0 + base + (1 if rank < extra else 0)
+
+
+def reduce_fisher(F_partial: torch.Tensor, keep_groups: bool = False, group=None) -> torch.Tensor:
+    """Token-sharded Fisher build, the exchange step: every rank built F [groups][d][d] over its
+    own tokens (s_g[t] depends only on token t's gradient row, so the blocks are sums over tokens
+    and the partial blocks add up to the whole). Sums them in place on every rank (all-reduce), or
+    with keep_groups=True returns only this rank's share of the groups (reduce-scatter over the
+    group dimension; groups must be a multiple of the world size)."""
+    world = dist.get_world_size(group) if dist.is_initialized() else 1
+    if world == 1:
+        return F_partial
+    if not keep_groups:
+        dist.all_reduce(F_partial, group=group)
+        return F_partial
+    groups = F_partial.shape[0]
+    if groups % world != 0:
+        raise ValueError(f"{groups} groups do not split over {world} ranks")
+    out = torch.empty((groups // world,) + tuple(F_partial.shape[1:]), dtype=F_partial.dtype,
+                      device=F_partial.device)
+    if dist.get_backend(group) == "nccl":
+        dist.reduce_scatter_tensor(out, F_partial.contiguous(), group=group)
+    else:   # backends without reduce-scatter: the full sum, then this rank's slice
+        dist.all_reduce(F_partial, group=group)
+        r = dist.get_rank(group)
+        out.copy_(F_partial[r * (groups // world):(r + 1) * (groups // world)])
+    return out
 
 
 def gpu_compute(lnq, wl, device):

@@ -176,3 +176,57 @@ def test_main_runs_the_decoder_block_on_two_gloo_ranks():
         assert line["rows"] == sum(l.d_out for l in layers)
         assert sums == want
     assert res[0][0]["ms"] == res[1][0]["ms"]
+
+
+def _fisher_rank(rank, world, port, out):
+    sys.path.insert(0, ROOT)
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        from oracle import oracle as orc
+        from post_weight_quantization_guided_b200 import shard
+        from post_weight_quantization_guided_b200 import workloads as wl
+        layer = wl.TINY
+        X = wl.make_x(layer).double()
+        G = wl.make_g(layer).double()
+        t0, t1 = shard.token_range(layer.n, rank, world)
+        Fp = torch.from_numpy(orc.fisher_full(X[t0:t1].numpy(), G[t0:t1].numpy(), layer.groups))
+        try:
+            mine = shard.reduce_fisher(Fp.clone(), keep_groups=True).numpy()
+        except ValueError:      # raised on every rank alike, before any collective
+            mine = None
+        every = shard.reduce_fisher(Fp.clone())
+        out[rank] = (every.numpy(), mine, (t0, t1))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.timeout(300)
+@pytest.mark.parametrize("world", [2, 3])
+def test_token_sharded_fisher_sums_to_the_whole(orc, world):
+    """gloo ranks each build the tiny layer's four blocks over their own tokens with the oracle
+    (with 3 ranks the 256 tokens do not split evenly). The all-reduce gives every rank the
+    whole-token blocks; the reduce-scatter path gives each rank its own groups, and refuses a
+    group count that does not split over the ranks."""
+    from post_weight_quantization_guided_b200 import workloads as wl
+    from post_weight_quantization_guided_b200 import shard
+    layer = wl.TINY
+    assert [shard.token_range(10, r, 3) for r in range(3)] == [(0, 4), (4, 7), (7, 10)]
+    with mp.get_context("spawn").Manager() as mgr:
+        out = mgr.dict()
+        mp.spawn(_fisher_rank, args=(world, _free_port(), out), nprocs=world, join=True)
+        res = dict(out)
+    F = orc.fisher_full(wl.make_x(layer).double().numpy(), wl.make_g(layer).double().numpy(),
+                        layer.groups)
+    spans = sorted(res[r][2] for r in range(world))
+    assert spans[0][0] == 0 and spans[-1][1] == layer.n
+    assert all(a[1] == b[0] for a, b in zip(spans, spans[1:]))
+    tol = dict(rtol=1e-12, atol=1e-12 * np.abs(F).max())
+    per = layer.groups // world
+    for r in range(world):
+        np.testing.assert_allclose(res[r][0], F, **tol)
+        if layer.groups % world == 0:
+            np.testing.assert_allclose(res[r][1], F[r * per:(r + 1) * per], **tol)
+        else:
+            assert res[r][1] is None
