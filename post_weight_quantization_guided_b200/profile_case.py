@@ -8,7 +8,9 @@ multiple of the group count) so that a capture stays small. It prints the object
 a run can be checked to have completed.
 
 With `--lut N` it then packs the codes and runs the lookup-table GEMV N times on one activation
-vector (the codes cycled through enough copies that they come from HBM).
+vector (the codes cycled through enough copies that they come from HBM). With `--diag N` it runs
+N calls of LNQ with diagonal Fisher blocks (the diagonals of the blocks just built, `--iters`
+iterations each, from the initial codebooks).
 """
 from __future__ import annotations
 
@@ -28,6 +30,8 @@ def main(argv=None) -> None:
     ap.add_argument("--rows", type=int, default=0, help="output rows (default: the workload's)")
     ap.add_argument("--iters", type=int, default=1)
     ap.add_argument("--lut", type=int, default=0, help="lookup-table GEMV calls after the run")
+    ap.add_argument("--diag", type=int, default=0,
+                    help="calls of LNQ with diagonal Fisher blocks after the run")
     args = ap.parse_args(argv)
     layer = WORKLOADS[args.workload]
     if args.rows:
@@ -53,6 +57,15 @@ def main(argv=None) -> None:
             api.lnq_lut_gemv(x, Ps[k % len(Ps)], C, layer.d_in, y=y)
         torch.cuda.synchronize()
         print(f"lut_gemv calls={args.lut} sum(y)={float(y.sum()):.6e}")
+    if args.diag:
+        Fd = torch.diagonal(F, dim1=1, dim2=2).contiguous()
+        C0, Q0 = api.lnq_init_codebook(W, layer.m)
+        for _ in range(args.diag):
+            C.copy_(C0)
+            Q.copy_(Q0)
+            api.lnq_quantize_rows_diag(Fd, W, layer.m, args.iters, C, Q, J, st)
+        torch.cuda.synchronize()
+        print(f"lnq_diag calls={args.diag} iters={args.iters} sum(J)={float(J.sum()):.6e}")
 
 
 if __name__ == "__main__":
