@@ -1,19 +1,25 @@
 """Benchmark of the GuidedQuant + LNQ hot path on B200.
 
-One step = the whole hot path on one synthetic Llama-2-7B q_proj layer (d_in = d_out = 4096,
-n = 16384 calibration tokens, 4 Fisher groups, 4-bit codebooks, 3 LNQ iterations):
-guided Fisher build (s_g reduction, operand scaling, tcgen05 SYRK), codebook initialisation,
-3 x (codebook step + assignment sweep), and the per-row objective.
+Headline workload: the seven linears of a Llama-2-7B-shaped decoder block (q, k, v, o 4096 x 4096;
+gate, up 4096 -> 11008; down 11008 -> 4096), n = 131072 calibration tokens, 4 Fisher groups,
+5 LNQ iterations, quantised at 4 bits (m = 16) and at 3 bits (m = 8). One step quantises the
+whole block at both bit widths: per layer the guided Fisher build (s_g reduction, then the
+tcgen05 SYRK with the diag(s_g) scaling fused into its operand load), then for each bit width the
+codebook initialisation, 5 x (codebook step + assignment sweep) and the per-row objective. F does
+not depend on the bit width, so each layer's F is built once and used by both.
 
-    python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+    python bench.py [--gpus N --steps K --warmup W] [--impl reference] [--no-q-proj]
 
-With N > 1 (launched by torchrun, one process per GPU) every rank quantises its own layer (the
-rows, groups and layers of the method are independent), so per-GPU work is fixed: weak scaling,
-with no collective on the data path. Rank 0 prints one JSON line.
+`value` is rows quantised per second over the whole step (both bit widths, Fisher build
+included); the line also gives, per bit width, the end-to-end block time (the Fisher builds plus
+that bit width's LNQ) and the LNQ-only rate d_out / (t_init + t_iterations) summed over layers.
+With N > 1 (torchrun, one process per GPU) every rank quantises its own block (seeds offset per
+rank): weak scaling, no collective on the data path. Rank 0 prints one JSON line.
 """
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
 import statistics
@@ -27,10 +33,12 @@ sys.path.insert(0, ROOT)
 import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
-METRIC = "LNQ rows quantized/s per layer (guided Fisher build + init + LNQ iterations)"
+METRIC = ("LNQ rows quantized/s per layer (guided Fisher build + init + LNQ iterations + "
+          "objective)")
 UNIT = "rows/s"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
                   "sm_max_mhz": 1965.0}
+FISHER_KERNELS = ("token_stats", "fisher_syrk")
 
 
 def load_peaks():
@@ -111,157 +119,177 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------------------------------
-# Algorithmic work per kernel: per-unit figure x the units one launch processes
+# Algorithmic work per launch: the per-unit figure times the units one launch processes
 # ------------------------------------------------------------------------------------------
-def algorithmic_work(layer, kernel: str, launches: int, moves_per_sweep: float):
-    """(amount, unit kind) per launch for a kernel of one step on `layer`."""
-    d, n, g, dout, m = layer.d_in, layer.n, layer.groups, layer.d_out, layer.m
+def launches_per_call(kernel, layer, iters):
+    """Launches of `kernel` made by one layer's Fisher build (Fisher kernels) or by one
+    init + lnq_quantize_rows(iters, with J) call (LNQ kernels)."""
+    guided = layer.g_kind != "ones"
+    fixed = {"token_stats": 1 if guided else 0, "fisher_syrk": 1, "lnq_init": 1,
+             "lnq_split_f16": 1, "lnq_objective": 1}
+    per_iter = ("lnq_operand_image", "lnq_mgemm", "lnq_solve", "lnq_sweep")
+    if kernel in fixed:
+        return fixed[kernel]
+    if kernel in per_iter:
+        return iters
+    if kernel in ("lnq_residual_scale", "lnq_residual_image", "lnq_residual_gemm"):
+        return 2 + iters        # -F w once, u = F r before every sweep and for the objective
+    return 0
+
+
+def algorithmic_work(layer, m, kernel, sweep_tail=None):
+    """(amount, unit) of one launch of `kernel` on `layer` at m codewords.
+
+    sweep_tail: for lnq_sweep, the measured sum over moved coordinates of (d - i) per launch."""
+    d, n, g, dout = layer.d_in, layer.n, layer.groups, layer.d_out
     if kernel == "fisher_syrk":
         # every unique entry of each symmetric block: 2 n flops for each of d(d+1)/2 entries
         return float(g) * n * d * (d + 1), "flop"
     if kernel == "token_stats":
         return 2.0 * n * (d + dout) + 4.0 * n * (g + 1), "byte"    # read X and G, write S and M
-    if kernel == "guided_operands":
-        return 2.0 * n * d * (2 + g) + 4.0 * n * (g + 1), "byte"   # read X, S, M; write A, B_g
     if kernel == "lnq_init":
         return 4.0 * dout * d + dout * d + 4.0 * dout * m, "byte"  # read W, write Q and C
     ld = (d + 7) // 8 * 8
     if kernel in ("lnq_operand_image", "lnq_residual_image"):
-        # write the right-operand image (N columns x d coordinates x 2 bytes per row tile), read Q
-        # and W once
-        rt = 256 // m if kernel == "lnq_operand_image" else 64
-        ncols = 256 if kernel == "lnq_operand_image" else 192
+        # write the right-operand image (256 columns x d coordinates x 2 bytes per row tile), read
+        # Q (and W for the residual) once
+        rt = 256 // m if kernel == "lnq_operand_image" else 128
         tiles = g * -(-(dout // g) // rt)
-        return tiles * ncols * (-(-d // 64) * 64) * 2.0 + 5.0 * dout * d, "byte"
+        reads = dout * d * (1.0 if kernel == "lnq_operand_image" else 5.0)
+        return tiles * 256 * (-(-d // 64) * 64) * 2.0 + reads, "byte"
     if kernel == "lnq_split_f16":
         return 4.0 * g * d * d + 4.0 * g * d * ld, "byte"           # read F, write 2 fp16 pieces
     if kernel == "lnq_residual_scale":
         return 5.0 * dout * d, "byte"                               # read W and Q
-    if kernel == "lnq_vgemm":
-        # the class-binned product V_j = F P_j over all rows: 2 d^2 m flops per row
-        return 2.0 * d * d * m * dout, "flop"
+    if kernel == "lnq_mgemm":
+        # the codebook step's M = P^T F P: d^2 / 2 FADD per row with the symmetry of F
+        return 0.5 * d * d * dout, "lane_op"
     if kernel == "lnq_residual_gemm":
-        return 2.0 * d * d * dout, "flop"                           # u = F r for every row
+        return 1.0 * d * d * dout, "lane_op"                        # u = F r: d^2 FMA per row
     if kernel == "lnq_solve":
-        return dout * (d * (4.0 * m + 4 + 1) + 8.0 * m), "byte"    # read V, uT, Q; write C, dC
+        # read the binned partial sums (m x m per 128 coordinates), U and Q; write C
+        halves = 2 * -(-d // 256)
+        return dout * (halves * m * m * 4.0 + d * 5.0 + 4.0 * m), "byte"
     if kernel == "lnq_sweep":
-        # coordinate descent: the triangular u update d^2/2 FMA per row (the blocked scheme does
-        # it whenever a block moved) plus 2 d m for the candidates and the V dc refresh
-        return dout * (d * d / 2.0 + 2.0 * d * m), "lane_op"
+        # the moves' updates of u (sum over moved coordinates of d - i FMA) plus the candidate
+        # comparisons (3 m per coordinate)
+        return float(sweep_tail or 0.0) + 3.0 * m * d * dout, "lane_op"
     if kernel == "lnq_objective":
-        return dout * d * (4.0 + 4 + 1), "byte"                     # read uT, W, Q
+        return dout * d * (4.0 + 4 + 1), "byte"                     # read U, W, Q
     return 0.0, "unknown"
 
 
-# tcgen05 work per unit of algorithmic work. Both products take F as two fp16 pieces: the
-# class-binned product against m exact one-hot columns per row (two products), the residual
-# product (F w once per call, F r for the objective) against three residual-piece columns (six).
-def hw_flop_factor(layer, kernel):
-    if kernel == "lnq_vgemm":
-        return 2.0
+# Executed tensor-core work of the products that run on tcgen05 (fp16 pieces, fp32 accumulate):
+#   lnq_mgemm: F's two pieces against m one-hot columns per row, over the upper block triangle
+#     (pair blocks of 256 coordinates; the K blocks of 64 from the diagonal block on);
+#   lnq_residual_gemm: three piece products per row (H1 R1, H1 R2, H2 R1) over all of F.
+def executed_tensor_flops(layer, m, kernel):
+    d, dout = layer.d_in, layer.d_out
+    nk, pairs = -(-d // 64), -(-d // 256)
+    if kernel == "lnq_mgemm":
+        kblocks = sum(nk - 4 * ip for ip in range(pairs))
+        return 2.0 * 2 * m * 256 * 64 * kblocks * dout
     if kernel == "lnq_residual_gemm":
-        return 6.0
+        return 2.0 * 3 * (pairs * 256) * (nk * 64) * dout
     return None
 
 
-# DRAM bytes per launch of the dominant kernel from an ncu capture (profiles/
-# dram_traffic_lnq_q_proj_rows1024.md: 1024 rows, scaled by 4 to the 4096-row launch), valid only
-# while the kernel's source is the one that was measured.
-TRAFFIC = {"lnq_vgemm": {"bytes": 4 * (1205451008 + 250055168), "source": "lnq_vgemm.cu",
-                         "sha256": "85b8ca24e3b69b4a4da631df276300ca7d62cb5a9e4e0d90557304f37f301c31"}}
+# DRAM bytes per launch of the dominant kernel from ncu captures of small cases, per row of the
+# launch at a given d_in (scaled by the rows a launch processes), valid only while the kernel's
+# source is the one that was measured.
+TRAFFIC = {}
 
 
-def measured_traffic(kernel):
-    import hashlib
+def measured_traffic(kernel, launches):
+    """Average DRAM bytes per launch over `launches` = [(layer, count)], or None."""
     rec = TRAFFIC.get(kernel)
-    if rec is None or rec["sha256"] is None:
+    if rec is None:
         return None
-    path = os.path.join(os.path.dirname(os.path.abspath(__file__)),
-                        "post_weight_quantization_guided_b200", "csrc", rec["source"])
+    path = os.path.join(ROOT, "post_weight_quantization_guided_b200", "csrc", rec["source"])
     try:
         digest = hashlib.sha256(open(path, "rb").read()).hexdigest()
     except OSError:
         return None
-    return rec["bytes"] if digest == rec["sha256"] else None
+    if digest != rec["sha256"]:
+        return None
+    total, count = 0.0, 0
+    for layer, c in launches:
+        per_row = rec["bytes_per_row"].get(layer.d_in)
+        if per_row is None:
+            return None
+        total += c * per_row * layer.d_out
+        count += c
+    return total / count if count else None
 
 
-def roofline_for(kernel, per_launch_work, unit, avg_ms, peaks, clocks, num_sms):
-    sec = avg_ms / 1e3
+def roofline(work, unit, ms, peaks, fp32_peak):
+    """Roofline object for `work` algorithmic units done in `ms` of device time."""
+    sec = ms / 1e3
     if unit == "flop":
-        peak = peaks["bf16_tflops"]
-        achieved = per_launch_work / sec / 1e12
+        peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+        achieved = work / sec / 1e12
         return {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak}
+                "frac": achieved / peak, "peak_kind": "bf16 dense, sustained (of measured)"}
     if unit == "byte":
         peak = peaks["hbm_gbs"]
-        achieved = per_launch_work / sec / 1e9
+        achieved = work / sec / 1e9
         return {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                "frac": achieved / peak}
-    # FP32 lane operations: 128 FP32 lanes per SM at the maximum SM clock
-    mhz = peaks.get("sm_max_mhz", 1965.0)
-    peak = num_sms * 128 * mhz * 1e6 / 1e12
-    achieved = per_launch_work / sec / 1e12
+                "frac": achieved / peak, "peak_kind": "HBM copy (of measured)"}
+    peak = fp32_peak["sustained"]
+    achieved = work / sec / 1e12
     return {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "Tlane-op/s",
-            "frac": achieved / peak}
+            "frac": achieved / peak,
+            "peak_kind": "FP32 FFMA lane-ops, sustained (of measured, this run's probe)"}
 
 
 # ------------------------------------------------------------------------------------------
-# Oracle (CPU) baseline on a bounded sample
+# FP32 lane-operation peak, measured with the library's FFMA probe
 # ------------------------------------------------------------------------------------------
-def cpu_baseline(layer, X, G, W, F_gpu, budget_s=20.0, threads=None):
-    """Oracle throughput in rows/s on a bounded sample of the same layer, extrapolated:
-    Fisher = measured 64x64 tiles of group 0 scaled to all groups' full blocks; LNQ = measured
-    rows of group 0 (init + all iterations on the GPU's F) scaled to all rows."""
-    from oracle import oracle as orc
-    threads = threads or os.cpu_count()
-    d, n, R = layer.d_in, layer.n, layer.rows_per_group
-    t_start = time.perf_counter()
-    s = np.empty(n)
-    Rg = layer.rows_per_group
-    for r0 in range(0, n, 4096):
-        Gh = G[r0:r0 + 4096, 0:Rg].double().cpu().numpy()
-        s[r0:r0 + Gh.shape[0]] = orc.group_scales(Gh, Gh.shape[0], Rg, 1)[0]
-    t_s = time.perf_counter() - t_start
-    tiles, t_tiles = 0, 0.0
-    rng = np.random.default_rng(0)
-    while t_tiles < budget_s * 0.3 and tiles < 64:
-        i0, k0 = (int(v) for v in rng.integers(0, d - 64, 2))
-        A = X[:, i0:i0 + 64].double().cpu().numpy()
-        B = X[:, k0:k0 + 64].double().cpu().numpy()
-        t0 = time.perf_counter()
-        orc.fisher_block(A, B, s, 1.0)
-        t_tiles += time.perf_counter() - t0
-        tiles += 1
-    fisher_s = (t_tiles / tiles) * layer.groups * (d / 64.0) ** 2 + t_s * layer.groups
-    Fh = F_gpu[0].double().cpu().numpy()
-    Wh = W[:R].double().cpu().numpy()
-    rows, t_rows = 0, 0.0
-    while t_rows < budget_s * 0.6 and rows < R:
-        k = min(threads, R - rows)
-        t0 = time.perf_counter()
-        orc.lnq_rows(Fh, Wh[rows:rows + k], layer.m, layer.iters, init=True, nthreads=threads)
-        t_rows += time.perf_counter() - t0
-        rows += k
-    lnq_s = t_rows / rows * layer.d_out
-    value = layer.d_out / (fisher_s + lnq_s)
-    return {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
-            "sample": (f"Fisher: {tiles} 64x64 tiles of group 0 (n={n}) extrapolated to "
-                       f"{layer.groups} full {d}x{d} blocks; LNQ: {rows} rows of group 0, init + "
-                       f"{layer.iters} iterations on the GPU's F, extrapolated to {layer.d_out} "
-                       f"rows; FP64, {threads} OpenMP threads"),
-            "fisher_s_extrapolated": fisher_s, "lnq_s_extrapolated": lnq_s}
+def measure_fp32_peak(device):
+    from post_weight_quantization_guided_b200 import binding as b
+    sink = torch.zeros(1, dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream(device)
+    iters = 1 << 14
+    for _ in range(3):
+        b.lnq_fp32_probe(iters, sink)
+    torch.cuda.synchronize(device)
+    best = 0.0
+    for _ in range(5):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        ops = b.lnq_fp32_probe(iters, sink)
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        best = max(best, ops / (e0.elapsed_time(e1) / 1e3))
+    # sustained: back-to-back launches for about two seconds
+    per_launch_s = ops / best
+    reps = max(4, int(2.0 / per_launch_s))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    total = 0
+    e0.record(stream)
+    for _ in range(reps):
+        total += b.lnq_fp32_probe(iters, sink)
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    sustained = total / (e0.elapsed_time(e1) / 1e3)
+    return {"burst": best / 1e12, "sustained": sustained / 1e12, "unit": "Tlane-op/s",
+            "how": f"FFMA probe over all SMs: best of 5 launches (burst), {reps} launches "
+                   "back to back (sustained)"}
 
 
 # ------------------------------------------------------------------------------------------
-# Main arm
-# ------------------------------------------------------------------------------------------
-# Multi-rank host logic (one layer per rank, weak scaling, no data-path collective)
+# Multi-rank host logic (one block per rank, weak scaling, no data-path collective)
 # ------------------------------------------------------------------------------------------
 def per_rank_layer(wl, rank):
-    """Rank r quantises its own q_proj-shaped layer: same shapes and distributions, seeds offset by
-    100 r, so the ranks' inputs differ."""
+    """Rank r's q_proj-shaped layer: same shapes and distributions, seeds offset by 100 r."""
     base = wl.Q_PROJ
     return wl.scaled(base, seed=base.seed + 100 * rank, x_seed=base.x_seed + 100 * rank)
+
+
+def per_rank_block(wl, rank, m):
+    """Rank r's decoder block at m codewords: the seeds of every layer offset by 100 r."""
+    return [wl.scaled(L, seed=L.seed + 100 * rank, x_seed=L.x_seed + 100 * rank)
+            for L in wl.decoder_block(m)]
 
 
 def max_over_ranks(values, world, device):
@@ -279,14 +307,411 @@ def job_throughput(world, rows_per_rank, ms_per_step):
 
 
 # ------------------------------------------------------------------------------------------
-def run_ours(args, rank, world, device):
+# Oracle (CPU) baseline on a bounded sample
+# ------------------------------------------------------------------------------------------
+def _oracle_lnq_rate(orc, F0, W0, m, iters, budget_s, threads):
+    """Rows per second of the oracle's LNQ (init + iters) on rows of W0 against F0."""
+    rows, t = 0, 0.0
+    while (t < budget_s or rows == 0) and rows < W0.shape[0]:
+        k = min(threads, W0.shape[0] - rows)
+        t0 = time.perf_counter()
+        orc.lnq_rows(F0, W0[rows:rows + k], m, iters, init=True, nthreads=threads)
+        t += time.perf_counter() - t0
+        rows += k
+    return rows / t, rows
+
+
+def _oracle_tile_seconds(orc, X, s, budget_s, rng, max_tiles=64):
+    """Seconds per 64 x 64 Fisher tile of the oracle over all of X's tokens."""
+    d = X.shape[1]
+    tiles, t = 0, 0.0
+    while (t < budget_s or tiles == 0) and tiles < max_tiles:
+        i0, k0 = (int(v) for v in rng.integers(0, d - 64, 2))
+        A = X[:, i0:i0 + 64].double().cpu().numpy()
+        B = X[:, k0:k0 + 64].double().cpu().numpy()
+        t0 = time.perf_counter()
+        orc.fisher_block(A, B, s, 1.0)
+        t += time.perf_counter() - t0
+        tiles += 1
+    return t / tiles, tiles
+
+
+def block_cpu_estimate(orc, layers16, tile_s, rates):
+    """Extrapolated oracle seconds for one step of the block: every layer's Fisher blocks (64 x 64
+    tiles) plus LNQ of every row at both bit widths. rates[(d_in, m)] = oracle rows/s."""
+    fisher = sum(L.groups * (-(-L.d_in // 64)) ** 2 * tile_s for L in layers16)
+    lnq = sum(L.d_out / rates[(L.d_in, m)] for L in layers16 for m in (16, 8))
+    return fisher, lnq
+
+
+def cpu_baseline_block(layers16, inputs, F_small, budget_s=20.0, threads=None):
+    """Oracle throughput in rows/s on a bounded sample of the block, extrapolated to one step:
+    64 x 64 Fisher tiles at n = 131072 (any tile costs the same) and LNQ rows (init + 5
+    iterations) of a d_in = 4096 and a d_in = 11008 layer at both bit widths, on the GPU's F."""
+    from oracle import oracle as orc
+    threads = threads or os.cpu_count()
+    rng = np.random.default_rng(0)
+    q = layers16[0]
+    X, G, _ = inputs(q)
+    R = q.rows_per_group
+    s = np.empty(q.n)
+    for r0 in range(0, q.n, 8192):
+        Gh = G[r0:r0 + 8192, 0:R].double().cpu().numpy()
+        s[r0:r0 + Gh.shape[0]] = orc.group_scales(Gh, Gh.shape[0], R, 1)[0]
+    tile_s, tiles = _oracle_tile_seconds(orc, X, s, budget_s * 0.25, rng)
+    rates, sampled = {}, []
+    for L in (layers16[0], layers16[-1]):
+        F0 = F_small[L.name]
+        W0 = inputs(L)[2][:L.rows_per_group].double().cpu().numpy()
+        for m in (16, 8):
+            rate, rows = _oracle_lnq_rate(orc, F0, W0, m, L.iters, budget_s * 0.18, threads)
+            rates[(L.d_in, m)] = rate
+            sampled.append(f"{rows} rows at d_in={L.d_in}, m={m}")
+    fisher_s, lnq_s = block_cpu_estimate(orc, layers16, tile_s, rates)
+    rows = 2 * sum(L.d_out for L in layers16)
+    return {"value": rows / (fisher_s + lnq_s), "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": (f"Fisher: {tiles} 64x64 tiles (n={q.n}) extrapolated to every layer's "
+                       f"{q.groups} blocks; LNQ (init + {q.iters} iterations, group 0 rows, on "
+                       f"the GPU's F): {', '.join(sampled)}, extrapolated to all rows of the "
+                       f"block at both bit widths; FP64, {threads} OpenMP threads"),
+            "fisher_s_extrapolated": fisher_s, "lnq_s_extrapolated": lnq_s}
+
+
+# ------------------------------------------------------------------------------------------
+# Main arm: the decoder block
+# ------------------------------------------------------------------------------------------
+class BlockInputs:
+    """Device-resident inputs of a block: X per distinct draw, G and W per layer."""
+
+    def __init__(self, wl, layers, device):
+        self.X, self.G, self.W = {}, {}, {}
+        for L in layers:
+            if L.x_seed not in self.X:
+                self.X[L.x_seed] = wl.make_x(L, device)
+            self.G[L.name] = wl.make_g(L, device)
+            self.W[L.name] = wl.make_w(L, device)
+
+    def __call__(self, L):
+        return self.X[L.x_seed], self.G[L.name], self.W[L.name]
+
+
+def run_block(args, rank, world, device):
     import post_weight_quantization_guided_b200 as lnq
     from post_weight_quantization_guided_b200 import binding as b
     from post_weight_quantization_guided_b200 import workloads as wl
 
     lnq.binding.lib()
-    layer = per_rank_layer(wl, rank)
     torch.cuda.set_device(device)
+    mset = (16, 8)
+    blocks = {m: per_rank_block(wl, rank, m) for m in mset}
+    layers = blocks[16]
+    nl = len(layers)
+    inputs = BlockInputs(wl, layers, device)
+    # outputs per (layer, m); one F buffer (the largest) reused layer by layer
+    out = {}
+    for m in mset:
+        for L in blocks[m]:
+            out[(L.name[:-len(f"_m{m}")], m)] = (
+                torch.empty((L.d_out, m), dtype=torch.float32, device=device),
+                torch.empty((L.d_out, L.d_in), dtype=torch.uint8, device=device),
+                torch.empty(L.d_out, dtype=torch.float64, device=device))
+    base = [L.name[:-len("_m16")] for L in layers]
+    dmax = max(L.d_in for L in layers)
+    Fbuf = torch.empty(max(L.groups * L.d_in * L.d_in for L in layers), dtype=torch.float32,
+                       device=device)
+    st = torch.empty(max(L.d_out for L in layers), dtype=torch.int32, device=device)
+    fsz = max(b.lnq_workspace_size(b.LNQ_OP_BUILD_FISHER, L.n, L.d_in, L.d_out, L.groups, 16)
+              for L in layers)
+    qsz = max(b.lnq_workspace_size(b.LNQ_OP_QUANTIZE_ROWS, 0, L.d_in, L.d_out, L.groups, m)
+              for L in layers for m in mset)
+    ws_f = torch.empty(fsz, dtype=torch.uint8, device=device)
+    ws_q = torch.empty(qsz, dtype=torch.uint8, device=device)
+    ws_i = torch.empty(256, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def F_of(L):
+        return Fbuf[:L.groups * L.d_in * L.d_in].view(L.groups, L.d_in, L.d_in)
+
+    def layer_fisher(k, src=None):
+        L = layers[k]
+        X, G, _ = src(L) if src else inputs(L)
+        lnq.lnq_build_fisher(X, G, L.groups, F=F_of(L), ws=ws_f)
+
+    def layer_lnq(k, m, src=None, dst=None):
+        L = blocks[m][k]
+        W = (src(layers[k]) if src else inputs(layers[k]))[2]
+        C, Q, J = (dst or out)[(base[k], m)]
+        lnq.lnq_init_codebook(W, m, C, Q, ws=ws_i)
+        lnq.lnq_quantize_rows(F_of(L), W, m, L.iters, C, Q, J, st[:L.d_out], ws=ws_q)
+
+    def step(evs=None):
+        if evs is not None:
+            evs[0].record(stream)
+        for k in range(nl):
+            layer_fisher(k)
+            if evs is not None:
+                evs[1 + 3 * k].record(stream)
+            for mi, m in enumerate(mset):
+                layer_lnq(k, m)
+                if evs is not None:
+                    evs[2 + 3 * k + mi].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+    assert b.lnq_workspace_check(ws_f) == b.LNQ_OK and b.lnq_workspace_check(ws_q) == b.LNQ_OK
+    fp32_peak = measure_fp32_peak(device)
+
+    # ---------------------------------------------------------------- device-timed region
+    # The block's inputs (6 GB of X, 11 GB of G) exceed L2 many times over, and every layer
+    # streams through them: no L2 flush is needed between steps.
+    sampler = ClockSampler(device.index) if rank == 0 else None
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(device)
+    if sampler:
+        sampler.start()
+    b.lnq_profile_read()
+    b.lnq_profile_enable(True)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(1 + 3 * nl)]
+           for _ in range(args.steps)]
+    for k in range(args.steps):
+        step(evs[k])
+    torch.cuda.synchronize(device)
+    if world > 1:
+        torch.distributed.barrier()
+    b.lnq_profile_enable(False)
+    prof = b.lnq_profile_read()
+    clocks = sampler.stop() if sampler else None
+    fisher_ms = lnq_ms = 0.0
+    lnq_m_ms = {m: 0.0 for m in mset}
+    total_ms = 0.0
+    for e in evs:
+        total_ms += e[0].elapsed_time(e[-1])
+        for k in range(nl):
+            prev = e[0] if k == 0 else e[3 * k]
+            fisher_ms += prev.elapsed_time(e[1 + 3 * k])
+            for mi, m in enumerate(mset):
+                t = e[1 + 3 * k + mi].elapsed_time(e[2 + 3 * k + mi])
+                lnq_m_ms[m] += t
+                lnq_ms += t
+    assert b.lnq_workspace_check(ws_f) == b.LNQ_OK and b.lnq_workspace_check(ws_q) == b.LNQ_OK
+    for key, (C, Q, J) in out.items():
+        assert bool(torch.isfinite(J).all()), key
+
+    # ---------------------------------------------------------------- sweep counters (untimed)
+    # The run is deterministic, so one more pass reads the moves every timed step made.
+    tails, moves = {}, {}
+    for k in range(nl):
+        layer_fisher(k)
+        for m in mset:
+            layer_lnq(k, m)
+            mv, tl = b.lnq_sweep_counters(ws_q)
+            moves[(k, m)], tails[(k, m)] = mv, tl
+    torch.cuda.synchronize(device)
+    # group 0's Fisher block of two layers for the oracle's LNQ sample
+    F_small = {}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        for L in (layers[0], layers[-1]):
+            X, G, _ = inputs(L)
+            Fs = lnq.lnq_build_fisher(X, G, L.groups, F=F_of(L), ws=ws_f)
+            F_small[L.name] = Fs[0].double().cpu().numpy()
+
+    # ---------------------------------------------------------------- end to end (host buffers)
+    # Every step copies the block's inputs from pinned host memory (each distinct X once, G and W
+    # per layer) and reads every result back (C, Q, J per layer and bit width), all inside the
+    # timed region. Copies run on a second stream with two device buffer sets, so layer k+1's
+    # inputs and layer k's results cross the bus while layer k's kernels run.
+    def pinned(t):
+        return torch.empty(t.shape, dtype=t.dtype, pin_memory=True).copy_(t)
+
+    pin_X = {sd: pinned(x) for sd, x in inputs.X.items()}
+    pin_G = {nm: pinned(g) for nm, g in inputs.G.items()}
+    pin_W = {nm: pinned(w) for nm, w in inputs.W.items()}
+    res_host = {key: [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in v]
+                for key, v in out.items()}
+    dev_X = [torch.empty(max(x.numel() for x in inputs.X.values()), dtype=torch.bfloat16,
+                         device=device) for _ in range(2)]
+    dev_G = [torch.empty(max(g.numel() for g in inputs.G.values()), dtype=torch.bfloat16,
+                         device=device) for _ in range(2)]
+    dev_W = [torch.empty(max(w.numel() for w in inputs.W.values()), dtype=torch.float32,
+                         device=device) for _ in range(2)]
+    res_dev = [{key: [torch.empty_like(t) for t in v] for key, v in out.items()
+                if key[0] == base[k]} for k in range(nl)]
+    h2d = (sum(x.numel() * 2 for x in pin_X.values()) + sum(g.numel() * 2 for g in pin_G.values())
+           + sum(w.numel() * 4 for w in pin_W.values()))
+    d2h = sum(t.numel() * t.element_size() for v in out.values() for t in v)
+    copy = torch.cuda.Stream(device)
+    e2e_steps = max(1, args.steps)
+    nseq = e2e_steps * nl
+    in_ready = [torch.cuda.Event() for _ in range(nseq)]
+    computed = [torch.cuda.Event() for _ in range(nseq)]
+    read_back = [torch.cuda.Event() for _ in range(nseq)]
+    # X draws in sequence order: a layer that shares the previous layer's X reuses its buffer;
+    # a new draw goes to the buffer the draw before the previous one used
+    draw_of, draw_first, draw_last = [], [], []
+    for sq in range(nseq):
+        new = sq == 0 or layers[(sq - 1) % nl].x_seed != layers[sq % nl].x_seed
+        if new:
+            draw_first.append(sq)
+            draw_last.append(sq)
+        draw_of.append(len(draw_first) - 1)
+        draw_last[-1] = sq
+
+    def views(sq):
+        L = layers[sq % nl]
+        u = sq % 2
+        X = dev_X[draw_of[sq] % 2][:L.n * L.d_in].view(L.n, L.d_in)
+        G = dev_G[u][:L.n * L.d_out].view(L.n, L.d_out)
+        W = dev_W[u][:L.d_out * L.d_in].view(L.d_out, L.d_in)
+        return X, G, W
+
+    def copy_inputs(sq):
+        L = layers[sq % nl]
+        X, G, W = views(sq)
+        with torch.cuda.stream(copy):
+            if sq >= 2:
+                copy.wait_event(computed[sq - 2])   # layer sq-2 is done with G/W buffer set
+            dr = draw_of[sq]
+            if draw_first[dr] == sq:
+                if dr >= 2:
+                    copy.wait_event(computed[draw_last[dr - 2]])   # done with this X buffer
+                X.copy_(pin_X[L.x_seed], non_blocking=True)
+            G.copy_(pin_G[L.name], non_blocking=True)
+            W.copy_(pin_W[L.name], non_blocking=True)
+            in_ready[sq].record(copy)
+
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    copy.wait_event(e0)
+    copy_inputs(0)
+    for sq in range(nseq):
+        k = sq % nl
+        if sq + 1 < nseq:
+            copy_inputs(sq + 1)
+        stream.wait_event(in_ready[sq])
+        if sq >= 2:
+            stream.wait_event(read_back[sq - 2])   # earlier results have left their buffers
+        src = (lambda _L, _sq=sq: views(_sq))
+        layer_fisher(k, src)
+        for m in mset:
+            layer_lnq(k, m, src, res_dev[k])
+        computed[sq].record(stream)
+        with torch.cuda.stream(copy):
+            copy.wait_event(computed[sq])
+            for m in mset:
+                for t_h, t_d in zip(res_host[(base[k], m)], res_dev[k][(base[k], m)]):
+                    t_h.copy_(t_d, non_blocking=True)
+            read_back[sq].record(copy)
+    stream.wait_stream(copy)
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    e2e_ms = e0.elapsed_time(e1)
+    for key, (C, Q, J) in out.items():
+        assert np.array_equal(res_host[key][1].numpy(), Q.cpu().numpy()), key
+    del pin_X, pin_G, pin_W, dev_X, dev_G, dev_W, res_dev
+
+    total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], world, device)
+    if rank != 0:
+        return None, None
+    rows_per_step = sum(L.d_out for L in layers) * len(mset)
+    ms_per_step = total_ms / args.steps
+    peaks = load_peaks()
+
+    # ---------------------------------------------------------------- per-kernel roofline
+    kernels = {}
+    all_ms = sum(v[1] for v in prof.values())
+    for name, (launches, ms) in prof.items():
+        work, unit, hw, lw = 0.0, None, 0.0, []
+        for k, L in enumerate(layers):
+            if name in FISHER_KERNELS:
+                c = launches_per_call(name, L, 0)
+                if c:
+                    w, unit = algorithmic_work(L, 16, name)
+                    work += c * w
+                    lw.append((L, c))
+                continue
+            for m in mset:
+                Lm = blocks[m][k]
+                c = launches_per_call(name, Lm, Lm.iters)
+                if not c:
+                    continue
+                tail = tails[(k, m)] / Lm.iters if name == "lnq_sweep" else None
+                w, unit = algorithmic_work(Lm, m, name, tail)
+                work += c * w
+                lw.append((Lm, c))
+                ex = executed_tensor_flops(Lm, m, name)
+                if ex is not None:
+                    hw += c * ex
+        work *= args.steps
+        hw *= args.steps
+        if unit is None or unit == "unknown":
+            continue
+        entry = {"launches_per_step": launches / args.steps, "avg_ms": ms / launches,
+                 "share": ms / all_ms, "roofline": roofline(work, unit, ms, peaks, fp32_peak)}
+        if hw:
+            tens = hw / (ms / 1e3) / 1e12
+            pk = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+            entry["tensor_executed"] = {"achieved": tens, "peak": pk, "unit": "TFLOP/s",
+                                        "frac": tens / pk}
+        entry["_launches"] = lw
+        if abs(sum(c for _, c in lw) * args.steps - launches) > 0:
+            entry["launch_count_mismatch"] = [sum(c for _, c in lw) * args.steps, launches]
+        kernels[name] = entry
+    dominant = max(kernels, key=lambda k: kernels[k]["share"])
+    roof = dict(kernels[dominant]["roofline"])
+    roof["kernel"] = dominant
+    roof["traffic"] = measured_traffic(dominant, kernels[dominant]["_launches"])
+    roof["peak_source"] = peaks["source"]
+    for v in kernels.values():
+        del v["_launches"]
+    fisher_flops = sum(algorithmic_work(L, 16, "fisher_syrk")[0] for L in layers)
+    sweep_moves = {f"m{m}": sum(moves[(k, m)] for k in range(nl)) for m in mset}
+    line = {
+        "metric": METRIC, "value": job_throughput(world, rows_per_step, ms_per_step),
+        "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16+f32",
+        "data": "synthetic (seeded draws with the decoder block's shapes and distributions)",
+        "config": {"workload": "llama2_7b_decoder_block_7_linears_n131072_m16_and_m8",
+                   "layers": [f"{L.name[:-4]} {L.d_in}->{L.d_out}" for L in layers],
+                   "n": layers[0].n, "groups": layers[0].groups, "m": list(mset),
+                   "iters": layers[0].iters, "rows_per_step": world * rows_per_step,
+                   "fisher_per_layer": "built once, used by both bit widths",
+                   "parallelism": f"block-per-gpu x{world}",
+                   "l2": "inputs larger than L2 (17 GB per step streamed), no flush"},
+        "gpu_launches": int(round(sum(v[0] for v in prof.values()) / args.steps)) * args.steps,
+        "e2e": {"value": job_throughput(world, rows_per_step, e2e_ms / e2e_steps), "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "block_ms": {f"m{m}": (fisher_ms + lnq_m_ms[m]) / args.steps for m in mset},
+        "fisher_ms_per_step": fisher_ms / args.steps,
+        "lnq_rows_per_s": {f"m{m}": sum(L.d_out for L in layers) / (lnq_m_ms[m] / args.steps
+                                                                      / 1e3) for m in mset},
+        "fisher_tflops": fisher_flops / (fisher_ms / args.steps / 1e3) / 1e12,
+        "sweep_moves_per_step": sweep_moves,
+        "roofline": roof,
+        "fp32_peak": fp32_peak,
+        "kernels": kernels,
+        "clocks": clocks,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline_block(layers, inputs, F_small,
+                                                  budget_s=args.cpu_budget)
+    return line, fp32_peak
+
+
+# ------------------------------------------------------------------------------------------
+# Secondary workload: one q_proj layer (the consumer and the diagonal variant run on its result)
+# ------------------------------------------------------------------------------------------
+def run_q_proj(args, rank, device, fp32_peak, steps=5, warmup=3):
+    import post_weight_quantization_guided_b200 as lnq
+    from post_weight_quantization_guided_b200 import binding as b
+    from post_weight_quantization_guided_b200 import workloads as wl
+
+    layer = per_rank_layer(wl, rank)
     X, G, W = wl.make_layer(layer, device)
     d, dout, m, it = layer.d_in, layer.d_out, layer.m, layer.iters
     F = torch.empty((layer.groups, d, d), dtype=torch.float32, device=device)
@@ -300,109 +725,44 @@ def run_ours(args, rank, world, device):
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=device)
     stream = torch.cuda.current_stream(device)
 
-    def step(Xs, Gs, Ws):
-        lnq.lnq_build_fisher(Xs, Gs, layer.groups, F=F, ws=ws_f)
-        lnq.lnq_init_codebook(Ws, m, C, Q, ws=ws_i)
-        lnq.lnq_quantize_rows(F, Ws, m, it, C, Q, J, st, ws=ws_q)
+    def step():
+        lnq.lnq_build_fisher(X, G, layer.groups, F=F, ws=ws_f)
+        lnq.lnq_init_codebook(W, m, C, Q, ws=ws_i)
+        lnq.lnq_quantize_rows(F, W, m, it, C, Q, J, st, ws=ws_q)
 
-    for _ in range(args.warmup):
-        step(X, G, W)
+    for _ in range(warmup):
+        step()
     torch.cuda.synchronize(device)
-    assert b.lnq_workspace_check(ws_f) == b.LNQ_OK
-
-    # ---------------------------------------------------------------- device-timed region
-    sampler = ClockSampler(device.index) if rank == 0 else None
-    if world > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize(device)
-    if sampler:
-        sampler.start()
     b.lnq_profile_read()
     b.lnq_profile_enable(True)
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(args.steps)]
-    for k in range(args.steps):
+    ms = 0.0
+    for k in range(steps):
         flush.fill_(k & 0xFF)           # evict L2 between timed steps (untimed)
-        evs[k][0].record(stream)
-        step(X, G, W)
-        evs[k][1].record(stream)
-    torch.cuda.synchronize(device)
-    if world > 1:
-        torch.distributed.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        step()
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        ms += e0.elapsed_time(e1)
     b.lnq_profile_enable(False)
     prof = b.lnq_profile_read()
-    clocks = sampler.stop() if sampler else None
-    step_ms = [a.elapsed_time(z) for a, z in evs]
-    total_ms = float(sum(step_ms))
-    assert b.lnq_workspace_check(ws_f) == b.LNQ_OK
-    Jh = J.cpu().numpy()
-    assert np.all(np.isfinite(Jh)) and int(st.abs().sum()) == 0
+    assert b.lnq_workspace_check(ws_q) == b.LNQ_OK
+    step()
+    mv, tail = b.lnq_sweep_counters(ws_q)
+    peaks = load_peaks()
+    kernels = {}
+    for name, (launches, kms) in prof.items():
+        w, unit = algorithmic_work(layer, m, name, tail / it if name == "lnq_sweep" else None)
+        if unit == "unknown":
+            continue
+        kernels[name] = {"avg_ms": kms / launches, "launches_per_step": launches / steps,
+                         "roofline": roofline(w * launches, unit, kms, peaks, fp32_peak)}
+    res = {"workload": layer.name, "steps": steps, "ms_per_step": ms / steps,
+           "rows_per_s": dout / (ms / steps / 1e3), "sweep_moves": mv, "sweep_tail": tail,
+           "kernels": kernels, "l2": "flushed between timed steps (256 MB write)"}
 
-    # ---------------------------------------------------------------- end to end (host buffers)
-    # Every step copies its inputs from pinned host memory and reads its results back, all inside
-    # the timed region. Copies run on a second stream with two device buffer sets, so step k+1's
-    # inputs and step k's results cross the bus while step k's kernels run (a stream of layers).
-    Xp, Gp, Wp = X.cpu().pin_memory(), G.cpu().pin_memory(), W.cpu().pin_memory()
-    Cp = [torch.empty_like(C, device="cpu").pin_memory() for _ in range(2)]
-    Qp = [torch.empty_like(Q, device="cpu").pin_memory() for _ in range(2)]
-    Jp = [torch.empty_like(J, device="cpu").pin_memory() for _ in range(2)]
-    Xd = [torch.empty_like(X) for _ in range(2)]
-    Gd = [torch.empty_like(G) for _ in range(2)]
-    Wd = [torch.empty_like(W) for _ in range(2)]
-    Cd = [torch.empty_like(C) for _ in range(2)]
-    Qd = [torch.empty_like(Q) for _ in range(2)]
-    Jd = [torch.empty_like(J) for _ in range(2)]
-    h2d = X.numel() * 2 + G.numel() * 2 + W.numel() * 4
-    d2h = C.numel() * 4 + Q.numel() + J.numel() * 8
-    e2e_steps = max(1, args.steps)
-    copy = torch.cuda.Stream(device)
-    in_ready = [torch.cuda.Event() for _ in range(e2e_steps)]
-    computed = [torch.cuda.Event() for _ in range(e2e_steps)]
-    read_back = [torch.cuda.Event() for _ in range(e2e_steps)]
-
-    def copy_inputs(k):
-        u = k % 2
-        with torch.cuda.stream(copy):
-            if k >= 2:
-                copy.wait_event(computed[k - 2])   # step k-2 is done with buffer set u
-            Xd[u].copy_(Xp, non_blocking=True)
-            Gd[u].copy_(Gp, non_blocking=True)
-            Wd[u].copy_(Wp, non_blocking=True)
-            in_ready[k].record(copy)
-
-    if world > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize(device)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    copy.wait_event(e0)
-    copy_inputs(0)
-    for k in range(e2e_steps):
-        u = k % 2
-        if k + 1 < e2e_steps:
-            copy_inputs(k + 1)
-        stream.wait_event(in_ready[k])
-        if k >= 2:
-            stream.wait_event(read_back[k - 2])    # step k-2's results have left buffer set u
-        lnq.lnq_build_fisher(Xd[u], Gd[u], layer.groups, F=F, ws=ws_f)
-        lnq.lnq_init_codebook(Wd[u], m, Cd[u], Qd[u], ws=ws_i)
-        lnq.lnq_quantize_rows(F, Wd[u], m, it, Cd[u], Qd[u], Jd[u], st, ws=ws_q)
-        computed[k].record(stream)
-        with torch.cuda.stream(copy):
-            copy.wait_event(computed[k])
-            Cp[u].copy_(Cd[u], non_blocking=True)
-            Qp[u].copy_(Qd[u], non_blocking=True)
-            Jp[u].copy_(Jd[u], non_blocking=True)
-            read_back[k].record(copy)
-    stream.wait_stream(copy)
-    e1.record(stream)
-    torch.cuda.synchronize(device)
-    e2e_ms = e0.elapsed_time(e1)
-    assert np.array_equal(Qp[(e2e_steps - 1) % 2].numpy(), Q.cpu().numpy())
-
-    # ---------------------------------------------------------------- consumer of (C, Q)
-    # The lookup-table GEMV on the step's codes (batch 1), outside the step's timed region: the
-    # packed codes are cycled through enough copies that they come from HBM, not L2.
+    # the consumer of (C, Q): the lookup-table GEMV on the step's codes (batch 1); the packed codes
+    # are cycled through enough copies that they come from HBM, not L2
     bits = m.bit_length() - 1
     Pk = lnq.lnq_pack_codes(Q, bits)
     copies = max(2, int(3 * 126e6 / (Pk.numel() * 4)) + 1)
@@ -412,7 +772,6 @@ def run_ours(args, rank, world, device):
     for k in range(4):
         lnq.lnq_lut_gemv(xg, Ps[k % copies], C, d, y=yg)
     torch.cuda.synchronize(device)
-    # one CUDA graph of `copies` calls, so the timing sees the device, not the host's call rate
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph):
         for k in range(copies):
@@ -427,13 +786,14 @@ def run_ours(args, rank, world, device):
     g1.record(stream)
     torch.cuda.synchronize(device)
     lut_us = g0.elapsed_time(g1) * 1e3 / (replays * copies)
-    del graph
+    del graph, Ps
     lut_bytes = Pk.numel() * 4 + C.numel() * 4 + d * 4 + dout * 4
-    del Ps
+    res_lut = {"workload": f"{layer.name}: {bits}-bit packed codes, batch 1",
+               "us_per_call": lut_us, "algorithmic_bytes": lut_bytes,
+               "achieved_gbs": lut_bytes / (lut_us * 1e-6) / 1e9, "peak_gbs": peaks["hbm_gbs"],
+               "frac": lut_bytes / (lut_us * 1e-6) / 1e9 / peaks["hbm_gbs"]}
 
-    # ---------------------------------------------------------------- diagonal Fisher blocks
-    # The same LNQ iterations with F_g replaced by its diagonal (one call from the initial state
-    # per repetition, outside the step's timed region).
+    # LNQ with diagonal Fisher blocks (the same iterations, F_g = diag of the step's F_g)
     Fd = torch.diagonal(F, dim1=1, dim2=2).contiguous()
     C0d, Q0d = lnq.lnq_init_codebook(W, m)
     Cx, Qx = C0d.clone(), Q0d.clone()
@@ -442,8 +802,7 @@ def run_ours(args, rank, world, device):
         Cx.copy_(C0d)
         Qx.copy_(Q0d)
         lnq.lnq_quantize_rows_diag(Fd, W, m, it, Cx, Qx, Jx)
-    reps = 10
-    diag_ms = 0.0
+    reps, diag_ms = 10, 0.0
     for _ in range(reps):
         Cx.copy_(C0d)
         Qx.copy_(Q0d)
@@ -453,118 +812,72 @@ def run_ours(args, rank, world, device):
         g1.record(stream)
         torch.cuda.synchronize(device)
         diag_ms += g0.elapsed_time(g1) / reps
-    # W read, codes read and written, codebooks read and written, objective written
     diag_bytes = dout * d * (4 + 1 + 1) + 2 * dout * m * 4 + dout * 8 + layer.groups * d * 4
-    del Fd, C0d, Q0d, Cx, Qx, Jx
-
-    # ---------------------------------------------------------------- max over ranks
-    total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], world, device)
-
-    if rank != 0:
-        return None
-    ms_per_step = total_ms / args.steps
-    value = job_throughput(world, dout, ms_per_step)
-    e2e_value = job_throughput(world, dout, e2e_ms / e2e_steps)
-
-    peaks = load_peaks()
-    num_sms = torch.cuda.get_device_properties(device).multi_processor_count
-    kernels = {}
-    for name, (launches, ms) in prof.items():
-        per_step = launches / args.steps
-        per_launch, unit = algorithmic_work(layer, name, launches, 0.0)
-        avg = ms / launches
-        kernels[name] = {"launches_per_step": per_step, "avg_ms": avg,
-                         "share": ms / sum(v[1] for v in prof.values()),
-                         "roofline": roofline_for(name, per_launch, unit, avg, peaks, clocks,
-                                                  num_sms)}
-        hf = hw_flop_factor(layer, name)
-        if hf is not None:
-            kernels[name]["roofline"]["hw_flop_factor"] = hf
-            kernels[name]["roofline"]["hw_frac"] = kernels[name]["roofline"]["frac"] * hf
-    dominant = max(kernels, key=lambda k: kernels[k]["share"])
-    roof = dict(kernels[dominant]["roofline"])
-    roof["kernel"] = dominant
-    roof["traffic"] = measured_traffic(dominant)
-    roof["peak_source"] = peaks["source"]
-    fisher_ms = sum(kernels[k]["avg_ms"] for k in ("token_stats", "guided_operands", "fisher_syrk")
-                    if k in kernels) or None
-    line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16+f32",
-        "data": "synthetic (seeded draws with the q_proj layer's shapes and distributions)",
-        "config": {"workload": layer.name, "d_in": d, "d_out": dout, "n": layer.n,
-                   "groups": layer.groups, "m": m, "iters": it,
-                   "rows_per_step": world * dout, "parallelism": f"layer-per-gpu x{world}",
-                   "l2": "flushed between timed steps (256 MB write)"},
-        "gpu_launches": int(sum(v[0] for v in prof.values()) / args.steps) * args.steps,
-        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h},
-        "roofline": roof,
-        # the whole Fisher build (statistics, operands, SYRK) at the unique-entry flop count
-        "fisher_tflops": (layer.groups * layer.n * d * (d + 1) / (fisher_ms / 1e3) / 1e12)
-        if fisher_ms else None,
-        "kernels": kernels,
-        "clocks": clocks,
-        # the consumer of (C, Q): y = x W^T read through the codebooks from the packed codes
-        "lut_gemv": {"workload": f"{layer.name}: {bits}-bit packed codes, batch 1",
-                     "us_per_call": lut_us, "algorithmic_bytes": lut_bytes,
-                     "achieved_gbs": lut_bytes / (lut_us * 1e-6) / 1e9,
-                     "peak_gbs": peaks["hbm_gbs"],
-                     "frac": lut_bytes / (lut_us * 1e-6) / 1e9 / peaks["hbm_gbs"]},
-        # LNQ with diagonal Fisher blocks (the same iterations, F_g = diag of the step's F_g)
-        "lnq_diag": {"workload": f"{layer.name}: {it} iterations, m = {m}",
-                     "ms_per_call": diag_ms, "rows_per_s": dout / (diag_ms / 1e3),
-                     "algorithmic_bytes": diag_bytes,
-                     "achieved_gbs": diag_bytes / (diag_ms * 1e-3) / 1e9,
-                     "frac_hbm": diag_bytes / (diag_ms * 1e-3) / 1e9 / peaks["hbm_gbs"]},
-    }
-    if world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(layer, X, G, W, F, budget_s=args.cpu_budget)
-    return line
+    res_diag = {"workload": f"{layer.name}: {it} iterations, m = {m}", "ms_per_call": diag_ms,
+                "rows_per_s": dout / (diag_ms / 1e3), "algorithmic_bytes": diag_bytes,
+                "achieved_gbs": diag_bytes / (diag_ms * 1e-3) / 1e9,
+                "frac_hbm": diag_bytes / (diag_ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}
+    return res, res_lut, res_diag
 
 
+# ------------------------------------------------------------------------------------------
+# Reference arm: the oracle on the host cores
+# ------------------------------------------------------------------------------------------
 def run_reference(args, rank, world):
     """The oracle (plain FP64 CPU code) on the host cores, same metric and workload, each step a
-    bounded sample extrapolated to the whole layer."""
+    bounded sample extrapolated to the whole block."""
     if rank != 0:
         return None
     from post_weight_quantization_guided_b200 import workloads as wl
     from oracle import oracle as orc
     orc.build()
-    layer = wl.Q_PROJ
-    X, G, W = wl.make_layer(layer, "cpu")
-    d = layer.d_in
-    s = orc.group_scales(G[:, :layer.rows_per_group].double().numpy(), layer.n,
-                         layer.rows_per_group, 1)[0]
-    # Untimed preparation: group 0's Fisher block as input for the LNQ sample (a plain float64
-    # product; the oracle's own Fisher routine is what the timed sample below measures).
-    Xh = X.double().numpy()
-    F0 = (Xh * s[:, None]).T @ Xh
-    vals = []
-    for k in range(args.warmup + args.steps):
-        t0 = time.perf_counter()
-        A = X[:, 0:64].double().numpy()
-        orc.fisher_block(A, A, s, 1.0)
-        t_tile = time.perf_counter() - t0
-        t1 = time.perf_counter()
-        orc.lnq_rows(F0, W[:8].double().numpy(), layer.m, layer.iters, init=True, nthreads=0)
-        t_rows = time.perf_counter() - t1
-        per_layer = t_tile * layer.groups * (d / 64.0) ** 2 + t_rows / 8 * layer.d_out
-        if k >= args.warmup:
-            vals.append(layer.d_out / per_layer)
-    value = statistics.median(vals)
+    layers = wl.decoder_block(16)
+    q, down = layers[0], layers[-1]
     threads = os.cpu_count()
+    # Untimed preparation: the q layer's inputs, and for the LNQ sample group 0's Fisher block of
+    # the q and down layers over their first 8192 tokens (a plain float64 product; the sample's
+    # cost per row does not depend on n).
+    Xq = wl.make_x(q)
+    Gq = wl.make_g(q)
+    Rq = q.rows_per_group
+    s = orc.group_scales(Gq[:, :Rq].double().numpy(), q.n, Rq, 1)[0]
+    prepared = {}
+    for L in (q, down):
+        Ls = wl.scaled(L, n=8192)
+        X = wl.make_x(Ls).double().numpy()
+        Gs = wl.make_g(Ls)
+        ss = orc.group_scales(Gs[:, :L.rows_per_group].double().numpy(), 8192,
+                              L.rows_per_group, 1)[0]
+        prepared[L.d_in] = ((X * ss[:, None]).T @ X,
+                            wl.make_w(L)[:threads].double().numpy())
+    vals = []
+    rng = np.random.default_rng(0)
+    for k in range(args.warmup + args.steps):
+        tile_s, _ = _oracle_tile_seconds(orc, Xq, s, 0.0, rng, max_tiles=1)
+        rates = {}
+        for dd, (F0, W0) in prepared.items():
+            for m in (16, 8):
+                rows = 1 if dd > 4096 else 2
+                t0 = time.perf_counter()
+                orc.lnq_rows(F0, W0[:rows], m, q.iters, init=True, nthreads=threads)
+                rates[(dd, m)] = rows / (time.perf_counter() - t0)
+        fisher_s, lnq_s = block_cpu_estimate(orc, layers, tile_s, rates)
+        if k >= args.warmup:
+            vals.append(2 * sum(L.d_out for L in layers) / (fisher_s + lnq_s))
+    value = statistics.median(vals)
+    sample = ("per step: one 64x64 Fisher tile (n=131072), LNQ (init + 5 iterations) of 2 rows at "
+              "d_in=4096 and 1 row at d_in=11008 for m=16 and m=8 (one OpenMP thread per row), "
+              "extrapolated to the whole block at both bit widths")
     return {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": 1e3 * layer.d_out / value, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "impl": "reference",
-            "config": {"workload": layer.name, "d_in": d, "d_out": layer.d_out, "n": layer.n,
-                       "groups": layer.groups, "m": layer.m, "iters": layer.iters},
+            "ms_per_step": 1e3 * 2 * sum(L.d_out for L in layers) / value,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": {"workload": "llama2_7b_decoder_block_7_linears_n131072_m16_and_m8",
+                       "layers": [f"{L.name[:-4]} {L.d_in}->{L.d_out}" for L in layers],
+                       "n": q.n, "groups": q.groups, "m": [16, 8], "iters": q.iters},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
-                             "sample": "per step: one 64x64 Fisher tile (n=16384) and 8 rows "
-                                       "of LNQ (init + 3 iterations), extrapolated to the layer"},
+                             "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
 
@@ -576,6 +889,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-q-proj", action="store_true",
+                    help="skip the secondary single-layer workload")
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", "0"))
@@ -592,7 +907,12 @@ def main():
                                              device_id=torch.device("cuda", local))
     device = torch.device("cuda", local)
     try:
-        line = run_ours(args, rank, world, device)
+        line, fp32_peak = run_block(args, rank, world, device)
+        if not args.no_q_proj and rank == 0:
+            torch.cuda.empty_cache()
+            qp = run_q_proj(args, rank, device, fp32_peak)
+            if line is not None:
+                line["q_proj"], line["lut_gemv"], line["lnq_diag"] = qp
     finally:
         if world > 1:
             torch.distributed.destroy_process_group()

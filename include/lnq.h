@@ -29,8 +29,11 @@
  *
  * Conventions for every entry point:
  *   - Pointers: every array pointer is DEVICE memory that the caller allocates and owns. The
- *     library allocates no device memory. It keeps no state between calls except a cached TMA
- *     encoder function pointer.
+ *     library allocates no device memory at run time. Its state between calls is a cached TMA
+ *     encoder function pointer, per-kernel occupancy figures, and, for lnq_build_fisher_noalloc
+ *     only, a static device array of LNQ_NOALLOC_SCRATCH_BYTES that is part of the library image
+ *     (every GPU that loads the library holds it) with its device address cached per device.
+ *     Calls that use that array must not overlap on the GPU.
  *   - Layout: all matrices are dense and row-major with no padding.
  *       X  [n][d_in]      bf16, passed as raw 16-bit patterns (uint16_t)
  *       G  [n][d_out]     bf16 (raw 16-bit), or NULL
@@ -96,10 +99,16 @@ LNQ_API size_t lnq_workspace_size(lnq_op op, int64_t n, int64_t d_in, int64_t d_
  *   X      [n][d_in] bf16; G [n][d_out] bf16 or NULL (all gradients 1, requires groups == 1)
  *   alpha  overall scale (1 gives X^T X for G == NULL; 1/n gives the blocks of the equation)
  *   F      out, [groups][d_in][d_in] fp32, both triangles written
- * Requirements: n >= 1; d_in >= 1 and d_in % 8 == 0; d_out >= 1; groups >= 1 and
- * d_out % groups == 0; X, G and F 16-byte aligned. Arithmetic: the s_g reduction in fp32. The
- * products run on tensor cores with bf16 operands and fp32 accumulation. When G != NULL, the
- * operand is bf16(sqrt(s_g[t]) * X[t][:]), rounded once. */
+ * Requirements: n >= 1; d_in >= 1 and d_in % 8 == 0 (X's rows are read by TMA, whose row
+ * strides must be multiples of 16 bytes); d_out >= 1; groups >= 1 and d_out % groups == 0; X, G
+ * and F 16-byte aligned.
+ * Arithmetic: s_g[t] is reduced in fp32. The products run on tensor cores with fp32
+ * accumulation. With G == NULL both operands are X in bf16 (exact products). With G != NULL the
+ * operands are one-sided fp16 with power-of-two scales: A[t] = X[t] 2^-e_t (exact; 2^e_t is the
+ * smallest power of two >= max_i |X[t][i]|) and B_g[t] = fp16(s_g[t] X[t] 2^(e_t - E_g)) (one
+ * rounding, 2^-11 relative; 2^E_g bounds s_g[t] max_i X[t][i]^2 over the tokens), so that
+ * F_g = alpha 2^E_g A^T B_g and every entry is within about 5e-4 sqrt(F_ii F_kk) of the exact
+ * value, even for a single token. */
 LNQ_API lnq_status lnq_build_fisher(const uint16_t *X, const uint16_t *G, int64_t n, int64_t d_in,
                             int64_t d_out, int groups, float alpha, float *F, void *ws,
                             size_t ws_bytes, lnq_stream_t stream);
@@ -116,8 +125,12 @@ LNQ_API lnq_status lnq_build_fisher(const uint16_t *X, const uint16_t *G, int64_
  *   that loads the library holds it until the process exits. The call itself allocates nothing
  *   (no cudaMalloc, no cudaFree, no allocating library routine).
  *   Set-up: the first call on each device looks up the array's device address
- *   (cudaGetSymbolAddress) with that device current. Make that first call before any stream
- *   capture, and call with the device that owns `stream` current.
+ *   (cudaGetSymbolAddress) with that device current and caches it. Make that first call before
+ *   any stream capture, and call with the device that owns `stream` current. The cached address
+ *   does not survive a cudaDeviceReset of that device: do not use the library across one.
+ *   Errors: a bounded in-kernel wait that gives up sets the flag in the array's header, which the
+ *   next call clears; read it with lnq_workspace_check(NULL, stream) after the call and before
+ *   the next one (LNQ_ERR_TIMEOUT means F is incomplete).
  *   Sharing: all calls share the one array, which keeps the last call's contents. Each call
  *   clears what must start at zero and overwrites the rest, but calls that overlap on the GPU
  *   (different streams or host threads) race on the array, so serialise them.
@@ -171,14 +184,37 @@ LNQ_API lnq_status lnq_quantize_rows_diag(const float *Fd, int groups, const flo
                                           uint8_t *Q, double *J_out, int32_t *row_status,
                                           lnq_stream_t stream);
 
-/* Per-row objective J[j] = r^T F_g r with r = C[j][Q[j]] - W[j] (fp32 products, fp64 sums). */
+/* Per-row objective J[j] = r^T F_g r with r = C[j][Q[j]] - W[j] ("GuidedQuant" blog, GuidedQuant
+ * section, third equation: the guided output error of row j is n r^T F_j r; LNQ section, first
+ * equation, with F_g in place of X^T X). Row j uses F[j / (d_out/groups)].
+ *   W, C, Q  as lnq_quantize_rows (read only); J [d_out] fp64 out
+ * Arithmetic: u = F r on tensor cores (F and r as fp16 pieces, fp32 accumulation), then J = r^T u
+ * with fp64 sums. Requirements and errors as lnq_quantize_rows; `ws` as for
+ * LNQ_OP_OBJECTIVE. */
 LNQ_API lnq_status lnq_objective(const float *F, int groups, const float *W, const float *C,
                          const uint8_t *Q, int64_t d_out, int64_t d_in, int m, double *J,
                          void *ws, size_t ws_bytes, lnq_stream_t stream);
 
 /* Synchronises `stream`, then reads and clears the flag that a bounded in-kernel wait sets when it
- * gives up. Returns LNQ_OK, LNQ_ERR_TIMEOUT or LNQ_ERR_CUDA. */
+ * gives up. ws == NULL checks the static scratch of lnq_build_fisher_noalloc on the current
+ * device. Returns LNQ_OK, LNQ_ERR_TIMEOUT or LNQ_ERR_CUDA. */
 LNQ_API lnq_status lnq_workspace_check(void *ws, lnq_stream_t stream);
+
+/* Work counters of the assignment sweeps of the last lnq_quantize_rows call that used `ws` (LNQ
+ * section, the coordinate loop): *moves = coordinates that changed codeword, summed over rows and
+ * iterations; *tail = the sum over those moves of (d_in - i), i the 0-based coordinate, which is
+ * the number of entries of u = F r that each move updates. Synchronises `stream`. Returns
+ * LNQ_ERR_INVALID_ARG for a NULL or misaligned ws or NULL outputs. */
+LNQ_API lnq_status lnq_sweep_counters(const void *ws, lnq_stream_t stream, int64_t *moves,
+                                      int64_t *tail);
+
+/* Measurement aid (no counterpart on the pages): enqueues a kernel of independent FP32 FFMA chains
+ * over every SM (8 blocks of 256 threads per SM, each thread `iters` x 8 FFMAs) so that the caller
+ * can time the device's FP32 lane-operation rate with CUDA events on `stream`. *lane_ops receives
+ * the number of FFMAs the launch performs. sink: device memory of at least one float, written
+ * never in practice (it keeps the chains live). Requirements: iters a positive multiple of 16. */
+LNQ_API lnq_status lnq_fp32_probe(int64_t iters, float *sink, int64_t *lane_ops,
+                                  lnq_stream_t stream);
 
 /* ---- Consumer of (C, Q): packed codes and the lookup-table GEMV ----------------------------
  * "GuidedQuant" (jinukkim.me blog), LNQ section, last sentence (LNQ runs on SqueezeLLM's CUDA

@@ -4,4 +4,6 @@ from .binding import (LNQ_OP_BUILD_FISHER, LNQ_OP_INIT_CODEBOOK, LNQ_OP_OBJECTIV
                       LNQ_OP_QUANTIZE_ROWS, LnqError, lnq_build_fisher, lnq_init_codebook,
                       lnq_objective, lnq_quantize_rows, lnq_set_wait_limit, lnq_status_string,
                       lnq_workspace_check, lnq_workspace_size, lnq_packed_words,
-                      lnq_pack_codes, lnq_lut_gemv, lnq_quantize_rows_diag)
+                      lnq_pack_codes, lnq_lut_gemv, lnq_quantize_rows_diag,
+                      lnq_sweep_counters, lnq_fp32_probe, lnq_build_fisher_noalloc,
+                      lnq_noalloc_check)

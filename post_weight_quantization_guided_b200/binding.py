@@ -23,7 +23,8 @@ LNQ_OP_BUILD_FISHER, LNQ_OP_INIT_CODEBOOK, LNQ_OP_QUANTIZE_ROWS, LNQ_OP_OBJECTIV
 EXPORTED = ("lnq_workspace_size", "lnq_build_fisher", "lnq_init_codebook", "lnq_quantize_rows",
             "lnq_objective", "lnq_workspace_check", "lnq_set_wait_limit", "lnq_status_string",
             "lnq_profile_enable", "lnq_profile_read", "lnq_build_fisher_noalloc",
-            "lnq_packed_words", "lnq_pack_codes", "lnq_lut_gemv", "lnq_quantize_rows_diag")
+            "lnq_packed_words", "lnq_pack_codes", "lnq_lut_gemv", "lnq_quantize_rows_diag",
+            "lnq_sweep_counters", "lnq_fp32_probe")
 
 _lib = None
 _VP, _I64, _INT, _SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
@@ -70,9 +71,12 @@ def lib():
         L.lnq_lut_gemv.argtypes = [_VP, _I64, _VP, _VP, _I64, _I64, _INT, _VP, _VP]
         L.lnq_quantize_rows_diag.argtypes = [_VP, _INT, _VP, _I64, _I64, _INT, _INT, _VP, _VP,
                                              _VP, _VP, _VP]
+        L.lnq_sweep_counters.argtypes = [_VP, _VP, ctypes.POINTER(_I64), ctypes.POINTER(_I64)]
+        L.lnq_fp32_probe.argtypes = [_I64, _VP, ctypes.POINTER(_I64), _VP]
         for name in ("lnq_build_fisher", "lnq_build_fisher_noalloc", "lnq_init_codebook",
                      "lnq_quantize_rows", "lnq_objective", "lnq_workspace_check",
-                     "lnq_pack_codes", "lnq_lut_gemv", "lnq_quantize_rows_diag"):
+                     "lnq_pack_codes", "lnq_lut_gemv", "lnq_quantize_rows_diag",
+                     "lnq_sweep_counters", "lnq_fp32_probe"):
             getattr(L, name).restype = _INT
         _lib = L
     return _lib
@@ -167,6 +171,12 @@ def lnq_build_fisher_noalloc(X: torch.Tensor, G: Optional[torch.Tensor], groups:
     return F
 
 
+def lnq_noalloc_check(stream=None) -> int:
+    """Synchronises the stream and reports (LNQ_OK / LNQ_ERR_TIMEOUT) whether a bounded wait of the
+    last lnq_build_fisher_noalloc call on the current device gave up; clears the flag."""
+    return int(lib().lnq_workspace_check(None, _stream(stream)))
+
+
 def lnq_init_codebook(W: torch.Tensor, m: int, C: Optional[torch.Tensor] = None,
                       Q: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
                       stream=None):
@@ -246,9 +256,26 @@ def lnq_objective(F: torch.Tensor, W: torch.Tensor, C: torch.Tensor, Q: torch.Te
     return J
 
 
-def lnq_workspace_check(ws: torch.Tensor, stream=None) -> int:
-    """Synchronises the stream and returns LNQ_OK or LNQ_ERR_TIMEOUT (see include/lnq.h)."""
+def lnq_workspace_check(ws: Optional[torch.Tensor], stream=None) -> int:
+    """Synchronises the stream and returns LNQ_OK or LNQ_ERR_TIMEOUT (see include/lnq.h); ws None
+    checks the static scratch of lnq_build_fisher_noalloc on the current device."""
     return int(lib().lnq_workspace_check(_ptr(ws), _stream(stream)))
+
+
+def lnq_sweep_counters(ws: torch.Tensor, stream=None):
+    """(moves, tail) of the sweeps of the last lnq_quantize_rows call on `ws` (synchronises)."""
+    mv, tl = ctypes.c_int64(0), ctypes.c_int64(0)
+    _check(lib().lnq_sweep_counters(_ptr(ws), _stream(stream), ctypes.byref(mv),
+                                    ctypes.byref(tl)), "lnq_sweep_counters")
+    return int(mv.value), int(tl.value)
+
+
+def lnq_fp32_probe(iters: int, sink: torch.Tensor, stream=None) -> int:
+    """Enqueues the FP32 FFMA probe kernel; returns the number of FFMAs it performs."""
+    ops = ctypes.c_int64(0)
+    _check(lib().lnq_fp32_probe(int(iters), _ptr(sink), ctypes.byref(ops), _stream(stream)),
+           "lnq_fp32_probe")
+    return int(ops.value)
 
 
 def lnq_packed_words(d_in: int, bits: int) -> int:

@@ -13,15 +13,13 @@
 
 namespace lnq {
 
-// Kernels and launchers defined in fisher.cu / lnq.cu.
+// Kernels and launchers defined in fisher.cu.
 __global__ void token_stats_kernel(const __nv_bfloat16 *, const __nv_bfloat16 *, int64_t, int64_t,
                                    int64_t, int, float *, float *, unsigned *);
-__global__ void guided_operands_kernel(const __nv_bfloat16 *, const float *, const float *,
-                                       const unsigned *, int64_t, int64_t, int, __half *,
-                                       __half *);
-cudaError_t fisher_syrk(const void *A, const void *B, bool f16, const unsigned *pimax, int64_t n,
-                        int64_t d, int groups, float alpha, float *F, DeviceErr err,
-                        cudaStream_t s, int num_sms);
+__global__ void token_scales_kernel(int64_t, int, float *, float *, const unsigned *);
+cudaError_t fisher_syrk(const __nv_bfloat16 *X, const float *S, const float *M,
+                        const unsigned *pimax, int64_t n, int64_t d, int groups, float alpha,
+                        float *F, DeviceErr err, cudaStream_t s, int num_sms);
 
 static std::atomic<long long> g_wait_limit{kDefaultWaitLimit};
 
@@ -40,32 +38,29 @@ static bool valid_m(int m) { return m == 2 || m == 4 || m == 8 || m == 16; }
 
 // Workspace layout (all offsets 256-byte aligned):
 //   BUILD_FISHER:   header | S [groups][n] f32 | M [n] f32 | pimax [groups] u32
-//                   | A [n][d_in] f16 | B [groups][n][d_in] f16
 //   QUANTIZE_ROWS:  header | status [d_out] i32 | Fh [groups][2][d_in][ld] f16 (ld = d_in
 //                   rounded up to a multiple of 8) | fexp [groups][d_in] i32 | rexp [d_out] i32
-//                   | V [d_out][d_in][m] f32 | U [d_out][d_in] f32 (u = F r) | dC [d_out][m] f32
-//                   | sweep history [CTAs][2 ceil(d_in / 128)][3][4 KB] (Delta pieces)
-//                   | right-operand image of the product [row tiles][K blocks][N][64] 16-bit
-//   OBJECTIVE:      the same layout (status, V and dC unused)
+//                   | Sb [2 ceil(d_in / 256)][d_out][m][m] f32 (class-binned partial sums)
+//                   | U [d_out][d_in] f32 (-F w) | Ur [d_out][d_in] f32 (u = F r)
+//                   | sweep history [CTAs][2 ceil(d_in / 128)][2][4 KB] (Delta pieces)
+//                   | right-operand image of the products [row tiles][K blocks][256][64] 16-bit
+//   OBJECTIVE:      the same layout (status, Sb and U unused)
 //   INIT:           header
 struct FisherWs {
-    size_t s_off, m_off, pi_off, a_off, b_off, total;
+    size_t s_off, m_off, pi_off, total;
 };
-static FisherWs fisher_ws(int64_t n, int64_t d_in, int groups)
+static FisherWs fisher_ws(int64_t n, int groups)
 {
     FisherWs w;
     w.s_off = kWsHeader;
     w.m_off = align_up(w.s_off + static_cast<size_t>(groups) * n * sizeof(float), 256);
     w.pi_off = align_up(w.m_off + static_cast<size_t>(n) * sizeof(float), 256);
-    w.a_off = align_up(w.pi_off + static_cast<size_t>(groups) * sizeof(unsigned), 256);
-    w.b_off = align_up(w.a_off + static_cast<size_t>(n) * d_in * 2, 256);
-    w.total = align_up(w.b_off + static_cast<size_t>(groups) * n * d_in * 2, 256);
+    w.total = align_up(w.pi_off + static_cast<size_t>(groups) * sizeof(unsigned), 256);
     return w;
 }
 
 struct LnqWs {
-    size_t st_off, fh_off, fexp_off, rexp_off, v_off, ut_off, dc_off, hist_off, img_off,
-        total;
+    size_t st_off, fh_off, fexp_off, rexp_off, sb_off, u_off, ur_off, hist_off, img_off, total;
 };
 static LnqWs lnq_ws(int64_t d_in, int64_t d_out, int groups, int m)
 {
@@ -75,10 +70,10 @@ static LnqWs lnq_ws(int64_t d_in, int64_t d_out, int groups, int m)
     const size_t ld = static_cast<size_t>((d_in + 7) / 8 * 8);  // fp16 piece row stride
     w.fexp_off = align_up(w.fh_off + static_cast<size_t>(groups) * 2 * d_in * ld * 2, 256);
     w.rexp_off = align_up(w.fexp_off + static_cast<size_t>(groups) * d_in * 4, 256);
-    w.v_off = align_up(w.rexp_off + static_cast<size_t>(d_out) * 4, 256);
-    w.ut_off = align_up(w.v_off + static_cast<size_t>(d_out) * d_in * m * 4, 256);
-    w.dc_off = align_up(w.ut_off + static_cast<size_t>(d_in) * d_out * 4, 256);
-    w.hist_off = align_up(w.dc_off + static_cast<size_t>(d_out) * m * 4, 256);
+    w.sb_off = align_up(w.rexp_off + static_cast<size_t>(d_out) * 4, 256);
+    w.u_off = align_up(w.sb_off + lnq_binned_bytes(d_in, d_out, m), 256);
+    w.ur_off = align_up(w.u_off + static_cast<size_t>(d_in) * d_out * 4, 256);
+    w.hist_off = align_up(w.ur_off + static_cast<size_t>(d_in) * d_out * 4, 256);
     w.img_off = align_up(w.hist_off + lnq_sweep_history_bytes(d_in, d_out, groups), 256);
     w.total = align_up(w.img_off + lnq_vgemm_image_bytes(d_in, d_out, groups, m), 256);
     return w;
@@ -92,9 +87,9 @@ static LnqWorkspace carve(void *ws, const LnqWs &lay)
     w.Fh = reinterpret_cast<__half *>(b + lay.fh_off);
     w.fexp = reinterpret_cast<int32_t *>(b + lay.fexp_off);
     w.rexp = reinterpret_cast<int32_t *>(b + lay.rexp_off);
-    w.V = reinterpret_cast<float *>(b + lay.v_off);
-    w.U = reinterpret_cast<float *>(b + lay.ut_off);
-    w.dC = reinterpret_cast<float *>(b + lay.dc_off);
+    w.Sb = reinterpret_cast<float *>(b + lay.sb_off);
+    w.U = reinterpret_cast<float *>(b + lay.u_off);
+    w.Ur = reinterpret_cast<float *>(b + lay.ur_off);
     w.hist = b + lay.hist_off;
     w.img = reinterpret_cast<uint16_t *>(b + lay.img_off);
     return w;
@@ -131,7 +126,7 @@ size_t lnq_workspace_size(lnq_op op, int64_t n, int64_t d_in, int64_t d_out, int
     case LNQ_OP_BUILD_FISHER:
         if (n < 1 || d_in < 1 || groups < 1)
             return 0;
-        return fisher_ws(n, d_in, groups).total;
+        return fisher_ws(n, groups).total;
     case LNQ_OP_QUANTIZE_ROWS:
     case LNQ_OP_OBJECTIVE:
         if (d_out < 1 || d_in < 1 || groups < 1 || !valid_m(m))
@@ -159,7 +154,7 @@ lnq_status lnq_build_fisher(const uint16_t *X, const uint16_t *G, int64_t n, int
         (G != nullptr && !aligned16(G)) || (G == nullptr && groups != 1) ||
         n > (int64_t(1) << 31) - 64 || d_in > (int64_t(1) << 30))
         return LNQ_ERR_INVALID_ARG;
-    const FisherWs lay = fisher_ws(n, d_in, groups);
+    const FisherWs lay = fisher_ws(n, groups);
     const size_t need = (G == nullptr) ? kWsHeader : lay.total;
     lnq_status st = check_ws(ws, ws_bytes, need);
     if (st != LNQ_OK)
@@ -175,8 +170,6 @@ lnq_status lnq_build_fisher(const uint16_t *X, const uint16_t *G, int64_t n, int
         float *S = reinterpret_cast<float *>(base + lay.s_off);
         float *M = reinterpret_cast<float *>(base + lay.m_off);
         unsigned *pimax = reinterpret_cast<unsigned *>(base + lay.pi_off);
-        __half *A = reinterpret_cast<__half *>(base + lay.a_off);
-        __half *B = reinterpret_cast<__half *>(base + lay.b_off);
         if (cudaMemsetAsync(pimax, 0, static_cast<size_t>(groups) * sizeof(unsigned), s) !=
             cudaSuccess)
             return LNQ_ERR_CUDA;
@@ -187,17 +180,17 @@ lnq_status lnq_build_fisher(const uint16_t *X, const uint16_t *G, int64_t n, int
                                  0, s>>>(Xb, reinterpret_cast<const __nv_bfloat16 *>(G), n, d_in,
                                          d_out, groups, S, M, pimax);
         }
-        const int64_t vecs = n * (d_in / 8);
         {
-            KernelTimer timer("guided_operands", s);
-            guided_operands_kernel<<<static_cast<unsigned>((vecs + threads - 1) / threads),
-                                     threads, 0, s>>>(Xb, S, M, pimax, n, d_in, groups, A, B);
+            KernelTimer timer("token_scales", s);
+            token_scales_kernel<<<static_cast<unsigned>((n + threads - 1) / threads), threads, 0,
+                                  s>>>(n, groups, S, M, pimax);
         }
         if (cudaGetLastError() != cudaSuccess)
             return LNQ_ERR_CUDA;
-        e = fisher_syrk(A, B, true, pimax, n, d_in, groups, alpha, F, err, s, device_sm_count());
+        e = fisher_syrk(Xb, S, M, pimax, n, d_in, groups, alpha, F, err, s, device_sm_count());
     } else {
-        e = fisher_syrk(Xb, Xb, false, nullptr, n, d_in, 1, alpha, F, err, s, device_sm_count());
+        e = fisher_syrk(Xb, nullptr, nullptr, nullptr, n, d_in, 1, alpha, F, err, s,
+                        device_sm_count());
     }
     if (e == cudaErrorNotSupported)
         return LNQ_ERR_UNSUPPORTED;
@@ -317,8 +310,12 @@ lnq_status lnq_lut_gemv(const float *x, int64_t nb, const uint32_t *P, const flo
 
 lnq_status lnq_workspace_check(void *ws, lnq_stream_t stream)
 {
-    if (ws == nullptr)
-        return LNQ_ERR_WORKSPACE;
+    if (ws == nullptr) {
+        // the static scratch of lnq_build_fisher_noalloc on the current device
+        ws = noalloc_scratch_address();
+        if (ws == nullptr)
+            return LNQ_ERR_CUDA;
+    }
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     uint32_t flags[2] = {0, 0};
     if (cudaMemcpyAsync(flags, ws, sizeof(flags), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
@@ -330,6 +327,22 @@ lnq_status lnq_workspace_check(void *ws, lnq_stream_t stream)
             return LNQ_ERR_CUDA;
         return LNQ_ERR_TIMEOUT;
     }
+    return LNQ_OK;
+}
+
+lnq_status lnq_sweep_counters(const void *ws, lnq_stream_t stream, int64_t *moves, int64_t *tail)
+{
+    if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0 || moves == nullptr ||
+        tail == nullptr)
+        return LNQ_ERR_INVALID_ARG;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    unsigned long long c[2] = {0ull, 0ull};
+    if (cudaMemcpyAsync(c, static_cast<const unsigned long long *>(ws) + kWsCounterWord, sizeof(c),
+                        cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+        return LNQ_ERR_CUDA;
+    *moves = static_cast<int64_t>(c[0]);
+    *tail = static_cast<int64_t>(c[1]);
     return LNQ_OK;
 }
 

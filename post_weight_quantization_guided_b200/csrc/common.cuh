@@ -20,8 +20,10 @@ namespace lnq {
 // Workspace header: the first 256 bytes of every workspace.
 //   word 0: error flags set by device code (sticky until lnq_workspace_check reads them)
 //   word 1: index of the first wait that gave up (debug aid)
+//   bytes 16-31: two 64-bit work counters of the assignment sweeps (lnq_sweep_counters)
 // ------------------------------------------------------------------------------------------
 constexpr size_t kWsHeader = 256;
+constexpr int kWsCounterWord = 2;  // first counter, in 64-bit words from the header's start
 constexpr uint32_t kErrTimeout = 1u;
 // Budget for waits that only wait on this CTA's own copies or MMAs on the error path; those finish
 // on their own, so this budget does not follow the testing knob.
@@ -376,6 +378,18 @@ __device__ __forceinline__ void umma_f16_pair(uint32_t d_tmem, uint64_t a_desc, 
         "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// The same MMA with the accumulator's old value halved first: D = A x B + D / 2 (the optional
+// scale-input-d operand of kind::f16, D scaled by 2^-1; exact in fp32).
+__device__ __forceinline__ void umma_f16_pair_halve_d(uint32_t d_tmem, uint64_t a_desc,
+                                                      uint64_t b_desc, uint32_t idesc)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p, 1;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(1u)
         : "memory");
 }
 

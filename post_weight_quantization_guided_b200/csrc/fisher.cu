@@ -6,26 +6,29 @@
 // within each group, so F_g uses s_g[t] = mean_{j in g} G[t,j]^2).
 //
 // Kernels:
-//   token_stats_kernel      per token t: s_g[t] for every group (16-byte loads of G, fp32 sums),
-//                           M_t = max_i |X[t,i]|, and per group the maximum of s_g[t] M_t^2.
-//   guided_operands_kernel  A = X scaled by a power of two per token (exact in fp16) and
-//                           B_g = fp16(s_g * X) scaled by powers of two (one rounding, 2^-11
-//                           relative), so that F_g = alpha * Pi_g * A^T B_g. Keeping X exact on
-//                           one side and fp16 on the other bounds the error of every F entry by
-//                           about 5e-4 * sqrt(F_ii F_kk) even for a single token; bf16 on both
-//                           sides can reach 8e-3.
-//   fisher_syrk_kernel      persistent tcgen05 GEMM over the upper-triangle 256 x 256 tiles of
-//                           every F_g, two CTAs (a cluster pair on two SMs) per tile. Each CTA's
-//                           TMA brings its 128 rows of A and its 128 of the tile's 256 columns of
-//                           B_g, as 64(t) x 64(i) boxes in the 128-byte-swizzled MN-major layout
-//                           (no transpose of X is needed), with the bytes of both counted on the
-//                           even CTA's barrier; the even CTA's thread issues
-//                           tcgen05.mma.cta_group::2.kind::f16 (M=256, N=256, K=16); each CTA's
-//                           four epilogue warps read its 128 rows from TMEM, scale and write them
-//                           and their mirror image. Two TMEM accumulators let the epilogue of one
-//                           tile overlap the main loop of the next. Per CTA and stage 32 KB feed
-//                           128 x 256 x 64 MACs (48 KB for a single CTA's tile of the same size).
-// Without gradients (G == NULL) the product is X^T X: A = B = X in bf16, no preparation pass.
+//   token_stats_kernel   per token t: s_g[t] for every group (16-byte loads of G, fp32 sums),
+//                        M_t = max_i |X[t,i]|, and per group the maximum of s_g[t] M_t^2.
+//   token_scales_kernel  per token t: the two operand factors below, in place of s_g[t] and M_t.
+//   fisher_syrk_kernel   persistent tcgen05 GEMM over the upper-triangle 256 x 256 tiles of every
+//                        F_g, two CTAs (a cluster pair on two SMs) per tile. Per stage of 64
+//                        tokens each CTA holds its 128 rows of the left operand and its 128 of the
+//                        tile's 256 columns of the right operand, in the 128-byte-swizzled
+//                        MN-major layout (64(t) x 64(i) boxes; X is never transposed). The even
+//                        CTA's thread issues tcgen05.mma.cta_group::2.kind::f16 (M=256, N=256,
+//                        K=16); each CTA's four epilogue warps read its 128 rows from TMEM, scale
+//                        them and write them and their mirror image. Two TMEM accumulators let the
+//                        epilogue of one tile overlap the main loop of the next.
+//     guided (G given):  the diag(s_g) scaling is fused into the operand load. Two groups of
+//                        eight producer warps per CTA read X (bf16) straight from global memory
+//                        with 16-byte loads, each group a whole stage (two stages in flight), and
+//                        write both operands into the stage in fp16:
+//                          A[t][i] = X[t][i] / P_t                  (P_t = pow2_ceil(M_t), exact)
+//                          B[t][k] = fp16(X[t][k] * s_g[t] P_t / Pi_g)   (Pi_g = pow2_ceil(max_t
+//                                                                    s_g[t] M_t^2), one rounding)
+//                        so that A^T B = X^T diag(s_g) X / Pi_g with |A| <= 1, |B| <= 2, and every
+//                        entry within about 5e-4 sqrt(F_ii F_kk) even for a single token (bf16 on
+//                        both sides can reach 8e-3). No scaled copy of X is ever written to HBM.
+//     plain (G == NULL): F = X^T X; TMA brings X in bf16 (exact products) for both operands.
 #include <cuda_fp16.h>
 
 #include "common.cuh"
@@ -113,42 +116,23 @@ __device__ __forceinline__ float pow2_ceil(float v)
     return __uint_as_float((u & 0x7F800000u) + 0x00800000u);
 }
 
-// Operands of the guided product, one thread per 8 consecutive elements of a token row:
-//   A[t][:]    = fp16(X[t][:] / P_t),                          P_t = pow2_ceil(M[t])  (exact)
-//   B[g][t][:] = fp16(X[t][:] * S[g][t] * P_t / Pi_g),         Pi_g = pow2_ceil(pimax[g])
-// so that A[t][i] * B[g][t][k] = s_g[t] X[t][i] X[t][k] / Pi_g with one fp16 rounding, |A| <= 1
-// and |B| <= 2. The GEMM epilogue multiplies by alpha * Pi_g.
-__global__ void guided_operands_kernel(const __nv_bfloat16 *__restrict__ X,
-                                       const float *__restrict__ S, const float *__restrict__ M,
-                                       const unsigned *__restrict__ pimax, int64_t n, int64_t d,
-                                       int groups, __half *__restrict__ A, __half *__restrict__ B)
+// Per-token operand factors of the guided product, in place of the statistics they come from:
+//   M[t]    <- 1 / P_t,                    P_t = pow2_ceil(M_t)           (exact)
+//   S[g][t] <- S[g][t] * P_t / Pi_g,       Pi_g = pow2_ceil(pimax[g])
+// so that the left operand X[t][:] / P_t is exact in fp16 (|.| <= 1), the right operand
+// fp16(X[t][:] * S[g][t] P_t / Pi_g) is rounded once (|.| <= 2), and their product is
+// s_g[t] X[t][i] X[t][k] / Pi_g. One thread per token.
+__global__ void token_scales_kernel(int64_t n, int groups, float *__restrict__ S,
+                                    float *__restrict__ M, const unsigned *__restrict__ pimax)
 {
-    const int64_t vec_per_row = d / 8;
-    const int64_t v = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-    if (v >= n * vec_per_row)
+    const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (t >= n)
         return;
-    const int64_t t = v / vec_per_row;
-    const uint4 x = __ldg(reinterpret_cast<const uint4 *>(X) + v);
-    const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&x);
-    float2 f[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e)
-        f[e] = __bfloat1622float2(h[e]);
     const float Pt = pow2_ceil(M[t]);
-    const float inv = 1.f / Pt;  // exact: Pt is a power of two
-    uint4 out;
-    __half2 *o = reinterpret_cast<__half2 *>(&out);
-#pragma unroll
-    for (int e = 0; e < 4; ++e)
-        o[e] = __floats2half2_rn(f[e].x * inv, f[e].y * inv);
-    reinterpret_cast<uint4 *>(A)[v] = out;
-    for (int g = 0; g < groups; ++g) {
-        const float factor = S[static_cast<int64_t>(g) * n + t] * Pt / pow2_ceil(__uint_as_float(pimax[g]));
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-            o[e] = __floats2half2_rn(f[e].x * factor, f[e].y * factor);
-        reinterpret_cast<uint4 *>(B + static_cast<int64_t>(g) * n * d)[v] = out;
-    }
+    for (int g = 0; g < groups; ++g)
+        S[static_cast<int64_t>(g) * n + t] =
+            S[static_cast<int64_t>(g) * n + t] * Pt / pow2_ceil(__uint_as_float(pimax[g]));
+    M[t] = 1.f / Pt;
 }
 
 // ------------------------------------------------------------------------------------------
@@ -158,24 +142,37 @@ namespace syrk {
 constexpr int BM = 128;          // tile rows (i) per CTA: TMEM lanes; the pair covers 2 BM
 constexpr int PM = 2 * BM;       // rows of a pair tile
 constexpr int BN = 256;          // tile columns (k), TMEM columns per accumulator
-constexpr int HALF = BN / 2;     // columns of the right operand each CTA loads
+constexpr int HALF = BN / 2;     // columns of the right operand each CTA holds
 constexpr int BK = 64;           // tokens per pipeline stage
 constexpr int STAGES = 6;
-constexpr int BOX = 64;          // TMA box: 64 elements (128 B) along i/k  x  64 tokens
+constexpr int BOX = 64;          // operand box: 64 elements (128 B) along i/k  x  64 tokens
 constexpr int BOX_BYTES = BOX * BK * 2;                  // 8 KB
 constexpr int A_BYTES = (BM / BOX) * BOX_BYTES;          // 16 KB
 constexpr int B_BYTES = (HALF / BOX) * BOX_BYTES;        // 16 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;           // 32 KB per CTA
-constexpr int NUM_THREADS = 192;                         // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
+// warp 0 TMA (plain), warp 1 MMA, warps 2-5 epilogue, then (guided) PROD_GROUPS groups of four
+// operand-producer warps; group k fills the stages of fills k, k + PROD_GROUPS, ...
+constexpr int PROD_GROUPS = 2;
+constexpr int GROUP_THREADS = 256;
+constexpr int PROD_THREADS = PROD_GROUPS * GROUP_THREADS;
+constexpr int PROD_TOKENS = BK / (GROUP_THREADS / 16);   // tokens per producer thread and fill: 8
+__host__ __device__ constexpr int num_threads(bool guided) { return guided ? 192 + PROD_THREADS : 192; }
 constexpr int TMEM_COLS = 2 * BN;                        // two accumulators
 constexpr size_t SMEM_BYTES = static_cast<size_t>(STAGES) * STAGE_BYTES + 1024 /*align*/ + 256;
 constexpr uint16_t PAIR = 0x3;                           // both CTAs of the cluster
 constexpr long long kPairDrainLimit = 1LL << 22;
 static_assert(SMEM_BYTES <= 232448, "shared memory");
+static_assert(BK % (GROUP_THREADS / 16) == 0 && STAGES % PROD_GROUPS == 0, "producer tiling");
+// the last 16-byte chunk a producer thread writes ends at the end of its operand's half stage
+static_assert(BOX_BYTES + (BK - 1) * 128 + 7 * 16 + 16 == A_BYTES && A_BYTES == B_BYTES,
+              "producer stores stay inside their stage");
 }  // namespace syrk
 
 struct SyrkParams {
     float *F;            // [groups][d][d]
+    const __nv_bfloat16 *X;  // [n][d] (guided: read by the producer warps)
+    const float *bfac;   // [groups][n] right-operand factor s_g[t] P_t / Pi_g (guided)
+    const float *ainv;   // [n] left-operand factor 1 / P_t (guided)
     const unsigned *pimax;  // [groups] per-group operand scale (guided), or nullptr
     int64_t n, d;
     int groups;
@@ -200,18 +197,41 @@ __device__ __forceinline__ void syrk_tile_coords(const SyrkParams &p, int tile, 
     bi = r;
 }
 
-template <bool kF16>
-__global__ void __launch_bounds__(syrk::NUM_THREADS, 1)
-    fisher_syrk_kernel(const __grid_constant__ CUtensorMap amap,
-                       const __grid_constant__ CUtensorMap bmap, SyrkParams p)
+// 16-byte read-only load that does not allocate in L1 (X is shared through L2).
+__device__ __forceinline__ uint4 ldg_nc_v4(const void *p)
+{
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(reinterpret_cast<uint64_t>(p)));
+    return v;
+}
+
+// 8 bf16 values times `scale`, rounded once to fp16.
+__device__ __forceinline__ uint4 scale_bf16x8_to_f16(uint4 x, float scale)
+{
+    const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&x);
+    uint4 out;
+    __half2 *o = reinterpret_cast<__half2 *>(&out);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const float2 f = __bfloat1622float2(h[e]);
+        o[e] = __floats2half2_rn(f.x * scale, f.y * scale);
+    }
+    return out;
+}
+
+template <bool kGuided>
+__device__ __forceinline__ void fisher_syrk_body(const CUtensorMap &amap, const CUtensorMap &bmap,
+                                                 const SyrkParams &p)
 {
     using namespace syrk;
     constexpr uint32_t IDESC = umma_idesc_f16kind(PM, BN, /*a_mn_major=*/true,
-                                                  /*b_mn_major=*/true, kF16);
+                                                  /*b_mn_major=*/true, kGuided);
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(align_up(reinterpret_cast<uintptr_t>(smem_raw), 1024));
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + STAGES * STAGE_BYTES);
-    uint64_t *full = bars;                  // [STAGES] (the even CTA's counts both CTAs' bytes)
+    uint64_t *full = bars;                  // [STAGES] (the even CTA's counts both CTAs' fills)
     uint64_t *empty = bars + STAGES;        // [STAGES]
     uint64_t *tfull = bars + 2 * STAGES;    // [2]
     uint64_t *tempty = bars + 2 * STAGES + 2;  // [2] (the even CTA's counts both epilogues)
@@ -226,7 +246,9 @@ __global__ void __launch_bounds__(syrk::NUM_THREADS, 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
-            mbar_init(&full[s], 1);
+            // guided: one arrival per warp of the filling producer group in both CTAs; plain: the
+            // even CTA's expect_tx arrival, with the TMA bytes of both CTAs
+            mbar_init(&full[s], kGuided ? 2 * (GROUP_THREADS / 32) : 1);
             mbar_init(&empty[s], 1);
         }
         for (int a = 0; a < 2; ++a) {
@@ -235,8 +257,10 @@ __global__ void __launch_bounds__(syrk::NUM_THREADS, 1)
         }
         mbar_init(drain, 1);
         fence_barrier_init();
-        tma_prefetch_desc(&amap);
-        tma_prefetch_desc(&bmap);
+        if (!kGuided) {
+            tma_prefetch_desc(&amap);
+            tma_prefetch_desc(&bmap);
+        }
     }
     if (warp == 1)
         tmem_alloc_pair(tmem_holder, TMEM_COLS);
@@ -248,10 +272,10 @@ __global__ void __launch_bounds__(syrk::NUM_THREADS, 1)
     const long long limit = p.err.limit;
 
     if (warp == 0) {
-        // ---------------------------------------------------------------- TMA producer
-        // Per stage: this CTA's 128 rows of A and its 128 of the tile's 256 columns of B_g, the
+        // ---------------------------------------------------------------- TMA producer (plain)
+        // Per stage: this CTA's 128 rows of A and its 128 of the tile's 256 columns of B, the
         // bytes of both CTAs counted on the even CTA's barrier (armed there for both).
-        if (lane == 0) {
+        if (!kGuided && lane == 0) {
             uint32_t fpar = 0u, fused = 0u;  // per stage: parity of the fills, ever filled
             int stage = 0;
             bool ok = true;
@@ -314,7 +338,9 @@ __global__ void __launch_bounds__(syrk::NUM_THREADS, 1)
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
                 for (int kb = 0; kb < nk; ++kb) {
-                    if (!mbar_wait(&full[stage], (fph >> stage) & 1u, limit)) {
+                    const bool got = kGuided ? mbar_wait_cluster(&full[stage], (fph >> stage) & 1u, limit)
+                                             : mbar_wait(&full[stage], (fph >> stage) & 1u, limit);
+                    if (!got) {
                         raise_error(p.err, kErrTimeout, 3);
                         ok = false;
                         break;
@@ -341,7 +367,7 @@ __global__ void __launch_bounds__(syrk::NUM_THREADS, 1)
             umma_commit_pair(drain, 0x1);
             mbar_wait(drain, 0, kDrainLimit);
         }
-    } else {
+    } else if (warp < 6) {
         // ---------------------------------------------------------------- epilogue (warps 2-5)
         const int quarter = warp & 3;  // TMEM lanes this warp may access
         const int row_in_tile = static_cast<int>(cr) * BM + quarter * 32 + lane;
@@ -367,7 +393,7 @@ __global__ void __launch_bounds__(syrk::NUM_THREADS, 1)
             syrk_tile_coords(p, tile, g, bi, bk);
             float *Fg = p.F + static_cast<int64_t>(g) * p.d * p.d;
             const float scale =
-                p.pimax ? p.alpha * pow2_ceil(__uint_as_float(p.pimax[g])) : p.alpha;
+                kGuided ? p.alpha * pow2_ceil(__uint_as_float(p.pimax[g])) : p.alpha;
             const int64_t i = static_cast<int64_t>(bi) * PM + row_in_tile;
             for (int chunk = 0; chunk < BN / 32; ++chunk) {
                 float v[32];
@@ -404,15 +430,90 @@ __global__ void __launch_bounds__(syrk::NUM_THREADS, 1)
             tc_fence_before();
             mbar_arrive_cluster(tempty_leader[acc]);
         }
+    } else if constexpr (kGuided) {
+        // ---------------------------------------------------------------- operand producers
+        // Group k fills the stages of fills k, k + PROD_GROUPS, ... (fill f: tile pair + (f / nk)
+        // npairs, tokens 64 (f % nk) ..). Thread pt of a group covers 8 consecutive coordinates
+        // (column c16 of 16-byte chunks, box c16 / 8) of both operands for the tokens tr + 16 j.
+        // Its element (t, 8 c16 ..) sits at row t of its box, 16-byte chunk (c16 % 8) ^ (t % 8):
+        // the 128-byte swizzle the MMA descriptors expect (t % 8 = tr % 8 for every j). A group issues
+        // all loads of its fill (X and the two per-token factors) before it waits for the stage, so
+        // the groups' fills overlap; each warp of the group arrives once on the even CTA's barrier.
+        const int pidx = threadIdx.x - 6 * 32;
+        const int grp = pidx / GROUP_THREADS;
+        const int pt = pidx % GROUP_THREADS;
+        const int c16 = pt & 15, tr = pt >> 4;
+        const uint32_t soff = static_cast<uint32_t>((c16 >> 3) * BOX_BYTES + tr * 128 +
+                                                    (((c16 & 7) ^ (tr & 7)) << 4));
+        const int64_t d = p.d, n = p.n;
+        const int total = ((p.num_tiles - pair + npairs - 1) / npairs) * nk;  // this pair's fills
+        const uint32_t full_leader_base = cluster_addr(&full[0], 0);
+        for (int f = grp; f < total; f += PROD_GROUPS) {
+            const int tile = pair + (f / nk) * npairs;
+            int g, bi, bk;
+            syrk_tile_coords(p, tile, g, bi, bk);
+            const int64_t i0 = static_cast<int64_t>(bi) * PM + static_cast<int64_t>(cr) * BM + 8 * c16;
+            const int64_t k0 = static_cast<int64_t>(bk) * BN + static_cast<int64_t>(cr) * HALF + 8 * c16;
+            const int64_t t0 = static_cast<int64_t>(f % nk) * BK + tr;
+            uint4 xa[PROD_TOKENS], xb[PROD_TOKENS];
+            float fa[PROD_TOKENS], fb[PROD_TOKENS];
+#pragma unroll
+            for (int j = 0; j < PROD_TOKENS; ++j) {
+                const int64_t t = t0 + (GROUP_THREADS / 16) * j;
+                const bool tin = t < n;
+                xa[j] = (tin && i0 < d) ? ldg_nc_v4(p.X + t * d + i0) : make_uint4(0u, 0u, 0u, 0u);
+                xb[j] = (tin && k0 < d) ? ldg_nc_v4(p.X + t * d + k0) : make_uint4(0u, 0u, 0u, 0u);
+                fa[j] = tin ? __ldg(p.ainv + t) : 0.f;
+                fb[j] = tin ? __ldg(p.bfac + static_cast<int64_t>(g) * n + t) : 0.f;
+            }
+            const int stage = f % STAGES;
+            int got = 0;
+            if (lane == 0)
+                got = mbar_wait(&empty[stage], ((f / STAGES) & 1) ^ 1, limit) ? 1 : 0;
+            got = __shfl_sync(0xffffffffu, got, 0);
+            if (!got) {
+                if (lane == 0)
+                    raise_error(p.err, kErrTimeout, 5);
+                break;
+            }
+            uint8_t *sa = smem + stage * STAGE_BYTES + soff;
+#pragma unroll
+            for (int j = 0; j < PROD_TOKENS; ++j) {
+                *reinterpret_cast<uint4 *>(sa + (GROUP_THREADS / 16) * j * 128) =
+                    scale_bf16x8_to_f16(xa[j], fa[j]);
+                *reinterpret_cast<uint4 *>(sa + A_BYTES + (GROUP_THREADS / 16) * j * 128) =
+                    scale_bf16x8_to_f16(xb[j], fb[j]);
+            }
+            fence_proxy_async_smem();  // the stores become visible to the tensor core
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive_cluster(full_leader_base + static_cast<uint32_t>(stage * 8));
+        }
     }
 
     // Both CTAs stay until the pair is done: the MMAs read both CTAs' shared memory and the
-    // copies and epilogues of both signal barriers in the even CTA.
+    // copies, producers and epilogues of both signal barriers in the even CTA.
     tc_fence_before();
     cluster_sync();
     tc_fence_after();
     if (warp == 1)
         tmem_dealloc_pair(tmem_base, TMEM_COLS);
+}
+
+// The two instantiations: plain (192 threads) and guided (704 threads: 22 warps, at most six on
+// each of the SM's four register-file quarters, so at most 80 registers per thread).
+__global__ void __launch_bounds__(syrk::num_threads(false), 1)
+    fisher_syrk_plain_kernel(const __grid_constant__ CUtensorMap amap,
+                             const __grid_constant__ CUtensorMap bmap, SyrkParams p)
+{
+    fisher_syrk_body<false>(amap, bmap, p);
+}
+
+__global__ void __launch_bounds__(syrk::num_threads(true), 1)
+    fisher_syrk_guided_kernel(const __grid_constant__ CUtensorMap amap,
+                              const __grid_constant__ CUtensorMap bmap, SyrkParams p)
+{
+    fisher_syrk_body<true>(amap, bmap, p);
 }
 
 }  // namespace lnq
@@ -422,6 +523,7 @@ __global__ void __launch_bounds__(syrk::NUM_THREADS, 1)
 // ------------------------------------------------------------------------------------------
 #include <cudaTypedefs.h>
 
+#include <cstring>
 #include <mutex>
 
 namespace lnq {
@@ -460,21 +562,31 @@ static bool encode_operand(CUtensorMap *map, const void *base, int64_t n, int64_
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// F_g = scale_g * A^T B_g, both triangles written, for A [n][d] and B [groups][n][d] (row-major):
-//   f16 == false: A = B = X in bf16 (groups == 1), scale = alpha;
-//   f16 == true:  the guided operands above, scale_g = alpha * pow2_ceil(pimax[g]).
-cudaError_t fisher_syrk(const void *A, const void *B, bool f16, const unsigned *pimax, int64_t n,
-                        int64_t d, int groups, float alpha, float *F, DeviceErr err,
-                        cudaStream_t s, int num_sms)
+// F_g = scale_g * (operands)^T (operands), both triangles written:
+//   S == nullptr: F = alpha X^T X, X read by TMA in bf16 (groups == 1);
+//   otherwise:    the guided blocks, operands formed by the producer warps from X and the factors
+//                 that token_scales_kernel left in S (right) and M (left),
+//                 scale_g = alpha * pow2_ceil(pimax[g]).
+cudaError_t fisher_syrk(const __nv_bfloat16 *X, const float *S, const float *M,
+                        const unsigned *pimax, int64_t n, int64_t d, int groups, float alpha,
+                        float *F, DeviceErr err, cudaStream_t s, int num_sms)
 {
     using namespace syrk;
+    const bool guided = S != nullptr;
     CUtensorMap amap, bmap;
-    if (tensor_map_encoder() == nullptr)
-        return cudaErrorNotSupported;
-    if (!encode_operand(&amap, A, n, d, 1, f16) || !encode_operand(&bmap, B, n, d, groups, f16))
-        return cudaErrorInvalidValue;
+    memset(&amap, 0, sizeof(amap));
+    memset(&bmap, 0, sizeof(bmap));
+    if (!guided) {
+        if (tensor_map_encoder() == nullptr)
+            return cudaErrorNotSupported;
+        if (!encode_operand(&amap, X, n, d, 1, false) || !encode_operand(&bmap, X, n, d, 1, false))
+            return cudaErrorInvalidValue;
+    }
     SyrkParams p;
     p.F = F;
+    p.X = X;
+    p.bfac = S;
+    p.ainv = M;
     p.pimax = pimax;
     p.n = n;
     p.d = d;
@@ -484,7 +596,7 @@ cudaError_t fisher_syrk(const void *A, const void *B, bool f16, const unsigned *
     p.tiles_per_group = p.nb * (p.nb + 1) / 2;
     p.num_tiles = p.tiles_per_group * groups;
     p.err = err;
-    auto kernel = f16 ? fisher_syrk_kernel<true> : fisher_syrk_kernel<false>;
+    auto kernel = guided ? fisher_syrk_guided_kernel : fisher_syrk_plain_kernel;
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(SMEM_BYTES));
     if (e != cudaSuccess)
@@ -495,19 +607,21 @@ cudaError_t fisher_syrk(const void *A, const void *B, bool f16, const unsigned *
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
-    cfg.blockDim = dim3(NUM_THREADS);
+    cfg.blockDim = dim3(num_threads(guided));
     cfg.dynamicSmemBytes = SMEM_BYTES;
     cfg.stream = s;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     // persistent: as many pairs as can be resident at once (one CTA per SM)
     static int resident[2] = {0, 0};
-    int &res = resident[f16 ? 1 : 0];
+    int &res = resident[guided ? 1 : 0];
     if (res == 0) {
         cfg.gridDim = dim3(static_cast<unsigned>(num_sms & ~1));
         int clusters = 0;
-        if (cudaOccupancyMaxActiveClusters(&clusters, kernel, &cfg) != cudaSuccess || clusters < 1)
+        if (cudaOccupancyMaxActiveClusters(&clusters, kernel, &cfg) != cudaSuccess || clusters < 1) {
+            (void)cudaGetLastError();   // a failed query is not an error of this call
             clusters = num_sms / 2;
+        }
         res = clusters;
     }
     int pairs = res < p.num_tiles ? res : p.num_tiles;

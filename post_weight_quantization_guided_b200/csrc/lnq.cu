@@ -236,6 +236,7 @@ cudaError_t lnq_iterate_launch(const float *F, int groups, const float *W, int64
                                const LnqWorkspace &w, DeviceErr err, int num_sms, cudaStream_t s)
 {
     cudaError_t e;
+    const int nhalves = static_cast<int>(2 * ((d + 255) / 256));
     if (iters > 0 || J != nullptr)
         if ((e = lnq_split_f16(F, d, groups, w.Fh, w.fexp, s)) != cudaSuccess)
             return e;
@@ -248,22 +249,29 @@ cudaError_t lnq_iterate_launch(const float *F, int groups, const float *W, int64
             return e;
     }
     for (int it = 0; it < iters; ++it) {
-        if ((e = lnq_vgemm(w.Fh, w.fexp, nullptr, groups, Q, W, C, w.V, nullptr, w.img, d, d_out,
+        // codebook step: M = P^T F P (binned over the upper block triangle), then the solve
+        if ((e = lnq_vgemm(w.Fh, w.fexp, nullptr, groups, Q, W, C, w.Sb, nullptr, w.img, d, d_out,
                            m, false, err, num_sms, s)) != cudaSuccess)
             return e;
-        if ((e = lnq_solve(w.V, w.U, Q, C, w.dC, w.status, d, d_out, m, s)) != cudaSuccess)
+        if ((e = lnq_solve(w.Sb, nhalves, w.U, Q, C, w.status, d, d_out, m, s)) != cudaSuccess)
             return e;
-        if ((e = lnq_sweep(F, w.Fh, w.fexp, groups, w.V, w.dC, w.U, C, Q, w.hist, d, d_out, m,
-                           err, s)) != cudaSuccess)
+        // the sweep's starting u = F (c[q] - w) for the new codebook
+        if ((e = lnq_residual_scale(Q, W, C, d, d_out, m, w.rexp, s)) != cudaSuccess)
+            return e;
+        if ((e = lnq_vgemm(w.Fh, w.fexp, w.rexp, groups, Q, W, C, nullptr, w.Ur, w.img, d, d_out,
+                           m, true, err, num_sms, s)) != cudaSuccess)
+            return e;
+        if ((e = lnq_sweep(F, w.Fh, w.fexp, groups, w.Ur, C, Q, w.hist, d, d_out, m, err, s)) !=
+            cudaSuccess)
             return e;
     }
     if (J != nullptr) {
         if ((e = lnq_residual_scale(Q, W, C, d, d_out, m, w.rexp, s)) != cudaSuccess)
             return e;
-        if ((e = lnq_vgemm(w.Fh, w.fexp, w.rexp, groups, Q, W, C, nullptr, w.U, w.img, d, d_out, m,
-                           true, err, num_sms, s)) != cudaSuccess)
+        if ((e = lnq_vgemm(w.Fh, w.fexp, w.rexp, groups, Q, W, C, nullptr, w.Ur, w.img, d, d_out,
+                           m, true, err, num_sms, s)) != cudaSuccess)
             return e;
-        if ((e = lnq_objective_from_u(w.U, W, C, Q, J, d, d_out, m, s)) != cudaSuccess)
+        if ((e = lnq_objective_from_u(w.Ur, W, C, Q, J, d, d_out, m, s)) != cudaSuccess)
             return e;
     }
     return cudaGetLastError();

@@ -8,9 +8,9 @@
 // One CTA per 32 rows of one Fisher group. Coordinates are taken in windows of 128 (the height
 // of a tensor-core tile), each window in four blocks of 32.
 //   * Before a window starts, its u is assembled left-looking: the value at the start of the
-//     sweep, U + V c (U = -F w and V = F P from lnq_vgemm, c the new codebook from lnq_solve,
-//     so U + V c = F (c[q] - w)), plus F[window][earlier coordinates] x Delta[earlier
-//     coordinates], Delta being the moves made so far in this sweep. That product runs on tcgen05
+//     sweep, u0 = F (c[q] - w) for the new codebook c (the residual product of lnq_vgemm.cu),
+//     plus F[window][earlier coordinates] x Delta[earlier coordinates], Delta being the moves
+//     made so far in this sweep. That product runs on tcgen05
 //     tensor cores: F as its two fp16 pieces with a power-of-two scale per row (the operand of
 //     lnq_vgemm, 22 bits per entry), Delta as two fp16 pieces with a power-of-two scale per
 //     row of W (22 bits), three piece products (F2 x D2, below 2^-22 of each term, is left out)
@@ -69,8 +69,7 @@ constexpr int OFF_STRIP = OFF_BS + 2 * H_CHUNK;
 constexpr int OFF_UW = OFF_STRIP + 2 * BLK * WIN * 4;
 constexpr int OFF_DL = OFF_UW + 2 * RB * UW_LD * 4;
 constexpr int OFF_C = OFF_DL + 2 * BLK * RB * 4;      // moves: two blocks in flight
-constexpr int OFF_DC = OFF_C + RB * 17 * 4;
-constexpr int OFF_QB = OFF_DC + RB * 16 * 4;
+constexpr int OFF_QB = OFF_C + RB * 17 * 4;
 constexpr int OFF_WM = OFF_QB + 2 * RB * (BLK + 8);   // codes: two blocks in flight
 constexpr int OFF_TS = (OFF_WM + MAX_WIN + 15) / 16 * 16;  // [2][RB] Delta scales 2^t, 2^-t
 constexpr int OFF_SRT = OFF_TS + 2 * RB * 4;               // [RB][17] sorted codebook
@@ -89,9 +88,7 @@ static_assert(OFF_QB % 8 == 0 && OFF_STRIP % 16 == 0, "vector accesses to the co
 
 struct SwParams {
     const float *F;      // [groups][d][d]
-    const float *V;      // [d_out][d][m]
-    const float *dC;     // [d_out][m] the new codebook (u at the start = U + V dC)
-    const float *U;      // [d_out][d] u = F r for the previous codebook
+    const float *U;      // [d_out][d] u = F r at the start of the sweep (codebook C, codes Q)
     const float *C;      // [d_out][m]
     uint8_t *Q;          // [d_out][d]
     uint8_t *hist;       // [CTAs][2 * windows][2][4 KB]
@@ -99,8 +96,18 @@ struct SwParams {
     int64_t d, d_out, rows_per_group;
     int strip_tma;       // F strips by TMA (d % 4 == 0, F 16-byte aligned) or by plain loads
     int blocks_per_group, nwin;
+    // work counters in the workspace header: [0] coordinates moved, [1] the sum over those moves
+    // of (d - i), the entries of u that each move updates
+    unsigned long long *counters;
     DeviceErr err;
 };
+
+// Sum of the positions of the set bits of a 32-bit mask.
+__device__ __forceinline__ unsigned bit_position_sum(unsigned m)
+{
+    return __popc(m & 0xAAAAAAAAu) + 2u * __popc(m & 0xCCCCCCCCu) + 4u * __popc(m & 0xF0F0F0F0u) +
+           8u * __popc(m & 0xFF00FF00u) + 16u * __popc(m & 0xFFFF0000u);
+}
 
 template <int M>
 __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
@@ -118,7 +125,6 @@ __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
     float *uwb = reinterpret_cast<float *>(smem + OFF_UW);           // [2][RB][UW_LD]
     float(*dl2)[BLK][RB] = reinterpret_cast<float(*)[BLK][RB]>(smem + OFF_DL);  // [2][BLK][RB] moves
     float(*c_s)[17] = reinterpret_cast<float(*)[17]>(smem + OFF_C);         // [RB][m]
-    float(*dc_s)[16] = reinterpret_cast<float(*)[16]>(smem + OFF_DC);       // [RB][m]
     // [2][RB][BLK + 8] codes of the current and the next block, rows 8-byte aligned
     uint8_t(*qb2)[RB][BLK + 8] = reinterpret_cast<uint8_t(*)[RB][BLK + 8]>(smem + OFF_QB);
     volatile uint8_t *wmask = smem + OFF_WM;                         // [window]: some row moved
@@ -188,7 +194,6 @@ __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
         const int r = e >> 4, b = e & 15;
         const bool in = r < nrows && b < M;
         c_s[r][b] = in ? p.C[(row0 + r) * M + b] : 0.f;
-        dc_s[r][b] = in ? p.dC[(row0 + r) * M + b] : 0.f;
     }
     if (threadIdx.x < RB) {
         // every Delta of row r is a difference of two of its codewords: |Delta| <= max c - min c
@@ -365,7 +370,7 @@ __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
     } else if (warp < 6) {
         // ---------------------------------------------------------------- window assembly
         // Thread = coordinate kl of the window (= TMEM lane; warp w reads lanes 32 (w % 4)..).
-        // u of window T for the CTA's rows: U (= -F w) + V c (c the new codebook), plus the
+        // u of window T for the CTA's rows: u0 = F (c[q] - w) at the start of the sweep, plus the
         // accumulator of the moves made before the window, written to the window buffer T & 1.
         const int quarter = warp & 3;
         const int kl = quarter * 32 + lane;
@@ -379,30 +384,6 @@ __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
 #pragma unroll
             for (int r = 0; r < RB; ++r)
                 u0[r] = (kin && r < nrows) ? p.U[(row0 + r) * d + k] : 0.f;
-            if (kin) {
-#pragma unroll
-                for (int r = 0; r < RB; ++r) {
-                    if (r < nrows) {
-                        const float *vk = p.V + ((row0 + r) * d + k) * M;
-                        float acc = u0[r];
-                        if constexpr (M >= 4) {
-#pragma unroll
-                            for (int b4 = 0; b4 < M / 4; ++b4) {
-                                const float4 v4 = reinterpret_cast<const float4 *>(vk)[b4];
-                                acc = fmaf(v4.x, dc_s[r][4 * b4], acc);
-                                acc = fmaf(v4.y, dc_s[r][4 * b4 + 1], acc);
-                                acc = fmaf(v4.z, dc_s[r][4 * b4 + 2], acc);
-                                acc = fmaf(v4.w, dc_s[r][4 * b4 + 3], acc);
-                            }
-                        } else {
-                            const float2 v2 = *reinterpret_cast<const float2 *>(vk);
-                            acc = fmaf(v2.x, dc_s[r][0], acc);
-                            acc = fmaf(v2.y, dc_s[r][1], acc);
-                        }
-                        u0[r] = acc;
-                    }
-                }
-            }
             if (T > 0) {
                 const int acc = T & 1;
                 int okw = 0;
@@ -616,6 +597,7 @@ __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
         fetch_codes(0, 0, t, SWEEP_THREADS);
         load_strip(0, 0, 0, t, SWEEP_THREADS);
         bool failed = false;
+        unsigned long long cmoves = 0ull, ctail = 0ull;  // warp 6: this lane's row's counters
         for (int T = 0; T < nwin; ++T) {
             const int64_t wstart = static_cast<int64_t>(T) * WIN;
             const int buf = T & 1;
@@ -758,6 +740,13 @@ __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
                     for (int v = 0; v < BLK / 4; ++v)
                         *reinterpret_cast<uint32_t *>(&qb_s[r][4 * v]) = qw[v];
                     rm2[cb][r] = rowmask;
+                    {
+                        const unsigned moved = static_cast<unsigned>(__popc(rowmask));
+                        cmoves += moved;
+                        ctail += static_cast<unsigned long long>(moved) *
+                                     static_cast<unsigned long long>(d - b0) -
+                                 bit_position_sum(rowmask);
+                    }
                     const unsigned wm = __reduce_or_sync(0xffffffffu, rowmask);
                     if (lane == 0)
                         mv2[cb] = wm;
@@ -793,6 +782,17 @@ __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
                 mbar_arrive(bs_ready);
             }
             mbar_arrive(&uw_free[buf]);
+        }
+        if (warp == 6) {
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                cmoves += __shfl_xor_sync(0xffffffffu, cmoves, o);
+                ctail += __shfl_xor_sync(0xffffffffu, ctail, o);
+            }
+            if (lane == 0 && p.counters != nullptr) {
+                atomicAdd(&p.counters[0], cmoves);
+                atomicAdd(&p.counters[1], ctail);
+            }
         }
         cp_async_wait_all();
         // after an early exit, let the strip copies in flight land (the last fill of buffer b
@@ -855,8 +855,8 @@ static cudaError_t sweep_m(const CUtensorMap &map, const CUtensorMap &smap, cons
 }
 
 cudaError_t lnq_sweep(const float *F, const __half *Fh, const int32_t *fexp, int groups,
-                      const float *V, const float *dC, const float *U, const float *C, uint8_t *Q,
-                      uint8_t *hist, int64_t d, int64_t d_out, int m, DeviceErr err, cudaStream_t s)
+                      const float *U, const float *C, uint8_t *Q, uint8_t *hist, int64_t d,
+                      int64_t d_out, int m, DeviceErr err, cudaStream_t s)
 {
     CUtensorMap map;
     if (!encode_f16_pieces(&map, Fh, d, groups))
@@ -867,8 +867,6 @@ cudaError_t lnq_sweep(const float *F, const __half *Fh, const int32_t *fexp, int
     SwParams p{};
     p.strip_tma = strip_tma ? 1 : 0;
     p.F = F;
-    p.V = V;
-    p.dC = dC;
     p.U = U;
     p.C = C;
     p.Q = Q;
@@ -879,6 +877,7 @@ cudaError_t lnq_sweep(const float *F, const __half *Fh, const int32_t *fexp, int
     p.rows_per_group = d_out / groups;
     p.blocks_per_group = static_cast<int>((p.rows_per_group + sw::RB - 1) / sw::RB);
     p.nwin = static_cast<int>((d + sw::WIN - 1) / sw::WIN);
+    p.counters = reinterpret_cast<unsigned long long *>(err.flags) + kWsCounterWord;
     p.err = err;
     const unsigned grid = static_cast<unsigned>(p.blocks_per_group) * static_cast<unsigned>(groups);
     switch (m) {

@@ -1,30 +1,38 @@
-// lnq_vgemm.cu -- the dense contraction of an LNQ iteration on tcgen05 tensor cores.
+// lnq_vgemm.cu -- the dense contractions of an LNQ iteration on tcgen05 tensor cores.
 //
 // Source: "GuidedQuant" (jinukkim.me blog), LNQ section. The codebook update
-// c <- (P^T F P)^-1 P^T F w needs, per output row j, the class-binned product V_j = F P_j (d x m;
-// P_j is the one-hot assignment): M_j = P_j^T V_j. P^T F w comes from y_j = F w_j, which does not
-// change between iterations, and the sweep starts from u_j = F r_j = V_j c_j - y_j with
-// r_j = c_j[q_j] - w_j. Two products serve all rows of one Fisher group, whose left operand F
-// they share:
+// c <- (P^T F P)^-1 P^T F w needs, per output row j, the m x m matrix M_j = P_j^T F P_j (P_j the
+// one-hot assignment, d x m), and the assignment sweep that follows starts from u_j = F r_j with
+// r_j = c_j[q_j] - w_j. Both come from products of F with right operands that stack the rows of
+// one Fisher group side by side, so that every row of the group shares the left operand F:
 //
-//      [V_j1 | V_j2 | ...] = F x [P_j1 | P_j2 | ...]        (m one-hot columns per row)
-//      [u_j1 | u_j2 | ...] = F x [r_j1 | r_j2 | ...]        (residual; r = -w gives -y)
+//   class-binned product (m > 0), over the upper block triangle only. With F = U + U^T, U the
+//     blocks of 256 x 256 coordinates on and above the diagonal with the diagonal blocks halved,
+//     M_j = P_j^T U P_j + (P_j^T U P_j)^T. For coordinate block I the product accumulates
+//     V'_I = (1/2) F_II P_I + sum_{K > I} F_IK P_K (the diagonal block first; the first MMA of the
+//     next block halves the accumulator exactly through its scale-input-d operand), and the
+//     epilogue bins V'_I by class: S_I[q][.] = sum over coordinates i of I in class q of V'_I[i][.].
+//     M_j is then the sum over I of S_I + S_I^T (lnq_solve.cu). Half of the dense product's work.
+//   residual product (m == 0): u_j = F r_j for every row, r = c[q] - w (the zero codebook gives
+//     -F w), used by the codebook's right-hand side, the sweep and the objective.
 //
-// This kernel computes either with tcgen05.mma.cta_group::2.kind::f16 on fp16 pieces:
-//   * each row i of F (fp32) is scaled by a power of two 2^fexp[i] that puts its largest entry
-//     in [2^14, 2^15) and split into two fp16 pieces H1 + H2, 22 significant bits of every
-//     entry;
-//   * the one-hot columns are 0/1 (exact in fp16), two piece products; r_j is scaled by 2^rexp[j]
-//     the same way and split into three fp16 pieces (33 bits, exact for fp32 r), one column each,
-//     six piece products;
-//   * accumulation is fp32 in TMEM; the epilogue removes the power-of-two scales exactly.
-// The right operand (one-hot columns or residual pieces) of every (row tile, K block) is written
-// once per call as an image in HBM and loaded by TMA like F. Two CTAs (a cluster pair on two SMs)
-// share one MMA of 256 coordinates (i) x 256 columns (RT = 256 / m rows of m one-hot columns, or
-// 85 rows of 3 residual pieces): each CTA loads the F tiles of its own 128 coordinates and half of
-// the right operand's rows (K-major, 128-byte swizzle, no multicast). The even CTA issues the
-// MMAs; each CTA's TMEM holds its 128 coordinates x all columns, and its epilogue writes V[j][i][b]
-// or U[j][i] (both contiguous across a warp's coordinates).
+// Precision: each row i of F (fp32) is scaled by a power of two 2^fexp[i] that puts its largest
+// entry in [2^14, 2^15) and split into two fp16 pieces H1 + H2 (22 significant bits of every
+// entry). One-hot columns are exact in fp16 (two piece products). A residual row is scaled by
+// 2^rexp[j] the same way and split into two fp16 pieces R1 + R2; three piece products
+// H1 R1 + H1 R2 + H2 R1 (H2 R2 is below 2^-22 of each term, the size of the pieces' own rounding)
+// accumulate in fp32 in TMEM, in segments of 8 K blocks whose sums the epilogue adds in fp32. The
+// epilogues remove the power-of-two scales exactly.
+//
+// Two CTAs (a cluster pair on two SMs) share one MMA of 256 coordinates (i) x 256 columns: each CTA
+// loads by TMA the F tiles of its own 128 coordinates and half (128 columns) of the right
+// operand's tile (K-major, 128-byte swizzle, no multicast). The even CTA issues the MMAs; each
+// CTA's TMEM holds its 128 coordinates x 256 columns, two accumulators alternating between tiles.
+// The right operand of every (row tile, K block) is written once per product as an image in HBM:
+//   one-hot: RT = 256 / m rows of m class columns;
+//   residual: 128 rows; CTA h of the pair holds R1 of rows 64h .. 64h + 63, then their R2.
+//   The H1 product takes all 256 columns; the H2 product takes only the R1 halves (N = 128) and
+//   accumulates them 64 columns further on, into the R2 columns of the same rows.
 #include <cuda_fp16.h>
 
 #include "common.cuh"
@@ -35,12 +43,19 @@ namespace lnq {
 
 namespace vg {
 constexpr int BM = 128;                          // coordinates per CTA; a pair covers 256
+constexpr int PAIR_KB = 2 * BM / 64;             // K blocks per pair block of coordinates
 constexpr int BK = 64;
-constexpr int A_TILE = BM * BK * 2;              // one bf16 piece of a 128 x 64 F tile: 16 KB
+constexpr int A_TILE = BM * BK * 2;              // one fp16 piece of a 128 x 64 F tile: 16 KB
 constexpr int B_STAGES = 4;                      // right-operand half tiles in flight
 constexpr int NUM_THREADS = 192;                 // w0 TMA, w1 MMA, w2-5 epilogue
 constexpr int EPI_THREADS = 128;
+constexpr int EPI_BAR = 1;                       // named barrier of the epilogue warps
 constexpr int TMEM_COLS = 512;
+constexpr int NCOLS = 256;                       // MMA N: columns of the right operand per tile
+constexpr int HALF = NCOLS / 2;                  // right-operand rows held by one CTA
+constexpr int B_BYTES = HALF * 128;              // HALF rows x 64 k of 16-bit values: 16 KB
+constexpr int VS_LD = 36;                        // floats per staged coordinate (32 + pad)
+constexpr int VS_BYTES = BM * VS_LD * 4;         // one staged 32-column chunk: 18 KB
 constexpr int MAX_DYN_SMEM = 232448;             // opt-in dynamic shared memory per block
 constexpr int BAR_BYTES = 512;
 constexpr uint16_t PAIR = 0x3;                   // both CTAs of the cluster
@@ -49,37 +64,28 @@ constexpr long long kPairDrainLimit = 1LL << 22;
 }  // namespace vg
 
 // Tile shapes. Both products take F as two fp16 pieces and the MMA is 256 columns wide, with two
-// TMEM accumulators that alternate between accumulation segments. The class-binned product
-// (M > 0, M one-hot columns per row) accumulates a whole tile in one segment. The residual product
-// (M == 0: three fp16 pieces of r per row) feeds the objective and the solve, where u = F r is
-// small against its terms: its segments are SEGK K blocks long and the epilogue adds each
-// finished segment into fp32 sums per row, so no tensor-core accumulation chain runs longer than
-// SEGK x 64 coordinates (the accumulator's rounding error grows with the chain). Each CTA holds
-// HALF = NCOLS / 2 rows of the right operand per stage.
+// TMEM accumulators. The class-binned product (M > 0: RT = 256 / M rows of M one-hot columns per
+// tile) accumulates a tile in one segment and its epilogue stages each 32-column chunk in shared
+// memory (two buffers) next to the tile's codes; the residual product (M == 0: 128 rows per tile)
+// accumulates segments of SEGK K blocks, which its epilogue adds into fp32 sums per row held in
+// registers.
 template <int M>
 struct VgShape {
     static constexpr int PIECES = 2;                    // fp16 pieces of F in the left operand
-    // MMA N: 256, or 192 (64 rows of three pieces) for the residual product, whose epilogue keeps
-    // a running sum per row in registers
-    static constexpr int NCOLS = M > 0 ? 256 : 192;
-    static constexpr int HALF = NCOLS / 2;              // right-operand rows held by one CTA
     static constexpr int SEGK = M > 0 ? 0 : 8;          // K blocks per segment (0: whole tile)
-    static constexpr int SETS = 2;                      // accumulators (segment double-buffer)
-    static constexpr int RES = M > 0 ? 0 : 3;           // residual-piece columns per row
-    static constexpr int RT = NCOLS / (M + RES);        // rows per tile
-    static constexpr int ONEHOT = RT * M;               // one-hot columns
-    static constexpr int USED = RT * (M + RES);         // columns carrying data
-    static constexpr int CHUNKS = (USED + 31) / 32;     // 32-column TMEM loads per accumulator
-    static constexpr int B_BYTES = HALF * 128;          // HALF rows x 64 k of 16-bit values
+    static constexpr int SETS = 2;                      // accumulators
+    static constexpr int RT = M > 0 ? vg::NCOLS / M : 128;  // rows per tile
+    static constexpr int EPI_BYTES = M > 0 ? 2 * vg::VS_BYTES + RT * vg::BM : 0;
     static constexpr int A_FIT = (vg::MAX_DYN_SMEM - 1024 - vg::BAR_BYTES -
-                                  vg::B_STAGES * B_BYTES) / vg::A_TILE;
+                                  vg::B_STAGES * vg::B_BYTES - EPI_BYTES) / vg::A_TILE;
     static constexpr int A_SLOTS = A_FIT < 12 ? A_FIT : 12;
     static constexpr size_t SMEM = 1024 + static_cast<size_t>(A_SLOTS) * vg::A_TILE +
-                                   vg::B_STAGES * B_BYTES + vg::BAR_BYTES;
-    static_assert(SETS * NCOLS <= vg::TMEM_COLS, "TMEM holds 512 fp32 columns");
+                                   vg::B_STAGES * vg::B_BYTES + EPI_BYTES + vg::BAR_BYTES;
+    static_assert(SETS * vg::NCOLS <= vg::TMEM_COLS, "TMEM holds 512 fp32 columns");
     static_assert(A_SLOTS >= 2 * PIECES, "at least two K blocks of F in flight");
     static_assert(A_SLOTS <= 32, "slot phases are kept in 32-bit masks");
     static_assert(SMEM <= vg::MAX_DYN_SMEM, "shared memory");
+    static_assert(M == 0 || (M <= 32 && (32 / (M > 0 ? M : 1)) * M == 32), "a 32-column chunk holds whole rows");
 };
 
 // Row stride (elements) of the fp16 pieces of F: TMA needs row strides that are multiples of 16 B.
@@ -149,23 +155,23 @@ __global__ void __launch_bounds__(256)
 }
 
 
-// The right operand of every (row tile, K block), written once per call of the product and then
-// loaded by TMA like F: NCOLS rows (the product's columns) x 64 coordinates, row-major
-// [row tiles][K blocks][NCOLS][64]. Column n < ONEHOT of a row tile is the indicator of class n % M
-// for its row n / M; ONEHOT <= n < USED is residual piece (n - ONEHOT) % 3 of row (n - ONEHOT) / 3;
-// the rest is zero, as is everything outside the problem. All values are fp16, residuals scaled by
-// 2^rexp (C == nullptr: the zero codebook, r = -w). Two writers follow.
+// The right operand of every (row tile, K block), written once per product and then loaded by TMA
+// like F: NCOLS rows (the product's columns) x 64 coordinates, row-major
+// [row tiles][K blocks][NCOLS][64], fp16. One-hot image (M > 0): row n of a row tile is the
+// indicator of class n % M for the tile's row n / M. Residual image (M == 0): rows 128 h .. 128 h +
+// 63 hold piece R1 of the tile's rows 64 h .. 64 h + 63 and rows 128 h + 64 .. 128 h + 127 their R2
+// (h = 0, 1: the half each CTA of the pair loads). Everything outside the problem is zero.
 
-// The one-hot image (M > 0) with one task per (row tile, row, 8 coordinates): the task reads its
-// 8 codes once and writes its row's M class columns (16 bytes each; a warp's 32 tasks cover 4
-// rows x 64 coordinates, so each class store fills 4 whole 128-byte rows of the image).
+// The one-hot image with one task per (row tile, row, 8 coordinates): the task reads its 8 codes
+// once and writes its row's M class columns (16 bytes each; a warp's 32 tasks cover 4 rows x 64
+// coordinates, so each class store fills 4 whole 128-byte rows of the image).
 template <int M>
 __global__ void __launch_bounds__(256)
     onehot_image_kernel(const uint8_t *__restrict__ Q, int64_t d, int64_t rows_per_group,
                         int row_tiles_per_group, int64_t ntasks, int nk, uint16_t *__restrict__ img)
 {
     using S = VgShape<M>;
-    static_assert(M > 0 && S::ONEHOT == S::NCOLS, "one-hot columns fill the tile");
+    static_assert(M > 0 && S::RT * M == vg::NCOLS, "one-hot columns fill the tile");
     const bool vec = (d & 7) == 0 && (reinterpret_cast<uintptr_t>(Q) & 7u) == 0;
     for (int64_t task = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; task < ntasks;
          task += static_cast<int64_t>(gridDim.x) * blockDim.x) {
@@ -198,7 +204,7 @@ __global__ void __launch_bounds__(256)
                         qv[e] = Q[j * d + k0 + e];
             }
         }
-        uint16_t *dst = img + (tb * S::NCOLS + static_cast<int64_t>(r) * M) * 64 + 8 * c;
+        uint16_t *dst = img + (tb * vg::NCOLS + static_cast<int64_t>(r) * M) * 64 + 8 * c;
 #pragma unroll
         for (int b = 0; b < M; ++b) {
             uint32_t out[4];
@@ -211,31 +217,31 @@ __global__ void __launch_bounds__(256)
     }
 }
 
-// The residual image (M == 0) with one task per (row tile, row, 8 coordinates): the task forms its
-// 8 residuals r = c[q] - w (C == nullptr: r = -w) once, scales them by 2^rexp of the row and
-// writes the row's three fp16 piece columns (16 bytes each).
+// The residual image with one task per (row tile, row, 8 coordinates): the task forms its 8
+// residuals r = c[q] - w (C == nullptr: r = -w) once, scales them by 2^rexp of the row and writes
+// the two fp16 pieces R1 = fp16(r), R2 = fp16(r - R1) (16 bytes each).
 __global__ void __launch_bounds__(256)
     residual_image_kernel(const uint8_t *__restrict__ Q, const float *__restrict__ W,
                           const float *__restrict__ C, const int32_t *__restrict__ rexp, int64_t d,
                           int64_t rows_per_group, int row_tiles_per_group, int64_t ntasks, int nk,
                           int m, uint16_t *__restrict__ img)
 {
-    using S = VgShape<0>;
+    constexpr int RT = VgShape<0>::RT;
     const bool vec = (d & 7) == 0 && (reinterpret_cast<uintptr_t>(Q) & 7u) == 0 &&
                      (reinterpret_cast<uintptr_t>(W) & 15u) == 0;
     for (int64_t task = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; task < ntasks;
          task += static_cast<int64_t>(gridDim.x) * blockDim.x) {
         const int c = static_cast<int>(task & 7);
-        const int r = static_cast<int>((task >> 3) % S::RT);
-        const int64_t tb = (task >> 3) / S::RT;
+        const int r = static_cast<int>((task >> 3) % RT);
+        const int64_t tb = (task >> 3) / RT;
         const int kb = static_cast<int>(tb % nk);
         const int rt_all = static_cast<int>(tb / nk);
         const int g = rt_all / row_tiles_per_group;
         const int rt = rt_all - g * row_tiles_per_group;
         const int64_t gstart = static_cast<int64_t>(g) * rows_per_group;
-        const int64_t j = gstart + static_cast<int64_t>(rt) * S::RT + r;
+        const int64_t j = gstart + static_cast<int64_t>(rt) * RT + r;
         const int64_t k0 = static_cast<int64_t>(kb) * 64 + 8 * c;
-        uint32_t out[3][4] = {{0u, 0u, 0u, 0u}, {0u, 0u, 0u, 0u}, {0u, 0u, 0u, 0u}};
+        uint32_t out[2][4] = {{0u, 0u, 0u, 0u}, {0u, 0u, 0u, 0u}};
         if (j < gstart + rows_per_group && k0 < d) {
             uint8_t qv[8];
             float wv[8];
@@ -263,33 +269,30 @@ __global__ void __launch_bounds__(256)
             for (int e = 0; e < 8; ++e) {
                 if (qv[e] == 0xFFu)
                     continue;
-                const float rv = (C != nullptr ? C[j * m + (qv[e] & (m - 1))] : 0.f) - wv[e];
-                uint16_t b0, b1, b2;
-                split3_f16(rv * sc, b0, b1, b2);
+                const float rv = ((C != nullptr ? C[j * m + (qv[e] & (m - 1))] : 0.f) - wv[e]) * sc;
+                const __half p1 = __float2half_rn(rv);
+                const __half p2 = __float2half_rn(rv - __half2float(p1));
                 const int sh = 16 * (e & 1);
-                out[0][e >> 1] |= static_cast<uint32_t>(b0) << sh;
-                out[1][e >> 1] |= static_cast<uint32_t>(b1) << sh;
-                out[2][e >> 1] |= static_cast<uint32_t>(b2) << sh;
+                out[0][e >> 1] |= static_cast<uint32_t>(__half_as_ushort(p1)) << sh;
+                out[1][e >> 1] |= static_cast<uint32_t>(__half_as_ushort(p2)) << sh;
             }
         }
-        uint16_t *dst = img + (tb * S::NCOLS + static_cast<int64_t>(r) * 3) * 64 + 8 * c;
+        const int base_row = (r >> 6) * vg::HALF + (r & 63);
+        uint16_t *dst = img + (tb * vg::NCOLS + base_row) * 64 + 8 * c;
 #pragma unroll
-        for (int pc = 0; pc < 3; ++pc)
-            *reinterpret_cast<uint4 *>(dst + static_cast<int64_t>(pc) * 64) =
+        for (int pc = 0; pc < 2; ++pc)
+            *reinterpret_cast<uint4 *>(dst + static_cast<int64_t>(pc) * 64 * 64) =
                 make_uint4(out[pc][0], out[pc][1], out[pc][2], out[pc][3]);
     }
 }
 
 struct VgParams {
     const uint8_t *Q;   // [d_out][d]
-    const float *W;     // [d_out][d]
-    const float *C;     // [d_out][m]
-    float *V;           // [d_out][d][m] (m > 0)
-    float *U;           // [d_out][d] u = F r per row
-    const int32_t *fexp;  // [groups][d] row scales of the fp16 pieces of F (fp16 mode)
-    const int32_t *rexp;  // [d_out] residual scales (fp16 mode)
+    float *S;           // [2 i_pairs][d_out][m][m] class-binned partial sums (m > 0)
+    float *U;           // [d_out][d] u = F r per row (m == 0)
+    const int32_t *fexp;  // [groups][d] row scales of the fp16 pieces of F
+    const int32_t *rexp;  // [d_out] residual scales
     int64_t d, d_out, rows_per_group;
-    int m;
     int row_tiles_per_group, i_pairs, num_tiles;
     DeviceErr err;
 };
@@ -311,6 +314,11 @@ __device__ __forceinline__ void vg_tile_coords(const VgParams &p, int tile, int 
     row_end = min(row0 + RT, gstart + p.rows_per_group);
 }
 
+// First K block of a tile: the class-binned product covers the upper block triangle (K blocks of
+// the diagonal pair block and beyond), the residual product all of K.
+template <int M>
+__device__ __forceinline__ int vg_first_kb(int ip) { return M > 0 ? ip * vg::PAIR_KB : 0; }
+
 template <int M>
 __global__ void __launch_bounds__(vg::NUM_THREADS, 1)
     lnq_vgemm_kernel(const __grid_constant__ CUtensorMap fmap, const __grid_constant__ CUtensorMap bmap,
@@ -319,12 +327,14 @@ __global__ void __launch_bounds__(vg::NUM_THREADS, 1)
     using namespace vg;
     using S = VgShape<M>;
     constexpr int NSLOT = S::A_SLOTS;
-    constexpr uint32_t IDESC = umma_idesc_f16kind(2 * BM, S::NCOLS, false, false, true);
+    constexpr uint32_t IDESC = umma_idesc_f16kind(2 * BM, NCOLS, false, false, true);
+    constexpr uint32_t IDESC_R1 = umma_idesc_f16kind(2 * BM, NCOLS / 2, false, false, true);
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(align_up(reinterpret_cast<uintptr_t>(smem_raw), 1024));
     uint8_t *a_base = smem;                                       // [NSLOT][16 KB]
     uint8_t *b_base = smem + NSLOT * A_TILE;                      // [B_STAGES][B_BYTES]
-    uint64_t *bars = reinterpret_cast<uint64_t *>(b_base + B_STAGES * S::B_BYTES);
+    uint8_t *e_base = b_base + B_STAGES * B_BYTES;                // epilogue staging (M > 0)
+    uint64_t *bars = reinterpret_cast<uint64_t *>(e_base + S::EPI_BYTES);
     uint64_t *a_full = bars;                                      // [NSLOT] (the even CTA's count)
     uint64_t *a_empty = a_full + NSLOT;                           // [NSLOT]
     uint64_t *b_full = a_empty + NSLOT;                           // [B_STAGES] (the even CTA's count)
@@ -381,16 +391,16 @@ __global__ void __launch_bounds__(vg::NUM_THREADS, 1)
                 int64_t row0, row_end;
                 vg_tile_coords<M>(p, tile, g, row0, row_end, ip, rt_all);
                 const int i0 = ip * 2 * BM + static_cast<int>(cr) * BM;
-                for (int kb = 0; kb < nk && ok; ++kb) {
+                for (int kb = vg_first_kb<M>(ip); kb < nk && ok; ++kb) {
                     if (!mbar_wait(&b_empty[bs], ((bpar >> bs) & 1u) ^ 1u, limit)) {
                         raise_error(p.err, kErrTimeout, 17);
                         ok = false;
                         break;
                     }
                     if (cr == 0)
-                        mbar_arrive_expect_tx(&b_full[bs], 2 * S::B_BYTES);
-                    tma_load_2d_pair(b_base + bs * S::B_BYTES, &bmap, cluster_addr(&b_full[bs], 0), 0,
-                                     (rt_all * nk + kb) * S::NCOLS + static_cast<int>(cr) * S::HALF);
+                        mbar_arrive_expect_tx(&b_full[bs], 2 * B_BYTES);
+                    tma_load_2d_pair(b_base + bs * B_BYTES, &bmap, cluster_addr(&b_full[bs], 0), 0,
+                                     (rt_all * nk + kb) * NCOLS + static_cast<int>(cr) * HALF);
                     bpar ^= 1u << bs;
                     bused |= 1u << bs;
                     bs = (bs + 1 == B_STAGES) ? 0 : bs + 1;
@@ -430,19 +440,28 @@ __global__ void __launch_bounds__(vg::NUM_THREADS, 1)
         }
     } else if (warp == 1) {
         // ---------------------------------------------------------------- MMA issue (even CTA)
-        // Per K block: wait for both CTAs' right-operand halves, then for each piece wait for
-        // both CTAs' F tiles, issue four K=16 MMAs (M = 256 over the pair) and release the slot
-        // in both CTAs; release the stage after the block, the accumulator after the segment.
+        // Per K block: wait for both CTAs' right-operand halves, then for each piece of F wait for
+        // both CTAs' tiles, issue four K=16 MMAs (M = 256 over the pair) and release the slot in
+        // both CTAs; release the stage after the block, the accumulator after the segment.
+        //   class-binned: H1 and H2 against all 256 columns; the first MMA after the diagonal pair
+        //     block (K block 4 of the tile) halves what the accumulator holds.
+        //   residual: H1 against all 256 columns, H2 against the R1 halves (N = 128) into the
+        //     columns 64 .. 191, which belong to the same rows.
         if (cr == 0 && lane == 0) {
             int slot = 0, bstage = 0;
             uint32_t aph = 0u, bph = 0u;  // phase parity per slot / stage
             bool ok = true;
             int itn = 0;  // segments issued: accumulator itn % SETS
-            const int segk = S::SEGK > 0 ? S::SEGK : nk;
             for (int tile = pair; tile < p.num_tiles && ok; tile += npairs) {
+                int g, ip, rt_all;
+                int64_t row0, row_end;
+                vg_tile_coords<M>(p, tile, g, row0, row_end, ip, rt_all);
+                const int klo = vg_first_kb<M>(ip);
+                const int segk = S::SEGK > 0 ? S::SEGK : nk - klo;
                 int acc = 0;
-                for (int kb = 0; kb < nk && ok; ++kb) {
-                    const bool seg_start = kb % segk == 0;
+                for (int kb = klo; kb < nk && ok; ++kb) {
+                    const int kr = kb - klo;
+                    const bool seg_start = kr % segk == 0;
                     if (seg_start) {
                         acc = itn % S::SETS;
                         if (!mbar_wait_cluster(&tempty[acc], ((itn / S::SETS) & 1) ^ 1, limit)) {
@@ -459,8 +478,8 @@ __global__ void __launch_bounds__(vg::NUM_THREADS, 1)
                     }
                     bph ^= 1u << bstage;
                     tc_fence_after();
-                    const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * S::NCOLS);
-                    const uint32_t sb = smem_u32(b_base + bstage * S::B_BYTES);
+                    const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * NCOLS);
+                    const uint32_t sb = smem_u32(b_base + bstage * B_BYTES);
                     for (int pc = 0; pc < S::PIECES; ++pc) {
                         if (!mbar_wait(&a_full[slot], (aph >> slot) & 1u, limit)) {
                             raise_error(p.err, kErrTimeout, 16);
@@ -475,8 +494,18 @@ __global__ void __launch_bounds__(vg::NUM_THREADS, 1)
                             // K-major, 128-byte swizzle: 16 k = 32 bytes along the row
                             const uint64_t ad = umma_desc_sw128(sa + kk * 32, 16, 1024);
                             const uint64_t bd = umma_desc_sw128(sb + kk * 32, 16, 1024);
-                            umma_f16_pair(d_tmem, ad, bd, IDESC,
-                                          (!seg_start || pc != 0 || kk != 0) ? 1u : 0u);
+                            const bool first = seg_start && pc == 0 && kk == 0;
+                            if constexpr (M > 0) {
+                                if (kr == PAIR_KB && pc == 0 && kk == 0)
+                                    umma_f16_pair_halve_d(d_tmem, ad, bd, IDESC);
+                                else
+                                    umma_f16_pair(d_tmem, ad, bd, IDESC, first ? 0u : 1u);
+                            } else {
+                                if (pc == 0)
+                                    umma_f16_pair(d_tmem, ad, bd, IDESC, first ? 0u : 1u);
+                                else
+                                    umma_f16_pair(d_tmem + NCOLS / 4, ad, bd, IDESC_R1, 1u);
+                            }
                         }
                         umma_commit_pair(&a_empty[slot], PAIR);
                         slot = (slot + 1 == NSLOT) ? 0 : slot + 1;
@@ -485,7 +514,7 @@ __global__ void __launch_bounds__(vg::NUM_THREADS, 1)
                         break;
                     umma_commit_pair(&b_empty[bstage], PAIR);
                     bstage = (bstage + 1 == B_STAGES) ? 0 : bstage + 1;
-                    if (kb % segk == segk - 1 || kb + 1 == nk) {
+                    if (kr % segk == segk - 1 || kb + 1 == nk) {
                         umma_commit_pair(&tfull[acc], PAIR);
                         ++itn;
                     }
@@ -498,89 +527,197 @@ __global__ void __launch_bounds__(vg::NUM_THREADS, 1)
         // ---------------------------------------------------------------- epilogue (warps 2-5)
         // This CTA's TMEM: lane = one of its 128 coordinates, columns = all of the tile's columns.
         const int quarter = warp & 3;
+        const int tid = quarter * 32 + lane;   // coordinate of this thread within the CTA's 128
         uint32_t tempty_leader[S::SETS];
 #pragma unroll
         for (int a = 0; a < S::SETS; ++a)
             tempty_leader[a] = cluster_addr(&tempty[a], 0);
         int itn = 0;  // segments read: accumulator itn % SETS
-        const int segk = S::SEGK > 0 ? S::SEGK : nk;
-        const int nseg = (nk + segk - 1) / segk;
         bool ok = true;
-        for (int tile = pair; tile < p.num_tiles && ok; tile += npairs) {
-            int g, ip, rt_all;
-            int64_t row0, row_end;
-            vg_tile_coords<M>(p, tile, g, row0, row_end, ip, rt_all);
-            const int64_t i = static_cast<int64_t>(ip) * 2 * BM + static_cast<int64_t>(cr) * BM +
-                              quarter * 32 + lane;
-            // the accumulator carries 2^fexp[i] (and 2^rexp[j] on residual columns)
-            const float inv_si =
-                pow2f(i < p.d ? -p.fexp[static_cast<int64_t>(g) * p.d + i] : 0);
-            // residual product: per row, the sum over segments of its three piece columns
-            float uacc[M > 0 ? 1 : S::RT];
-#pragma unroll
-            for (int r = 0; r < (M > 0 ? 1 : S::RT); ++r)
-                uacc[r] = 0.f;
-            for (int sg = 0; sg < nseg; ++sg, ++itn) {
+        auto wait_acc = [&](int acc) -> bool {
+            int okw = 0;
+            if (lane == 0)
+                okw = mbar_wait(&tfull[acc], (itn / S::SETS) & 1, limit) ? 1 : 0;
+            okw = __shfl_sync(0xffffffffu, okw, 0);
+            if (!okw) {
+                if (lane == 0)
+                    raise_error(p.err, kErrTimeout, 15);
+                return false;
+            }
+            __syncwarp();
+            tc_fence_after();
+            return true;
+        };
+        if constexpr (M > 0) {
+            // Class binning. Per 32-column chunk (32 / M rows of M columns) all 128 threads stage
+            // their coordinate's values in shared memory, then thread (pair pidx = row-in-chunk x
+            // class q, part h) adds the values of the coordinates 4 ii + h (ii = 0..31) that have
+            // class q, and the four parts combine in a fixed order: S[q][.] of the row.
+            float *vs = reinterpret_cast<float *>(e_base);                 // [2][BM][VS_LD]
+            uint8_t *qs = e_base + 2 * VS_BYTES;                           // [RT][BM] codes
+            const int h = lane >> 3;
+            const int pidx = (lane & 7) | (quarter << 3);
+            const int rin = pidx / M, qcls = pidx % M;
+            constexpr int ROWS_PER_CHUNK = 32 / M;
+            const bool qvec = (p.d & 15) == 0 && (reinterpret_cast<uintptr_t>(p.Q) & 15u) == 0;
+            for (int tile = pair; tile < p.num_tiles && ok; tile += npairs) {
+                int g, ip, rt_all;
+                int64_t row0, row_end;
+                vg_tile_coords<M>(p, tile, g, row0, row_end, ip, rt_all);
+                const int64_t ibase = static_cast<int64_t>(ip) * 2 * BM + static_cast<int64_t>(cr) * BM;
+                const int ih = 2 * ip + static_cast<int>(cr);
+                const bool halve_here = nk - vg_first_kb<M>(ip) <= PAIR_KB;  // no later block
                 const int acc = itn % S::SETS;
+                // All four warps take one verdict on the accumulator (so that none of them waits at
+                // a named barrier the others have left); the barrier also ends the previous tile's
+                // binning, so its codes may be overwritten.
                 int okw = 0;
                 if (lane == 0)
                     okw = mbar_wait(&tfull[acc], (itn / S::SETS) & 1, limit) ? 1 : 0;
                 okw = __shfl_sync(0xffffffffu, okw, 0);
-                if (!okw) {
-                    if (lane == 0)
+                if (!named_bar_and(EPI_BAR, EPI_THREADS, okw)) {
+                    if (tid == 0)
                         raise_error(p.err, kErrTimeout, 15);
                     ok = false;
                     break;
                 }
-                __syncwarp();
                 tc_fence_after();
-#pragma unroll
-                for (int ch = 0; ch < S::CHUNKS; ++ch) {
+                // the tile's codes at this CTA's coordinates (0xFF: no coordinate or no row)
+                for (int e = tid; e < S::RT * (BM / 16); e += EPI_THREADS) {
+                    const int r = e / (BM / 16), c16 = e % (BM / 16);
+                    const int64_t j = row0 + r, k = ibase + 16 * c16;
+                    uint4 qv = make_uint4(0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu, 0xFFFFFFFFu);
+                    if (j < row_end && k < p.d) {
+                        if (qvec && k + 16 <= p.d) {
+                            qv = *reinterpret_cast<const uint4 *>(p.Q + j * p.d + k);
+                        } else {
+                            uint8_t *b = reinterpret_cast<uint8_t *>(&qv);
+                            for (int e2 = 0; e2 < 16; ++e2)
+                                if (k + e2 < p.d)
+                                    b[e2] = p.Q[j * p.d + k + e2];
+                        }
+                    }
+                    *reinterpret_cast<uint4 *>(qs + r * BM + 16 * c16) = qv;
+                }
+                const int64_t i = ibase + tid;
+                // the accumulator carries 2^fexp[i]; tiles without a block after the diagonal one
+                // are halved here
+                const float inv_si = pow2f(i < p.d ? -p.fexp[static_cast<int64_t>(g) * p.d + i] : 0) *
+                                     (halve_here ? 0.5f : 1.f);
+#pragma unroll 1
+                for (int ch = 0; ch < NCOLS / 32; ++ch) {
                     float v[32];
                     tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
-                                           static_cast<uint32_t>(acc * S::NCOLS + ch * 32),
+                                           static_cast<uint32_t>(acc * NCOLS + ch * 32),
                                        v);
+                    if (ch + 1 == NCOLS / 32) {
+                        tc_fence_before();
+                        mbar_arrive_cluster(tempty_leader[acc]);   // the accumulator is free
+                    }
+                    float *vrow = vs + (ch & 1) * (BM * VS_LD) + tid * VS_LD;
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const int col = ch * 32 + e;
-                        if constexpr (M > 0) {
-                            // M divides 32, so each row's M columns sit inside one chunk.
-                            if (col < S::ONEHOT && col % M == 0) {
-                                const int64_t j = row0 + col / M;
-                                if (j < row_end && i < p.d) {
-                                    float *dst = p.V + (j * p.d + i) * M;
-                                    if constexpr (M >= 4) {
+                    for (int e4 = 0; e4 < 8; ++e4)
+                        *reinterpret_cast<float4 *>(vrow + 4 * e4) =
+                            make_float4(v[4 * e4] * inv_si, v[4 * e4 + 1] * inv_si,
+                                        v[4 * e4 + 2] * inv_si, v[4 * e4 + 3] * inv_si);
+                    named_bar_sync(EPI_BAR, EPI_THREADS);      // the chunk (and the codes) staged
+                    const int rr = ch * ROWS_PER_CHUNK + rin;  // row of the tile
+                    const float *vcol = vs + (ch & 1) * (BM * VS_LD) + rin * M;
+                    const uint8_t *qrow = qs + rr * BM;
+                    float sacc[M];
 #pragma unroll
-                                        for (int b4 = 0; b4 < M / 4; ++b4)
-                                            reinterpret_cast<float4 *>(dst)[b4] = make_float4(
-                                                v[e + 4 * b4] * inv_si, v[e + 4 * b4 + 1] * inv_si,
-                                                v[e + 4 * b4 + 2] * inv_si,
-                                                v[e + 4 * b4 + 3] * inv_si);
-                                    } else {
-                                        *reinterpret_cast<float2 *>(dst) =
-                                            make_float2(v[e] * inv_si, v[e + 1] * inv_si);
-                                    }
+                    for (int c = 0; c < M; ++c)
+                        sacc[c] = 0.f;
+#pragma unroll 8
+                    for (int ii = 0; ii < BM / 4; ++ii) {
+                        const int il = 4 * ii + h;
+                        const bool mine = qrow[il] == qcls;
+                        const float *vv = vcol + il * VS_LD;
+                        if constexpr (M >= 4) {
+#pragma unroll
+                            for (int c4 = 0; c4 < M / 4; ++c4) {
+                                const float4 x = *reinterpret_cast<const float4 *>(vv + 4 * c4);
+                                if (mine) {
+                                    sacc[4 * c4] += x.x;
+                                    sacc[4 * c4 + 1] += x.y;
+                                    sacc[4 * c4 + 2] += x.z;
+                                    sacc[4 * c4 + 3] += x.w;
                                 }
                             }
                         } else {
-                            if (col < S::USED)
-                                uacc[col / 3] += v[e];
+                            const float2 x = *reinterpret_cast<const float2 *>(vv);
+                            if (mine) {
+                                sacc[0] += x.x;
+                                sacc[1] += x.y;
+                            }
                         }
                     }
-                    if constexpr (M == 0) {
-                        // the chunk's sums are complete here, before the next chunk is loaded
-                        // (otherwise the additions may be deferred and every chunk kept live)
+                    // parts h and h ^ 1, then the two pairs: the same order on every lane
 #pragma unroll
-                        for (int r = (ch * 32) / 3; r <= (ch * 32 + 31) / 3 && r < S::RT; ++r)
-                            asm volatile("" : "+f"(uacc[r]));
+                    for (int c = 0; c < M; ++c) {
+                        sacc[c] += __shfl_xor_sync(0xffffffffu, sacc[c], 8);
+                        sacc[c] += __shfl_xor_sync(0xffffffffu, sacc[c], 16);
+                    }
+                    const int64_t j = row0 + rr;
+                    if (h == 0 && j < row_end) {
+                        float *dst = p.S + ((static_cast<int64_t>(ih) * p.d_out + j) * M + qcls) * M;
+                        if constexpr (M >= 4) {
+#pragma unroll
+                            for (int c4 = 0; c4 < M / 4; ++c4)
+                                reinterpret_cast<float4 *>(dst)[c4] =
+                                    make_float4(sacc[4 * c4], sacc[4 * c4 + 1], sacc[4 * c4 + 2],
+                                                sacc[4 * c4 + 3]);
+                        } else {
+                            *reinterpret_cast<float2 *>(dst) = make_float2(sacc[0], sacc[1]);
+                        }
                     }
                 }
-                tc_fence_before();
-                mbar_arrive_cluster(tempty_leader[acc]);
+                ++itn;
             }
-            if (!ok)
-                break;
-            if constexpr (M == 0) {
+        } else {
+            // Residual sums: per segment, each of the tile's 128 rows adds its columns (R1 column,
+            // and the R2 column that also holds H2 x R1) into an fp32 sum held in registers.
+            const int nseg = (nk + S::SEGK - 1) / S::SEGK;
+            for (int tile = pair; tile < p.num_tiles && ok; tile += npairs) {
+                int g, ip, rt_all;
+                int64_t row0, row_end;
+                vg_tile_coords<M>(p, tile, g, row0, row_end, ip, rt_all);
+                const int64_t i = static_cast<int64_t>(ip) * 2 * BM + static_cast<int64_t>(cr) * BM + tid;
+                const float inv_si = pow2f(i < p.d ? -p.fexp[static_cast<int64_t>(g) * p.d + i] : 0);
+                float uacc[S::RT];
+#pragma unroll
+                for (int r = 0; r < S::RT; ++r)
+                    uacc[r] = 0.f;
+                for (int sg = 0; sg < nseg; ++sg, ++itn) {
+                    const int acc = itn % S::SETS;
+                    if (!wait_acc(acc)) {
+                        ok = false;
+                        break;
+                    }
+#pragma unroll
+                    for (int ch = 0; ch < NCOLS / 32; ++ch) {
+                        float v[32];
+                        tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
+                                               static_cast<uint32_t>(acc * NCOLS + ch * 32),
+                                           v);
+                        // column c belongs to row (c / 128) * 64 + c % 64
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) {
+                            const int col = ch * 32 + e;
+                            uacc[(col >> 7) * 64 + (col & 63)] += v[e];
+                        }
+                        // the chunk's sums are complete here, before the next chunk is loaded
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) {
+                            const int col = ch * 32 + e;
+                            asm volatile("" : "+f"(uacc[(col >> 7) * 64 + (col & 63)]));
+                        }
+                    }
+                    tc_fence_before();
+                    mbar_arrive_cluster(tempty_leader[acc]);
+                }
+                if (!ok)
+                    break;
                 if (i < p.d) {
 #pragma unroll
                     for (int r = 0; r < S::RT; ++r) {
@@ -648,15 +785,15 @@ bool encode_f16_pieces(CUtensorMap *map, const __half *Fh, int64_t d, int groups
     return encode_pieces_map(map, Fh, d, groups * 2, CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
 }
 
-// Right-operand image rows for m (M > 0 layout) or for the residual-only product: the workspace
-// holds the larger of the two.
+// Right-operand image rows for m (M > 0 layout) or for the residual product: the workspace holds
+// the larger of the two.
 template <int M>
 static int64_t image_rows_m(int64_t d, int64_t d_out, int groups)
 {
     using S = VgShape<M>;
     const int64_t R = d_out / groups;
     const int64_t nk = (d + vg::BK - 1) / vg::BK;
-    return groups * ((R + S::RT - 1) / S::RT) * nk * S::NCOLS;
+    return groups * ((R + S::RT - 1) / S::RT) * nk * vg::NCOLS;
 }
 
 size_t lnq_vgemm_image_bytes(int64_t d, int64_t d_out, int groups, int m)
@@ -674,8 +811,16 @@ size_t lnq_vgemm_image_bytes(int64_t d, int64_t d_out, int groups, int m)
     return static_cast<size_t>(rows) * 64 * 2;
 }
 
+// Class-binned partial sums: one m x m block per row and per 128 coordinates.
+size_t lnq_binned_bytes(int64_t d, int64_t d_out, int m)
+{
+    const int64_t halves = 2 * ((d + 2 * vg::BM - 1) / (2 * vg::BM));
+    return static_cast<size_t>(halves) * d_out * m * m * sizeof(float);
+}
+
 template <int M>
-static cudaError_t launch_vgemm_m(const CUtensorMap &map, VgParams p, uint16_t *img, int num_sms,
+static cudaError_t launch_vgemm_m(const CUtensorMap &map, VgParams p, const float *W,
+                                  const float *C, int m, uint16_t *img, int num_sms,
                                   cudaStream_t s, const char *name)
 {
     using S = VgShape<M>;
@@ -684,7 +829,7 @@ static cudaError_t launch_vgemm_m(const CUtensorMap &map, VgParams p, uint16_t *
     const int64_t groups = p.d_out / p.rows_per_group;
     const int nk = static_cast<int>((p.d + vg::BK - 1) / vg::BK);
     const int64_t num_rt_all = groups * p.row_tiles_per_group;
-    const int64_t img_rows = num_rt_all * nk * S::NCOLS;
+    const int64_t img_rows = num_rt_all * nk * vg::NCOLS;
     if (img_rows > 0x7fffffffLL || num_rt_all * p.i_pairs > 0x7fffffffLL)
         return cudaErrorInvalidValue;
     p.num_tiles = static_cast<int>(num_rt_all * p.i_pairs);
@@ -700,8 +845,8 @@ static cudaError_t launch_vgemm_m(const CUtensorMap &map, VgParams p, uint16_t *
                 p.Q, p.d, p.rows_per_group, p.row_tiles_per_group, ntasks, nk, img);
         } else {
             residual_image_kernel<<<static_cast<unsigned>(tblocks), 256, 0, s>>>(
-                p.Q, p.W, p.C, p.rexp, p.d, p.rows_per_group, p.row_tiles_per_group, ntasks, nk,
-                p.m, img);
+                p.Q, W, C, p.rexp, p.d, p.rows_per_group, p.row_tiles_per_group, ntasks, nk, m,
+                img);
         }
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess)
@@ -714,10 +859,11 @@ static cudaError_t launch_vgemm_m(const CUtensorMap &map, VgParams p, uint16_t *
             return cudaErrorInvalidValue;
         cuuint64_t dims[2] = {64, static_cast<cuuint64_t>(img_rows)};
         cuuint64_t strides[1] = {128};
-        cuuint32_t box[2] = {64, static_cast<cuuint32_t>(S::HALF)};
+        cuuint32_t box[2] = {64, static_cast<cuuint32_t>(vg::HALF)};
         cuuint32_t estr[2] = {1, 1};
-        if (encode(&bmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, img, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+        if (encode(&bmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, img, dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return cudaErrorInvalidValue;
     }
@@ -744,8 +890,10 @@ static cudaError_t launch_vgemm_m(const CUtensorMap &map, VgParams p, uint16_t *
         cfg.gridDim = dim3(static_cast<unsigned>(num_sms & ~1));
         int clusters = 0;
         if (cudaOccupancyMaxActiveClusters(&clusters, lnq_vgemm_kernel<M>, &cfg) != cudaSuccess ||
-            clusters < 1)
+            clusters < 1) {
+            (void)cudaGetLastError();   // a failed query is not an error of this call
             clusters = num_sms / 2;
+        }
         resident[slot] = clusters;
     }
     int pairs = resident[slot];
@@ -761,36 +909,34 @@ static cudaError_t launch_vgemm_m(const CUtensorMap &map, VgParams p, uint16_t *
     return cudaGetLastError();
 }
 
-// V = F P for every row (m in {2,4,8,16}) or, with residual_only, U = F r with the residual scales
-// rexp (C == nullptr: the zero codebook, U = -F w), both from the fp16 pieces (Fh, fexp).
-cudaError_t lnq_vgemm(const __half *Fh, const int32_t *fexp,
-                      const int32_t *rexp, int groups, const uint8_t *Q, const float *W,
-                      const float *C, float *V, float *U, uint16_t *img, int64_t d, int64_t d_out,
-                      int m, bool residual_only, DeviceErr err, int num_sms, cudaStream_t s)
+// The class-binned partial sums Sb of M = P^T F P for every row (m in {2,4,8,16}), or, with
+// residual_only, U = F r with the residual scales rexp (C == nullptr: the zero codebook, U = -F w),
+// both from the fp16 pieces (Fh, fexp).
+cudaError_t lnq_vgemm(const __half *Fh, const int32_t *fexp, const int32_t *rexp, int groups,
+                      const uint8_t *Q, const float *W, const float *C, float *Sb, float *U,
+                      uint16_t *img, int64_t d, int64_t d_out, int m, bool residual_only,
+                      DeviceErr err, int num_sms, cudaStream_t s)
 {
     CUtensorMap map;
     if (!encode_f16_pieces(&map, Fh, d, groups))
         return cudaErrorInvalidValue;
     VgParams p{};
     p.Q = Q;
-    p.W = W;
-    p.C = C;
-    p.V = V;
+    p.S = Sb;
     p.U = U;
     p.fexp = fexp;
     p.rexp = rexp;
     p.d = d;
     p.d_out = d_out;
     p.rows_per_group = d_out / groups;
-    p.m = m;
     p.err = err;
     if (residual_only)
-        return launch_vgemm_m<0>(map, p, img, num_sms, s, "lnq_residual_gemm");
+        return launch_vgemm_m<0>(map, p, W, C, m, img, num_sms, s, "lnq_residual_gemm");
     switch (m) {
-    case 2: return launch_vgemm_m<2>(map, p, img, num_sms, s, "lnq_vgemm");
-    case 4: return launch_vgemm_m<4>(map, p, img, num_sms, s, "lnq_vgemm");
-    case 8: return launch_vgemm_m<8>(map, p, img, num_sms, s, "lnq_vgemm");
-    case 16: return launch_vgemm_m<16>(map, p, img, num_sms, s, "lnq_vgemm");
+    case 2: return launch_vgemm_m<2>(map, p, W, C, m, img, num_sms, s, "lnq_mgemm");
+    case 4: return launch_vgemm_m<4>(map, p, W, C, m, img, num_sms, s, "lnq_mgemm");
+    case 8: return launch_vgemm_m<8>(map, p, W, C, m, img, num_sms, s, "lnq_mgemm");
+    case 16: return launch_vgemm_m<16>(map, p, W, C, m, img, num_sms, s, "lnq_mgemm");
     }
     return cudaErrorInvalidValue;
 }

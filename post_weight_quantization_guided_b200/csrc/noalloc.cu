@@ -14,6 +14,7 @@
 #include <mutex>
 
 #include "common.cuh"
+#include "lnq_internal.cuh"
 
 namespace lnq {
 namespace {
@@ -24,8 +25,12 @@ constexpr int kMaxDevices = 64;
 std::mutex g_addr_mu;
 void *g_addr[kMaxDevices] = {};
 
+}  // namespace
+
 // Device address of the scratch array on the current device; nullptr if it cannot be found.
-void *scratch_address()
+// Looked up once per device and cached: the cached address does not survive a cudaDeviceReset of
+// that device (the library must not be used across one).
+void *noalloc_scratch_address()
 {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
@@ -40,7 +45,6 @@ void *scratch_address()
     return g_addr[dev];
 }
 
-}  // namespace
 }  // namespace lnq
 
 extern "C" LNQ_API lnq_status lnq_build_fisher_noalloc(const uint16_t *X, const uint16_t *G,
@@ -55,7 +59,7 @@ extern "C" LNQ_API lnq_status lnq_build_fisher_noalloc(const uint16_t *X, const 
                             : lnq_workspace_size(LNQ_OP_BUILD_FISHER, n, d_in, d_out, groups, 0);
     if (need > static_cast<size_t>(LNQ_NOALLOC_SCRATCH_BYTES))
         return LNQ_ERR_WORKSPACE;
-    void *scratch = lnq::scratch_address();
+    void *scratch = lnq::noalloc_scratch_address();
     if (scratch == nullptr)
         return LNQ_ERR_CUDA;
     // The regular entry point zeroes what must start at zero (the error header and the per-group

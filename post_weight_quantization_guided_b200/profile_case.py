@@ -7,7 +7,8 @@ the objective on a named synthetic workload, optionally with fewer output rows (
 multiple of the group count) so that a capture stays small. It prints the objective's sum so that
 a run can be checked to have completed.
 
-With `--lut N` it then packs the codes and runs the lookup-table GEMV N times on one activation
+With `--fisher-only` it stops after building the blocks twice (`--tokens` shortens n). With
+`--lut N` it then packs the codes and runs the lookup-table GEMV N times on one activation
 vector (the codes cycled through enough copies that they come from HBM). With `--diag N` it runs
 N calls of LNQ with diagonal Fisher blocks (the diagonals of the blocks just built, `--iters`
 iterations each, from the initial codebooks).
@@ -32,15 +33,25 @@ def main(argv=None) -> None:
     ap.add_argument("--lut", type=int, default=0, help="lookup-table GEMV calls after the run")
     ap.add_argument("--diag", type=int, default=0,
                     help="calls of LNQ with diagonal Fisher blocks after the run")
+    ap.add_argument("--fisher-only", action="store_true",
+                    help="build the Fisher blocks (twice) and stop")
+    ap.add_argument("--tokens", type=int, default=0, help="calibration tokens (default: the workload's)")
     args = ap.parse_args(argv)
     layer = WORKLOADS[args.workload]
     if args.rows:
         if args.rows % layer.groups:
             raise SystemExit(f"--rows must be a multiple of {layer.groups}")
         layer = wl.scaled(layer, d_out=args.rows)
+    if args.tokens:
+        layer = wl.scaled(layer, n=args.tokens)
     dev = torch.device("cuda:0")
     X, G, W = wl.make_layer(layer, dev)
     F = api.lnq_build_fisher(X, G, layer.groups)
+    if args.fisher_only:
+        api.lnq_build_fisher(X, G, layer.groups, F=F)
+        torch.cuda.synchronize()
+        print(f"{layer.name} n={layer.n} fisher sum(diag)={float(torch.diagonal(F, dim1=1, dim2=2).sum()):.6e}")
+        return
     C, Q = api.lnq_init_codebook(W, layer.m)
     J = torch.empty(layer.d_out, dtype=torch.float64, device=dev)
     st = torch.empty(layer.d_out, dtype=torch.int32, device=dev)

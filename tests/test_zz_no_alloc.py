@@ -39,7 +39,7 @@ def _max_rel(F1, F2):
 
 def test_rejects_problems_beyond_the_static_scratch(b):
     fake = 0x100000
-    n, d_in, d_out, groups = 65536, 4096, 4096, 4       # needs ~2.7 GB of scratch
+    n, d_in, d_out, groups = 1 << 22, 4096, 4096, 8     # s_g alone needs 128 MiB of scratch
     assert b.lnq_workspace_size(b.LNQ_OP_BUILD_FISHER, n, d_in, d_out, groups) > 64 << 20
     st = b.lib().lnq_build_fisher_noalloc(fake, fake, n, d_in, d_out, groups, ctypes.c_float(1.0),
                                           fake, None)
@@ -75,3 +75,30 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls(b):
     F_na = b.lnq_build_fisher_noalloc(X, None, 1)
     torch.cuda.synchronize()
     assert _max_rel(F_na, F_ref) <= F_TOL
+
+
+@pytest.mark.gpu
+def test_noalloc_timeout_is_reported_through_the_static_scratch(b):
+    """A bounded wait that gives up inside the no-allocation call sets the flag in the static
+    array's header; lnq_workspace_check(NULL) reads it as LNQ_ERR_TIMEOUT, and the next call with
+    the default limit is correct again."""
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from post_weight_quantization_guided_b200 import workloads as wl
+    dev = torch.device("cuda:0")
+    layer = wl.scaled(wl.TINY, n=512, d_in=256, d_out=8, groups=2)
+    X, G, _ = wl.make_layer(layer, dev)
+    F_ref = b.lnq_build_fisher(X, G, layer.groups)
+    F_na = torch.empty_like(F_ref)
+    assert b.lnq_noalloc_check() == b.LNQ_OK
+    try:
+        b.lnq_set_wait_limit(0)
+        b.lnq_build_fisher_noalloc(X, G, layer.groups, F=F_na)
+        assert b.lnq_noalloc_check() == b.LNQ_ERR_TIMEOUT
+    finally:
+        b.lnq_set_wait_limit(-1)
+    assert b.lnq_noalloc_check() == b.LNQ_OK                # the check cleared the flag
+    b.lnq_build_fisher_noalloc(X, G, layer.groups, F=F_na)
+    assert b.lnq_noalloc_check() == b.LNQ_OK
+    assert _max_rel(F_na, F_ref) <= F_TOL
+
