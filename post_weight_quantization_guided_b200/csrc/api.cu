@@ -15,11 +15,11 @@ namespace lnq {
 
 // Kernels and launchers defined in fisher.cu.
 __global__ void token_stats_kernel(const __nv_bfloat16 *, const __nv_bfloat16 *, int64_t, int64_t,
-                                   int64_t, int, float *, float *, unsigned *);
-__global__ void token_scales_kernel(int64_t, int, float *, float *, const unsigned *);
+                                   int64_t, int64_t, int, float *, float *, unsigned *);
+__global__ void token_scales_kernel(int64_t, int64_t, int, float *, float *, const unsigned *);
 cudaError_t fisher_syrk(const __nv_bfloat16 *X, const float *S, const float *M,
-                        const unsigned *pimax, int64_t n, int64_t d, int groups, float alpha,
-                        float *F, DeviceErr err, cudaStream_t s, int num_sms);
+                        const unsigned *pimax, int64_t n, int64_t ld, int64_t d, int groups,
+                        float alpha, float *F, DeviceErr err, cudaStream_t s, int num_sms);
 
 static std::atomic<long long> g_wait_limit{kDefaultWaitLimit};
 
@@ -37,7 +37,8 @@ static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 
 static bool valid_m(int m) { return m == 2 || m == 4 || m == 8 || m == 16; }
 
 // Workspace layout (all offsets 256-byte aligned):
-//   BUILD_FISHER:   header | S [groups][n] f32 | M [n] f32 | pimax [groups] u32
+//   BUILD_FISHER:   header | S [groups][ld] f32 | M [ld] f32 | pimax [groups] u32
+//                   (ld = n rounded up to a multiple of 64)
 //   QUANTIZE_ROWS:  header | status [d_out] i32 | Fh [groups][2][d_in][ld] f16 (ld = d_in
 //                   rounded up to a multiple of 8) | fexp [groups][d_in] i32 | rexp [d_out] i32
 //                   | Sb [2 ceil(d_in / 256)][d_out][m][m] f32 (class-binned partial sums)
@@ -49,12 +50,14 @@ static bool valid_m(int m) { return m == 2 || m == 4 || m == 8 || m == 16; }
 struct FisherWs {
     size_t s_off, m_off, pi_off, total;
 };
+static int64_t fisher_ld(int64_t n) { return (n + 63) / 64 * 64; }
 static FisherWs fisher_ws(int64_t n, int groups)
 {
     FisherWs w;
+    const int64_t ld = fisher_ld(n);
     w.s_off = kWsHeader;
-    w.m_off = align_up(w.s_off + static_cast<size_t>(groups) * n * sizeof(float), 256);
-    w.pi_off = align_up(w.m_off + static_cast<size_t>(n) * sizeof(float), 256);
+    w.m_off = align_up(w.s_off + static_cast<size_t>(groups) * ld * sizeof(float), 256);
+    w.pi_off = align_up(w.m_off + static_cast<size_t>(ld) * sizeof(float), 256);
     w.total = align_up(w.pi_off + static_cast<size_t>(groups) * sizeof(unsigned), 256);
     return w;
 }
@@ -177,19 +180,20 @@ lnq_status lnq_build_fisher(const uint16_t *X, const uint16_t *G, int64_t n, int
         {
             KernelTimer timer("token_stats", s);
             token_stats_kernel<<<static_cast<unsigned>((n * 32 + threads - 1) / threads), threads,
-                                 0, s>>>(Xb, reinterpret_cast<const __nv_bfloat16 *>(G), n, d_in,
-                                         d_out, groups, S, M, pimax);
+                                 0, s>>>(Xb, reinterpret_cast<const __nv_bfloat16 *>(G), n,
+                                         fisher_ld(n), d_in, d_out, groups, S, M, pimax);
         }
         {
             KernelTimer timer("token_scales", s);
-            token_scales_kernel<<<static_cast<unsigned>((n + threads - 1) / threads), threads, 0,
-                                  s>>>(n, groups, S, M, pimax);
+            token_scales_kernel<<<static_cast<unsigned>((fisher_ld(n) + threads - 1) / threads),
+                                  threads, 0, s>>>(n, fisher_ld(n), groups, S, M, pimax);
         }
         if (cudaGetLastError() != cudaSuccess)
             return LNQ_ERR_CUDA;
-        e = fisher_syrk(Xb, S, M, pimax, n, d_in, groups, alpha, F, err, s, device_sm_count());
+        e = fisher_syrk(Xb, S, M, pimax, n, fisher_ld(n), d_in, groups, alpha, F, err, s,
+                        device_sm_count());
     } else {
-        e = fisher_syrk(Xb, nullptr, nullptr, nullptr, n, d_in, 1, alpha, F, err, s,
+        e = fisher_syrk(Xb, nullptr, nullptr, nullptr, n, n, d_in, 1, alpha, F, err, s,
                         device_sm_count());
     }
     if (e == cudaErrorNotSupported)

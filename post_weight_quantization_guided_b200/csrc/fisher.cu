@@ -18,10 +18,12 @@
 //                        K=16); each CTA's four epilogue warps read its 128 rows from TMEM, scale
 //                        them and write them and their mirror image. Two TMEM accumulators let the
 //                        epilogue of one tile overlap the main loop of the next.
-//     guided (G given):  the diag(s_g) scaling is fused into the operand load. Two groups of
-//                        eight producer warps per CTA read X (bf16) straight from global memory
-//                        with 16-byte loads, each group a whole stage (two stages in flight), and
-//                        write both operands into the stage in fp16:
+//     guided (G given):  the diag(s_g) scaling is fused into the operand load. TMA brings the
+//                        stage's X tiles (bf16, the same boxes as the plain path) and the stage's
+//                        64 per-token factors of both operands into the stage; four groups of four
+//                        converter warps, each on every fourth stage, then rewrite every
+//                        16-byte chunk in place as fp16 (same swizzled
+//                        position: the chunk's row is its token):
 //                          A[t][i] = X[t][i] / P_t                  (P_t = pow2_ceil(M_t), exact)
 //                          B[t][k] = fp16(X[t][k] * s_g[t] P_t / Pi_g)   (Pi_g = pow2_ceil(max_t
 //                                                                    s_g[t] M_t^2), one rounding)
@@ -68,11 +70,12 @@ __device__ __forceinline__ float sum_squares_bf16(const __nv_bfloat16 *__restric
     return acc;
 }
 
-// One warp per token t: S[g][t] = mean_{j in g} G[t,j]^2 for every group, M[t] = max_i |X[t,i]|,
-// and pimax[g] = max over tokens of S[g][t] * M[t]^2 (positive floats compare as their bits).
+// One warp per token t: S[g][t] = mean_{j in g} G[t,j]^2 for every group (row stride ld),
+// M[t] = max_i |X[t,i]|, and pimax[g] = max over tokens of S[g][t] * M[t]^2 (positive floats compare
+// as their bits).
 __global__ void token_stats_kernel(const __nv_bfloat16 *__restrict__ X,
-                                   const __nv_bfloat16 *__restrict__ G, int64_t n, int64_t d,
-                                   int64_t d_out, int groups, float *__restrict__ S,
+                                   const __nv_bfloat16 *__restrict__ G, int64_t n, int64_t ld,
+                                   int64_t d, int64_t d_out, int groups, float *__restrict__ S,
                                    float *__restrict__ M, unsigned *__restrict__ pimax)
 {
     const int64_t t = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
@@ -99,7 +102,7 @@ __global__ void token_stats_kernel(const __nv_bfloat16 *__restrict__ X,
     for (int g = 0; g < groups; ++g) {
         const float sg = sum_squares_bf16(G + t * d_out + g * R, R, lane) / static_cast<float>(R);
         if (lane == 0) {
-            S[static_cast<int64_t>(g) * n + t] = sg;
+            S[static_cast<int64_t>(g) * ld + t] = sg;
             atomicMax(&pimax[g], __float_as_uint(sg * mx * mx));
         }
     }
@@ -121,17 +124,24 @@ __device__ __forceinline__ float pow2_ceil(float v)
 //   S[g][t] <- S[g][t] * P_t / Pi_g,       Pi_g = pow2_ceil(pimax[g])
 // so that the left operand X[t][:] / P_t is exact in fp16 (|.| <= 1), the right operand
 // fp16(X[t][:] * S[g][t] P_t / Pi_g) is rounded once (|.| <= 2), and their product is
-// s_g[t] X[t][i] X[t][k] / Pi_g. One thread per token.
-__global__ void token_scales_kernel(int64_t n, int groups, float *__restrict__ S,
+// s_g[t] X[t][i] X[t][k] / Pi_g. One thread per token of the padded range: tokens n .. ld - 1
+// get zero factors (the SYRK's stages copy whole blocks of 64).
+__global__ void token_scales_kernel(int64_t n, int64_t ld, int groups, float *__restrict__ S,
                                     float *__restrict__ M, const unsigned *__restrict__ pimax)
 {
     const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-    if (t >= n)
+    if (t >= ld)
         return;
+    if (t >= n) {
+        for (int g = 0; g < groups; ++g)
+            S[static_cast<int64_t>(g) * ld + t] = 0.f;
+        M[t] = 0.f;
+        return;
+    }
     const float Pt = pow2_ceil(M[t]);
     for (int g = 0; g < groups; ++g)
-        S[static_cast<int64_t>(g) * n + t] =
-            S[static_cast<int64_t>(g) * n + t] * Pt / pow2_ceil(__uint_as_float(pimax[g]));
+        S[static_cast<int64_t>(g) * ld + t] =
+            S[static_cast<int64_t>(g) * ld + t] * Pt / pow2_ceil(__uint_as_float(pimax[g]));
     M[t] = 1.f / Pt;
 }
 
@@ -145,34 +155,35 @@ constexpr int BN = 256;          // tile columns (k), TMEM columns per accumulat
 constexpr int HALF = BN / 2;     // columns of the right operand each CTA holds
 constexpr int BK = 64;           // tokens per pipeline stage
 constexpr int STAGES = 6;
-constexpr int BOX = 64;          // operand box: 64 elements (128 B) along i/k  x  64 tokens
+constexpr int BOX = 64;          // operand box: 64 elements (128 B) along i/k  x  BK tokens
 constexpr int BOX_BYTES = BOX * BK * 2;                  // 8 KB
 constexpr int A_BYTES = (BM / BOX) * BOX_BYTES;          // 16 KB
 constexpr int B_BYTES = (HALF / BOX) * BOX_BYTES;        // 16 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;           // 32 KB per CTA
-// warp 0 TMA (plain), warp 1 MMA, warps 2-5 epilogue, then (guided) PROD_GROUPS groups of four
-// operand-producer warps; group k fills the stages of fills k, k + PROD_GROUPS, ...
-constexpr int PROD_GROUPS = 2;
-constexpr int GROUP_THREADS = 256;
-constexpr int PROD_THREADS = PROD_GROUPS * GROUP_THREADS;
-constexpr int PROD_TOKENS = BK / (GROUP_THREADS / 16);   // tokens per producer thread and fill: 8
-__host__ __device__ constexpr int num_threads(bool guided) { return guided ? 192 + PROD_THREADS : 192; }
+// warp 0 TMA, warp 1 MMA, warps 2-5 epilogue, then (guided) CONV_GROUPS groups of four converter
+// warps; group k converts the stages of fills k, k + CONV_GROUPS, ...
+constexpr int CONV_GROUPS = 4;
+constexpr int GROUP_THREADS = 128;
+constexpr int CONV_THREADS = CONV_GROUPS * GROUP_THREADS;
+constexpr int GROUP_WARPS = GROUP_THREADS / 32;
+constexpr int SCALE_BYTES = 2 * BK * 4;                  // the stage's factors of both operands
+__host__ __device__ constexpr int num_threads(bool guided) { return guided ? 192 + CONV_THREADS : 192; }
 constexpr int TMEM_COLS = 2 * BN;                        // two accumulators
-constexpr size_t SMEM_BYTES = static_cast<size_t>(STAGES) * STAGE_BYTES + 1024 /*align*/ + 256;
+constexpr int NUM_BARS = 3 * STAGES + 5;                 // full, empty, raw_full; tfull, tempty, drain
+constexpr int BAR_BYTES = (NUM_BARS * 8 + 4 + 15) / 16 * 16;   // + the TMEM address holder
+constexpr size_t SMEM_BYTES = static_cast<size_t>(STAGES) * (STAGE_BYTES + SCALE_BYTES) +
+                              1024 /*align*/ + BAR_BYTES;
 constexpr uint16_t PAIR = 0x3;                           // both CTAs of the cluster
 constexpr long long kPairDrainLimit = 1LL << 22;
 static_assert(SMEM_BYTES <= 232448, "shared memory");
-static_assert(BK % (GROUP_THREADS / 16) == 0 && STAGES % PROD_GROUPS == 0, "producer tiling");
-// the last 16-byte chunk a producer thread writes ends at the end of its operand's half stage
-static_assert(BOX_BYTES + (BK - 1) * 128 + 7 * 16 + 16 == A_BYTES && A_BYTES == B_BYTES,
-              "producer stores stay inside their stage");
+static_assert((A_BYTES / 16) % GROUP_THREADS == 0 && A_BYTES == B_BYTES, "converter tiling");
 }  // namespace syrk
 
 struct SyrkParams {
     float *F;            // [groups][d][d]
-    const __nv_bfloat16 *X;  // [n][d] (guided: read by the producer warps)
-    const float *bfac;   // [groups][n] right-operand factor s_g[t] P_t / Pi_g (guided)
-    const float *ainv;   // [n] left-operand factor 1 / P_t (guided)
+    const float *bfac;   // [groups][ld] right-operand factor s_g[t] P_t / Pi_g (guided)
+    const float *ainv;   // [ld] left-operand factor 1 / P_t (guided)
+    int64_t ld;          // n rounded up to a multiple of 64 (guided factor rows)
     const unsigned *pimax;  // [groups] per-group operand scale (guided), or nullptr
     int64_t n, d;
     int groups;
@@ -197,28 +208,26 @@ __device__ __forceinline__ void syrk_tile_coords(const SyrkParams &p, int tile, 
     bi = r;
 }
 
-// 16-byte read-only load that does not allocate in L1 (X is shared through L2).
-__device__ __forceinline__ uint4 ldg_nc_v4(const void *p)
-{
-    uint4 v;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "l"(reinterpret_cast<uint64_t>(p)));
-    return v;
-}
-
-// 8 bf16 values times `scale`, rounded once to fp16.
+// 8 bf16 values times `scale`, rounded once to fp16: each pair is widened to fp32 (exact), both
+// halves are multiplied by one packed fp32 multiply (round to nearest, as two scalar ones) and
+// rounded to fp16 by one packed conversion.
 __device__ __forceinline__ uint4 scale_bf16x8_to_f16(uint4 x, float scale)
 {
-    const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&x);
-    uint4 out;
-    __half2 *o = reinterpret_cast<__half2 *>(&out);
+    const uint64_t sc2 = (static_cast<uint64_t>(__float_as_uint(scale)) << 32) | __float_as_uint(scale);
+    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+    uint32_t r[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-        const float2 f = __bfloat1622float2(h[e]);
-        o[e] = __floats2half2_rn(f.x * scale, f.y * scale);
+        // low element in the low word, high element in the high word
+        const uint64_t pair = (static_cast<uint64_t>(w[e] & 0xFFFF0000u) << 32) | (w[e] << 16);
+        uint64_t prod;
+        asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(prod) : "l"(pair), "l"(sc2));
+        asm("cvt.rn.f16x2.f32 %0, %1, %2;"
+            : "=r"(r[e])
+            : "f"(__uint_as_float(static_cast<uint32_t>(prod >> 32))),
+              "f"(__uint_as_float(static_cast<uint32_t>(prod))));
     }
-    return out;
+    return make_uint4(r[0], r[1], r[2], r[3]);
 }
 
 template <bool kGuided>
@@ -230,13 +239,15 @@ __device__ __forceinline__ void fisher_syrk_body(const CUtensorMap &amap, const 
                                                   /*b_mn_major=*/true, kGuided);
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(align_up(reinterpret_cast<uintptr_t>(smem_raw), 1024));
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + STAGES * STAGE_BYTES);
+    float *scales = reinterpret_cast<float *>(smem + STAGES * STAGE_BYTES);  // [STAGES][2][BK]
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + STAGES * (STAGE_BYTES + SCALE_BYTES));
     uint64_t *full = bars;                  // [STAGES] (the even CTA's counts both CTAs' fills)
     uint64_t *empty = bars + STAGES;        // [STAGES]
     uint64_t *tfull = bars + 2 * STAGES;    // [2]
     uint64_t *tempty = bars + 2 * STAGES + 2;  // [2] (the even CTA's counts both epilogues)
     uint64_t *drain = bars + 2 * STAGES + 4;
-    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 5);
+    uint64_t *raw_full = bars + 2 * STAGES + 5;  // [STAGES] guided: this CTA's copies landed
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + 3 * STAGES + 5);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -246,10 +257,11 @@ __device__ __forceinline__ void fisher_syrk_body(const CUtensorMap &amap, const 
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
-            // guided: one arrival per warp of the filling producer group in both CTAs; plain: the
-            // even CTA's expect_tx arrival, with the TMA bytes of both CTAs
-            mbar_init(&full[s], kGuided ? 2 * (GROUP_THREADS / 32) : 1);
+            // guided: one arrival per converter warp of both CTAs; plain: the even CTA's
+            // expect_tx arrival, with the TMA bytes of both CTAs
+            mbar_init(&full[s], kGuided ? 2 * GROUP_WARPS : 1);
             mbar_init(&empty[s], 1);
+            mbar_init(&raw_full[s], 1);
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(&tfull[a], 1);
@@ -257,10 +269,8 @@ __device__ __forceinline__ void fisher_syrk_body(const CUtensorMap &amap, const 
         }
         mbar_init(drain, 1);
         fence_barrier_init();
-        if (!kGuided) {
-            tma_prefetch_desc(&amap);
-            tma_prefetch_desc(&bmap);
-        }
+        tma_prefetch_desc(&amap);
+        tma_prefetch_desc(&bmap);
     }
     if (warp == 1)
         tmem_alloc_pair(tmem_holder, TMEM_COLS);
@@ -271,11 +281,60 @@ __device__ __forceinline__ void fisher_syrk_body(const CUtensorMap &amap, const 
     const int nk = static_cast<int>((p.n + BK - 1) / BK);
     const long long limit = p.err.limit;
 
-    if (warp == 0) {
+    if (warp == 0 && kGuided) {
+        // ---------------------------------------------------------------- TMA producer (guided)
+        // Per stage: this CTA's X tiles of both operands (bf16) and the stage's factors, counted
+        // on this CTA's raw_full barrier; the converters turn them into the operands in place.
+        if (lane == 0) {
+            int stage = 0, use = 0;
+            uint32_t used = 0u;
+            bool ok = true;
+            for (int tile = pair; tile < p.num_tiles && ok; tile += npairs) {
+                int g, bi, bk;
+                syrk_tile_coords(p, tile, g, bi, bk);
+                const int i0 = bi * PM + static_cast<int>(cr) * BM;
+                const int k0 = bk * BN + static_cast<int>(cr) * HALF;
+                const float *bf = p.bfac + static_cast<int64_t>(g) * p.ld;
+                for (int kb = 0; kb < nk; ++kb) {
+                    if (!mbar_wait(&empty[stage], (use & 1) ^ 1, limit)) {
+                        raise_error(p.err, kErrTimeout, 1);
+                        ok = false;
+                        break;
+                    }
+                    uint8_t *sa = smem + stage * STAGE_BYTES;
+                    float *sc = scales + stage * 2 * BK;
+                    mbar_arrive_expect_tx(&raw_full[stage], STAGE_BYTES + SCALE_BYTES);
+                    const int t0 = kb * BK;
+                    for (int b = 0; b < BM / BOX; ++b)
+                        tma_load_3d(sa + b * BOX_BYTES, &amap, &raw_full[stage], i0 + b * BOX, t0, 0);
+                    for (int b = 0; b < HALF / BOX; ++b)
+                        tma_load_3d(sa + A_BYTES + b * BOX_BYTES, &amap, &raw_full[stage],
+                                    k0 + b * BOX, t0, 0);
+                    bulk_load(sc, p.ainv + t0, BK * 4, &raw_full[stage]);
+                    bulk_load(sc + BK, bf + t0, BK * 4, &raw_full[stage]);
+                    used |= 1u << stage;
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        ++use;
+                    }
+                }
+            }
+            if (!ok) {
+                // let this CTA's copies land before it exits: wait for the last armed phase of
+                // every stage (its parity is that of the number of completed uses)
+                for (int s = 0; s < STAGES; ++s) {
+                    if (!((used >> s) & 1u))
+                        continue;
+                    const int last_use = s < stage ? use : use - 1;
+                    mbar_wait(&raw_full[s], last_use & 1, kDrainLimit);
+                }
+            }
+        }
+    } else if (warp == 0) {
         // ---------------------------------------------------------------- TMA producer (plain)
         // Per stage: this CTA's 128 rows of A and its 128 of the tile's 256 columns of B, the
         // bytes of both CTAs counted on the even CTA's barrier (armed there for both).
-        if (!kGuided && lane == 0) {
+        if (lane == 0) {
             uint32_t fpar = 0u, fused = 0u;  // per stage: parity of the fills, ever filled
             int stage = 0;
             bool ok = true;
@@ -431,58 +490,45 @@ __device__ __forceinline__ void fisher_syrk_body(const CUtensorMap &amap, const 
             mbar_arrive_cluster(tempty_leader[acc]);
         }
     } else if constexpr (kGuided) {
-        // ---------------------------------------------------------------- operand producers
-        // Group k fills the stages of fills k, k + PROD_GROUPS, ... (fill f: tile pair + (f / nk)
-        // npairs, tokens 64 (f % nk) ..). Thread pt of a group covers 8 consecutive coordinates
-        // (column c16 of 16-byte chunks, box c16 / 8) of both operands for the tokens tr + 16 j.
-        // Its element (t, 8 c16 ..) sits at row t of its box, 16-byte chunk (c16 % 8) ^ (t % 8):
-        // the 128-byte swizzle the MMA descriptors expect (t % 8 = tr % 8 for every j). A group issues
-        // all loads of its fill (X and the two per-token factors) before it waits for the stage, so
-        // the groups' fills overlap; each warp of the group arrives once on the even CTA's barrier.
-        const int pidx = threadIdx.x - 6 * 32;
-        const int grp = pidx / GROUP_THREADS;
-        const int pt = pidx % GROUP_THREADS;
-        const int c16 = pt & 15, tr = pt >> 4;
-        const uint32_t soff = static_cast<uint32_t>((c16 >> 3) * BOX_BYTES + tr * 128 +
-                                                    (((c16 & 7) ^ (tr & 7)) << 4));
-        const int64_t d = p.d, n = p.n;
-        const int total = ((p.num_tiles - pair + npairs - 1) / npairs) * nk;  // this pair's fills
+        // ---------------------------------------------------------------- operand converters
+        // Group k converts the stages of fills k, k + CONV_GROUPS, ... once this CTA's copies have
+        // landed: every 16-byte chunk of the two operand halves (8 coordinates of one token row of
+        // a box) is rewritten in place as fp16, scaled by its token's factor; the chunk's token is
+        // its row in the box, whatever the swizzle. Thread q of a group takes chunks q, q + 128, ...
+        // of each operand. Each warp arrives once on the even CTA's barrier.
+        const int cq = threadIdx.x - 6 * 32;
+        const int grp = cq / GROUP_THREADS;
+        const int q = cq % GROUP_THREADS;
+        constexpr int PER_THREAD = A_BYTES / 16 / GROUP_THREADS;  // chunks per operand
         const uint32_t full_leader_base = cluster_addr(&full[0], 0);
-        for (int f = grp; f < total; f += PROD_GROUPS) {
-            const int tile = pair + (f / nk) * npairs;
-            int g, bi, bk;
-            syrk_tile_coords(p, tile, g, bi, bk);
-            const int64_t i0 = static_cast<int64_t>(bi) * PM + static_cast<int64_t>(cr) * BM + 8 * c16;
-            const int64_t k0 = static_cast<int64_t>(bk) * BN + static_cast<int64_t>(cr) * HALF + 8 * c16;
-            const int64_t t0 = static_cast<int64_t>(f % nk) * BK + tr;
-            uint4 xa[PROD_TOKENS], xb[PROD_TOKENS];
-            float fa[PROD_TOKENS], fb[PROD_TOKENS];
-#pragma unroll
-            for (int j = 0; j < PROD_TOKENS; ++j) {
-                const int64_t t = t0 + (GROUP_THREADS / 16) * j;
-                const bool tin = t < n;
-                xa[j] = (tin && i0 < d) ? ldg_nc_v4(p.X + t * d + i0) : make_uint4(0u, 0u, 0u, 0u);
-                xb[j] = (tin && k0 < d) ? ldg_nc_v4(p.X + t * d + k0) : make_uint4(0u, 0u, 0u, 0u);
-                fa[j] = tin ? __ldg(p.ainv + t) : 0.f;
-                fb[j] = tin ? __ldg(p.bfac + static_cast<int64_t>(g) * n + t) : 0.f;
-            }
-            const int stage = f % STAGES;
+        const int total = ((p.num_tiles - pair + npairs - 1) / npairs) * nk;  // this pair's stages
+        for (int f = grp; f < total; f += CONV_GROUPS) {
+            const int stage = f % STAGES, use = f / STAGES;
             int got = 0;
             if (lane == 0)
-                got = mbar_wait(&empty[stage], ((f / STAGES) & 1) ^ 1, limit) ? 1 : 0;
+                got = mbar_wait(&raw_full[stage], use & 1, limit) ? 1 : 0;
             got = __shfl_sync(0xffffffffu, got, 0);
             if (!got) {
                 if (lane == 0)
                     raise_error(p.err, kErrTimeout, 5);
                 break;
             }
-            uint8_t *sa = smem + stage * STAGE_BYTES + soff;
+            uint8_t *sa = smem + stage * STAGE_BYTES;
+            const float *sc = scales + stage * 2 * BK;
 #pragma unroll
-            for (int j = 0; j < PROD_TOKENS; ++j) {
-                *reinterpret_cast<uint4 *>(sa + (GROUP_THREADS / 16) * j * 128) =
-                    scale_bf16x8_to_f16(xa[j], fa[j]);
-                *reinterpret_cast<uint4 *>(sa + A_BYTES + (GROUP_THREADS / 16) * j * 128) =
-                    scale_bf16x8_to_f16(xb[j], fb[j]);
+            for (int opnd = 0; opnd < 2; ++opnd) {
+                uint8_t *base = sa + opnd * A_BYTES;
+                uint4 x[PER_THREAD];
+#pragma unroll
+                for (int k = 0; k < PER_THREAD; ++k)
+                    x[k] = *reinterpret_cast<const uint4 *>(base + (q + GROUP_THREADS * k) * 16);
+#pragma unroll
+                for (int k = 0; k < PER_THREAD; ++k) {
+                    const int c = q + GROUP_THREADS * k;     // chunk of this operand's half stage
+                    const int tok = (c >> 3) & (BK - 1);      // its row in its BK-row box
+                    *reinterpret_cast<uint4 *>(base + c * 16) =
+                        scale_bf16x8_to_f16(x[k], sc[opnd * BK + tok]);
+                }
             }
             fence_proxy_async_smem();  // the stores become visible to the tensor core
             __syncwarp();
@@ -564,29 +610,27 @@ static bool encode_operand(CUtensorMap *map, const void *base, int64_t n, int64_
 
 // F_g = scale_g * (operands)^T (operands), both triangles written:
 //   S == nullptr: F = alpha X^T X, X read by TMA in bf16 (groups == 1);
-//   otherwise:    the guided blocks, operands formed by the producer warps from X and the factors
-//                 that token_scales_kernel left in S (right) and M (left),
-//                 scale_g = alpha * pow2_ceil(pimax[g]).
+//   otherwise:    the guided blocks, operands converted in the stages from X and the factors that
+//                 token_scales_kernel left in S (right, row stride ld) and M (left), ld >= n a
+//                 multiple of BK, scale_g = alpha * pow2_ceil(pimax[g]).
 cudaError_t fisher_syrk(const __nv_bfloat16 *X, const float *S, const float *M,
-                        const unsigned *pimax, int64_t n, int64_t d, int groups, float alpha,
-                        float *F, DeviceErr err, cudaStream_t s, int num_sms)
+                        const unsigned *pimax, int64_t n, int64_t ld, int64_t d, int groups,
+                        float alpha, float *F, DeviceErr err, cudaStream_t s, int num_sms)
 {
     using namespace syrk;
     const bool guided = S != nullptr;
     CUtensorMap amap, bmap;
-    memset(&amap, 0, sizeof(amap));
-    memset(&bmap, 0, sizeof(bmap));
-    if (!guided) {
-        if (tensor_map_encoder() == nullptr)
-            return cudaErrorNotSupported;
-        if (!encode_operand(&amap, X, n, d, 1, false) || !encode_operand(&bmap, X, n, d, 1, false))
-            return cudaErrorInvalidValue;
-    }
+    if (tensor_map_encoder() == nullptr)
+        return cudaErrorNotSupported;
+    if (!encode_operand(&amap, X, n, d, 1, false) || !encode_operand(&bmap, X, n, d, 1, false))
+        return cudaErrorInvalidValue;
     SyrkParams p;
     p.F = F;
-    p.X = X;
     p.bfac = S;
     p.ainv = M;
+    p.ld = ld;
+    if (guided && ld % BK != 0)
+        return cudaErrorInvalidValue;   // the stages copy whole blocks of BK factors
     p.pimax = pimax;
     p.n = n;
     p.d = d;
