@@ -165,7 +165,9 @@ def algorithmic_work(layer, m, kernel, sweep_tail=None):
         # the codebook step's M = P^T F P: d^2 / 2 FADD per row with the symmetry of F
         return 0.5 * d * d * dout, "lane_op"
     if kernel == "lnq_residual_gemm":
-        return 1.0 * d * d * dout, "lane_op"                        # u = F r: d^2 FMA per row
+        # u = F r for every row: a dense contraction of F with the residual columns, 2 d^2 flops
+        # per row (executed as three fp16 piece products on tensor cores)
+        return 2.0 * d * d * dout, "flop"
     if kernel == "lnq_solve":
         # read the binned partial sums (m x m per 128 coordinates), U and Q; write C
         halves = 2 * -(-d // 256)
