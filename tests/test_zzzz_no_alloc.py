@@ -8,8 +8,8 @@ within the F tolerance on two calls in a row (so leftovers of one call do not le
 next), it allocates no device memory, and it refuses problems larger than the array before
 touching the device.
 
-This file sorts after the parity tests so that a run stopping at the first failure has already
-run them.
+This file sorts after every other test file, so that a run stopping at the first failure has
+already run all of them.
 """
 import ctypes
 
