@@ -174,8 +174,12 @@ LNQ_API lnq_status lnq_quantize_rows(const float *F, int groups, const float *W,
  *   W, C, Q     as lnq_quantize_rows (C, Q in/out; codes are read modulo m)
  *   J_out       [d_out] fp64 out, sum_i f_i (C[j][Q[j][i]] - W[j][i])^2, or NULL
  *   row_status  [d_out] int32 out, or NULL
- * Arithmetic: class sums, cost changes and the objective in fp64, in a fixed order; results are
- * bit-identical from run to run. Needs no workspace.
+ * Arithmetic: the class sums are exact integer sums of per-coordinate fixed-point terms
+ * (rint(f_i w_i 2^s_w), rint(f_i 2^s_f), every term at most 2^41 for the row's scales); a class
+ * whose f sum is under n_a 2^24 units is summed directly in fp64 instead. Moves are decided by
+ * fp32 midpoints and confirmed by the fp64 change; objective terms in fp32, summed in fp64 in a
+ * fixed order. Results are bit-identical from run to run and across any split of the iterations
+ * over calls. Needs no workspace.
  * Requirements: non-NULL Fd, W, C, Q; m in {2, 4, 8, 16}; 1 <= d_in <= 16384; 1 <= d_out < 2^31;
  * groups >= 1 and d_out % groups == 0; iters >= 0. Otherwise LNQ_ERR_INVALID_ARG before any
  * device work; a launch failure is LNQ_ERR_CUDA. */

@@ -282,6 +282,32 @@ def test_lnq_diag_q_proj_full_size_sampled_rows(orc, lnq, wl):
     assert torch.equal(C3, C) and torch.equal(Q3, Q)
 
 
+def test_lnq_diag_small_weight_class(orc, lnq):
+    # A class whose weights f_i are 1e-9 of the row's largest: its fixed-point f sum is too coarse
+    # (mean f under 2^-17 of the largest), so the kernel sums that class directly in fp64; the
+    # codebook must still match the oracle's weighted mean to the usual tolerance.
+    gen = torch.Generator().manual_seed(11)
+    d, rows = 64, 4
+    f = torch.ones(1, d)
+    f[0, 48:] = 1e-9
+    W = torch.randn(rows, d, generator=gen) * 0.01
+    W[:, 48:] += 5.0
+    lnq_follow_parity(orc, lnq, f.to(_dev()), W.contiguous().to(_dev()), 4, 3, diag=True)
+
+
+def test_lnq_diag_mixed_sign_weights(orc, lnq):
+    # f_i < 0 on a tenth of the coordinates (small in size, so the rows keep J > 0): those
+    # coordinates take the codeword with the most negative fp64 change, the rest their nearest.
+    gen = torch.Generator().manual_seed(12)
+    d, rows, groups = 256, 8, 2
+    f = torch.exp(torch.randn(groups, d, generator=gen))
+    neg = torch.rand(groups, d, generator=gen) < 0.1
+    f[neg] = -0.0005 * f[neg]
+    W = torch.randn(rows, d, generator=gen) * 0.02
+    summary, _, _ = lnq_follow_parity(orc, lnq, f.to(_dev()), W.to(_dev()), 8, 3, diag=True)
+    assert summary["moves"] > 0
+
+
 def test_lnq_diag_singular_rows(orc, lnq):
     # Row 0 (group 0): f = 0 on coordinates 0..3, which hold the row's only large values, so a
     # codeword used only there has no weight: the row keeps its codebook and reports
