@@ -242,8 +242,9 @@ LNQ_API lnq_status lnq_pack_codes(const uint8_t *Q, int64_t d_out, int64_t d_in,
  * quantised weights W^ = C[Q], read from the packed codes.
  *   x [nb][d_in] fp32, P packed as above, C [d_out][2^bits] fp32, y [nb][d_out] fp32 out; all
  *   device memory, caller-owned.
- * Arithmetic: fp32 products and sums (each lane sums its words in order, then a fixed-order warp
- * tree), so results are bit-identical from run to run.
+ * Arithmetic: fp32 products and sums in a fixed order (per row, each lane sums its words in order;
+ * the 32 lanes by a fixed shuffle butterfly; the 16 warps that split d_in in order), so results
+ * are bit-identical from run to run.
  * Requirements: bits in 1..4, 1 <= nb <= 8, d_out >= 1, d_in >= 1, non-NULL pointers; otherwise
  * LNQ_ERR_INVALID_ARG. */
 LNQ_API lnq_status lnq_lut_gemv(const float *x, int64_t nb, const uint32_t *P, const float *C,

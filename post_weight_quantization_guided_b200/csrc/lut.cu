@@ -13,20 +13,27 @@
 //
 // Kernels:
 //   pack_codes_kernel  one thread per output word: reads its codes, writes the word.
-//   lut_gemv_kernel    one warp per output row: the row's codebook in shared memory, lane l takes
-//                      words l, l + 32, ... (coalesced; 8 loads in flight per lane before any is
-//                      decoded), decodes each code once and multiplies it
-//                      with the NB (1..8, a template parameter) activation vectors (read through the read-only cache; they
-//                      are shared by every row), fp32 sums per lane, then a fixed-order warp tree.
-//                      Bound: HBM, the packed codes read once (d_out * words * 4 bytes).
+//   lut_gemv_kernel    K split over the 16 warps of a CTA: lane l of warp w takes the words
+//                      w * 32 + l + 512 s of every row, so one set of its activation values serves
+//                      every row. A CTA takes R rows at a time (R = 32 / NB, rounded down to a
+//                      power of two): their codebooks in shared memory, the R packed words of each
+//                      of its slices loaded before any is decoded (R loads in flight per lane),
+//                      each code decoded once and multiplied with the NB activation vectors, code
+//                      position by code position so that the R rows' sums are independent chains.
+//                      Per row a lane sums its words in order; the 32 lanes' sums of the R rows are
+//                      reduced by a transposing butterfly of shuffles (lane l ends with row
+//                      l / (32 / R)), and the 16 warps' sums are added in order.
+//                      Bound: HBM, the packed codes read once (d_out * words * 4 bytes); in
+//                      practice the issue rate (about 7 instructions per code: decode, address,
+//                      lookup, product, and the loop and reduction around them).
 #include "common.cuh"
 #include "lnq_internal.cuh"
 #include "profile.cuh"
 
 namespace lnq {
 
-constexpr int kLutWarps = 8;      // rows per CTA
-constexpr int kLutUnroll = 8;     // words a lane has in flight before decoding them
+constexpr int kLutWarps = 16;                  // K split: warps of a CTA
+constexpr int kLutThreads = kLutWarps * 32;
 
 __host__ __device__ inline int64_t lut_words(int64_t d_in, int bits)
 {
@@ -55,8 +62,29 @@ __global__ void __launch_bounds__(256)
     }
 }
 
-template <int BITS, int NB>
-__global__ void __launch_bounds__(kLutWarps * 32)
+// v[r] of every lane summed over the 32 lanes: a butterfly that halves the vector at each step,
+// so that lane l ends with the sum for row l / (32 / R). Fixed order, so bit-identical runs.
+template <int R>
+__device__ __forceinline__ float lut_transpose_sum(float (&v)[R], int lane)
+{
+#pragma unroll
+    for (int n = R / 2, o = 16; n >= 1; n >>= 1, o >>= 1) {
+        const bool upper = (lane & o) != 0;
+#pragma unroll
+        for (int c = 0; c < n; ++c) {
+            const float send = upper ? v[c] : v[c + n];
+            const float keep = upper ? v[c + n] : v[c];
+            v[c] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+        }
+    }
+#pragma unroll
+    for (int o = 16 / R; o >= 1; o >>= 1)
+        v[0] += __shfl_xor_sync(0xffffffffu, v[0], o);
+    return v[0];
+}
+
+template <int BITS, int NB, int R>
+__global__ void __launch_bounds__(kLutThreads, 1)
     lut_gemv_kernel(const float *__restrict__ x, const uint32_t *__restrict__ P,
                     const float *__restrict__ C, int64_t d_out, int64_t d_in,
                     float *__restrict__ y)
@@ -64,76 +92,66 @@ __global__ void __launch_bounds__(kLutWarps * 32)
     constexpr int PER = 32 / BITS;
     constexpr int M = 1 << BITS;
     constexpr uint32_t MASK = (1u << BITS) - 1u;
-    __shared__ float cs[kLutWarps][M];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    static_assert(R >= 1 && R <= 32 && (R & (R - 1)) == 0, "rows per block: a power of two");
+    __shared__ float cs[R][M];
+    __shared__ float part[NB][kLutWarps][R];
+    const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
     const int64_t words = lut_words(d_in, BITS);
-    const bool vec = (PER % 4 == 0) && (d_in % 4 == 0) && (reinterpret_cast<uintptr_t>(x) & 15u) == 0;
-    for (int64_t j = static_cast<int64_t>(blockIdx.x) * kLutWarps + warp; j < d_out;
-         j += static_cast<int64_t>(gridDim.x) * kLutWarps) {
-        if (lane < M)
-            cs[warp][lane] = C[j * M + lane];
-        __syncwarp();
-        float acc[NB];
+    const int64_t nslice = (words + kLutThreads - 1) / kLutThreads;
+    for (int64_t j0 = static_cast<int64_t>(blockIdx.x) * R; j0 < d_out;
+         j0 += static_cast<int64_t>(gridDim.x) * R) {
+        __syncthreads();   // the previous rows' codebooks and partial sums are read
+        for (int e = t; e < R * M; e += kLutThreads) {
+            const int64_t j = j0 + e / M;
+            cs[e / M][e % M] = j < d_out ? C[j * M + e % M] : 0.f;
+        }
+        __syncthreads();
+        float acc[NB][R];
 #pragma unroll
         for (int b = 0; b < NB; ++b)
-            acc[b] = 0.f;
-        const uint32_t *pj = P + j * words;
-        for (int64_t w0 = lane; w0 < words; w0 += 32 * kLutUnroll) {
-          // the lane's next kLutUnroll words, all loads issued before the first is used
-          uint32_t wd[kLutUnroll];
 #pragma unroll
-          for (int u = 0; u < kLutUnroll; ++u) {
-            const int64_t w = w0 + 32 * u;
-            wd[u] = w < words ? __ldg(pj + w) : 0u;
-          }
+            for (int r = 0; r < R; ++r)
+                acc[b][r] = 0.f;
+        for (int64_t s = 0; s < nslice; ++s) {
+            const int64_t w = s * kLutThreads + warp * 32 + lane;
+            const bool win = w < words;
+            uint32_t wd[R];
 #pragma unroll
-          for (int u = 0; u < kLutUnroll; ++u) {
-            const int64_t w = w0 + 32 * u;
-            if (w >= words)
-                continue;
-            const uint32_t word = wd[u];
-            const int64_t i0 = w * PER;
-            float wv[PER];
+            for (int r = 0; r < R; ++r)
+                wd[r] = (win && j0 + r < d_out) ? __ldg(P + (j0 + r) * words + w) : 0u;
 #pragma unroll
-            for (int t = 0; t < PER; ++t)
-                wv[t] = cs[warp][(word >> (t * BITS)) & MASK];
-            if (vec && i0 + PER <= d_in) {
+            for (int tt = 0; tt < PER; ++tt) {
+                const int64_t i = w * PER + tt;
+                float xv[NB];
 #pragma unroll
-                for (int b = 0; b < NB; ++b) {
-                    const float4 *xb = reinterpret_cast<const float4 *>(x + b * d_in + i0);
+                for (int b = 0; b < NB; ++b)
+                    xv[b] = (win && i < d_in) ? __ldg(x + b * d_in + i) : 0.f;
 #pragma unroll
-                    for (int t4 = 0; t4 < PER / 4; ++t4) {
-                        const float4 v = __ldg(xb + t4);
-                        acc[b] = fmaf(v.x, wv[4 * t4], acc[b]);
-                        acc[b] = fmaf(v.y, wv[4 * t4 + 1], acc[b]);
-                        acc[b] = fmaf(v.z, wv[4 * t4 + 2], acc[b]);
-                        acc[b] = fmaf(v.w, wv[4 * t4 + 3], acc[b]);
-                    }
-                }
-            } else {
+                for (int r = 0; r < R; ++r) {
+                    const float v = cs[r][(wd[r] >> (tt * BITS)) & MASK];
 #pragma unroll
-                for (int b = 0; b < NB; ++b) {
-#pragma unroll
-                    for (int t = 0; t < PER; ++t)
-                        if (i0 + t < d_in)
-                            acc[b] = fmaf(__ldg(x + b * d_in + i0 + t), wv[t], acc[b]);
+                    for (int b = 0; b < NB; ++b)
+                        acc[b][r] = fmaf(v, xv[b], acc[b][r]);
                 }
             }
-          }
         }
-        // fixed-order warp tree
 #pragma unroll
         for (int b = 0; b < NB; ++b) {
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1)
-                acc[b] += __shfl_xor_sync(0xffffffffu, acc[b], o);
+            const float sum = lut_transpose_sum<R>(acc[b], lane);
+            if ((lane & (32 / R - 1)) == 0)
+                part[b][warp][lane / (32 / R)] = sum;
         }
-        if (lane == 0) {
+        __syncthreads();
+        for (int e = t; e < NB * R; e += kLutThreads) {
+            const int b = e / R, r = e % R;
+            if (j0 + r < d_out) {
+                float sum = 0.f;
 #pragma unroll
-            for (int b = 0; b < NB; ++b)
-                y[b * d_out + j] = acc[b];
+                for (int w2 = 0; w2 < kLutWarps; ++w2)
+                    sum += part[b][w2][r];
+                y[b * d_out + j0 + r] = sum;
+            }
         }
-        __syncwarp();  // the row's codebook is read before the next row overwrites it
     }
 }
 
@@ -158,11 +176,13 @@ template <int BITS, int NB>
 static cudaError_t lut_gemv_nb(const float *x, const uint32_t *P, const float *C, int64_t d_out,
                                int64_t d_in, float *y, int num_sms, cudaStream_t s)
 {
-    int64_t blocks = (d_out + kLutWarps - 1) / kLutWarps;
-    if (blocks > static_cast<int64_t>(num_sms) * 16)
-        blocks = static_cast<int64_t>(num_sms) * 16;
+    // rows per block: 32 / NB rounded down to a power of two (NB * R <= 32 accumulators)
+    constexpr int R = NB == 1 ? 32 : (NB == 2 ? 16 : (NB <= 4 ? 8 : 4));
+    int64_t blocks = (d_out + R - 1) / R;
+    if (blocks > static_cast<int64_t>(num_sms))
+        blocks = static_cast<int64_t>(num_sms);
     KernelTimer timer("lnq_lut_gemv", s);
-    lut_gemv_kernel<BITS, NB><<<static_cast<unsigned>(blocks), kLutWarps * 32, 0, s>>>(
+    lut_gemv_kernel<BITS, NB, R><<<static_cast<unsigned>(blocks), kLutThreads, 0, s>>>(
         x, P, C, d_out, d_in, y);
     return cudaGetLastError();
 }

@@ -409,6 +409,33 @@ def test_lut_pack_and_gemv(orc, lnq, bits, d_out, d_in, nb):
     assert np.all(err <= 1e-5 * scale + 1e-30), float((err / (scale + 1e-30)).max())
 
 
+@pytest.mark.parametrize("case", ["many_row_blocks_and_slices", "unaligned_words"])
+def test_lut_gemv_large_and_unaligned(orc, lnq, case):
+    """Several row blocks per CTA and several K slices per lane (3000 x 16384), and packed words
+    that start off a 16-byte boundary."""
+    bits, nb = 4, 2
+    d_out, d_in = (3000, 16384) if case == "many_row_blocks_and_slices" else (300, 1000)
+    m = 1 << bits
+    g = torch.Generator().manual_seed(91 + d_in)
+    Q = torch.randint(0, m, (d_out, d_in), generator=g, dtype=torch.uint8)
+    C = torch.randn(d_out, m, generator=g)
+    x = torch.randn(nb, d_in, generator=g)
+    P = lnq.lnq_pack_codes(Q.to(_dev()), bits)
+    if case == "unaligned_words":
+        buf = torch.empty(P.numel() + 1, dtype=P.dtype, device=P.device)
+        buf[1:].copy_(P.reshape(-1))
+        P = buf[1:].view(P.shape)
+        assert P.data_ptr() % 16 != 0
+    y = lnq.lnq_lut_gemv(x.to(_dev()), P, C.to(_dev()), d_in)
+    torch.cuda.synchronize()
+    Qn, Cn, xn = Q.numpy(), C.double().numpy(), x.double().numpy()
+    yo = orc.lut_gemv(xn, Cn, Qn)
+    W_hat = np.take_along_axis(Cn, Qn.astype(np.int64), axis=1)
+    scale = np.abs(xn) @ np.abs(W_hat).T
+    err = np.abs(y.double().cpu().numpy() - yo)
+    assert np.all(err <= 1e-5 * scale + 1e-30), float((err / (scale + 1e-30)).max())
+
+
 def test_lut_gemv_on_a_quantised_layer(orc, lnq, wl):
     """The consumer on the tiny layer's own LNQ result (C, Q after three iterations)."""
     layer = wl.TINY
