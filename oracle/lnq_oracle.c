@@ -22,6 +22,11 @@
  *               (single-batch inference is memory-bound; weights stored as low-bit indices) and
  *               GANQ abstract (lookup-table based mixed-precision GEMM): the consumer of (C, Q)
  *               multiplies activations by W^ = C[Q] read through each row's codebook.
+ *   [GANQ]      scime.ai summary of GANQ (GPU-adaptive non-uniform quantization), Approach
+ *               paragraph: the same per-row problem, solved by alternating a Cholesky /
+ *               back-substitution assignment of the codebook indices with the closed-form
+ *               least-squares codebook update, batched on the GPU. Prior art, here only as a
+ *               comparison solver.
  *
  * READINGS (the pages leave these open; each routine below states the one it takes):
  *   R1 groups are contiguous, equal slices of output rows; s_g is the plain mean of squared
@@ -37,6 +42,14 @@
  *   R6 packed codes (the pages fix no format): bits = log2(m); each row is a run of 32-bit words
  *      holding floor(32 / bits) codes each, code i of the row in word i / floor(32 / bits) at bit
  *      (i mod floor(32 / bits)) * bits; unused high bits and the tail of the last word are zero.
+ *   R7 GANQ-style assignment: the Cholesky factor is lower, F = L L^T, so with r = c[q] - w the
+ *      objective is ||L^T r||^2 = sum_i z_i^2, z_i = sum_{k >= i} L[k][i] r_k. Back-substitution
+ *      visits i = d-1 down to 0 and gives coordinate i the codeword nearest to
+ *      t_i = w_i - (sum_{k > i} L[k][i] r_k) / L[i][i] (the smallest |z_i| given the later
+ *      coordinates; ties to the lower index). No damping or preconditioning. An iteration is the
+ *      codebook step (R5) followed by this assignment. A non-positive pivot of the factorisation
+ *      means the group is not positive definite: its rows keep their codes and report
+ *      ORC_ROW_NOT_PD.
  *
  * Build:  gcc -O2 -fopenmp -shared -fPIC lnq_oracle.c -o liblnq_oracle.so -lm
  */
@@ -50,6 +63,7 @@
 
 #define ORC_ROW_OK 0
 #define ORC_ROW_SINGULAR 1
+#define ORC_ROW_NOT_PD 2
 
 /* ------------------------------------------------------------------------------------------ */
 /* Fisher blocks [GQ-eq3], readings R1, R2                                                      */
@@ -392,6 +406,110 @@ void orc_follow_iteration(const double *F, int64_t d, const double *W, int64_t n
         status[j] = orc_codebook_row(F, d, w, m, q, c);
         orc_sweep_row(F, d, w, m, c, q, Q_hint + j * d, tie_rel, tie_abs ? tie_abs[j] : 0.0,
                       stats + 4 * j, NULL);
+        J_out[j] = orc_objective_row(F, d, w, c, q);
+    }
+}
+
+/* ------------------------------------------------------------------------------------------ */
+/* GANQ-style comparison solver [GANQ], reading R7                                              */
+/* ------------------------------------------------------------------------------------------ */
+
+/* Cholesky factor F = L L^T (Cholesky-Banachiewicz, row by row, FP64); L is d x d row-major,
+ * lower, zero above the diagonal. Returns 0, or 1 at the first non-positive pivot (L partial). */
+int orc_cholesky(const double *F, int64_t d, double *L)
+{
+    for (int64_t i = 0; i < d * d; ++i)
+        L[i] = 0.0;
+    for (int64_t i = 0; i < d; ++i) {
+        for (int64_t j = 0; j <= i; ++j) {
+            double sum = F[i * d + j];
+            for (int64_t k = 0; k < j; ++k)
+                sum -= L[i * d + k] * L[j * d + k];
+            if (i == j) {
+                if (!(sum > 0.0))
+                    return 1;
+                L[i * d + i] = sqrt(sum);
+            } else {
+                L[i * d + j] = sum / L[j * d + j];
+            }
+        }
+    }
+    return 0;
+}
+
+/* Back-substitution assignment of one row (R7): i = d-1 down to 0, coordinate i takes the codeword
+ * nearest to t_i = w_i - (sum_{k > i} L[k][i] r_k) / L[i][i], with r_k = c[q_k] - w_k of the
+ * coordinates already visited; the cost of candidate a is L[i][i]^2 (c_a - t_i)^2 = z_i^2.
+ * Follow mode (hint != NULL): where the hint differs and its cost is within `band` of the best
+ * cost, the hint is taken (a tie-follow); otherwise this choice stays (a mismatch).
+ * stats (may be NULL): [0] codes changed from the input, [1] tie-follows, [2] mismatches. */
+void orc_ganq_assign_row(const double *L, int64_t d, const double *w, int m, const double *c,
+                         uint8_t *q, const uint8_t *hint, double band, int64_t *stats)
+{
+    double *r = (double *)calloc((size_t)d, sizeof(double));
+    int64_t changed = 0, follows = 0, mismatches = 0;
+    for (int64_t i = d - 1; i >= 0; --i) {
+        double s = 0.0;
+        for (int64_t k = i + 1; k < d; ++k)
+            s += L[k * d + i] * r[k];
+        const double lii = L[i * d + i];
+        const double t = w[i] - s / lii;
+        int best = 0;
+        double bcost = lii * lii * (c[0] - t) * (c[0] - t);
+        for (int a = 1; a < m; ++a) {
+            const double cost = lii * lii * (c[a] - t) * (c[a] - t);
+            if (cost < bcost) {
+                bcost = cost;
+                best = a;
+            }
+        }
+        if (hint != NULL && hint[i] != best) {
+            const double hc = lii * lii * (c[hint[i]] - t) * (c[hint[i]] - t);
+            if (hc - bcost <= band) {
+                best = hint[i];
+                follows += 1;
+            } else {
+                mismatches += 1;
+            }
+        }
+        if (best != q[i])
+            changed += 1;
+        q[i] = (uint8_t)best;
+        r[i] = c[best] - w[i];
+    }
+    if (stats) {
+        stats[0] = changed;
+        stats[1] = follows;
+        stats[2] = mismatches;
+    }
+    free(r);
+}
+
+/* One GANQ-style iteration for `nrows` rows sharing F (and its factor L, from orc_cholesky):
+ * the codebook step (R5) from (C_start, Q_start), then the back-substitution assignment (R7),
+ * following Q_hint inside the band (Q_hint may be NULL). band (nrows, may be NULL): per-row
+ * absolute tie band. Out: C_out, Q_out, J_out (objective from its definition), stats (nrows x 3),
+ * status (nrows: codebook status). */
+void orc_ganq_iteration(const double *F, const double *L, int64_t d, const double *W,
+                        int64_t nrows, int m, const double *C_start, const uint8_t *Q_start,
+                        const uint8_t *Q_hint, const double *band, double *C_out,
+                        uint8_t *Q_out, double *J_out, int64_t *stats, int32_t *status,
+                        int nthreads)
+{
+#ifdef _OPENMP
+    if (nthreads > 0)
+        omp_set_num_threads(nthreads);
+#pragma omp parallel for schedule(dynamic, 1)
+#endif
+    for (int64_t j = 0; j < nrows; ++j) {
+        const double *w = W + j * d;
+        double *c = C_out + j * m;
+        uint8_t *q = Q_out + j * d;
+        memcpy(c, C_start + j * m, (size_t)m * sizeof(double));
+        memcpy(q, Q_start + j * d, (size_t)d);
+        status[j] = orc_codebook_row(F, d, w, m, q, c);
+        orc_ganq_assign_row(L, d, w, m, c, q, Q_hint ? Q_hint + j * d : NULL,
+                            band ? band[j] : 0.0, stats ? stats + 3 * j : NULL);
         J_out[j] = orc_objective_row(F, d, w, c, q);
     }
 }

@@ -55,6 +55,12 @@ def _bind(path: str):
     lib.orc_sweep_row.restype = ctypes.c_double
     lib.orc_lnq_rows.argtypes = [_DP, _I64, _DP, _I64, ctypes.c_int, ctypes.c_int,
                                  ctypes.c_int, _DP, _U8P, _DP, _I32P, ctypes.c_int]
+    lib.orc_cholesky.argtypes = [_DP, _I64, _DP]
+    lib.orc_cholesky.restype = ctypes.c_int
+    lib.orc_ganq_assign_row.argtypes = [_DP, _I64, _DP, ctypes.c_int, _DP, _U8P, _U8P,
+                                        ctypes.c_double, _I64P]
+    lib.orc_ganq_iteration.argtypes = [_DP, _DP, _I64, _DP, _I64, ctypes.c_int, _DP, _U8P, _U8P,
+                                       _DP, _DP, _U8P, _DP, _I64P, _I32P, ctypes.c_int]
     lib.orc_follow_iteration.argtypes = [_DP, _I64, _DP, _I64, ctypes.c_int, _DP, _U8P,
                                          _U8P, ctypes.c_double, _DP, _DP, _U8P, _DP, _I64P,
                                          _I32P, ctypes.c_int]
@@ -240,6 +246,47 @@ def follow_iteration(F, W, m: int, C_start, Q_start, Q_hint, tie_rel: float,
 
 
 _U32P = ctypes.POINTER(ctypes.c_uint32)
+
+
+def cholesky(F):
+    """(L, ok): the lower Cholesky factor F = L L^T in FP64; ok is False at a non-positive
+    pivot (reading R7)."""
+    F = _f64(F)
+    d = F.shape[0]
+    L = np.zeros((d, d), dtype=np.float64)
+    bad = _load().orc_cholesky(_p(F, _DP), d, _p(L, _DP))
+    return L, bad == 0
+
+
+def ganq_assign_row(L, w, c, q, hint=None, band: float = 0.0):
+    """The back-substitution assignment of one row (reading R7); returns (q, stats) with stats
+    [changed, tie-follows, mismatches]."""
+    L, w, c = _f64(L), _f64(w), _f64(c)
+    q = _u8(q).copy()
+    stats = np.zeros(3, dtype=np.int64)
+    hp = None if hint is None else _p(_u8(hint), _U8P)
+    _load().orc_ganq_assign_row(_p(L, _DP), L.shape[0], _p(w, _DP), c.shape[0], _p(c, _DP),
+                                _p(q, _U8P), hp, float(band), _p(stats, _I64P))
+    return q, stats
+
+
+def ganq_iteration(F, L, W, m: int, C_start, Q_start, Q_hint=None, band=None, nthreads: int = 0):
+    """One GANQ-style iteration (codebook step, then back-substitution assignment) for rows
+    sharing F; returns (C, Q, J, stats [rows x 3], status)."""
+    F, L, W = _f64(F), _f64(L), _f64(W)
+    nrows, d = W.shape
+    C = np.empty((nrows, m), dtype=np.float64)
+    Q = np.empty((nrows, d), dtype=np.uint8)
+    J = np.empty(nrows, dtype=np.float64)
+    stats = np.zeros((nrows, 3), dtype=np.int64)
+    status = np.zeros(nrows, dtype=np.int32)
+    hp = None if Q_hint is None else _p(_u8(Q_hint), _U8P)
+    bp = None if band is None else _p(_f64(band), _DP)
+    _load().orc_ganq_iteration(_p(F, _DP), _p(L, _DP), d, _p(W, _DP), nrows, m,
+                               _p(_f64(C_start), _DP), _p(_u8(Q_start), _U8P), hp, bp,
+                               _p(C, _DP), _p(Q, _U8P), _p(J, _DP), _p(stats, _I64P),
+                               _p(status, _I32P), nthreads)
+    return C, Q, J, stats, status
 
 
 def packed_words(d_in: int, bits: int) -> int:
