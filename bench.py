@@ -819,7 +819,41 @@ def run_q_proj(args, rank, device, fp32_peak, steps=5, warmup=3):
                 "rows_per_s": dout / (diag_ms / 1e3), "algorithmic_bytes": diag_bytes,
                 "achieved_gbs": diag_bytes / (diag_ms * 1e-3) / 1e9,
                 "frac_hbm": diag_bytes / (diag_ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}
-    return res, res_lut, res_diag
+
+    # A/B: the GANQ-style solver (Cholesky / back-substitution assignment, the same codebook
+    # step) against LNQ on the same F, W and initial codebooks, the same number of iterations
+    ws_g = b.workspace(b.LNQ_OP_GANQ_ROWS, 0, d, dout, layer.groups, m, device)
+    Cg, Qg = C0d.clone(), Q0d.clone()
+    Jg = torch.empty(dout, dtype=torch.float64, device=device)
+    lnq.lnq_ganq_rows(F, W, m, it, Cg, Qg, Jg, ws=ws_g)       # warm-up
+    torch.cuda.synchronize(device)
+    reps, ganq_ms = 3, 0.0
+    b.lnq_profile_read()
+    b.lnq_profile_enable(True)
+    for _ in range(reps):
+        Cg.copy_(C0d)
+        Qg.copy_(Q0d)
+        flush.fill_(0x3C)
+        g0.record(stream)
+        lnq.lnq_ganq_rows(F, W, m, it, Cg, Qg, Jg, ws=ws_g)
+        g1.record(stream)
+        torch.cuda.synchronize(device)
+        ganq_ms += g0.elapsed_time(g1) / reps
+    b.lnq_profile_enable(False)
+    gprof = b.lnq_profile_read()
+    Cl, Ql = C0d.clone(), Q0d.clone()
+    Jl = torch.empty(dout, dtype=torch.float64, device=device)
+    lnq.lnq_quantize_rows(F, W, m, it, Cl, Ql, Jl, ws=ws_q)
+    torch.cuda.synchronize(device)
+    del ws_g
+    res_ganq = {"workload": f"{layer.name}: {it} iterations, m = {m}, from the same initial "
+                            "codebooks as LNQ",
+                "ms_per_call": ganq_ms, "rows_per_s": dout / (ganq_ms / 1e3),
+                "kernels_ms_per_call": {k: v[1] / reps for k, v in gprof.items()},
+                "sum_J": float(Jg.sum()), "lnq_sum_J": float(Jl.sum()),
+                "J_ratio_vs_lnq": float(Jg.sum()) / float(Jl.sum()),
+                "rows_lower_than_lnq": int((Jg < Jl).sum())}
+    return res, res_lut, res_diag, res_ganq
 
 
 # ------------------------------------------------------------------------------------------
@@ -914,7 +948,7 @@ def main():
             torch.cuda.empty_cache()
             qp = run_q_proj(args, rank, device, fp32_peak)
             if line is not None:
-                line["q_proj"], line["lut_gemv"], line["lnq_diag"] = qp
+                line["q_proj"], line["lut_gemv"], line["lnq_diag"], line["ganq_ab"] = qp
     finally:
         if world > 1:
             torch.distributed.destroy_process_group()

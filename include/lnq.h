@@ -80,14 +80,15 @@ typedef enum {
 } lnq_status;
 
 /* Per-row outcome written to row_status by lnq_quantize_rows. */
-enum { LNQ_ROW_OK = 0, LNQ_ROW_SINGULAR = 1 };
+enum { LNQ_ROW_OK = 0, LNQ_ROW_SINGULAR = 1, LNQ_ROW_NOT_PD = 2 };
 
 /* Operation selector for lnq_workspace_size. */
 typedef enum {
     LNQ_OP_BUILD_FISHER = 0,
     LNQ_OP_INIT_CODEBOOK = 1,
     LNQ_OP_QUANTIZE_ROWS = 2,
-    LNQ_OP_OBJECTIVE = 3
+    LNQ_OP_OBJECTIVE = 3,
+    LNQ_OP_GANQ_ROWS = 4
 } lnq_op;
 
 /* Bytes of device workspace the operation needs for these sizes (0 if the sizes are invalid).
@@ -187,6 +188,28 @@ LNQ_API lnq_status lnq_quantize_rows_diag(const float *Fd, int groups, const flo
                                           int64_t d_out, int64_t d_in, int m, int iters, float *C,
                                           uint8_t *Q, double *J_out, int32_t *row_status,
                                           lnq_stream_t stream);
+
+/* A GANQ-style comparison solver on the same per-row problem: `iters` iterations of the
+ * codebook step of lnq_quantize_rows followed by a Cholesky / back-substitution assignment.
+ * scime.ai summary of GANQ (GPU-adaptive non-uniform quantization), Approach paragraph
+ * (alternating Cholesky / back-substitution index assignment and closed-form least-squares
+ * codebook, batched on the GPU). Reading: F_g = L L^T with L lower (factorised once per call in
+ * fp64); with r = C[j][Q[j]] - W[j], coordinates are visited from the last to the first and each
+ * takes the codeword nearest to t_i = w_i - (sum_{k > i} L[k][i] r_k) / L[i][i]; no damping.
+ *   F, W, C, Q, J_out  as lnq_quantize_rows (C, Q in/out; codes are read modulo m)
+ *   row_status  [d_out] int32 out, or NULL: LNQ_ROW_SINGULAR as lnq_quantize_rows; LNQ_ROW_NOT_PD
+ *               for rows of a group whose factorisation met a non-positive pivot (their codes are
+ *               kept; the codebook step still runs)
+ *   ws          lnq_workspace_size(LNQ_OP_GANQ_ROWS, 0, d_in, d_out, groups, m) bytes, 256-byte
+ *               aligned (the QUANTIZE_ROWS workspace plus an fp64 and an fp32 copy of every F_g
+ *               and a residual per weight).
+ * Arithmetic: factorisation in fp64; the back-substituted sums in fp32 from the fp32 factor, in a
+ * fixed order, so results are bit-identical from run to run.
+ * Requirements and errors as lnq_quantize_rows. */
+LNQ_API lnq_status lnq_ganq_rows(const float *F, int groups, const float *W, int64_t d_out,
+                                 int64_t d_in, int m, int iters, float *C, uint8_t *Q,
+                                 double *J_out, int32_t *row_status, void *ws, size_t ws_bytes,
+                                 lnq_stream_t stream);
 
 /* Per-row objective J[j] = r^T F_g r with r = C[j][Q[j]] - W[j] ("GuidedQuant" blog, GuidedQuant
  * section, third equation: the guided output error of row j is n r^T F_j r; LNQ section, first

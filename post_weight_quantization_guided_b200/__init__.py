@@ -6,4 +6,4 @@ from .binding import (LNQ_OP_BUILD_FISHER, LNQ_OP_INIT_CODEBOOK, LNQ_OP_OBJECTIV
                       lnq_workspace_check, lnq_workspace_size, lnq_packed_words,
                       lnq_pack_codes, lnq_lut_gemv, lnq_quantize_rows_diag,
                       lnq_sweep_counters, lnq_fp32_probe, lnq_build_fisher_noalloc,
-                      lnq_noalloc_check)
+                      lnq_noalloc_check, lnq_ganq_rows, LNQ_OP_GANQ_ROWS, LNQ_ROW_NOT_PD)

@@ -17,14 +17,15 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "liblnq.so")
 # Status codes and selectors (include/lnq.h).
 LNQ_OK, LNQ_ERR_INVALID_ARG, LNQ_ERR_CUDA, LNQ_ERR_WORKSPACE, LNQ_ERR_UNSUPPORTED, \
     LNQ_ERR_TIMEOUT = range(6)
-LNQ_ROW_OK, LNQ_ROW_SINGULAR = 0, 1
-LNQ_OP_BUILD_FISHER, LNQ_OP_INIT_CODEBOOK, LNQ_OP_QUANTIZE_ROWS, LNQ_OP_OBJECTIVE = range(4)
+LNQ_ROW_OK, LNQ_ROW_SINGULAR, LNQ_ROW_NOT_PD = 0, 1, 2
+(LNQ_OP_BUILD_FISHER, LNQ_OP_INIT_CODEBOOK, LNQ_OP_QUANTIZE_ROWS, LNQ_OP_OBJECTIVE,
+ LNQ_OP_GANQ_ROWS) = range(5)
 
 EXPORTED = ("lnq_workspace_size", "lnq_build_fisher", "lnq_init_codebook", "lnq_quantize_rows",
             "lnq_objective", "lnq_workspace_check", "lnq_set_wait_limit", "lnq_status_string",
             "lnq_profile_enable", "lnq_profile_read", "lnq_build_fisher_noalloc",
             "lnq_packed_words", "lnq_pack_codes", "lnq_lut_gemv", "lnq_quantize_rows_diag",
-            "lnq_sweep_counters", "lnq_fp32_probe")
+            "lnq_sweep_counters", "lnq_fp32_probe", "lnq_ganq_rows")
 
 _lib = None
 _VP, _I64, _INT, _SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
@@ -52,6 +53,7 @@ def lib():
         L.lnq_init_codebook.argtypes = [_VP, _I64, _I64, _INT, _VP, _VP, _VP, _SZ, _VP]
         L.lnq_quantize_rows.argtypes = [_VP, _INT, _VP, _I64, _I64, _INT, _INT, _VP, _VP, _VP,
                                         _VP, _VP, _SZ, _VP]
+        L.lnq_ganq_rows.argtypes = L.lnq_quantize_rows.argtypes
         L.lnq_objective.argtypes = [_VP, _INT, _VP, _VP, _VP, _I64, _I64, _INT, _VP, _VP, _SZ,
                                     _VP]
         L.lnq_workspace_check.argtypes = [_VP, _VP]
@@ -76,7 +78,7 @@ def lib():
         for name in ("lnq_build_fisher", "lnq_build_fisher_noalloc", "lnq_init_codebook",
                      "lnq_quantize_rows", "lnq_objective", "lnq_workspace_check",
                      "lnq_pack_codes", "lnq_lut_gemv", "lnq_quantize_rows_diag",
-                     "lnq_sweep_counters", "lnq_fp32_probe"):
+                     "lnq_sweep_counters", "lnq_fp32_probe", "lnq_ganq_rows"):
             getattr(L, name).restype = _INT
         _lib = L
     return _lib
@@ -215,6 +217,30 @@ def lnq_quantize_rows(F: torch.Tensor, W: torch.Tensor, m: int, iters: int, C: t
     _check(lib().lnq_quantize_rows(_ptr(F), groups, _ptr(W), d_out, d_in, m, iters, _ptr(C),
                                    _ptr(Q), _ptr(J_out), _ptr(row_status), _ptr(ws), ws.numel(),
                                    _stream(stream)), "lnq_quantize_rows")
+    return C, Q, J_out, row_status
+
+
+def lnq_ganq_rows(F: torch.Tensor, W: torch.Tensor, m: int, iters: int, C: torch.Tensor,
+                  Q: torch.Tensor, J_out: Optional[torch.Tensor] = None,
+                  row_status: Optional[torch.Tensor] = None,
+                  ws: Optional[torch.Tensor] = None, stream=None):
+    """`iters` GANQ-style iterations (codebook step, Cholesky / back-substitution assignment) in
+    place on (C, Q); returns (C, Q, J_out, row_status)."""
+    groups, d_in, _ = F.shape
+    d_out = W.shape[0]
+    _need(F, torch.float32, (groups, d_in, d_in), "F")
+    _need(W, torch.float32, (d_out, d_in), "W")
+    _need(C, torch.float32, (d_out, m), "C")
+    _need(Q, torch.uint8, (d_out, d_in), "Q")
+    if J_out is not None:
+        _need(J_out, torch.float64, (d_out,), "J_out")
+    if row_status is not None:
+        _need(row_status, torch.int32, (d_out,), "row_status")
+    if ws is None:
+        ws = workspace(LNQ_OP_GANQ_ROWS, 0, d_in, d_out, groups, m, device=W.device)
+    _check(lib().lnq_ganq_rows(_ptr(F), groups, _ptr(W), d_out, d_in, m, iters, _ptr(C),
+                               _ptr(Q), _ptr(J_out), _ptr(row_status), _ptr(ws), ws.numel(),
+                               _stream(stream)), "lnq_ganq_rows")
     return C, Q, J_out, row_status
 
 

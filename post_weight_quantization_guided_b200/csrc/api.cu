@@ -46,6 +46,9 @@ static bool valid_m(int m) { return m == 2 || m == 4 || m == 8 || m == 16; }
 //                   | sweep history [CTAs][2 ceil(d_in / 128)][2][4 KB] (Delta pieces)
 //                   | right-operand image of the products [row tiles][K blocks][256][64] 16-bit
 //   OBJECTIVE:      the same layout (status, Sb and U unused)
+//   GANQ_ROWS:      the QUANTIZE_ROWS layout, then A [groups][d_in][d_in] f64 (the factorisation)
+//                   | L [groups][d_in][d_in] f32 | 1 / L_ii [groups][d_in] f32
+//                   | R [d_out][d_in] f32 (residuals) | factor status [groups] i32
 //   INIT:           header
 struct FisherWs {
     size_t s_off, m_off, pi_off, total;
@@ -137,6 +140,10 @@ size_t lnq_workspace_size(lnq_op op, int64_t n, int64_t d_in, int64_t d_out, int
         return lnq_ws(d_in, d_out, groups, m).total;
     case LNQ_OP_INIT_CODEBOOK:
         return kWsHeader;
+    case LNQ_OP_GANQ_ROWS:
+        if (d_out < 1 || d_in < 1 || groups < 1 || !valid_m(m))
+            return 0;
+        return lnq_ws(d_in, d_out, groups, m).total + lnq_ganq_extra_bytes(d_in, d_out, groups);
     }
     return 0;
 }
@@ -234,6 +241,34 @@ lnq_status lnq_quantize_rows(const float *F, int groups, const float *W, int64_t
         return LNQ_ERR_CUDA;
     if (lnq_iterate_launch(F, groups, W, d_out, d_in, m, iters, C, Q, J_out, w, err,
                            device_sm_count(), s) != cudaSuccess)
+        return LNQ_ERR_CUDA;
+    if (row_status != nullptr &&
+        cudaMemcpyAsync(row_status, w.status, static_cast<size_t>(d_out) * sizeof(int32_t),
+                        cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+        return LNQ_ERR_CUDA;
+    return LNQ_OK;
+}
+
+lnq_status lnq_ganq_rows(const float *F, int groups, const float *W, int64_t d_out, int64_t d_in,
+                         int m, int iters, float *C, uint8_t *Q, double *J_out,
+                         int32_t *row_status, void *ws, size_t ws_bytes, lnq_stream_t stream)
+{
+    if (F == nullptr || W == nullptr || C == nullptr || Q == nullptr || groups < 1 ||
+        d_out < 1 || d_out % groups != 0 || d_in < 1 || d_in > 16384 || !valid_m(m) ||
+        iters < 0 || d_out > (int64_t(1) << 31) - 1)
+        return LNQ_ERR_INVALID_ARG;
+    const LnqWs lay = lnq_ws(d_in, d_out, groups, m);
+    lnq_status st = check_ws(ws, ws_bytes, lay.total + lnq_ganq_extra_bytes(d_in, d_out, groups));
+    if (st != LNQ_OK)
+        return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const LnqWorkspace w = carve(ws, lay);
+    DeviceErr err{reinterpret_cast<uint32_t *>(ws), g_wait_limit.load()};
+    if (cudaMemsetAsync(ws, 0, lay.fh_off, s) != cudaSuccess)   // header and row status
+        return LNQ_ERR_CUDA;
+    if (lnq_ganq_launch(F, groups, W, d_out, d_in, m, iters, C, Q, J_out, w,
+                        static_cast<uint8_t *>(ws) + lay.total, err, device_sm_count(), s) !=
+        cudaSuccess)
         return LNQ_ERR_CUDA;
     if (row_status != nullptr &&
         cudaMemcpyAsync(row_status, w.status, static_cast<size_t>(d_out) * sizeof(int32_t),

@@ -72,6 +72,13 @@ cudaError_t lnq_lut_gemv_launch(const float *x, int nb, const uint32_t *P, const
                                 int64_t d_out, int64_t d_in, int bits, float *y, int num_sms,
                                 cudaStream_t s);
 
+// ganq.cu
+size_t lnq_ganq_extra_bytes(int64_t d, int64_t d_out, int groups);
+cudaError_t lnq_ganq_launch(const float *F, int groups, const float *W, int64_t d_out, int64_t d,
+                            int m, int iters, float *C, uint8_t *Q, double *J,
+                            const LnqWorkspace &w, void *extra, DeviceErr err, int num_sms,
+                            cudaStream_t s);
+
 // lnq_diag.cu
 cudaError_t lnq_diag_launch(const float *Fd, int groups, const float *W, int64_t d_out, int64_t d,
                             int m, int iters, float *C, uint8_t *Q, double *J, int32_t *status,

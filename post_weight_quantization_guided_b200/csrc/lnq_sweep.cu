@@ -109,6 +109,72 @@ __device__ __forceinline__ unsigned bit_position_sum(unsigned m)
            8u * __popc(m & 0xFF00FF00u) + 16u * __popc(m & 0xFFFF0000u);
 }
 
+// The decisions of one block for one row (lane = row). With F_ii > 0, candidate a changes the
+// objective by F_ii ((c_a - t)^2 - (cur - t)^2), t = cur - u_i / F_ii, so the best candidate is
+// the codeword nearest to t: a binary search of the sorted codebook's midpoints, held in
+// registers, halving the candidate values and midpoints at each level (selects only, no loads on
+// the chain). Its change delta (2 u_i + delta F_ii) is then evaluated and the coordinate moves only
+// if that is strictly negative. (F_ii = 0 gives t = -+inf, the extreme codeword, which is the best
+// one for a linear change.) The later coordinates of the block are corrected in registers from
+// the block's rows of the F strip. The shared-memory views are restrict-qualified, so that the
+// loads of later coordinates may be issued ahead of the stores of earlier ones.
+template <int M>
+__device__ __forceinline__ unsigned sweep_decide_block(
+    float (&ub)[sw::BLK], uint32_t (&qw)[sw::BLK / 4], const uint32_t (&qo)[sw::BLK / 4],
+    const float *__restrict__ crow, const uint8_t *__restrict__ ordrow,
+    const float *__restrict__ finv, const float *__restrict__ fdg, const float *__restrict__ st,
+    float *__restrict__ dlcol, const float (&mid)[M > 1 ? M - 1 : 1], const float (&sv)[M],
+    bool vr, int nb)
+{
+    using namespace sw;
+    unsigned rowmask = 0u;
+#pragma unroll
+    for (int ii = 0; ii < BLK; ++ii) {
+        const float u = ub[ii];
+        const float cur = crow[(qo[ii >> 2] >> (8 * (ii & 3))) & 0xFFu];
+        const float tt = fmaf(-u, finv[ii], cur);
+        float V[M], Mi[M];
+#pragma unroll
+        for (int k = 0; k < M; ++k) {
+            V[k] = sv[k];
+            Mi[k] = k + 1 < M ? mid[k + 1 < M ? k : 0] : 0.f;
+        }
+        int pos = 0;
+#pragma unroll
+        for (int S = M; S > 1; S >>= 1) {
+            const int h = S / 2;
+            const bool up = tt > Mi[h - 1];
+#pragma unroll
+            for (int k = 0; k < h; ++k)
+                V[k] = up ? V[k + h] : V[k];
+#pragma unroll
+            for (int k = 0; k + 1 < h; ++k)
+                Mi[k] = up ? Mi[k + h] : Mi[k];
+            pos += up ? h : 0;
+        }
+        const float da = V[0] - cur;
+        const float D = da * fmaf(da, fdg[ii], 2.f * u);
+        // a strictly negative change implies c != cur
+        const bool mv = vr && ii < nb && D < 0.f;
+        const float dlt = mv ? da : 0.f;
+        rowmask |= (mv ? 1u : 0u) << ii;
+        const int sh = 8 * (ii & 3);
+        const uint32_t nq =
+            (qw[ii >> 2] & ~(0xFFu << sh)) | (static_cast<uint32_t>(ordrow[pos]) << sh);
+        qw[ii >> 2] = mv ? nq : qw[ii >> 2];
+#pragma unroll
+        for (int v = (ii + 1) / 4; v < BLK / 4; ++v) {
+            const float4 f4 = *reinterpret_cast<const float4 *>(st + ii * WIN + 4 * v);
+            if (4 * v > ii) ub[4 * v] = fmaf(dlt, f4.x, ub[4 * v]);
+            if (4 * v + 1 > ii) ub[4 * v + 1] = fmaf(dlt, f4.y, ub[4 * v + 1]);
+            if (4 * v + 2 > ii) ub[4 * v + 2] = fmaf(dlt, f4.z, ub[4 * v + 2]);
+            if (4 * v + 3 > ii) ub[4 * v + 3] = fmaf(dlt, f4.w, ub[4 * v + 3]);
+        }
+        dlcol[ii * RB] = dlt;
+    }
+    return rowmask;
+}
+
 template <int M>
 __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
     sweep_kernel(const __grid_constant__ CUtensorMap fmap, const __grid_constant__ CUtensorMap smap,
@@ -577,6 +643,7 @@ __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
         // warp 6 (lane = row): the row's codebook sorted, equal values in index order, and the
         // midpoints between neighbours, for the decisions of the whole sweep
         float mid[M > 1 ? M - 1 : 1];
+        float sv[M];   // the sorted codebook
         if (warp == 6) {
             const int r = lane;
             for (int a = 0; a < M; ++a) {
@@ -593,6 +660,9 @@ __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
 #pragma unroll
             for (int k = 0; k + 1 < M; ++k)
                 mid[k] = 0.5f * (srt_s[r][k] + srt_s[r][k + 1]);
+#pragma unroll
+            for (int k = 0; k < M; ++k)
+                sv[k] = srt_s[r][k];
         }
         fetch_codes(0, 0, t, SWEEP_THREADS);
         load_strip(0, 0, 0, t, SWEEP_THREADS);
@@ -696,46 +766,9 @@ __global__ void __launch_bounds__(sw::NUM_THREADS, 1)
 #pragma unroll
                     for (int ii = 0; ii < BLK; ++ii)
                         ub[ii] = uw[r * UW_LD + lb * BLK + ii];
-                    unsigned rowmask = 0u;
-#pragma unroll
-                    for (int ii = 0; ii < BLK; ++ii) {
-                        const float u = ub[ii];
-                        const float cur = c_s[r][(qo[ii >> 2] >> (8 * (ii & 3))) & 0xFFu];
-                        const float tt = fmaf(-u, finv_s[ii], cur);
-                        // number of midpoints below t, summed as a balanced tree of floats (exact
-                        // small integers; floating-point adds keep the tree's order, so the count is
-                        // four additions deep)
-                        float cnt[M];
-#pragma unroll
-                        for (int k = 0; k < M; ++k)
-                            cnt[k] = (k + 1 < M && tt > mid[k < M - 1 ? k : 0]) ? 1.f : 0.f;
-#pragma unroll
-                        for (int w2 = 1; w2 < M; w2 *= 2) {
-#pragma unroll
-                            for (int k = 0; k + w2 < M; k += 2 * w2)
-                                cnt[k] += cnt[k + w2];
-                        }
-                        const int pos = static_cast<int>(cnt[0]);
-                        const float da = srt_s[r][pos] - cur;
-                        const float D = da * fmaf(da, fdg_s[ii], 2.f * u);
-                        // a strictly negative change implies c != cur
-                        const bool mv = vr && ii < nb && D < 0.f;
-                        const float dlt = mv ? da : 0.f;
-                        rowmask |= (mv ? 1u : 0u) << ii;
-                        const int sh = 8 * (ii & 3);
-                        const uint32_t nq = (qw[ii >> 2] & ~(0xFFu << sh)) |
-                                            (static_cast<uint32_t>(ord_s[r][pos]) << sh);
-                        qw[ii >> 2] = mv ? nq : qw[ii >> 2];
-#pragma unroll
-                        for (int v = (ii + 1) / 4; v < BLK / 4; ++v) {
-                            const float4 f4 = *reinterpret_cast<const float4 *>(st + ii * WIN + 4 * v);
-                            if (4 * v > ii) ub[4 * v] = fmaf(dlt, f4.x, ub[4 * v]);
-                            if (4 * v + 1 > ii) ub[4 * v + 1] = fmaf(dlt, f4.y, ub[4 * v + 1]);
-                            if (4 * v + 2 > ii) ub[4 * v + 2] = fmaf(dlt, f4.z, ub[4 * v + 2]);
-                            if (4 * v + 3 > ii) ub[4 * v + 3] = fmaf(dlt, f4.w, ub[4 * v + 3]);
-                        }
-                        dl2[cb][ii][r] = dlt;
-                    }
+                    const unsigned rowmask = sweep_decide_block<M>(
+                        ub, qw, qo, c_s[r], ord_s[r], finv_s, fdg_s, st, &dl2[cb][0][r], mid, sv,
+                        vr, nb);
 #pragma unroll
                     for (int v = 0; v < BLK / 4; ++v)
                         *reinterpret_cast<uint32_t *>(&qb_s[r][4 * v]) = qw[v];

@@ -31,7 +31,7 @@ def test_header_declares_the_entry_points():
                             "lnq_workspace_check", "lnq_workspace_size", "lnq_profile_enable",
                             "lnq_profile_read", "lnq_build_fisher_noalloc", "lnq_packed_words",
                             "lnq_pack_codes", "lnq_lut_gemv", "lnq_quantize_rows_diag",
-                            "lnq_sweep_counters", "lnq_fp32_probe"])
+                            "lnq_sweep_counters", "lnq_fp32_probe", "lnq_ganq_rows"])
 
 
 def test_packed_words_and_argument_checks(L):
@@ -67,6 +67,12 @@ def test_workspace_sizes(L):
     assert b.lnq_workspace_size(b.LNQ_OP_QUANTIZE_ROWS, 0, d, dout, g, 16) >= 256 + dout * 4
     assert b.lnq_workspace_size(b.LNQ_OP_INIT_CODEBOOK, 0, d, dout, 1, 16) == 256
     assert b.lnq_workspace_size(b.LNQ_OP_BUILD_FISHER, 0, d, dout, g, 16) == 0
+    # the GANQ-style solver: the QUANTIZE_ROWS workspace plus an fp64 and an fp32 factor per group,
+    # the reciprocal pivots, a residual per weight and the factor statuses
+    q = b.lnq_workspace_size(b.LNQ_OP_QUANTIZE_ROWS, 0, d, dout, g, 16)
+    extra = g * d * d * 12 + g * d * 4 + dout * d * 4 + g * 4
+    sz = b.lnq_workspace_size(b.LNQ_OP_GANQ_ROWS, 0, d, dout, g, 16)
+    assert q + extra <= sz <= q + extra + 5 * 256
 
 
 def _fisher(L, **kw):
@@ -118,6 +124,24 @@ def test_quantize_rows_diag_rejects_bad_arguments(L, kw):
     a.update(kw)
     assert L.lnq_quantize_rows_diag(a["F"], a["groups"], a["W"], a["d_out"], a["d_in"], a["m"],
                                     a["iters"], a["C"], a["Q"], None, None, None) == 1
+
+
+@pytest.mark.parametrize("kw", [
+    dict(m=3), dict(iters=-1), dict(groups=5), dict(d_out=0), dict(d_in=0), dict(d_in=16385),
+    dict(F=None), dict(C=None), dict(Q=None), dict(W=None),
+])
+def test_ganq_rows_rejects_bad_arguments(L, kw):
+    a = dict(F=FAKE, groups=4, W=FAKE, d_out=64, d_in=128, m=8, iters=3, C=FAKE, Q=FAKE)
+    a.update(kw)
+    assert L.lnq_ganq_rows(a["F"], a["groups"], a["W"], a["d_out"], a["d_in"], a["m"], a["iters"],
+                           a["C"], a["Q"], None, None, FAKE, 1 << 40, None) == 1
+
+
+def test_ganq_rows_rejects_small_workspace(L):
+    from post_weight_quantization_guided_b200 import binding as b
+    need = b.lnq_workspace_size(b.LNQ_OP_GANQ_ROWS, 0, 128, 64, 4, 8)
+    assert L.lnq_ganq_rows(FAKE, 4, FAKE, 64, 128, 8, 3, FAKE, FAKE, None, None, FAKE, need - 256,
+                           None) == 3
 
 
 def test_quantize_rows_rejects_small_workspace(L):
