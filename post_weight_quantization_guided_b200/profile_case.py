@@ -11,7 +11,8 @@ With `--fisher-only` it stops after building the blocks twice (`--tokens` shorte
 `--lut N` it then packs the codes and runs the lookup-table GEMV N times on one activation
 vector (the codes cycled through enough copies that they come from HBM). With `--diag N` it runs
 N calls of LNQ with diagonal Fisher blocks (the diagonals of the blocks just built, `--iters`
-iterations each, from the initial codebooks).
+iterations each, from the initial codebooks). With `--ganq N` it runs N calls of the GANQ-style
+comparison solver (`--iters` iterations each, from the initial codebooks).
 """
 from __future__ import annotations
 
@@ -33,6 +34,8 @@ def main(argv=None) -> None:
     ap.add_argument("--lut", type=int, default=0, help="lookup-table GEMV calls after the run")
     ap.add_argument("--diag", type=int, default=0,
                     help="calls of LNQ with diagonal Fisher blocks after the run")
+    ap.add_argument("--ganq", type=int, default=0,
+                    help="calls of the GANQ-style comparison solver after the run")
     ap.add_argument("--fisher-only", action="store_true",
                     help="build the Fisher blocks (twice) and stop")
     ap.add_argument("--tokens", type=int, default=0, help="calibration tokens (default: the workload's)")
@@ -77,6 +80,14 @@ def main(argv=None) -> None:
             api.lnq_quantize_rows_diag(Fd, W, layer.m, args.iters, C, Q, J, st)
         torch.cuda.synchronize()
         print(f"lnq_diag calls={args.diag} iters={args.iters} sum(J)={float(J.sum()):.6e}")
+    if args.ganq:
+        C0, Q0 = api.lnq_init_codebook(W, layer.m)
+        for _ in range(args.ganq):
+            C.copy_(C0)
+            Q.copy_(Q0)
+            api.lnq_ganq_rows(F, W, layer.m, args.iters, C, Q, J, st)
+        torch.cuda.synchronize()
+        print(f"ganq calls={args.ganq} iters={args.iters} sum(J)={float(J.sum()):.6e}")
 
 
 if __name__ == "__main__":
