@@ -196,9 +196,10 @@ def executed_tensor_flops(layer, m, kernel):
     return None
 
 
-# DRAM bytes per launch of the dominant kernel from ncu captures of small cases, per row of the
-# launch at a given d_in (scaled by the rows a launch processes), valid only while the kernel's
-# source is the one that was measured.
+# DRAM bytes per launch of the dominant kernel from ncu captures (dram__bytes_read.sum +
+# dram__bytes_write.sum of one launch, the block's own layer shapes with 16384 calibration
+# tokens, which do not change this kernel's work), per output row for each (d_in, m), valid only
+# while the kernel's source is the one that was measured.
 TRAFFIC = {}
 
 
@@ -216,7 +217,7 @@ def measured_traffic(kernel, launches):
         return None
     total, count = 0.0, 0
     for layer, c in launches:
-        per_row = rec["bytes_per_row"].get(layer.d_in)
+        per_row = rec["bytes_per_row"].get(f"{layer.d_in}/{layer.m}")
         if per_row is None:
             return None
         total += c * per_row * layer.d_out

@@ -23,11 +23,11 @@
 //   chol_update_kernel   the trailing lower triangle minus the panel's outer product, in 64 x 64
 //                        tiles (each thread 4 x 4 outputs, the two panel slices in shared memory).
 //   chol_finish_kernel   L (fp32, zero above the diagonal) and 1 / L[i][i].
-//   ganq_assign_kernel   32 rows of one group per CTA, coordinates in blocks of 32 from the last:
+//   ganq_assign_kernel   16 rows of one group per CTA, coordinates in blocks of 32 from the last:
 //                        (1) all 256 threads form s[row][i] = sum_{k past the block} L[k][i] r_k
-//                        for the block's 32 coordinates (32 x 32 outputs, k in chunks of 128
-//                        through shared memory, the next chunk loaded while the current one is
-//                        summed, fp32); (2) one warp (lane = row) decides the block from the
+//                        for the block's 32 coordinates (16 x 32 outputs, k in chunks of 128
+//                        through a ring of three shared-memory stages filled by asynchronous
+//                        copies, two chunks in flight while one is summed, fp32); (2) one warp (lane = row) decides the block from the
 //                        last coordinate to the first, adding the block's own earlier decisions from
 //                        its diagonal tile of L in registers, and finds the nearest codeword by a
 //                        binary search of the sorted codebook's midpoints in registers; (3) the
@@ -41,7 +41,7 @@ namespace lnq {
 
 constexpr int kCholB = 32;       // panel width of the blocked factorisation
 constexpr int kCholTile = 64;    // output tile of the trailing update
-constexpr int kGanqRows = 32;    // rows per CTA of the assignment
+constexpr int kGanqRows = 16;    // rows per CTA of the assignment
 constexpr int kGanqBlk = 32;     // coordinates per decision block
 constexpr int kGanqThreads = 256;
 
@@ -202,53 +202,72 @@ __global__ void chol_finish_kernel(const double *__restrict__ A, int64_t d, int 
 }
 
 constexpr int kGanqKc = 128;     // k per chunk of step (1)
+constexpr int kGanqLL = kGanqKc * kGanqBlk / 4 / kGanqThreads;     // float4 loads of L per thread
+constexpr int kGanqRL = kGanqRows * kGanqKc / 4 / kGanqThreads;    // float4 loads of R per thread
+constexpr int kGanqOut = kGanqRows * kGanqBlk / kGanqThreads;      // outputs of step (1) per thread
+static_assert(kGanqLL * 4 * kGanqThreads == kGanqKc * kGanqBlk, "L chunk split");
+static_assert(kGanqRL * 4 * kGanqThreads == kGanqRows * kGanqKc, "R chunk split");
+static_assert(kGanqOut == 2, "two outputs per thread in step (1)");
 
-// One chunk of step (1) into registers: L[kc + a][b0 .. b0 + 31] for a < kGanqKc and
-// R[j0 + row][kc .. kc + kGanqKc - 1] for the CTA's rows; zeros past d and past the rows. kVec: d is
-// a multiple of 4, so both come as float4.
+constexpr int kGanqStages = 3;   // chunks in flight in step (1)
+constexpr int kGanqRcLd = kGanqKc + 4;                               // row stride of a staged R chunk
+constexpr int kGanqStage = kGanqKc * kGanqBlk + kGanqRows * kGanqRcLd;   // floats per stage
+constexpr size_t kGanqSmem = static_cast<size_t>(kGanqStages) * kGanqStage * sizeof(float);
+
+__device__ __forceinline__ void cp_async16_zfill(void *dst, const void *src, bool valid)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src),
+                 "r"(valid ? 16 : 0)
+                 : "memory");
+}
+
+template <int N>
+__device__ __forceinline__ void cp_async_wait_group()
+{
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// One chunk of step (1) into a stage: L[kc + a][b0 .. b0 + 31] for a < kGanqKc (lc, [Kc][32])
+// and R[j0 + row][kc .. kc + kGanqKc - 1] for the CTA's rows (rc, [rows][Kc + 4]); zeros past d
+// and past the rows. kVec (d a multiple of 4): 16-byte asynchronous copies with zero fill;
+// otherwise plain loads and stores.
 template <bool kVec>
-__device__ __forceinline__ void ganq_load_chunk(const float *__restrict__ Lg,
-                                                const float *__restrict__ R, int64_t d,
-                                                int64_t b0, int bw, int64_t j0, int nr,
-                                                int64_t kc, float4 (&pl)[4], float4 (&pr)[4])
+__device__ __forceinline__ void ganq_issue_chunk(float *stage, const float *__restrict__ Lg,
+                                                 const float *__restrict__ R, int64_t d,
+                                                 int64_t b0, int bw, int64_t j0, int nr,
+                                                 int64_t kc)
 {
     const int t = threadIdx.x;
+    float *lc = stage;
+    float *rc = stage + kGanqKc * kGanqBlk;
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < kGanqLL; ++u) {
         const int e = t + kGanqThreads * u;
-        {   // L: row a = e / 8, columns 4 (e % 8) .. + 3
-            const int a = e >> 3, c4 = (e & 7) * 4;
-            const int64_t k = kc + a;
-            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (k < d) {
-                const float *src = Lg + k * d + b0 + c4;
-                if (kVec && c4 + 4 <= bw) {
-                    v = __ldg(reinterpret_cast<const float4 *>(src));
-                } else {
-                    v.x = c4 < bw ? __ldg(src) : 0.f;
-                    v.y = c4 + 1 < bw ? __ldg(src + 1) : 0.f;
-                    v.z = c4 + 2 < bw ? __ldg(src + 2) : 0.f;
-                    v.w = c4 + 3 < bw ? __ldg(src + 3) : 0.f;
-                }
-            }
-            pl[u] = v;
+        const int a = e >> 3, c4 = (e & 7) * 4;   // L row a, columns c4 .. c4 + 3
+        const int64_t k = kc + a;
+        float *dst = lc + a * kGanqBlk + c4;
+        const float *src = Lg + (k < d ? k : 0) * d + b0 + c4;
+        if (kVec) {
+            cp_async16_zfill(dst, k < d && c4 + 4 <= bw ? src : Lg, k < d && c4 + 4 <= bw);
+        } else {
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+                dst[c] = (k < d && c4 + c < bw) ? __ldg(src + c) : 0.f;
         }
-        {   // R: row e / 32, k 4 (e % 32) .. + 3
-            const int row = e >> 5, k4 = (e & 31) * 4;
-            const int64_t k = kc + k4;
-            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (row < nr) {
-                const float *src = R + (j0 + row) * d + k;
-                if (kVec && k + 4 <= d) {
-                    v = *reinterpret_cast<const float4 *>(src);
-                } else {
-                    v.x = k < d ? src[0] : 0.f;
-                    v.y = k + 1 < d ? src[1] : 0.f;
-                    v.z = k + 2 < d ? src[2] : 0.f;
-                    v.w = k + 3 < d ? src[3] : 0.f;
-                }
-            }
-            pr[u] = v;
+    }
+#pragma unroll
+    for (int u = 0; u < kGanqRL; ++u) {
+        const int e = t + kGanqThreads * u;
+        const int row = e >> 5, k4 = (e & 31) * 4;   // R row, k offsets k4 .. k4 + 3
+        const int64_t k = kc + k4;
+        float *dst = rc + row * kGanqRcLd + k4;
+        const float *src = R + (j0 + (row < nr ? row : 0)) * d + (k < d ? k : 0);
+        if (kVec) {
+            cp_async16_zfill(dst, row < nr && k + 4 <= d ? src : R, row < nr && k + 4 <= d);
+        } else {
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+                dst[c] = (row < nr && k + c < d) ? src[c] : 0.f;
         }
     }
 }
@@ -261,18 +280,15 @@ __global__ void __launch_bounds__(kGanqThreads)
                        float *__restrict__ R, int32_t *__restrict__ status, int64_t d,
                        int64_t rows_per_group, int ctas_per_group)
 {
-    // step (1) uses lc and rc; steps (2) and (3) reuse the same bytes for ss, ws, rs and ld
-    // (barriers separate the steps)
-    __shared__ __align__(16) float smraw[kGanqKc * kGanqBlk + kGanqRows * (kGanqKc + 4)];
-    auto lc = reinterpret_cast<float(*)[kGanqBlk]>(smraw);                          // [Kc][32]
-    auto rc = reinterpret_cast<float(*)[kGanqKc + 4]>(smraw + kGanqKc * kGanqBlk);  // [rows][Kc]
-    auto ss = reinterpret_cast<float(*)[kGanqBlk + 1]>(smraw);            // s of the block
-    auto ws = ss + kGanqRows;                                             // w of the block
-    auto rs = ws + kGanqRows;                                             // r of the block
-    auto ld = reinterpret_cast<float(*)[kGanqBlk]>(smraw + 3 * kGanqRows * (kGanqBlk + 1));
-    static_assert(3 * kGanqRows * (kGanqBlk + 1) + kGanqBlk * kGanqBlk <=
-                      kGanqKc * kGanqBlk + kGanqRows * (kGanqKc + 4),
-                  "the decision tiles fit in the chunk buffers");
+    // step (1) uses the ring of chunk stages; steps (2) and (3) reuse the first stage's bytes for
+    // ss, ws, rs and ld (barriers separate the steps)
+    extern __shared__ __align__(16) float ganq_sm[];
+    auto ss = reinterpret_cast<float(*)[kGanqBlk + 1]>(ganq_sm);           // s of the block
+    auto ws = ss + kGanqRows;                                              // w of the block
+    auto rs = ws + kGanqRows;                                              // r of the block
+    auto ld = reinterpret_cast<float(*)[kGanqBlk]>(ganq_sm + 3 * kGanqRows * (kGanqBlk + 1));
+    static_assert(3 * kGanqRows * (kGanqBlk + 1) + kGanqBlk * kGanqBlk <= kGanqStage,
+                  "the decision tiles fit in one chunk stage");
     __shared__ float iv[kGanqBlk];                      // 1 / L[i][i] of the block
     __shared__ uint8_t qs[kGanqRows][kGanqBlk];
     const int g = blockIdx.x / ctas_per_group;
@@ -320,61 +336,60 @@ __global__ void __launch_bounds__(kGanqThreads)
         const int64_t kstart = b0 + bw;
         // (1) s[row][c] = sum_{k >= kstart} L[k][b0 + c] r[row][k]: chunks of kGanqKc through
         // shared memory, the next chunk's loads in flight while the current one is summed
-        const int srow = t >> 3, scol = (t & 7) * 4;
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
-        float4 pl[4], pr[4];
-        if (kstart < d) {
-            ganq_load_chunk<kVec>(Lg, R, d, b0, bw, j0, nr, kstart, pl, pr);
+        const int srow = t / (kGanqBlk / kGanqOut), scol = (t % (kGanqBlk / kGanqOut)) * kGanqOut;
+        float acc[kGanqOut] = {0.f, 0.f};
+        const int64_t nch = kstart < d ? (d - kstart + kGanqKc - 1) / kGanqKc : 0;
+        // kGanqStages - 1 chunks in flight ahead of the one being summed; one commit group per
+        // chunk slot (empty groups past the last chunk keep the count uniform)
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int e = t + kGanqThreads * u;
-                *reinterpret_cast<float4 *>(&lc[e >> 3][(e & 7) * 4]) = pl[u];
-                *reinterpret_cast<float4 *>(&rc[e >> 5][(e & 31) * 4]) = pr[u];
-            }
+        for (int c = 0; c < kGanqStages - 1; ++c) {
+            if (c < nch)
+                ganq_issue_chunk<kVec>(ganq_sm + c * kGanqStage, Lg, R, d, b0, bw, j0, nr,
+                                       kstart + c * kGanqKc);
+            cp_async_commit();
         }
-        __syncthreads();
-        for (int64_t kc = kstart; kc < d; kc += kGanqKc) {
-            const bool more = kc + kGanqKc < d;
-            if (more)
-                ganq_load_chunk<kVec>(Lg, R, d, b0, bw, j0, nr, kc + kGanqKc, pl, pr);
+        for (int64_t c = 0; c < nch; ++c) {
+            cp_async_wait_group<kGanqStages - 2>();
+            __syncthreads();    // chunk c visible; every thread is done with chunk c - 1
+            const int64_t cn = c + kGanqStages - 1;
+            if (cn < nch)
+                ganq_issue_chunk<kVec>(ganq_sm + (cn % kGanqStages) * kGanqStage, Lg, R, d, b0, bw,
+                                       j0, nr, kstart + cn * kGanqKc);
+            cp_async_commit();
+            const float *lc = ganq_sm + (c % kGanqStages) * kGanqStage;
+            const float *rc = lc + kGanqKc * kGanqBlk;
 #pragma unroll 4
             for (int k = 0; k < kGanqKc; k += 4) {
-                const float4 r4 = *reinterpret_cast<const float4 *>(&rc[srow][k]);
+                const float4 r4 = *reinterpret_cast<const float4 *>(rc + srow * kGanqRcLd + k);
                 const float rv[4] = {r4.x, r4.y, r4.z, r4.w};
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
-                    const float4 l4 = *reinterpret_cast<const float4 *>(&lc[k + kk][scol]);
-                    acc[0] = fmaf(rv[kk], l4.x, acc[0]);
-                    acc[1] = fmaf(rv[kk], l4.y, acc[1]);
-                    acc[2] = fmaf(rv[kk], l4.z, acc[2]);
-                    acc[3] = fmaf(rv[kk], l4.w, acc[3]);
+                    const float2 l2 =
+                        *reinterpret_cast<const float2 *>(lc + (k + kk) * kGanqBlk + scol);
+                    acc[0] = fmaf(rv[kk], l2.x, acc[0]);
+                    acc[1] = fmaf(rv[kk], l2.y, acc[1]);
                 }
-            }
-            __syncthreads();
-            if (more) {
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int e = t + kGanqThreads * u;
-                    *reinterpret_cast<float4 *>(&lc[e >> 3][(e & 7) * 4]) = pl[u];
-                    *reinterpret_cast<float4 *>(&rc[e >> 5][(e & 31) * 4]) = pr[u];
-                }
-                __syncthreads();
             }
         }
+        cp_async_wait_group<0>();
+        __syncthreads();        // every thread is done with the stages before they are reused
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
+        for (int c = 0; c < kGanqOut; ++c)
             ss[srow][scol + c] = acc[c];
         // the block's w, its diagonal tile of L and the reciprocal pivots
-        for (int x = t; x < kGanqBlk * kGanqBlk; x += kGanqThreads) {
+        for (int x = t; x < kGanqRows * kGanqBlk; x += kGanqThreads) {
             const int a = x / kGanqBlk, b = x % kGanqBlk;
             ws[a][b] = (a < nr && b < bw) ? W[(j0 + a) * d + b0 + b] : 0.f;
+        }
+        for (int x = t; x < kGanqBlk * kGanqBlk; x += kGanqThreads) {
+            const int a = x / kGanqBlk, b = x % kGanqBlk;
             ld[a][b] = (a < bw && b < bw) ? Lg[(b0 + a) * d + b0 + b] : 0.f;
         }
         if (t < bw)
             iv[t] = invd[g * d + b0 + t];
         __syncthreads();
         // (2) decisions, last coordinate first
-        if (warp == 0) {
+        if (warp == 0 && lane < kGanqRows) {
             float sacc[kGanqBlk];
 #pragma unroll
             for (int c = 0; c < kGanqBlk; ++c)
@@ -446,13 +461,16 @@ static cudaError_t ganq_assign_m(const float *L, const float *invd, const int32_
     const int64_t rpg = d_out / groups;
     const int cpg = static_cast<int>((rpg + kGanqRows - 1) / kGanqRows);
     KernelTimer timer("ganq_assign", s);
-    if (d % 4 == 0)
-        ganq_assign_kernel<M, true><<<static_cast<unsigned>(cpg) * groups, kGanqThreads, 0, s>>>(
+    auto launch = [&](auto kernel) -> cudaError_t {
+        cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(kGanqSmem));
+        if (e != cudaSuccess)
+            return e;
+        kernel<<<static_cast<unsigned>(cpg) * groups, kGanqThreads, kGanqSmem, s>>>(
             L, invd, gstatus, W, C, Q, R, status, d, rpg, cpg);
-    else
-        ganq_assign_kernel<M, false><<<static_cast<unsigned>(cpg) * groups, kGanqThreads, 0, s>>>(
-            L, invd, gstatus, W, C, Q, R, status, d, rpg, cpg);
-    return cudaGetLastError();
+        return cudaGetLastError();
+    };
+    return d % 4 == 0 ? launch(ganq_assign_kernel<M, true>) : launch(ganq_assign_kernel<M, false>);
 }
 
 cudaError_t lnq_ganq_launch(const float *F, int groups, const float *W, int64_t d_out, int64_t d,

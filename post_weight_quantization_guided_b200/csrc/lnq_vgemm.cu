@@ -49,6 +49,7 @@ constexpr int A_TILE = BM * BK * 2;              // one fp16 piece of a 128 x 64
 constexpr int B_STAGES = 4;                      // right-operand half tiles in flight
 constexpr int NUM_THREADS = 192;                 // w0 TMA, w1 MMA, w2-5 epilogue
 constexpr int EPI_THREADS = 128;
+constexpr int IP_BLOCK = 9;   // pair blocks per block of the tile order (see vg_tile_coords)
 constexpr int EPI_BAR = 1;                       // named barrier of the epilogue warps
 constexpr int TMEM_COLS = 512;
 constexpr int NCOLS = 256;                       // MMA N: columns of the right operand per tile
@@ -298,17 +299,34 @@ struct VgParams {
 };
 
 // Tile -> (group, rows [row0, row_end), coordinate pair block ip, row tile rt_all over all
-// groups). Consecutive tiles share a row tile, so the pairs running at the same time read the same
-// right-operand tiles, and a group's F pieces (fp16: 2 d^2 x 2 bytes) stay in L2 across its rows.
+// groups). Within a group the tiles run in blocks of IP_BLOCK pair blocks: row tile by row tile,
+// and within a row tile the block's pair blocks. The pairs running at the same time then cover
+// about 8 row tiles x IP_BLOCK pair blocks of one group: each F piece tile is read by the 8 row
+// tiles at once and each right-operand tile by the IP_BLOCK pair blocks, so both come from L2
+// after their first read even when a group's F pieces (2 d^2 x 2 bytes) are far larger than L2.
 template <int M>
 __device__ __forceinline__ void vg_tile_coords(const VgParams &p, int tile, int &g, int64_t &row0,
                                                int64_t &row_end, int &ip, int &rt_all)
 {
     constexpr int RT = VgShape<M>::RT;
-    ip = tile % p.i_pairs;
-    rt_all = tile / p.i_pairs;
-    g = rt_all / p.row_tiles_per_group;
-    const int rt = rt_all - g * p.row_tiles_per_group;
+    const int per_group = p.row_tiles_per_group * p.i_pairs;
+    g = tile / per_group;
+    int o = tile - g * per_group;
+    const int full = p.i_pairs / vg::IP_BLOCK;               // whole blocks of pair blocks
+    const int per_full = p.row_tiles_per_group * vg::IP_BLOCK;
+    int ipb, width;
+    if (o < full * per_full) {
+        ipb = o / per_full;
+        o -= ipb * per_full;
+        width = vg::IP_BLOCK;
+    } else {
+        ipb = full;
+        o -= full * per_full;
+        width = p.i_pairs - full * vg::IP_BLOCK;
+    }
+    const int rt = o / width;
+    ip = ipb * vg::IP_BLOCK + (o - rt * width);
+    rt_all = g * p.row_tiles_per_group + rt;
     const int64_t gstart = static_cast<int64_t>(g) * p.rows_per_group;
     row0 = gstart + static_cast<int64_t>(rt) * RT;
     row_end = min(row0 + RT, gstart + p.rows_per_group);

@@ -23,7 +23,9 @@ import torch
 from . import binding as api
 from . import workloads as wl
 
-WORKLOADS = {"tiny": wl.TINY, "q_proj": wl.Q_PROJ, "down_proj": wl.DOWN_PROJ, "up_proj": wl.UP_PROJ}
+WORKLOADS = {"tiny": wl.TINY, "q_proj": wl.Q_PROJ, "down_proj": wl.DOWN_PROJ, "up_proj": wl.UP_PROJ,
+             "block_q": wl.decoder_block(16)[0], "block_gate": wl.decoder_block(16)[4],
+             "block_down": wl.decoder_block(16)[6]}
 
 
 def main(argv=None) -> None:
@@ -39,6 +41,7 @@ def main(argv=None) -> None:
     ap.add_argument("--fisher-only", action="store_true",
                     help="build the Fisher blocks (twice) and stop")
     ap.add_argument("--tokens", type=int, default=0, help="calibration tokens (default: the workload's)")
+    ap.add_argument("--m", type=int, default=0, help="codewords per row (default: the workload's)")
     args = ap.parse_args(argv)
     layer = WORKLOADS[args.workload]
     if args.rows:
@@ -47,6 +50,8 @@ def main(argv=None) -> None:
         layer = wl.scaled(layer, d_out=args.rows)
     if args.tokens:
         layer = wl.scaled(layer, n=args.tokens)
+    if args.m:
+        layer = wl.scaled(layer, m=args.m)
     dev = torch.device("cuda:0")
     X, G, W = wl.make_layer(layer, dev)
     F = api.lnq_build_fisher(X, G, layer.groups)
