@@ -198,9 +198,19 @@ def executed_tensor_flops(layer, m, kernel):
 
 # DRAM bytes per launch of the dominant kernel from ncu captures (dram__bytes_read.sum +
 # dram__bytes_write.sum of one launch, the block's own layer shapes with 16384 calibration
-# tokens, which do not change this kernel's work), per output row for each (d_in, m), valid only
-# while the kernel's source is the one that was measured.
-TRAFFIC = {}
+# tokens, which do not change this kernel's work), per output row for each (d_in, d_out, m),
+# valid only while the kernel's source is the one that was measured.
+TRAFFIC = {
+    "lnq_mgemm": {
+        "source": "lnq_vgemm.cu",
+        "sha256": "eb71dc725b8bf11887f2350945960880c807ff5d1ff296aa89c87c9375f79969",
+        "bytes_per_row": {
+            "4096/4096/16": 1177223168 / 4096, "4096/4096/8": 609373696 / 4096,
+            "4096/11008/16": 2883097856 / 11008, "4096/11008/8": 1477671936 / 11008,
+            "11008/4096/16": 34628989696 / 4096, "11008/4096/8": 17168465408 / 4096,
+        },
+    },
+}
 
 
 def measured_traffic(kernel, launches):
@@ -217,7 +227,7 @@ def measured_traffic(kernel, launches):
         return None
     total, count = 0.0, 0
     for layer, c in launches:
-        per_row = rec["bytes_per_row"].get(f"{layer.d_in}/{layer.m}")
+        per_row = rec["bytes_per_row"].get(f"{layer.d_in}/{layer.d_out}/{layer.m}")
         if per_row is None:
             return None
         total += c * per_row * layer.d_out
