@@ -99,15 +99,17 @@ __device__ __forceinline__ double diag_scale(int e)
     return __longlong_as_double(static_cast<long long>(41 - e + 1023) << 52);
 }
 
-// Adds or removes coordinate i = (fi, wi) at class q.
+// Adds or removes coordinate i = (fi, wi) at class q (scale_w, scale_f: the row's 2^s_w, 2^s_f,
+// read once by the caller).
 template <int M>
 __device__ __forceinline__ void diag_class_add(DiagShared<M> &sh, int i, int q, float fi,
-                                               float wi, bool remove)
+                                               float wi, bool remove, double scale_w,
+                                               double scale_f)
 {
     // exact products in fp64, scaled by powers of two (exact), rounded to integers
     const long long tw = __double2ll_rn(static_cast<double>(fi) * static_cast<double>(wi) *
-                                        sh.scale_w);
-    const long long tf = __double2ll_rn(static_cast<double>(fi) * sh.scale_f);
+                                        scale_w);
+    const long long tf = __double2ll_rn(static_cast<double>(fi) * scale_f);
     const int sg = remove ? -1 : 1;
     const int slot = (i >> 2) & 31;
     atomicAdd(&sh.lim[0][q][slot], sg * static_cast<int>(tw & 0x1fffff));
@@ -166,9 +168,10 @@ __device__ __forceinline__ void diag_drain(DiagShared<M> &sh, float *ws, uint8_t
         const int q = qs[i];
         const int a = diag_assign_full<M>(sh, fi, wi, q);
         if (a != q) {
+            const double sw = sh.scale_w, sf = sh.scale_f;
             qs[i] = static_cast<uint8_t>(a);
-            diag_class_add<M>(sh, i, q, fi, wi, true);
-            diag_class_add<M>(sh, i, a, fi, wi, false);
+            diag_class_add<M>(sh, i, q, fi, wi, true, sw, sf);
+            diag_class_add<M>(sh, i, a, fi, wi, false, sw, sf);
         }
         if (kObjective)
             jr += diag_cost(sh.cb[a], fi, wi);
@@ -203,13 +206,26 @@ __device__ __forceinline__ double diag_assign_pass(DiagShared<M> &sh, float *ws,
     const int nq = (d + 3) / 4;
     int qc = 0;                     // warp-uniform queue length
     double jr = 0.0;
+    // the quad of the next step is loaded before this one is tested (a drain only touches the
+    // coordinates this warp has already tested, never the quad loaded ahead)
+    float4 wn = make_float4(0.f, 0.f, 0.f, 0.f), fn = wn;
+    uint32_t qn = 0u;
+    if (warp * 32 + lane < nq) {
+        wn = reinterpret_cast<const float4 *>(ws)[warp * 32 + lane];
+        qn = reinterpret_cast<const uint32_t *>(qs)[warp * 32 + lane];
+    }
+    fn = diag_f4<kVec>(f, warp * 32 + lane, d);
     for (int k0 = warp * 32; k0 < nq; k0 += kDiagThreads) {
+        const float4 wv = wn, fv = fn;
+        const uint32_t qv = qn;
+        {
+            const int kx = k0 + kDiagThreads + lane;
+            const bool xin = kx < nq;
+            wn = xin ? reinterpret_cast<const float4 *>(ws)[kx] : make_float4(0.f, 0.f, 0.f, 0.f);
+            qn = xin ? reinterpret_cast<const uint32_t *>(qs)[kx] : 0u;
+            fn = diag_f4<kVec>(f, kx, d);
+        }
         const int k = k0 + lane;
-        const bool kin = k < nq;
-        const float4 wv = kin ? reinterpret_cast<const float4 *>(ws)[k]
-                              : make_float4(0.f, 0.f, 0.f, 0.f);
-        const uint32_t qv = kin ? reinterpret_cast<const uint32_t *>(qs)[k] : 0u;
-        const float4 fv = diag_f4<kVec>(f, k, d);
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
             const float fi = f4_at(fv, u), wi = f4_at(wv, u);
@@ -347,7 +363,7 @@ __device__ __forceinline__ void diag_codebook(DiagShared<M> &sh, const float *ws
 
 // kVec: d % 4 == 0, W and Fd 16-byte aligned and Q 4-byte aligned (rows as whole quads).
 template <int M, bool kVec>
-__global__ void __launch_bounds__(kDiagThreads, 8)
+__global__ void __launch_bounds__(kDiagThreads, M == 16 ? 6 : 8)
     diag_lnq_kernel(const float *__restrict__ Fd, const float *__restrict__ W, int d,
                     int64_t rows_per_group, int iters, float *__restrict__ C,
                     uint8_t *__restrict__ Q, double *__restrict__ J, int32_t *__restrict__ status)
@@ -447,15 +463,19 @@ __global__ void __launch_bounds__(kDiagThreads, 8)
             jr += diag_cost(sh.cb[qs[i]], __ldg(f + i), ws[i]);
     } else {
         // the class sums of the starting codes (thread t takes quads t, t + 128, ...: slot = lane)
+        //  (the next quad's f is loaded before this one is added)
+        const double sw = sh.scale_w, sf = sh.scale_f;
+        float4 fn = diag_f4<kVec>(f, t, d);
         for (int k = t; k < (d + 3) / 4; k += kDiagThreads) {
-            const float4 fv = diag_f4<kVec>(f, k, d);
+            const float4 fv = fn;
+            fn = diag_f4<kVec>(f, k + kDiagThreads, d);
             const float4 wv = reinterpret_cast<const float4 *>(ws)[k];
             const uint32_t qv = reinterpret_cast<const uint32_t *>(qs)[k];
 #pragma unroll
             for (int u = 0; u < 4; ++u)
                 if (4 * k + u < d)
                     diag_class_add<M>(sh, 4 * k + u, (qv >> (8 * u)) & 0xffu, f4_at(fv, u),
-                                      f4_at(wv, u), false);
+                                      f4_at(wv, u), false, sw, sf);
         }
         for (int it = 0; it < iters; ++it) {
             __syncthreads();
