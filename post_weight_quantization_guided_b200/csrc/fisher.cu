@@ -435,7 +435,7 @@ __device__ __forceinline__ void fisher_syrk_body(const CUtensorMap &amap, const 
         for (int tile = pair; tile < p.num_tiles; tile += npairs, ++it) {
             const int acc = it & 1;
             const int use = it >> 1;
-            // One lane waits and the warp follows its verdict, so the warp-collective TMEM loads
+            // One lane waits and the warp follows its outcome, so the warp-collective TMEM loads
             // below are executed by all 32 lanes or by none.
             int ok = 0;
             if (lane == 0)
