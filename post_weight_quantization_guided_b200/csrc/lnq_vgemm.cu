@@ -586,7 +586,7 @@ __global__ void __launch_bounds__(vg::NUM_THREADS, 1)
                 const int ih = 2 * ip + static_cast<int>(cr);
                 const bool halve_here = nk - vg_first_kb<M>(ip) <= PAIR_KB;  // no later block
                 const int acc = itn % S::SETS;
-                // All four warps take one decision on the accumulator (so that none of them waits at
+                // All four warps take one verdict on the accumulator (so that none of them waits at
                 // a named barrier the others have left); the barrier also ends the previous tile's
                 // binning, so its codes may be overwritten.
                 int okw = 0;
