@@ -238,16 +238,19 @@ def measured_traffic(kernel, launches):
 def roofline(work, unit, ms, peaks, fp32_peak):
     """Roofline object for `work` algorithmic units done in `ms` of device time."""
     sec = ms / 1e3
+    src = peaks.get("source", "measured")
     if unit == "flop":
-        peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+        sustained = "bf16_tflops_sustained" in peaks
+        peak = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
         achieved = work / sec / 1e12
+        kind = f"bf16 dense, {'sustained' if sustained else 'burst'} (of {src})"
         return {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "peak_kind": "bf16 dense, sustained (of measured)"}
+                "frac": achieved / peak, "peak_kind": kind}
     if unit == "byte":
         peak = peaks["hbm_gbs"]
         achieved = work / sec / 1e9
         return {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                "frac": achieved / peak, "peak_kind": "HBM copy (of measured)"}
+                "frac": achieved / peak, "peak_kind": f"HBM copy (of {src})"}
     peak = fp32_peak["sustained"]
     achieved = work / sec / 1e12
     return {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "Tlane-op/s",
