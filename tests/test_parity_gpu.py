@@ -137,6 +137,26 @@ def test_lnq_q_proj_full_size_sampled_rows(orc, lnq, wl):
     assert summary["moves"] > 0
 
 
+def test_lnq_q_proj_one_call_equals_one_iteration_calls(lnq, wl):
+    """The bench's form of the call (all iterations and the objective in one lnq_quantize_rows)
+    ends bit for bit in the state of one-iteration calls, whose every step the follow-mode test
+    above checks against the oracle: 32 sweep windows, so the per-window move flags of one call
+    carry nothing into the next iteration."""
+    layer = wl.Q_PROJ
+    X, G, W = wl.make_layer(layer, _dev())
+    F = lnq.lnq_build_fisher(X, G, layer.groups)
+    del X, G
+    C, Q = lnq.lnq_init_codebook(W, layer.m)
+    Ca, Qa = C.clone(), Q.clone()
+    J = torch.empty(W.shape[0], dtype=torch.float64, device=W.device)
+    Ja = torch.empty_like(J)
+    lnq.lnq_quantize_rows(F, W, layer.m, layer.iters, C, Q, J)
+    for _ in range(layer.iters):
+        lnq.lnq_quantize_rows(F, W, layer.m, 1, Ca, Qa, Ja)
+    torch.cuda.synchronize()
+    assert torch.equal(C, Ca) and torch.equal(Q, Qa) and torch.equal(J, Ja)
+
+
 def test_lnq_down_proj_full_size_sampled_rows(orc, lnq, wl):
     """d_in = 11008 (86 sweep windows, a ragged last one), m = 8, four iterations, one group."""
     layer = wl.DOWN_PROJ
