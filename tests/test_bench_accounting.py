@@ -105,3 +105,33 @@ def test_traffic_needs_the_measured_source(monkeypatch):
     monkeypatch.setitem(bench.TRAFFIC, "lnq_mgemm", changed)
     assert bench.measured_traffic("lnq_mgemm", [(L, 3)]) is None
     assert bench.measured_traffic("lnq_sweep", [(L, 3)]) is None
+
+
+def test_cpu_baseline_leg_runs_on_a_small_block(orc):
+    """The bench's oracle leg on CPU tensors of a scaled block: it samples Fisher tiles and LNQ
+    rows of the first and last layer and extrapolates to one step of every layer."""
+    import numpy as np
+    import torch
+    blk = wl.decoder_block(16)
+    layers = [wl.scaled(L, d_in=128 if L.d_in == 4096 else 160, d_out=32 if L.d_out == 4096 else 48,
+                        n=128, iters=2) for L in blk]
+    cache = {}
+
+    def inputs(L):
+        if L.name not in cache:
+            cache[L.name] = wl.make_layer(L, torch.device("cpu"))
+        return cache[L.name]
+
+    F_small = {}
+    for L in (layers[0], layers[-1]):
+        X, G, _ = inputs(L)
+        Gh = G[:, :L.rows_per_group].double().numpy()
+        s = orc.group_scales(Gh, L.n, L.rows_per_group, 1)[0]
+        Xh = X.double().numpy()
+        F_small[L.name] = orc.fisher_block(Xh, Xh, s, 1.0)
+    out = bench.cpu_baseline_block(layers, inputs, F_small, budget_s=0.2, threads=2)
+    assert out["kind"] == "oracle" and out["cores"] == 2 and out["unit"] == bench.UNIT
+    rows = 2 * sum(L.d_out for L in layers)
+    secs = out["fisher_s_extrapolated"] + out["lnq_s_extrapolated"]
+    assert secs > 0 and out["value"] == pytest.approx(rows / secs)
+    assert np.isfinite(out["value"]) and "d_in=160" in out["sample"]
